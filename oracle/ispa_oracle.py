@@ -1,0 +1,304 @@
+"""fp64 CPU oracle of the ISPA hot path.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product package imports, links or
+executes this module; only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may.  It is deliberately plain and slow: every
+function follows the definition it cites in float64, with NumPy matmuls,
+LAPACK's Cholesky and triangular solves as the only library steps, and no
+blocking, fusion or reordering beyond what the definition states.
+
+Sources (the five web pages about arXiv 2607.00712, "Towards Memory-Efficient
+Autoregressive Video Generation via Instance-Specific Parametric Absorption"):
+
+* [EN-notes]   en.papernotes.org note, section "Key Designs" 1-3, "Loss &
+                Training", "Main Results" / "Ablation Study" (Table 2).
+* [ZH-notes]   papernotes.org note, the Chinese version of the same sections.
+* [DE-summary] gist.science/de, "Technisches Resümee", section 2 "Methodik",
+                items "Dual-Stream Warmup", "Layer Absorb", "Speichereffiziente
+                Inferenz" and "Dynamische Layerauswahl".
+
+Readings taken where the pages are silent or garbled (each one is also
+listed in the design notes of the repository):
+
+* softmax scale 1/sqrt(d); log-sum-exp in natural log with the scale included;
+* no mask inside a group: the current chunk attends to itself bidirectionally;
+* local group = sink frames union current frames, history = frames strictly
+  between them; an empty group has L = -inf and O = 0;
+* the merge (the pages cite Eq. 9-12 without printing them) is the standard
+  log-sum-exp combination of two disjoint softmax groups;
+* W is applied to row vectors, y = a W, W of shape [D_in, D_out];
+* the ridge penalty is squared Frobenius (the DE summary writes ||.||_2^2);
+* epsilon is taken over all warmup rows, without the lambda term;
+* K = floor(x N); ties in epsilon go to the lower layer index.
+
+Parity pins for every function live in ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, List, Sequence, Tuple
+
+import numpy as np
+import scipy.linalg
+
+NEG_INF = -np.inf
+
+
+# ---------------------------------------------------------------------------
+# attention over one KV group  [EN-notes, Key Designs 1]
+# ---------------------------------------------------------------------------
+def attend_group(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> Tuple[np.ndarray, np.ndarray]:
+    """Softmax attention of queries q [n, d] over one key group k, v [m, d].
+
+    Returns the group's normalised output O [n, d] and its log-sum-exp
+    L [n] = log(sum_j exp(scale * q.k_j)).  Each group "returns both its
+    weighted value output and the LSE state associated with softmax
+    normalization" [EN-notes, Key Designs 1].  An empty group returns O = 0 and
+    L = -inf, so that it carries no attention mass in a merge.
+    """
+    q = np.asarray(q, np.float64)
+    n = q.shape[0]
+    if k.shape[0] == 0:
+        return np.zeros((n, v.shape[1])), np.full(n, NEG_INF)
+    s = scale * (q @ np.asarray(k, np.float64).T)          # [n, m] scores
+    m = s.max(axis=1)
+    e = np.exp(s - m[:, None])
+    l = e.sum(axis=1)
+    O = (e @ np.asarray(v, np.float64)) / l[:, None]
+    return O, m + np.log(l)
+
+
+def lse_merge(o_a: np.ndarray, l_a: np.ndarray, o_b: np.ndarray, l_b: np.ndarray):
+    """Recover attention over the union of two disjoint groups from each group's (O, L).
+
+    The full output is a combination "using LSE-derived weights"; "an ordinary
+    average would be incorrect because the groups generally carry different
+    amounts of total attention mass" [EN-notes, Key Designs 1].  With
+    L = log(exp(L_a) + exp(L_b)), O = exp(L_a - L) O_a + exp(L_b - L) O_b.
+    Both groups empty gives L = -inf, O = 0.
+    """
+    l_a = np.asarray(l_a, np.float64)
+    l_b = np.asarray(l_b, np.float64)
+    L = np.logaddexp(l_a, l_b)
+    both_empty = np.isneginf(L)
+    Ls = np.where(both_empty, 0.0, L)
+    w_a = np.where(np.isneginf(l_a), 0.0, np.exp(np.where(np.isneginf(l_a), 0.0, l_a) - Ls))
+    w_b = np.where(np.isneginf(l_b), 0.0, np.exp(np.where(np.isneginf(l_b), 0.0, l_b) - Ls))
+    O = w_a[..., None] * np.asarray(o_a, np.float64) + w_b[..., None] * np.asarray(o_b, np.float64)
+    return O, L
+
+
+def _local_rows(shape) -> np.ndarray:
+    frames = sorted(set(range(0, shape.sink_frames)) | set(range(shape.cur_begin, shape.cur_end)))
+    return np.array([r for f in frames for r in range(f * shape.tpf, (f + 1) * shape.tpf)], dtype=np.int64)
+
+
+def _hist_rows(shape) -> np.ndarray:
+    return np.arange(shape.hist_begin * shape.tpf, shape.hist_end * shape.tpf, dtype=np.int64)
+
+
+def split_attention(shape, q, k, v, scale: float = None, rows: Sequence[int] = None,
+                    row_block: int = 512) -> Dict[str, np.ndarray]:
+    """Decomposable two-group attention of one chunk  [EN-notes, Key Designs 1; DE-summary 2].
+
+    q [B, Lq, H, d]; k, v [B, kv_frames*tpf, H, d].  The same queries attend
+    separately to the local group (sink frames and current frames) and to the
+    history group (the frames in between); the two results are merged by their
+    LSE into the full-context output.  ``rows`` restricts the query rows (all by
+    default).  Returns O_* [B, n, H, d] and L_* [B, n, H] for loc, hist, full.
+    """
+    d = q.shape[-1]
+    scale = 1.0 / math.sqrt(d) if not scale else scale
+    B, Lq, H, _ = q.shape
+    rows = np.arange(Lq) if rows is None else np.asarray(rows)
+    n = len(rows)
+    loc_idx, hist_idx = _local_rows(shape), _hist_rows(shape)
+    out = {key: np.zeros((B, n, H, d)) for key in ("O_loc", "O_hist", "O_full")}
+    out.update({key: np.zeros((B, n, H)) for key in ("L_loc", "L_hist", "L_full")})
+    for b in range(B):
+        for h in range(H):
+            kl, vl = k[b, loc_idx, h, :], v[b, loc_idx, h, :]
+            kh, vh = k[b, hist_idx, h, :], v[b, hist_idx, h, :]
+            for r0 in range(0, n, row_block):
+                rr = rows[r0:r0 + row_block]
+                qq = np.asarray(q[b, rr, h, :], np.float64)
+                o_l, l_l = attend_group(qq, kl, vl, scale)
+                o_h, l_h = attend_group(qq, kh, vh, scale)
+                o_f, l_f = lse_merge(o_l, l_l, o_h, l_h)
+                sl = slice(r0, r0 + len(rr))
+                out["O_loc"][b, sl, h], out["L_loc"][b, sl, h] = o_l, l_l
+                out["O_hist"][b, sl, h], out["L_hist"][b, sl, h] = o_h, l_h
+                out["O_full"][b, sl, h], out["L_full"][b, sl, h] = o_f, l_f
+    return out
+
+
+def full_attention(shape, q, k, v, scale: float = None, rows: Sequence[int] = None,
+                   row_block: int = 512) -> Tuple[np.ndarray, np.ndarray]:
+    """Monolithic softmax attention over every KV frame (the F-layer path after the switch).
+
+    F-layers "continue using the full-context path" [EN-notes, Key Designs 3;
+    DE-summary 2, "Speichereffiziente Inferenz"].
+    """
+    d = q.shape[-1]
+    scale = 1.0 / math.sqrt(d) if not scale else scale
+    B, Lq, H, _ = q.shape
+    rows = np.arange(Lq) if rows is None else np.asarray(rows)
+    n = len(rows)
+    O = np.zeros((B, n, H, d))
+    L = np.zeros((B, n, H))
+    for b in range(B):
+        for h in range(H):
+            for r0 in range(0, n, row_block):
+                rr = rows[r0:r0 + row_block]
+                o, l = attend_group(q[b, rr, h, :], k[b, :, h, :], v[b, :, h, :], scale)
+                O[b, r0:r0 + len(rr), h], L[b, r0:r0 + len(rr), h] = o, l
+    return O, L
+
+
+def heads_to_rows(O: np.ndarray) -> np.ndarray:
+    """[B, n, H, d] -> [B*n, H*d]: one activation row per query token, heads concatenated."""
+    B, n, H, d = O.shape
+    return np.asarray(O, np.float64).reshape(B * n, H * d)
+
+
+# ---------------------------------------------------------------------------
+# absorption statistics and the closed-form solve
+# [EN-notes, Key Designs 2; DE-summary 2, "Layer Absorb"]
+# ---------------------------------------------------------------------------
+def residual(A_loc: np.ndarray, A_full: np.ndarray, W: np.ndarray) -> np.ndarray:
+    """Projected output residual R = (A_full - A_loc) W, taken before the output projection."""
+    return (np.asarray(A_full, np.float64) - np.asarray(A_loc, np.float64)) @ np.asarray(W, np.float64)
+
+
+def absorption_stats(A_loc: np.ndarray, A_full: np.ndarray, W: np.ndarray):
+    """Sufficient statistics of the warmup rows: G = A_loc^T A_loc, C = A_loc^T R, r2 = ||R||_F^2.
+
+    The pages accumulate "activation outer products and activation-residual
+    cross-statistics" during the forward passes [EN-notes, Key Designs 2]; the
+    DE summary's closed form uses exactly G and C.
+    """
+    A = np.asarray(A_loc, np.float64)
+    R = residual(A, A_full, W)
+    return A.T @ A, A.T @ R, float(np.sum(R * R))
+
+
+def ridge_lambda(G: np.ndarray, lam: float, relative: bool) -> float:
+    """lambda as given, or lam * tr(G) / D when ``relative``."""
+    return float(lam) * float(np.trace(G)) / G.shape[0] if relative else float(lam)
+
+
+def cholesky_lower(A: np.ndarray) -> np.ndarray:
+    """Lower Cholesky factor of a symmetric positive-definite matrix (LAPACK potrf)."""
+    return np.linalg.cholesky(np.asarray(A, np.float64))
+
+
+def ridge_solve(G: np.ndarray, C: np.ndarray, lam: float) -> np.ndarray:
+    """Delta W = (G + lambda I)^-1 C  [DE-summary 2, "Layer Absorb"].
+
+    The minimiser of ||A_loc (W + dW) - A_full W||^2 + lambda ||dW||^2 is
+    dW = (A_loc^T A_loc + lambda I)^-1 A_loc^T (A_full - A_loc) W.  The "single
+    D x D matrix inversion" [EN-notes, Key Designs 2] is applied as a Cholesky
+    factorisation LL^T = G + lambda I and two triangular solves.
+    """
+    G = np.asarray(G, np.float64)
+    M = G + lam * np.eye(G.shape[0])
+    Lf = cholesky_lower(M)
+    Y = scipy.linalg.solve_triangular(Lf, np.asarray(C, np.float64), lower=True)
+    return scipy.linalg.solve_triangular(Lf.T, Y, lower=False)
+
+
+def eps_direct(A_loc: np.ndarray, A_full: np.ndarray, W: np.ndarray, dW: np.ndarray) -> float:
+    """epsilon = ||A_loc (W + dW) - A_full W||_F^2 over all warmup rows [EN-notes, Key Designs 2]."""
+    A = np.asarray(A_loc, np.float64)
+    W = np.asarray(W, np.float64)
+    E = A @ (W + np.asarray(dW, np.float64)) - np.asarray(A_full, np.float64) @ W
+    return float(np.sum(E * E))
+
+
+def eps_from_stats(G: np.ndarray, C: np.ndarray, r2: float, dW: np.ndarray) -> float:
+    """The same epsilon expanded over the statistics: r2 - 2<dW, C> + <dW, G dW>.
+
+    ||A dW - R||^2 = ||R||^2 - 2 tr(dW^T A^T R) + tr(dW^T A^T A dW).
+    """
+    dW = np.asarray(dW, np.float64)
+    return float(r2 - 2.0 * np.sum(dW * C) + np.sum(dW * (np.asarray(G, np.float64) @ dW)))
+
+
+# ---------------------------------------------------------------------------
+# layer selection  [EN-notes, Key Designs 3; DE-summary 2, "Dynamische Layerauswahl"]
+# ---------------------------------------------------------------------------
+def num_selected(x: float, N: int) -> int:
+    """ISPA-x converts K = x N layers; read as floor(x N), never above the budget."""
+    return int(math.floor(x * N + 1e-9))
+
+
+def select_layers(eps: Sequence[float], K: int):
+    """Sort layers by increasing epsilon and take the K lowest as L-layers.
+
+    Ties go to the lower layer index (stable sort).  Returns (is_local uint8 [N],
+    idx int32 [K] ascending by layer index).
+    """
+    eps = np.asarray(eps, np.float64)
+    N = eps.shape[0]
+    order = sorted(range(N), key=lambda i: (eps[i], i))
+    chosen = sorted(order[:K])
+    is_local = np.zeros(N, np.uint8)
+    is_local[chosen] = 1
+    return is_local, np.array(chosen, np.int32)
+
+
+def kv_retained_fraction(x: float, hist_frac: float) -> float:
+    """KV kept relative to full caching when a fraction x of layers drops its history.
+
+    An L-layer keeps sink + current entries and evicts history; F-layers keep
+    everything [EN-notes, Key Designs 3].  With h = history / all KV entries of a
+    layer, the kept fraction is (1 - x) + x (1 - h) = 1 - x h.
+    """
+    return 1.0 - x * hist_frac
+
+
+# ---------------------------------------------------------------------------
+# post-switch L-layer  [DE-summary 2, "Speichereffiziente Inferenz"]
+# ---------------------------------------------------------------------------
+def local_projection(shape, q, k, v, W: np.ndarray, dW: np.ndarray = None, scale: float = None,
+                     rows: Sequence[int] = None) -> np.ndarray:
+    """Y = A_loc (W + dW): attention over sink + current only, projected with W_new = W + dW.
+
+    Returns Y [B, n, D_out].
+    """
+    d = q.shape[-1]
+    scale = 1.0 / math.sqrt(d) if not scale else scale
+    B, Lq, H, _ = q.shape
+    rows = np.arange(Lq) if rows is None else np.asarray(rows)
+    loc_idx = _local_rows(shape)
+    O = np.zeros((B, len(rows), H, d))
+    for b in range(B):
+        for h in range(H):
+            O[b, :, h], _ = attend_group(q[b, rows, h, :], k[b, loc_idx, h, :], v[b, loc_idx, h, :], scale)
+    Weff = np.asarray(W, np.float64) + (0.0 if dW is None else np.asarray(dW, np.float64))
+    return (heads_to_rows(O) @ Weff).reshape(B, len(rows), -1)
+
+
+# ---------------------------------------------------------------------------
+# one layer's warmup -> transition, and a whole model's selection
+# ---------------------------------------------------------------------------
+def absorb_layer(chunks: List[Dict[str, np.ndarray]], W: np.ndarray, lam: float, lam_relative: bool):
+    """Warmup over chunks of one layer, then its closed-form absorption.
+
+    ``chunks`` holds the split-attention outputs of every warmup chunk (dicts
+    from :func:`split_attention`).  Rows of all chunks are stacked (the
+    statistics are "accumulated during forward passes").  Returns G, C, r2,
+    lambda, dW, eps (direct form) and the stacked rows.
+    """
+    A_loc = np.concatenate([heads_to_rows(c["O_loc"]) for c in chunks], axis=0)
+    A_full = np.concatenate([heads_to_rows(c["O_full"]) for c in chunks], axis=0)
+    G, C, r2 = absorption_stats(A_loc, A_full, W)
+    lam_eff = ridge_lambda(G, lam, lam_relative)
+    dW = ridge_solve(G, C, lam_eff)
+    return dict(G=G, C=C, r2=r2, lam=lam_eff, dW=dW, eps=eps_direct(A_loc, A_full, W, dW),
+                A_loc=A_loc, A_full=A_full)
+
+
+def attention_flops(n_query: int, n_key: int, H: int, d: int) -> float:
+    """Dot-product FLOPs of one attention call: QK^T and PV, 2 flops per multiply-add."""
+    return 4.0 * n_query * n_key * H * d

@@ -1,0 +1,425 @@
+"""Pins of the fp64 oracle to facts fixed by the ISPA pages and by mathematics.
+
+No test here compares the oracle with itself: each one checks it against a
+brute-force computation written independently (pure-Python loops), a closed
+form, an invariant, a LAPACK/NumPy routine solving the same problem another
+way, or a value printed on the pages.  The mutation tests at the end plant a
+plausible mistake in a copy of an oracle function and check that a pin
+catches it.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import ispa_oracle as orc
+import synth_inputs as si
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------------------
+# brute-force softmax attention, independent of the oracle (pure Python)
+# ---------------------------------------------------------------------------
+def brute_attention(q, k, v, scale):
+    """Softmax attention of each query over all rows of k/v, with math.exp loops."""
+    n, d = len(q), len(q[0])
+    O = np.zeros((n, len(v[0]) if len(v) else d))
+    L = np.zeros(n)
+    for i in range(n):
+        s = [scale * sum(float(q[i][t]) * float(kj[t]) for t in range(d)) for kj in k]
+        if not s:
+            O[i] = 0.0
+            L[i] = -math.inf
+            continue
+        mx = max(s)
+        w = [math.exp(x - mx) for x in s]
+        tot = math.fsum(w)
+        for j, wj in enumerate(w):
+            O[i] += (wj / tot) * np.asarray(v[j], np.float64)
+        L[i] = mx + math.log(tot)
+    return O, L
+
+
+def _rand(g, *shape, std=1.0):
+    return g.standard_normal(shape) * std
+
+
+# ---------------------------------------------------------------------------
+# P1: per-group attention and the merge equal monolithic softmax
+# ---------------------------------------------------------------------------
+def check_group_vs_brute(attend, seed=0):
+    g = np.random.default_rng(seed)
+    ok = True
+    for n, m, d in [(3, 5, 4), (1, 1, 2), (4, 9, 8)]:
+        q, k, v = _rand(g, n, d), _rand(g, m, d), _rand(g, m, d)
+        scale = 1.0 / math.sqrt(d)
+        O, L = attend(q, k, v, scale)
+        Ob, Lb = brute_attention(q, k, v, scale)
+        ok &= np.allclose(O, Ob, rtol=1e-12, atol=1e-13) and np.allclose(L, Lb, rtol=1e-13, atol=1e-13)
+    return bool(ok)
+
+
+def test_group_attention_bruteforce():
+    assert check_group_vs_brute(orc.attend_group)
+
+
+def test_group_attention_closed_forms():
+    g = np.random.default_rng(1)
+    d, m = 8, 7
+    q = _rand(g, 3, d)
+    kvec = _rand(g, d)
+    k = np.tile(kvec, (m, 1))              # identical keys -> uniform weights
+    v = _rand(g, m, d)
+    O, L = orc.attend_group(q, k, v, 0.5)
+    s = 0.5 * (q @ kvec)
+    assert np.allclose(O, np.tile(v.mean(axis=0), (3, 1)), atol=1e-14)
+    assert np.allclose(L, s + math.log(m), atol=1e-13)
+    O1, L1 = orc.attend_group(q, k[:1], v[:1], 0.5)   # single key -> O = v, L = s
+    assert np.allclose(O1, np.tile(v[0], (3, 1)), atol=1e-15)
+    assert np.allclose(L1, s, atol=1e-15)
+    O0, L0 = orc.attend_group(q, k[:0], v[:0], 0.5)   # empty group
+    assert np.all(O0 == 0) and np.all(np.isneginf(L0))
+
+
+def check_merge_vs_monolithic(merge, seed=2):
+    """Random two-way splits of a key set: merged (O, L) == attention over the union."""
+    g = np.random.default_rng(seed)
+    ok = True
+    for trial in range(40):
+        d = int(g.choice([2, 4, 8]))
+        n, m = int(g.integers(1, 5)), int(g.integers(1, 40))
+        mult = [1.0, 30.0][trial % 2]      # x30 scores stress overflow handling
+        q, k, v = _rand(g, n, d) * mult, _rand(g, m, d), _rand(g, m, d)
+        perm = g.permutation(m)
+        cut = int(g.integers(0, m + 1))    # cut == 0 or m leaves one group empty
+        a, b = perm[:cut], perm[cut:]
+        oa, la = orc.attend_group(q, k[a], v[a], 0.3)
+        ob, lb = orc.attend_group(q, k[b], v[b], 0.3)
+        O, L = merge(oa, la, ob, lb)
+        Ob, Lb = brute_attention(q, k, v, 0.3)
+        ok &= np.allclose(O, Ob, rtol=1e-10, atol=1e-12) and np.allclose(L, Lb, rtol=1e-12, atol=1e-10)
+    return bool(ok)
+
+
+def test_merge_equals_monolithic_softmax():
+    assert check_merge_vs_monolithic(orc.lse_merge)
+
+
+def test_merge_dominant_history_and_empty_groups():
+    g = np.random.default_rng(3)
+    d = 4
+    q = _rand(g, 2, d)
+    k_loc, v_loc = _rand(g, 3, d), _rand(g, 3, d)
+    # history keys aligned with q and scaled so its LSE exceeds the local one by > 50 nats
+    k_hist = np.stack([q[0] * 60.0, q[1] * 60.0])
+    v_hist = _rand(g, 2, d)
+    ol, ll = orc.attend_group(q, k_loc, v_loc, 1.0)
+    oh, lh = orc.attend_group(q, k_hist, v_hist, 1.0)
+    assert np.all(lh - ll > 50)
+    O, L = orc.lse_merge(ol, ll, oh, lh)
+    Ob, Lb = brute_attention(q, np.vstack([k_loc, k_hist]), np.vstack([v_loc, v_hist]), 1.0)
+    assert np.allclose(O, Ob, atol=1e-12) and np.allclose(L, Lb, atol=1e-9)
+    # empty history: full == local exactly
+    e_o, e_l = np.zeros_like(ol), np.full(2, -np.inf)
+    O2, L2 = orc.lse_merge(ol, ll, e_o, e_l)
+    assert np.array_equal(O2, ol) and np.array_equal(L2, ll)
+    # both empty
+    O3, L3 = orc.lse_merge(e_o, e_l, e_o, e_l)
+    assert np.all(O3 == 0) and np.all(np.isneginf(L3))
+
+
+# ---------------------------------------------------------------------------
+# P2: merge symmetry and associativity
+# ---------------------------------------------------------------------------
+def test_merge_symmetry_and_associativity():
+    g = np.random.default_rng(4)
+    d, n = 8, 5
+    q = _rand(g, n, d)
+    groups = [(_rand(g, m, d), _rand(g, m, d)) for m in (3, 7, 11)]
+    parts = [orc.attend_group(q, k, v, 0.4) for k, v in groups]
+    ab = orc.lse_merge(*parts[0], *parts[1])
+    ba = orc.lse_merge(*parts[1], *parts[0])
+    assert np.allclose(ab[0], ba[0], atol=1e-15) and np.allclose(ab[1], ba[1], atol=1e-15)
+    left = orc.lse_merge(*ab, *parts[2])
+    bc = orc.lse_merge(*parts[1], *parts[2])
+    right = orc.lse_merge(*parts[0], *bc)
+    assert np.allclose(left[0], right[0], atol=1e-14) and np.allclose(left[1], right[1], atol=1e-13)
+    kall = np.vstack([k for k, _ in groups])
+    vall = np.vstack([v for _, v in groups])
+    Ob, Lb = brute_attention(q, kall, vall, 0.4)
+    assert np.allclose(left[0], Ob, atol=1e-12) and np.allclose(left[1], Lb, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# split attention over frame layouts: groups partition the KV (no frame twice)
+# ---------------------------------------------------------------------------
+def test_split_attention_layouts_bruteforce():
+    g = np.random.default_rng(5)
+    shapes = [si.random_groups_shape(g, max_frames=4, d=4, H=2, tpf=3, B=1) for _ in range(6)]
+    # first chunk of a video: the current chunk is the sink itself (union, no double count)
+    shapes.append(si.AttnShape(B=1, H=1, d=4, tpf=2, sink_frames=2, hist_begin=2, hist_end=2,
+                               cur_begin=0, cur_end=2, kv_frames=2))
+    # sink overlapping part of the current chunk
+    shapes.append(si.AttnShape(B=1, H=1, d=4, tpf=2, sink_frames=2, hist_begin=2, hist_end=2,
+                               cur_begin=1, cur_end=3, kv_frames=3))
+    for sh in shapes:
+        q = _rand(g, sh.B, sh.Lq, sh.H, sh.d)
+        k = _rand(g, sh.B, sh.Lkv, sh.H, sh.d)
+        v = _rand(g, sh.B, sh.Lkv, sh.H, sh.d)
+        out = orc.split_attention(sh, q, k, v)
+        frames_loc = sorted(set(range(sh.sink_frames)) | set(range(sh.cur_begin, sh.cur_end)))
+        rows_loc = [f * sh.tpf + t for f in frames_loc for t in range(sh.tpf)]
+        rows_hist = list(range(sh.hist_begin * sh.tpf, sh.hist_end * sh.tpf))
+        assert not set(rows_loc) & set(rows_hist)
+        for h in range(sh.H):
+            sc = 1.0 / math.sqrt(sh.d)
+            Ol, Ll = brute_attention(q[0, :, h], k[0, rows_loc, h], v[0, rows_loc, h], sc)
+            Of, Lf = brute_attention(q[0, :, h], k[0, rows_loc + rows_hist, h], v[0, rows_loc + rows_hist, h], sc)
+            assert np.allclose(out["O_loc"][0, :, h], Ol, atol=1e-12)
+            assert np.allclose(out["L_loc"][0, :, h], Ll, atol=1e-12)
+            assert np.allclose(out["O_full"][0, :, h], Of, atol=1e-12)
+            assert np.allclose(out["L_full"][0, :, h], Lf, atol=1e-12)
+        if sh.hist_end == sh.hist_begin:
+            assert np.all(np.isneginf(out["L_hist"])) and np.all(out["O_hist"] == 0)
+
+
+def test_full_attention_is_merge_of_groups():
+    sh = si.TINY
+    d = si.iid_qkv(sh, "f32", ("pin", "full"))
+    out = orc.split_attention(sh, d["q"], d["k"], d["v"])
+    O, L = orc.full_attention(sh, d["q"], d["k"], d["v"])
+    assert np.allclose(out["O_full"], O, atol=1e-13) and np.allclose(out["L_full"], L, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# P3: exact absorption; P4: normal equations; P5: library cross-checks
+# ---------------------------------------------------------------------------
+def _absorb_problem(seed, T=200, D=12, Dout=10):
+    g = np.random.default_rng(seed)
+    A_loc = _rand(g, T, D)
+    A_full = A_loc + 0.3 * _rand(g, T, D)
+    W = _rand(g, D, Dout) / math.sqrt(D)
+    return A_loc, A_full, W
+
+
+def check_exact_absorption(stats, solve, eps_fn, seed=6):
+    g = np.random.default_rng(seed)
+    T, D, Dout = 60, 8, 6
+    A_loc = _rand(g, T, D)
+    M = np.eye(D) + 0.4 * _rand(g, D, D)
+    A_full = A_loc @ M
+    W = _rand(g, D, Dout)
+    G, C, r2 = stats(A_loc, A_full, W)
+    dW = solve(G, C, 0.0)
+    e = eps_fn(A_loc, A_full, W, dW)
+    return bool(np.allclose(dW, (M - np.eye(D)) @ W, atol=1e-10) and e <= 1e-20 * r2 + 1e-24)
+
+
+def test_exact_absorption_closed_form():
+    assert check_exact_absorption(orc.absorption_stats, orc.ridge_solve, orc.eps_direct)
+
+
+def check_normal_equations(stats, solve, lam=0.7, seed=7):
+    A_loc, A_full, W = _absorb_problem(seed)
+    G, C, r2 = stats(A_loc, A_full, W)
+    dW = solve(G, C, lam)
+    R = (A_full - A_loc) @ W
+    resid = A_loc.T @ (A_loc @ dW - R) + lam * dW
+    return bool(np.abs(resid).max() <= 1e-9 * np.abs(A_loc.T @ R).max())
+
+
+def test_normal_equations():
+    assert check_normal_equations(orc.absorption_stats, orc.ridge_solve, lam=0.7)
+    assert check_normal_equations(orc.absorption_stats, orc.ridge_solve, lam=0.0)
+
+
+def test_ridge_against_lstsq_and_svd_filter():
+    A_loc, A_full, W = _absorb_problem(8)
+    G, C, r2 = orc.absorption_stats(A_loc, A_full, W)
+    R = (A_full - A_loc) @ W
+    dW0 = orc.ridge_solve(G, C, 0.0)
+    ls = np.linalg.lstsq(A_loc, R, rcond=None)[0]
+    assert np.allclose(dW0, ls, atol=1e-10)
+    lam = 3.0
+    U, s, Vt = np.linalg.svd(A_loc, full_matrices=False)
+    svd_sol = Vt.T @ np.diag(s / (s ** 2 + lam)) @ U.T @ R
+    assert np.allclose(orc.ridge_solve(G, C, lam), svd_sol, atol=1e-11)
+    big = orc.ridge_solve(G, C, 1e12)
+    assert np.abs(big).max() < 1e-8
+    assert orc.eps_direct(A_loc, A_full, W, big) == pytest.approx(r2, rel=1e-6)
+
+
+def test_stats_are_the_gram_and_cross_products():
+    # G and C written as explicit row sums (sum_t a_t a_t^T) in Python loops
+    A_loc, A_full, W = _absorb_problem(9, T=15, D=4, Dout=3)
+    G, C, r2 = orc.absorption_stats(A_loc, A_full, W)
+    Gb = np.zeros((4, 4)); Cb = np.zeros((4, 3)); r2b = 0.0
+    for t in range(15):
+        a = A_loc[t]
+        r = [sum((A_full[t, i] - A_loc[t, i]) * W[i, j] for i in range(4)) for j in range(3)]
+        for i in range(4):
+            for j in range(4):
+                Gb[i, j] += a[i] * a[j]
+            for j in range(3):
+                Cb[i, j] += a[i] * r[j]
+        r2b += sum(x * x for x in r)
+    assert np.allclose(G, Gb, atol=1e-12) and np.allclose(C, Cb, atol=1e-12)
+    assert r2 == pytest.approx(r2b, rel=1e-13)
+
+
+def test_cholesky_factor():
+    g = np.random.default_rng(10)
+    X = _rand(g, 30, 9)
+    A = X.T @ X + 0.1 * np.eye(9)
+    L = orc.cholesky_lower(A)
+    assert np.allclose(np.triu(L, 1), 0) and np.all(np.diag(L) > 0)
+    assert np.allclose(L @ L.T, A, atol=1e-12)
+
+
+def test_relative_lambda():
+    G = np.diag([1.0, 2.0, 3.0, 6.0])
+    assert orc.ridge_lambda(G, 1e-4, True) == pytest.approx(1e-4 * 12.0 / 4)
+    assert orc.ridge_lambda(G, 1e-3, False) == 1e-3
+
+
+# ---------------------------------------------------------------------------
+# P9: epsilon two ways
+# ---------------------------------------------------------------------------
+def test_eps_direct_equals_stats_form():
+    for seed, lam in [(11, 0.0), (12, 0.5), (13, 50.0)]:
+        A_loc, A_full, W = _absorb_problem(seed)
+        G, C, r2 = orc.absorption_stats(A_loc, A_full, W)
+        dW = orc.ridge_solve(G, C, lam)
+        e1 = orc.eps_direct(A_loc, A_full, W, dW)
+        e2 = orc.eps_from_stats(G, C, r2, dW)
+        assert e1 == pytest.approx(e2, rel=1e-10, abs=1e-10 * r2)
+        # the ridge solution never does worse than no correction
+        assert e1 <= r2 * (1 + 1e-12)
+
+
+# ---------------------------------------------------------------------------
+# P6: selection == brute force over subsets
+# ---------------------------------------------------------------------------
+def check_selection_bruteforce(select, seed=14):
+    g = np.random.default_rng(seed)
+    ok = True
+    for N in range(1, 9):
+        for _ in range(5):
+            eps = np.round(g.random(N) * 4) / 4         # frequent ties
+            for K in range(0, N + 1):
+                mask, idx = select(eps, K)
+                combos = list(itertools.combinations(range(N), K))
+                best_sum = min(float(np.sum(eps[list(c)])) for c in combos)
+                # minimal total epsilon; among equal totals the lower layer indices win
+                expected = min(c for c in combos if float(np.sum(eps[list(c)])) == best_sum)
+                ok &= list(idx) == list(expected) and int(mask.sum()) == K and all(mask[list(idx)] == 1)
+    return bool(ok)
+
+
+def test_selection_bruteforce():
+    assert check_selection_bruteforce(orc.select_layers)
+
+
+def test_num_selected():
+    assert orc.num_selected(0.5, 30) == 15 and orc.num_selected(0.5, 40) == 20
+    assert orc.num_selected(0.25, 30) == 7 and orc.num_selected(0.25, 40) == 10
+    assert orc.num_selected(0.0, 30) == 0 and orc.num_selected(0.7, 10) == 7
+    assert orc.num_selected(0.3, 10) == 3 and orc.num_selected(1.0, 7) == 7
+
+
+# ---------------------------------------------------------------------------
+# P7: KV accounting reproduces the pages' Table 2
+# ---------------------------------------------------------------------------
+def test_kv_retained_reproduces_table2():
+    with open(os.path.join(GOLDEN, "table2_kv_retained.json")) as f:
+        rows = json.load(f)["rows"]
+    by = {}
+    for r in rows:
+        by.setdefault(r["backbone"], []).append(r)
+    for backbone, rs in by.items():
+        # one history fraction h = 1 - 1/n (n an integer frame ratio) must explain every row
+        fits = []
+        for n in range(2, 40):
+            h = 1.0 - 1.0 / n
+            if all(abs(100 * orc.kv_retained_fraction(r["x"], h) - r["remaining_pct"]) <= 0.05 + 1e-9 for r in rs):
+                fits.append(n)
+        assert fits, backbone
+    # LongLive's three rows share one history fraction (11/12)
+    assert all(abs(100 * orc.kv_retained_fraction(r["x"], 11 / 12) - r["remaining_pct"]) <= 0.05
+               for r in by["LongLive"])
+
+
+# ---------------------------------------------------------------------------
+# P8: the split costs the same dot products as full attention
+# ---------------------------------------------------------------------------
+def test_flop_identity():
+    for sh in (si.SHAPE_1P3B, si.SHAPE_14B, si.TINY):
+        nl, nh = len(sh.local_rows), len(sh.hist_rows)
+        assert nl + nh == sh.Lkv
+        f_split = orc.attention_flops(sh.Lq, nl, sh.H, sh.d) + orc.attention_flops(sh.Lq, nh, sh.H, sh.d)
+        assert f_split == orc.attention_flops(sh.Lq, sh.Lkv, sh.H, sh.d)
+    assert orc.attention_flops(4680, 32760, 12, 128) == pytest.approx(0.942e12, rel=1e-3)
+
+
+def test_local_projection_definition():
+    sh = si.TINY
+    d = si.iid_qkv(sh, "f32", ("pin", "proj"))
+    W = si.projection_weight(sh.D, sh.D, ("pin", "proj"))
+    dW = 0.01 * np.random.default_rng(15).standard_normal((sh.D, sh.D))
+    Y = orc.local_projection(sh, d["q"], d["k"], d["v"], W, dW)
+    out = orc.split_attention(sh, d["q"], d["k"], d["v"])
+    assert np.allclose(Y[0], orc.heads_to_rows(out["O_loc"]) @ (W + dW), atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# mutation tests: plausible mistakes planted in copies of oracle functions
+# ---------------------------------------------------------------------------
+def test_mutant_plain_average_merge_is_caught():
+    def average_merge(oa, la, ob, lb):
+        L = np.logaddexp(la, lb)
+        return 0.5 * (oa + ob), L
+    assert not check_merge_vs_monolithic(average_merge)
+
+
+def test_mutant_swapped_merge_weights_is_caught():
+    def swapped(oa, la, ob, lb):
+        L = np.logaddexp(la, lb)
+        wa, wb = np.exp(la - L), np.exp(lb - L)
+        return wb[..., None] * oa + wa[..., None] * ob, L
+    assert not check_merge_vs_monolithic(swapped)
+
+
+def test_mutant_missing_scale_is_caught():
+    def unscaled(q, k, v, scale):
+        return orc.attend_group(q, k, v, 1.0)
+    assert not check_group_vs_brute(unscaled)
+
+
+def test_mutant_residual_sign_is_caught():
+    def wrong_sign_stats(A_loc, A_full, W):
+        G, C, r2 = orc.absorption_stats(A_loc, A_full, W)
+        return G, -C, r2
+    assert not check_exact_absorption(wrong_sign_stats, orc.ridge_solve, orc.eps_direct)
+
+
+def test_mutant_transposed_cross_stat_is_caught():
+    def transposed(A_loc, A_full, W):
+        R = (A_full - A_loc) @ W
+        return A_loc.T @ A_loc, (R.T @ A_loc).T[:, ::-1], float(np.sum(R * R))
+    assert not check_exact_absorption(transposed, orc.ridge_solve, orc.eps_direct)
+
+
+def test_mutant_dropped_lambda_is_caught():
+    def no_lambda(G, C, lam):
+        return orc.ridge_solve(G, C, 0.0)
+    assert not check_normal_equations(orc.absorption_stats, no_lambda, lam=0.7)
+
+
+def test_mutant_largest_eps_selection_is_caught():
+    def largest(eps, K):
+        return orc.select_layers(-np.asarray(eps), K)
+    assert not check_selection_bruteforce(largest)
