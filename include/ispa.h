@@ -1,0 +1,237 @@
+/*
+ * ispa.h -- C ABI of the ISPA hot path on NVIDIA B200 (sm_100a).
+ *
+ * ISPA (Instance-Specific Parametric Absorption) compresses the KV cache of an
+ * autoregressive video generator.  During a short warmup every layer runs a
+ * decomposable two-group attention, accumulates absorption statistics, and at
+ * the transition solves a closed-form ridge problem per layer; the K layers
+ * with the smallest reconstruction error then drop their history and project
+ * with W + dW.
+ *
+ * Passages cited below (all about arXiv 2607.00712, "Towards Memory-Efficient
+ * Autoregressive Video Generation via Instance-Specific Parametric Absorption"):
+ *   [EN-notes]   en.papernotes.org note, "Key Designs" 1-3 and "Loss & Training".
+ *   [DE-summary] gist.science/de, "Technisches Resümee", section 2 "Methodik"
+ *                ("Dual-Stream Warmup", "Layer Absorb", "Speichereffiziente
+ *                Inferenz", "Dynamische Layerauswahl").
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *     allocates no memory; calls that need scratch take a caller-owned
+ *     workspace whose size is given by the matching *_workspace_bytes query.
+ *   - Every call validates its arguments on the host before touching the GPU
+ *     and returns ISPA_ERR_INVALID_ARG / ISPA_ERR_UNSUPPORTED without launching
+ *     anything.  Otherwise it enqueues kernels on `stream` and returns without
+ *     synchronising (ISPA_ERR_CUDA if a launch fails).
+ *   - Conditions found on the device (a non positive-definite matrix, a bounded
+ *     wait that timed out) are recorded in a per-device error word and are
+ *     reported by ispa_check_device_error(), which synchronises the stream.
+ *   - Tensor pointers must be 16-byte aligned.  Row-major, C-contiguous layouts.
+ *   - ispa_last_error() returns a thread-local description of the last failure.
+ *   - Matrices act on row vectors: y = a W with W of shape [D_in, D_out].
+ */
+#ifndef ISPA_H
+#define ISPA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t.  NULL selects the legacy default stream. */
+typedef struct CUstream_st *ispa_stream_t;
+
+typedef enum {
+  ISPA_OK = 0,
+  ISPA_ERR_INVALID_ARG = 1, /* bad pointer, size, range or alignment           */
+  ISPA_ERR_UNSUPPORTED = 2, /* valid but not compiled (dtype / head_dim combo)  */
+  ISPA_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed       */
+  ISPA_ERR_NOT_SPD = 4,     /* G + lambda I had a non-positive Cholesky pivot    */
+  ISPA_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up                */
+} ispa_status;
+
+typedef enum { ISPA_F32 = 0, ISPA_BF16 = 1 } ispa_dtype;
+
+/* Arithmetic of the absorption-statistics GEMMs. */
+typedef enum {
+  ISPA_PREC_TF32 = 0, /* tcgen05 kind::tf32, operands rounded to nearest tf32, fp32 accumulate */
+  ISPA_PREC_F32 = 1   /* fp32 FFMA (CUDA cores), for fp32 workloads that need fp32 accuracy   */
+} ispa_precision;
+
+/* Returns a static version string. */
+const char *ispa_version(void);
+
+/* Thread-local text of the last error reported by this thread ("" if none). */
+const char *ispa_last_error(void);
+
+/*
+ * Synchronises `stream`, then reads and clears the error word of the current
+ * device.  Returns ISPA_OK, ISPA_ERR_NOT_SPD or ISPA_ERR_TIMEOUT (or
+ * ISPA_ERR_CUDA if the synchronisation itself failed).  `detail` (optional,
+ * host) receives the code's argument: the 1-based failing pivot for NOT_SPD,
+ * the kernel's wait-site id for TIMEOUT.
+ */
+ispa_status ispa_check_device_error(ispa_stream_t stream, int *detail);
+
+/* ------------------------------------------------------------------------- */
+/* Two-group attention                                                        */
+/* ------------------------------------------------------------------------- */
+/*
+ * Frame layout of one attention call.  Each instance's K/V buffer holds
+ * kv_frames * tokens_per_frame token rows, frame-ordered.  The queries are the
+ * current chunk: frames [cur_begin, cur_end), so Lq = (cur_end - cur_begin) *
+ * tokens_per_frame.
+ *   local group   = frames [0, sink_frames) united with [cur_begin, cur_end)
+ *                   (a frame in both counts once);
+ *   history group = frames [hist_begin, hist_end); it must not intersect the
+ *                   local group.  hist_begin == hist_end means no history.
+ * "The local group contains the initial sink frame and current frame; the
+ * historical group contains the intervening frames" [EN-notes, Key Designs 1].
+ * A post-switch F-layer (full context) is the same call with
+ * sink_frames = cur_begin and an empty history.
+ */
+typedef struct {
+  int B;                /* independent instances (batch)                        */
+  int H;                /* heads                                                */
+  int head_dim;         /* d: 128 for bf16 inputs; 32, 64 or 128 for fp32       */
+  int tokens_per_frame; /* tpf >= 1                                             */
+  int sink_frames;      /* local part 1: frames [0, sink_frames)                */
+  int hist_begin, hist_end;
+  int cur_begin, cur_end;
+  int kv_frames;        /* frames held per instance; row stride of K/V          */
+  ispa_dtype in_dtype;  /* dtype of Q, K, V                                     */
+  ispa_dtype out_dtype; /* dtype of the O outputs                               */
+  float softmax_scale;  /* <= 0 selects 1/sqrt(head_dim)                        */
+} ispa_attn_desc;
+
+/*
+ * Decomposable dual-stream attention [EN-notes, Key Designs 1; DE-summary 2,
+ * "Dual-Stream Warmup"]: the same queries attend separately to the local and
+ * the history group; each group emits its normalised output O and its
+ * log-sum-exp L = log sum_j exp(scale * q.k_j) (natural log, scale included).
+ * With o_full/lse_full given, the kernel also merges the two groups by their
+ * LSE into the full-context output (the fused form of ispa_lse_merge).
+ *
+ *   q          [B, Lq, H, d]                 in_dtype
+ *   k, v       [B, kv_frames*tpf, H, d]      in_dtype
+ *   o_loc      [B, Lq, H, d] out_dtype, lse_loc  [B, Lq, H] fp32   (required)
+ *   o_hist     [B, Lq, H, d] out_dtype, lse_hist [B, Lq, H] fp32   (both or neither)
+ *   o_full     [B, Lq, H, d] out_dtype, lse_full [B, Lq, H] fp32   (both or neither)
+ * An empty group yields O = 0 and L = -inf.  Compiled paths: bf16 in with
+ * head_dim 128 (tcgen05 tensor cores, fp32 accumulation) and fp32 in with
+ * head_dim 32/64/128 (fp32 CUDA cores).  Outputs may not alias inputs.
+ */
+ispa_status ispa_attn_split(const ispa_attn_desc *desc, const void *q, const void *k,
+                            const void *v, void *o_loc, float *lse_loc, void *o_hist,
+                            float *lse_hist, void *o_full, float *lse_full,
+                            ispa_stream_t stream);
+
+/*
+ * LSE-weighted merge of two disjoint groups' results [EN-notes, Key Designs 1]:
+ *   L = log(exp(L_a) + exp(L_b)),  O = exp(L_a - L) O_a + exp(L_b - L) O_b.
+ * o_* [rows, H, d] (o_dtype), lse_* [rows, H] fp32, rows = B * Lq.  Both
+ * groups empty (-inf) gives O = 0, L = -inf.  o_out may alias o_a or o_b
+ * (element-wise in place); lse_out must not overlap lse_a or lse_b.
+ * head_dim % 8 == 0.
+ */
+ispa_status ispa_lse_merge(int rows, int H, int head_dim, ispa_dtype o_dtype, const void *o_a,
+                           const float *lse_a, const void *o_b, const float *lse_b, void *o_out,
+                           float *lse_out, ispa_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* Absorption statistics                                                      */
+/* ------------------------------------------------------------------------- */
+size_t ispa_accum_stats_workspace_bytes(int T, int D, int Dout, ispa_precision prec);
+
+/*
+ * Warmup accumulation [EN-notes, Key Designs 2; DE-summary 2, "Layer Absorb"]:
+ *   R = (A_full - A_loc) W,   G += A_loc^T A_loc,   C += A_loc^T R,   r2 += ||R||_F^2
+ * for one batch of T activation rows taken immediately before the output
+ * projection.
+ *   a_loc, a_full [T, D] fp32 (D = H * head_dim, heads concatenated)
+ *   W             [D, Dout] fp32
+ *   G             [D, D] fp32, accumulated in place; ONLY the upper triangle
+ *                 (i <= j) is written and later read, the strict lower
+ *                 triangle is left as it was
+ *   C             [D, Dout] fp32, accumulated in place
+ *   r2            one double, accumulated in place
+ *   workspace     >= ispa_accum_stats_workspace_bytes(T, D, Dout, prec) bytes
+ * Zero G, C and r2 before the first batch of an instance.  T = 0 is a no-op.
+ * ISPA_PREC_TF32 needs D % 32 == 0 and Dout % 32 == 0.
+ */
+ispa_status ispa_accum_stats(int T, int D, int Dout, const float *a_loc, const float *a_full,
+                             const float *W, float *G, float *C, double *r2,
+                             ispa_precision prec, void *workspace, size_t workspace_bytes,
+                             ispa_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* Closed-form absorption                                                     */
+/* ------------------------------------------------------------------------- */
+size_t ispa_ridge_workspace_bytes(int D, int Dout);
+
+/*
+ * Closed-form ridge solve [DE-summary 2, "Layer Absorb"; EN-notes, Key Designs 2]:
+ *   dW  = (G + lambda I)^-1 C      (Cholesky LL^T = G + lambda I, two triangular solves)
+ *   eps = ||A_loc (W + dW) - A_full W||_F^2 = r2 - 2<dW, C> + <dW, G dW>
+ * lambda_eff = lambda, or lambda * trace(G) / D when lambda_relative != 0.
+ * refine_steps extra steps of iterative refinement with fp64 residuals
+ * (0 = plain fp32 solve).
+ *   G [D, D] fp32 (upper triangle read), C [D, Dout] fp32, r2 one double: inputs,
+ *   left unchanged.  dW [D, Dout] fp32 and eps (one double) are outputs.
+ * A non-positive pivot records ISPA_ERR_NOT_SPD (see ispa_check_device_error)
+ * and fills dW with NaN.  Asynchronous.
+ */
+ispa_status ispa_ridge_solve(int D, int Dout, const float *G, const float *C, const double *r2,
+                             float lambda, int lambda_relative, int refine_steps, float *dW,
+                             double *eps, void *workspace, size_t workspace_bytes,
+                             ispa_stream_t stream);
+
+/*
+ * Instance-specific layer selection [EN-notes, Key Designs 3; DE-summary 2,
+ * "Dynamische Layerauswahl"]: sort the N layers by increasing eps and take
+ * the K lowest as L-layers; equal eps goes to the lower layer index.
+ *   eps      [N] double (device), is_local [N] uint8 (1 = L-layer),
+ *   idx      [K] int32, the chosen layer indices in ascending order.
+ * 0 <= K <= N <= 4096.  NaN eps sorts after every number.
+ */
+ispa_status ispa_select_layers(int N, const double *eps, int K, unsigned char *is_local, int *idx,
+                               ispa_stream_t stream);
+
+/*
+ * W_new = W + dW for a layer that switches [DE-summary 2, "Speichereffiziente
+ * Inferenz"].  W [D, Dout] in w_dtype, dW [D, Dout] fp32, W_new [D, Dout] in
+ * out_dtype (rounded to nearest even).  W_new may alias W when the dtypes match.
+ */
+ispa_status ispa_absorb_weight(int D, int Dout, const void *W, ispa_dtype w_dtype, const float *dW,
+                               void *W_new, ispa_dtype out_dtype, ispa_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* Post-switch layer                                                          */
+/* ------------------------------------------------------------------------- */
+size_t ispa_attn_local_proj_workspace_bytes(const ispa_attn_desc *desc);
+
+/*
+ * Post-switch layer step [DE-summary 2, "Speichereffiziente Inferenz";
+ * EN-notes, Key Designs 3]: attention of the current chunk over the local group
+ * only (the history range of desc is ignored), then the output projection
+ *   y = A_loc W_proj,
+ * with W_proj = W + dW for an L-layer (from ispa_absorb_weight) or the original
+ * W for an F-layer (whose desc then sets sink_frames = cur_begin so that the
+ * local group spans every frame).
+ *   q, k, v   as for ispa_attn_split (bf16, head_dim 128)
+ *   W_proj    [D, Dout] bf16,  D = H * head_dim,  Dout % 16 == 0
+ *   y         [B, Lq, Dout] in y_dtype
+ *   workspace >= ispa_attn_local_proj_workspace_bytes(desc) (holds A_loc in bf16)
+ */
+ispa_status ispa_attn_local_proj(const ispa_attn_desc *desc, const void *q, const void *k,
+                                 const void *v, const void *W_proj, int Dout, void *y,
+                                 ispa_dtype y_dtype, void *workspace, size_t workspace_bytes,
+                                 ispa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ISPA_H */

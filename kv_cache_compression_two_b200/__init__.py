@@ -1,0 +1,203 @@
+"""Python binding of libispa, the B200 (sm_100a) ISPA hot path.
+
+Argument marshalling only: every step of the path runs in the CUDA kernels of
+``libispa.so`` (built in-tree by :mod:`kv_cache_compression_two_b200.build`).
+Importing this package fails loudly when the library is missing; there is no
+CPU or PyTorch fallback.
+
+Tensor arguments may be ``torch.Tensor`` objects (their ``data_ptr()`` is
+passed; the binding checks device, dtype and contiguity) or raw integer device
+addresses.  ``stream`` may be a ``torch.cuda.Stream``, a raw ``cudaStream_t``
+integer or ``None`` (the current torch stream when torch is initialised,
+otherwise the legacy default stream).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libispa.so")
+
+ISPA_OK, ISPA_ERR_INVALID_ARG, ISPA_ERR_UNSUPPORTED, ISPA_ERR_CUDA, ISPA_ERR_NOT_SPD, ISPA_ERR_TIMEOUT = range(6)
+ISPA_F32, ISPA_BF16 = 0, 1
+ISPA_PREC_TF32, ISPA_PREC_F32 = 0, 1
+
+STATUS_NAMES = {0: "ISPA_OK", 1: "ISPA_ERR_INVALID_ARG", 2: "ISPA_ERR_UNSUPPORTED", 3: "ISPA_ERR_CUDA",
+                4: "ISPA_ERR_NOT_SPD", 5: "ISPA_ERR_TIMEOUT"}
+
+# Every entry point declared in include/ispa.h.
+EXPORTED = ("ispa_version", "ispa_last_error", "ispa_check_device_error", "ispa_attn_split", "ispa_lse_merge",
+            "ispa_accum_stats_workspace_bytes", "ispa_accum_stats", "ispa_ridge_workspace_bytes", "ispa_ridge_solve",
+            "ispa_select_layers", "ispa_absorb_weight", "ispa_attn_local_proj_workspace_bytes",
+            "ispa_attn_local_proj")
+
+
+class IspaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class AttnDesc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("tokens_per_frame", ctypes.c_int), ("sink_frames", ctypes.c_int), ("hist_begin", ctypes.c_int),
+                ("hist_end", ctypes.c_int), ("cur_begin", ctypes.c_int), ("cur_end", ctypes.c_int),
+                ("kv_frames", ctypes.c_int), ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
+                ("softmax_scale", ctypes.c_float)]
+
+
+def attn_desc(shape, in_dtype: int, out_dtype: int, softmax_scale: float = 0.0) -> AttnDesc:
+    """Builds an AttnDesc from any object with the frame-layout attributes (B, H, d, tpf, ...)."""
+    return AttnDesc(shape.B, shape.H, shape.d, shape.tpf, shape.sink_frames, shape.hist_begin, shape.hist_end,
+                    shape.cur_begin, shape.cur_end, shape.kv_frames, in_dtype, out_dtype, softmax_scale)
+
+
+_lib = None
+_vp, _ci, _cf, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libispa.so (once).  Raises ImportError when it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libispa.so not found at {LIB_PATH}; build it with "
+                          "`python -m kv_cache_compression_two_b200.build` (needs nvcc)")
+    L = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "ispa_version": (ctypes.c_char_p, []),
+        "ispa_last_error": (ctypes.c_char_p, []),
+        "ispa_check_device_error": (_ci, [_vp, ctypes.POINTER(_ci)]),
+        "ispa_attn_split": (_ci, [ctypes.POINTER(AttnDesc)] + [_vp] * 9 + [_vp]),
+        "ispa_lse_merge": (_ci, [_ci, _ci, _ci, _ci, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+        "ispa_accum_stats_workspace_bytes": (_sz, [_ci, _ci, _ci, _ci]),
+        "ispa_accum_stats": (_ci, [_ci, _ci, _ci, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _vp, _sz, _vp]),
+        "ispa_ridge_workspace_bytes": (_sz, [_ci, _ci]),
+        "ispa_ridge_solve": (_ci, [_ci, _ci, _vp, _vp, _vp, _cf, _ci, _ci, _vp, _vp, _vp, _sz, _vp]),
+        "ispa_select_layers": (_ci, [_ci, _vp, _ci, _vp, _vp, _vp]),
+        "ispa_absorb_weight": (_ci, [_ci, _ci, _vp, _ci, _vp, _vp, _ci, _vp]),
+        "ispa_attn_local_proj_workspace_bytes": (_sz, [ctypes.POINTER(AttnDesc)]),
+        "ispa_attn_local_proj": (_ci, [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _ci, _vp, _ci, _vp, _sz, _vp]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def _ptr(x, *, dtype=None, name="tensor") -> Optional[int]:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    import torch
+    if not isinstance(x, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, an int address or None")
+    if not x.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if not x.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if dtype is not None and x.dtype not in dtype:
+        raise ValueError(f"{name}: dtype {x.dtype} not in {dtype}")
+    return x.data_ptr()
+
+
+def _stream(s) -> Optional[int]:
+    if s is None:
+        try:
+            import torch
+            if torch.cuda.is_available() and torch.cuda.is_initialized():
+                return torch.cuda.current_stream().cuda_stream
+        except Exception:
+            pass
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(status: int) -> None:
+    if status != ISPA_OK:
+        raise IspaError(status, lib().ispa_last_error().decode(errors="replace"))
+
+
+def _dt(t) -> int:
+    import torch
+    return ISPA_BF16 if t.dtype == torch.bfloat16 else ISPA_F32
+
+
+def version() -> str:
+    return lib().ispa_version().decode()
+
+
+def ispa_check_device_error(stream=None) -> int:
+    detail = ctypes.c_int(0)
+    _check(lib().ispa_check_device_error(_stream(stream), ctypes.byref(detail)))
+    return detail.value
+
+
+def ispa_attn_split(desc: AttnDesc, q, k, v, o_loc, lse_loc, o_hist=None, lse_hist=None, o_full=None, lse_full=None,
+                    stream=None) -> None:
+    _check(lib().ispa_attn_split(ctypes.byref(desc), _ptr(q, name="q"), _ptr(k, name="k"), _ptr(v, name="v"),
+                                 _ptr(o_loc, name="o_loc"), _ptr(lse_loc, name="lse_loc"), _ptr(o_hist, name="o_hist"),
+                                 _ptr(lse_hist, name="lse_hist"), _ptr(o_full, name="o_full"),
+                                 _ptr(lse_full, name="lse_full"), _stream(stream)))
+
+
+def ispa_lse_merge(rows: int, H: int, head_dim: int, o_dtype: int, o_a, lse_a, o_b, lse_b, o_out, lse_out,
+                   stream=None) -> None:
+    _check(lib().ispa_lse_merge(rows, H, head_dim, o_dtype, _ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b),
+                                _ptr(o_out), _ptr(lse_out), _stream(stream)))
+
+
+def ispa_accum_stats_workspace_bytes(T: int, D: int, Dout: int, prec: int = ISPA_PREC_TF32) -> int:
+    return int(lib().ispa_accum_stats_workspace_bytes(T, D, Dout, prec))
+
+
+def ispa_accum_stats(T: int, D: int, Dout: int, a_loc, a_full, W, G, C, r2, prec: int = ISPA_PREC_TF32,
+                     workspace=None, workspace_bytes: int = 0, stream=None) -> None:
+    if workspace is not None and not isinstance(workspace, int):
+        workspace_bytes = workspace_bytes or workspace.numel() * workspace.element_size()
+    _check(lib().ispa_accum_stats(T, D, Dout, _ptr(a_loc), _ptr(a_full), _ptr(W), _ptr(G), _ptr(C), _ptr(r2), prec,
+                                  _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def ispa_ridge_workspace_bytes(D: int, Dout: int) -> int:
+    return int(lib().ispa_ridge_workspace_bytes(D, Dout))
+
+
+def ispa_ridge_solve(D: int, Dout: int, G, C, r2, lam: float, lambda_relative: bool, refine_steps: int, dW, eps,
+                     workspace, workspace_bytes: int = 0, stream=None) -> None:
+    if workspace is not None and not isinstance(workspace, int):
+        workspace_bytes = workspace_bytes or workspace.numel() * workspace.element_size()
+    _check(lib().ispa_ridge_solve(D, Dout, _ptr(G), _ptr(C), _ptr(r2), float(lam), int(bool(lambda_relative)),
+                                  int(refine_steps), _ptr(dW), _ptr(eps), _ptr(workspace), workspace_bytes,
+                                  _stream(stream)))
+
+
+def ispa_select_layers(N: int, eps, K: int, is_local, idx, stream=None) -> None:
+    _check(lib().ispa_select_layers(N, _ptr(eps), K, _ptr(is_local), _ptr(idx), _stream(stream)))
+
+
+def ispa_absorb_weight(D: int, Dout: int, W, w_dtype: int, dW, W_new, out_dtype: int, stream=None) -> None:
+    _check(lib().ispa_absorb_weight(D, Dout, _ptr(W), w_dtype, _ptr(dW), _ptr(W_new), out_dtype, _stream(stream)))
+
+
+def ispa_attn_local_proj_workspace_bytes(desc: AttnDesc) -> int:
+    return int(lib().ispa_attn_local_proj_workspace_bytes(ctypes.byref(desc)))
+
+
+def ispa_attn_local_proj(desc: AttnDesc, q, k, v, W_proj, Dout: int, y, y_dtype: int, workspace,
+                         workspace_bytes: int = 0, stream=None) -> None:
+    if workspace is not None and not isinstance(workspace, int):
+        workspace_bytes = workspace_bytes or workspace.numel() * workspace.element_size()
+    _check(lib().ispa_attn_local_proj(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(W_proj), Dout, _ptr(y),
+                                      y_dtype, _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+lib()

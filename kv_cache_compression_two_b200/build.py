@@ -1,0 +1,104 @@
+"""Builds libispa.so in-tree for sm_100a with nvcc.
+
+Every .cu file under csrc/ is compiled in parallel to an object under _build/,
+then linked with the static CUDA runtime into ``libispa.so`` next to this file.
+Objects are rebuilt when their source, a header or the flags change.
+
+    python -m kv_cache_compression_two_b200.build [--force] [--verbose]
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures
+import glob
+import hashlib
+import os
+import shutil
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+CSRC = os.path.join(HERE, "csrc")
+BUILD = os.path.join(HERE, "_build")
+LIB = os.path.join(HERE, "libispa.so")
+
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",
+                     "-I" + os.path.join(ROOT, "include"), "-Xptxas", "-warn-spills"]
+
+
+def nvcc() -> str:
+    for cand in (os.environ.get("NVCC"), shutil.which("nvcc"), "/usr/local/cuda/bin/nvcc"):
+        if cand and os.path.exists(cand):
+            return cand
+    raise RuntimeError("nvcc not found; the CUDA toolkit is required to build libispa")
+
+
+def _digest(paths, extra: str) -> str:
+    h = hashlib.sha256(extra.encode())
+    for p in sorted(paths):
+        with open(p, "rb") as f:
+            h.update(p.encode())
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def build(force: bool = False, verbose: bool = False, jobs: int = 0) -> str:
+    """Compiles (if needed) and returns the path of libispa.so."""
+    os.makedirs(BUILD, exist_ok=True)
+    sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    headers = sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) +
+                     glob.glob(os.path.join(ROOT, "include", "*.h")))
+    flags_key = " ".join(NVCC_FLAGS)
+    header_key = _digest(headers, flags_key)
+    compiler = nvcc()
+
+    def compile_one(src: str) -> str:
+        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        stamp = obj + ".key"
+        key = _digest([src], header_key)
+        if not force and os.path.exists(obj) and os.path.exists(stamp) and open(stamp).read() == key:
+            return obj
+        cmd = [compiler] + NVCC_FLAGS + ["-c", src, "-o", obj]
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        res = subprocess.run(cmd, capture_output=True, text=True)
+        if res.returncode != 0:
+            raise RuntimeError(f"nvcc failed on {os.path.basename(src)}:\n{res.stderr}")
+        if verbose and res.stderr.strip():
+            print(res.stderr, flush=True)
+        with open(stamp, "w") as f:
+            f.write(key)
+        return obj
+
+    n = jobs or min(len(sources), os.cpu_count() or 4)
+    with concurrent.futures.ThreadPoolExecutor(max_workers=n) as ex:
+        objs = list(ex.map(compile_one, sources))
+    link_key = _digest(objs, flags_key)
+    stamp = LIB + ".key"
+    if force or not os.path.exists(LIB) or not os.path.exists(stamp) or open(stamp).read() != link_key:
+        tmp = LIB + ".tmp"
+        cmd = [compiler] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs + ["-lpthread", "-ldl", "-lrt"]
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        res = subprocess.run(cmd, capture_output=True, text=True)
+        if res.returncode != 0:
+            raise RuntimeError(f"link failed:\n{res.stderr}")
+        os.replace(tmp, LIB)
+        with open(stamp, "w") as f:
+            f.write(link_key)
+    return LIB
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("--verbose", action="store_true")
+    args = ap.parse_args(argv)
+    print(build(force=args.force, verbose=args.verbose))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

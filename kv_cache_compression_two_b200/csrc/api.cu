@@ -1,0 +1,335 @@
+// api.cu -- the extern "C" entry points of libispa: argument validation,
+// group-range normalisation, error reporting and dispatch to the kernels.
+#include <math.h>
+#include <mutex>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "internal.h"
+
+// Per-device error word: [0] ispa_status of the first device-side failure, [1] its detail.
+__device__ int g_ispa_device_error[2];
+
+namespace ispa {
+
+static thread_local char t_last_error[512] = "";
+
+ispa_status fail(ispa_status st, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof(t_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+ispa_status cuda_status(cudaError_t e, const char *what) {
+  if (e == cudaSuccess) return ISPA_OK;
+  return fail(ISPA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int *g_err_addr[kMaxDevices] = {};
+int g_sms[kMaxDevices] = {};
+long long g_wait_limit_ns = 2000000000LL;  // 2 s per device-side wait
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+}  // namespace
+
+ispa_status device_err(DevErr *out) {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return fail(ISPA_ERR_CUDA, "no current CUDA device");
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_err_addr[dev]) {
+    void *p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_ispa_device_error);
+    if (e != cudaSuccess) return cuda_status(e, "cudaGetSymbolAddress(error word)");
+    g_err_addr[dev] = static_cast<int *>(p);
+  }
+  out->word = g_err_addr[dev];
+  out->limit_ns = g_wait_limit_ns;
+  return ISPA_OK;
+}
+
+int sm_count() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  if (!g_sms[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    g_sms[dev] = n > 0 ? n : 148;
+  }
+  return g_sms[dev];
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+ispa_status make_tmap(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *base, const uint64_t *dims,
+                      const uint64_t *strides_bytes, const uint32_t *box, CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(ISPA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint64_t d[5], st[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) st[i] = strides_bytes[i];
+  CUresult r = fn(m, dt, (cuuint32_t)rank, const_cast<void *>(base), d, st, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(ISPA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return ISPA_OK;
+}
+
+}  // namespace ispa
+
+using namespace ispa;
+
+namespace {
+
+bool dtype_ok(ispa_dtype d) { return d == ISPA_F32 || d == ISPA_BF16; }
+
+// Validates an attention descriptor and turns frame ranges into token ranges.
+ispa_status attn_ranges(const ispa_attn_desc *d, GroupRanges *g, float *scale) {
+  if (!d) return fail(ISPA_ERR_INVALID_ARG, "desc is NULL");
+  if (d->B < 1 || d->H < 1 || d->tokens_per_frame < 1)
+    return fail(ISPA_ERR_INVALID_ARG, "B, H and tokens_per_frame must be >= 1");
+  if (d->head_dim != 32 && d->head_dim != 64 && d->head_dim != 128)
+    return fail(ISPA_ERR_INVALID_ARG, "head_dim must be 32, 64 or 128 (got %d)", d->head_dim);
+  if (!dtype_ok(d->in_dtype) || !dtype_ok(d->out_dtype)) return fail(ISPA_ERR_INVALID_ARG, "bad dtype");
+  const int F = d->kv_frames;
+  if (F < 1) return fail(ISPA_ERR_INVALID_ARG, "kv_frames must be >= 1");
+  if (d->sink_frames < 0 || d->sink_frames > F) return fail(ISPA_ERR_INVALID_ARG, "sink_frames out of [0, kv_frames]");
+  if (!(0 <= d->cur_begin && d->cur_begin < d->cur_end && d->cur_end <= F))
+    return fail(ISPA_ERR_INVALID_ARG, "current chunk [%d, %d) invalid for kv_frames %d", d->cur_begin, d->cur_end, F);
+  if (!(0 <= d->hist_begin && d->hist_begin <= d->hist_end && d->hist_end <= F))
+    return fail(ISPA_ERR_INVALID_ARG, "history [%d, %d) invalid for kv_frames %d", d->hist_begin, d->hist_end, F);
+  const bool hist = d->hist_end > d->hist_begin;
+  if (hist && (d->hist_begin < d->sink_frames || (d->hist_begin < d->cur_end && d->cur_begin < d->hist_end)))
+    return fail(ISPA_ERR_INVALID_ARG, "history group overlaps the local group");
+  const long long tpf = d->tokens_per_frame;
+  if ((long long)F * tpf > (1LL << 30) || (long long)d->B * F * tpf * d->H * d->head_dim > (1LL << 40))
+    return fail(ISPA_ERR_INVALID_ARG, "tensor too large");
+  // local = [0, S) u [cb, ce), merged when they touch
+  int lb[2], le[2], n = 0;
+  const int S = d->sink_frames, cb = d->cur_begin, ce = d->cur_end;
+  if (S > 0) {
+    if (cb <= S) {
+      lb[n] = 0;
+      le[n++] = ce > S ? ce : S;
+    } else {
+      lb[n] = 0;
+      le[n++] = S;
+      lb[n] = cb;
+      le[n++] = ce;
+    }
+  } else {
+    lb[n] = cb;
+    le[n++] = ce;
+  }
+  g->n_loc = n;
+  for (int i = 0; i < n; ++i) {
+    g->loc_begin[i] = (int)(lb[i] * tpf);
+    g->loc_end[i] = (int)(le[i] * tpf);
+  }
+  g->hist_begin = (int)(d->hist_begin * tpf);
+  g->hist_end = (int)(d->hist_end * tpf);
+  g->q_begin = (int)(cb * tpf);
+  g->Lq = (int)((ce - cb) * tpf);
+  g->Lkv = (int)(F * tpf);
+  *scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.f / sqrtf((float)d->head_dim);
+  if (!isfinite(*scale)) return fail(ISPA_ERR_INVALID_ARG, "softmax_scale must be finite");
+  return ISPA_OK;
+}
+
+bool ptr_ok(const void *p) { return p != nullptr && aligned16(p); }
+
+}  // namespace
+
+extern "C" {
+
+const char *ispa_version(void) { return "ispa-b200 0.1 (sm_100a)"; }
+
+const char *ispa_last_error(void) { return t_last_error; }
+
+ispa_status ispa_check_device_error(ispa_stream_t stream, int *detail) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_status(e, "stream synchronize");
+  DevErr de;
+  ispa_status st = device_err(&de);
+  if (st != ISPA_OK) return st;
+  int host[2] = {0, 0};
+  e = cudaMemcpy(host, de.word, sizeof(host), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_status(e, "read device error word");
+  if (host[0] != 0) {
+    const int zero[2] = {0, 0};
+    cudaMemcpy(de.word, zero, sizeof(zero), cudaMemcpyHostToDevice);
+  }
+  if (detail) *detail = host[1];
+  if (host[0] == ISPA_ERR_NOT_SPD) return fail(ISPA_ERR_NOT_SPD, "G + lambda I is not positive definite (pivot %d)", host[1]);
+  if (host[0] == ISPA_ERR_TIMEOUT) return fail(ISPA_ERR_TIMEOUT, "device-side wait timed out (site %d)", host[1]);
+  if (host[0] != 0) return fail(ISPA_ERR_CUDA, "device error code %d", host[0]);
+  return ISPA_OK;
+}
+
+ispa_status ispa_attn_split(const ispa_attn_desc *desc, const void *q, const void *k, const void *v, void *o_loc,
+                            float *lse_loc, void *o_hist, float *lse_hist, void *o_full, float *lse_full,
+                            ispa_stream_t stream) {
+  GroupRanges g;
+  float scale;
+  ispa_status st = attn_ranges(desc, &g, &scale);
+  if (st != ISPA_OK) return st;
+  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v)) return fail(ISPA_ERR_INVALID_ARG, "q, k, v must be 16-byte aligned device pointers");
+  if (!ptr_ok(o_loc) || !ptr_ok(lse_loc)) return fail(ISPA_ERR_INVALID_ARG, "o_loc and lse_loc are required (16-byte aligned)");
+  if ((o_hist == nullptr) != (lse_hist == nullptr)) return fail(ISPA_ERR_INVALID_ARG, "o_hist and lse_hist: both or neither");
+  if ((o_full == nullptr) != (lse_full == nullptr)) return fail(ISPA_ERR_INVALID_ARG, "o_full and lse_full: both or neither");
+  if ((o_hist && !ptr_ok(o_hist)) || (lse_hist && !ptr_ok(lse_hist)) || (o_full && !ptr_ok(o_full)) ||
+      (lse_full && !ptr_ok(lse_full)))
+    return fail(ISPA_ERR_INVALID_ARG, "outputs must be 16-byte aligned");
+  if (desc->in_dtype == ISPA_BF16) {
+    if (desc->head_dim != 128) return fail(ISPA_ERR_UNSUPPORTED, "bf16 attention is compiled for head_dim 128 only");
+    return launch_attn_tc(*desc, g, scale, q, k, v, o_loc, lse_loc, o_hist, lse_hist, o_full, lse_full,
+                          (cudaStream_t)stream);
+  }
+  return launch_attn_simt(*desc, g, scale, (const float *)q, (const float *)k, (const float *)v, o_loc, lse_loc, o_hist,
+                          lse_hist, o_full, lse_full, (cudaStream_t)stream);
+}
+
+ispa_status ispa_lse_merge(int rows, int H, int head_dim, ispa_dtype o_dtype, const void *o_a, const float *lse_a,
+                           const void *o_b, const float *lse_b, void *o_out, float *lse_out, ispa_stream_t stream) {
+  if (rows < 0 || H < 1 || head_dim < 8 || head_dim % 8 != 0 || !dtype_ok(o_dtype))
+    return fail(ISPA_ERR_INVALID_ARG, "rows >= 0, H >= 1, head_dim a positive multiple of 8");
+  if (rows == 0) return ISPA_OK;
+  if (o_dtype == ISPA_F32 && head_dim % 4 != 0) return fail(ISPA_ERR_INVALID_ARG, "head_dim");
+  if (!ptr_ok(o_a) || !ptr_ok(o_b) || !ptr_ok(o_out) || !lse_a || !lse_b || !lse_out)
+    return fail(ISPA_ERR_INVALID_ARG, "pointers must be non-NULL, O pointers 16-byte aligned");
+  const size_t n = (size_t)rows * H;
+  const char *lo = (const char *)lse_out;
+  auto overlap = [&](const float *p) { return lo < (const char *)(p + n) && (const char *)p < lo + n * 4; };
+  if (overlap(lse_a) || overlap(lse_b)) return fail(ISPA_ERR_INVALID_ARG, "lse_out must not overlap lse_a or lse_b");
+  return launch_lse_merge(rows, H, head_dim, o_dtype, o_a, lse_a, o_b, lse_b, o_out, lse_out, (cudaStream_t)stream);
+}
+
+size_t ispa_accum_stats_workspace_bytes(int T, int D, int Dout, ispa_precision prec) {
+  if (T < 0 || D < 1 || Dout < 1) return 0;
+  return stats_workspace_bytes(T, D, Dout, prec);
+}
+
+ispa_status ispa_accum_stats(int T, int D, int Dout, const float *a_loc, const float *a_full, const float *W, float *G,
+                             float *C, double *r2, ispa_precision prec, void *workspace, size_t workspace_bytes,
+                             ispa_stream_t stream) {
+  if (T < 0 || D < 1 || Dout < 1) return fail(ISPA_ERR_INVALID_ARG, "T >= 0, D >= 1, Dout >= 1");
+  if (prec != ISPA_PREC_TF32 && prec != ISPA_PREC_F32) return fail(ISPA_ERR_INVALID_ARG, "bad precision");
+  if (prec == ISPA_PREC_TF32 && (D % 32 != 0 || Dout % 32 != 0))
+    return fail(ISPA_ERR_INVALID_ARG, "ISPA_PREC_TF32 needs D and Dout multiples of 32");
+  if ((long long)T * D > (1LL << 34) || (long long)D * Dout > (1LL << 31))
+    return fail(ISPA_ERR_INVALID_ARG, "sizes too large");
+  if (!ptr_ok(a_loc) || !ptr_ok(a_full) || !ptr_ok(W) || !ptr_ok(G) || !ptr_ok(C) || !r2)
+    return fail(ISPA_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
+  if (T == 0) return ISPA_OK;
+  const size_t need = stats_workspace_bytes(T, D, Dout, prec);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return fail(ISPA_ERR_INVALID_ARG, "workspace needs %zu bytes (16-byte aligned)", need);
+  return launch_stats(T, D, Dout, a_loc, a_full, W, G, C, r2, prec, workspace, (cudaStream_t)stream);
+}
+
+size_t ispa_ridge_workspace_bytes(int D, int Dout) {
+  if (D < 1 || Dout < 1) return 0;
+  return ridge_workspace_bytes(D, Dout);
+}
+
+ispa_status ispa_ridge_solve(int D, int Dout, const float *G, const float *C, const double *r2, float lambda,
+                             int lambda_relative, int refine_steps, float *dW, double *eps, void *workspace,
+                             size_t workspace_bytes, ispa_stream_t stream) {
+  if (D < 1 || Dout < 1 || D > 32768 || (long long)D * Dout > (1LL << 31))
+    return fail(ISPA_ERR_INVALID_ARG, "1 <= D <= 32768, Dout >= 1");
+  if (!(lambda >= 0.f) || !isfinite(lambda)) return fail(ISPA_ERR_INVALID_ARG, "lambda must be finite and >= 0");
+  if (refine_steps < 0 || refine_steps > 16) return fail(ISPA_ERR_INVALID_ARG, "refine_steps in [0, 16]");
+  if (!ptr_ok(G) || !ptr_ok(C) || !r2 || !ptr_ok(dW) || !eps)
+    return fail(ISPA_ERR_INVALID_ARG, "pointers must be non-NULL, matrices 16-byte aligned");
+  const size_t need = ridge_workspace_bytes(D, Dout);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return fail(ISPA_ERR_INVALID_ARG, "workspace needs %zu bytes (16-byte aligned)", need);
+  return launch_ridge(D, Dout, G, C, r2, lambda, lambda_relative, refine_steps, dW, eps, workspace,
+                      (cudaStream_t)stream);
+}
+
+ispa_status ispa_select_layers(int N, const double *eps, int K, unsigned char *is_local, int *idx,
+                               ispa_stream_t stream) {
+  if (N < 0 || N > 4096 || K < 0 || K > N) return fail(ISPA_ERR_INVALID_ARG, "need 0 <= K <= N <= 4096");
+  if (N == 0) return ISPA_OK;
+  if (!eps || !is_local || (K > 0 && !idx)) return fail(ISPA_ERR_INVALID_ARG, "NULL pointer");
+  return launch_select(N, eps, K, is_local, idx, (cudaStream_t)stream);
+}
+
+ispa_status ispa_absorb_weight(int D, int Dout, const void *W, ispa_dtype w_dtype, const float *dW, void *W_new,
+                               ispa_dtype out_dtype, ispa_stream_t stream) {
+  if (D < 1 || Dout < 1 || ((long long)D * Dout) % 4 != 0 || (long long)D * Dout > (1LL << 34))
+    return fail(ISPA_ERR_INVALID_ARG, "D * Dout must be a positive multiple of 4");
+  if (!dtype_ok(w_dtype) || !dtype_ok(out_dtype)) return fail(ISPA_ERR_INVALID_ARG, "bad dtype");
+  if (!ptr_ok(W) || !ptr_ok(dW) || !ptr_ok(W_new)) return fail(ISPA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (W_new == W && w_dtype != out_dtype) return fail(ISPA_ERR_INVALID_ARG, "in-place needs matching dtypes");
+  return launch_absorb_weight(D, Dout, W, w_dtype, dW, W_new, out_dtype, (cudaStream_t)stream);
+}
+
+size_t ispa_attn_local_proj_workspace_bytes(const ispa_attn_desc *desc) {
+  GroupRanges g;
+  float scale;
+  if (attn_ranges(desc, &g, &scale) != ISPA_OK) return 0;
+  const size_t a = (size_t)desc->B * g.Lq * desc->H * desc->head_dim * 2;
+  const size_t l = (size_t)desc->B * g.Lq * desc->H * 4;
+  return ((a + 255) & ~size_t(255)) + ((l + 255) & ~size_t(255));
+}
+
+ispa_status ispa_attn_local_proj(const ispa_attn_desc *desc, const void *q, const void *k, const void *v,
+                                 const void *W_proj, int Dout, void *y, ispa_dtype y_dtype, void *workspace,
+                                 size_t workspace_bytes, ispa_stream_t stream) {
+  GroupRanges g;
+  float scale;
+  ispa_status st = attn_ranges(desc, &g, &scale);
+  if (st != ISPA_OK) return st;
+  if (desc->in_dtype != ISPA_BF16 || desc->head_dim != 128)
+    return fail(ISPA_ERR_UNSUPPORTED, "post-switch projection is compiled for bf16 inputs with head_dim 128");
+  if (Dout < 16 || Dout % 16 != 0) return fail(ISPA_ERR_INVALID_ARG, "Dout must be a positive multiple of 16");
+  if (!dtype_ok(y_dtype)) return fail(ISPA_ERR_INVALID_ARG, "bad y dtype");
+  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(W_proj) || !ptr_ok(y))
+    return fail(ISPA_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
+  const size_t need = ispa_attn_local_proj_workspace_bytes(desc);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return fail(ISPA_ERR_INVALID_ARG, "workspace needs %zu bytes (16-byte aligned)", need);
+  ispa_attn_desc d = *desc;
+  d.hist_begin = d.hist_end = 0;
+  d.out_dtype = ISPA_BF16;
+  g.hist_begin = g.hist_end = 0;
+  const size_t a_bytes = (((size_t)d.B * g.Lq * d.H * d.head_dim * 2) + 255) & ~size_t(255);
+  void *a_loc = workspace;
+  float *lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + a_bytes);
+  st = launch_attn_tc(d, g, scale, q, k, v, a_loc, lse, nullptr, nullptr, nullptr, nullptr, (cudaStream_t)stream);
+  if (st != ISPA_OK) return st;
+  const int D = d.H * d.head_dim;
+  return launch_gemm_bf16(d.B * g.Lq, Dout, D, a_loc, W_proj, y, y_dtype, (cudaStream_t)stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,293 @@
+// gemm_tc.cuh -- tcgen05 GEMM building block (sm_100a).
+//
+// D[128 x 128 tile] = sum over K of A_tile * B_tile, accumulated in tensor
+// memory (128 lanes x 128 fp32 columns), with operands staged by TMA into
+// 128-byte-swizzled shared memory through a 4-stage mbarrier pipeline.
+//
+// Warp roles (192 threads):
+//   warp 0      TMA producer (one elected lane)
+//   warp 1      TMEM allocator + MMA issuer (one elected lane)
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator rows, then the
+//               problem-specific store (each thread owns one output row)
+//
+// Operand staging.  Every operand tile is 16 KB: 128 rows (M or N) by one
+// 128-byte swizzle span of K for K-major operands, or BK rows of K by 128
+// M/N elements (several 128-byte boxes) for MN-major operands.  Per stage the
+// MMA warp issues 4 instructions of K = 8 (tf32) or K = 16 (bf16).
+//
+// Up to two sub-problems that share A (same M, K) but have different B and
+// outputs run in one launch: blockIdx.x enumerates the tiles of problem 0,
+// then those of problem 1.  Tiles may be restricted to the upper triangle
+// (used for the symmetric Gram matrix).
+#pragma once
+
+#include "common.cuh"
+
+namespace ispa {
+namespace tcg {
+
+constexpr int BM = 128, BN = 128, STAGES = 4;
+constexpr int TILE_BYTES = 16384;
+constexpr int SMEM_BYTES = STAGES * 2 * TILE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int THREADS = 192;
+
+enum Epi : int {
+  EPI_STORE_F32 = 0,      // out = acc
+  EPI_STORE_TF32_SQ = 1,  // out = tf32_rn(acc); r2 += sum acc^2
+  EPI_ACCUM_F32 = 2,      // out += acc
+  EPI_STORE_BF16 = 3      // out = bf16_rn(acc)
+};
+
+struct SubProblem {
+  int N;          // columns of this problem's output
+  int tiles_n;    // ceil(N / BN)
+  int upper;      // 1: only tiles/elements with row <= col
+  int epi;        // Epi
+  void *out;      // [M, N] row-major, ld = ldo
+  long long ldo;
+};
+
+struct Params {
+  int M, K;
+  int tiles_m;
+  int n_tiles0;   // tiles of problem 0 (upper-triangle filter already applied)
+  int n_tiles;    // tiles of both problems (the grid size)
+  int kind_tf32;  // 1: kind::tf32 (fp32 operands), 0: kind::f16 with bf16 operands
+  int a_mn, b_mn; // operand majorness (1 = MN-major)
+  uint32_t idesc;
+  double *r2;     // EPI_STORE_TF32_SQ accumulator
+  SubProblem p[2];
+  DevErr err;
+};
+
+// Enumerates upper-triangle tiles (tile row tm <= tile col tn covering some i <= j).
+__host__ __device__ inline int upper_tile_count(int tiles_m, int tiles_n) {
+  int c = 0;
+  for (int tm = 0; tm < tiles_m; ++tm) {
+    const int first = (tm * BM) / BN;  // first tile column whose block has a col >= row
+    c += tiles_n > first ? tiles_n - first : 0;
+  }
+  return c;
+}
+
+__device__ inline void tile_coords(const Params &P, int t, int &prob, int &tm, int &tn) {
+  prob = t < P.n_tiles0 ? 0 : 1;
+  if (prob == 1) t -= P.n_tiles0;
+  const SubProblem &sp = P.p[prob];
+  if (!sp.upper) {
+    tm = t / sp.tiles_n;
+    tn = t - tm * sp.tiles_n;
+    return;
+  }
+  for (tm = 0; tm < P.tiles_m; ++tm) {
+    const int first = (tm * BM) / BN;
+    const int cnt = sp.tiles_n > first ? sp.tiles_n - first : 0;
+    if (t < cnt) {
+      tn = first + t;
+      return;
+    }
+    t -= cnt;
+  }
+  tn = 0;
+}
+
+template <int EPI>
+__device__ __forceinline__ void epilogue_chunk(const Params &P, const SubProblem &sp, int row, int col0,
+                                               const uint32_t (&r)[32], double &sq) {
+  if (row >= P.M) return;
+  const int N = sp.N;
+  if (EPI == EPI_STORE_BF16) {
+    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(sp.out) + (long long)row * sp.ldo + col0;
+    if (col0 + 32 <= N) {
+      uint4 *o4 = reinterpret_cast<uint4 *>(o);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+        w.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+        w.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+        w.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+        o4[v] = w;
+      }
+    } else {
+      for (int j = 0; j < 32 && col0 + j < N; ++j) o[j] = __float2bfloat16_rn(__uint_as_float(r[j]));
+    }
+    return;
+  }
+  float *o = reinterpret_cast<float *>(sp.out) + (long long)row * sp.ldo + col0;
+  const bool full = col0 + 32 <= N && (!sp.upper || col0 >= row);
+  if (full) {
+    float4 *o4 = reinterpret_cast<float4 *>(o);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      float4 x = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]), __uint_as_float(r[4 * v + 2]),
+                             __uint_as_float(r[4 * v + 3]));
+      if (EPI == EPI_STORE_TF32_SQ) {
+        sq += (double)x.x * x.x + (double)x.y * x.y + (double)x.z * x.z + (double)x.w * x.w;
+        x = make_float4(to_tf32_rn(x.x), to_tf32_rn(x.y), to_tf32_rn(x.z), to_tf32_rn(x.w));
+      }
+      if (EPI == EPI_ACCUM_F32) {
+        const float4 y = o4[v];
+        x.x += y.x;
+        x.y += y.y;
+        x.z += y.z;
+        x.w += y.w;
+      }
+      o4[v] = x;
+    }
+  } else {
+    for (int j = 0; j < 32; ++j) {
+      const int c = col0 + j;
+      if (c >= N) break;
+      if (sp.upper && c < row) continue;
+      float x = __uint_as_float(r[j]);
+      if (EPI == EPI_STORE_TF32_SQ) {
+        sq += (double)x * x;
+        x = to_tf32_rn(x);
+      }
+      if (EPI == EPI_ACCUM_F32) x += o[j];
+      o[j] = x;
+    }
+  }
+}
+
+#ifdef ISPA_DEFINE_GEMM_KERNEL
+// tma maps: ta = A operand; tb[prob] = B operand of each sub-problem.
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb0,
+                const __grid_constant__ CUtensorMap tb1, Params P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + STAGES * TILE_BYTES;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + 2 * STAGES * TILE_BYTES);
+  uint64_t *empty = full + STAGES;
+  uint64_t *done = empty + STAGES;
+  uint64_t *drain = done + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int prob, tm, tn;
+  tile_coords(P, blockIdx.x, prob, tm, tn);
+  const SubProblem &sp = P.p[prob];
+  const CUtensorMap *tB = prob == 0 ? &tb0 : &tb1;
+  const int m0 = tm * BM, n0 = tn * BN;
+  const int k_tiles = (P.K + (P.kind_tf32 ? 31 : 63)) / (P.kind_tf32 ? 32 : 64);
+  const int bk = P.kind_tf32 ? 32 : 64;         // K elements per stage
+  const int e128 = P.kind_tf32 ? 32 : 64;       // elements per 128-byte row
+  const uint32_t kstep_kmajor = 32;             // bytes per MMA K-step inside a K-major row
+  const uint32_t kstep_mn = P.kind_tf32 ? 1024 : 2048;  // bytes per MMA K-step in an MN-major tile
+  const uint32_t mn_box_bytes = (uint32_t)bk * 128;     // one 128-byte-wide MN-major box
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    mbar_init(done, 1);
+    mbar_init(drain, 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&ta);
+    tma_prefetch_desc(tB);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, BN);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t pending = 0;  // bit s: a load into stage s may still be in flight
+      uint32_t issued_phase = 0;
+      for (int kt = 0; kt < k_tiles; ++kt) {
+        const int s = kt % STAGES;
+        const uint32_t ph = (kt / STAGES) & 1;
+        if (!wait_parity(empty + s, ph ^ 1, P.err, abort, 1)) break;
+        mbar_arrive_expect_tx(full + s, 2 * TILE_BYTES);
+        const int k0 = kt * bk;
+        uint8_t *a = sA + s * TILE_BYTES;
+        uint8_t *b = sB + s * TILE_BYTES;
+        if (!P.a_mn) {
+          tma_load_2d(a, &ta, full + s, k0, m0);
+        } else {
+          for (int c = 0; c < BM / e128; ++c) tma_load_2d(a + c * mn_box_bytes, &ta, full + s, m0 + c * e128, k0);
+        }
+        if (!P.b_mn) {
+          tma_load_2d(b, tB, full + s, k0, n0);
+        } else {
+          for (int c = 0; c < BN / e128; ++c) tma_load_2d(b + c * mn_box_bytes, tB, full + s, n0 + c * e128, k0);
+        }
+        pending |= 1u << s;
+        issued_phase = (issued_phase & ~(1u << s)) | (ph << s);
+      }
+      if (*abort) {
+        for (int s = 0; s < STAGES; ++s)
+          if (pending & (1u << s)) wait_parity_drain(full + s, (issued_phase >> s) & 1, P.err);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = true;
+      for (int kt = 0; kt < k_tiles; ++kt) {
+        const int s = kt % STAGES;
+        const uint32_t ph = (kt / STAGES) & 1;
+        if (!wait_parity(full + s, ph, P.err, abort, 2)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(sA + s * TILE_BYTES);
+        const uint32_t b_base = smem_u32(sB + s * TILE_BYTES);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t ad = P.a_mn ? smem_desc_sw128(a_base + ks * kstep_mn, mn_box_bytes, 1024)
+                                     : smem_desc_sw128(a_base + ks * kstep_kmajor, 16, 1024);
+          const uint64_t bd = P.b_mn ? smem_desc_sw128(b_base + ks * kstep_mn, mn_box_bytes, 1024)
+                                     : smem_desc_sw128(b_base + ks * kstep_kmajor, 16, 1024);
+          mma_ss(tmem, ad, bd, P.idesc, (kt > 0 || ks > 0) ? 1u : 0u, P.kind_tf32);
+        }
+        mma_commit(empty + s);
+      }
+      mma_commit(ok ? done : drain);
+      if (!ok) wait_parity_drain(drain, 0, P.err);
+    }
+  } else {
+    // epilogue warps 2..5: TMEM lane quarter = warp % 4
+    const int quarter = warp & 3;
+    const int row = m0 + quarter * 32 + lane;
+    double sq = 0.0;
+    if (wait_parity(done, 0, P.err, abort, 3)) {
+      tc_fence_after();
+      const int n_chunks = min(BN, sp.N - n0 + 31) / 32;
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + c * 32, r);
+        tmem_wait_ld();
+        if (c >= n_chunks) continue;
+        switch (sp.epi) {
+          case EPI_STORE_F32: epilogue_chunk<EPI_STORE_F32>(P, sp, row, n0 + c * 32, r, sq); break;
+          case EPI_STORE_TF32_SQ: epilogue_chunk<EPI_STORE_TF32_SQ>(P, sp, row, n0 + c * 32, r, sq); break;
+          case EPI_ACCUM_F32: epilogue_chunk<EPI_ACCUM_F32>(P, sp, row, n0 + c * 32, r, sq); break;
+          default: epilogue_chunk<EPI_STORE_BF16>(P, sp, row, n0 + c * 32, r, sq); break;
+        }
+      }
+    }
+    if (sp.epi == EPI_STORE_TF32_SQ) {
+      sq = warp_sum_d(sq);
+      if (lane == 0 && P.r2) atomicAdd(P.r2, sq);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, BN);
+}
+#endif  // ISPA_DEFINE_GEMM_KERNEL
+
+}  // namespace tcg
+}  // namespace ispa

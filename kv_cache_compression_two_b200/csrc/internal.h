@@ -1,0 +1,69 @@
+// internal.h -- host-side declarations shared by the translation units of libispa.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/ispa.h"
+#include "common.cuh"
+
+namespace ispa {
+
+// Records a printf-style message as this thread's last error and returns `st`.
+ispa_status fail(ispa_status st, const char *fmt, ...);
+// ISPA_OK, or ISPA_ERR_CUDA with the CUDA error text.
+ispa_status cuda_status(cudaError_t e, const char *what);
+// Error word and wait limit of the current device (fetched once per device).
+ispa_status device_err(DevErr *out);
+// SM count of the current device.
+int sm_count();
+
+// Encodes a tiled TMA descriptor (driver entry point resolved at run time).
+//   dims[0] is the contiguous dimension; strides_bytes has rank-1 entries.
+ispa_status make_tmap(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *base,
+                      const uint64_t *dims, const uint64_t *strides_bytes, const uint32_t *box,
+                      CUtensorMapSwizzle swizzle);
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Token ranges of the two groups of one attention call (half-open, in rows).
+struct GroupRanges {
+  int n_loc;            // 0, 1 or 2 local ranges (sink, current), disjoint and ordered
+  int loc_begin[2], loc_end[2];
+  int hist_begin, hist_end;
+  int q_begin;          // first K/V row of the current chunk (queries' own frames)
+  int Lq, Lkv;
+};
+
+// ---- launchers (each returns ISPA_OK or ISPA_ERR_CUDA) ----
+ispa_status launch_lse_merge(int rows, int H, int d, ispa_dtype dt, const void *oa, const float *la,
+                             const void *ob, const float *lb, void *oo, float *lo, cudaStream_t s);
+ispa_status launch_select(int N, const double *eps, int K, unsigned char *is_local, int *idx,
+                          cudaStream_t s);
+ispa_status launch_absorb_weight(int D, int Dout, const void *W, ispa_dtype wdt, const float *dW,
+                                 void *Wn, ispa_dtype odt, cudaStream_t s);
+ispa_status launch_attn_simt(const ispa_attn_desc &d, const GroupRanges &g, float scale, const float *q,
+                             const float *k, const float *v, void *o_loc, float *l_loc, void *o_hist,
+                             float *l_hist, void *o_full, float *l_full, cudaStream_t s);
+ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float scale, const void *q,
+                           const void *k, const void *v, void *o_loc, float *l_loc, void *o_hist,
+                           float *l_hist, void *o_full, float *l_full, cudaStream_t s);
+
+// stats
+size_t stats_workspace_bytes(int T, int D, int Dout, ispa_precision prec);
+ispa_status launch_stats(int T, int D, int Dout, const float *a_loc, const float *a_full, const float *W,
+                         float *G, float *C, double *r2, ispa_precision prec, void *ws, cudaStream_t s);
+
+// ridge
+size_t ridge_workspace_bytes(int D, int Dout);
+ispa_status launch_ridge(int D, int Dout, const float *G, const float *C, const double *r2, float lambda,
+                         int lambda_relative, int refine_steps, float *dW, double *eps, void *ws,
+                         cudaStream_t s);
+
+// bf16 projection GEMM y[M, N] = A[M, K] * B[K, N] (A, B bf16 row-major) on tcgen05
+ispa_status launch_gemm_bf16(int M, int N, int K, const void *A, const void *B, void *Y, ispa_dtype ydt,
+                             cudaStream_t s);
+
+}  // namespace ispa

@@ -1,0 +1,316 @@
+// ridge.cu -- closed-form absorption: dW = (G + lambda I)^-1 C and epsilon.
+//
+// Blocked right-looking Cholesky in fp32 (block NB = 64):
+//   for each diagonal block k:  factor L_kk (one CTA, shared memory),
+//                               L_ik = A_ik L_kk^-T for the rows below (one thread per row),
+//                               A_ij -= L_ik L_jk^T on the trailing lower triangle (SIMT GEMM).
+// then the blocked forward and backward substitutions on the Dout right-hand
+// sides, optional iterative refinement with residuals accumulated in fp64,
+// and epsilon = r2 - 2<dW, C> + <dW, G dW> with fp64 reductions.
+#include "internal.h"
+#include "simt_gemm.cuh"
+
+namespace ispa {
+
+namespace {
+
+constexpr int NB = 64;
+
+struct Ws {
+  float *L;      // [D, D] lower Cholesky factor (working copy)
+  float *Rres;   // [D, Dout] refinement residual / correction
+  double *acc;   // [0] <dW, C>  [1] <dW, G dW>  [2] trace(G)  [3] lambda_eff
+  int *flag;     // non-zero once a pivot failed
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+Ws carve(void *base, int D, int Dout) {
+  char *p = static_cast<char *>(base);
+  Ws w;
+  w.L = reinterpret_cast<float *>(p);
+  p += align256((size_t)D * D * sizeof(float));
+  w.Rres = reinterpret_cast<float *>(p);
+  p += align256((size_t)D * Dout * sizeof(float));
+  w.acc = reinterpret_cast<double *>(p);
+  p += 64;
+  w.flag = reinterpret_cast<int *>(p);
+  return w;
+}
+
+__global__ void trace_kernel(int D, const float *__restrict__ G, double *acc) {
+  double s = 0.0;
+  for (int i = threadIdx.x; i < D; i += blockDim.x) s += (double)G[(long long)i * D + i];
+  s = warp_sum_d(s);
+  __shared__ double part[32];
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += part[w];
+    acc[2] = t;
+  }
+}
+
+__global__ void init_kernel(int D, int Dout, const float *__restrict__ G, const float *__restrict__ C,
+                            float lambda, int relative, Ws w, float *dW) {
+  const double lam = relative ? (double)lambda * w.acc[2] / D : (double)lambda;
+  const float lamf = (float)lam;
+  const long long nDD = (long long)D * D, nDO = (long long)D * Dout;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  const long long t0 = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (t0 == 0) {
+    w.acc[0] = 0.0;
+    w.acc[1] = 0.0;
+    w.acc[3] = (double)lamf;
+    *w.flag = 0;
+  }
+  for (long long e = t0; e < nDD; e += stride) {
+    const int i = (int)(e / D), j = (int)(e - (long long)i * D);
+    float x = 0.f;
+    if (i >= j) x = G[(long long)j * D + i] + (i == j ? lamf : 0.f);
+    w.L[e] = x;
+  }
+  for (long long e = t0; e < nDO; e += stride) dW[e] = C[e];
+}
+
+// Factors the nb x nb diagonal block at kb0 in place (nb <= 64), one CTA of 64 threads.
+__global__ void __launch_bounds__(64) potrf_diag_kernel(int D, int kb0, float *L, int *flag, DevErr err) {
+  __shared__ float A[NB][NB + 1];
+  const int nb = min(NB, D - kb0);
+  const int t = threadIdx.x;
+  for (int r = 0; r < nb; ++r)
+    if (t < nb) A[r][t] = L[(long long)(kb0 + r) * D + kb0 + t];
+  __syncthreads();
+  for (int c = 0; c < nb; ++c) {
+    if (t == 0) {
+      float piv = A[c][c];
+      if (!(piv > 0.f)) {
+        if (atomicExch(flag, 1) == 0) report_error(err, ISPA_ERR_NOT_SPD, kb0 + c + 1);
+        piv = __int_as_float(0x7fc00000);
+      }
+      A[c][c] = sqrtf(piv);
+    }
+    __syncthreads();
+    if (t > c && t < nb) A[t][c] /= A[c][c];
+    __syncthreads();
+    if (t > c && t < nb) {
+      const float lic = A[t][c];
+      for (int j = c + 1; j <= t; ++j) A[t][j] -= lic * A[j][c];
+    }
+    __syncthreads();
+  }
+  for (int r = 0; r < nb; ++r)
+    if (t <= r) L[(long long)(kb0 + r) * D + kb0 + t] = A[r][t];
+}
+
+// Rows i >= kb0 + 64: L[i, kb] = A[i, kb] L_kk^-T  (forward substitution per row).
+__global__ void __launch_bounds__(64) trsm_panel_kernel(int D, int kb0, float *L) {
+  __shared__ float Lk[NB][NB + 1];
+  const int t = threadIdx.x;
+  for (int r = 0; r < NB; ++r) Lk[r][t] = L[(long long)(kb0 + r) * D + kb0 + t];
+  __syncthreads();
+  const int i = kb0 + NB + blockIdx.x * NB + t;
+  if (i >= D) return;
+  float x[NB];
+  float *row = L + (long long)i * D + kb0;
+#pragma unroll
+  for (int c = 0; c < NB; ++c) x[c] = row[c];
+#pragma unroll
+  for (int c = 0; c < NB; ++c) {
+    float s = x[c];
+#pragma unroll
+    for (int p = 0; p < c; ++p) s -= Lk[c][p] * x[p];
+    x[c] = s / Lk[c][c];
+  }
+#pragma unroll
+  for (int c = 0; c < NB; ++c) row[c] = x[c];
+}
+
+// Loads the diagonal block padded to NB x NB with the identity beyond nb.
+__device__ __forceinline__ void load_diag_padded(float (*Lk)[NB + 1], const float *L, int D, int kb0, int nb) {
+  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
+    const int r = e / NB, c = e - r * NB;
+    float x;
+    if (r < nb && c < nb)
+      x = (c <= r) ? L[(long long)(kb0 + r) * D + kb0 + c] : 0.f;
+    else
+      x = (r == c) ? 1.f : 0.f;
+    Lk[r][c] = x;
+  }
+}
+
+// Y[kb rows, :] = L_kk^-1 Y[kb rows, :]   (one thread per right-hand-side column)
+__global__ void __launch_bounds__(128) trsv_fwd_kernel(int D, int Dout, int kb0, const float *L, float *Y) {
+  __shared__ float Lk[NB][NB + 1];
+  const int nb = min(NB, D - kb0);
+  load_diag_padded(Lk, L, D, kb0, nb);
+  __syncthreads();
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= Dout) return;
+  float y[NB];
+#pragma unroll
+  for (int p = 0; p < NB; ++p) y[p] = p < nb ? Y[(long long)(kb0 + p) * Dout + j] : 0.f;
+#pragma unroll
+  for (int r = 0; r < NB; ++r) {
+    float s = y[r];
+#pragma unroll
+    for (int p = 0; p < r; ++p) s -= Lk[r][p] * y[p];
+    y[r] = s / Lk[r][r];
+  }
+#pragma unroll
+  for (int p = 0; p < NB; ++p)
+    if (p < nb) Y[(long long)(kb0 + p) * Dout + j] = y[p];
+}
+
+// Y[kb rows, :] = L_kk^-T Y[kb rows, :]
+__global__ void __launch_bounds__(128) trsv_bwd_kernel(int D, int Dout, int kb0, const float *L, float *Y) {
+  __shared__ float Lk[NB][NB + 1];
+  const int nb = min(NB, D - kb0);
+  load_diag_padded(Lk, L, D, kb0, nb);
+  __syncthreads();
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= Dout) return;
+  float y[NB];
+#pragma unroll
+  for (int p = 0; p < NB; ++p) y[p] = p < nb ? Y[(long long)(kb0 + p) * Dout + j] : 0.f;
+#pragma unroll
+  for (int r = NB - 1; r >= 0; --r) {
+    float s = y[r];
+#pragma unroll
+    for (int c = r + 1; c < NB; ++c) s -= Lk[c][r] * y[c];
+    y[r] = s / Lk[r][r];
+  }
+#pragma unroll
+  for (int p = 0; p < NB; ++p)
+    if (p < nb) Y[(long long)(kb0 + p) * Dout + j] = y[p];
+}
+
+// Rres = C - (G + lambda I) X, accumulated in fp64.
+struct EpiResidual {
+  float *out;
+  const float *C, *X;
+  const double *acc;
+  int ld;
+  __device__ void begin() {}
+  __device__ void end() {}
+  __device__ void operator()(int m, int n, double a) {
+    const long long o = (long long)m * ld + n;
+    out[o] = (float)((double)C[o] - a - acc[3] * (double)X[o]);
+  }
+};
+
+// acc[1] += sum dW[m][n] * (G dW)[m][n]
+struct EpiDotG {
+  const float *dW;
+  double *acc;
+  int ld;
+  double part;
+  __device__ void begin() { part = 0.0; }
+  __device__ void operator()(int m, int n, float a) { part += (double)dW[(long long)m * ld + n] * (double)a; }
+  __device__ void end() {
+    const double s = warp_sum_d(part);
+    if ((threadIdx.x & 31) == 0) atomicAdd(acc + 1, s);
+  }
+};
+
+__global__ void add_kernel(long long n, float *__restrict__ X, const float *__restrict__ dX) {
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x)
+    X[e] += dX[e];
+}
+
+__global__ void dot_kernel(long long n, const float *__restrict__ a, const float *__restrict__ b, double *out) {
+  double s = 0.0;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x)
+    s += (double)a[e] * (double)b[e];
+  s = warp_sum_d(s);
+  if ((threadIdx.x & 31) == 0) atomicAdd(out, s);
+}
+
+__global__ void finalize_kernel(long long n, const double *__restrict__ r2, Ws w, float *dW, double *eps) {
+  const bool bad = *w.flag != 0;
+  if (blockIdx.x == 0 && threadIdx.x == 0)
+    *eps = bad ? __longlong_as_double(0x7ff8000000000000LL) : (*r2 - 2.0 * w.acc[0] + w.acc[1]);
+  if (!bad) return;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x)
+    dW[e] = __int_as_float(0x7fc00000);
+}
+
+// Forward then backward blocked substitution on Y [D, Dout] in place.
+cudaError_t cholesky_solve(int D, int Dout, const float *L, float *Y, cudaStream_t s) {
+  const int cgrid = (Dout + 127) / 128;
+  for (int kb0 = 0; kb0 < D; kb0 += NB) {
+    const int nb = min(NB, D - kb0);
+    trsv_fwd_kernel<<<cgrid, 128, 0, s>>>(D, Dout, kb0, L, Y);
+    const int below = D - kb0 - nb;
+    if (below > 0) {
+      cudaError_t e = simt_gemm<OP_N, OP_N, float, 0>(
+          below, Dout, nb, Operand{L + (long long)(kb0 + nb) * D + kb0, nullptr, D},
+          Operand{Y + (long long)kb0 * Dout, nullptr, Dout},
+          EpiAxpby{Y + (long long)(kb0 + nb) * Dout, Dout, -1.f, 1.f, 0}, s);
+      if (e != cudaSuccess) return e;
+    }
+  }
+  const int last0 = ((D - 1) / NB) * NB;
+  for (int kb0 = last0; kb0 >= 0; kb0 -= NB) {
+    const int nb = min(NB, D - kb0);
+    trsv_bwd_kernel<<<cgrid, 128, 0, s>>>(D, Dout, kb0, L, Y);
+    if (kb0 > 0) {
+      cudaError_t e = simt_gemm<OP_T, OP_N, float, 0>(kb0, Dout, nb, Operand{L + (long long)kb0 * D, nullptr, D},
+                                                      Operand{Y + (long long)kb0 * Dout, nullptr, Dout},
+                                                      EpiAxpby{Y, Dout, -1.f, 1.f, 0}, s);
+      if (e != cudaSuccess) return e;
+    }
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t ridge_workspace_bytes(int D, int Dout) {
+  return align256((size_t)D * D * sizeof(float)) + align256((size_t)D * Dout * sizeof(float)) + 256;
+}
+
+ispa_status launch_ridge(int D, int Dout, const float *G, const float *C, const double *r2, float lambda,
+                         int lambda_relative, int refine_steps, float *dW, double *eps, void *ws_base,
+                         cudaStream_t s) {
+  DevErr err;
+  ispa_status st = device_err(&err);
+  if (st != ISPA_OK) return st;
+  Ws w = carve(ws_base, D, Dout);
+  const int grid = sm_count() * 4;
+  trace_kernel<<<1, 256, 0, s>>>(D, G, w.acc);
+  init_kernel<<<grid, 256, 0, s>>>(D, Dout, G, C, lambda, lambda_relative, w, dW);
+  for (int kb0 = 0; kb0 < D; kb0 += NB) {
+    potrf_diag_kernel<<<1, 64, 0, s>>>(D, kb0, w.L, w.flag, err);
+    const int below = D - kb0 - NB;
+    if (below > 0) {
+      trsm_panel_kernel<<<(below + NB - 1) / NB, 64, 0, s>>>(D, kb0, w.L);
+      const int j0 = kb0 + NB;
+      cudaError_t e = simt_gemm<OP_N, OP_T, float, 1>(
+          below, below, NB, Operand{w.L + (long long)j0 * D + kb0, nullptr, D},
+          Operand{w.L + (long long)j0 * D + kb0, nullptr, D},
+          EpiAxpby{w.L + (long long)j0 * D + j0, D, -1.f, 1.f, 1}, s);
+      if (e != cudaSuccess) return cuda_status(e, "ridge trailing update");
+    }
+  }
+  cudaError_t e = cholesky_solve(D, Dout, w.L, dW, s);
+  if (e != cudaSuccess) return cuda_status(e, "ridge solve");
+  const long long nDO = (long long)D * Dout;
+  for (int r = 0; r < refine_steps; ++r) {
+    e = simt_gemm<OP_SYM_UPPER, OP_N, double, 0>(D, Dout, D, Operand{G, nullptr, D}, Operand{dW, nullptr, Dout},
+                                                 EpiResidual{w.Rres, C, dW, w.acc, Dout}, s);
+    if (e != cudaSuccess) return cuda_status(e, "ridge residual");
+    e = cholesky_solve(D, Dout, w.L, w.Rres, s);
+    if (e != cudaSuccess) return cuda_status(e, "ridge refinement solve");
+    add_kernel<<<grid, 256, 0, s>>>(nDO, dW, w.Rres);
+  }
+  dot_kernel<<<grid, 256, 0, s>>>(nDO, dW, C, w.acc);
+  e = simt_gemm<OP_SYM_UPPER, OP_N, float, 0>(D, Dout, D, Operand{G, nullptr, D}, Operand{dW, nullptr, Dout},
+                                              EpiDotG{dW, w.acc, Dout, 0.0}, s);
+  if (e != cudaSuccess) return cuda_status(e, "ridge G dW");
+  finalize_kernel<<<grid, 256, 0, s>>>(nDO, r2, w, dW, eps);
+  return cuda_status(cudaGetLastError(), "ridge launch");
+}
+
+}  // namespace ispa

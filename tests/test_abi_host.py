@@ -1,0 +1,123 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+declared in include/ispa.h, and rejects invalid arguments before touching the
+GPU (no CUDA call is made on these paths, so they run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import kv_cache_compression_two_b200 as ispa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "ispa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ispa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = ispa.lib()
+    declared = header_functions()
+    assert len(declared) >= 12
+    for name in declared:
+        assert hasattr(L, name), name
+    assert set(declared) == set(ispa.EXPORTED)
+
+
+def test_version_string():
+    assert "sm_100a" in ispa.version()
+
+
+def _desc(**kw):
+    base = dict(B=1, H=2, head_dim=128, tokens_per_frame=16, sink_frames=1, hist_begin=1, hist_end=4, cur_begin=4,
+                cur_end=5, kv_frames=5, in_dtype=ispa.ISPA_BF16, out_dtype=ispa.ISPA_F32, softmax_scale=0.0)
+    base.update(kw)
+    return ispa.AttnDesc(**base)
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def _split(desc, ptrs=None):
+    p = ptrs or [FAKE] * 9
+    return ispa.lib().ispa_attn_split(ctypes.byref(desc), *p, None)
+
+
+@pytest.mark.parametrize("kw,frag", [
+    (dict(head_dim=96), "head_dim"),
+    (dict(B=0), "B, H"),
+    (dict(kv_frames=0), "kv_frames"),
+    (dict(cur_begin=5, cur_end=5), "current chunk"),
+    (dict(cur_end=6), "current chunk"),
+    (dict(hist_begin=0, hist_end=2), "overlaps"),
+    (dict(hist_begin=3, hist_end=5), "overlaps"),
+    (dict(sink_frames=6), "sink_frames"),
+    (dict(in_dtype=7), "dtype"),
+])
+def test_attn_split_rejects_bad_layouts(kw, frag):
+    st = _split(_desc(**kw))
+    assert st == ispa.ISPA_ERR_INVALID_ARG
+    assert frag in ispa.lib().ispa_last_error().decode()
+
+
+def test_attn_split_rejects_null_and_misaligned():
+    assert ispa.lib().ispa_attn_split(None, *([FAKE] * 9), None) == ispa.ISPA_ERR_INVALID_ARG
+    p = [FAKE] * 9
+    p[0] = FAKE + 4
+    assert _split(_desc(), p) == ispa.ISPA_ERR_INVALID_ARG
+    p = [FAKE] * 9
+    p[5] = None  # o_hist without lse_hist
+    p[6] = FAKE
+    p[5], p[6] = None, FAKE
+    assert _split(_desc(), p) == ispa.ISPA_ERR_INVALID_ARG
+
+
+def test_bf16_other_head_dims_unsupported():
+    st = _split(_desc(head_dim=64))
+    assert st == ispa.ISPA_ERR_UNSUPPORTED
+
+
+def test_stats_and_ridge_validation():
+    L = ispa.lib()
+    assert L.ispa_accum_stats(10, 48, 64, *([FAKE] * 5), FAKE, ispa.ISPA_PREC_TF32, FAKE, 1 << 30,
+                              None) == ispa.ISPA_ERR_INVALID_ARG  # D % 32
+    assert L.ispa_accum_stats(10, 64, 64, *([FAKE] * 5), FAKE, ispa.ISPA_PREC_TF32, FAKE, 16,
+                              None) == ispa.ISPA_ERR_INVALID_ARG  # workspace too small
+    assert "workspace" in L.ispa_last_error().decode()
+    assert L.ispa_ridge_solve(64, 64, FAKE, FAKE, FAKE, ctypes.c_float(-1.0), 0, 0, FAKE, FAKE, FAKE, 1 << 30,
+                              None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_ridge_solve(64, 64, FAKE, FAKE, FAKE, ctypes.c_float(1.0), 0, 99, FAKE, FAKE, FAKE, 1 << 30,
+                              None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_select_layers(4, FAKE, 5, FAKE, FAKE, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_select_layers(5000, FAKE, 5, FAKE, FAKE, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_lse_merge(10, 2, 12, ispa.ISPA_F32, *([FAKE] * 6), None) == ispa.ISPA_ERR_INVALID_ARG
+    # lse_out overlapping lse_a is rejected (in-place O is allowed, in-place LSE is not)
+    assert L.ispa_lse_merge(10, 2, 64, ispa.ISPA_F32, FAKE, FAKE, FAKE, FAKE + 4096, FAKE + 8192, FAKE,
+                            None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_absorb_weight(3, 3, FAKE, 0, FAKE, FAKE, 0, None) == ispa.ISPA_ERR_INVALID_ARG
+
+
+def test_workspace_queries():
+    L = ispa.lib()
+    D, Dout, T = 1536, 1536, 4680
+    ridge = L.ispa_ridge_workspace_bytes(D, Dout)
+    assert ridge >= 2 * D * Dout * 4
+    tf32 = L.ispa_accum_stats_workspace_bytes(T, D, Dout, ispa.ISPA_PREC_TF32)
+    assert tf32 >= (2 * T * D + D * Dout + T * Dout) * 4
+    assert L.ispa_accum_stats_workspace_bytes(T, D, Dout, ispa.ISPA_PREC_F32) >= T * Dout * 4
+    d = _desc(H=12, tokens_per_frame=1560, sink_frames=3, hist_begin=3, hist_end=18, cur_begin=18, cur_end=21,
+              kv_frames=21)
+    assert L.ispa_attn_local_proj_workspace_bytes(ctypes.byref(d)) >= 4680 * 1536 * 2
+    assert L.ispa_ridge_workspace_bytes(0, 5) == 0
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    import importlib
+    import sys
+    monkeypatch.setattr(ispa, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(ispa, "_lib", None)
+    with pytest.raises(ImportError):
+        ispa.lib()

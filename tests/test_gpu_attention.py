@@ -1,0 +1,153 @@
+"""GPU parity of the two-group attention (and its fused merge) against the fp64 oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import kv_cache_compression_two_b200 as ispa
+import synth_inputs as si
+from oracle import ispa_oracle as orc
+from gpu_helpers import assert_bf16_out, assert_lse, dev, host, max_over_rms, nan_like, normwise
+
+pytestmark = pytest.mark.gpu
+
+
+def run_split(shape, in_dt, out_dt, key, fused=True, want_hist=True):
+    data = si.iid_qkv(shape, "bf16" if in_dt == ispa.ISPA_BF16 else "f32", key)
+    tin = torch.bfloat16 if in_dt == ispa.ISPA_BF16 else torch.float32
+    tout = torch.bfloat16 if out_dt == ispa.ISPA_BF16 else torch.float32
+    q, k, v = dev(data["q"], tin), dev(data["k"], tin), dev(data["v"], tin)
+    B, Lq, H, d = shape.B, shape.Lq, shape.H, shape.d
+    o = {n: nan_like((B, Lq, H, d), tout) for n in ("loc", "hist", "full")}
+    l = {n: nan_like((B, Lq, H), torch.float32) for n in ("loc", "hist", "full")}
+    desc = ispa.attn_desc(shape, in_dt, out_dt)
+    ispa.ispa_attn_split(desc, q, k, v, o["loc"], l["loc"], o["hist"] if want_hist else None,
+                         l["hist"] if want_hist else None, o["full"] if fused else None, l["full"] if fused else None)
+    ispa.ispa_check_device_error()
+    torch.cuda.synchronize()
+    return data, {n: host(t) for n, t in o.items()}, {n: host(t) for n, t in l.items()}
+
+
+def check(shape, data, O, L, in_dt, out_dt, fused=True, rows=None, want_hist=True):
+    ref = orc.split_attention(shape, data["q"], data["k"], data["v"], rows=rows)
+    names = ["loc"] + (["hist"] if want_hist else []) + (["full"] if fused else [])
+    sel = slice(None) if rows is None else np.asarray(rows)
+    for n in names:
+        got_o, got_l = O[n][:, sel], L[n][:, sel]
+        ref_o, ref_l = ref["O_" + n], ref["L_" + n]
+        if in_dt == ispa.ISPA_F32:
+            if np.abs(ref_o).max() > 0:
+                assert normwise(got_o, ref_o) <= 1e-5, (n, normwise(got_o, ref_o))
+            else:
+                assert np.all(got_o == 0)
+            assert_lse(got_l, ref_l, 1e-5 * max(1.0, float(np.abs(ref_l[np.isfinite(ref_l)]).max(initial=1.0))))
+        else:
+            if np.all(ref_o == 0):
+                assert np.all(got_o == 0), n
+            elif out_dt == ispa.ISPA_BF16:
+                assert_bf16_out(got_o, ref_o)
+            else:
+                assert max_over_rms(got_o, ref_o) <= 1e-2, (n, max_over_rms(got_o, ref_o))
+            assert_lse(got_l, ref_l, 1e-3)
+
+
+# ---------------------------------------------------------------- fp32 (CUDA cores)
+def test_tiny_fp32_matches_oracle():
+    sh = si.TINY
+    for chunk in range(4):
+        data, O, L = run_split(sh, ispa.ISPA_F32, ispa.ISPA_F32, ("gpu", "tiny", chunk))
+        check(sh, data, O, L, ispa.ISPA_F32, ispa.ISPA_F32)
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+def test_fp32_random_layouts(d):
+    g = np.random.default_rng(100 + d)
+    for trial in range(4):
+        sh = si.random_groups_shape(g, max_frames=6, d=d)
+        data, O, L = run_split(sh, ispa.ISPA_F32, ispa.ISPA_F32, ("gpu", "f32rand", d, trial))
+        check(sh, data, O, L, ispa.ISPA_F32, ispa.ISPA_F32)
+
+
+# ---------------------------------------------------------------- bf16 (tcgen05)
+BF16_SHAPES = [
+    # several query tiles with a ragged tail, local group split in two ranges, ragged KV tiles
+    si.AttnShape(B=2, H=2, d=128, tpf=50, sink_frames=2, hist_begin=2, hist_end=7, cur_begin=7, cur_end=10,
+                 kv_frames=10),
+    # no history: full == local, empty history group
+    si.AttnShape(B=1, H=3, d=128, tpf=37, sink_frames=1, hist_begin=1, hist_end=1, cur_begin=1, cur_end=5,
+                 kv_frames=5),
+    # first chunk: the sink is the current chunk itself (one merged local range)
+    si.AttnShape(B=1, H=1, d=128, tpf=200, sink_frames=2, hist_begin=2, hist_end=2, cur_begin=0, cur_end=2,
+                 kv_frames=2),
+    # exact multiples of the 128 tiles, long history
+    si.AttnShape(B=1, H=2, d=128, tpf=128, sink_frames=1, hist_begin=1, hist_end=9, cur_begin=9, cur_end=10,
+                 kv_frames=10),
+    # single-token frames
+    si.AttnShape(B=3, H=1, d=128, tpf=1, sink_frames=1, hist_begin=1, hist_end=40, cur_begin=40, cur_end=43,
+                 kv_frames=43),
+]
+
+
+@pytest.mark.parametrize("idx", range(len(BF16_SHAPES)))
+def test_bf16_layouts_fp32_out(idx):
+    sh = BF16_SHAPES[idx]
+    data, O, L = run_split(sh, ispa.ISPA_BF16, ispa.ISPA_F32, ("gpu", "bf16", idx))
+    check(sh, data, O, L, ispa.ISPA_BF16, ispa.ISPA_F32)
+
+
+@pytest.mark.parametrize("idx", [0, 1])
+def test_bf16_layouts_bf16_out(idx):
+    sh = BF16_SHAPES[idx]
+    data, O, L = run_split(sh, ispa.ISPA_BF16, ispa.ISPA_BF16, ("gpu", "bf16o", idx))
+    check(sh, data, O, L, ispa.ISPA_BF16, ispa.ISPA_BF16)
+
+
+def test_bf16_optional_outputs():
+    sh = BF16_SHAPES[0]
+    data, O, L = run_split(sh, ispa.ISPA_BF16, ispa.ISPA_F32, ("gpu", "opt"), fused=False, want_hist=True)
+    check(sh, data, O, L, ispa.ISPA_BF16, ispa.ISPA_F32, fused=False)
+    assert np.all(np.isnan(O["full"]))  # untouched
+    data, O, L = run_split(sh, ispa.ISPA_BF16, ispa.ISPA_F32, ("gpu", "opt2"), fused=True, want_hist=False)
+    check(sh, data, O, L, ispa.ISPA_BF16, ispa.ISPA_F32, fused=True, want_hist=False)
+    assert np.all(np.isnan(O["hist"]))
+
+
+def test_bf16_large_scores_and_rescaling():
+    """Scores scaled up so the running maximum moves by far more than the rescale threshold."""
+    sh = si.AttnShape(B=1, H=1, d=128, tpf=64, sink_frames=1, hist_begin=1, hist_end=6, cur_begin=6, cur_end=8,
+                      kv_frames=8)
+    data = si.iid_qkv(sh, "bf16", ("gpu", "big"))
+    ramp = np.linspace(0.2, 3.0, sh.Lkv, dtype=np.float32)[None, :, None, None]
+    data["k"] = si.round_to_bf16(data["k"] * ramp)
+    q, k, v = dev(data["q"], torch.bfloat16), dev(data["k"], torch.bfloat16), dev(data["v"], torch.bfloat16)
+    o = {n: nan_like((1, sh.Lq, 1, 128), torch.float32) for n in ("loc", "hist", "full")}
+    l = {n: nan_like((1, sh.Lq, 1), torch.float32) for n in ("loc", "hist", "full")}
+    ispa.ispa_attn_split(ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_F32), q, k, v, o["loc"], l["loc"], o["hist"],
+                         l["hist"], o["full"], l["full"])
+    torch.cuda.synchronize()
+    check(sh, data, {n: host(t) for n, t in o.items()}, {n: host(t) for n, t in l.items()}, ispa.ISPA_BF16,
+          ispa.ISPA_F32)
+
+
+def test_bf16_fused_merge_equals_separate_merge():
+    sh = BF16_SHAPES[0]
+    data, O, L = run_split(sh, ispa.ISPA_BF16, ispa.ISPA_F32, ("gpu", "fm"))
+    oa, ob = dev(O["loc"]), dev(O["hist"])
+    la, lb = dev(L["loc"]), dev(L["hist"])
+    oo, lo = torch.empty_like(oa), torch.empty_like(la)
+    ispa.ispa_lse_merge(sh.B * sh.Lq, sh.H, 128, ispa.ISPA_F32, oa, la, ob, lb, oo, lo)
+    torch.cuda.synchronize()
+    assert np.abs(host(oo) - O["full"]).max() <= 1e-6 * np.abs(O["full"]).max()
+    assert np.abs(host(lo) - L["full"]).max() <= 1e-5
+
+
+def test_bf16_full_size_1p3b_sampled_rows():
+    """The 1.3B-shaped layer (4680 queries, 32760 keys, 12 heads) at full size, sampled rows."""
+    sh = si.SHAPE_1P3B
+    data, O, L = run_split(sh, ispa.ISPA_BF16, ispa.ISPA_F32, ("gpu", "full1p3b"))
+    rows = np.r_[0:3, 127:130, 2000:2003, 4600:4680:7, 4679]
+    check(sh, data, O, L, ispa.ISPA_BF16, ispa.ISPA_F32, rows=rows)
+    # unwritten outputs would still hold NaN
+    for n in ("loc", "hist", "full"):
+        assert not np.isnan(O[n]).any() and not np.isnan(L[n]).any()

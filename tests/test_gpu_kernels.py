@@ -1,0 +1,238 @@
+"""GPU parity of the LSE merge, statistics, ridge solve, selection, weight
+correction and post-switch projection against the fp64 oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import kv_cache_compression_two_b200 as ispa
+import synth_inputs as si
+from oracle import ispa_oracle as orc
+from gpu_helpers import assert_bf16_out, assert_lse, dev, host, max_over_rms, nan_like, normwise, rel_fro
+
+pytestmark = pytest.mark.gpu
+
+
+# ---------------------------------------------------------------- LSE merge
+@pytest.mark.parametrize("o_dt", [ispa.ISPA_F32, ispa.ISPA_BF16])
+def test_lse_merge_with_edge_cases(o_dt):
+    g = np.random.default_rng(7)
+    rows, H, d = 515, 3, 128
+    oa = g.standard_normal((rows, H, d)).astype(np.float32)
+    ob = g.standard_normal((rows, H, d)).astype(np.float32)
+    la = (g.standard_normal((rows, H)) * 5).astype(np.float32)
+    lb = (g.standard_normal((rows, H)) * 5).astype(np.float32)
+    la[0, :] = -np.inf                      # empty first group
+    lb[1, :] = -np.inf                      # empty second group
+    la[2, :] = -np.inf; lb[2, :] = -np.inf  # both empty
+    oa[0] = 0; ob[1] = 0; oa[2] = 0; ob[2] = 0
+    la[3, :] = 80.0; lb[3, :] = 10.0        # one group dominates by 70 nats
+    tdt = torch.bfloat16 if o_dt == ispa.ISPA_BF16 else torch.float32
+    if o_dt == ispa.ISPA_BF16:
+        oa, ob = si.round_to_bf16(oa), si.round_to_bf16(ob)
+    A, Bo = dev(oa, tdt), dev(ob, tdt)
+    LA, LB = dev(la), dev(lb)
+    out, lout = nan_like((rows, H, d), tdt), nan_like((rows, H), torch.float32)
+    ispa.ispa_lse_merge(rows, H, d, o_dt, A, LA, Bo, LB, out, lout)
+    torch.cuda.synchronize()
+    ref_o, ref_l = orc.lse_merge(oa, la, ob, lb)
+    got_o, got_l = host(out), host(lout)
+    assert_lse(got_l, ref_l, 1e-5 * np.abs(ref_l[np.isfinite(ref_l)]).max())
+    if o_dt == ispa.ISPA_F32:
+        assert np.abs(got_o - ref_o).max() <= 1e-6 * np.abs(ref_o).max()
+    else:
+        assert_bf16_out(got_o, ref_o, tol=1e-3)
+    assert np.all(got_o[2] == 0)
+    # in place on O
+    ispa.ispa_lse_merge(rows, H, d, o_dt, A, LA, Bo, LB, A, lout)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(A), got_o)
+
+
+# ---------------------------------------------------------------- selection
+def test_select_layers_matches_oracle_with_ties():
+    g = np.random.default_rng(8)
+    for N in (1, 2, 7, 30, 40, 129, 1000):
+        eps = np.round(g.random(N) * 8) / 8
+        for K in sorted({0, 1, N // 4, N // 2, N}):
+            e = dev(eps, torch.float64)
+            mask = torch.full((N,), 7, dtype=torch.uint8, device="cuda")
+            idx = torch.full((max(K, 1),), -1, dtype=torch.int32, device="cuda")
+            ispa.ispa_select_layers(N, e, K, mask, idx)
+            torch.cuda.synchronize()
+            rm, ri = orc.select_layers(eps, K)
+            assert np.array_equal(mask.cpu().numpy(), rm)
+            assert np.array_equal(idx.cpu().numpy()[:K], ri)
+
+
+def test_select_layers_nan_sorts_last():
+    eps = np.array([0.5, np.nan, 0.1, np.nan, 0.3])
+    mask = torch.zeros(5, dtype=torch.uint8, device="cuda")
+    idx = torch.zeros(4, dtype=torch.int32, device="cuda")
+    ispa.ispa_select_layers(5, dev(eps, torch.float64), 4, mask, idx)
+    torch.cuda.synchronize()
+    assert mask.cpu().tolist() == [1, 1, 1, 0, 1]
+    assert idx.cpu().tolist() == [0, 1, 2, 4]
+
+
+# ---------------------------------------------------------------- statistics
+def _stats_inputs(T, D, Dout, seed):
+    g = np.random.default_rng(seed)
+    # rows shaped like attention outputs: a common mean plus smaller fluctuations
+    mu = g.standard_normal(D) * 0.1
+    A_loc = (mu + 0.02 * g.standard_normal((T, D))).astype(np.float32)
+    A_full = (A_loc + 0.01 * g.standard_normal((T, D)) + 0.05 * mu).astype(np.float32)
+    W = (g.standard_normal((D, Dout)) / math.sqrt(D)).astype(np.float32)
+    return A_loc, A_full, W
+
+
+def _run_stats(T, D, Dout, prec, seed, batches=1):
+    A_loc, A_full, W = _stats_inputs(T * batches, D, Dout, seed)
+    G = torch.zeros((D, D), device="cuda")
+    C = torch.zeros((D, Dout), device="cuda")
+    r2 = torch.zeros(1, dtype=torch.float64, device="cuda")
+    ws = torch.empty(ispa.ispa_accum_stats_workspace_bytes(T, D, Dout, prec), dtype=torch.uint8, device="cuda")
+    Wd = dev(W)
+    for bi in range(batches):
+        sl = slice(bi * T, (bi + 1) * T)
+        ispa.ispa_accum_stats(T, D, Dout, dev(A_loc[sl]), dev(A_full[sl]), Wd, G, C, r2, prec, ws)
+    torch.cuda.synchronize()
+    Gr, Cr, r2r = orc.absorption_stats(A_loc.astype(np.float64), A_full.astype(np.float64), W.astype(np.float64))
+    return host(G), host(C), float(r2.item()), Gr, Cr, r2r
+
+
+@pytest.mark.parametrize("T,D,Dout,batches", [(300, 256, 192, 1), (128, 128, 128, 3), (4680, 1536, 1536, 1),
+                                              (77, 64, 96, 2)])
+def test_stats_tf32(T, D, Dout, batches):
+    G, C, r2, Gr, Cr, r2r = _run_stats(T, D, Dout, ispa.ISPA_PREC_TF32, 9, batches)
+    iu = np.triu_indices(D)
+    assert rel_fro(G[iu], Gr[iu]) <= 1e-3, rel_fro(G[iu], Gr[iu])
+    assert rel_fro(C, Cr) <= 1e-3, rel_fro(C, Cr)
+    assert abs(r2 - r2r) <= 1e-3 * r2r
+
+
+@pytest.mark.parametrize("T,D,Dout,batches", [(16, 64, 64, 4), (70, 96, 80, 1)])
+def test_stats_fp32(T, D, Dout, batches):
+    G, C, r2, Gr, Cr, r2r = _run_stats(T, D, Dout, ispa.ISPA_PREC_F32, 10, batches)
+    iu = np.triu_indices(D)
+    assert normwise(G[iu], Gr[iu]) <= 1e-5
+    assert normwise(C, Cr) <= 1e-5
+    assert abs(r2 - r2r) <= 1e-5 * r2r
+
+
+def test_stats_lower_triangle_untouched():
+    D = 128
+    A_loc, A_full, W = _stats_inputs(64, D, D, 11)
+    G = torch.full((D, D), 3.0, device="cuda")
+    C = torch.zeros((D, D), device="cuda")
+    r2 = torch.zeros(1, dtype=torch.float64, device="cuda")
+    ws = torch.empty(ispa.ispa_accum_stats_workspace_bytes(64, D, D, 0), dtype=torch.uint8, device="cuda")
+    ispa.ispa_accum_stats(64, D, D, dev(A_loc), dev(A_full), dev(W), G, C, r2, ispa.ISPA_PREC_TF32, ws)
+    torch.cuda.synchronize()
+    Gh = host(G)
+    il = np.tril_indices(D, -1)
+    assert np.all(Gh[il] == 3.0)
+
+
+# ---------------------------------------------------------------- ridge solve
+def _spd_problem(D, Dout, T, seed, cond_boost=1.0):
+    g = np.random.default_rng(seed)
+    A = g.standard_normal((T, D)) * np.linspace(1.0, cond_boost, D)
+    R = A @ g.standard_normal((D, Dout)) * 0.1 + 0.05 * g.standard_normal((T, Dout))
+    G = (A.T @ A).astype(np.float32)
+    C = (A.T @ R).astype(np.float32)
+    r2 = float(np.sum(R * R))
+    return G, C, r2
+
+
+def _run_ridge(G, C, r2, lam, rel, refine):
+    D, Dout = C.shape
+    dW = nan_like((D, Dout), torch.float32)
+    eps = torch.zeros(1, dtype=torch.float64, device="cuda")
+    ws = torch.empty(ispa.ispa_ridge_workspace_bytes(D, Dout), dtype=torch.uint8, device="cuda")
+    ispa.ispa_ridge_solve(D, Dout, dev(np.triu(G)), dev(C), dev(np.array([r2]), torch.float64), lam, rel, refine, dW,
+                          eps, ws)
+    ispa.ispa_check_device_error()
+    return host(dW), float(eps.item())
+
+
+@pytest.mark.parametrize("D,Dout,refine", [(64, 64, 0), (200, 136, 0), (1536, 1536, 0), (64, 64, 3), (333, 77, 2)])
+def test_ridge_solve_matches_oracle(D, Dout, refine):
+    G, C, r2 = _spd_problem(D, Dout, 3 * D, D + Dout)
+    Gs = np.triu(G).astype(np.float64)
+    Gs = Gs + np.triu(Gs, 1).T  # the symmetric matrix the upper triangle stands for
+    lam = orc.ridge_lambda(Gs, 1e-4, True)
+    dW, eps = _run_ridge(G, C, r2, 1e-4, True, refine)
+    lam32 = float(np.float32(lam))
+    ref = orc.ridge_solve(Gs, C.astype(np.float64), lam32)
+    err = rel_fro(dW, ref)
+    assert err <= (1e-5 if refine else 1e-2), err
+    ref_eps = orc.eps_from_stats(Gs, C.astype(np.float64), r2, dW.astype(np.float64))
+    assert abs(eps - ref_eps) <= 1e-6 * r2, (eps, ref_eps, r2)
+
+
+def test_ridge_absolute_lambda_and_identity():
+    D = 96
+    G = np.eye(D, dtype=np.float32) * 2.0
+    C = np.random.default_rng(3).standard_normal((D, D)).astype(np.float32)
+    dW, eps = _run_ridge(G, C, 10.0, 0.5, False, 0)
+    assert np.abs(dW - C / 2.5).max() <= 1e-6 * np.abs(C).max()
+
+
+def test_ridge_not_spd_reports_and_fills_nan():
+    D = 80
+    G = np.eye(D, dtype=np.float32)
+    G[40, 40] = -5.0
+    C = np.ones((D, D), dtype=np.float32)
+    dW = nan_like((D, D), torch.float32)
+    eps = torch.zeros(1, dtype=torch.float64, device="cuda")
+    ws = torch.empty(ispa.ispa_ridge_workspace_bytes(D, D), dtype=torch.uint8, device="cuda")
+    ispa.ispa_ridge_solve(D, D, dev(G), dev(C), dev(np.array([1.0]), torch.float64), 0.0, False, 0, dW, eps, ws)
+    with pytest.raises(ispa.IspaError) as ei:
+        ispa.ispa_check_device_error()
+    assert ei.value.status == ispa.ISPA_ERR_NOT_SPD
+    assert torch.isnan(dW).all().item() and math.isnan(eps.item())
+    assert ispa.ispa_check_device_error() == 0  # cleared
+
+
+# ---------------------------------------------------------------- weight correction
+def test_absorb_weight_rounding():
+    g = np.random.default_rng(4)
+    D, Dout = 64, 96
+    W = si.round_to_bf16(g.standard_normal((D, Dout)).astype(np.float32))
+    dW = (0.01 * g.standard_normal((D, Dout))).astype(np.float32)
+    out = torch.empty((D, Dout), dtype=torch.bfloat16, device="cuda")
+    ispa.ispa_absorb_weight(D, Dout, dev(W, torch.bfloat16), ispa.ISPA_BF16, dev(dW), out, ispa.ISPA_BF16)
+    out32 = torch.empty((D, Dout), dtype=torch.float32, device="cuda")
+    ispa.ispa_absorb_weight(D, Dout, dev(W), ispa.ISPA_F32, dev(dW), out32, ispa.ISPA_F32)
+    torch.cuda.synchronize()
+    exact = (W + dW).astype(np.float32)
+    assert np.array_equal(host(out32).astype(np.float32), exact)
+    assert np.array_equal(host(out).astype(np.float32), si.round_to_bf16(exact))
+
+
+# ---------------------------------------------------------------- post-switch projection
+@pytest.mark.parametrize("y_dt", [ispa.ISPA_F32, ispa.ISPA_BF16])
+def test_attn_local_proj(y_dt):
+    sh = si.AttnShape(B=2, H=2, d=128, tpf=45, sink_frames=2, hist_begin=2, hist_end=6, cur_begin=6, cur_end=9,
+                      kv_frames=9)
+    data = si.iid_qkv(sh, "bf16", ("gpu", "proj"))
+    D, Dout = sh.D, 192
+    W = si.projection_weight(D, Dout, ("gpu", "proj"), "bf16")
+    dW = (0.02 * np.random.default_rng(5).standard_normal((D, Dout))).astype(np.float32)
+    Wn = torch.empty((D, Dout), dtype=torch.bfloat16, device="cuda")
+    ispa.ispa_absorb_weight(D, Dout, dev(W, torch.bfloat16), ispa.ISPA_BF16, dev(dW), Wn, ispa.ISPA_BF16)
+    desc = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_BF16)
+    ws = torch.empty(ispa.ispa_attn_local_proj_workspace_bytes(desc), dtype=torch.uint8, device="cuda")
+    tdt = torch.bfloat16 if y_dt == ispa.ISPA_BF16 else torch.float32
+    y = nan_like((sh.B, sh.Lq, Dout), tdt)
+    ispa.ispa_attn_local_proj(desc, dev(data["q"], torch.bfloat16), dev(data["k"], torch.bfloat16),
+                              dev(data["v"], torch.bfloat16), Wn, Dout, y, y_dt, ws)
+    torch.cuda.synchronize()
+    ref = orc.local_projection(sh, data["q"], data["k"], data["v"], W, dW)
+    got = host(y)
+    if y_dt == ispa.ISPA_BF16:
+        assert_bf16_out(got, ref)
+    else:
+        assert max_over_rms(got, ref) <= 1e-2, max_over_rms(got, ref)
