@@ -67,6 +67,13 @@ const char *ispa_version(void);
 const char *ispa_last_error(void);
 
 /*
+ * Number of kernels this library has enqueued in this process, over all
+ * threads and devices (a monotonically increasing diagnostic counter; the
+ * difference across a region counts the library's launches in it).
+ */
+uint64_t ispa_launch_count(void);
+
+/*
  * Synchronises `stream`, then reads and clears the error word of the current
  * device.  Returns ISPA_OK, ISPA_ERR_NOT_SPD or ISPA_ERR_TIMEOUT (or
  * ISPA_ERR_CUDA if the synchronisation itself failed).  `detail` (optional,

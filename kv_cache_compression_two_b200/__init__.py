@@ -28,7 +28,7 @@ STATUS_NAMES = {0: "ISPA_OK", 1: "ISPA_ERR_INVALID_ARG", 2: "ISPA_ERR_UNSUPPORTE
                 4: "ISPA_ERR_NOT_SPD", 5: "ISPA_ERR_TIMEOUT"}
 
 # Every entry point declared in include/ispa.h.
-EXPORTED = ("ispa_version", "ispa_last_error", "ispa_check_device_error", "ispa_attn_split", "ispa_lse_merge",
+EXPORTED = ("ispa_version", "ispa_last_error", "ispa_launch_count", "ispa_check_device_error", "ispa_attn_split", "ispa_lse_merge",
             "ispa_accum_stats_workspace_bytes", "ispa_accum_stats", "ispa_ridge_workspace_bytes", "ispa_ridge_solve",
             "ispa_select_layers", "ispa_absorb_weight", "ispa_attn_local_proj_workspace_bytes",
             "ispa_attn_local_proj")
@@ -65,11 +65,12 @@ def lib() -> ctypes.CDLL:
         return _lib
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"libispa.so not found at {LIB_PATH}; build it with "
-                          "`python -m kv_cache_compression_two_b200.build` (needs nvcc)")
+                          "`python kv_cache_compression_two_b200/build.py` (needs nvcc)")
     L = ctypes.CDLL(LIB_PATH)
     sig = {
         "ispa_version": (ctypes.c_char_p, []),
         "ispa_last_error": (ctypes.c_char_p, []),
+        "ispa_launch_count": (ctypes.c_uint64, []),
         "ispa_check_device_error": (_ci, [_vp, ctypes.POINTER(_ci)]),
         "ispa_attn_split": (_ci, [ctypes.POINTER(AttnDesc)] + [_vp] * 9 + [_vp]),
         "ispa_lse_merge": (_ci, [_ci, _ci, _ci, _ci, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
@@ -133,6 +134,11 @@ def _dt(t) -> int:
 
 def version() -> str:
     return lib().ispa_version().decode()
+
+
+def launch_count() -> int:
+    """Kernels enqueued by libispa so far in this process."""
+    return int(lib().ispa_launch_count())
 
 
 def ispa_check_device_error(stream=None) -> int:

@@ -4,7 +4,9 @@ Every .cu file under csrc/ is compiled in parallel to an object under _build/,
 then linked with the static CUDA runtime into ``libispa.so`` next to this file.
 Objects are rebuilt when their source, a header or the flags change.
 
-    python -m kv_cache_compression_two_b200.build [--force] [--verbose]
+    python kv_cache_compression_two_b200/build.py [--force] [--verbose]
+
+(run by path: importing the package loads the library it builds)
 """
 from __future__ import annotations
 

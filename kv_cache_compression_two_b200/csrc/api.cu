@@ -11,9 +11,14 @@
 // Per-device error word: [0] ispa_status of the first device-side failure, [1] its detail.
 __device__ int g_ispa_device_error[2];
 
+#include <atomic>
+
 namespace ispa {
 
 static thread_local char t_last_error[512] = "";
+static std::atomic<unsigned long long> g_launches{0};
+
+void note_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 
 ispa_status fail(ispa_status st, const char *fmt, ...) {
   va_list ap;
@@ -173,6 +178,8 @@ extern "C" {
 const char *ispa_version(void) { return "ispa-b200 0.1 (sm_100a)"; }
 
 const char *ispa_last_error(void) { return t_last_error; }
+
+uint64_t ispa_launch_count(void) { return (uint64_t)g_launches.load(std::memory_order_relaxed); }
 
 ispa_status ispa_check_device_error(ispa_stream_t stream, int *detail) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);

@@ -151,6 +151,7 @@ ispa_status launch_d(const ispa_attn_desc &d, const GroupRanges &g, float scale,
   dim3 grid((g.Lq + kWarps - 1) / kWarps, d.H, d.B);
   attn_simt_kernel<D, TO><<<grid, kWarps * 32, 0, s>>>(g, d.H, scale, q, k, v, (TO *)o_loc, l_loc,
                                                        (TO *)o_hist, l_hist, (TO *)o_full, l_full);
+  note_launch();
   return cuda_status(cudaGetLastError(), "attn_simt launch");
 }
 

@@ -442,6 +442,7 @@ ispa_status launch_typed(const CUtensorMap &tq, const CUtensorMap &tk, const CUt
   }
   dim3 grid(P.q_tiles * P.H, B);
   attn_tc_kernel<TO><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, P);
+  note_launch();
   return cuda_status(cudaGetLastError(), "tcgen05 attention launch");
 }
 

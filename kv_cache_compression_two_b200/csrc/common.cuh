@@ -17,6 +17,9 @@
 
 namespace ispa {
 
+// Host side: counts kernels enqueued by the library (see ispa_launch_count).
+void note_launch(int n = 1);
+
 // ---------------------------------------------------------------------------
 // device error word: [0] = ispa_status code (first one wins), [1] = detail
 // ---------------------------------------------------------------------------
@@ -226,14 +229,23 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 //     groups SBO bytes apart; LBO unused.
 //   MN-major operand: 128 B along M/N per row, 8-row groups along K SBO bytes
 //     apart, consecutive 128 B chunks along M/N LBO bytes apart.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+//   layout 2 = SWIZZLE_128B (16-byte chunks XOR row mod 8, 8-row atoms);
+//   layout 1 = SWIZZLE_128B_BASE32B (32-byte chunks XOR row mod 4, 4-row atoms),
+//   the form 32-bit (tf32) MN-major operands need; TMA writes it with
+//   CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                              uint32_t layout) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
   d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
   d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1 << 46;  // descriptor version (sm_100)
-  d |= (uint64_t)2 << 61;  // SWIZZLE_128B
+  d |= (uint64_t)layout << 61;
   return d;
+}
+
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return smem_desc(saddr, lbo_bytes, sbo_bytes, 2);
 }
 
 // Instruction descriptor for kind::f16 / kind::tf32 with fp32 accumulation.

@@ -96,6 +96,7 @@ ispa_status launch_lse_merge(int rows, int H, int d, ispa_dtype dt, const void *
   else
     lse_merge_bf16_kernel<<<grid, 256, 0, s>>>(n_vec, vph, (const uint4 *)oa, la, (const uint4 *)ob, lb,
                                                (uint4 *)oo, lo);
+  note_launch();
   return cuda_status(cudaGetLastError(), "lse_merge launch");
 }
 
@@ -140,6 +141,7 @@ ispa_status launch_absorb_weight(int D, int Dout, const void *W, ispa_dtype wdt,
   else
     absorb_weight_kernel<__nv_bfloat16, __nv_bfloat16>
         <<<grid, 256, 0, s>>>(n4, (const __nv_bfloat16 *)W, d4, (__nv_bfloat16 *)Wn);
+  note_launch();
   return cuda_status(cudaGetLastError(), "absorb_weight launch");
 }
 
@@ -179,6 +181,7 @@ __global__ void __launch_bounds__(1024) select_kernel(int N, const double *__res
 ispa_status launch_select(int N, const double *eps, int K, unsigned char *is_local, int *idx, cudaStream_t s) {
   if (N == 0) return ISPA_OK;
   select_kernel<<<1, 1024, 0, s>>>(N, eps, K, is_local, idx);
+  note_launch();
   return cuda_status(cudaGetLastError(), "select launch");
 }
 

@@ -18,6 +18,7 @@ ispa_status launch_tc_gemm(const CUtensorMap &ta, const CUtensorMap &tb0, const 
     configured_device = dev;
   }
   tcg::gemm_kernel<<<P.n_tiles, tcg::THREADS, tcg::SMEM_BYTES, s>>>(ta, tb0, tb1, P);
+  note_launch();
   return cuda_status(cudaGetLastError(), "tcgen05 gemm launch");
 }
 

@@ -243,11 +243,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         const uint32_t a_base = smem_u32(sA + s * TILE_BYTES);
         const uint32_t b_base = smem_u32(sB + s * TILE_BYTES);
+        // MN-major: bf16 uses 8-row SWIZZLE_128B atoms (SBO = 1024 B between them),
+        // tf32 uses 4-row SWIZZLE_128B_BASE32B atoms (SBO = 512 B).
+        const uint32_t mn_layout = P.kind_tf32 ? 1u : 2u;
+        const uint32_t mn_sbo = P.kind_tf32 ? 512u : 1024u;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t ad = P.a_mn ? smem_desc_sw128(a_base + ks * kstep_mn, mn_box_bytes, 1024)
+          const uint64_t ad = P.a_mn ? smem_desc(a_base + ks * kstep_mn, mn_box_bytes, mn_sbo, mn_layout)
                                      : smem_desc_sw128(a_base + ks * kstep_kmajor, 16, 1024);
-          const uint64_t bd = P.b_mn ? smem_desc_sw128(b_base + ks * kstep_mn, mn_box_bytes, 1024)
+          const uint64_t bd = P.b_mn ? smem_desc(b_base + ks * kstep_mn, mn_box_bytes, mn_sbo, mn_layout)
                                      : smem_desc_sw128(b_base + ks * kstep_kmajor, 16, 1024);
           mma_ss(tmem, ad, bd, P.idesc, (kt > 0 || ks > 0) ? 1u : 0u, P.kind_tf32);
         }

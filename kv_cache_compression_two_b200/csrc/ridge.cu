@@ -242,6 +242,7 @@ cudaError_t cholesky_solve(int D, int Dout, const float *L, float *Y, cudaStream
   for (int kb0 = 0; kb0 < D; kb0 += NB) {
     const int nb = min(NB, D - kb0);
     trsv_fwd_kernel<<<cgrid, 128, 0, s>>>(D, Dout, kb0, L, Y);
+    note_launch();
     const int below = D - kb0 - nb;
     if (below > 0) {
       cudaError_t e = simt_gemm<OP_N, OP_N, float, 0>(
@@ -255,6 +256,7 @@ cudaError_t cholesky_solve(int D, int Dout, const float *L, float *Y, cudaStream
   for (int kb0 = last0; kb0 >= 0; kb0 -= NB) {
     const int nb = min(NB, D - kb0);
     trsv_bwd_kernel<<<cgrid, 128, 0, s>>>(D, Dout, kb0, L, Y);
+    note_launch();
     if (kb0 > 0) {
       cudaError_t e = simt_gemm<OP_T, OP_N, float, 0>(kb0, Dout, nb, Operand{L + (long long)kb0 * D, nullptr, D},
                                                       Operand{Y + (long long)kb0 * Dout, nullptr, Dout},
@@ -281,11 +283,14 @@ ispa_status launch_ridge(int D, int Dout, const float *G, const float *C, const 
   const int grid = sm_count() * 4;
   trace_kernel<<<1, 256, 0, s>>>(D, G, w.acc);
   init_kernel<<<grid, 256, 0, s>>>(D, Dout, G, C, lambda, lambda_relative, w, dW);
+  note_launch(2);
   for (int kb0 = 0; kb0 < D; kb0 += NB) {
     potrf_diag_kernel<<<1, 64, 0, s>>>(D, kb0, w.L, w.flag, err);
+    note_launch();
     const int below = D - kb0 - NB;
     if (below > 0) {
       trsm_panel_kernel<<<(below + NB - 1) / NB, 64, 0, s>>>(D, kb0, w.L);
+      note_launch();
       const int j0 = kb0 + NB;
       cudaError_t e = simt_gemm<OP_N, OP_T, float, 1>(
           below, below, NB, Operand{w.L + (long long)j0 * D + kb0, nullptr, D},
@@ -304,12 +309,15 @@ ispa_status launch_ridge(int D, int Dout, const float *G, const float *C, const 
     e = cholesky_solve(D, Dout, w.L, w.Rres, s);
     if (e != cudaSuccess) return cuda_status(e, "ridge refinement solve");
     add_kernel<<<grid, 256, 0, s>>>(nDO, dW, w.Rres);
+    note_launch();
   }
   dot_kernel<<<grid, 256, 0, s>>>(nDO, dW, C, w.acc);
+  note_launch();
   e = simt_gemm<OP_SYM_UPPER, OP_N, float, 0>(D, Dout, D, Operand{G, nullptr, D}, Operand{dW, nullptr, Dout},
                                               EpiDotG{dW, w.acc, Dout, 0.0}, s);
   if (e != cudaSuccess) return cuda_status(e, "ridge G dW");
   finalize_kernel<<<grid, 256, 0, s>>>(nDO, r2, w, dW, eps);
+  note_launch();
   return cuda_status(cudaGetLastError(), "ridge launch");
 }
 

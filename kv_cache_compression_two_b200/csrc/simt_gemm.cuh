@@ -95,6 +95,7 @@ inline cudaError_t simt_gemm(int M, int N, int K, Operand A, Operand B, Epi epi,
   if (M <= 0 || N <= 0) return cudaSuccess;
   dim3 grid((N + 63) / 64, (M + 63) / 64);
   simt_gemm_kernel<KA, KB, Acc, TRI, Epi><<<grid, 256, 0, s>>>(M, N, K, A, B, epi);
+  note_launch();
   return cudaGetLastError();
 }
 

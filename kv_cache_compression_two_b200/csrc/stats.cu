@@ -72,11 +72,15 @@ TF32Ws carve_tf32(void *ws, int T, int D, int Dout) {
   return w;
 }
 
-ispa_status map2d_f32(CUtensorMap *m, const void *base, int inner, int outer, int box_inner, int box_outer) {
+// fp32 map of a row-major [outer, inner] matrix.  K-major operands use the
+// 128-byte swizzle; MN-major tf32 operands the 128-byte swizzle with 32-byte atoms.
+ispa_status map2d_f32(CUtensorMap *m, const void *base, int inner, int outer, int box_inner, int box_outer,
+                      bool mn_major) {
   const uint64_t dims[2] = {(uint64_t)inner, (uint64_t)outer};
   const uint64_t strides[1] = {(uint64_t)inner * 4};
   const uint32_t box[2] = {(uint32_t)box_inner, (uint32_t)box_outer};
-  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box,
+                   mn_major ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace
@@ -112,14 +116,15 @@ ispa_status launch_stats(int T, int D, int Dout, const float *a_loc, const float
   const long long n4_rows = (long long)T * D / 4, n4_w = (long long)D * Dout / 4;
   prep_tf32_kernel<<<sm_count() * 8, 256, 0, s>>>(n4_rows, n4_w, (const float4 *)a_loc, (const float4 *)a_full,
                                                   (const float4 *)W, (float4 *)w.dA, (float4 *)w.Ar, (float4 *)w.Wr);
+  note_launch();
   st = cuda_status(cudaGetLastError(), "stats prep launch");
   if (st != ISPA_OK) return st;
 
   // launch 1: R = dA W
   {
     CUtensorMap ta, tb;
-    if ((st = map2d_f32(&ta, w.dA, D, T, 32, 128)) != ISPA_OK) return st;
-    if ((st = map2d_f32(&tb, w.Wr, Dout, D, 32, 32)) != ISPA_OK) return st;
+    if ((st = map2d_f32(&ta, w.dA, D, T, 32, 128, false)) != ISPA_OK) return st;
+    if ((st = map2d_f32(&tb, w.Wr, Dout, D, 32, 32, true)) != ISPA_OK) return st;
     tcg::Params P{};
     P.M = T;
     P.K = D;
@@ -139,8 +144,8 @@ ispa_status launch_stats(int T, int D, int Dout, const float *a_loc, const float
   // launch 2: G (upper) += Ar^T Ar, C += Ar^T R
   {
     CUtensorMap ta, tr;
-    if ((st = map2d_f32(&ta, w.Ar, D, T, 32, 32)) != ISPA_OK) return st;
-    if ((st = map2d_f32(&tr, w.R, Dout, T, 32, 32)) != ISPA_OK) return st;
+    if ((st = map2d_f32(&ta, w.Ar, D, T, 32, 32, true)) != ISPA_OK) return st;
+    if ((st = map2d_f32(&tr, w.R, Dout, T, 32, 32, true)) != ISPA_OK) return st;
     tcg::Params P{};
     P.M = D;
     P.K = T;
