@@ -96,6 +96,11 @@ def reduce_over_ranks(value: float, op: str, device) -> float:
     return float(t.item())
 
 
+def aggregate_value(flops_per_step: float, max_ms_per_step: float, world: int) -> float:
+    """Whole-job TFLOP/s: every replica's work over the slowest replica's step time."""
+    return world * flops_per_step / (max_ms_per_step * 1e-3) / 1e12
+
+
 def barrier(device):
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized():
@@ -207,6 +212,7 @@ def run_ours(args, world, rank, local):
     W_new = torch.empty((D, D), device=dev, dtype=torch.bfloat16)
     y = {n: torch.empty((B, Lq, D), device=dev, dtype=torch.bfloat16) for n in ("L", "F")}
     desc_warm = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_F32)
+    ws_attn = torch.empty(ispa.ispa_attn_split_workspace_bytes(desc_warm), device=dev, dtype=torch.uint8)
     desc_L = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_BF16)
     import dataclasses
     shF = dataclasses.replace(sh, sink_frames=sh.cur_begin, hist_begin=0, hist_end=0)
@@ -225,7 +231,7 @@ def run_ours(args, world, rank, local):
         if timed_components:
             ev_attn[0].record(stream)
         ispa.ispa_attn_split(desc_warm, Lw.dev["q"], Lw.dev["k"], Lw.dev["v"], o["loc"], l["loc"], o["hist"],
-                             l["hist"], o["full"], l["full"], stream=stream)
+                             l["hist"], o["full"], l["full"], workspace=ws_attn, stream=stream)
         if timed_components:
             ev_attn[1].record(stream)
         ispa.ispa_accum_stats(T, D, D, o["loc"], o["full"], W32, G, C, r2, ispa.ISPA_PREC_TF32, ws_stats,
@@ -410,8 +416,9 @@ def run_attn_only(args):
     o = {n: torch.empty((sh.B, sh.Lq, sh.H, 128), **f32) for n in ("loc", "hist", "full")}
     l = {n: torch.empty((sh.B, sh.Lq, sh.H), **f32) for n in ("loc", "hist", "full")}
     desc = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_F32)
+    ws = torch.empty(ispa.ispa_attn_split_workspace_bytes(desc), device=dev, dtype=torch.uint8)
     run = lambda: ispa.ispa_attn_split(desc, L.dev["q"], L.dev["k"], L.dev["v"], o["loc"], l["loc"], o["hist"],
-                                       l["hist"], o["full"], l["full"])
+                                       l["hist"], o["full"], l["full"], workspace=ws)
     for _ in range(args.warmup):
         run()
     torch.cuda.synchronize()
@@ -472,7 +479,7 @@ def main(argv=None):
     r = run_ours(args, world, rank, local)
     if rank == 0:
         work = r["work"]
-        value = world * work["total"] / (r["ms_step"] * 1e-3) / 1e12
+        value = aggregate_value(work["total"], r["ms_step"], world)
         peaks = {}
         try:
             peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))

@@ -129,11 +129,18 @@ typedef struct {
  * An empty group yields O = 0 and L = -inf.  Compiled paths: bf16 in with
  * head_dim 128 (tcgen05 tensor cores, fp32 accumulation) and fp32 in with
  * head_dim 32/64/128 (fp32 CUDA cores).  Outputs may not alias inputs.
+ * Every K/V row that a group's 128-row tiles cover must hold finite values.
+ *   workspace  >= ispa_attn_split_workspace_bytes(desc) bytes, 16-byte aligned
+ *              (0 for fp32 inputs; for bf16 inputs it holds a power-of-two
+ *              scaled fp16 copy of the V rows in use, so that the softmax
+ *              weights enter the PV product with 11 significant bits).
  */
+size_t ispa_attn_split_workspace_bytes(const ispa_attn_desc *desc);
+
 ispa_status ispa_attn_split(const ispa_attn_desc *desc, const void *q, const void *k,
                             const void *v, void *o_loc, float *lse_loc, void *o_hist,
-                            float *lse_hist, void *o_full, float *lse_full,
-                            ispa_stream_t stream);
+                            float *lse_hist, void *o_full, float *lse_full, void *workspace,
+                            size_t workspace_bytes, ispa_stream_t stream);
 
 /*
  * LSE-weighted merge of two disjoint groups' results [EN-notes, Key Designs 1]:
@@ -230,7 +237,8 @@ size_t ispa_attn_local_proj_workspace_bytes(const ispa_attn_desc *desc);
  *   q, k, v   as for ispa_attn_split (bf16, head_dim 128)
  *   W_proj    [D, Dout] bf16,  D = H * head_dim,  Dout % 16 == 0
  *   y         [B, Lq, Dout] in y_dtype
- *   workspace >= ispa_attn_local_proj_workspace_bytes(desc) (holds A_loc in bf16)
+ *   workspace >= ispa_attn_local_proj_workspace_bytes(desc) (holds A_loc in bf16
+ *             and the attention workspace)
  */
 ispa_status ispa_attn_local_proj(const ispa_attn_desc *desc, const void *q, const void *k,
                                  const void *v, const void *W_proj, int Dout, void *y,

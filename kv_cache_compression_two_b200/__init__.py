@@ -28,7 +28,7 @@ STATUS_NAMES = {0: "ISPA_OK", 1: "ISPA_ERR_INVALID_ARG", 2: "ISPA_ERR_UNSUPPORTE
                 4: "ISPA_ERR_NOT_SPD", 5: "ISPA_ERR_TIMEOUT"}
 
 # Every entry point declared in include/ispa.h.
-EXPORTED = ("ispa_version", "ispa_last_error", "ispa_launch_count", "ispa_check_device_error", "ispa_attn_split", "ispa_lse_merge",
+EXPORTED = ("ispa_version", "ispa_last_error", "ispa_launch_count", "ispa_check_device_error", "ispa_attn_split_workspace_bytes", "ispa_attn_split", "ispa_lse_merge",
             "ispa_accum_stats_workspace_bytes", "ispa_accum_stats", "ispa_ridge_workspace_bytes", "ispa_ridge_solve",
             "ispa_select_layers", "ispa_absorb_weight", "ispa_attn_local_proj_workspace_bytes",
             "ispa_attn_local_proj")
@@ -72,7 +72,8 @@ def lib() -> ctypes.CDLL:
         "ispa_last_error": (ctypes.c_char_p, []),
         "ispa_launch_count": (ctypes.c_uint64, []),
         "ispa_check_device_error": (_ci, [_vp, ctypes.POINTER(_ci)]),
-        "ispa_attn_split": (_ci, [ctypes.POINTER(AttnDesc)] + [_vp] * 9 + [_vp]),
+        "ispa_attn_split_workspace_bytes": (_sz, [ctypes.POINTER(AttnDesc)]),
+        "ispa_attn_split": (_ci, [ctypes.POINTER(AttnDesc)] + [_vp] * 10 + [_sz, _vp]),
         "ispa_lse_merge": (_ci, [_ci, _ci, _ci, _ci, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
         "ispa_accum_stats_workspace_bytes": (_sz, [_ci, _ci, _ci, _ci]),
         "ispa_accum_stats": (_ci, [_ci, _ci, _ci, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _vp, _sz, _vp]),
@@ -147,12 +148,23 @@ def ispa_check_device_error(stream=None) -> int:
     return detail.value
 
 
+def _ws(workspace, workspace_bytes):
+    if workspace is not None and not isinstance(workspace, int):
+        return _ptr(workspace, name="workspace"), workspace_bytes or workspace.numel() * workspace.element_size()
+    return workspace, workspace_bytes
+
+
+def ispa_attn_split_workspace_bytes(desc: AttnDesc) -> int:
+    return int(lib().ispa_attn_split_workspace_bytes(ctypes.byref(desc)))
+
+
 def ispa_attn_split(desc: AttnDesc, q, k, v, o_loc, lse_loc, o_hist=None, lse_hist=None, o_full=None, lse_full=None,
-                    stream=None) -> None:
+                    workspace=None, workspace_bytes: int = 0, stream=None) -> None:
+    ws, nbytes = _ws(workspace, workspace_bytes)
     _check(lib().ispa_attn_split(ctypes.byref(desc), _ptr(q, name="q"), _ptr(k, name="k"), _ptr(v, name="v"),
                                  _ptr(o_loc, name="o_loc"), _ptr(lse_loc, name="lse_loc"), _ptr(o_hist, name="o_hist"),
                                  _ptr(lse_hist, name="lse_hist"), _ptr(o_full, name="o_full"),
-                                 _ptr(lse_full, name="lse_full"), _stream(stream)))
+                                 _ptr(lse_full, name="lse_full"), ws, nbytes, _stream(stream)))
 
 
 def ispa_lse_merge(rows: int, H: int, head_dim: int, o_dtype: int, o_a, lse_a, o_b, lse_b, o_out, lse_out,

@@ -201,13 +201,24 @@ ispa_status ispa_check_device_error(ispa_stream_t stream, int *detail) {
   return ISPA_OK;
 }
 
+size_t ispa_attn_split_workspace_bytes(const ispa_attn_desc *desc) {
+  GroupRanges g;
+  float scale;
+  if (attn_ranges(desc, &g, &scale) != ISPA_OK) return 0;
+  if (desc->in_dtype != ISPA_BF16) return 0;
+  return attn_tc_workspace_bytes(desc->B, desc->H, g.Lkv);
+}
+
 ispa_status ispa_attn_split(const ispa_attn_desc *desc, const void *q, const void *k, const void *v, void *o_loc,
                             float *lse_loc, void *o_hist, float *lse_hist, void *o_full, float *lse_full,
-                            ispa_stream_t stream) {
+                            void *workspace, size_t workspace_bytes, ispa_stream_t stream) {
   GroupRanges g;
   float scale;
   ispa_status st = attn_ranges(desc, &g, &scale);
   if (st != ISPA_OK) return st;
+  const size_t need = ispa_attn_split_workspace_bytes(desc);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+    return fail(ISPA_ERR_INVALID_ARG, "workspace needs %zu bytes (16-byte aligned)", need);
   if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v)) return fail(ISPA_ERR_INVALID_ARG, "q, k, v must be 16-byte aligned device pointers");
   if (!ptr_ok(o_loc) || !ptr_ok(lse_loc)) return fail(ISPA_ERR_INVALID_ARG, "o_loc and lse_loc are required (16-byte aligned)");
   if ((o_hist == nullptr) != (lse_hist == nullptr)) return fail(ISPA_ERR_INVALID_ARG, "o_hist and lse_hist: both or neither");
@@ -217,7 +228,7 @@ ispa_status ispa_attn_split(const ispa_attn_desc *desc, const void *q, const voi
     return fail(ISPA_ERR_INVALID_ARG, "outputs must be 16-byte aligned");
   if (desc->in_dtype == ISPA_BF16) {
     if (desc->head_dim != 128) return fail(ISPA_ERR_UNSUPPORTED, "bf16 attention is compiled for head_dim 128 only");
-    return launch_attn_tc(*desc, g, scale, q, k, v, o_loc, lse_loc, o_hist, lse_hist, o_full, lse_full,
+    return launch_attn_tc(*desc, g, scale, q, k, v, o_loc, lse_loc, o_hist, lse_hist, o_full, lse_full, workspace,
                           (cudaStream_t)stream);
   }
   return launch_attn_simt(*desc, g, scale, (const float *)q, (const float *)k, (const float *)v, o_loc, lse_loc, o_hist,
@@ -307,7 +318,8 @@ size_t ispa_attn_local_proj_workspace_bytes(const ispa_attn_desc *desc) {
   if (attn_ranges(desc, &g, &scale) != ISPA_OK) return 0;
   const size_t a = (size_t)desc->B * g.Lq * desc->H * desc->head_dim * 2;
   const size_t l = (size_t)desc->B * g.Lq * desc->H * 4;
-  return ((a + 255) & ~size_t(255)) + ((l + 255) & ~size_t(255));
+  return ((a + 255) & ~size_t(255)) + ((l + 255) & ~size_t(255)) +
+         attn_tc_workspace_bytes(desc->B, desc->H, g.Lkv);
 }
 
 ispa_status ispa_attn_local_proj(const ispa_attn_desc *desc, const void *q, const void *k, const void *v,
@@ -331,9 +343,12 @@ ispa_status ispa_attn_local_proj(const ispa_attn_desc *desc, const void *q, cons
   d.out_dtype = ISPA_BF16;
   g.hist_begin = g.hist_end = 0;
   const size_t a_bytes = (((size_t)d.B * g.Lq * d.H * d.head_dim * 2) + 255) & ~size_t(255);
+  const size_t l_bytes = (((size_t)d.B * g.Lq * d.H * 4) + 255) & ~size_t(255);
   void *a_loc = workspace;
   float *lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + a_bytes);
-  st = launch_attn_tc(d, g, scale, q, k, v, a_loc, lse, nullptr, nullptr, nullptr, nullptr, (cudaStream_t)stream);
+  void *attn_ws = static_cast<char *>(workspace) + a_bytes + l_bytes;
+  st = launch_attn_tc(d, g, scale, q, k, v, a_loc, lse, nullptr, nullptr, nullptr, nullptr, attn_ws,
+                      (cudaStream_t)stream);
   if (st != ISPA_OK) return st;
   const int D = d.H * d.head_dim;
   return launch_gemm_bf16(d.B * g.Lq, Dout, D, a_loc, W_proj, y, y_dtype, (cudaStream_t)stream);

@@ -53,10 +53,105 @@ struct AttnParams {
   int r_begin[3], r_end[3];
   int n_loc_tiles, n_tiles;
   float scale_log2;        // softmax scale * log2(e)
+  const float *v_unscale;  // [B * H]: 2^-s of the fp16 copy of V (see prepare_v)
   void *o_loc, *o_hist, *o_full;
   float *l_loc, *l_hist, *l_full;
   DevErr err;
 };
+
+// ---------------------------------------------------------------------------
+// fp16 copy of V.  P = exp(S - m) is rounded to 16 bits before the PV product;
+// in fp16 (11 significant bits) that rounding is 8x finer than in bf16, which
+// keeps the output error well inside the parity tolerance.  tcgen05 kind::f16
+// needs both operands in the same type, so V is converted once per call:
+// each head of each instance is scaled by a power of two 2^s so that its
+// largest |v| lies in [2^14, 2^15) (exact in fp16, far from overflow), and the
+// epilogue multiplies O by 2^-s (exact).  Only the rows the tiles read are
+// converted: every range rounded up to whole 128-row tiles.
+// ---------------------------------------------------------------------------
+struct VPrep {
+  int B, H, Lkv;
+  int n_ext;
+  int ext_begin[3], ext_end[3];  // row extents the tiles touch
+};
+
+// Per-(instance, head) max |v|.  Each thread keeps one 16-byte column group c8
+// (8 values of one head) and walks rows; the 16 lanes that cover one head
+// combine by shuffles and one lane per head issues the atomic.
+__global__ void __launch_bounds__(256) v_amax_kernel(VPrep p, const __nv_bfloat16 *__restrict__ v,
+                                                     unsigned int *amax_bits) {
+  const int D = p.H * kD;
+  const int vec_per_row = D / 8;                       // multiple of 16 (kD / 8 = 16 per head)
+  const int b = blockIdx.y;
+  const int lanes = gridDim.x * blockDim.x;
+  const int row_step = lanes / vec_per_row;            // rows advanced per pass (>= 1 by the launch)
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+  const int c8 = tid % vec_per_row;
+  const int r0 = tid / vec_per_row;
+  float m = 0.f;
+  if (r0 < row_step) {
+    for (int e = 0; e < p.n_ext; ++e)
+      for (int row = p.ext_begin[e] + r0; row < p.ext_end[e]; row += row_step) {
+        const uint4 in = __ldg(reinterpret_cast<const uint4 *>(v + ((long long)b * p.Lkv + row) * D) + c8);
+        const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[j]));
+          m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+      }
+  }
+  // vec_per_row = 16 H and warps start at multiples of 32, so lanes 16k..16k+15
+  // hold the 16 column groups of one head of one row: reduce them by shuffles.
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 15) == 0 && r0 < row_step) atomicMax(amax_bits + b * p.H + (c8 * 8) / kD, __float_as_uint(m));
+}
+
+__device__ __forceinline__ int v_exponent(unsigned int amax_bits) {
+  const float a = __uint_as_float(amax_bits);
+  if (!(a > 0.f) || !isfinite(a)) return 0;
+  return 14 - ilogbf(a);  // a * 2^s in [2^14, 2^15)
+}
+
+__global__ void __launch_bounds__(256) v_to_f16_kernel(VPrep p, const __nv_bfloat16 *__restrict__ v,
+                                                       const unsigned int *__restrict__ amax_bits, __half *v16,
+                                                       float *v_unscale) {
+  const int D = p.H * kD;
+  const int vec_per_row = D / 8;
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < p.B * p.H; i += blockDim.x) v_unscale[i] = ldexpf(1.f, -v_exponent(amax_bits[i]));
+  for (int e = 0; e < p.n_ext; ++e) {
+    const long long rows = p.ext_end[e] - p.ext_begin[e];
+    const long long n = (long long)p.B * rows * vec_per_row;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+      const int c8 = (int)(i % vec_per_row);
+      const long long br = i / vec_per_row;
+      const int b = (int)(br / rows);
+      const long long row = p.ext_begin[e] + br % rows;
+      const int h = (c8 * 8) / kD;
+      const float scale = ldexpf(1.f, v_exponent(amax_bits[b * p.H + h]));
+      const long long off = ((long long)b * p.Lkv + row) * D + c8 * 8;
+      const uint4 in = *reinterpret_cast<const uint4 *>(v + off);
+      const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[j]));
+        const float lo = fminf(fmaxf(f.x * scale, -65504.f), 65504.f);
+        const float hi = fminf(fmaxf(f.y * scale, -65504.f), 65504.f);
+        __half2 hh = __floats2half2_rn(lo, hi);
+        o[j] = *reinterpret_cast<uint32_t *>(&hh);
+      }
+      *reinterpret_cast<uint4 *>(v16 + off) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
 
 struct SmemLayout {
   uint8_t q[kTileBytes];
@@ -225,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_qk = make_idesc(128, 128, 1, 0, 0);
-      const uint32_t idesc_pv = make_idesc(128, 128, 1, 0, 1);
+      const uint32_t idesc_pv = make_idesc(128, 128, 0, 0, 1);  // fp16 P (TMEM) x fp16 V (smem)
       const uint32_t q_addr = smem_u32(sm.q);
       bool ok = wait_parity(&sm.q_full, 0, P.err, abort, 21);
       for (int j = 0; ok && j <= P.n_tiles; ++j) {
@@ -310,12 +405,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int t = 0; t < 32; ++t) s[c * 32 + t] = __uint_as_float(raw[t]);
       }
-      float mt = -INFINITY;
+      // row maximum with 8 independent partial maxima (no 128-long dependency chain)
+      float mx[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) mx[t] = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 128; ++c) {
         if (c >= n_valid) s[c] = -INFINITY;
-        mt = fmaxf(mt, s[c]);
+        mx[c & 7] = fmaxf(mx[c & 7], s[c]);
       }
+      float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       mt *= P.scale_log2;
       if (grp_first) {
         m_ref = mt;
@@ -339,9 +438,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_st16(lane_base + kColO + c * 16, o);
         }
       }
-      // P = exp2(s * scale * log2e - m_ref), packed to bf16 pairs into TMEM P[j % 2].
+      // P = exp2(s * scale * log2e - m_ref) <= 2^8, packed to fp16 pairs into TMEM P[j % 2].
       const float neg_m = -m_ref;
-      float lsum = 0.f;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
@@ -349,13 +448,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < 16; ++t) {
           const float p0 = ex2(fmaf(s[c * 32 + 2 * t], P.scale_log2, neg_m));
           const float p1 = ex2(fmaf(s[c * 32 + 2 * t + 1], P.scale_log2, neg_m));
-          lsum += p0 + p1;
-          pk[t] = pack_bf16x2(p0, p1);
+          ls[t & 3] += p0 + p1;
+          pk[t] = pack_f16x2(p0, p1);
         }
         tmem_st16(lane_base + kColP0 + (uint32_t)(j & 1) * 64 + c * 16, pk);
       }
       tmem_wait_st();
-      l += lsum;
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       tc_fence_before();
       mbar_arrive(&sm.p_full[j & 1]);
 
@@ -369,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const bool is_loc = j < P.n_loc_tiles;
-      const float inv_l = 1.f / l;
+      const float inv_l = P.v_unscale[b * P.H + h] / l;  // undoes the power-of-two scaling of V too
       const float L = (m_ref + log2f(l)) * 0.69314718055994530942f;
       float wa = 1.f, wb = 0.f, L_full = L;
       if (is_loc) {
@@ -446,27 +545,62 @@ ispa_status launch_typed(const CUtensorMap &tq, const CUtensorMap &tk, const CUt
   return cuda_status(cudaGetLastError(), "tcgen05 attention launch");
 }
 
-ispa_status map3d_bf16(CUtensorMap *m, const void *base, int D, int rows, int B) {
+ispa_status map3d_16(CUtensorMap *m, const void *base, int D, int rows, int B, CUtensorMapDataType dt) {
   const uint64_t dims[3] = {(uint64_t)D, (uint64_t)rows, (uint64_t)B};
   const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)D * 2 * (uint64_t)rows};
   const uint32_t box[3] = {64, 128, 1};
-  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  return make_tmap(m, dt, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
+
+size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
+size_t attn_tc_workspace_bytes(int B, int H, int Lkv) {
+  return a256((size_t)B * Lkv * H * kD * 2) + 2 * a256((size_t)B * H * 4);
+}
+
 ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float scale, const void *q,
                            const void *k, const void *v, void *o_loc, float *l_loc, void *o_hist, float *l_hist,
-                           void *o_full, float *l_full, cudaStream_t s) {
+                           void *o_full, float *l_full, void *workspace, cudaStream_t s) {
   if (g.Lq == 0) return ISPA_OK;
   AttnParams P{};
   ispa_status st = device_err(&P.err);
   if (st != ISPA_OK) return st;
   const int D = d.H * kD;
+
+  // ---- fp16 copy of the V rows the tiles read (workspace)
+  char *ws = static_cast<char *>(workspace);
+  __half *v16 = reinterpret_cast<__half *>(ws);
+  unsigned int *amax = reinterpret_cast<unsigned int *>(ws + a256((size_t)d.B * g.Lkv * D * 2));
+  float *v_unscale = reinterpret_cast<float *>(ws + a256((size_t)d.B * g.Lkv * D * 2) + a256((size_t)d.B * d.H * 4));
+  VPrep vp{};
+  vp.B = d.B;
+  vp.H = d.H;
+  vp.Lkv = g.Lkv;
+  auto add_ext = [&](int beg, int end) {
+    if (end <= beg) return;
+    const int tiles = (end - beg + kTileK - 1) / kTileK;
+    vp.ext_begin[vp.n_ext] = beg;
+    vp.ext_end[vp.n_ext] = min(g.Lkv, beg + tiles * kTileK);
+    ++vp.n_ext;
+  };
+  for (int r = 0; r < g.n_loc; ++r) add_ext(g.loc_begin[r], g.loc_end[r]);
+  add_ext(g.hist_begin, g.hist_end);
+  cudaError_t e = cudaMemsetAsync(amax, 0, (size_t)d.B * d.H * 4, s);
+  if (e != cudaSuccess) return cuda_status(e, "attention workspace clear");
+  const int vec_per_row = D / 8;
+  const int amax_blocks = max((vec_per_row + 255) / 256, (sm_count() * 8 + d.B - 1) / d.B);
+  v_amax_kernel<<<dim3(amax_blocks, d.B), 256, 0, s>>>(vp, static_cast<const __nv_bfloat16 *>(v), amax);
+  v_to_f16_kernel<<<sm_count() * 8, 256, 0, s>>>(vp, static_cast<const __nv_bfloat16 *>(v), amax, v16, v_unscale);
+  note_launch(2);
+  if ((st = cuda_status(cudaGetLastError(), "V conversion launch")) != ISPA_OK) return st;
+  P.v_unscale = v_unscale;
+
   CUtensorMap tq, tk, tv;
-  if ((st = map3d_bf16(&tq, q, D, g.Lq, d.B)) != ISPA_OK) return st;
-  if ((st = map3d_bf16(&tk, k, D, g.Lkv, d.B)) != ISPA_OK) return st;
-  if ((st = map3d_bf16(&tv, v, D, g.Lkv, d.B)) != ISPA_OK) return st;
+  if ((st = map3d_16(&tq, q, D, g.Lq, d.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) != ISPA_OK) return st;
+  if ((st = map3d_16(&tk, k, D, g.Lkv, d.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) != ISPA_OK) return st;
+  if ((st = map3d_16(&tv, v16, D, g.Lkv, d.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16)) != ISPA_OK) return st;
   P.H = d.H;
   P.Lq = g.Lq;
   P.q_tiles = (g.Lq + kTileQ - 1) / kTileQ;

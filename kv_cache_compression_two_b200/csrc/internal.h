@@ -47,9 +47,11 @@ ispa_status launch_absorb_weight(int D, int Dout, const void *W, ispa_dtype wdt,
 ispa_status launch_attn_simt(const ispa_attn_desc &d, const GroupRanges &g, float scale, const float *q,
                              const float *k, const float *v, void *o_loc, float *l_loc, void *o_hist,
                              float *l_hist, void *o_full, float *l_full, cudaStream_t s);
+// workspace: an fp16 copy of V (see attn_tc.cu) plus per-head scales
+size_t attn_tc_workspace_bytes(int B, int H, int Lkv);
 ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float scale, const void *q,
                            const void *k, const void *v, void *o_loc, float *l_loc, void *o_hist,
-                           float *l_hist, void *o_full, float *l_full, cudaStream_t s);
+                           float *l_hist, void *o_full, float *l_full, void *workspace, cudaStream_t s);
 
 // stats
 size_t stats_workspace_bytes(int T, int D, int Dout, ispa_precision prec);

@@ -43,7 +43,7 @@ FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
 
 def _split(desc, ptrs=None):
     p = ptrs or [FAKE] * 9
-    return ispa.lib().ispa_attn_split(ctypes.byref(desc), *p, None)
+    return ispa.lib().ispa_attn_split(ctypes.byref(desc), *p, FAKE, 1 << 40, None)
 
 
 @pytest.mark.parametrize("kw,frag", [
@@ -64,7 +64,10 @@ def test_attn_split_rejects_bad_layouts(kw, frag):
 
 
 def test_attn_split_rejects_null_and_misaligned():
-    assert ispa.lib().ispa_attn_split(None, *([FAKE] * 9), None) == ispa.ISPA_ERR_INVALID_ARG
+    assert ispa.lib().ispa_attn_split(None, *([FAKE] * 9), FAKE, 1 << 40, None) == ispa.ISPA_ERR_INVALID_ARG
+    # workspace too small for the bf16 path
+    assert ispa.lib().ispa_attn_split(ctypes.byref(_desc()), *([FAKE] * 9), FAKE, 16, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert "workspace" in ispa.lib().ispa_last_error().decode()
     p = [FAKE] * 9
     p[0] = FAKE + 4
     assert _split(_desc(), p) == ispa.ISPA_ERR_INVALID_ARG
@@ -110,7 +113,10 @@ def test_workspace_queries():
     assert L.ispa_accum_stats_workspace_bytes(T, D, Dout, ispa.ISPA_PREC_F32) >= T * Dout * 4
     d = _desc(H=12, tokens_per_frame=1560, sink_frames=3, hist_begin=3, hist_end=18, cur_begin=18, cur_end=21,
               kv_frames=21)
-    assert L.ispa_attn_local_proj_workspace_bytes(ctypes.byref(d)) >= 4680 * 1536 * 2
+    assert L.ispa_attn_local_proj_workspace_bytes(ctypes.byref(d)) >= 4680 * 1536 * 2 + 32760 * 1536 * 2
+    assert L.ispa_attn_split_workspace_bytes(ctypes.byref(d)) >= 32760 * 1536 * 2
+    d.in_dtype = ispa.ISPA_F32
+    assert L.ispa_attn_split_workspace_bytes(ctypes.byref(d)) == 0
     assert L.ispa_ridge_workspace_bytes(0, 5) == 0
 
 

@@ -22,8 +22,10 @@ def run_split(shape, in_dt, out_dt, key, fused=True, want_hist=True):
     o = {n: nan_like((B, Lq, H, d), tout) for n in ("loc", "hist", "full")}
     l = {n: nan_like((B, Lq, H), torch.float32) for n in ("loc", "hist", "full")}
     desc = ispa.attn_desc(shape, in_dt, out_dt)
+    ws = torch.empty(max(1, ispa.ispa_attn_split_workspace_bytes(desc)), dtype=torch.uint8, device="cuda")
     ispa.ispa_attn_split(desc, q, k, v, o["loc"], l["loc"], o["hist"] if want_hist else None,
-                         l["hist"] if want_hist else None, o["full"] if fused else None, l["full"] if fused else None)
+                         l["hist"] if want_hist else None, o["full"] if fused else None, l["full"] if fused else None,
+                         workspace=ws)
     ispa.ispa_check_device_error()
     torch.cuda.synchronize()
     return data, {n: host(t) for n, t in o.items()}, {n: host(t) for n, t in l.items()}
@@ -123,8 +125,9 @@ def test_bf16_large_scores_and_rescaling():
     q, k, v = dev(data["q"], torch.bfloat16), dev(data["k"], torch.bfloat16), dev(data["v"], torch.bfloat16)
     o = {n: nan_like((1, sh.Lq, 1, 128), torch.float32) for n in ("loc", "hist", "full")}
     l = {n: nan_like((1, sh.Lq, 1), torch.float32) for n in ("loc", "hist", "full")}
-    ispa.ispa_attn_split(ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_F32), q, k, v, o["loc"], l["loc"], o["hist"],
-                         l["hist"], o["full"], l["full"])
+    desc = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_F32)
+    ws = torch.empty(ispa.ispa_attn_split_workspace_bytes(desc), dtype=torch.uint8, device="cuda")
+    ispa.ispa_attn_split(desc, q, k, v, o["loc"], l["loc"], o["hist"], l["hist"], o["full"], l["full"], workspace=ws)
     torch.cuda.synchronize()
     check(sh, data, {n: host(t) for n, t in o.items()}, {n: host(t) for n, t in l.items()}, ispa.ISPA_BF16,
           ispa.ISPA_F32)

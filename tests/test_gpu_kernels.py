@@ -232,7 +232,10 @@ def test_attn_local_proj(y_dt):
     torch.cuda.synchronize()
     ref = orc.local_projection(sh, data["q"], data["k"], data["v"], W, dW)
     got = host(y)
+    # y = A_loc W_new with both operands in bf16 (the post-switch layer computes in bf16): every
+    # product carries two bf16 roundings (relative RMS 2 * 2^-9 / sqrt(3) combined ~1.6e-3), so the
+    # largest of ~5e4 outputs sits near 5 sigma ~ 8e-3 of RMS; the bound is 2e-2 of RMS.
     if y_dt == ispa.ISPA_BF16:
-        assert_bf16_out(got, ref)
+        assert_bf16_out(got, ref, tol=2e-2)
     else:
-        assert max_over_rms(got, ref) <= 1e-2, max_over_rms(got, ref)
+        assert max_over_rms(got, ref) <= 2e-2, max_over_rms(got, ref)

@@ -1,0 +1,136 @@
+"""End-to-end GPU parity: warmup -> statistics -> ridge solve -> selection, against the oracle.
+
+Stage-wise comparison: every stage is checked against the oracle applied to
+the GPU's own inputs of that stage (so that the conditioning of G + lambda I
+does not amplify the rounding of an earlier stage into a later one), and the
+end-to-end deviation is reported alongside."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import kv_cache_compression_two_b200 as ispa
+import synth_inputs as si
+from oracle import ispa_oracle as orc
+from gpu_helpers import dev, host, normwise, rel_fro
+
+pytestmark = pytest.mark.gpu
+
+
+def _attn(sh, data, in_dt, tin):
+    B, Lq, H, d = sh.B, sh.Lq, sh.H, sh.d
+    o = {n: torch.empty((B, Lq, H, d), device="cuda") for n in ("loc", "full")}
+    l = {n: torch.empty((B, Lq, H), device="cuda") for n in ("loc", "full")}
+    desc = ispa.attn_desc(sh, in_dt, ispa.ISPA_F32)
+    ws = torch.empty(max(1, ispa.ispa_attn_split_workspace_bytes(desc)), dtype=torch.uint8, device="cuda")
+    ispa.ispa_attn_split(desc, dev(data["q"], tin), dev(data["k"], tin), dev(data["v"], tin), o["loc"], l["loc"],
+                         None, None, o["full"], l["full"], workspace=ws)
+    return o
+
+
+def _absorb_gpu(rows_loc, rows_full, W, prec, lam_rel, refine):
+    """Accumulates the statistics over chunks of rows and solves; returns host arrays."""
+    D, Dout = W.shape
+    G = torch.zeros((D, D), device="cuda")
+    C = torch.zeros((D, Dout), device="cuda")
+    r2 = torch.zeros(1, dtype=torch.float64, device="cuda")
+    Wd = dev(W)
+    for a_loc, a_full in zip(rows_loc, rows_full):
+        T = a_loc.shape[0]
+        ws = torch.empty(ispa.ispa_accum_stats_workspace_bytes(T, D, Dout, prec), dtype=torch.uint8, device="cuda")
+        ispa.ispa_accum_stats(T, D, Dout, a_loc, a_full, Wd, G, C, r2, prec, ws)
+    dW = torch.empty((D, Dout), device="cuda")
+    eps = torch.zeros(1, dtype=torch.float64, device="cuda")
+    rws = torch.empty(ispa.ispa_ridge_workspace_bytes(D, Dout), dtype=torch.uint8, device="cuda")
+    ispa.ispa_ridge_solve(D, Dout, G, C, r2, lam_rel, True, refine, dW, eps, rws)
+    ispa.ispa_check_device_error()
+    return host(G), host(C), float(r2.item()), host(dW), float(eps.item())
+
+
+def _sym(G_upper):
+    U = np.triu(G_upper)
+    return U + np.triu(U, 1).T
+
+
+def test_tiny_fp32_warmup_to_absorption():
+    """Tiny fp32 case: 2 heads x 32, 16 tokens/frame, sink 1 + history 6 + current 1, 4 warmup chunks."""
+    sh = si.TINY
+    W = si.projection_weight(sh.D, sh.D, ("pipe", "tiny"))
+    loc_d, full_d, chunks = [], [], []
+    for c in range(4):
+        data = si.iid_qkv(sh, "f32", ("pipe", "tiny", c))
+        o = _attn(sh, data, ispa.ISPA_F32, torch.float32)
+        ref = orc.split_attention(sh, data["q"], data["k"], data["v"])
+        assert normwise(host(o["loc"]), ref["O_loc"]) <= 1e-5
+        assert normwise(host(o["full"]), ref["O_full"]) <= 1e-5
+        chunks.append(ref)
+        loc_d.append(o["loc"].reshape(sh.Lq, sh.D))
+        full_d.append(o["full"].reshape(sh.Lq, sh.D))
+    G, C, r2, dW, eps = _absorb_gpu(loc_d, full_d, W, ispa.ISPA_PREC_F32, 1e-4, 3)
+    # statistics from the GPU's attention rows (stage-wise) and from the oracle's (end to end)
+    A_loc = np.concatenate([host(t) for t in loc_d])
+    A_full = np.concatenate([host(t) for t in full_d])
+    Gs, Cs, r2s = orc.absorption_stats(A_loc, A_full, W)
+    iu = np.triu_indices(sh.D)
+    assert normwise(G[iu], Gs[iu]) <= 1e-5 and normwise(C, Cs) <= 1e-5 and abs(r2 - r2s) <= 1e-5 * r2s
+    # solve from the GPU's statistics, with the same lambda rule
+    Gg = _sym(G)
+    lam = float(np.float32(orc.ridge_lambda(Gg, 1e-4, True)))
+    dW_ref = orc.ridge_solve(Gg, C.astype(np.float64), lam)
+    assert rel_fro(dW, dW_ref) <= 1e-5, rel_fro(dW, dW_ref)
+    eps_ref = orc.eps_direct(A_loc, A_full, W, dW)
+    assert abs(eps - eps_ref) <= 1e-5 * r2
+    # end to end against the oracle's own warmup (reported; amplified by cond(G + lambda I))
+    full = orc.absorb_layer(chunks, W, 1e-4, True)
+    print(f"tiny end-to-end: dW rel {rel_fro(dW, full['dW']):.2e}, eps {eps:.6e} vs {full['eps']:.6e}, "
+          f"r2 {full['r2']:.6e}")
+
+
+def _drift_chunk(sh, layer, chunk, prefix):
+    cq = si.chunk_qkv(sh, "bf16", layer, chunk, ("pipe", "model"))
+    return {"q": cq["q"], "k": si.assemble_kv(prefix["k"], cq["k"], sh),
+            "v": si.assemble_kv(prefix["v"], cq["v"], sh)}
+
+
+def test_reduced_model_selection_matches_oracle():
+    """Drift-history model (6 layers, 2 heads x 128, 64 tokens/frame, sink 3 + history 15 + chunk 3),
+    4 warmup chunks per layer, ISPA-0.5: the selected set equals the oracle's."""
+    sh = si.video_shape(2, 15, tpf=64)
+    N, chunks, x = 6, 4, 0.5
+    K = orc.num_selected(x, N)
+    eps_gpu, eps_ref, dW_err = [], [], []
+    for layer in range(N):
+        prefix = si.drift_layer_kv(sh, "bf16", layer, ("pipe", "model"))
+        W = si.projection_weight(sh.D, sh.D, ("pipe", "model", layer), "bf16")
+        loc_d, full_d, ref_chunks = [], [], []
+        for c in range(chunks):
+            data = _drift_chunk(sh, layer, c, prefix)
+            o = _attn(sh, data, ispa.ISPA_BF16, torch.bfloat16)
+            loc_d.append(o["loc"].reshape(sh.Lq, sh.D))
+            full_d.append(o["full"].reshape(sh.Lq, sh.D))
+            ref_chunks.append(orc.split_attention(sh, data["q"], data["k"], data["v"]))
+        G, C, r2, dW, eps = _absorb_gpu(loc_d, full_d, W, ispa.ISPA_PREC_TF32, 1e-4, 0)
+        # stage-wise solve check
+        Gg = _sym(G)
+        dW_stage = orc.ridge_solve(Gg, C.astype(np.float64), float(np.float32(orc.ridge_lambda(Gg, 1e-4, True))))
+        dW_err.append(rel_fro(dW, dW_stage))
+        full = orc.absorb_layer(ref_chunks, W, 1e-4, True)
+        eps_gpu.append(eps)
+        eps_ref.append(full["eps"])
+        assert rel_fro(G[np.triu_indices(sh.D)], full["G"][np.triu_indices(sh.D)]) <= 1e-3
+        assert rel_fro(C, full["C"]) <= 1e-3
+    assert max(dW_err) <= 1e-2, dW_err
+    e = torch.tensor(eps_gpu, dtype=torch.float64, device="cuda")
+    mask = torch.zeros(N, dtype=torch.uint8, device="cuda")
+    idx = torch.zeros(K, dtype=torch.int32, device="cuda")
+    ispa.ispa_select_layers(N, e, K, mask, idx)
+    torch.cuda.synchronize()
+    _, ref_idx = orc.select_layers(eps_ref, K)
+    srt = np.sort(eps_ref)
+    gap = (srt[K] - srt[K - 1]) / srt[K]
+    rel = [abs(a - b) / b for a, b in zip(eps_gpu, eps_ref)]
+    print(f"eps gpu {np.round(eps_gpu, 6)} ref {np.round(eps_ref, 6)}; boundary gap {gap:.3e}; "
+          f"max rel eps dev {max(rel):.3e}")
+    assert gap > 2 * max(rel), "selection boundary is a tie within the propagated error"
+    assert idx.cpu().numpy().tolist() == ref_idx.tolist()
