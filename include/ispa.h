@@ -203,6 +203,32 @@ ispa_status ispa_ridge_solve(int D, int Dout, const float *G, const float *C, co
                              ispa_stream_t stream);
 
 /*
+ * Allocation-free form of ispa_ridge_solve.  The paper has no counterpart:
+ * this entry point exists for callers that cannot allocate device memory for
+ * the solver's workspace -- for example a video generator's per-chunk loop
+ * that must never call cudaMalloc or cudaFree (both can synchronise the whole
+ * device and stall the streams that are still generating frames), or a host
+ * application whose device memory is wholly owned by another allocator.
+ *
+ * Same arguments and results as ispa_ridge_solve, without the workspace.  Its
+ * scratch is a static array inside the library of ISPA_RIDGE_NOALLOC_MAX_D^2 +
+ * ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_DOUT floats (8 MiB), which
+ * every GPU that loads the library holds until the process exits; the call
+ * itself allocates nothing.  D > ISPA_RIDGE_NOALLOC_MAX_D or Dout >
+ * ISPA_RIDGE_NOALLOC_MAX_DOUT returns ISPA_ERR_INVALID_ARG.  The first call on
+ * a device looks up the array's device address (cudaGetSymbolAddress); make
+ * that first call before any stream capture.  All calls share the one array
+ * and every call rewrites the parts it reads before reading them, so calls
+ * that overlap on the GPU (other streams, other host threads) race: serialise
+ * them.
+ */
+#define ISPA_RIDGE_NOALLOC_MAX_D 1024
+#define ISPA_RIDGE_NOALLOC_MAX_DOUT 1024
+ispa_status ispa_ridge_solve_noalloc(int D, int Dout, const float *G, const float *C, const double *r2,
+                                     float lambda, int lambda_relative, int refine_steps, float *dW,
+                                     double *eps, ispa_stream_t stream);
+
+/*
  * Instance-specific layer selection [EN-notes, Key Designs 3; DE-summary 2,
  * "Dynamische Layerauswahl"]: sort the N layers by increasing eps and take
  * the K lowest as L-layers; equal eps goes to the lower layer index.

@@ -31,7 +31,8 @@ STATUS_NAMES = {0: "ISPA_OK", 1: "ISPA_ERR_INVALID_ARG", 2: "ISPA_ERR_UNSUPPORTE
 EXPORTED = ("ispa_version", "ispa_last_error", "ispa_launch_count", "ispa_check_device_error", "ispa_attn_split_workspace_bytes", "ispa_attn_split", "ispa_lse_merge",
             "ispa_accum_stats_workspace_bytes", "ispa_accum_stats", "ispa_ridge_workspace_bytes", "ispa_ridge_solve",
             "ispa_select_layers", "ispa_absorb_weight", "ispa_attn_local_proj_workspace_bytes",
-            "ispa_attn_local_proj")
+            "ispa_attn_local_proj", "ispa_ridge_solve_noalloc")
+RIDGE_NOALLOC_MAX_D = RIDGE_NOALLOC_MAX_DOUT = 1024
 
 
 class IspaError(RuntimeError):
@@ -79,6 +80,7 @@ def lib() -> ctypes.CDLL:
         "ispa_accum_stats": (_ci, [_ci, _ci, _ci, _vp, _vp, _vp, _vp, _vp, _vp, _ci, _vp, _sz, _vp]),
         "ispa_ridge_workspace_bytes": (_sz, [_ci, _ci]),
         "ispa_ridge_solve": (_ci, [_ci, _ci, _vp, _vp, _vp, _cf, _ci, _ci, _vp, _vp, _vp, _sz, _vp]),
+        "ispa_ridge_solve_noalloc": (_ci, [_ci, _ci, _vp, _vp, _vp, _cf, _ci, _ci, _vp, _vp, _vp]),
         "ispa_select_layers": (_ci, [_ci, _vp, _ci, _vp, _vp, _vp]),
         "ispa_absorb_weight": (_ci, [_ci, _ci, _vp, _ci, _vp, _vp, _ci, _vp]),
         "ispa_attn_local_proj_workspace_bytes": (_sz, [ctypes.POINTER(AttnDesc)]),
@@ -196,6 +198,14 @@ def ispa_ridge_solve(D: int, Dout: int, G, C, r2, lam: float, lambda_relative: b
     _check(lib().ispa_ridge_solve(D, Dout, _ptr(G), _ptr(C), _ptr(r2), float(lam), int(bool(lambda_relative)),
                                   int(refine_steps), _ptr(dW), _ptr(eps), _ptr(workspace), workspace_bytes,
                                   _stream(stream)))
+
+
+def ispa_ridge_solve_noalloc(D: int, Dout: int, G, C, r2, lam: float, lambda_relative: bool, refine_steps: int, dW,
+                             eps, stream=None) -> None:
+    """ispa_ridge_solve without a workspace, for callers that cannot allocate device memory
+    (D, Dout <= 1024; the scratch is a static array inside the library, shared by all calls)."""
+    _check(lib().ispa_ridge_solve_noalloc(D, Dout, _ptr(G), _ptr(C), _ptr(r2), float(lam), int(bool(lambda_relative)),
+                                          int(refine_steps), _ptr(dW), _ptr(eps), _stream(stream)))
 
 
 def ispa_select_layers(N: int, eps, K: int, is_local, idx, stream=None) -> None:

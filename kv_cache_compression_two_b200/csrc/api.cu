@@ -294,6 +294,25 @@ ispa_status ispa_ridge_solve(int D, int Dout, const float *G, const float *C, co
                       (cudaStream_t)stream);
 }
 
+ispa_status ispa_ridge_solve_noalloc(int D, int Dout, const float *G, const float *C, const double *r2, float lambda,
+                                     int lambda_relative, int refine_steps, float *dW, double *eps,
+                                     ispa_stream_t stream) {
+  if (D < 1 || Dout < 1 || D > ISPA_RIDGE_NOALLOC_MAX_D || Dout > ISPA_RIDGE_NOALLOC_MAX_DOUT)
+    return fail(ISPA_ERR_INVALID_ARG,
+                "ispa_ridge_solve_noalloc: need 1 <= D <= %d and 1 <= Dout <= %d (got D=%d, Dout=%d); use "
+                "ispa_ridge_solve with a workspace for larger sizes",
+                ISPA_RIDGE_NOALLOC_MAX_D, ISPA_RIDGE_NOALLOC_MAX_DOUT, D, Dout);
+  if (!(lambda >= 0.f) || !isfinite(lambda)) return fail(ISPA_ERR_INVALID_ARG, "lambda must be finite and >= 0");
+  if (refine_steps < 0 || refine_steps > 16) return fail(ISPA_ERR_INVALID_ARG, "refine_steps in [0, 16]");
+  if (!ptr_ok(G) || !ptr_ok(C) || !r2 || !ptr_ok(dW) || !eps)
+    return fail(ISPA_ERR_INVALID_ARG, "pointers must be non-NULL, matrices 16-byte aligned");
+  void *scratch = nullptr;
+  ispa_status st = ridge_noalloc_scratch(&scratch);
+  if (st != ISPA_OK) return st;
+  return launch_ridge(D, Dout, G, C, r2, lambda, lambda_relative, refine_steps, dW, eps, scratch,
+                      (cudaStream_t)stream);
+}
+
 ispa_status ispa_select_layers(int N, const double *eps, int K, unsigned char *is_local, int *idx,
                                ispa_stream_t stream) {
   if (N < 0 || N > 4096 || K < 0 || K > N) return fail(ISPA_ERR_INVALID_ARG, "need 0 <= K <= N <= 4096");

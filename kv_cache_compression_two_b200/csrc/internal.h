@@ -63,6 +63,8 @@ size_t ridge_workspace_bytes(int D, int Dout);
 ispa_status launch_ridge(int D, int Dout, const float *G, const float *C, const double *r2, float lambda,
                          int lambda_relative, int refine_steps, float *dW, double *eps, void *ws,
                          cudaStream_t s);
+// Device address of the static scratch array of ispa_ridge_solve_noalloc on the current device.
+ispa_status ridge_noalloc_scratch(void **out);
 
 // bf16 projection GEMM y[M, N] = A[M, K] * B[K, N] (A, B bf16 row-major) on tcgen05
 ispa_status launch_gemm_bf16(int M, int N, int K, const void *A, const void *B, void *Y, ispa_dtype ydt,

@@ -7,6 +7,8 @@
 // then the blocked forward and backward substitutions on the Dout right-hand
 // sides, optional iterative refinement with residuals accumulated in fp64,
 // and epsilon = r2 - 2<dW, C> + <dW, G dW> with fp64 reductions.
+#include <mutex>
+
 #include "internal.h"
 #include "simt_gemm.cuh"
 
@@ -271,6 +273,39 @@ cudaError_t cholesky_solve(int D, int Dout, const float *L, float *Y, cudaStream
 
 size_t ridge_workspace_bytes(int D, int Dout) {
   return align256((size_t)D * D * sizeof(float)) + align256((size_t)D * Dout * sizeof(float)) + 256;
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant (ispa_ridge_solve_noalloc).  Its scratch -- the
+// working copy of the Cholesky factor, the refinement residual and a few
+// accumulators -- lives in this file-scope device array instead of a
+// caller-supplied workspace.  Every device that loads the library holds the
+// array until the process exits.  Host code must not pass the symbol itself to
+// a kernel (on the host it only names a host-side shadow); the device address
+// is looked up once per device with cudaGetSymbolAddress.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = (size_t)ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_D * 4 +
+                                        (size_t)ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_DOUT * 4 + 256;
+static __device__ __align__(256) unsigned char g_ridge_scratch[kNoAllocScratchBytes];
+
+ispa_status ridge_noalloc_scratch(void **out) {
+  static std::mutex mu;
+  static void *addr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(ISPA_ERR_CUDA, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_ridge_scratch);
+    if (e != cudaSuccess) return cuda_status(e, "cudaGetSymbolAddress(ridge scratch)");
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  static_assert(kNoAllocScratchBytes >= (size_t)ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_D * 4 + 256,
+                "scratch smaller than the largest workspace it must hold");
+  return ISPA_OK;
 }
 
 ispa_status launch_ridge(int D, int Dout, const float *G, const float *C, const double *r2, float lambda,
