@@ -1,49 +1,53 @@
 // attn_tc.cu -- two-group attention on tcgen05 tensor cores (bf16 in, fp32 accumulate, d = 128).
 //
-// One CTA computes one 128-query tile of one head of one instance and walks the
-// KV tiles of the local group (sink range, then current range) followed by the
-// history group.  Each group keeps its own online-softmax state; at the end of
-// a group the normalised output and its log-sum-exp are written, and after the
-// history group the optional fused merge combines both groups by their LSE.
+// One CTA computes two 128-query tiles (A and B, 256 queries) of one head of
+// one instance and walks the KV tiles of the local group (sink range, then
+// current range) followed by the history group.  Both query tiles share every
+// K/V tile, which halves the operand traffic from L2 per FLOP -- the limit of a
+// single-tile design on this part.  Each group keeps its own online-softmax
+// state; at the end of a group the normalised output and its log-sum-exp are
+// written, and after the history group the optional fused merge combines both
+// groups by their LSE.
 //
-// Warp roles (192 threads, one CTA per SM):
-//   warp 0      TMA producer: Q once, then K and V tiles (128 keys x 128 dims)
-//               through two-stage rings with separate K and V barriers.
-//   warp 1      TMEM allocator and MMA issuer:
-//                 S_j = Q K_j^T       -> TMEM S[j % 2]   (A, B from shared memory)
-//                 O  += P_j V_j       -> TMEM O          (A = P from TMEM, B = V)
-//               issue order S_0, S_1, PV_0, S_2, PV_1, ... so that the
-//               softmax of tile j overlaps the MMAs of tiles j+1 and j-1.
-//   warps 2..5  softmax / correction / epilogue, one query row per thread
-//               (TMEM lane = row).  P_j is written as packed bf16 to TMEM
-//               P[j % 2] (K/2 32-bit columns per row).  The running maximum is
-//               only moved (and O rescaled) when a row's tile maximum exceeds
-//               it by more than 2^8, so O is rarely touched off the MMA path.
+// Warp roles (320 threads, one CTA per SM):
+//   warp 0      TMA producer: Q_A and Q_B once, then K and V tiles (128 keys x
+//               128 dims) through two-stage rings with separate K and V barriers.
+//   warp 1      TMEM allocator and MMA issuer, per KV tile j:
+//                 PV_{j-1}(A), S_j(A), PV_{j-1}(B), S_j(B)
+//               with S_j(X) = Q_X K_j^T (bf16, operands in shared memory) and
+//               PV_j(X): O_X += P_j(X) V_j (fp16 P read from TMEM as operand A,
+//               fp16 V from shared memory), so the softmax of one query tile
+//               overlaps the MMAs of the other.
+//   warps 2-5   softmax / correction / epilogue of query tile A, one row per
+//   warps 6-9   thread (TMEM lane = row); the same for query tile B.
 //
-// TMEM columns: S0 [0,128) S1 [128,256) O [256,384) P0 [384,448) P1 [448,512).
+// TMEM columns: S_A [0,128) S_B [128,256) O_A [256,384) O_B [384,512).  P_j(X)
+// is written as packed fp16 into columns [0,64) of S_X after the softmax has
+// read S_j(X); tcgen05.mma operations issued by one thread execute in order,
+// so PV_j(X) has read P before S_{j+1}(X) overwrites the columns.
 //
-// Ordering argument (every TMEM buffer has one writer at a time):
-//   * S_j overwrites S[j%2] only after P_{j-2} was published, i.e. after the
-//     softmax of tile j-2 finished its tcgen05.ld of that buffer.
-//   * The softmax of tile j writes P[j%2] after S_j completed; S_j's commit
-//     covers every earlier MMA, including PV_{j-2} which read P[j%2].
-//   * O is rescaled by the softmax of tile j only after PV_{j-1} completed
-//     (o_done) and before PV_j is issued (PV_j waits for P_j).
-//   * At the end of the local group the epilogue reads O after PV of that tile
-//     and releases it (o_free) before the first history PV overwrites it.
+// Ordering argument:
+//   * S_{j+1}(X) is issued after the softmax published P_j(X), i.e. after it
+//     finished its tcgen05.ld of S_j(X).
+//   * S_j(X) is issued after PV_{j-1}(X); its commit (s_full) therefore also
+//     covers PV_{j-1}(X), so while the softmax of tile j runs no MMA touches
+//     O_X and it may rescale O_X directly; PV_j(X) waits for P_j(X).
+//   * At the end of the local group the epilogue reads O_X after PV of that
+//     tile (o_done) and releases it (o_free) before the first history PV
+//     overwrites it.
 #include "internal.h"
 
 namespace ispa {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // producer, MMA, one softmax warpgroup per query tile
 constexpr int kTileQ = 128, kTileK = 128, kD = 128;
 constexpr int kBoxBytes = 128 * 128;          // 128 rows x 64 bf16
 constexpr int kTileBytes = 2 * kBoxBytes;     // 128 rows x 128 bf16
-constexpr int kStages = 2;
+constexpr int kStagesK = 3, kStagesV = 2;  // K is needed one MMA step earlier than V
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColO = 256, kColP0 = 384;
+constexpr uint32_t kColS = 0, kColO = 256;  // + 128 * query tile
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 
 struct AttnParams {
@@ -154,14 +158,14 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 }
 
 struct SmemLayout {
-  uint8_t q[kTileBytes];
-  uint8_t k[kStages][kTileBytes];
-  uint8_t v[kStages][kTileBytes];
+  uint8_t q[2][kTileBytes];
+  uint8_t k[kStagesK][kTileBytes];
+  uint8_t v[kStagesV][kTileBytes];
   uint64_t q_full;
-  uint64_t k_full[kStages], k_empty[kStages];
-  uint64_t v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_full[2];
-  uint64_t o_done, o_free, drain;
+  uint64_t k_full[kStagesK], k_empty[kStagesK];
+  uint64_t v_full[kStagesV], v_empty[kStagesV];
+  uint64_t s_full[2], p_full[2], o_done[2], o_free[2];  // per query tile
+  uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -189,6 +193,27 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Packed fp32 pair arithmetic (sm_100): one instruction for two lanes of work.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
 }
 
 template <typename TO>
@@ -247,26 +272,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       *reinterpret_cast<SmemLayout *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   volatile int *abort = &sm.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x % P.q_tiles;
+  const int qt = blockIdx.x % P.q_tiles;  // pair of 128-query tiles
   const int h = blockIdx.x / P.q_tiles;
   const int b = blockIdx.y;
-  const int q0 = qt * kTileQ;
+  const int q0 = qt * 2 * kTileQ;
   const bool has_hist = P.n_tiles > P.n_loc_tiles;
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kStagesK; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
+    }
+    for (int s = 0; s < kStagesV; ++s) {
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.p_full[s], 128);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&sm.s_full[x], 1);
+      mbar_init(&sm.p_full[x], 128);
+      mbar_init(&sm.o_done[x], 1);
+      mbar_init(&sm.o_free[x], 128);
     }
-    mbar_init(&sm.o_done, 1);
-    mbar_init(&sm.o_free, 128);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
     fence_mbar_init();
@@ -286,88 +313,93 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const int x0 = h * kD;
-      mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
-      tma_load_3d(sm.q, &tq, &sm.q_full, x0, q0, b);
-      tma_load_3d(sm.q + kBoxBytes, &tq, &sm.q_full, x0 + 64, q0, b);
+      mbar_arrive_expect_tx(&sm.q_full, 2 * kTileBytes);
+      for (int x = 0; x < 2; ++x) {
+        tma_load_3d(sm.q[x], &tq, &sm.q_full, x0, q0 + x * kTileQ, b);
+        tma_load_3d(sm.q[x] + kBoxBytes, &tq, &sm.q_full, x0 + 64, q0 + x * kTileQ, b);
+      }
       uint32_t k_pend = 0, v_pend = 0, k_ph = 0, v_ph = 0;
       TileIter it;
       it.start(P);
       for (int j = 0; j < P.n_tiles; ++j, it.next(P)) {
-        const int s = j % kStages;
-        const uint32_t ph = (j / kStages) & 1;
-        if (!wait_parity(&sm.k_empty[s], ph ^ 1, P.err, abort, 11)) break;
-        mbar_arrive_expect_tx(&sm.k_full[s], kTileBytes);
-        tma_load_3d(sm.k[s], &tk, &sm.k_full[s], x0, it.t0, b);
-        tma_load_3d(sm.k[s] + kBoxBytes, &tk, &sm.k_full[s], x0 + 64, it.t0, b);
-        k_pend |= 1u << s;
-        k_ph = (k_ph & ~(1u << s)) | (ph << s);
-        if (!wait_parity(&sm.v_empty[s], ph ^ 1, P.err, abort, 12)) break;
-        mbar_arrive_expect_tx(&sm.v_full[s], kTileBytes);
-        tma_load_3d(sm.v[s], &tv, &sm.v_full[s], x0, it.t0, b);
-        tma_load_3d(sm.v[s] + kBoxBytes, &tv, &sm.v_full[s], x0 + 64, it.t0, b);
-        v_pend |= 1u << s;
-        v_ph = (v_ph & ~(1u << s)) | (ph << s);
+        const int sk = j % kStagesK, sv = j % kStagesV;
+        const uint32_t phk = (j / kStagesK) & 1, phv = (j / kStagesV) & 1;
+        if (!wait_parity(&sm.k_empty[sk], phk ^ 1, P.err, abort, 11)) break;
+        mbar_arrive_expect_tx(&sm.k_full[sk], kTileBytes);
+        tma_load_3d(sm.k[sk], &tk, &sm.k_full[sk], x0, it.t0, b);
+        tma_load_3d(sm.k[sk] + kBoxBytes, &tk, &sm.k_full[sk], x0 + 64, it.t0, b);
+        k_pend |= 1u << sk;
+        k_ph = (k_ph & ~(1u << sk)) | (phk << sk);
+        if (!wait_parity(&sm.v_empty[sv], phv ^ 1, P.err, abort, 12)) break;
+        mbar_arrive_expect_tx(&sm.v_full[sv], kTileBytes);
+        tma_load_3d(sm.v[sv], &tv, &sm.v_full[sv], x0, it.t0, b);
+        tma_load_3d(sm.v[sv] + kBoxBytes, &tv, &sm.v_full[sv], x0 + 64, it.t0, b);
+        v_pend |= 1u << sv;
+        v_ph = (v_ph & ~(1u << sv)) | (phv << sv);
       }
       if (*abort) {  // let copies in flight land before the CTA exits
         wait_parity_drain(&sm.q_full, 0, P.err);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < kStagesK; ++s)
           if (k_pend & (1u << s)) wait_parity_drain(&sm.k_full[s], (k_ph >> s) & 1, P.err);
+        for (int s = 0; s < kStagesV; ++s)
           if (v_pend & (1u << s)) wait_parity_drain(&sm.v_full[s], (v_ph >> s) & 1, P.err);
-        }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc_qk = make_idesc(128, 128, 1, 0, 0);
-      const uint32_t idesc_pv = make_idesc(128, 128, 0, 0, 1);  // fp16 P (TMEM) x fp16 V (smem)
-      const uint32_t q_addr = smem_u32(sm.q);
-      bool ok = wait_parity(&sm.q_full, 0, P.err, abort, 21);
-      for (int j = 0; ok && j <= P.n_tiles; ++j) {
-        if (j < P.n_tiles) {
-          const int s = j % kStages;
-          if (!wait_parity(&sm.k_full[s], (j / kStages) & 1, P.err, abort, 22)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(sm.k[s]);
-          const uint32_t d_s = tmem + kColS0 + (uint32_t)(j & 1) * 128;
+      const uint32_t idesc_qk = make_idesc(128, 128, 1, 0, 0);  // bf16 Q x bf16 K, both K-major
+      const uint32_t idesc_pv = make_idesc(128, 128, 0, 0, 1);  // fp16 P (TMEM) x fp16 V (MN-major)
+      auto issue_s = [&](int j, int x) {  // S_j(x) = Q_x K_j^T
+        const uint32_t q_addr = smem_u32(sm.q[x]);
+        const uint32_t k_addr = smem_u32(sm.k[j % kStagesK]);
+        const uint32_t d_s = tmem + kColS + (uint32_t)x * 128;
 #pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) {
-            const uint32_t off = (uint32_t)(kk >> 2) * kBoxBytes + (uint32_t)(kk & 3) * 32;
-            mma_ss(d_s, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024), idesc_qk,
-                   kk > 0 ? 1u : 0u, 0);
-          }
-          mma_commit(&sm.k_empty[s]);
-          mma_commit(&sm.s_full[j & 1]);
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (uint32_t)(kk >> 2) * kBoxBytes + (uint32_t)(kk & 3) * 32;
+          mma_ss(d_s, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024), idesc_qk,
+                 kk > 0 ? 1u : 0u, 0);
         }
-        if (j >= 1) {
-          const int i = j - 1;
-          const int s = i % kStages;
-          if (!wait_parity(&sm.p_full[i & 1], (i >> 1) & 1, P.err, abort, 23)) {
-            ok = false;
-            break;
-          }
-          if (i == P.n_loc_tiles && !wait_parity(&sm.o_free, 0, P.err, abort, 24)) {
-            ok = false;
-            break;
-          }
-          if (!wait_parity(&sm.v_full[s], (i / kStages) & 1, P.err, abort, 25)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const bool first = (i == 0) || (i == P.n_loc_tiles);
-          const uint32_t v_addr = smem_u32(sm.v[s]);
-          const uint32_t a_p = tmem + kColP0 + (uint32_t)(i & 1) * 64;
+        mma_commit(&sm.s_full[x]);
+      };
+      auto issue_pv = [&](int j, int x) {  // O_x (+)= P_j(x) V_j, P in the first 64 columns of S_x
+        const bool first = (j == 0) || (j == P.n_loc_tiles);
+        const uint32_t v_addr = smem_u32(sm.v[j % kStagesV]);
+        const uint32_t a_p = tmem + kColS + (uint32_t)x * 128;
 #pragma unroll
-          for (int kk = 0; kk < kTileK / 16; ++kk) {
-            mma_ts(tmem + kColO, a_p + kk * 8, smem_desc_sw128(v_addr + kk * 2048, kBoxBytes, 1024), idesc_pv,
-                   (first && kk == 0) ? 0u : 1u);
+        for (int kk = 0; kk < kTileK / 16; ++kk)
+          mma_ts(tmem + kColO + (uint32_t)x * 128, a_p + kk * 8,
+                 smem_desc_sw128(v_addr + kk * 2048, kBoxBytes, 1024), idesc_pv, (first && kk == 0) ? 0u : 1u);
+        mma_commit(&sm.o_done[x]);
+      };
+      bool ok = wait_parity(&sm.q_full, 0, P.err, abort, 21) &&
+                wait_parity(&sm.k_full[0], 0, P.err, abort, 22);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(0, 1);
+        mma_commit(&sm.k_empty[0]);
+      }
+      for (int j = 0; ok && j < P.n_tiles; ++j) {
+        const int sv = j % kStagesV;
+        const bool more = j + 1 < P.n_tiles;
+        const int sk1 = (j + 1) % kStagesK;
+        for (int x = 0; x < 2 && ok; ++x) {
+          ok = wait_parity(&sm.p_full[x], (uint32_t)(j & 1), P.err, abort, 23);
+          if (ok && j == P.n_loc_tiles) ok = wait_parity(&sm.o_free[x], 0, P.err, abort, 24);
+          if (ok && x == 0) ok = wait_parity(&sm.v_full[sv], (j / kStagesV) & 1, P.err, abort, 25);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(j, x);
+          if (x == 1) mma_commit(&sm.v_empty[sv]);
+          if (more) {
+            // K_{j+1} is waited for only after PV_j(x) is queued
+            if (x == 0) ok = wait_parity(&sm.k_full[sk1], ((j + 1) / kStagesK) & 1, P.err, abort, 26);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(j + 1, x);
+            if (x == 1) mma_commit(&sm.k_empty[sk1]);
           }
-          mma_commit(&sm.v_empty[s]);
-          mma_commit(&sm.o_done);
         }
       }
       if (!ok) {
@@ -377,11 +409,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
+    const int x = (warp - 2) >> 2;  // query tile of this warpgroup
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // row inside the tile == TMEM lane
-    const int qrow = q0 + r;
+    const int qrow = q0 + x * kTileQ + r;
     const bool row_ok = qrow < P.Lq;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t col_s = kColS + (uint32_t)x * 128, col_o = kColO + (uint32_t)x * 128;
     const long long head_row = ((long long)b * P.Lq + (row_ok ? qrow : 0)) * P.H + h;
     TO *o_loc = reinterpret_cast<TO *>(P.o_loc) + head_row * kD;
     TO *o_hist = P.o_hist ? reinterpret_cast<TO *>(P.o_hist) + head_row * kD : nullptr;
@@ -393,78 +427,70 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool grp_first = (j == 0) || (j == P.n_loc_tiles);
       const bool grp_last = (j == P.n_loc_tiles - 1) || (j == P.n_tiles - 1);
       const int n_valid = it.valid(P);
-      bool ok = wait_parity(&sm.s_full[j & 1], (j >> 1) & 1, P.err, abort, 31);
+      bool ok = wait_parity(&sm.s_full[x], (uint32_t)(j & 1), P.err, abort, 31);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      float s[128];
+      uint32_t sr[4][32];  // S row of this thread (fp32 bits), straight from TMEM
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t raw[32];
-        tmem_ld32(lane_base + kColS0 + (uint32_t)(j & 1) * 128 + c * 32, raw);
-        tmem_wait_ld();
+      for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + col_s + c * 32, sr[c]);
+      tmem_wait_ld();
+      if (n_valid < kTileK) {  // ragged tile: keys past the range end get -inf
 #pragma unroll
-        for (int t = 0; t < 32; ++t) s[c * 32 + t] = __uint_as_float(raw[t]);
+        for (int c = 0; c < 128; ++c)
+          if (c >= n_valid) sr[c >> 5][c & 31] = 0xff800000u;
       }
-      // row maximum with 8 independent partial maxima (no 128-long dependency chain)
       float mx[8];
 #pragma unroll
       for (int t = 0; t < 8; ++t) mx[t] = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        if (c >= n_valid) s[c] = -INFINITY;
-        mx[c & 7] = fmaxf(mx[c & 7], s[c]);
-      }
-      float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      mt *= P.scale_log2;
+      for (int c = 0; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(sr[c >> 5][c & 31]));
+      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+                       P.scale_log2;
       if (grp_first) {
         m_ref = mt;
         l = 0.f;
       } else if (__any_sync(0xffffffffu, mt > m_ref + kRescaleThreshold)) {
-        // PV_{j-1} must have landed in O before it is rescaled; PV_j waits for P_j.
-        ok = wait_parity(&sm.o_done, (uint32_t)((j - 1) & 1), P.err, abort, 32);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        tc_fence_after();
+        // O_x is quiescent here (PV_{j-1}(x) completed before S_j(x)); PV_j(x) waits for P_j(x).
         const float m_new = fmaxf(m_ref, mt);
         const float f = ex2(m_ref - m_new);
         m_ref = m_new;
         l *= f;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t o[16];
-          tmem_ld16(lane_base + kColO + c * 16, o);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + col_o + c * 32, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int t = 0; t < 16; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * f);
-          tmem_st16(lane_base + kColO + c * 16, o);
+          for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * f);
+          tmem_st16(lane_base + col_o + c * 32, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
+          tmem_st16(lane_base + col_o + c * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
         }
       }
-      // P = exp2(s * scale * log2e - m_ref) <= 2^8, packed to fp16 pairs into TMEM P[j % 2].
-      const float neg_m = -m_ref;
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      // P = exp2(s * scale * log2e - m_ref) <= 2^8, packed to fp16 pairs into columns [0, 64) of S_x.
+      const float2 sc2 = make_float2(P.scale_log2, P.scale_log2), nm2 = make_float2(-m_ref, -m_ref);
+      float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
-          const float p0 = ex2(fmaf(s[c * 32 + 2 * t], P.scale_log2, neg_m));
-          const float p1 = ex2(fmaf(s[c * 32 + 2 * t + 1], P.scale_log2, neg_m));
-          ls[t & 3] += p0 + p1;
-          pk[t] = pack_f16x2(p0, p1);
+          const float2 x = ffma2(make_float2(__uint_as_float(sr[c][2 * t]), __uint_as_float(sr[c][2 * t + 1])), sc2, nm2);
+          const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+          ls[t & 1] = fadd2(ls[t & 1], pp);
+          pk[t] = pack_f16x2(pp.x, pp.y);
         }
-        tmem_st16(lane_base + kColP0 + (uint32_t)(j & 1) * 64 + c * 16, pk);
+        tmem_st16(lane_base + col_s + c * 16, pk);
       }
       tmem_wait_st();
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
       tc_fence_before();
-      mbar_arrive(&sm.p_full[j & 1]);
+      mbar_arrive(&sm.p_full[x]);
 
       if (!grp_last) continue;
-      // ---- end of a group: O of this group is complete once PV_j has landed.
-      // o_done counts PVs; a parity wait is only exact when the barrier is at
-      // most one phase behind, so first wait for PV_{j-1} (PV_{j-2} is covered
-      // by the commit of S_j), then for PV_j.
-      ok = j == 0 || wait_parity(&sm.o_done, (uint32_t)((j - 1) & 1), P.err, abort, 33);
-      ok = ok && wait_parity(&sm.o_done, (uint32_t)(j & 1), P.err, abort, 34);
+      // ---- end of a group: O_x is final once PV_j(x) has landed (o_done counts the
+      // PVs of this tile; PV_{j-1}(x) completed before S_j(x), so the wait is exact).
+      ok = wait_parity(&sm.o_done[x], (uint32_t)(j & 1), P.err, abort, 33);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const bool is_loc = j < P.n_loc_tiles;
@@ -476,32 +502,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (row_ok) P.l_loc[head_row] = L;
       } else {
         if (row_ok && P.l_hist) P.l_hist[head_row] = L;
-        const float mx = fmaxf(L_loc, L);
-        const float ea = expf(L_loc - mx), eb = expf(L - mx), se = ea + eb;
+        const float mxl = fmaxf(L_loc, L);
+        const float ea = expf(L_loc - mxl), eb = expf(L - mxl), se = ea + eb;
         wa = ea / se;
         wb = eb / se;
-        L_full = mx + logf(se);
+        L_full = mxl + logf(se);
       }
       TO *dst = is_loc ? o_loc : o_hist;
       const bool write_full = o_full != nullptr && (!is_loc || !has_hist);
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t raw[32];
-        tmem_ld32(lane_base + kColO + c * 32, raw);
+        tmem_ld32(lane_base + col_o + c * 32, raw);
         tmem_wait_ld();
-        float x[32];
+        float xo[32];
 #pragma unroll
-        for (int t = 0; t < 32; ++t) x[t] = __uint_as_float(raw[t]) * inv_l;
+        for (int t = 0; t < 32; ++t) xo[t] = __uint_as_float(raw[t]) * inv_l;
         if (!row_ok) continue;
-        if (dst) store_row32<TO>(dst + c * 32, x);
+        if (dst) store_row32<TO>(dst + c * 32, xo);
         if (write_full) {
           if (!is_loc) {
             float y[32];
             load_row32<TO>(o_loc + c * 32, y);
 #pragma unroll
-            for (int t = 0; t < 32; ++t) x[t] = wa * y[t] + wb * x[t];
+            for (int t = 0; t < 32; ++t) xo[t] = wa * y[t] + wb * xo[t];
           }
-          store_row32<TO>(o_full + c * 32, x);
+          store_row32<TO>(o_full + c * 32, xo);
         }
       }
       if (write_full && row_ok) P.l_full[head_row] = L_full;
@@ -515,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (is_loc && has_hist) {
         tc_fence_before();
-        mbar_arrive(&sm.o_free);
+        mbar_arrive(&sm.o_free[x]);
       }
     }
   }
@@ -603,7 +629,7 @@ ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float 
   if ((st = map3d_16(&tv, v16, D, g.Lkv, d.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16)) != ISPA_OK) return st;
   P.H = d.H;
   P.Lq = g.Lq;
-  P.q_tiles = (g.Lq + kTileQ - 1) / kTileQ;
+  P.q_tiles = (g.Lq + 2 * kTileQ - 1) / (2 * kTileQ);  // pairs of query tiles
   P.n_ranges = 0;
   P.n_loc_tiles = 0;
   for (int r = 0; r < g.n_loc; ++r) {

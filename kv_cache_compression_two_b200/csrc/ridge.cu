@@ -1,12 +1,13 @@
 // ridge.cu -- closed-form absorption: dW = (G + lambda I)^-1 C and epsilon.
 //
 // Blocked right-looking Cholesky in fp32 (block NB = 64):
-//   for each diagonal block k:  factor L_kk (one CTA, shared memory),
-//                               L_ik = A_ik L_kk^-T for the rows below (one thread per row),
+//   for each diagonal block k:  factor L_kk and invert it (one CTA, shared memory),
+//                               L_ik = A_ik Linv_kk^T for the rows below (SIMT GEMM),
 //                               A_ij -= L_ik L_jk^T on the trailing lower triangle (SIMT GEMM).
 // then the blocked forward and backward substitutions on the Dout right-hand
-// sides, optional iterative refinement with residuals accumulated in fp64,
-// and epsilon = r2 - 2<dW, C> + <dW, G dW> with fp64 reductions.
+// sides (diagonal blocks applied as GEMMs with Linv_kk), optional iterative
+// refinement with residuals accumulated in fp64, and
+// epsilon = r2 - 2<dW, C> + <dW, G dW> with fp64 reductions.
 #include <mutex>
 
 #include "internal.h"
@@ -20,6 +21,7 @@ constexpr int NB = 64;
 
 struct Ws {
   float *L;      // [D, D] lower Cholesky factor (working copy)
+  float *Linv;   // [ceil(D / 64), 64, 64] inverses of the diagonal blocks of L
   float *Rres;   // [D, Dout] refinement residual / correction
   double *acc;   // [0] <dW, C>  [1] <dW, G dW>  [2] trace(G)  [3] lambda_eff
   int *flag;     // non-zero once a pivot failed
@@ -32,6 +34,8 @@ Ws carve(void *base, int D, int Dout) {
   Ws w;
   w.L = reinterpret_cast<float *>(p);
   p += align256((size_t)D * D * sizeof(float));
+  w.Linv = reinterpret_cast<float *>(p);
+  p += align256((size_t)((D + NB - 1) / NB) * NB * NB * sizeof(float));
   w.Rres = reinterpret_cast<float *>(p);
   p += align256((size_t)D * Dout * sizeof(float));
   w.acc = reinterpret_cast<double *>(p);
@@ -76,15 +80,23 @@ __global__ void init_kernel(int D, int Dout, const float *__restrict__ G, const 
   for (long long e = t0; e < nDO; e += stride) dW[e] = C[e];
 }
 
-// Factors the nb x nb diagonal block at kb0 in place (nb <= 64), one CTA of 64 threads.
-__global__ void __launch_bounds__(64) potrf_diag_kernel(int D, int kb0, float *L, int *flag, DevErr err) {
+// Factors the nb x nb diagonal block at kb0 in place (nb <= 64) and writes the
+// inverse of its lower factor, padded to 64 x 64 with the identity, to Linv.
+// One CTA of 512 threads: per column one pivot, a scaled column and a rank-1
+// update of the trailing triangle spread over all threads; the inverse is
+// formed row by row (X = L^-1 solves L X = I), each row's entries in parallel.
+__global__ void __launch_bounds__(512) potrf_inv_kernel(int D, int kb0, float *L, float *Linv, int *flag,
+                                                        DevErr err) {
   __shared__ float A[NB][NB + 1];
+  __shared__ float X[NB][NB + 1];
   const int nb = min(NB, D - kb0);
   const int t = threadIdx.x;
-  for (int r = 0; r < nb; ++r)
-    if (t < nb) A[r][t] = L[(long long)(kb0 + r) * D + kb0 + t];
+  for (int e = t; e < NB * NB; e += blockDim.x) {
+    const int r = e / NB, c = e % NB;
+    A[r][c] = (r < nb && c < nb) ? L[(long long)(kb0 + r) * D + kb0 + c] : (r == c ? 1.f : 0.f);
+  }
   __syncthreads();
-  for (int c = 0; c < nb; ++c) {
+  for (int c = 0; c < NB; ++c) {
     if (t == 0) {
       float piv = A[c][c];
       if (!(piv > 0.f)) {
@@ -94,98 +106,40 @@ __global__ void __launch_bounds__(64) potrf_diag_kernel(int D, int kb0, float *L
       A[c][c] = sqrtf(piv);
     }
     __syncthreads();
-    if (t > c && t < nb) A[t][c] /= A[c][c];
+    const float inv_d = 1.f / A[c][c];
+    if (t > c && t < NB) A[t][c] *= inv_d;
     __syncthreads();
-    if (t > c && t < nb) {
-      const float lic = A[t][c];
-      for (int j = c + 1; j <= t; ++j) A[t][j] -= lic * A[j][c];
+    // rank-1 update of the trailing lower triangle: 8 threads per row i = t / 8,
+    // each taking the columns j = c+1+q, c+9+q, ... (q = t % 8) up to i
+    {
+      const int i = t >> 3, q = t & 7;
+      if (i > c) {
+        const float lic = A[i][c];
+        for (int j = c + 1 + q; j <= i; j += 8) A[i][j] -= lic * A[j][c];
+      }
     }
     __syncthreads();
   }
-  for (int r = 0; r < nb; ++r)
-    if (t <= r) L[(long long)(kb0 + r) * D + kb0 + t] = A[r][t];
-}
-
-// Rows i >= kb0 + 64: L[i, kb] = A[i, kb] L_kk^-T  (forward substitution per row).
-__global__ void __launch_bounds__(64) trsm_panel_kernel(int D, int kb0, float *L) {
-  __shared__ float Lk[NB][NB + 1];
-  const int t = threadIdx.x;
-  for (int r = 0; r < NB; ++r) Lk[r][t] = L[(long long)(kb0 + r) * D + kb0 + t];
-  __syncthreads();
-  const int i = kb0 + NB + blockIdx.x * NB + t;
-  if (i >= D) return;
-  float x[NB];
-  float *row = L + (long long)i * D + kb0;
-#pragma unroll
-  for (int c = 0; c < NB; ++c) x[c] = row[c];
-#pragma unroll
-  for (int c = 0; c < NB; ++c) {
-    float s = x[c];
-#pragma unroll
-    for (int p = 0; p < c; ++p) s -= Lk[c][p] * x[p];
-    x[c] = s / Lk[c][c];
+  // X = L^-1 (lower), row by row: X[r][j] = (delta_rj - sum_{j<=p<r} L[r][p] X[p][j]) / L[r][r].
+  // 8 threads share one entry j = t / 8 (partial sums over p = q, q+8, ...), combined by shuffles.
+  {
+    const int j = t >> 3, q = t & 7;
+    for (int r = 0; r < NB; ++r) {
+      float s = 0.f;
+      if (j <= r)
+        for (int p = j + q; p < r; p += 8) s += A[r][p] * X[p][j];
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      s += __shfl_xor_sync(0xffffffffu, s, 4);
+      if (q == 0) X[r][j] = (j <= r) ? (((j == r) ? 1.f : 0.f) - s) / A[r][r] : 0.f;
+      __syncthreads();
+    }
   }
-#pragma unroll
-  for (int c = 0; c < NB; ++c) row[c] = x[c];
-}
-
-// Loads the diagonal block padded to NB x NB with the identity beyond nb.
-__device__ __forceinline__ void load_diag_padded(float (*Lk)[NB + 1], const float *L, int D, int kb0, int nb) {
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
-    const int r = e / NB, c = e - r * NB;
-    float x;
-    if (r < nb && c < nb)
-      x = (c <= r) ? L[(long long)(kb0 + r) * D + kb0 + c] : 0.f;
-    else
-      x = (r == c) ? 1.f : 0.f;
-    Lk[r][c] = x;
+  for (int e = t; e < NB * NB; e += blockDim.x) {
+    const int r = e / NB, c = e % NB;
+    Linv[e] = X[r][c];
+    if (r < nb && c <= r) L[(long long)(kb0 + r) * D + kb0 + c] = A[r][c];
   }
-}
-
-// Y[kb rows, :] = L_kk^-1 Y[kb rows, :]   (one thread per right-hand-side column)
-__global__ void __launch_bounds__(128) trsv_fwd_kernel(int D, int Dout, int kb0, const float *L, float *Y) {
-  __shared__ float Lk[NB][NB + 1];
-  const int nb = min(NB, D - kb0);
-  load_diag_padded(Lk, L, D, kb0, nb);
-  __syncthreads();
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= Dout) return;
-  float y[NB];
-#pragma unroll
-  for (int p = 0; p < NB; ++p) y[p] = p < nb ? Y[(long long)(kb0 + p) * Dout + j] : 0.f;
-#pragma unroll
-  for (int r = 0; r < NB; ++r) {
-    float s = y[r];
-#pragma unroll
-    for (int p = 0; p < r; ++p) s -= Lk[r][p] * y[p];
-    y[r] = s / Lk[r][r];
-  }
-#pragma unroll
-  for (int p = 0; p < NB; ++p)
-    if (p < nb) Y[(long long)(kb0 + p) * Dout + j] = y[p];
-}
-
-// Y[kb rows, :] = L_kk^-T Y[kb rows, :]
-__global__ void __launch_bounds__(128) trsv_bwd_kernel(int D, int Dout, int kb0, const float *L, float *Y) {
-  __shared__ float Lk[NB][NB + 1];
-  const int nb = min(NB, D - kb0);
-  load_diag_padded(Lk, L, D, kb0, nb);
-  __syncthreads();
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= Dout) return;
-  float y[NB];
-#pragma unroll
-  for (int p = 0; p < NB; ++p) y[p] = p < nb ? Y[(long long)(kb0 + p) * Dout + j] : 0.f;
-#pragma unroll
-  for (int r = NB - 1; r >= 0; --r) {
-    float s = y[r];
-#pragma unroll
-    for (int c = r + 1; c < NB; ++c) s -= Lk[c][r] * y[c];
-    y[r] = s / Lk[r][r];
-  }
-#pragma unroll
-  for (int p = 0; p < NB; ++p)
-    if (p < nb) Y[(long long)(kb0 + p) * Dout + j] = y[p];
 }
 
 // Rres = C - (G + lambda I) X, accumulated in fp64.
@@ -221,6 +175,15 @@ __global__ void add_kernel(long long n, float *__restrict__ X, const float *__re
     X[e] += dX[e];
 }
 
+// out[i][j] = G[min(i,j)][max(i,j)]: the full symmetric matrix from its upper triangle.
+__global__ void symmetrize_kernel(int D, const float *__restrict__ G, float *out) {
+  const long long n = (long long)D * D;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
+    const int i = (int)(e / D), j = (int)(e - (long long)i * D);
+    out[e] = i <= j ? G[e] : G[(long long)j * D + i];
+  }
+}
+
 __global__ void dot_kernel(long long n, const float *__restrict__ a, const float *__restrict__ b, double *out) {
   double s = 0.0;
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x)
@@ -238,31 +201,38 @@ __global__ void finalize_kernel(long long n, const double *__restrict__ r2, Ws w
     dW[e] = __int_as_float(0x7fc00000);
 }
 
-// Forward then backward blocked substitution on Y [D, Dout] in place.
-cudaError_t cholesky_solve(int D, int Dout, const float *L, float *Y, cudaStream_t s) {
-  const int cgrid = (Dout + 127) / 128;
+// Forward then backward blocked substitution on Y [D, Dout] in place, using the
+// inverted diagonal blocks: Y_k <- Linv_kk Y_k (a small GEMM whose CTAs each
+// read their whole 64-row block column before writing it, so it may run in
+// place), then the update of the remaining block rows.
+cudaError_t cholesky_solve(int D, int Dout, const float *L, const float *Linv, float *Y, cudaStream_t s) {
   for (int kb0 = 0; kb0 < D; kb0 += NB) {
     const int nb = min(NB, D - kb0);
-    trsv_fwd_kernel<<<cgrid, 128, 0, s>>>(D, Dout, kb0, L, Y);
-    note_launch();
+    const float *Li = Linv + (long long)(kb0 / NB) * NB * NB;
+    cudaError_t e = simt_gemm<OP_N, OP_N, float, 0>(nb, Dout, nb, Operand{Li, nullptr, NB},
+                                                    Operand{Y + (long long)kb0 * Dout, nullptr, Dout},
+                                                    EpiAxpby{Y + (long long)kb0 * Dout, Dout, 1.f, 0.f, 0}, s);
+    if (e != cudaSuccess) return e;
     const int below = D - kb0 - nb;
     if (below > 0) {
-      cudaError_t e = simt_gemm<OP_N, OP_N, float, 0>(
-          below, Dout, nb, Operand{L + (long long)(kb0 + nb) * D + kb0, nullptr, D},
-          Operand{Y + (long long)kb0 * Dout, nullptr, Dout},
-          EpiAxpby{Y + (long long)(kb0 + nb) * Dout, Dout, -1.f, 1.f, 0}, s);
+      e = simt_gemm<OP_N, OP_N, float, 0>(below, Dout, nb, Operand{L + (long long)(kb0 + nb) * D + kb0, nullptr, D},
+                                          Operand{Y + (long long)kb0 * Dout, nullptr, Dout},
+                                          EpiAxpby{Y + (long long)(kb0 + nb) * Dout, Dout, -1.f, 1.f, 0}, s);
       if (e != cudaSuccess) return e;
     }
   }
   const int last0 = ((D - 1) / NB) * NB;
   for (int kb0 = last0; kb0 >= 0; kb0 -= NB) {
     const int nb = min(NB, D - kb0);
-    trsv_bwd_kernel<<<cgrid, 128, 0, s>>>(D, Dout, kb0, L, Y);
-    note_launch();
+    const float *Li = Linv + (long long)(kb0 / NB) * NB * NB;
+    cudaError_t e = simt_gemm<OP_T, OP_N, float, 0>(nb, Dout, nb, Operand{Li, nullptr, NB},
+                                                    Operand{Y + (long long)kb0 * Dout, nullptr, Dout},
+                                                    EpiAxpby{Y + (long long)kb0 * Dout, Dout, 1.f, 0.f, 0}, s);
+    if (e != cudaSuccess) return e;
     if (kb0 > 0) {
-      cudaError_t e = simt_gemm<OP_T, OP_N, float, 0>(kb0, Dout, nb, Operand{L + (long long)kb0 * D, nullptr, D},
-                                                      Operand{Y + (long long)kb0 * Dout, nullptr, Dout},
-                                                      EpiAxpby{Y, Dout, -1.f, 1.f, 0}, s);
+      e = simt_gemm<OP_T, OP_N, float, 0>(kb0, Dout, nb, Operand{L + (long long)kb0 * D, nullptr, D},
+                                          Operand{Y + (long long)kb0 * Dout, nullptr, Dout},
+                                          EpiAxpby{Y, Dout, -1.f, 1.f, 0}, s);
       if (e != cudaSuccess) return e;
     }
   }
@@ -272,7 +242,8 @@ cudaError_t cholesky_solve(int D, int Dout, const float *L, float *Y, cudaStream
 }  // namespace
 
 size_t ridge_workspace_bytes(int D, int Dout) {
-  return align256((size_t)D * D * sizeof(float)) + align256((size_t)D * Dout * sizeof(float)) + 256;
+  return align256((size_t)D * D * sizeof(float)) + align256((size_t)((D + NB - 1) / NB) * NB * NB * sizeof(float)) +
+         align256((size_t)D * Dout * sizeof(float)) + 256;
 }
 
 // ---------------------------------------------------------------------------
@@ -285,6 +256,7 @@ size_t ridge_workspace_bytes(int D, int Dout) {
 // is looked up once per device with cudaGetSymbolAddress.
 // ---------------------------------------------------------------------------
 constexpr size_t kNoAllocScratchBytes = (size_t)ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_D * 4 +
+                                        (size_t)ISPA_RIDGE_NOALLOC_MAX_D * NB * 4 +
                                         (size_t)ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_DOUT * 4 + 256;
 static __device__ __align__(256) unsigned char g_ridge_scratch[kNoAllocScratchBytes];
 
@@ -303,8 +275,8 @@ ispa_status ridge_noalloc_scratch(void **out) {
     addr[dev] = p;
   }
   *out = addr[dev];
-  static_assert(kNoAllocScratchBytes >= (size_t)ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_D * 4 + 256,
-                "scratch smaller than the largest workspace it must hold");
+  static_assert(ISPA_RIDGE_NOALLOC_MAX_D % NB == 0 && ISPA_RIDGE_NOALLOC_MAX_D % 64 == 0,
+                "the largest workspace must fit the scratch exactly");
   return ISPA_OK;
 }
 
@@ -320,36 +292,47 @@ ispa_status launch_ridge(int D, int Dout, const float *G, const float *C, const 
   init_kernel<<<grid, 256, 0, s>>>(D, Dout, G, C, lambda, lambda_relative, w, dW);
   note_launch(2);
   for (int kb0 = 0; kb0 < D; kb0 += NB) {
-    potrf_diag_kernel<<<1, 64, 0, s>>>(D, kb0, w.L, w.flag, err);
+    float *Li = w.Linv + (long long)(kb0 / NB) * NB * NB;
+    potrf_inv_kernel<<<1, 512, 0, s>>>(D, kb0, w.L, Li, w.flag, err);
     note_launch();
     const int below = D - kb0 - NB;
     if (below > 0) {
-      trsm_panel_kernel<<<(below + NB - 1) / NB, 64, 0, s>>>(D, kb0, w.L);
-      note_launch();
+      // panel: L[i, kb] = A[i, kb] Linv_kk^T for the rows below (in place: each CTA owns whole rows)
+      float *panel = w.L + (long long)(kb0 + NB) * D + kb0;
+      cudaError_t e = simt_gemm<OP_N, OP_T, float, 0>(below, NB, NB, Operand{panel, nullptr, D},
+                                                      Operand{Li, nullptr, NB}, EpiAxpby{panel, D, 1.f, 0.f, 0}, s);
+      if (e != cudaSuccess) return cuda_status(e, "ridge panel");
       const int j0 = kb0 + NB;
-      cudaError_t e = simt_gemm<OP_N, OP_T, float, 1>(
-          below, below, NB, Operand{w.L + (long long)j0 * D + kb0, nullptr, D},
-          Operand{w.L + (long long)j0 * D + kb0, nullptr, D},
-          EpiAxpby{w.L + (long long)j0 * D + j0, D, -1.f, 1.f, 1}, s);
+      e = simt_gemm<OP_N, OP_T, float, 1>(below, below, NB, Operand{w.L + (long long)j0 * D + kb0, nullptr, D},
+                                          Operand{w.L + (long long)j0 * D + kb0, nullptr, D},
+                                          EpiAxpby{w.L + (long long)j0 * D + j0, D, -1.f, 1.f, 1}, s);
       if (e != cudaSuccess) return cuda_status(e, "ridge trailing update");
     }
   }
-  cudaError_t e = cholesky_solve(D, Dout, w.L, dW, s);
+  cudaError_t e = cholesky_solve(D, Dout, w.L, w.Linv, dW, s);
   if (e != cudaSuccess) return cuda_status(e, "ridge solve");
   const long long nDO = (long long)D * Dout;
   for (int r = 0; r < refine_steps; ++r) {
     e = simt_gemm<OP_SYM_UPPER, OP_N, double, 0>(D, Dout, D, Operand{G, nullptr, D}, Operand{dW, nullptr, Dout},
                                                  EpiResidual{w.Rres, C, dW, w.acc, Dout}, s);
     if (e != cudaSuccess) return cuda_status(e, "ridge residual");
-    e = cholesky_solve(D, Dout, w.L, w.Rres, s);
+    e = cholesky_solve(D, Dout, w.L, w.Linv, w.Rres, s);
     if (e != cudaSuccess) return cuda_status(e, "ridge refinement solve");
     add_kernel<<<grid, 256, 0, s>>>(nDO, dW, w.Rres);
     note_launch();
   }
   dot_kernel<<<grid, 256, 0, s>>>(nDO, dW, C, w.acc);
   note_launch();
-  e = simt_gemm<OP_SYM_UPPER, OP_N, float, 0>(D, Dout, D, Operand{G, nullptr, D}, Operand{dW, nullptr, Dout},
-                                              EpiDotG{dW, w.acc, Dout, 0.0}, s);
+  if (D % 4 == 0 && Dout % 4 == 0) {
+    // the factor is no longer needed: expand G to the full symmetric matrix there
+    // so that the G dW product reads both operands row-major with 16-byte loads
+    symmetrize_kernel<<<grid, 256, 0, s>>>(D, G, w.L);
+    note_launch();
+    e = simt_gemm_nn128(D, Dout, D, w.L, D, dW, Dout, EpiDotG{dW, w.acc, Dout, 0.0}, s);
+  } else {
+    e = simt_gemm<OP_SYM_UPPER, OP_N, float, 0>(D, Dout, D, Operand{G, nullptr, D}, Operand{dW, nullptr, Dout},
+                                                EpiDotG{dW, w.acc, Dout, 0.0}, s);
+  }
   if (e != cudaSuccess) return cuda_status(e, "ridge G dW");
   finalize_kernel<<<grid, 256, 0, s>>>(nDO, r2, w, dW, eps);
   note_launch();

@@ -99,6 +99,112 @@ inline cudaError_t simt_gemm(int M, int N, int K, Operand A, Operand B, Epi epi,
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Larger-tile variant for big row-major products C = A[M,K] B[K,N] (both
+// operands plain row-major, lda/ldb multiples of 4, 16-byte aligned bases):
+// 128 x 128 output tile, 256 threads with 8 x 8 accumulators each (two 4 x 4
+// quadrants 64 apart in each dimension, so shared-memory reads are float4 and
+// conflict-free), K staged 8 at a time through double-buffered shared memory
+// with the next stage prefetched into registers.
+// ---------------------------------------------------------------------------
+template <class Epi>
+__global__ void __launch_bounds__(256) simt_gemm_nn128_kernel(int M, int N, int K, const float *__restrict__ A,
+                                                              long long lda, const float *__restrict__ B,
+                                                              long long ldb, Epi epi) {
+  __shared__ __align__(16) float As[2][8][128];
+  __shared__ __align__(16) float Bs[2][8][128];
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int m0 = blockIdx.y * 128, n0 = blockIdx.x * 128;
+  // A tile 128 x 8: thread loads row (tid >> 1), 4 k values at (tid & 1) * 4
+  const int a_row = tid >> 1, a_k = (tid & 1) * 4;
+  // B tile 8 x 128: thread loads k row (tid >> 5), 4 columns at (tid & 31) * 4
+  const int b_k = tid >> 5, b_col = (tid & 31) * 4;
+  auto load_a = [&](int k0, float4 &v) {
+    const int gm = m0 + a_row, gk = k0 + a_k;
+    if (gm < M && gk + 3 < K) {
+      v = *reinterpret_cast<const float4 *>(A + (long long)gm * lda + gk);
+    } else {
+      float t[4];
+      for (int i = 0; i < 4; ++i) t[i] = (gm < M && gk + i < K) ? A[(long long)gm * lda + gk + i] : 0.f;
+      v = make_float4(t[0], t[1], t[2], t[3]);
+    }
+  };
+  auto load_b = [&](int k0, float4 &v) {
+    const int gk = k0 + b_k, gn = n0 + b_col;
+    if (gk < K && gn + 3 < N) {
+      v = *reinterpret_cast<const float4 *>(B + (long long)gk * ldb + gn);
+    } else {
+      float t[4];
+      for (int i = 0; i < 4; ++i) t[i] = (gk < K && gn + i < N) ? B[(long long)gk * ldb + gn + i] : 0.f;
+      v = make_float4(t[0], t[1], t[2], t[3]);
+    }
+  };
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  float4 ra, rb;
+  load_a(0, ra);
+  load_b(0, rb);
+  int buf = 0;
+  As[0][a_k + 0][a_row] = ra.x;
+  As[0][a_k + 1][a_row] = ra.y;
+  As[0][a_k + 2][a_row] = ra.z;
+  As[0][a_k + 3][a_row] = ra.w;
+  *reinterpret_cast<float4 *>(&Bs[0][b_k][b_col]) = rb;
+  __syncthreads();
+  for (int k0 = 0; k0 < K; k0 += 8) {
+    const bool more = k0 + 8 < K;
+    if (more) {
+      load_a(k0 + 8, ra);
+      load_b(k0 + 8, rb);
+    }
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4 *>(&As[buf][kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4 *>(&As[buf][kk][ty * 4 + 64]);
+      const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][tx * 4 + 64]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    if (more) {
+      const int nb = buf ^ 1;
+      As[nb][a_k + 0][a_row] = ra.x;
+      As[nb][a_k + 1][a_row] = ra.y;
+      As[nb][a_k + 2][a_row] = ra.z;
+      As[nb][a_k + 3][a_row] = ra.w;
+      *reinterpret_cast<float4 *>(&Bs[nb][b_k][b_col]) = rb;
+      __syncthreads();
+      buf = nb;
+    }
+  }
+  epi.begin();
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int m = m0 + ty * 4 + (i & 3) + (i >> 2) * 64, n = n0 + tx * 4 + (j & 3) + (j >> 2) * 64;
+      if (m < M && n < N) epi(m, n, acc[i][j]);
+    }
+  epi.end();
+}
+
+template <class Epi>
+inline cudaError_t simt_gemm_nn128(int M, int N, int K, const float *A, long long lda, const float *B, long long ldb,
+                                   Epi epi, cudaStream_t s) {
+  if (M <= 0 || N <= 0) return cudaSuccess;
+  dim3 grid((N + 127) / 128, (M + 127) / 128);
+  simt_gemm_nn128_kernel<Epi><<<grid, 256, 0, s>>>(M, N, K, A, lda, B, ldb, epi);
+  note_launch();
+  return cudaGetLastError();
+}
+
 // ---- common epilogues ----
 // out[m*ld + n] = beta * out[...] + alpha * acc   (restricted by `tri`: 0 all, 1 m>=n, 2 m<=n)
 struct EpiAxpby {
