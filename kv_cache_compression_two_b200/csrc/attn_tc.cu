@@ -9,7 +9,8 @@
 // written, and after the history group the optional fused merge combines both
 // groups by their LSE.
 //
-// Warp roles (320 threads, one CTA per SM):
+// Warp roles (384 threads, one CTA per SM; setmaxnreg moves registers from the
+// control warpgroup, 64 per thread, to the softmax warpgroups, 216 per thread):
 //   warp 0      TMA producer: Q_A and Q_B once, then K and V tiles (128 keys x
 //               128 dims) through two-stage rings with separate K and V barriers.
 //   warp 1      TMEM allocator and MMA issuer, per KV tile j:
@@ -18,8 +19,9 @@
 //               PV_j(X): O_X += P_j(X) V_j (fp16 P read from TMEM as operand A,
 //               fp16 V from shared memory), so the softmax of one query tile
 //               overlaps the MMAs of the other.
-//   warps 2-5   softmax / correction / epilogue of query tile A, one row per
-//   warps 6-9   thread (TMEM lane = row); the same for query tile B.
+//   warps 2-3   idle (they complete the control warpgroup).
+//   warps 4-7   softmax / correction / epilogue of query tile A, one row per
+//   warps 8-11  thread (TMEM lane = row); the same for query tile B.
 //
 // TMEM columns: S_A [0,128) S_B [128,256) O_A [256,384) O_B [384,512).  P_j(X)
 // is written as packed fp16 into columns [0,64) of S_X after the softmax has
@@ -41,7 +43,9 @@ namespace ispa {
 
 namespace {
 
-constexpr int kThreads = 320;  // producer, MMA, one softmax warpgroup per query tile
+constexpr int kThreads = 384;  // control warpgroup (producer, MMA, 2 idle) + one softmax warpgroup per query tile
+constexpr int kRegsControl = 64, kRegsSoftmax = 216;
+constexpr int kMinLaunchRegs = (128 * kRegsControl + 256 * kRegsSoftmax + kThreads - 1) / kThreads;
 constexpr int kTileQ = 128, kTileK = 128, kD = 128;
 constexpr int kBoxBytes = 128 * 128;          // 128 rows x 64 bf16
 constexpr int kTileBytes = 2 * kBoxBytes;     // 128 rows x 128 bf16
@@ -309,6 +313,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
+  // Register split: the control warpgroup (warps 0-3: producer, MMA issuer, two
+  // idle warps) gives registers to the two softmax warpgroups.  The block is
+  // launched with 384 x 168; 128 x kRegsControl + 256 x kRegsSoftmax must not
+  // exceed that (the launcher checks the compiled count before launching).
+  // Each role sits inside the branch that set its register budget, so the
+  // compiler allocates every role against its own limit.
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -407,9 +419,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         wait_parity_drain(&sm.drain, 0, P.err);
       }
     }
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // ------------------------------------------------------------ softmax + epilogue
-    const int x = (warp - 2) >> 2;  // query tile of this warpgroup
+    const int x = (warp - 4) >> 2;  // query tile of this warpgroup
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // row inside the tile == TMEM lane
     const int qrow = q0 + x * kTileQ + r;
@@ -563,6 +577,15 @@ ispa_status launch_typed(const CUtensorMap &tq, const CUtensorMap &tk, const CUt
       e = cudaFuncSetAttribute(attn_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kSmemBytes);
     if (e != cudaSuccess) return cuda_status(e, "attention smem attribute");
+    // setmaxnreg.inc waits for registers the block does not have if the launch
+    // allocation is smaller than the split; refuse to launch in that case.
+    cudaFuncAttributes fa[2];
+    e = cudaFuncGetAttributes(&fa[0], attn_tc_kernel<float>);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa[1], attn_tc_kernel<__nv_bfloat16>);
+    if (e != cudaSuccess) return cuda_status(e, "attention attributes");
+    if (fa[0].numRegs < kMinLaunchRegs || fa[1].numRegs < kMinLaunchRegs)
+      return fail(ISPA_ERR_CUDA, "attention kernel compiled with %d/%d registers, the register split needs %d",
+                  fa[0].numRegs, fa[1].numRegs, kMinLaunchRegs);
     configured_device = dev;
   }
   dim3 grid(P.q_tiles * P.H, B);
