@@ -195,7 +195,9 @@ size_t ispa_ridge_workspace_bytes(int D, int Dout);
  *   G [D, D] fp32 (upper triangle read), C [D, Dout] fp32, r2 one double: inputs,
  *   left unchanged.  dW [D, Dout] fp32 and eps (one double) are outputs.
  * A non-positive pivot records ISPA_ERR_NOT_SPD (see ispa_check_device_error)
- * and fills dW with NaN.  Asynchronous.
+ * and fills dW with NaN.  D above the device limit (the solve keeps a D x 8
+ * panel of the right-hand side in shared memory: D <= 6080 with 227 KiB per
+ * block) returns ISPA_ERR_UNSUPPORTED.  Asynchronous.
  */
 ispa_status ispa_ridge_solve(int D, int Dout, const float *G, const float *C, const double *r2,
                              float lambda, int lambda_relative, int refine_steps, float *dW,

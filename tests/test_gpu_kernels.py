@@ -172,6 +172,22 @@ def test_ridge_solve_matches_oracle(D, Dout, refine):
     assert abs(eps - ref_eps) <= 1e-6 * r2, (eps, ref_eps, r2)
 
 
+@pytest.mark.parametrize("D,Dout,T,refine,tol", [
+    (768, 96, 384, 3, 1e-5),     # fewer samples than dimensions: G is rank-deficient, cond(G + lambda I) ~ 6e4
+    (5120, 40, 15360, 0, 1e-2),  # the 14B model's width (40 heads x 128), 80 diagonal blocks
+])
+def test_ridge_solve_rank_deficient_and_wide(D, Dout, T, refine, tol):
+    G, C, r2 = _spd_problem(D, Dout, T, 7 + D)
+    Gs = np.triu(G).astype(np.float64)
+    Gs = Gs + np.triu(Gs, 1).T
+    lam32 = float(np.float32(orc.ridge_lambda(Gs, 1e-4, True)))
+    dW, eps = _run_ridge(G, C, r2, 1e-4, True, refine)
+    ref = orc.ridge_solve(Gs, C.astype(np.float64), lam32)
+    assert rel_fro(dW, ref) <= tol, rel_fro(dW, ref)
+    ref_eps = orc.eps_from_stats(Gs, C.astype(np.float64), r2, dW.astype(np.float64))
+    assert abs(eps - ref_eps) <= 1e-6 * r2, (eps, ref_eps, r2)
+
+
 def test_ridge_absolute_lambda_and_identity():
     D = 96
     G = np.eye(D, dtype=np.float32) * 2.0
