@@ -187,7 +187,7 @@ size_t ispa_ridge_workspace_bytes(int D, int Dout);
 
 /*
  * Closed-form ridge solve [DE-summary 2, "Layer Absorb"; EN-notes, Key Designs 2]:
- *   dW  = (G + lambda I)^-1 C      (Cholesky LL^T = G + lambda I, two triangular solves)
+ *   dW  = (G + lambda I)^-1 C      (Cholesky LL^T = G + lambda I, dW = L^-T (L^-1 C))
  *   eps = ||A_loc (W + dW) - A_full W||_F^2 = r2 - 2<dW, C> + <dW, G dW>
  * lambda_eff = lambda, or lambda * trace(G) / D when lambda_relative != 0.
  * refine_steps extra steps of iterative refinement with fp64 residuals
@@ -195,9 +195,7 @@ size_t ispa_ridge_workspace_bytes(int D, int Dout);
  *   G [D, D] fp32 (upper triangle read), C [D, Dout] fp32, r2 one double: inputs,
  *   left unchanged.  dW [D, Dout] fp32 and eps (one double) are outputs.
  * A non-positive pivot records ISPA_ERR_NOT_SPD (see ispa_check_device_error)
- * and fills dW with NaN.  D above the device limit (the solve keeps a D x 8
- * panel of the right-hand side in shared memory: D <= 6080 with 227 KiB per
- * block) returns ISPA_ERR_UNSUPPORTED.  Asynchronous.
+ * and fills dW with NaN.  Asynchronous.
  */
 ispa_status ispa_ridge_solve(int D, int Dout, const float *G, const float *C, const double *r2,
                              float lambda, int lambda_relative, int refine_steps, float *dW,
@@ -213,9 +211,10 @@ ispa_status ispa_ridge_solve(int D, int Dout, const float *G, const float *C, co
  * application whose device memory is wholly owned by another allocator.
  *
  * Same arguments and results as ispa_ridge_solve, without the workspace.  Its
- * scratch is a static array inside the library of ISPA_RIDGE_NOALLOC_MAX_D^2 +
- * ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_DOUT floats (8 MiB), which
- * every GPU that loads the library holds until the process exits; the call
+ * scratch is a static array inside the library sized for the largest problem
+ * (2.25 ISPA_RIDGE_NOALLOC_MAX_D^2 + 64 ISPA_RIDGE_NOALLOC_MAX_D +
+ * 2 ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_DOUT floats, 17.25 MiB),
+ * which every GPU that loads the library holds until the process exits; the call
  * itself allocates nothing.  D > ISPA_RIDGE_NOALLOC_MAX_D or Dout >
  * ISPA_RIDGE_NOALLOC_MAX_DOUT returns ISPA_ERR_INVALID_ARG.  The first call on
  * a device looks up the array's device address (cudaGetSymbolAddress); make

@@ -290,8 +290,6 @@ ispa_status ispa_ridge_solve(int D, int Dout, const float *G, const float *C, co
   const size_t need = ridge_workspace_bytes(D, Dout);
   if (!workspace || workspace_bytes < need || !aligned16(workspace))
     return fail(ISPA_ERR_INVALID_ARG, "workspace needs %zu bytes (16-byte aligned)", need);
-  const int max_d = ridge_max_dim();
-  if (D > max_d) return fail(ISPA_ERR_UNSUPPORTED, "ridge solve supports D <= %d on this device (got %d)", max_d, D);
   return launch_ridge(D, Dout, G, C, r2, lambda, lambda_relative, refine_steps, dW, eps, workspace,
                       (cudaStream_t)stream);
 }

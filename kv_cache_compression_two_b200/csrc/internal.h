@@ -60,9 +60,6 @@ ispa_status launch_stats(int T, int D, int Dout, const float *a_loc, const float
 
 // ridge
 size_t ridge_workspace_bytes(int D, int Dout);
-// Largest D the ridge solve supports on the current device (its solve keeps a
-// D x 8 panel in shared memory); 0 if the device cannot be queried.
-int ridge_max_dim();
 ispa_status launch_ridge(int D, int Dout, const float *G, const float *C, const double *r2, float lambda,
                          int lambda_relative, int refine_steps, float *dW, double *eps, void *ws,
                          cudaStream_t s);

@@ -8,18 +8,20 @@
 //   diagonal tile (i, i) also stores L_ik^T into the upper tile (k, i), and the
 //   CTA of tile (k+1, k+1) -- block 0, dispatched first -- goes on to factor
 //   that tile and invert its factor, so the next launch finds Linv_{k+1} ready.
-// The lower tiles keep the Schur-complement inputs A_ik; the factor itself is
-// kept as U = L^T in the upper tiles plus the inverses of the diagonal blocks,
-// which is all the triangular solves read.  Both solves run in ONE launch: the
-// right-hand sides are independent, so each CTA takes a panel of 8 columns and
-// carries it through the forward (L z = c) and backward (L^T x = z) block
-// substitutions in shared memory.  Then optional iterative refinement with
-// residuals C - (G + lambda I) X accumulated in fp64, and
-// epsilon = r2 - 2<dW, C> + <dW, G dW> with fp64 reductions.
+// One more launch copies L^T from the upper tiles into the lower ones.  Then
+// X = L^-1 by recursive 2 x 2 block inversion (batched GEMMs, one pair per
+// recursion depth), and the solve is two triangular GEMMs,
+//   dW = X^T (X C),
+// fully parallel instead of a chain of block substitutions; the same X serves
+// the optional iterative refinement (residual C - (G + lambda I) dW with fp64
+// accumulation, dW += X^T (X residual)).  epsilon = r2 - 2<dW, C> + <dW, G dW>
+// with fp64 reductions.
 //
 // Sizes are padded to Dp = 64 * ceil(D / 64) with an identity block, which is
 // decoupled from the problem and keeps every tile whole.
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "internal.h"
 #include "simt_gemm.cuh"
@@ -29,13 +31,14 @@ namespace ispa {
 namespace {
 
 constexpr int NB = 64;
-constexpr int kSolveW = 8;   // right-hand-side columns per CTA of the solve
-constexpr int kRedLd = 68;   // row stride of the solve's cross-warp partial sums
 
 struct Ws {
-  float *M;      // [Dp, Dp] lower tiles: G + lambda I, then Schur inputs; upper tiles: U = L^T
+  float *M;      // [Dp, Dp] lower tiles: G + lambda I, Schur inputs, finally L; upper tiles: L^T
   float *Linv;   // [nb, 64, 64] inverses of the diagonal blocks of L (row-major, lower)
-  float *Rres;   // [D, Dout] refinement residual / correction
+  float *X;      // [Dp, Dp] L^-1 (lower; zero above the diagonal)
+  float *T;      // [Dp * Dp / 4] products of the recursive inversion
+  float *Y;      // [D, Doutp] L^-1 times the right-hand side
+  float *Rres;   // [D, Dout] refinement residual
   double *acc;   // [0] <dW, C>  [1] <dW, G dW>  [2] trace(G)  [3] lambda_eff
   int *flag;     // non-zero once a pivot failed
 };
@@ -43,25 +46,45 @@ struct Ws {
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 int padded(int D) { return (D + NB - 1) / NB * NB; }
 
-Ws carve(void *base, int D, int Dout) {
+int padded4(int n) { return (n + 3) / 4 * 4; }
+
+// Workspace layout; carve() and ridge_workspace_bytes() share it.
+size_t carve_bytes(int D, int Dout, Ws *w, void *base) {
   const size_t Dp = (size_t)padded(D);
-  char *p = static_cast<char *>(base);
+  char *b = static_cast<char *>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char *q = b ? b + off : nullptr;
+    off += align256(bytes);
+    return q;
+  };
+  float *M = reinterpret_cast<float *>(take(Dp * Dp * sizeof(float)));
+  float *Linv = reinterpret_cast<float *>(take(Dp * NB * sizeof(float)));
+  float *X = reinterpret_cast<float *>(take(Dp * Dp * sizeof(float)));
+  float *T = reinterpret_cast<float *>(take(Dp * Dp / 4 * sizeof(float)));
+  float *Y = reinterpret_cast<float *>(take((size_t)D * padded4(Dout) * sizeof(float)));
+  float *R = reinterpret_cast<float *>(take((size_t)D * Dout * sizeof(float)));
+  char *tail = take(256);
+  if (w) {
+    w->M = M;
+    w->Linv = Linv;
+    w->X = X;
+    w->T = T;
+    w->Y = Y;
+    w->Rres = R;
+    w->acc = reinterpret_cast<double *>(tail);
+    w->flag = reinterpret_cast<int *>(tail + 64);
+  }
+  return off;
+}
+
+Ws carve(void *base, int D, int Dout) {
   Ws w;
-  w.M = reinterpret_cast<float *>(p);
-  p += align256(Dp * Dp * sizeof(float));
-  w.Linv = reinterpret_cast<float *>(p);
-  p += align256(Dp * NB * sizeof(float));
-  w.Rres = reinterpret_cast<float *>(p);
-  p += align256((size_t)D * Dout * sizeof(float));
-  w.acc = reinterpret_cast<double *>(p);
-  p += 64;
-  w.flag = reinterpret_cast<int *>(p);
+  carve_bytes(D, Dout, &w, base);
   return w;
 }
 
-size_t solve_smem_bytes(int Dp) {
-  return sizeof(float) * ((size_t)Dp * kSolveW + 8 * kSolveW * kRedLd + NB * kSolveW + NB * (NB + 1));
-}
+
 
 __global__ void trace_kernel(int D, const float *__restrict__ G, double *acc) {
   double s = 0.0;
@@ -78,12 +101,11 @@ __global__ void trace_kernel(int D, const float *__restrict__ G, double *acc) {
 }
 
 // M = G + lambda I on the lower tiles (diagonal tiles whole), identity on the
-// padding; dW = C as the right-hand side.
-__global__ void init_kernel(int D, int Dp, int Dout, const float *__restrict__ G, const float *__restrict__ C,
-                            float lambda, int relative, Ws w, float *dW) {
+// padding.
+__global__ void init_kernel(int D, int Dp, const float *__restrict__ G, float lambda, int relative, Ws w) {
   const double lam = relative ? (double)lambda * w.acc[2] / D : (double)lambda;
   const float lamf = (float)lam;
-  const long long nDD = (long long)Dp * Dp, nDO = (long long)D * Dout;
+  const long long nDD = (long long)Dp * Dp;
   const long long stride = (long long)gridDim.x * blockDim.x;
   const long long t0 = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   if (t0 == 0) {
@@ -99,7 +121,6 @@ __global__ void init_kernel(int D, int Dp, int Dout, const float *__restrict__ G
     if (i < D && j < D) x = G[(long long)min(i, j) * D + max(i, j)] + (i == j ? lamf : 0.f);
     w.M[e] = x;
   }
-  for (long long e = t0; e < nDO; e += stride) dW[e] = C[e];
 }
 
 // ---------------------------------------------------------------------------
@@ -156,71 +177,231 @@ __device__ __forceinline__ void store_acc_t(TileT &T, const float acc[4][4]) {
   }
 }
 
-// Factors the symmetric 64 x 64 matrix S (row-major in shared memory, only the
-// lower triangle read, visible to all threads on entry) as L L^T and writes
-// L^-1 (row-major, lower) to Linv_out.  Forward elimination of [S | I] with
-// Cholesky scaling turns it into [L^T | L^-1]: at pivot p, row p is divided by
-// sqrt(s_pp) and every row r > p loses s_pr / s_pp times the unscaled pivot
-// row.  256 threads; thread t owns row r = t / 4 and columns 16 (t % 4) .. +15
-// of both halves in registers; the pivot row is published through shared
-// memory (prow: 2 x 128 floats, 16-byte aligned, distinct from S; double-
-// buffered, so one barrier per pivot).
-__device__ void factor_invert_tile(const float *S, float *prow, float *__restrict__ Linv_out, int pivot_base,
-                                   int *flag, const DevErr &err) {
-  const int t = threadIdx.x, r = t >> 2, c0 = (t & 3) * 16;
-  float a[16], b[16];
-#pragma unroll
-  for (int jj = 0; jj < 16; ++jj) {
-    const int c = c0 + jj;
-    a[jj] = c <= r ? S[r * NB + c] : S[c * NB + r];
-    b[jj] = c == r ? 1.f : 0.f;
-  }
-  for (int p = 0; p < NB; ++p) {
-    float *pr = prow + (p & 1) * 2 * NB;
-    if (r == p) {
-#pragma unroll
-      for (int jj = 0; jj < 16; jj += 4) {
-        *reinterpret_cast<float4 *>(pr + c0 + jj) = make_float4(a[jj], a[jj + 1], a[jj + 2], a[jj + 3]);
-        *reinterpret_cast<float4 *>(pr + NB + c0 + jj) = make_float4(b[jj], b[jj + 1], b[jj + 2], b[jj + 3]);
-      }
-    }
-    __syncthreads();
-    const float d2 = pr[p];
-    if (t == 0 && !(d2 > 0.f) && atomicExch(flag, 1) == 0) report_error(err, ISPA_ERR_NOT_SPD, pivot_base + p + 1);
-    const float inv = 1.f / sqrtf(d2);  // NaN or inf after a failed pivot; the result is then discarded
-    if (r == p) {
-#pragma unroll
-      for (int jj = 0; jj < 16; ++jj) {
-        a[jj] *= inv;
-        b[jj] *= inv;
-      }
-    } else if (r > p) {
-      const float g = pr[r] * inv * inv;
-#pragma unroll
-      for (int jj = 0; jj < 16; jj += 4) {
-        const float4 pa = *reinterpret_cast<const float4 *>(pr + c0 + jj);
-        const float4 pb = *reinterpret_cast<const float4 *>(pr + NB + c0 + jj);
-        a[jj] = fmaf(-g, pa.x, a[jj]);
-        a[jj + 1] = fmaf(-g, pa.y, a[jj + 1]);
-        a[jj + 2] = fmaf(-g, pa.z, a[jj + 2]);
-        a[jj + 3] = fmaf(-g, pa.w, a[jj + 3]);
-        b[jj] = fmaf(-g, pb.x, b[jj]);
-        b[jj + 1] = fmaf(-g, pb.y, b[jj + 1]);
-        b[jj + 2] = fmaf(-g, pb.z, b[jj + 2]);
-        b[jj + 3] = fmaf(-g, pb.w, b[jj + 3]);
-      }
-    }
-  }
-#pragma unroll
-  for (int jj = 0; jj < 16; jj += 4)
-    *reinterpret_cast<float4 *>(Linv_out + r * NB + c0 + jj) = make_float4(b[jj], b[jj + 1], b[jj + 2], b[jj + 3]);
+// Factors the symmetric 64 x 64 matrix S (row-major in shared memory, lower
+// triangle and diagonal blocks read, visible to all threads on entry) as
+// L L^T and writes L^-1 (row-major, zero above the diagonal) to Linv_out.
+// Block forward elimination of [S | I] with Cholesky scaling, four pivots per
+// step: with C the four current pivot columns, D their 4 x 4 diagonal block
+// and M the inverse of D's Cholesky factor, every row r of the left half below
+// the block loses (C_r M^T)(C_c M^T)^T in column c, the four pivot rows of the
+// right half become M times themselves, and every right-half row below them
+// loses (C_r M^T) times those new rows.  The left half is only needed below
+// and right of the pivots, and by symmetry its pivot rows equal its pivot
+// columns.
+// kFactorThreads threads, each owning one 4 x 4 block in registers: thread
+// (I, J) = (t / 16, t % 16) of the first 256 owns block (I, J) of the left
+// half if I >= J and block (J, I) of the right half if I < J; threads 256..271
+// own the diagonal blocks of the right half.  Per step the owners publish the
+// four pivot columns of the left half and the four pivot rows of the right
+// half, and the owner of D publishes the inverse of D's Cholesky factor, which
+// it formed as soon as its own last update landed (double-buffered, so one
+// barrier per step); every thread then reads the values its block needs.  Entries that are no
+// longer read (columns left of the pivots, the upper part of the left diagonal
+// blocks) are updated without masks; rows of the right half above the pivots
+// are left alone.  bcast: kFactorBcast floats, 16-byte aligned, distinct from S.
+constexpr int kFactorThreads = 288;
+constexpr int kFactorBcast = 2 * 528;  // floats of the factor routine's broadcast buffers
+
+// Inverse m (lower triangular) of the Cholesky factor of the symmetric 4 x 4
+// block d (lower triangle read).  Returns the index of the first non-positive
+// pivot, or -1.
+__device__ __forceinline__ int chol4_inverse(const float d[4][4], float m[4][4]) {
+  const float i0 = rsqrtf(d[0][0]);
+  const float l10 = d[1][0] * i0, l20 = d[2][0] * i0, l30 = d[3][0] * i0;
+  const float s11 = d[1][1] - l10 * l10;
+  const float i1 = rsqrtf(s11);
+  const float l21 = (d[2][1] - l20 * l10) * i1, l31 = (d[3][1] - l30 * l10) * i1;
+  const float s22 = d[2][2] - l20 * l20 - l21 * l21;
+  const float i2 = rsqrtf(s22);
+  const float l32 = (d[3][2] - l30 * l20 - l31 * l21) * i2;
+  const float s33 = d[3][3] - l30 * l30 - l31 * l31 - l32 * l32;
+  const float i3 = rsqrtf(s33);  // NaN after a failed pivot; the result is then discarded
+  m[0][0] = i0;
+  m[1][1] = i1;
+  m[2][2] = i2;
+  m[3][3] = i3;
+  m[1][0] = -l10 * i0 * i1;
+  m[2][1] = -l21 * i1 * i2;
+  m[2][0] = -(l20 * i0 + l21 * m[1][0]) * i2;
+  m[3][2] = -l32 * i2 * i3;
+  m[3][1] = -(l31 * i1 + l32 * m[2][1]) * i3;
+  m[3][0] = -(l30 * i0 + l31 * m[1][0] + l32 * m[2][0]) * i3;
+  m[0][1] = m[0][2] = m[0][3] = m[1][2] = m[1][3] = m[2][3] = 0.f;
+  return !(d[0][0] > 0.f) ? 0 : !(s11 > 0.f) ? 1 : !(s22 > 0.f) ? 2 : !(s33 > 0.f) ? 3 : -1;
 }
 
-// Factor and invert the first diagonal block.  One CTA of 256 threads.
-__global__ void __launch_bounds__(256) chol_first_kernel(int Dp, const float *__restrict__ M, float *Linv, int *flag,
-                                                          DevErr err) {
+__device__ void factor_invert_tile(const float *S, float *bcast, float *__restrict__ Linv_out, int pivot_base,
+                                   int *flag, const DevErr &err) {
+  const int t = threadIdx.x;
+  bool is_b = false, active = true;
+  int R = 0, Cb = 0;  // first row and first column of the owned block
+  if (t < 256) {
+    const int I = t >> 4, J = t & 15;
+    is_b = I < J;
+    R = 4 * (is_b ? J : I);
+    Cb = 4 * (is_b ? I : J);
+  } else if (t < 272) {
+    is_b = true;
+    R = Cb = 4 * (t - 256);
+  } else {
+    active = false;
+  }
+  float x[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      x[i][j] = is_b ? (R + i == Cb + j ? 1.f : 0.f) : (active ? S[(R + i) * NB + Cb + j] : 0.f);
+
+  // The owner of each diagonal block of the left half factors it as soon as
+  // its last update lands (block 0: now) and publishes the inverse factor with
+  // the pivot columns, so no other thread repeats that dependent chain.
+  float mnext[4][4];
+  if (t == 0) {
+    const int bad = chol4_inverse(x, mnext);
+    if (bad >= 0 && atomicExch(flag, 1) == 0) report_error(err, ISPA_ERR_NOT_SPD, pivot_base + bad + 1);
+  }
+  for (int P = 0; P < NB / 4; ++P) {
+    const int p0 = 4 * P;
+    float *cb = bcast + (P & 1) * 528;  // [4 pivot columns][64 rows]
+    float *rb = cb + 256;               // [4 pivot rows][64 columns] of the right half
+    float *mb = cb + 512;               // [4][4] inverse factor of the pivot block
+    if (active && !is_b && Cb == p0) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<float4 *>(cb + j * NB + R) = make_float4(x[0][j], x[1][j], x[2][j], x[3][j]);
+      if (R == p0) {
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+          *reinterpret_cast<float4 *>(mb + 4 * a) = make_float4(mnext[a][0], mnext[a][1], mnext[a][2], mnext[a][3]);
+      }
+    }
+    if (is_b && R == p0) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<float4 *>(rb + i * NB + Cb) = make_float4(x[i][0], x[i][1], x[i][2], x[i][3]);
+    }
+    __syncthreads();
+
+    // the inverse factor of this step's pivot block, published by its owner
+    float m[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const float4 v = *reinterpret_cast<const float4 *>(mb + 4 * a);
+      m[a][0] = v.x;
+      m[a][1] = v.y;
+      m[a][2] = v.z;
+      m[a][3] = v.w;
+    }
+
+    if (!active || (is_b && (R < p0 || Cb > p0 + 3))) continue;  // nothing of this block changes
+
+    // l_r = C_r M^T for this block's rows
+    float cr[4][4], lr[4][4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float4 v = *reinterpret_cast<const float4 *>(cb + k * NB + R);
+      cr[0][k] = v.x;
+      cr[1][k] = v.y;
+      cr[2][k] = v.z;
+      cr[3][k] = v.w;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float s = 0.f;
+#pragma unroll
+        for (int k = 0; k <= j; ++k) s = fmaf(cr[i][k], m[j][k], s);
+        lr[i][j] = s;
+      }
+
+    if (!is_b) {
+      float lc[4][4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float4 v = *reinterpret_cast<const float4 *>(cb + k * NB + Cb);
+        cr[0][k] = v.x;
+        cr[1][k] = v.y;
+        cr[2][k] = v.z;
+        cr[3][k] = v.w;
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float s = 0.f;
+#pragma unroll
+          for (int k = 0; k <= j; ++k) s = fmaf(cr[i][k], m[j][k], s);
+          lc[i][j] = s;
+        }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float s = x[i][j];
+#pragma unroll
+          for (int a = 0; a < 4; ++a) s = fmaf(-lr[i][a], lc[j][a], s);
+          x[i][j] = s;
+        }
+      if (R == Cb && R == p0 + 4) {  // the next pivot block is final now
+        const int bad = chol4_inverse(x, mnext);
+        if (bad >= 0 && atomicExch(flag, 1) == 0) report_error(err, ISPA_ERR_NOT_SPD, pivot_base + R + bad + 1);
+      }
+    } else {
+      // the new pivot rows of the right half at this block's columns: M times the old ones
+      float bp[4][4], bn[4][4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const float4 v = *reinterpret_cast<const float4 *>(rb + a * NB + Cb);
+        bp[a][0] = v.x;
+        bp[a][1] = v.y;
+        bp[a][2] = v.z;
+        bp[a][3] = v.w;
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float s = 0.f;
+#pragma unroll
+          for (int k = 0; k <= a; ++k) s = fmaf(m[a][k], bp[k][j], s);
+          bn[a][j] = s;
+        }
+      if (R == p0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) x[i][j] = bn[i][j];
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            float s = x[i][j];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) s = fmaf(-lr[i][a], bn[a][j], s);
+            x[i][j] = s;
+          }
+      }
+    }
+  }
+  if (is_b) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<float4 *>(Linv_out + (R + i) * NB + Cb) = make_float4(x[i][0], x[i][1], x[i][2], x[i][3]);
+  } else if (active && R != Cb) {  // the mirrored block above the diagonal of L^-1 is zero
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<float4 *>(Linv_out + (Cb + i) * NB + R) = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// Factor and invert the first diagonal block.  One CTA of kFactorThreads threads.
+__global__ void __launch_bounds__(kFactorThreads) chol_first_kernel(int Dp, const float *__restrict__ M, float *Linv,
+                                                                     int *flag, DevErr err) {
   __shared__ __align__(16) float S[NB * NB];
-  __shared__ __align__(16) float prow[4 * NB];
+  __shared__ __align__(16) float prow[kFactorBcast];
   for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) S[e] = M[(long long)(e / NB) * Dp + e % NB];
   __syncthreads();
   factor_invert_tile(S, prow, Linv, 0, flag, err);
@@ -231,11 +412,14 @@ __global__ void __launch_bounds__(256) chol_first_kernel(int Dp, const float *__
 // numbered row by row so that block 0 is the next diagonal tile (k+1, k+1).
 // Reads only column-k tiles and Linv_k; writes only trailing tiles, upper
 // tiles (k, i) and Linv_{k+1}, so no CTA reads what another CTA writes.
-__global__ void __launch_bounds__(256) chol_step_kernel(int Dp, int k, float *M, float *Linv, int *flag, DevErr err) {
+__global__ void __launch_bounds__(kFactorThreads) chol_step_kernel(int Dp, int k, float *M, float *Linv, int *flag,
+                                                                    DevErr err) {
   __shared__ __align__(16) TileT sX;
   __shared__ __align__(16) TileT sY;
   __shared__ __align__(16) TileT sL;
-  const int t = threadIdx.x, ty = t >> 4, tx = t & 15;
+  // threads 0..255 do the tile work; all kFactorThreads factor the next diagonal block
+  const int t = threadIdx.x, ty = (t >> 4) & 15, tx = t & 15;
+  const bool worker = t < 256;
   const int lin = blockIdx.x;
   int ii = (int)((sqrtf(8.f * lin + 1.f) - 1.f) * 0.5f);
   while ((ii + 1) * (ii + 2) / 2 <= lin) ++ii;
@@ -243,208 +427,94 @@ __global__ void __launch_bounds__(256) chol_step_kernel(int Dp, int k, float *M,
   const int i = k + 1 + ii, j = k + 1 + (lin - ii * (ii + 1) / 2);
   const bool diag = i == j;
   const long long ld = Dp;
-
-  load_tile_t(sX, M + (long long)i * NB * ld + k * NB, ld);
-  if (!diag) load_tile_t(sY, M + (long long)j * NB * ld + k * NB, ld);
-  load_tile_t(sL, Linv + (long long)k * NB * NB, NB);
-  float aij[4][4];
   float *tile = M + (long long)i * NB * ld + j * NB;
+
+  float aij[4][4];
+  if (worker) {
+    load_tile_t(sX, M + (long long)i * NB * ld + k * NB, ld);
+    if (!diag) load_tile_t(sY, M + (long long)j * NB * ld + k * NB, ld);
+    load_tile_t(sL, Linv + (long long)k * NB * NB, NB);
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const float4 v = *reinterpret_cast<const float4 *>(tile + (long long)(4 * ty + a) * ld + 4 * tx);
-    aij[a][0] = v.x;
-    aij[a][1] = v.y;
-    aij[a][2] = v.z;
-    aij[a][3] = v.w;
+    for (int a = 0; a < 4; ++a) {
+      const float4 v = *reinterpret_cast<const float4 *>(tile + (long long)(4 * ty + a) * ld + 4 * tx);
+      aij[a][0] = v.x;
+      aij[a][1] = v.y;
+      aij[a][2] = v.z;
+      aij[a][3] = v.w;
+    }
   }
   __syncthreads();
 
   // panel tiles: L_ik = A_ik Linv_kk^T, L_jk = A_jk Linv_kk^T
   float p1[4][4], p2[4][4];
-  tile_xyt(sX, sL, p1);
-  if (!diag) tile_xyt(sY, sL, p2);
-  __syncthreads();
-  store_acc_t(sX, p1);
-  if (!diag) store_acc_t(sY, p2);
-  __syncthreads();
-
-  if (diag) {
-    // upper tile (k, i) = L_ik^T: its row q is column q of L_ik
-#pragma unroll
-    for (int pass = 0; pass < 4; ++pass) {
-      const int q = (t >> 4) + 16 * pass, c = t & 15;
-      const float4 v = *reinterpret_cast<const float4 *>(&sX[q][tgrp(c, q)]);
-      *reinterpret_cast<float4 *>(M + (long long)(k * NB + q) * ld + i * NB + 4 * c) = v;
-    }
+  if (worker) {
+    tile_xyt(sX, sL, p1);
+    if (!diag) tile_xyt(sY, sL, p2);
   }
+  __syncthreads();
+  if (worker) {
+    store_acc_t(sX, p1);
+    if (!diag) store_acc_t(sY, p2);
+  }
+  __syncthreads();
 
-  // trailing update A_ij -= L_ik L_jk^T
-  float upd[4][4];
-  tile_xyt(sX, diag ? sX : sY, upd);
+  if (worker) {
+    if (diag) {
+      // upper tile (k, i) = L_ik^T: its row q is column q of L_ik
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
+      for (int pass = 0; pass < 4; ++pass) {
+        const int q = (t >> 4) + 16 * pass, c = t & 15;
+        const float4 v = *reinterpret_cast<const float4 *>(&sX[q][tgrp(c, q)]);
+        *reinterpret_cast<float4 *>(M + (long long)(k * NB + q) * ld + i * NB + 4 * c) = v;
+      }
+    }
+    // trailing update A_ij -= L_ik L_jk^T
+    float upd[4][4];
+    tile_xyt(sX, diag ? sX : sY, upd);
 #pragma unroll
-    for (int b = 0; b < 4; ++b) aij[a][b] -= upd[a][b];
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) aij[a][b] -= upd[a][b];
+  }
 
   if (i == k + 1) {
     // the next diagonal block: factor and invert it for the next launch
     // (nothing reads the tile itself again, so it is not stored)
     __syncthreads();  // all reads of sX and sY are done
     float *S = &sY[0][0];
+    if (worker) {
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
-      *reinterpret_cast<float4 *>(S + (4 * ty + a) * NB + 4 * tx) = make_float4(aij[a][0], aij[a][1], aij[a][2],
-                                                                              aij[a][3]);
+      for (int a = 0; a < 4; ++a)
+        *reinterpret_cast<float4 *>(S + (4 * ty + a) * NB + 4 * tx) =
+            make_float4(aij[a][0], aij[a][1], aij[a][2], aij[a][3]);
+    }
     __syncthreads();
     factor_invert_tile(S, &sX[0][0], Linv + (long long)(k + 1) * NB * NB, (k + 1) * NB, flag, err);
-  } else {
+  } else if (worker) {
 #pragma unroll
     for (int a = 0; a < 4; ++a)
-      *reinterpret_cast<float4 *>(tile + (long long)(4 * ty + a) * ld + 4 * tx) = make_float4(aij[a][0], aij[a][1],
-                                                                                            aij[a][2], aij[a][3]);
+      *reinterpret_cast<float4 *>(tile + (long long)(4 * ty + a) * ld + 4 * tx) =
+          make_float4(aij[a][0], aij[a][1], aij[a][2], aij[a][3]);
   }
 }
 
-// Both triangular solves for a panel of kSolveW right-hand-side columns, in
-// place on X [D, Dout]: forward L z = c (block row b: z_b = Linv_bb (c_b -
-// sum over k < 64 b of U[k][64 b + r] z_k)), then backward L^T x = z (x_b =
-// Linv_bb^T (z_b - sum over k >= 64 (b + 1) of U[64 b + r][k] x_k)).  The panel
-// lives in shared memory for the whole launch.  256 threads (8 warps).
-//   forward:  lanes take row pairs of the block (coalesced along a row of U),
-//             warps split k; the eight partial sums meet in shared memory.
-//   backward: warps take 8 rows each, lanes split k (coalesced along a row of
-//             U); a butterfly over the lanes leaves each lane two of the sums.
-__global__ void __launch_bounds__(256) chol_solve_kernel(int D, int Dp, int Dout, const float *__restrict__ M,
-                                                         const float *__restrict__ Linv, float *X) {
-  extern __shared__ __align__(16) float smem[];
-  float *z = smem;                                // [Dp][8]
-  float *red = z + (size_t)Dp * kSolveW;          // [8 warps][8 columns][kRedLd]
-  float *tv = red + 8 * kSolveW * kRedLd;         // [64][8]
-  float *sL = tv + NB * kSolveW;                  // [64][65]
-  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int col0 = blockIdx.x * kSolveW, ncol = min(kSolveW, Dout - col0);
-  const int nb = Dp / NB;
+// Lower tile (i, k) = transpose of upper tile (k, i) for every k < i, after the
+// factorisation: the lower triangle then holds L itself (the Schur inputs it
+// held are no longer needed), so that both triangular solves read tiles whose
+// rows run along the output rows.  One CTA per tile pair, 256 threads.
+__global__ void __launch_bounds__(256) upper_to_lower_kernel(int Dp, float *M) {
+  __shared__ float s[NB][NB + 1];
+  const int lin = blockIdx.x;
+  int a = (int)((sqrtf(8.f * lin + 1.f) - 1.f) * 0.5f);
+  while ((a + 1) * (a + 2) / 2 <= lin) ++a;
+  while (a * (a + 1) / 2 > lin) --a;
+  const int i = a + 1, k = lin - a * (a + 1) / 2;  // k <= a < i
   const long long ld = Dp;
-  const int r = t >> 2, cc = (t & 3) * 2;  // this thread's two outputs of a block row
-
-  for (int e = t; e < Dp * kSolveW; e += blockDim.x) {
-    const int row = e / kSolveW, c = e % kSolveW;
-    z[e] = (row < D && c < ncol) ? X[(long long)row * Dout + col0 + c] : 0.f;
-  }
+  const float *src = M + (long long)k * NB * ld + i * NB;
+  float *dst = M + (long long)i * NB * ld + k * NB;
+  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) s[e / NB][e % NB] = src[(e / NB) * ld + e % NB];
   __syncthreads();
-
-  auto stage_linv = [&](int b) {
-    const float *src = Linv + (long long)b * NB * NB;
-    for (int e = t; e < NB * NB; e += blockDim.x) sL[(e / NB) * (NB + 1) + e % NB] = src[e];
-  };
-
-  // ------------------------------------------------------------------ forward
-  for (int b = 0; b < nb; ++b) {
-    const int rb = b * NB;
-    float acc[2][kSolveW];
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-      for (int c = 0; c < kSolveW; ++c) acc[i][c] = 0.f;
-    const float *ucol = M + rb + 2 * lane;
-#pragma unroll 4
-    for (int k = warp; k < rb; k += 8) {
-      const float2 u = *reinterpret_cast<const float2 *>(ucol + (long long)k * ld);
-      const float4 z0 = *reinterpret_cast<const float4 *>(z + k * kSolveW);
-      const float4 z1 = *reinterpret_cast<const float4 *>(z + k * kSolveW + 4);
-      const float zk[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-#pragma unroll
-      for (int c = 0; c < kSolveW; ++c) {
-        acc[0][c] = fmaf(u.x, zk[c], acc[0][c]);
-        acc[1][c] = fmaf(u.y, zk[c], acc[1][c]);
-      }
-    }
-#pragma unroll
-    for (int c = 0; c < kSolveW; ++c)
-      *reinterpret_cast<float2 *>(red + (warp * kSolveW + c) * kRedLd + 2 * lane) = make_float2(acc[0][c], acc[1][c]);
-    stage_linv(b);
-    __syncthreads();
-    {
-      float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) {
-        s0 += red[(w * kSolveW + cc) * kRedLd + r];
-        s1 += red[(w * kSolveW + cc + 1) * kRedLd + r];
-      }
-      const float2 zc = *reinterpret_cast<const float2 *>(z + (rb + r) * kSolveW + cc);
-      *reinterpret_cast<float2 *>(tv + r * kSolveW + cc) = make_float2(zc.x - s0, zc.y - s1);
-    }
-    __syncthreads();
-    {
-      float o0 = 0.f, o1 = 0.f;
-#pragma unroll 8
-      for (int q = 0; q < NB; ++q) {
-        const float l = sL[r * (NB + 1) + q];
-        const float2 v = *reinterpret_cast<const float2 *>(tv + q * kSolveW + cc);
-        o0 = fmaf(l, v.x, o0);
-        o1 = fmaf(l, v.y, o1);
-      }
-      *reinterpret_cast<float2 *>(z + (rb + r) * kSolveW + cc) = make_float2(o0, o1);
-    }
-    __syncthreads();
-  }
-
-  // ----------------------------------------------------------------- backward
-  for (int b = nb - 1; b >= 0; --b) {
-    const int rb = b * NB;
-    float v[64];  // v[i * 8 + c]: row rb + 8 warp + i, column c
-#pragma unroll
-    for (int e = 0; e < 64; ++e) v[e] = 0.f;
-    const float *urow = M + (long long)(rb + 8 * warp) * ld;
-#pragma unroll 2
-    for (int k = rb + NB + lane; k < Dp; k += 32) {
-      const float4 z0 = *reinterpret_cast<const float4 *>(z + k * kSolveW);
-      const float4 z1 = *reinterpret_cast<const float4 *>(z + k * kSolveW + 4);
-      const float zk[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float u = urow[(long long)i * ld + k];
-#pragma unroll
-        for (int c = 0; c < kSolveW; ++c) v[i * 8 + c] = fmaf(u, zk[c], v[i * 8 + c]);
-      }
-    }
-    // reduce-scatter over the lanes: afterwards lane l holds the sums of
-    // entries 2 l and 2 l + 1, i.e. row 8 warp + l / 4, columns 2 (l % 4) + {0, 1}
-#pragma unroll
-    for (int lvl = 0; lvl < 5; ++lvl) {
-      const int half = 32 >> lvl, off = 16 >> lvl;
-      const bool upper = (lane & off) != 0;
-#pragma unroll
-      for (int m = 0; m < half; ++m) {
-        const float keep = upper ? v[half + m] : v[m];
-        const float send = upper ? v[m] : v[half + m];
-        v[m] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-      }
-    }
-    stage_linv(b);
-    {
-      const float2 zc = *reinterpret_cast<const float2 *>(z + (rb + r) * kSolveW + cc);
-      *reinterpret_cast<float2 *>(tv + r * kSolveW + cc) = make_float2(zc.x - v[0], zc.y - v[1]);
-    }
-    __syncthreads();
-    {
-      float o0 = 0.f, o1 = 0.f;
-#pragma unroll 8
-      for (int q = 0; q < NB; ++q) {
-        const float l = sL[q * (NB + 1) + r];
-        const float2 w2 = *reinterpret_cast<const float2 *>(tv + q * kSolveW + cc);
-        o0 = fmaf(l, w2.x, o0);
-        o1 = fmaf(l, w2.y, o1);
-      }
-      *reinterpret_cast<float2 *>(z + (rb + r) * kSolveW + cc) = make_float2(o0, o1);
-    }
-    __syncthreads();
-  }
-
-  for (int e = t; e < D * kSolveW; e += blockDim.x) {
-    const int row = e / kSolveW, c = e % kSolveW;
-    if (c < ncol) X[(long long)row * Dout + col0 + c] = z[e];
-  }
+  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) dst[(e / NB) * ld + e % NB] = s[e % NB][e / NB];
 }
 
 // Rres = C - (G + lambda I) X, accumulated in fp64.
@@ -475,11 +545,6 @@ struct EpiDotG {
   }
 };
 
-__global__ void add_kernel(long long n, float *__restrict__ X, const float *__restrict__ dX) {
-  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x)
-    X[e] += dX[e];
-}
-
 // out[i][j] = G[min(i,j)][max(i,j)]: the full symmetric matrix from its upper triangle.
 __global__ void symmetrize_kernel(int D, const float *__restrict__ G, float *out) {
   const long long n = (long long)D * D;
@@ -506,35 +571,119 @@ __global__ void finalize_kernel(long long n, const double *__restrict__ r2, Ws w
     dW[e] = __int_as_float(0x7fc00000);
 }
 
-// Solves (G + lambda I) X = Y in place on Y [D, Dout] with the factorisation in w.
-cudaError_t cholesky_solve(int D, int Dout, const Ws &w, float *Y, cudaStream_t s) {
-  const int Dp = padded(D);
-  const size_t smem = solve_smem_bytes(Dp);
-  cudaError_t e = cudaFuncSetAttribute(chol_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  chol_solve_kernel<<<(Dout + kSolveW - 1) / kSolveW, 256, smem, s>>>(D, Dp, Dout, w.M, w.Linv, Y);
+// X = 0 with the inverses of L's diagonal blocks on its diagonal tiles.
+__global__ void x_init_kernel(int Dp, const float *__restrict__ Linv, float *X) {
+  const long long n = (long long)Dp * Dp;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
+    const int i = (int)(e / Dp), j = (int)(e - (long long)i * Dp);
+    X[e] = (i / NB == j / NB) ? Linv[(long long)(i / NB) * NB * NB + (i % NB) * NB + j % NB] : 0.f;
+  }
+}
+
+// Launches the jobs in batches of kMaxGemmJobs.  With split_k, K is cut into
+// chunks so that about two CTAs per SM have work (balancing the triangular
+// K ranges); the outputs must then already hold beta C (zero for beta = 0).
+cudaError_t launch_gemm_batch(const GemmJob *jobs, int n, bool a_trans, bool split_k, cudaStream_t s) {
+  for (int b0 = 0; b0 < n; b0 += kMaxGemmJobs) {
+    GemmBatch batch{};
+    const int cnt = n - b0 < kMaxGemmJobs ? n - b0 : kMaxGemmJobs;
+    int max_m = 0, max_n = 0, max_k = 0, vec = 1;
+    long long tiles = 0;
+    for (int i = 0; i < cnt; ++i) {
+      const GemmJob &j = jobs[b0 + i];
+      batch.job[i] = j;
+      max_m = max_m > j.M ? max_m : j.M;
+      max_n = max_n > j.N ? max_n : j.N;
+      max_k = max_k > j.K ? max_k : j.K;
+      tiles += (long long)((j.M + 127) / 128) * ((j.N + 127) / 128);
+      if ((j.lda | j.ldb) % 4 != 0 || !aligned16(j.A) || !aligned16(j.B)) vec = 0;
+    }
+    if (max_m == 0 || max_n == 0) continue;
+    int nsplit = 1, kchunk = max_k;
+    if (split_k && tiles > 0) {
+      const long long want = (2LL * sm_count() + tiles - 1) / tiles;
+      const int most = max_k / 128 > 1 ? max_k / 128 : 1;
+      nsplit = (int)(want < most ? want : most);
+      if (nsplit < 1) nsplit = 1;
+      kchunk = ((max_k + nsplit - 1) / nsplit + 7) / 8 * 8;
+      nsplit = (max_k + kchunk - 1) / kchunk;
+    }
+    dim3 grid((max_n + 127) / 128, (max_m + 127) / 128, cnt * nsplit);
+    if (a_trans)
+      simt_gemm_batched_kernel<true><<<grid, 256, 0, s>>>(batch, vec, nsplit, kchunk);
+    else
+      simt_gemm_batched_kernel<false><<<grid, 256, 0, s>>>(batch, vec, nsplit, kchunk);
+    note_launch();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+// X = L^-1 by recursive 2 x 2 block inversion over ranges of diagonal blocks:
+//   [L11 0; L21 L22]^-1 = [X11 0; -X22 L21 X11  X22],
+// the ranges of one recursion depth combined in one batched launch per
+// product, deepest first (the leaves are the diagonal-block inverses).
+void split_ranges(int lo, int hi, int depth, std::vector<std::vector<std::pair<int, int>>> &levels) {
+  if (hi - lo <= 1) return;
+  const int mid = lo + (hi - lo) / 2;
+  if ((int)levels.size() <= depth) levels.resize(depth + 1);
+  levels[depth].push_back({lo, hi});
+  split_ranges(lo, mid, depth + 1, levels);
+  split_ranges(mid, hi, depth + 1, levels);
+}
+
+cudaError_t invert_factor(int Dp, const Ws &w, cudaStream_t s) {
+  const int nb = Dp / NB;
+  x_init_kernel<<<sm_count() * 4, 256, 0, s>>>(Dp, w.Linv, w.X);
   note_launch();
-  return cudaGetLastError();
+  std::vector<std::vector<std::pair<int, int>>> levels;
+  split_ranges(0, nb, 0, levels);
+  std::vector<GemmJob> first, second;
+  for (int d = (int)levels.size() - 1; d >= 0; --d) {
+    first.clear();
+    second.clear();
+    long long t_off = 0;
+    for (const auto &r : levels[d]) {
+      const int lo = r.first * NB, mid = (r.first + (r.second - r.first) / 2) * NB, hi = r.second * NB;
+      const int n1 = mid - lo, n2 = hi - mid;
+      float *T = w.T + t_off;  // [n2, n1]
+      t_off += (long long)n2 * n1;
+      // T = L21 X11   (X11 lower: B[k][n] = 0 for k < n)
+      first.push_back(GemmJob{w.M + (long long)mid * Dp + lo, w.X + (long long)lo * Dp + lo, T, Dp, Dp, n1, n2, n1,
+                              n1, kTriBLower, 1.f, 0.f});
+      // X21 = -X22 T  (X22 lower: A[m][k] = 0 for k > m)
+      second.push_back(GemmJob{w.X + (long long)mid * Dp + mid, T, w.X + (long long)mid * Dp + lo, Dp, n1, Dp, n2,
+                               n1, n2, kTriALower, -1.f, 0.f});
+    }
+    // T starts at zero (split-K accumulates into it); X21 is still zero from x_init
+    cudaError_t e = cudaMemsetAsync(w.T, 0, (size_t)t_off * sizeof(float), s);
+    if (e == cudaSuccess) e = launch_gemm_batch(first.data(), (int)first.size(), false, true, s);
+    if (e == cudaSuccess) e = launch_gemm_batch(second.data(), (int)second.size(), false, true, s);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+// out = beta out + A^-1 rhs = beta out + X^T (X rhs), rhs and out [D, Dout]
+// (beta 0 or 1).
+cudaError_t apply_inverse(int D, int Dout, const Ws &w, const float *rhs, float *out, float beta, cudaStream_t s) {
+  const int Dp = padded(D), ldy = padded4(Dout);
+  // split-K accumulates into its outputs: Y starts at zero, out at beta out
+  cudaError_t e = cudaMemsetAsync(w.Y, 0, (size_t)D * ldy * sizeof(float), s);
+  if (e == cudaSuccess && beta == 0.f) e = cudaMemsetAsync(out, 0, (size_t)D * Dout * sizeof(float), s);
+  if (e != cudaSuccess) return e;
+  const GemmJob y{w.X, rhs, w.Y, Dp, Dout, ldy, D, Dout, D, kTriALower, 1.f, 0.f};
+  e = launch_gemm_batch(&y, 1, false, true, s);
+  if (e != cudaSuccess) return e;
+  // X^T is upper triangular: op(A)[m][k] = X[k][m] = 0 for k < m
+  const GemmJob x{w.X, w.Y, out, Dp, ldy, Dout, D, Dout, D, kTriAUpper, 1.f, beta};
+  return launch_gemm_batch(&x, 1, true, true, s);
 }
 
 }  // namespace
 
-size_t ridge_workspace_bytes(int D, int Dout) {
-  const size_t Dp = (size_t)padded(D);
-  return align256(Dp * Dp * sizeof(float)) + align256(Dp * NB * sizeof(float)) +
-         align256((size_t)D * Dout * sizeof(float)) + 256;
-}
-
-int ridge_max_dim() {
-  // the solve keeps a Dp x 8 panel in shared memory
-  int dev = 0, optin = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
-    return 0;
-  const size_t fixed = solve_smem_bytes(0);
-  if ((size_t)optin <= fixed) return 0;
-  return (int)(((size_t)optin - fixed) / (sizeof(float) * kSolveW)) / NB * NB;
-}
+size_t ridge_workspace_bytes(int D, int Dout) { return carve_bytes(D, Dout, nullptr, nullptr); }
 
 // ---------------------------------------------------------------------------
 // Allocation-free variant (ispa_ridge_solve_noalloc).  Its scratch -- the
@@ -545,9 +694,14 @@ int ridge_max_dim() {
 // a kernel (on the host it only names a host-side shadow); the device address
 // is looked up once per device with cudaGetSymbolAddress.
 // ---------------------------------------------------------------------------
-constexpr size_t kNoAllocScratchBytes = (size_t)ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_D * 4 +
-                                        (size_t)ISPA_RIDGE_NOALLOC_MAX_D * NB * 4 +
-                                        (size_t)ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_DOUT * 4 + 256;
+// the workspace of the largest size (D a multiple of 64 and Dout of 4, so
+// every part is a multiple of 256 bytes): factor copy, inverse, inversion
+// products, diagonal-block inverses, two D x Dout buffers, accumulators
+constexpr size_t kNoAllocScratchBytes =
+    (size_t)ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_D * 4 * 2 +
+    (size_t)ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_D +
+    (size_t)ISPA_RIDGE_NOALLOC_MAX_D * NB * 4 + (size_t)ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_DOUT * 4 * 2 +
+    256;
 static __device__ __align__(256) unsigned char g_ridge_scratch[kNoAllocScratchBytes];
 
 ispa_status ridge_noalloc_scratch(void **out) {
@@ -565,7 +719,8 @@ ispa_status ridge_noalloc_scratch(void **out) {
     addr[dev] = p;
   }
   *out = addr[dev];
-  static_assert(ISPA_RIDGE_NOALLOC_MAX_D % NB == 0, "the largest workspace must fit the scratch exactly");
+  static_assert(ISPA_RIDGE_NOALLOC_MAX_D % NB == 0 && ISPA_RIDGE_NOALLOC_MAX_DOUT % 64 == 0,
+                "the largest workspace must fit the scratch exactly");
   return ISPA_OK;
 }
 
@@ -579,25 +734,29 @@ ispa_status launch_ridge(int D, int Dout, const float *G, const float *C, const 
   const int Dp = padded(D), nb = Dp / NB;
   const int grid = sm_count() * 4;
   trace_kernel<<<1, 256, 0, s>>>(D, G, w.acc);
-  init_kernel<<<grid, 256, 0, s>>>(D, Dp, Dout, G, C, lambda, lambda_relative, w, dW);
-  chol_first_kernel<<<1, 256, 0, s>>>(Dp, w.M, w.Linv, w.flag, err);
+  init_kernel<<<grid, 256, 0, s>>>(D, Dp, G, lambda, lambda_relative, w);
+  chol_first_kernel<<<1, kFactorThreads, 0, s>>>(Dp, w.M, w.Linv, w.flag, err);
   note_launch(3);
   for (int k = 0; k + 1 < nb; ++k) {
     const int m = nb - k - 1;
-    chol_step_kernel<<<m * (m + 1) / 2, 256, 0, s>>>(Dp, k, w.M, w.Linv, w.flag, err);
+    chol_step_kernel<<<m * (m + 1) / 2, kFactorThreads, 0, s>>>(Dp, k, w.M, w.Linv, w.flag, err);
     note_launch();
   }
-  cudaError_t e = cholesky_solve(D, Dout, w, dW, s);
+  if (nb > 1) {
+    upper_to_lower_kernel<<<nb * (nb - 1) / 2, 256, 0, s>>>(Dp, w.M);
+    note_launch();
+  }
+  cudaError_t e = invert_factor(Dp, w, s);
+  if (e != cudaSuccess) return cuda_status(e, "ridge inverse");
+  e = apply_inverse(D, Dout, w, C, dW, 0.f, s);
   if (e != cudaSuccess) return cuda_status(e, "ridge solve");
   const long long nDO = (long long)D * Dout;
   for (int r = 0; r < refine_steps; ++r) {
     e = simt_gemm<OP_SYM_UPPER, OP_N, double, 0>(D, Dout, D, Operand{G, nullptr, D}, Operand{dW, nullptr, Dout},
                                                  EpiResidual{w.Rres, C, dW, w.acc, Dout}, s);
     if (e != cudaSuccess) return cuda_status(e, "ridge residual");
-    e = cholesky_solve(D, Dout, w, w.Rres, s);
+    e = apply_inverse(D, Dout, w, w.Rres, dW, 1.f, s);
     if (e != cudaSuccess) return cuda_status(e, "ridge refinement solve");
-    add_kernel<<<grid, 256, 0, s>>>(nDO, dW, w.Rres);
-    note_launch();
   }
   dot_kernel<<<grid, 256, 0, s>>>(nDO, dW, C, w.acc);
   note_launch();

@@ -223,3 +223,153 @@ struct EpiAxpby {
 };
 
 }  // namespace ispa
+
+namespace ispa {
+
+// ---------------------------------------------------------------------------
+// Batched 128 x 128-tile GEMM for the triangular products of the ridge solve:
+//   C = alpha op(A) B + beta C,  op(A) = A [M, K] or A^T (A stored [K, M]),
+// B [K, N], all row-major.  One z-slice of the grid per job.  A triangle that
+// is zero is skipped at tile granularity through the K range of each output
+// tile (the skipped region must hold zeros or lie outside the triangle):
+//   kTriALower: op(A)[m][k] = 0 for k > m   ->  k <  m0 + 128
+//   kTriAUpper: op(A)[m][k] = 0 for k < m   ->  k >= m0
+//   kTriBLower: B[k][n] = 0 for k < n       ->  k >= n0
+// Operands are read with 16-byte loads when every leading dimension is a
+// multiple of 4 and every base 16-byte aligned (vec), element by element
+// otherwise.  The inner loop is the one of simt_gemm_nn128_kernel.
+// ---------------------------------------------------------------------------
+enum { kTriNone = 0, kTriALower = 1, kTriAUpper = 2, kTriBLower = 3 };
+
+struct GemmJob {
+  const float *A;
+  const float *B;
+  float *C;
+  long long lda, ldb, ldc;
+  int M, N, K, tri;
+  float alpha, beta;
+};
+
+constexpr int kMaxGemmJobs = 32;
+struct GemmBatch {
+  GemmJob job[kMaxGemmJobs];
+};
+
+// Split K: with nsplit > 1, grid z-slice z handles job z / nsplit and the K
+// chunk z % nsplit of length kchunk (a multiple of 8) of every output tile's
+// K range, and adds alpha times its partial product to C with atomics (C must
+// then hold beta C already: zero for beta = 0).
+template <bool AT>
+__global__ void __launch_bounds__(256, 2) simt_gemm_batched_kernel(GemmBatch batch, int vec, int nsplit, int kchunk) {
+  const GemmJob &j = batch.job[blockIdx.z / nsplit];
+  const int chunk = blockIdx.z % nsplit;
+  const int m0 = blockIdx.y * 128, n0 = blockIdx.x * 128;
+  if (m0 >= j.M || n0 >= j.N) return;
+  int k_lo = 0, k_hi = j.K;
+  if (j.tri == kTriALower) k_hi = min(j.K, m0 + 128);
+  if (j.tri == kTriAUpper) k_lo = m0;
+  if (j.tri == kTriBLower) k_lo = n0;
+  if (nsplit > 1) {
+    k_lo += chunk * kchunk;
+    k_hi = min(k_hi, k_lo + kchunk);
+    if (k_lo >= k_hi) return;
+  }
+  __shared__ __align__(16) float As[2][8][128];
+  __shared__ __align__(16) float Bs[2][8][128];
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  // A tile 128 (m) x 8 (k): row-major A: thread takes row tid / 2, 4 k at (tid & 1) * 4;
+  //                          transposed A: thread takes k row tid / 32, 4 m at (tid & 31) * 4
+  // B tile 8 (k) x 128 (n): thread takes k row tid / 32, 4 columns at (tid & 31) * 4
+  const int a_r = AT ? (tid >> 5) : (tid >> 1), a_c = AT ? (tid & 31) * 4 : (tid & 1) * 4;
+  const int b_k = tid >> 5, b_col = (tid & 31) * 4;
+  auto load_a = [&](int k0, float (&v)[4]) {
+    if (!AT) {
+      const int gm = m0 + a_r, gk = k0 + a_c;
+      if (vec && gm < j.M && gk + 3 < k_hi) {
+        const float4 t = *reinterpret_cast<const float4 *>(j.A + (long long)gm * j.lda + gk);
+        v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+      } else {
+        for (int i = 0; i < 4; ++i)
+          v[i] = (gm < j.M && gk + i < k_hi) ? j.A[(long long)gm * j.lda + gk + i] : 0.f;
+      }
+    } else {
+      const int gk = k0 + a_r, gm = m0 + a_c;
+      if (vec && gk < k_hi && gm + 3 < j.M) {
+        const float4 t = *reinterpret_cast<const float4 *>(j.A + (long long)gk * j.lda + gm);
+        v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+      } else {
+        for (int i = 0; i < 4; ++i)
+          v[i] = (gk < k_hi && gm + i < j.M) ? j.A[(long long)gk * j.lda + gm + i] : 0.f;
+      }
+    }
+  };
+  auto load_b = [&](int k0, float (&v)[4]) {
+    const int gk = k0 + b_k, gn = n0 + b_col;
+    if (vec && gk < k_hi && gn + 3 < j.N) {
+      const float4 t = *reinterpret_cast<const float4 *>(j.B + (long long)gk * j.ldb + gn);
+      v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+    } else {
+      for (int i = 0; i < 4; ++i) v[i] = (gk < k_hi && gn + i < j.N) ? j.B[(long long)gk * j.ldb + gn + i] : 0.f;
+    }
+  };
+  auto stage = [&](int buf, const float (&ra)[4], const float (&rb)[4]) {
+    if (!AT) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) As[buf][a_c + i][a_r] = ra[i];
+    } else {
+      *reinterpret_cast<float4 *>(&As[buf][a_r][a_c]) = make_float4(ra[0], ra[1], ra[2], ra[3]);
+    }
+    *reinterpret_cast<float4 *>(&Bs[buf][b_k][b_col]) = make_float4(rb[0], rb[1], rb[2], rb[3]);
+  };
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[i][c] = 0.f;
+  float ra[4], rb[4];
+  load_a(k_lo, ra);
+  load_b(k_lo, rb);
+  int buf = 0;
+  stage(0, ra, rb);
+  __syncthreads();
+  for (int k0 = k_lo; k0 < k_hi; k0 += 8) {
+    const bool more = k0 + 8 < k_hi;
+    if (more) {
+      load_a(k0 + 8, ra);
+      load_b(k0 + 8, rb);
+    }
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4 *>(&As[buf][kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4 *>(&As[buf][kk][ty * 4 + 64]);
+      const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][tx * 4 + 64]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[i][c] = fmaf(a[i], b[c], acc[i][c]);
+    }
+    if (more) {
+      stage(buf ^ 1, ra, rb);
+      __syncthreads();
+      buf ^= 1;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int m = m0 + ty * 4 + (i & 3) + (i >> 2) * 64, n = n0 + tx * 4 + (c & 3) + (c >> 2) * 64;
+      if (m < j.M && n < j.N) {
+        float *p = j.C + (long long)m * j.ldc + n;
+        if (nsplit > 1)
+          atomicAdd(p, j.alpha * acc[i][c]);
+        else
+          *p = j.alpha * acc[i][c] + (j.beta == 0.f ? 0.f : j.beta * *p);
+      }
+    }
+}
+
+}  // namespace ispa
