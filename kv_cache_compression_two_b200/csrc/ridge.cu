@@ -177,30 +177,8 @@ __device__ __forceinline__ void store_acc_t(TileT &T, const float acc[4][4]) {
   }
 }
 
-// Factors the symmetric 64 x 64 matrix S (row-major in shared memory, lower
-// triangle and diagonal blocks read, visible to all threads on entry) as
-// L L^T and writes L^-1 (row-major, zero above the diagonal) to Linv_out.
-// Block forward elimination of [S | I] with Cholesky scaling, four pivots per
-// step: with C the four current pivot columns, D their 4 x 4 diagonal block
-// and M the inverse of D's Cholesky factor, every row r of the left half below
-// the block loses (C_r M^T)(C_c M^T)^T in column c, the four pivot rows of the
-// right half become M times themselves, and every right-half row below them
-// loses (C_r M^T) times those new rows.  The left half is only needed below
-// and right of the pivots, and by symmetry its pivot rows equal its pivot
-// columns.
-// kFactorThreads threads, each owning one 4 x 4 block in registers: thread
-// (I, J) = (t / 16, t % 16) of the first 256 owns block (I, J) of the left
-// half if I >= J and block (J, I) of the right half if I < J; threads 256..271
-// own the diagonal blocks of the right half.  Per step the owners publish the
-// four pivot columns of the left half and the four pivot rows of the right
-// half, and the owner of D publishes the inverse of D's Cholesky factor, which
-// it formed as soon as its own last update landed (double-buffered, so one
-// barrier per step); every thread then reads the values its block needs.  Entries that are no
-// longer read (columns left of the pivots, the upper part of the left diagonal
-// blocks) are updated without masks; rows of the right half above the pivots
-// are left alone.  bcast: kFactorBcast floats, 16-byte aligned, distinct from S.
 constexpr int kFactorThreads = 288;
-constexpr int kFactorBcast = 2 * 528;  // floats of the factor routine's broadcast buffers
+constexpr int kFactorBcast = 8 * 64 + 16;  // floats of the factor routine's broadcast buffers
 
 // Inverse m (lower triangular) of the Cholesky factor of the symmetric 4 x 4
 // block d (lower triangle read).  Returns the index of the first non-positive
@@ -230,7 +208,32 @@ __device__ __forceinline__ int chol4_inverse(const float d[4][4], float m[4][4])
   return !(d[0][0] > 0.f) ? 0 : !(s11 > 0.f) ? 1 : !(s22 > 0.f) ? 2 : !(s33 > 0.f) ? 3 : -1;
 }
 
-__device__ void factor_invert_tile(const float *S, float *bcast, float *__restrict__ Linv_out, int pivot_base,
+// Factors the symmetric 64 x 64 matrix S (row-major in shared memory, lower
+// triangle and diagonal blocks read, visible to all threads on entry) as
+// L L^T and writes L^-1 (row-major, zero above the diagonal) to Linv_out.
+// Block forward elimination of [S | I] with Cholesky scaling, four pivots per
+// step: with C the four current pivot columns, D their 4 x 4 diagonal block
+// and M the inverse of D's Cholesky factor, every row r of the left half below
+// the block loses l_r l_c^T in column c (l = C M^T), the four pivot rows of the
+// right half become M times themselves, and every right-half row below them
+// loses l_r times those new rows.  The left half is only needed below and
+// right of the pivots; by symmetry its pivot rows equal its pivot columns.
+// kFactorThreads threads, each owning one 4 x 4 block in registers: thread
+// (I, J) = (t / 16, t % 16) of the first 256 owns block (I, J) of the left
+// half if I >= J and block (J, I) of the right half if I < J; threads 256..271
+// own the diagonal blocks of the right half.  Two barriers per step:
+//   phase A: the owners of the pivot block column form l for their rows, the
+//            owners of the pivot rows of the right half form M times them,
+//            both into shared memory (M was published by the owner of D, who
+//            factored D as soon as its own last update landed);
+//   phase B: every block applies its rank-4 update from those vectors, and the
+//            owner of the next pivot block factors it and publishes its M.
+// Entries that are no longer read (columns left of the pivots, the upper part
+// of the left diagonal blocks) are updated without masks; rows of the right
+// half above the pivots are left alone.  bcast: kFactorBcast floats, 16-byte
+// aligned, distinct from S.
+__device__ __forceinline__ void factor_invert_tile(const float *S, float *bcast, float *__restrict__ Linv_out,
+                                                   int pivot_base,
                                    int *flag, const DevErr &err) {
   const int t = threadIdx.x;
   bool is_b = false, active = true;
@@ -252,138 +255,108 @@ __device__ void factor_invert_tile(const float *S, float *bcast, float *__restri
 #pragma unroll
     for (int j = 0; j < 4; ++j)
       x[i][j] = is_b ? (R + i == Cb + j ? 1.f : 0.f) : (active ? S[(R + i) * NB + Cb + j] : 0.f);
+  float *lbuf = bcast;               // [64 rows][4]: l = C M^T of the pivot block column
+  float *bbuf = bcast + 4 * NB;      // [4 rows][64]: new pivot rows of the right half
+  float *mb = bcast + 8 * NB;        // [4][4]: M of the current pivot block
 
-  // The owner of each diagonal block of the left half factors it as soon as
-  // its last update lands (block 0: now) and publishes the inverse factor with
-  // the pivot columns, so no other thread repeats that dependent chain.
-  float mnext[4][4];
-  if (t == 0) {
-    const int bad = chol4_inverse(x, mnext);
-    if (bad >= 0 && atomicExch(flag, 1) == 0) report_error(err, ISPA_ERR_NOT_SPD, pivot_base + bad + 1);
-  }
+  auto publish_m = [&](int pivot0) {  // factor the pivot block held in x, publish its M
+    float m[4][4];
+    const int bad = chol4_inverse(x, m);
+    if (bad >= 0 && atomicExch(flag, 1) == 0) report_error(err, ISPA_ERR_NOT_SPD, pivot_base + pivot0 + bad + 1);
+#pragma unroll
+    for (int a = 0; a < 4; ++a) *reinterpret_cast<float4 *>(mb + 4 * a) = make_float4(m[a][0], m[a][1], m[a][2], m[a][3]);
+  };
+  if (t == 0) publish_m(0);
+
   for (int P = 0; P < NB / 4; ++P) {
     const int p0 = 4 * P;
-    float *cb = bcast + (P & 1) * 528;  // [4 pivot columns][64 rows]
-    float *rb = cb + 256;               // [4 pivot rows][64 columns] of the right half
-    float *mb = cb + 512;               // [4][4] inverse factor of the pivot block
-    if (active && !is_b && Cb == p0) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        *reinterpret_cast<float4 *>(cb + j * NB + R) = make_float4(x[0][j], x[1][j], x[2][j], x[3][j]);
-      if (R == p0) {
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-          *reinterpret_cast<float4 *>(mb + 4 * a) = make_float4(mnext[a][0], mnext[a][1], mnext[a][2], mnext[a][3]);
-      }
-    }
-    if (is_b && R == p0) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        *reinterpret_cast<float4 *>(rb + i * NB + Cb) = make_float4(x[i][0], x[i][1], x[i][2], x[i][3]);
-    }
-    __syncthreads();
-
-    // the inverse factor of this step's pivot block, published by its owner
-    float m[4][4];
-#pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const float4 v = *reinterpret_cast<const float4 *>(mb + 4 * a);
-      m[a][0] = v.x;
-      m[a][1] = v.y;
-      m[a][2] = v.z;
-      m[a][3] = v.w;
-    }
-
-    if (!active || (is_b && (R < p0 || Cb > p0 + 3))) continue;  // nothing of this block changes
-
-    // l_r = C_r M^T for this block's rows
-    float cr[4][4], lr[4][4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float4 v = *reinterpret_cast<const float4 *>(cb + k * NB + R);
-      cr[0][k] = v.x;
-      cr[1][k] = v.y;
-      cr[2][k] = v.z;
-      cr[3][k] = v.w;
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float s = 0.f;
-#pragma unroll
-        for (int k = 0; k <= j; ++k) s = fmaf(cr[i][k], m[j][k], s);
-        lr[i][j] = s;
-      }
-
-    if (!is_b) {
-      float lc[4][4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float4 v = *reinterpret_cast<const float4 *>(cb + k * NB + Cb);
-        cr[0][k] = v.x;
-        cr[1][k] = v.y;
-        cr[2][k] = v.z;
-        cr[3][k] = v.w;
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float s = 0.f;
-#pragma unroll
-          for (int k = 0; k <= j; ++k) s = fmaf(cr[i][k], m[j][k], s);
-          lc[i][j] = s;
-        }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float s = x[i][j];
-#pragma unroll
-          for (int a = 0; a < 4; ++a) s = fmaf(-lr[i][a], lc[j][a], s);
-          x[i][j] = s;
-        }
-      if (R == Cb && R == p0 + 4) {  // the next pivot block is final now
-        const int bad = chol4_inverse(x, mnext);
-        if (bad >= 0 && atomicExch(flag, 1) == 0) report_error(err, ISPA_ERR_NOT_SPD, pivot_base + R + bad + 1);
-      }
-    } else {
-      // the new pivot rows of the right half at this block's columns: M times the old ones
-      float bp[4][4], bn[4][4];
+    __syncthreads();  // M of this step is visible; the previous step's phase B is done
+    // ---- phase A
+    const bool col_owner = active && !is_b && Cb == p0;
+    const bool row_owner = is_b && R == p0;
+    if (col_owner || row_owner) {
+      float m[4][4];
 #pragma unroll
       for (int a = 0; a < 4; ++a) {
-        const float4 v = *reinterpret_cast<const float4 *>(rb + a * NB + Cb);
-        bp[a][0] = v.x;
-        bp[a][1] = v.y;
-        bp[a][2] = v.z;
-        bp[a][3] = v.w;
+        const float4 v = *reinterpret_cast<const float4 *>(mb + 4 * a);
+        m[a][0] = v.x;
+        m[a][1] = v.y;
+        m[a][2] = v.z;
+        m[a][3] = v.w;
       }
+      if (col_owner) {  // l_r = C_r M^T for this block's four rows
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+        for (int i = 0; i < 4; ++i) {
+          float l[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float s = 0.f;
+          for (int jj = 0; jj < 4; ++jj) {
+            float s = 0.f;
 #pragma unroll
-          for (int k = 0; k <= a; ++k) s = fmaf(m[a][k], bp[k][j], s);
-          bn[a][j] = s;
-        }
-      if (R == p0) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) x[i][j] = bn[i][j];
-      } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float s = x[i][j];
-#pragma unroll
-            for (int a = 0; a < 4; ++a) s = fmaf(-lr[i][a], bn[a][j], s);
-            x[i][j] = s;
+            for (int k = 0; k <= jj; ++k) s = fmaf(x[i][k], m[jj][k], s);
+            l[jj] = s;
           }
+          *reinterpret_cast<float4 *>(lbuf + (R + i) * 4) = make_float4(l[0], l[1], l[2], l[3]);
+        }
+      } else {  // the pivot rows of the right half: M times them
+        float bn[4][4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            float s = 0.f;
+#pragma unroll
+            for (int k = 0; k <= a; ++k) s = fmaf(m[a][k], x[k][jj], s);
+            bn[a][jj] = s;
+          }
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          *reinterpret_cast<float4 *>(bbuf + a * NB + Cb) = make_float4(bn[a][0], bn[a][1], bn[a][2], bn[a][3]);
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) x[a][jj] = bn[a][jj];
+        }
       }
+    }
+    __syncthreads();
+    // ---- phase B
+    if (active && (!is_b || (R > p0 && Cb <= p0 + 3))) {
+      float lr[4][4], v[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 a = *reinterpret_cast<const float4 *>(lbuf + (R + i) * 4);
+        lr[i][0] = a.x;
+        lr[i][1] = a.y;
+        lr[i][2] = a.z;
+        lr[i][3] = a.w;
+      }
+      if (!is_b) {  // v[j][a] = l of column Cb + j
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const float4 a = *reinterpret_cast<const float4 *>(lbuf + (Cb + jj) * 4);
+          v[jj][0] = a.x;
+          v[jj][1] = a.y;
+          v[jj][2] = a.z;
+          v[jj][3] = a.w;
+        }
+      } else {  // v[j][a] = new pivot row a at column Cb + j
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          const float4 b = *reinterpret_cast<const float4 *>(bbuf + a * NB + Cb);
+          v[0][a] = b.x;
+          v[1][a] = b.y;
+          v[2][a] = b.z;
+          v[3][a] = b.w;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          float s = x[i][jj];
+#pragma unroll
+          for (int a = 0; a < 4; ++a) s = fmaf(-lr[i][a], v[jj][a], s);
+          x[i][jj] = s;
+        }
+      if (!is_b && R == Cb && R == p0 + 4) publish_m(R);  // the next pivot block is final now
     }
   }
   if (is_b) {
@@ -581,8 +554,9 @@ __global__ void x_init_kernel(int Dp, const float *__restrict__ Linv, float *X) 
 }
 
 // Launches the jobs in batches of kMaxGemmJobs.  With split_k, K is cut into
-// chunks so that about two CTAs per SM have work (balancing the triangular
-// K ranges); the outputs must then already hold beta C (zero for beta = 0).
+// chunks so that every SM gets a few CTAs (balancing the triangular K ranges
+// and giving the small products of the inversion enough parallelism); the
+// outputs must then already hold beta C (zero for beta = 0).
 cudaError_t launch_gemm_batch(const GemmJob *jobs, int n, bool a_trans, bool split_k, cudaStream_t s) {
   for (int b0 = 0; b0 < n; b0 += kMaxGemmJobs) {
     GemmBatch batch{};
@@ -601,18 +575,36 @@ cudaError_t launch_gemm_batch(const GemmJob *jobs, int n, bool a_trans, bool spl
     if (max_m == 0 || max_n == 0) continue;
     int nsplit = 1, kchunk = max_k;
     if (split_k && tiles > 0) {
-      const long long want = (2LL * sm_count() + tiles - 1) / tiles;
-      const int most = max_k / 128 > 1 ? max_k / 128 : 1;
-      nsplit = (int)(want < most ? want : most);
-      if (nsplit < 1) nsplit = 1;
-      kchunk = ((max_k + nsplit - 1) / nsplit + 7) / 8 * 8;
+      // chunks of kPipeBK-multiples, about four CTAs per SM in total (the
+      // chunks past a tile's triangle are empty, so roughly two do work)
+      const long long units = tiles * ((max_k + kPipeBK - 1) / kPipeBK);
+      const long long per = units / (4LL * sm_count());
+      kchunk = (int)(per > 1 ? per : 1) * kPipeBK;
       nsplit = (max_k + kchunk - 1) / kchunk;
     }
     dim3 grid((max_n + 127) / 128, (max_m + 127) / 128, cnt * nsplit);
-    if (a_trans)
+    if (vec) {  // 16-byte operands: the cp.async pipeline
+      static thread_local int configured_device = -1;
+      int dev = 0;
+      cudaGetDevice(&dev);
+      if (configured_device != dev) {
+        cudaError_t e = cudaFuncSetAttribute(simt_gemm_pipe_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kPipeSmemBytes);
+        if (e == cudaSuccess)
+          e = cudaFuncSetAttribute(simt_gemm_pipe_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)kPipeSmemBytes);
+        if (e != cudaSuccess) return e;
+        configured_device = dev;
+      }
+      if (a_trans)
+        simt_gemm_pipe_kernel<true><<<grid, 256, kPipeSmemBytes, s>>>(batch, nsplit, kchunk);
+      else
+        simt_gemm_pipe_kernel<false><<<grid, 256, kPipeSmemBytes, s>>>(batch, nsplit, kchunk);
+    } else if (a_trans) {
       simt_gemm_batched_kernel<true><<<grid, 256, 0, s>>>(batch, vec, nsplit, kchunk);
-    else
+    } else {
       simt_gemm_batched_kernel<false><<<grid, 256, 0, s>>>(batch, vec, nsplit, kchunk);
+    }
     note_launch();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -373,3 +373,127 @@ __global__ void __launch_bounds__(256, 2) simt_gemm_batched_kernel(GemmBatch bat
 }
 
 }  // namespace ispa
+
+namespace ispa {
+
+// ---------------------------------------------------------------------------
+// Pipelined form of simt_gemm_batched_kernel (same jobs, triangles and split
+// K), for 16-byte-aligned operands with leading dimensions that are multiples
+// of 4: K advances 16 at a time through a kPipeStages-deep cp.async ring, so
+// the L2 latency of a stage hides behind the arithmetic of the stages ahead.
+// Transposed A ([K, M] in memory) and B are copied as they are ([k][m],
+// [k][n]); row-major A is kept as [m][k] (row stride kPipeALd) and read as
+// broadcast scalars.  Edges are zero-filled by the copy (src-size < 16).
+// ---------------------------------------------------------------------------
+constexpr int kPipeStages = 4, kPipeBK = 16, kPipeALd = 20;
+constexpr int kPipeStageFloats = 128 * kPipeALd + kPipeBK * 128;  // A (either layout) + B
+constexpr size_t kPipeSmemBytes = sizeof(float) * kPipeStages * kPipeStageFloats;
+
+__device__ __forceinline__ void cp_async16_zfill(void *dst, const void *src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+template <bool AT>
+__global__ void __launch_bounds__(256, 2) simt_gemm_pipe_kernel(GemmBatch batch, int nsplit, int kchunk) {
+  extern __shared__ __align__(16) float pipe_smem[];
+  const GemmJob &j = batch.job[blockIdx.z / nsplit];
+  const int chunk = blockIdx.z % nsplit;
+  const int m0 = blockIdx.y * 128, n0 = blockIdx.x * 128;
+  if (m0 >= j.M || n0 >= j.N) return;
+  int k_lo = 0, k_hi = j.K;
+  if (j.tri == kTriALower) k_hi = min(j.K, m0 + 128);
+  if (j.tri == kTriAUpper) k_lo = m0;
+  if (j.tri == kTriBLower) k_lo = n0;
+  if (nsplit > 1) {
+    k_lo += chunk * kchunk;
+    k_hi = min(k_hi, k_lo + kchunk);
+  }
+  if (k_lo >= k_hi) {
+    if (nsplit > 1) return;  // nothing to add
+  }
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int nk = k_hi > k_lo ? (k_hi - k_lo + kPipeBK - 1) / kPipeBK : 0;
+
+  auto issue = [&](int kb) {
+    float *As = pipe_smem + (kb % kPipeStages) * kPipeStageFloats;
+    float *Bs = As + 128 * kPipeALd;
+    const int k0 = k_lo + kb * kPipeBK;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int e = tid + 256 * u;
+      {  // B: 16 rows x 32 chunks of 4 columns
+        const int r = e >> 5, c = (e & 31) * 4, gk = k0 + r, gn = n0 + c;
+        const int nv = (gk < k_hi) ? max(0, min(4, j.N - gn)) : 0;
+        cp_async16_zfill(Bs + r * 128 + c, nv ? j.B + (long long)gk * j.ldb + gn : j.B, nv * 4);
+      }
+      if (AT) {  // A^T: 16 rows (k) x 32 chunks of 4 m
+        const int r = e >> 5, c = (e & 31) * 4, gk = k0 + r, gm = m0 + c;
+        const int nv = (gk < k_hi) ? max(0, min(4, j.M - gm)) : 0;
+        cp_async16_zfill(As + r * 128 + c, nv ? j.A + (long long)gk * j.lda + gm : j.A, nv * 4);
+      } else {  // A: 128 rows (m) x 4 chunks of 4 k
+        const int r = e >> 2, c = (e & 3) * 4, gm = m0 + r, gk = k0 + c;
+        const int nv = (gm < j.M) ? max(0, min(4, k_hi - gk)) : 0;
+        cp_async16_zfill(As + r * kPipeALd + c, nv ? j.A + (long long)gm * j.lda + gk : j.A, nv * 4);
+      }
+    }
+  };
+
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[i][c] = 0.f;
+#pragma unroll
+  for (int s = 0; s < kPipeStages - 1; ++s) {
+    if (s < nk) issue(s);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  for (int kb = 0; kb < nk; ++kb) {
+    asm volatile("cp.async.wait_group %0;" ::"n"(kPipeStages - 2) : "memory");
+    __syncthreads();  // stage kb landed for every thread; stage kb - 1 is free
+    if (kb + kPipeStages - 1 < nk) issue(kb + kPipeStages - 1);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    const float *As = pipe_smem + (kb % kPipeStages) * kPipeStageFloats;
+    const float *Bs = As + 128 * kPipeALd;
+#pragma unroll
+    for (int kk = 0; kk < kPipeBK; ++kk) {
+      float a[8];
+      if (AT) {
+        const float4 a0 = *reinterpret_cast<const float4 *>(As + kk * 128 + ty * 4);
+        const float4 a1 = *reinterpret_cast<const float4 *>(As + kk * 128 + ty * 4 + 64);
+        a[0] = a0.x; a[1] = a0.y; a[2] = a0.z; a[3] = a0.w;
+        a[4] = a1.x; a[5] = a1.y; a[6] = a1.z; a[7] = a1.w;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          a[i] = As[(ty * 4 + i) * kPipeALd + kk];
+          a[4 + i] = As[(ty * 4 + 64 + i) * kPipeALd + kk];
+        }
+      }
+      const float4 b0 = *reinterpret_cast<const float4 *>(Bs + kk * 128 + tx * 4);
+      const float4 b1 = *reinterpret_cast<const float4 *>(Bs + kk * 128 + tx * 4 + 64);
+      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[i][c] = fmaf(a[i], b[c], acc[i][c]);
+    }
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int m = m0 + ty * 4 + (i & 3) + (i >> 2) * 64, n = n0 + tx * 4 + (c & 3) + (c >> 2) * 64;
+      if (m < j.M && n < j.N) {
+        float *p = j.C + (long long)m * j.ldc + n;
+        if (nsplit > 1)
+          atomicAdd(p, j.alpha * acc[i][c]);
+        else
+          *p = j.alpha * acc[i][c] + (j.beta == 0.f ? 0.f : j.beta * *p);
+      }
+    }
+}
+
+}  // namespace ispa
