@@ -37,6 +37,13 @@
 //   * At the end of the local group the epilogue reads O_X after PV of that
 //     tile (o_done) and releases it (o_free) before the first history PV
 //     overwrites it.
+#include <functional>
+#include <map>
+#include <mutex>
+#include <queue>
+#include <tuple>
+#include <vector>
+
 #include "internal.h"
 
 namespace ispa {
@@ -55,7 +62,12 @@ constexpr uint32_t kColS = 0, kColO = 256;  // + 128 * query tile
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 
 struct AttnParams {
-  int H, Lq, q_tiles;
+  int H, Lq;
+  // Work items over the B * H (instance, head) slots g = b * H + h, each with
+  // q_tiles 128-query tiles: first the CTAs with two tiles -- pair_base + 1
+  // pairs for slots g < pair_extra, pair_base for the others -- then the CTAs
+  // with one tile for the rest (see choose_pairs).
+  int q_tiles, pair_base, pair_extra, n_pair_items;
   int n_ranges;            // ranges 0..n_ranges-1; the first n_loc_ranges are local
   int n_loc_ranges;
   int r_begin[3], r_end[3];
@@ -276,10 +288,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       *reinterpret_cast<SmemLayout *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   volatile int *abort = &sm.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x % P.q_tiles;  // pair of 128-query tiles
-  const int h = blockIdx.x / P.q_tiles;
-  const int b = blockIdx.y;
-  const int q0 = qt * 2 * kTileQ;
+  // work item: (instance, head, first query tile, one or two tiles)
+  int nx = 2, b, h, q0;
+  {
+    const int pe = P.pair_extra, pb = P.pair_base;
+    int item = blockIdx.x, g, k;
+    if (item < P.n_pair_items) {
+      if (item < pe * (pb + 1)) {
+        g = item / (pb + 1);
+        k = item % (pb + 1);
+      } else {
+        item -= pe * (pb + 1);
+        g = pe + item / pb;
+        k = item % pb;
+      }
+      q0 = 2 * k * kTileQ;
+    } else {
+      nx = 1;
+      item -= P.n_pair_items;
+      const int s_hi = P.q_tiles - 2 * (pb + 1), s_lo = P.q_tiles - 2 * pb;  // singles per slot
+      if (item < pe * s_hi) {
+        g = item / s_hi;
+        k = 2 * (pb + 1) + item % s_hi;
+      } else {
+        item -= pe * s_hi;
+        g = pe + item / s_lo;
+        k = 2 * pb + item % s_lo;
+      }
+      q0 = k * kTileQ;
+    }
+    b = g / P.H;
+    h = g % P.H;
+  }
   const bool has_hist = P.n_tiles > P.n_loc_tiles;
 
   if (threadIdx.x == 0) {
@@ -325,8 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const int x0 = h * kD;
-      mbar_arrive_expect_tx(&sm.q_full, 2 * kTileBytes);
-      for (int x = 0; x < 2; ++x) {
+      mbar_arrive_expect_tx(&sm.q_full, nx * kTileBytes);
+      for (int x = 0; x < nx; ++x) {
         tma_load_3d(sm.q[x], &tq, &sm.q_full, x0, q0 + x * kTileQ, b);
         tma_load_3d(sm.q[x] + kBoxBytes, &tq, &sm.q_full, x0 + 64, q0 + x * kTileQ, b);
       }
@@ -388,29 +428,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                 wait_parity(&sm.k_full[0], 0, P.err, abort, 22);
       if (ok) {
         tc_fence_after();
-        issue_s(0, 0);
-        issue_s(0, 1);
+        for (int x = 0; x < nx; ++x) issue_s(0, x);
         mma_commit(&sm.k_empty[0]);
       }
       for (int j = 0; ok && j < P.n_tiles; ++j) {
         const int sv = j % kStagesV;
         const bool more = j + 1 < P.n_tiles;
         const int sk1 = (j + 1) % kStagesK;
-        for (int x = 0; x < 2 && ok; ++x) {
+        for (int x = 0; x < nx && ok; ++x) {
           ok = wait_parity(&sm.p_full[x], (uint32_t)(j & 1), P.err, abort, 23);
           if (ok && j == P.n_loc_tiles) ok = wait_parity(&sm.o_free[x], 0, P.err, abort, 24);
           if (ok && x == 0) ok = wait_parity(&sm.v_full[sv], (j / kStagesV) & 1, P.err, abort, 25);
           if (!ok) break;
           tc_fence_after();
           issue_pv(j, x);
-          if (x == 1) mma_commit(&sm.v_empty[sv]);
+          if (x == nx - 1) mma_commit(&sm.v_empty[sv]);
           if (more) {
             // K_{j+1} is waited for only after PV_j(x) is queued
             if (x == 0) ok = wait_parity(&sm.k_full[sk1], ((j + 1) / kStagesK) & 1, P.err, abort, 26);
             if (!ok) break;
             tc_fence_after();
             issue_s(j + 1, x);
-            if (x == 1) mma_commit(&sm.k_empty[sk1]);
+            if (x == nx - 1) mma_commit(&sm.k_empty[sk1]);
           }
         }
       }
@@ -424,6 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // ------------------------------------------------------------ softmax + epilogue
     const int x = (warp - 4) >> 2;  // query tile of this warpgroup
+    if (x < nx) {
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // row inside the tile == TMEM lane
     const int qrow = q0 + x * kTileQ + r;
@@ -558,11 +598,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&sm.o_free[x]);
       }
     }
+    }  // x < nx
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+// Splits the T query tiles of each of the `slots` (instance, head) pairs into
+// CTAs of two tiles (best use of each K/V tile) and of one tile.  The two-tile
+// CTAs are numbered first and the hardware dispatches CTAs roughly in order,
+// so the one-tile CTAs fill the last wave.  The number of two-tile CTAs is
+// chosen by simulating that greedy dispatch on n_sm SMs with a one-tile CTA
+// costing kSingleCost of a two-tile one; results are cached per shape.
+void choose_pairs(int T, int slots, int n_sm, int *pair_base, int *pair_extra) {
+  constexpr double kSingleCost = 0.67;  // measured ratio of one-tile to two-tile CTA time
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int>, std::pair<int, int>> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_tuple(T, slots, n_sm);
+  auto hit = cache.find(key);
+  if (hit == cache.end()) {
+    const long long max_pairs = (long long)slots * (T / 2);
+    const long long tiles = (long long)slots * T;
+    double best = 1e300;
+    long long best_n = max_pairs;
+    for (long long n = max_pairs; n >= 0; --n) {
+      std::priority_queue<double, std::vector<double>, std::greater<double>> q;
+      for (int i = 0; i < n_sm; ++i) q.push(0.0);
+      double end = 0.0;
+      const long long n_single = tiles - 2 * n;
+      for (long long i = 0; i < n + n_single; ++i) {
+        const double t1 = q.top() + (i < n ? 1.0 : kSingleCost);
+        q.pop();
+        end = t1 > end ? t1 : end;
+        q.push(t1);
+      }
+      if (end < best - 1e-9) {
+        best = end;
+        best_n = n;
+      }
+      if (n + n_sm < best_n) break;  // far fewer pairs than the best only adds singles
+    }
+    hit = cache.emplace(key, std::make_pair((int)(best_n / slots), (int)(best_n % slots))).first;
+  }
+  *pair_base = hit->second.first;
+  *pair_extra = hit->second.second;
 }
 
 template <typename TO>
@@ -588,7 +670,7 @@ ispa_status launch_typed(const CUtensorMap &tq, const CUtensorMap &tk, const CUt
                   fa[0].numRegs, fa[1].numRegs, kMinLaunchRegs);
     configured_device = dev;
   }
-  dim3 grid(P.q_tiles * P.H, B);
+  dim3 grid(B * P.H * P.q_tiles - P.n_pair_items);  // every pair CTA stands for two tiles
   attn_tc_kernel<TO><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, P);
   note_launch();
   return cuda_status(cudaGetLastError(), "tcgen05 attention launch");
@@ -652,7 +734,9 @@ ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float 
   if ((st = map3d_16(&tv, v16, D, g.Lkv, d.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16)) != ISPA_OK) return st;
   P.H = d.H;
   P.Lq = g.Lq;
-  P.q_tiles = (g.Lq + 2 * kTileQ - 1) / (2 * kTileQ);  // pairs of query tiles
+  P.q_tiles = (g.Lq + kTileQ - 1) / kTileQ;
+  choose_pairs(P.q_tiles, d.B * d.H, sm_count(), &P.pair_base, &P.pair_extra);
+  P.n_pair_items = d.B * d.H * P.pair_base + P.pair_extra;
   P.n_ranges = 0;
   P.n_loc_tiles = 0;
   for (int r = 0; r < g.n_loc; ++r) {
