@@ -126,10 +126,15 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=subprocess.PIPE,
+                                          "--format=csv,noheader,nounits", "-lms", "50"], stdout=subprocess.PIPE,
                                          stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            # the timed region starts only once the sampler is running
+            deadline = time.time() + 5.0
+            while not self.lines and time.time() < deadline and self.proc.poll() is None:
+                time.sleep(0.01)
+            self.lines.clear()
         except OSError:
             self.proc = None
         return self
@@ -165,6 +170,33 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+# DRAM traffic of the attention kernel (dram__bytes_read.sum + dram__bytes_write.sum
+# of one launch on this workload, from an ncu capture) is recorded in profiles/
+# with the SHA-256 of the kernel source it was measured on; once the source
+# differs the figure no longer describes the kernel and the line reports null.
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_tc_traffic.json")
+KERNEL_SOURCES = [os.path.join(ROOT, "kv_cache_compression_two_b200", "csrc", f) for f in ("attn_tc.cu", "common.cuh")]
+
+
+def kernel_source_digest():
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic():
+    try:
+        rec = json.load(open(TRAFFIC_FILE))
+    except (OSError, ValueError):
+        return None
+    if rec.get("workload") != WORKLOAD.name or rec.get("kernel_source_sha256") != kernel_source_digest():
+        return None
+    return rec.get("dram_bytes_per_launch")
 
 
 # ---------------------------------------------------------------------------
@@ -438,7 +470,7 @@ def run_attn_only(args):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-rows", type=int, default=32, help="query rows of the oracle sample (0: skip it)")
@@ -501,7 +533,7 @@ def main(argv=None):
                 "step_gflop": work["total"] / 1e9},
             "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (two-group attention + fused merge)",
                          "achieved": achieved, "peak": peak, "peak_source": peak_src, "unit": "TFLOP/s",
-                         "frac": achieved / peak, "traffic": None},
+                         "frac": achieved / peak, "traffic": measured_traffic()},
             "gpu_launches": r["launches"],
             "clocks": r["clocks"],
             "e2e": {"value": world * work["total"] / (r["e2e_ms"] * 1e-3) / 1e12, "unit": "TFLOP/s",
