@@ -436,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool more = j + 1 < P.n_tiles;
         const int sk1 = (j + 1) % kStagesK;
         for (int x = 0; x < nx && ok; ++x) {
-          ok = wait_parity(&sm.p_full[x], (uint32_t)(j & 1), P.err, abort, 23);
+          ok = wait_parity_spin(&sm.p_full[x], (uint32_t)(j & 1), P.err, abort, 23);
           if (ok && j == P.n_loc_tiles) ok = wait_parity(&sm.o_free[x], 0, P.err, abort, 24);
           if (ok && x == 0) ok = wait_parity(&sm.v_full[sv], (j / kStagesV) & 1, P.err, abort, 25);
           if (!ok) break;
@@ -481,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool grp_first = (j == 0) || (j == P.n_loc_tiles);
       const bool grp_last = (j == P.n_loc_tiles - 1) || (j == P.n_tiles - 1);
       const int n_valid = it.valid(P);
-      bool ok = wait_parity(&sm.s_full[x], (uint32_t)(j & 1), P.err, abort, 31);
+      bool ok = wait_parity_spin(&sm.s_full[x], (uint32_t)(j & 1), P.err, abort, 31);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       uint32_t sr[4][32];  // S row of this thread (fp32 bits), straight from TMEM

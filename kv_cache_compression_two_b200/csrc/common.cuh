@@ -78,6 +78,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-suspending probe of the phase (mbarrier.test_wait): the thread keeps its
+// issue slot instead of being parked, so it resumes within a few cycles of
+// the phase completing.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase of `bar` with the given parity to complete.  Returns
 // false (after setting the error word and *abort) when the time limit passes,
 // or as soon as another thread of the CTA has set *abort.
@@ -88,6 +103,25 @@ __device__ __forceinline__ bool wait_parity(uint64_t *bar, uint32_t parity, cons
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63u) == 0) {
+      if (*abort) return false;
+      if (globaltimer() - t0 > (unsigned long long)e.limit_ns) {
+        report_error(e, ISPA_ERR_TIMEOUT, site);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// The same bounded wait with non-suspending probes, for the short hand-offs on
+// a kernel's critical path where the wake-up delay of a parked thread shows.
+__device__ __forceinline__ bool wait_parity_spin(uint64_t *bar, uint32_t parity, const DevErr &e,
+                                                 volatile int *abort, int site) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((i & 255u) == 0) {
       if (*abort) return false;
       if (globaltimer() - t0 > (unsigned long long)e.limit_ns) {
         report_error(e, ISPA_ERR_TIMEOUT, site);
