@@ -1,73 +1,58 @@
 // attn_tc.cu -- two-group attention on tcgen05 tensor cores (bf16 in, fp32 accumulate, d = 128).
 //
-// One CTA computes two 128-query tiles (A and B, 256 queries) of one head of
-// one instance and walks the KV tiles of the local group (sink range, then
-// current range) followed by the history group.  Both query tiles share every
-// K/V tile, which halves the operand traffic from L2 per FLOP -- the limit of a
-// single-tile design on this part.  Each group keeps its own online-softmax
-// state; at the end of a group the normalised output and its log-sum-exp are
-// written, and after the history group the optional fused merge combines both
-// groups by their LSE.
+// One CTA computes one 128-query tile of one head of one instance and walks the
+// KV tiles of the local group (sink range, then current range) followed by the
+// history group.  Each group keeps its own online-softmax state; at the end of
+// a group the normalised output and its log-sum-exp are written, and after the
+// history group the optional fused merge combines both groups by their LSE.
 //
-// Warp roles (384 threads, one CTA per SM; setmaxnreg moves registers from the
-// control warpgroup, 64 per thread, to the softmax warpgroups, 216 per thread):
-//   warp 0      TMA producer: Q_A and Q_B once, then K and V tiles (128 keys x
-//               128 dims) through two-stage rings with separate K and V barriers.
-//   warp 1      TMEM allocator and MMA issuer, per KV tile j:
-//                 PV_{j-1}(A), S_j(A), PV_{j-1}(B), S_j(B)
-//               with S_j(X) = Q_X K_j^T (bf16, operands in shared memory) and
-//               PV_j(X): O_X += P_j(X) V_j (fp16 P read from TMEM as operand A,
-//               fp16 V from shared memory), so the softmax of one query tile
-//               overlaps the MMAs of the other.
-//   warps 2-3   idle (they complete the control warpgroup).
-//   warps 4-7   softmax / correction / epilogue of query tile A, one row per
-//   warps 8-11  thread (TMEM lane = row); the same for query tile B.
+// Warp roles (256 threads, one CTA per SM):
+//   warps 0, 2  TMA producers of the K and of the V tiles (128 keys x 128
+//               dims), each through a three-stage ring with full/empty barriers.
+//   warp 1      TMEM allocator and MMA issuer.  S_j = Q K_j^T (bf16; Q from
+//               tensor memory, K from shared memory) into S buffer j % 2, and
+//               PV_j: O += P_j V_j (fp16 P from tensor memory, fp16 V from shared
+//               memory).  Order: S_0, S_1, then per tile j: PV_j, S_{j+2}.
+//   warp 3      idle.
+//   warps 4-7   Q into tensor memory once; then per tile the softmax (one row
+//               per thread, TMEM lane = row), the correction of O when the
+//               running maximum grows, and the group epilogues.
 //
-// TMEM columns: S_A [0,128) S_B [128,256) O_A [256,384) O_B [384,512).  P_j(X)
-// is written as packed fp16 into columns [0,64) of S_X after the softmax has
-// read S_j(X); tcgen05.mma operations issued by one thread execute in order,
-// so PV_j(X) has read P before S_{j+1}(X) overwrites the columns.
+// TMEM columns: O [0,128), S buffers [128,256) and [256,384), Q [384,448)
+// (bf16 pairs).  P_j is written as packed fp16 into the first 64 columns of
+// the buffer that held S_j.  Because S is double-buffered, S_{j+1} is already
+// computed while the softmax works on S_j, so the softmax runs back to back
+// and the tensor pipe works on PV_j and S_{j+2} meanwhile.
 //
-// Ordering argument:
-//   * S_{j+1}(X) is issued after the softmax published P_j(X), i.e. after it
-//     finished its tcgen05.ld of S_j(X).
-//   * S_j(X) is issued after PV_{j-1}(X); its commit (s_full) therefore also
-//     covers PV_{j-1}(X), so while the softmax of tile j runs no MMA touches
-//     O_X and it may rescale O_X directly; PV_j(X) waits for P_j(X).
-//   * At the end of the local group the epilogue reads O_X after PV of that
-//     tile (o_done) and releases it (o_free) before the first history PV
-//     overwrites it.
-#include <functional>
-#include <map>
-#include <mutex>
-#include <queue>
-#include <tuple>
-#include <vector>
-
+// Ordering argument (tcgen05.mma operations issued by one thread execute in
+// order, and a commit fires once all earlier operations have completed):
+//   * S_{j+2} reuses the buffer of S_j / P_j: it is issued after PV_j (which
+//     reads P_j) and after P_j was published, i.e. after the softmax finished
+//     reading S_j.
+//   * When the softmax of tile j starts (S_j complete), PV_{j-2} has completed
+//     (S_j was issued after it); PV_{j-1} may still run, so a correction of O
+//     first waits for PV_{j-1} (o_done); PV_j itself waits for P_j.
+//   * At the end of the local group the epilogue reads O after PV of that tile
+//     (o_done) and releases it (o_free) before the first history PV, which
+//     starts O afresh, is issued.
 #include "internal.h"
 
 namespace ispa {
 
 namespace {
 
-constexpr int kThreads = 384;  // control warpgroup (producer, MMA, 2 idle) + one softmax warpgroup per query tile
-constexpr int kRegsControl = 64, kRegsSoftmax = 216;
-constexpr int kMinLaunchRegs = (128 * kRegsControl + 256 * kRegsSoftmax + kThreads - 1) / kThreads;
+constexpr int kThreads = 256;  // warps 0-3: K producer, MMA issuer, V producer, idle; warps 4-7: softmax
 constexpr int kTileQ = 128, kTileK = 128, kD = 128;
 constexpr int kBoxBytes = 128 * 128;          // 128 rows x 64 bf16
 constexpr int kTileBytes = 2 * kBoxBytes;     // 128 rows x 128 bf16
-constexpr int kStagesK = 3, kStagesV = 2;  // K is needed one MMA step earlier than V
+constexpr int kStagesK = 3, kStagesV = 3;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColO = 256;  // + 128 * query tile
+constexpr uint32_t kColO = 0, kColS = 128, kColQ = 384;  // S buffer b at kColS + 128 b
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 
 struct AttnParams {
   int H, Lq;
-  // Work items over the B * H (instance, head) slots g = b * H + h, each with
-  // q_tiles 128-query tiles: first the CTAs with two tiles -- pair_base + 1
-  // pairs for slots g < pair_extra, pair_base for the others -- then the CTAs
-  // with one tile for the rest (see choose_pairs).
-  int q_tiles, pair_base, pair_extra, n_pair_items;
+  int q_tiles;             // 128-query tiles per (instance, head); CTA x: slot x / q_tiles, tile x % q_tiles
   int n_ranges;            // ranges 0..n_ranges-1; the first n_loc_ranges are local
   int n_loc_ranges;
   int r_begin[3], r_end[3];
@@ -174,13 +159,15 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 }
 
 struct SmemLayout {
-  uint8_t q[2][kTileBytes];
   uint8_t k[kStagesK][kTileBytes];
   uint8_t v[kStagesV][kTileBytes];
-  uint64_t q_full;
   uint64_t k_full[kStagesK], k_empty[kStagesK];
   uint64_t v_full[kStagesV], v_empty[kStagesV];
-  uint64_t s_full[2], p_full[2], o_done[2], o_free[2];  // per query tile
+  uint64_t q_ready;   // Q is in tensor memory (128 arrivals)
+  uint64_t s_full[2]; // S_j complete in buffer j % 2
+  uint64_t p_full[2]; // P_j written into buffer j % 2 (128 arrivals)
+  uint64_t o_done;    // one phase per PV_j
+  uint64_t o_free;    // the local-group epilogue has read O (128 arrivals)
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -281,49 +268,19 @@ __device__ __forceinline__ void load_row32<__nv_bfloat16>(const __nv_bfloat16 *s
 
 template <typename TO>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                   const __grid_constant__ CUtensorMap tv, AttnParams P) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                   const __nv_bfloat16 *__restrict__ q, AttnParams P) {
   extern __shared__ uint8_t smem_raw[];
   SmemLayout &sm =
       *reinterpret_cast<SmemLayout *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   volatile int *abort = &sm.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // work item: (instance, head, first query tile, one or two tiles)
-  int nx = 2, b, h, q0;
-  {
-    const int pe = P.pair_extra, pb = P.pair_base;
-    int item = blockIdx.x, g, k;
-    if (item < P.n_pair_items) {
-      if (item < pe * (pb + 1)) {
-        g = item / (pb + 1);
-        k = item % (pb + 1);
-      } else {
-        item -= pe * (pb + 1);
-        g = pe + item / pb;
-        k = item % pb;
-      }
-      q0 = 2 * k * kTileQ;
-    } else {
-      nx = 1;
-      item -= P.n_pair_items;
-      const int s_hi = P.q_tiles - 2 * (pb + 1), s_lo = P.q_tiles - 2 * pb;  // singles per slot
-      if (item < pe * s_hi) {
-        g = item / s_hi;
-        k = 2 * (pb + 1) + item % s_hi;
-      } else {
-        item -= pe * s_hi;
-        g = pe + item / s_lo;
-        k = 2 * pb + item % s_lo;
-      }
-      q0 = k * kTileQ;
-    }
-    b = g / P.H;
-    h = g % P.H;
-  }
+  const int slot = blockIdx.x / P.q_tiles;  // (instance, head) = b * H + h
+  const int b = slot / P.H, h = slot % P.H;
+  const int q0 = (blockIdx.x % P.q_tiles) * kTileQ;
   const bool has_hist = P.n_tiles > P.n_loc_tiles;
 
   if (threadIdx.x == 0) {
-    mbar_init(&sm.q_full, 1);
     for (int s = 0; s < kStagesK; ++s) {
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
@@ -332,18 +289,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.v_full[s], 1);
       mbar_init(&sm.v_empty[s], 1);
     }
-    for (int x = 0; x < 2; ++x) {
-      mbar_init(&sm.s_full[x], 1);
-      mbar_init(&sm.p_full[x], 128);
-      mbar_init(&sm.o_done[x], 1);
-      mbar_init(&sm.o_free[x], 128);
+    mbar_init(&sm.q_ready, 128);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.s_full[s], 1);
+      mbar_init(&sm.p_full[s], 128);
     }
+    mbar_init(&sm.o_done, 1);
+    mbar_init(&sm.o_free, 128);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tq);
     tma_prefetch_desc(&tk);
     tma_prefetch_desc(&tv);
   }
@@ -353,104 +310,82 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  // Register split: the control warpgroup (warps 0-3: producer, MMA issuer, two
-  // idle warps) gives registers to the two softmax warpgroups.  The block is
-  // launched with 384 x 168; 128 x kRegsControl + 256 x kRegsSoftmax must not
-  // exceed that (the launcher checks the compiled count before launching).
-  // Each role sits inside the branch that set its register budget, so the
-  // compiler allocates every role against its own limit.
-  if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || warp == 2) {
+    // ------------------------------------------------------------ producers: K (warp 0), V (warp 2)
     if (lane == 0) {
+      const bool is_k = warp == 0;
+      const int n_stages = is_k ? kStagesK : kStagesV;
+      const CUtensorMap *map = is_k ? &tk : &tv;
+      uint64_t *full = is_k ? sm.k_full : sm.v_full;
+      uint64_t *empty = is_k ? sm.k_empty : sm.v_empty;
       const int x0 = h * kD;
-      mbar_arrive_expect_tx(&sm.q_full, nx * kTileBytes);
-      for (int x = 0; x < nx; ++x) {
-        tma_load_3d(sm.q[x], &tq, &sm.q_full, x0, q0 + x * kTileQ, b);
-        tma_load_3d(sm.q[x] + kBoxBytes, &tq, &sm.q_full, x0 + 64, q0 + x * kTileQ, b);
-      }
-      uint32_t k_pend = 0, v_pend = 0, k_ph = 0, v_ph = 0;
+      uint32_t pend = 0, ph_bits = 0;
       TileIter it;
       it.start(P);
       for (int j = 0; j < P.n_tiles; ++j, it.next(P)) {
-        const int sk = j % kStagesK, sv = j % kStagesV;
-        const uint32_t phk = (j / kStagesK) & 1, phv = (j / kStagesV) & 1;
-        if (!wait_parity(&sm.k_empty[sk], phk ^ 1, P.err, abort, 11)) break;
-        mbar_arrive_expect_tx(&sm.k_full[sk], kTileBytes);
-        tma_load_3d(sm.k[sk], &tk, &sm.k_full[sk], x0, it.t0, b);
-        tma_load_3d(sm.k[sk] + kBoxBytes, &tk, &sm.k_full[sk], x0 + 64, it.t0, b);
-        k_pend |= 1u << sk;
-        k_ph = (k_ph & ~(1u << sk)) | (phk << sk);
-        if (!wait_parity(&sm.v_empty[sv], phv ^ 1, P.err, abort, 12)) break;
-        mbar_arrive_expect_tx(&sm.v_full[sv], kTileBytes);
-        tma_load_3d(sm.v[sv], &tv, &sm.v_full[sv], x0, it.t0, b);
-        tma_load_3d(sm.v[sv] + kBoxBytes, &tv, &sm.v_full[sv], x0 + 64, it.t0, b);
-        v_pend |= 1u << sv;
-        v_ph = (v_ph & ~(1u << sv)) | (phv << sv);
+        const int st = j % n_stages;
+        const uint32_t ph = (j / n_stages) & 1;
+        if (!wait_parity(&empty[st], ph ^ 1, P.err, abort, is_k ? 11 : 12)) break;
+        uint8_t *dst = is_k ? sm.k[st] : sm.v[st];
+        mbar_arrive_expect_tx(&full[st], kTileBytes);
+        tma_load_3d(dst, map, &full[st], x0, it.t0, b);
+        tma_load_3d(dst + kBoxBytes, map, &full[st], x0 + 64, it.t0, b);
+        pend |= 1u << st;
+        ph_bits = (ph_bits & ~(1u << st)) | (ph << st);
       }
       if (*abort) {  // let copies in flight land before the CTA exits
-        wait_parity_drain(&sm.q_full, 0, P.err);
-        for (int s = 0; s < kStagesK; ++s)
-          if (k_pend & (1u << s)) wait_parity_drain(&sm.k_full[s], (k_ph >> s) & 1, P.err);
-        for (int s = 0; s < kStagesV; ++s)
-          if (v_pend & (1u << s)) wait_parity_drain(&sm.v_full[s], (v_ph >> s) & 1, P.err);
+        for (int st = 0; st < n_stages; ++st)
+          if (pend & (1u << st)) wait_parity_drain(&full[st], (ph_bits >> st) & 1, P.err);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc_qk = make_idesc(128, 128, 1, 0, 0);  // bf16 Q x bf16 K, both K-major
+      const uint32_t idesc_qk = make_idesc(128, 128, 1, 0, 0);  // bf16 Q (TMEM) x bf16 K (K-major)
       const uint32_t idesc_pv = make_idesc(128, 128, 0, 0, 1);  // fp16 P (TMEM) x fp16 V (MN-major)
-      auto issue_s = [&](int j, int x) {  // S_j(x) = Q_x K_j^T
-        const uint32_t q_addr = smem_u32(sm.q[x]);
+      auto issue_s = [&](int j) {  // S_j = Q K_j^T into buffer j & 1
         const uint32_t k_addr = smem_u32(sm.k[j % kStagesK]);
-        const uint32_t d_s = tmem + kColS + (uint32_t)x * 128;
+        const uint32_t d_s = tmem + kColS + (uint32_t)(j & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (uint32_t)(kk >> 2) * kBoxBytes + (uint32_t)(kk & 3) * 32;
-          mma_ss(d_s, smem_desc_sw128(q_addr + off, 16, 1024), smem_desc_sw128(k_addr + off, 16, 1024), idesc_qk,
-                 kk > 0 ? 1u : 0u, 0);
+          mma_ts(d_s, tmem + kColQ + (uint32_t)kk * 8, smem_desc_sw128(k_addr + off, 16, 1024), idesc_qk,
+                 kk > 0 ? 1u : 0u);
         }
-        mma_commit(&sm.s_full[x]);
+        mma_commit(&sm.s_full[j & 1]);
+        mma_commit(&sm.k_empty[j % kStagesK]);
       };
-      auto issue_pv = [&](int j, int x) {  // O_x (+)= P_j(x) V_j, P in the first 64 columns of S_x
+      auto issue_pv = [&](int j) {  // O (+)= P_j V_j, P_j in the first 64 columns of buffer j & 1
         const bool first = (j == 0) || (j == P.n_loc_tiles);
         const uint32_t v_addr = smem_u32(sm.v[j % kStagesV]);
-        const uint32_t a_p = tmem + kColS + (uint32_t)x * 128;
+        const uint32_t a_p = tmem + kColS + (uint32_t)(j & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < kTileK / 16; ++kk)
-          mma_ts(tmem + kColO + (uint32_t)x * 128, a_p + kk * 8,
-                 smem_desc_sw128(v_addr + kk * 2048, kBoxBytes, 1024), idesc_pv, (first && kk == 0) ? 0u : 1u);
-        mma_commit(&sm.o_done[x]);
+          mma_ts(tmem + kColO, a_p + kk * 8, smem_desc_sw128(v_addr + kk * 2048, kBoxBytes, 1024), idesc_pv,
+                 (first && kk == 0) ? 0u : 1u);
+        mma_commit(&sm.o_done);
+        mma_commit(&sm.v_empty[j % kStagesV]);
       };
-      bool ok = wait_parity(&sm.q_full, 0, P.err, abort, 21) &&
-                wait_parity(&sm.k_full[0], 0, P.err, abort, 22);
-      if (ok) {
+      bool ok = wait_parity(&sm.q_ready, 0, P.err, abort, 20);
+      for (int j = 0; ok && j < 2 && j < P.n_tiles; ++j) {
+        ok = wait_parity(&sm.k_full[j % kStagesK], (j / kStagesK) & 1, P.err, abort, 21);
+        if (!ok) break;
         tc_fence_after();
-        for (int x = 0; x < nx; ++x) issue_s(0, x);
-        mma_commit(&sm.k_empty[0]);
+        issue_s(j);
       }
       for (int j = 0; ok && j < P.n_tiles; ++j) {
-        const int sv = j % kStagesV;
-        const bool more = j + 1 < P.n_tiles;
-        const int sk1 = (j + 1) % kStagesK;
-        for (int x = 0; x < nx && ok; ++x) {
-          ok = wait_parity_spin(&sm.p_full[x], (uint32_t)(j & 1), P.err, abort, 23);
-          if (ok && j == P.n_loc_tiles) ok = wait_parity(&sm.o_free[x], 0, P.err, abort, 24);
-          if (ok && x == 0) ok = wait_parity(&sm.v_full[sv], (j / kStagesV) & 1, P.err, abort, 25);
+        ok = wait_parity_spin(&sm.p_full[j & 1], (uint32_t)(j >> 1) & 1, P.err, abort, 23);
+        if (ok && j == P.n_loc_tiles) ok = wait_parity(&sm.o_free, 0, P.err, abort, 24);
+        if (ok) ok = wait_parity(&sm.v_full[j % kStagesV], (j / kStagesV) & 1, P.err, abort, 25);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(j);
+        const int jn = j + 2;  // S runs two tiles ahead, into the buffer PV_j has just read
+        if (jn < P.n_tiles) {
+          ok = wait_parity(&sm.k_full[jn % kStagesK], (jn / kStagesK) & 1, P.err, abort, 26);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(j, x);
-          if (x == nx - 1) mma_commit(&sm.v_empty[sv]);
-          if (more) {
-            // K_{j+1} is waited for only after PV_j(x) is queued
-            if (x == 0) ok = wait_parity(&sm.k_full[sk1], ((j + 1) / kStagesK) & 1, P.err, abort, 26);
-            if (!ok) break;
-            tc_fence_after();
-            issue_s(j + 1, x);
-            if (x == nx - 1) mma_commit(&sm.k_empty[sk1]);
-          }
+          issue_s(jn);
         }
       }
       if (!ok) {
@@ -458,22 +393,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         wait_parity_drain(&sm.drain, 0, P.err);
       }
     }
-  }
-  } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+  } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
-    const int x = (warp - 4) >> 2;  // query tile of this warpgroup
-    if (x < nx) {
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // row inside the tile == TMEM lane
-    const int qrow = q0 + x * kTileQ + r;
+    const int qrow = q0 + r;
     const bool row_ok = qrow < P.Lq;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t col_s = kColS + (uint32_t)x * 128, col_o = kColO + (uint32_t)x * 128;
     const long long head_row = ((long long)b * P.Lq + (row_ok ? qrow : 0)) * P.H + h;
     TO *o_loc = reinterpret_cast<TO *>(P.o_loc) + head_row * kD;
     TO *o_hist = P.o_hist ? reinterpret_cast<TO *>(P.o_hist) + head_row * kD : nullptr;
     TO *o_full = P.o_full ? reinterpret_cast<TO *>(P.o_full) + head_row * kD : nullptr;
+    // This row of Q into TMEM as the A operand of S = Q K^T: column c holds
+    // elements 2c and 2c + 1 (zeros past the end of the sequence).
+    {
+      const uint4 *src = reinterpret_cast<const uint4 *>(q + head_row * kD);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t w[16];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint4 v = row_ok ? __ldg(src + c * 4 + u) : make_uint4(0u, 0u, 0u, 0u);
+          w[4 * u] = v.x;
+          w[4 * u + 1] = v.y;
+          w[4 * u + 2] = v.z;
+          w[4 * u + 3] = v.w;
+        }
+        tmem_st16(lane_base + kColQ + c * 16, w);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sm.q_ready);
+    }
     float m_ref = 0.f, l = 0.f, L_loc = -INFINITY;
     TileIter it;
     it.start(P);
@@ -481,7 +432,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool grp_first = (j == 0) || (j == P.n_loc_tiles);
       const bool grp_last = (j == P.n_loc_tiles - 1) || (j == P.n_tiles - 1);
       const int n_valid = it.valid(P);
-      bool ok = wait_parity_spin(&sm.s_full[x], (uint32_t)(j & 1), P.err, abort, 31);
+      const uint32_t col_s = kColS + (uint32_t)(j & 1) * 128;
+      bool ok = wait_parity_spin(&sm.s_full[j & 1], (uint32_t)(j >> 1) & 1, P.err, abort, 31);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       uint32_t sr[4][32];  // S row of this thread (fp32 bits), straight from TMEM
@@ -505,7 +457,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_ref = mt;
         l = 0.f;
       } else if (__any_sync(0xffffffffu, mt > m_ref + kRescaleThreshold)) {
-        // O_x is quiescent here (PV_{j-1}(x) completed before S_j(x)); PV_j(x) waits for P_j(x).
+        // O may still be accumulating PV_{j-1}; it is final once that PV lands (PV_j
+        // waits for P_j, which this warpgroup has not published yet).
+        ok = wait_parity(&sm.o_done, (uint32_t)(j - 1) & 1, P.err, abort, 32);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
         const float m_new = fmaxf(m_ref, mt);
         const float f = ex2(m_ref - m_new);
         m_ref = m_new;
@@ -513,15 +469,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
-          tmem_ld32(lane_base + col_o + c * 32, o);
+          tmem_ld32(lane_base + kColO + c * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * f);
-          tmem_st16(lane_base + col_o + c * 32, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
-          tmem_st16(lane_base + col_o + c * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
+          tmem_st16(lane_base + kColO + c * 32, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
+          tmem_st16(lane_base + kColO + c * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
         }
       }
-      // P = exp2(s * scale * log2e - m_ref) <= 2^8, packed to fp16 pairs into columns [0, 64) of S_x.
+      // P = exp2(s * scale * log2e - m_ref) <= 2^8, packed to fp16 pairs into columns [0, 64) of the buffer.
       const float2 sc2 = make_float2(P.scale_log2, P.scale_log2), nm2 = make_float2(-m_ref, -m_ref);
       float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
@@ -539,12 +495,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
       tc_fence_before();
-      mbar_arrive(&sm.p_full[x]);
+      mbar_arrive(&sm.p_full[j & 1]);
 
       if (!grp_last) continue;
-      // ---- end of a group: O_x is final once PV_j(x) has landed (o_done counts the
-      // PVs of this tile; PV_{j-1}(x) completed before S_j(x), so the wait is exact).
-      ok = wait_parity(&sm.o_done[x], (uint32_t)(j & 1), P.err, abort, 33);
+      // ---- end of a group: O is final once PV_j has landed (PV_{j+1} needs P_{j+1},
+      // which this warpgroup has not produced, so the wait cannot alias).
+      ok = wait_parity(&sm.o_done, (uint32_t)j & 1, P.err, abort, 33);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const bool is_loc = j < P.n_loc_tiles;
@@ -567,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t raw[32];
-        tmem_ld32(lane_base + col_o + c * 32, raw);
+        tmem_ld32(lane_base + kColO + c * 32, raw);
         tmem_wait_ld();
         float xo[32];
 #pragma unroll
@@ -595,10 +551,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (is_loc && has_hist) {
         tc_fence_before();
-        mbar_arrive(&sm.o_free[x]);
+        mbar_arrive(&sm.o_free);
       }
     }
-    }  // x < nx
   }
   tc_fence_before();
   __syncthreads();
@@ -606,49 +561,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
-// Splits the T query tiles of each of the `slots` (instance, head) pairs into
-// CTAs of two tiles (best use of each K/V tile) and of one tile.  The two-tile
-// CTAs are numbered first and the hardware dispatches CTAs roughly in order,
-// so the one-tile CTAs fill the last wave.  The number of two-tile CTAs is
-// chosen by simulating that greedy dispatch on n_sm SMs with a one-tile CTA
-// costing kSingleCost of a two-tile one; results are cached per shape.
-void choose_pairs(int T, int slots, int n_sm, int *pair_base, int *pair_extra) {
-  constexpr double kSingleCost = 0.67;  // measured ratio of one-tile to two-tile CTA time
-  static std::mutex mu;
-  static std::map<std::tuple<int, int, int>, std::pair<int, int>> cache;
-  std::lock_guard<std::mutex> lock(mu);
-  const auto key = std::make_tuple(T, slots, n_sm);
-  auto hit = cache.find(key);
-  if (hit == cache.end()) {
-    const long long max_pairs = (long long)slots * (T / 2);
-    const long long tiles = (long long)slots * T;
-    double best = 1e300;
-    long long best_n = max_pairs;
-    for (long long n = max_pairs; n >= 0; --n) {
-      std::priority_queue<double, std::vector<double>, std::greater<double>> q;
-      for (int i = 0; i < n_sm; ++i) q.push(0.0);
-      double end = 0.0;
-      const long long n_single = tiles - 2 * n;
-      for (long long i = 0; i < n + n_single; ++i) {
-        const double t1 = q.top() + (i < n ? 1.0 : kSingleCost);
-        q.pop();
-        end = t1 > end ? t1 : end;
-        q.push(t1);
-      }
-      if (end < best - 1e-9) {
-        best = end;
-        best_n = n;
-      }
-      if (n + n_sm < best_n) break;  // far fewer pairs than the best only adds singles
-    }
-    hit = cache.emplace(key, std::make_pair((int)(best_n / slots), (int)(best_n % slots))).first;
-  }
-  *pair_base = hit->second.first;
-  *pair_extra = hit->second.second;
-}
-
 template <typename TO>
-ispa_status launch_typed(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv, const AttnParams &P,
+ispa_status launch_typed(const CUtensorMap &tk, const CUtensorMap &tv, const __nv_bfloat16 *q, const AttnParams &P,
                          int B, cudaStream_t s) {
   static thread_local int configured_device = -1;
   int dev = 0;
@@ -659,19 +573,10 @@ ispa_status launch_typed(const CUtensorMap &tq, const CUtensorMap &tk, const CUt
       e = cudaFuncSetAttribute(attn_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                kSmemBytes);
     if (e != cudaSuccess) return cuda_status(e, "attention smem attribute");
-    // setmaxnreg.inc waits for registers the block does not have if the launch
-    // allocation is smaller than the split; refuse to launch in that case.
-    cudaFuncAttributes fa[2];
-    e = cudaFuncGetAttributes(&fa[0], attn_tc_kernel<float>);
-    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa[1], attn_tc_kernel<__nv_bfloat16>);
-    if (e != cudaSuccess) return cuda_status(e, "attention attributes");
-    if (fa[0].numRegs < kMinLaunchRegs || fa[1].numRegs < kMinLaunchRegs)
-      return fail(ISPA_ERR_CUDA, "attention kernel compiled with %d/%d registers, the register split needs %d",
-                  fa[0].numRegs, fa[1].numRegs, kMinLaunchRegs);
     configured_device = dev;
   }
-  dim3 grid(B * P.H * P.q_tiles - P.n_pair_items);  // every pair CTA stands for two tiles
-  attn_tc_kernel<TO><<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, P);
+  dim3 grid(B * P.H * P.q_tiles);
+  attn_tc_kernel<TO><<<grid, kThreads, kSmemBytes, s>>>(tk, tv, q, P);
   note_launch();
   return cuda_status(cudaGetLastError(), "tcgen05 attention launch");
 }
@@ -728,15 +633,12 @@ ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float 
   if ((st = cuda_status(cudaGetLastError(), "V conversion launch")) != ISPA_OK) return st;
   P.v_unscale = v_unscale;
 
-  CUtensorMap tq, tk, tv;
-  if ((st = map3d_16(&tq, q, D, g.Lq, d.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) != ISPA_OK) return st;
+  CUtensorMap tk, tv;
   if ((st = map3d_16(&tk, k, D, g.Lkv, d.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) != ISPA_OK) return st;
   if ((st = map3d_16(&tv, v16, D, g.Lkv, d.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16)) != ISPA_OK) return st;
   P.H = d.H;
   P.Lq = g.Lq;
   P.q_tiles = (g.Lq + kTileQ - 1) / kTileQ;
-  choose_pairs(P.q_tiles, d.B * d.H, sm_count(), &P.pair_base, &P.pair_extra);
-  P.n_pair_items = d.B * d.H * P.pair_base + P.pair_extra;
   P.n_ranges = 0;
   P.n_loc_tiles = 0;
   for (int r = 0; r < g.n_loc; ++r) {
@@ -760,8 +662,9 @@ ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float 
   P.l_loc = l_loc;
   P.l_hist = l_hist;
   P.l_full = l_full;
-  if (d.out_dtype == ISPA_F32) return launch_typed<float>(tq, tk, tv, P, d.B, s);
-  return launch_typed<__nv_bfloat16>(tq, tk, tv, P, d.B, s);
+  const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(q);
+  if (d.out_dtype == ISPA_F32) return launch_typed<float>(tk, tv, qb, P, d.B, s);
+  return launch_typed<__nv_bfloat16>(tk, tv, qb, P, d.B, s);
 }
 
 }  // namespace ispa
