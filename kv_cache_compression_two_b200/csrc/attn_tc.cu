@@ -343,25 +343,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_qk = make_idesc(128, 128, 1, 0, 0);  // bf16 Q (TMEM) x bf16 K (K-major)
       const uint32_t idesc_pv = make_idesc(128, 128, 0, 0, 1);  // fp16 P (TMEM) x fp16 V (MN-major)
+      // Descriptors of every ring stage, built once: each MMA then costs the
+      // issuing thread (which shares its scheduler with a softmax warp) only an
+      // add.  The start-address field (bits 0-13, address / 16) does not carry
+      // out for shared-memory offsets below 256 KiB.
+      uint64_t dk[kStagesK], dv[kStagesV];
+#pragma unroll
+      for (int st = 0; st < kStagesK; ++st) dk[st] = smem_desc_sw128(smem_u32(sm.k[st]), 16, 1024);
+#pragma unroll
+      for (int st = 0; st < kStagesV; ++st) dv[st] = smem_desc_sw128(smem_u32(sm.v[st]), kBoxBytes, 1024);
+      auto pick = [](const uint64_t *d, int n, int st) {  // register-resident select of d[st]
+        uint64_t r = d[0];
+#pragma unroll
+        for (int i = 1; i < n; ++i) r = st == i ? d[i] : r;
+        return r;
+      };
       auto issue_s = [&](int j) {  // S_j = Q K_j^T into buffer j & 1
-        const uint32_t k_addr = smem_u32(sm.k[j % kStagesK]);
+        const uint64_t kd = pick(dk, kStagesK, j % kStagesK);
         const uint32_t d_s = tmem + kColS + (uint32_t)(j & 1) * 128;
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (uint32_t)(kk >> 2) * kBoxBytes + (uint32_t)(kk & 3) * 32;
-          mma_ts(d_s, tmem + kColQ + (uint32_t)kk * 8, smem_desc_sw128(k_addr + off, 16, 1024), idesc_qk,
-                 kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < kD / 16; ++kk)
+          mma_ts(d_s, tmem + kColQ + (uint32_t)kk * 8, kd + (uint64_t)(((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4),
+                 idesc_qk, kk > 0 ? 1u : 0u);
         mma_commit(&sm.s_full[j & 1]);
         mma_commit(&sm.k_empty[j % kStagesK]);
       };
       auto issue_pv = [&](int j) {  // O (+)= P_j V_j, P_j in the first 64 columns of buffer j & 1
         const bool first = (j == 0) || (j == P.n_loc_tiles);
-        const uint32_t v_addr = smem_u32(sm.v[j % kStagesV]);
+        const uint64_t vd = pick(dv, kStagesV, j % kStagesV);
         const uint32_t a_p = tmem + kColS + (uint32_t)(j & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < kTileK / 16; ++kk)
-          mma_ts(tmem + kColO, a_p + kk * 8, smem_desc_sw128(v_addr + kk * 2048, kBoxBytes, 1024), idesc_pv,
+          mma_ts(tmem + kColO, a_p + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
                  (first && kk == 0) ? 0u : 1u);
         mma_commit(&sm.o_done);
         mma_commit(&sm.v_empty[j % kStagesV]);
