@@ -177,8 +177,8 @@ __device__ __forceinline__ void store_acc_t(TileT &T, const float acc[4][4]) {
   }
 }
 
-constexpr int kFactorThreads = 288;
-constexpr int kFactorBcast = 8 * 64 + 16;  // floats of the factor routine's broadcast buffers
+constexpr int kFactorThreads = 256;
+constexpr int kFactorBcast = 2 * 8 * NB;  // floats of the factor routine's broadcast buffers (two generations)
 
 // Inverse m (lower triangular) of the Cholesky factor of the symmetric 4 x 4
 // block d (lower triangle read).  Returns the index of the first non-positive
@@ -214,138 +214,126 @@ __device__ __forceinline__ int chol4_inverse(const float d[4][4], float m[4][4])
 // Block forward elimination of [S | I] with Cholesky scaling, four pivots per
 // step: with C the four current pivot columns, D their 4 x 4 diagonal block
 // and M the inverse of D's Cholesky factor, every row r of the left half below
-// the block loses l_r l_c^T in column c (l = C M^T), the four pivot rows of the
-// right half become M times themselves, and every right-half row below them
-// loses l_r times those new rows.  The left half is only needed below and
-// right of the pivots; by symmetry its pivot rows equal its pivot columns.
-// kFactorThreads threads, each owning one 4 x 4 block in registers: thread
-// (I, J) = (t / 16, t % 16) of the first 256 owns block (I, J) of the left
-// half if I >= J and block (J, I) of the right half if I < J; threads 256..271
-// own the diagonal blocks of the right half.  Two barriers per step:
-//   phase A: the owners of the pivot block column form l for their rows, the
-//            owners of the pivot rows of the right half form M times them,
-//            both into shared memory (M was published by the owner of D, who
-//            factored D as soon as its own last update landed);
-//   phase B: every block applies its rank-4 update from those vectors, and the
-//            owner of the next pivot block factors it and publishes its M.
-// Entries that are no longer read (columns left of the pivots, the upper part
-// of the left diagonal blocks) are updated without masks; rows of the right
-// half above the pivots are left alone.  bcast: kFactorBcast floats, 16-byte
-// aligned, distinct from S.
+// the pivots loses l_r l_c^T in column c (l = C M^T), the pivot rows of the
+// right half become bn = M times themselves, and every right-half row below
+// them loses l_r bn.  Only the lower triangle of the left half below and right
+// of the pivots is kept, and the lower triangle of the right half, which ends
+// as L^-1.
+//
+// Ownership: one 4 x 4 block per thread, in registers.  Block column J of the
+// left half (block rows J..15) and block row J of the right half left of the
+// diagonal (block columns 0..J-1) are 16 blocks, the group of J; warp w holds
+// the groups of J = w (lanes 0..15) and J = 15 - w (lanes 16..31), so every
+// warp stays busy until its later group is done.  Lane k of group J owns left
+// block (J + k, J) for k < 16 - J (k = 0: the diagonal block) and right block
+// (J, k - 16 + J) otherwise; the right diagonal block (J, J) is M_J, which
+// lane 0 keeps once pivot J is factored.
+//
+// One barrier per pivot step.  In step P every block still in play applies its
+// rank-4 update from the l and bn of pivot P in shared memory.  Right after its
+// own update, group P + 1 -- whose blocks are then final for pivot P + 1 --
+// factors its diagonal block on lane 0, passes M to the group by shuffles, and
+// writes l (left lanes) and bn (right lanes, which keep bn as their final
+// value) into the other of two buffers for the next step.  bcast: kFactorBcast
+// floats, 16-byte aligned, distinct from S.  kFactorThreads threads.
 __device__ __forceinline__ void factor_invert_tile(const float *S, float *bcast, float *__restrict__ Linv_out,
-                                                   int pivot_base,
-                                   int *flag, const DevErr &err) {
-  const int t = threadIdx.x;
-  bool is_b = false, active = true;
-  int R = 0, Cb = 0;  // first row and first column of the owned block
-  if (t < 256) {
-    const int I = t >> 4, J = t & 15;
-    is_b = I < J;
-    R = 4 * (is_b ? J : I);
-    Cb = 4 * (is_b ? I : J);
-  } else if (t < 272) {
-    is_b = true;
-    R = Cb = 4 * (t - 256);
-  } else {
-    active = false;
-  }
+                                                   int pivot_base, int *flag, const DevErr &err) {
+  const int t = threadIdx.x, w = t >> 5, lane = t & 31;
+  const int J = lane < 16 ? w : 15 - w;  // this lane's group
+  const int k = lane & 15;
+  const bool left = k < 16 - J;
+  const int rb = left ? J + k : J;       // block row of the owned block
+  const int cb = left ? J : k - 16 + J;  // block column
+  const int last = w > 15 - w ? w : 15 - w;  // the warp has work in steps P < last
   float x[4][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      x[i][j] = is_b ? (R + i == Cb + j ? 1.f : 0.f) : (active ? S[(R + i) * NB + Cb + j] : 0.f);
-  float *lbuf = bcast;               // [64 rows][4]: l = C M^T of the pivot block column
-  float *bbuf = bcast + 4 * NB;      // [4 rows][64]: new pivot rows of the right half
-  float *mb = bcast + 8 * NB;        // [4][4]: M of the current pivot block
+  for (int i = 0; i < 4; ++i) {
+    const float4 v = left ? *reinterpret_cast<const float4 *>(S + (4 * rb + i) * NB + 4 * cb)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    x[i][0] = v.x;
+    x[i][1] = v.y;
+    x[i][2] = v.z;
+    x[i][3] = v.w;
+  }
 
-  auto publish_m = [&](int pivot0) {  // factor the pivot block held in x, publish its M
-    float m[4][4];
-    const int bad = chol4_inverse(x, m);
-    if (bad >= 0 && atomicExch(flag, 1) == 0) report_error(err, ISPA_ERR_NOT_SPD, pivot_base + pivot0 + bad + 1);
-#pragma unroll
-    for (int a = 0; a < 4; ++a) *reinterpret_cast<float4 *>(mb + 4 * a) = make_float4(m[a][0], m[a][1], m[a][2], m[a][3]);
-  };
-  if (t == 0) publish_m(0);
-
-  for (int P = 0; P < NB / 4; ++P) {
-    const int p0 = 4 * P;
-    __syncthreads();  // M of this step is visible; the previous step's phase B is done
-    // ---- phase A
-    const bool col_owner = active && !is_b && Cb == p0;
-    const bool row_owner = is_b && R == p0;
-    if (col_owner || row_owner) {
+  // Pivot step Q of group Q; called by the whole warp that holds the group.
+  auto pivot = [&](int Q) {
+    const bool mine = J == Q;
+    if (mine && k == 0) {
       float m[4][4];
+      const int bad = chol4_inverse(x, m);
+      if (bad >= 0 && atomicExch(flag, 1) == 0) report_error(err, ISPA_ERR_NOT_SPD, pivot_base + 4 * Q + bad + 1);
 #pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        const float4 v = *reinterpret_cast<const float4 *>(mb + 4 * a);
-        m[a][0] = v.x;
-        m[a][1] = v.y;
-        m[a][2] = v.z;
-        m[a][3] = v.w;
-      }
-      if (col_owner) {  // l_r = C_r M^T for this block's four rows
+      for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float l[4];
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            float s = 0.f;
-#pragma unroll
-            for (int k = 0; k <= jj; ++k) s = fmaf(x[i][k], m[jj][k], s);
-            l[jj] = s;
-          }
-          *reinterpret_cast<float4 *>(lbuf + (R + i) * 4) = make_float4(l[0], l[1], l[2], l[3]);
-        }
-      } else {  // the pivot rows of the right half: M times them
-        float bn[4][4];
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            float s = 0.f;
-#pragma unroll
-            for (int k = 0; k <= a; ++k) s = fmaf(m[a][k], x[k][jj], s);
-            bn[a][jj] = s;
-          }
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          *reinterpret_cast<float4 *>(bbuf + a * NB + Cb) = make_float4(bn[a][0], bn[a][1], bn[a][2], bn[a][3]);
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj) x[a][jj] = bn[a][jj];
-        }
-      }
+        for (int b = 0; b < 4; ++b) x[a][b] = m[a][b];
     }
-    __syncthreads();
-    // ---- phase B
-    if (active && (!is_b || (R > p0 && Cb <= p0 + 3))) {
-      float lr[4][4], v[4][4];
+    const int src = Q == w ? 0 : 16;
+    float mq[4][4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 a = *reinterpret_cast<const float4 *>(lbuf + (R + i) * 4);
-        lr[i][0] = a.x;
-        lr[i][1] = a.y;
-        lr[i][2] = a.z;
-        lr[i][3] = a.w;
-      }
-      if (!is_b) {  // v[j][a] = l of column Cb + j
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) mq[a][b] = b <= a ? __shfl_sync(0xffffffffu, x[a][b], src) : 0.f;
+    float *lb = bcast + (Q & 1) * 8 * NB, *bb = lb + 4 * NB;
+    if (!mine) return;
+    if (k == 0) {  // the diagonal block of bn is M itself
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+        *reinterpret_cast<float4 *>(bb + a * NB + 4 * Q) = make_float4(x[a][0], x[a][1], x[a][2], x[a][3]);
+    } else if (left) {  // l = C M^T for this block's four rows, component-major
+      float l[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-          const float4 a = *reinterpret_cast<const float4 *>(lbuf + (Cb + jj) * 4);
-          v[jj][0] = a.x;
-          v[jj][1] = a.y;
-          v[jj][2] = a.z;
-          v[jj][3] = a.w;
-        }
-      } else {  // v[j][a] = new pivot row a at column Cb + j
+          float s = 0.f;
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          const float4 b = *reinterpret_cast<const float4 *>(bbuf + a * NB + Cb);
-          v[0][a] = b.x;
-          v[1][a] = b.y;
-          v[2][a] = b.z;
-          v[3][a] = b.w;
+          for (int q = 0; q <= jj; ++q) s = fmaf(x[i][q], mq[jj][q], s);
+          l[i][jj] = s;
         }
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+        *reinterpret_cast<float4 *>(lb + jj * NB + 4 * rb) = make_float4(l[0][jj], l[1][jj], l[2][jj], l[3][jj]);
+    } else {  // right block (Q, cb): bn = M x, its final value
+      float bn[4][4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          float s = 0.f;
+#pragma unroll
+          for (int q = 0; q <= a; ++q) s = fmaf(mq[a][q], x[q][jj], s);
+          bn[a][jj] = s;
+        }
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        *reinterpret_cast<float4 *>(bb + a * NB + 4 * cb) = make_float4(bn[a][0], bn[a][1], bn[a][2], bn[a][3]);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) x[a][jj] = bn[a][jj];
+      }
+    }
+  };
+
+  if (w == 0) pivot(0);
+  for (int P = 0; P < NB / 4 - 1; ++P) {
+    __syncthreads();  // l and bn of pivot P are visible; the buffer written next is no longer read
+    if (P >= last) continue;
+    if (J > P && (left || cb <= P)) {
+      const float *lb = bcast + (P & 1) * 8 * NB;
+      const float *vs = (left ? lb : lb + 4 * NB) + 4 * cb;  // l of column block J, or bn at block column cb
+      float lr[4][4], v[4][4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const float4 c = *reinterpret_cast<const float4 *>(lb + a * NB + 4 * rb);
+        lr[0][a] = c.x;
+        lr[1][a] = c.y;
+        lr[2][a] = c.z;
+        lr[3][a] = c.w;
+        const float4 d = *reinterpret_cast<const float4 *>(vs + a * NB);
+        v[0][a] = d.x;
+        v[1][a] = d.y;
+        v[2][a] = d.z;
+        v[3][a] = d.w;
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i)
@@ -356,17 +344,24 @@ __device__ __forceinline__ void factor_invert_tile(const float *S, float *bcast,
           for (int a = 0; a < 4; ++a) s = fmaf(-lr[i][a], v[jj][a], s);
           x[i][jj] = s;
         }
-      if (!is_b && R == Cb && R == p0 + 4) publish_m(R);  // the next pivot block is final now
     }
+    const int q = P + 1;
+    if (q == w || q == 15 - w) pivot(q);
   }
-  if (is_b) {
+  // row J of L^-1: right blocks, M_J on the diagonal, zeros above it
+  float *o = Linv_out + (4 * J) * NB;
+  if (!left) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      *reinterpret_cast<float4 *>(Linv_out + (R + i) * NB + Cb) = make_float4(x[i][0], x[i][1], x[i][2], x[i][3]);
-  } else if (active && R != Cb) {  // the mirrored block above the diagonal of L^-1 is zero
+      *reinterpret_cast<float4 *>(o + i * NB + 4 * cb) = make_float4(x[i][0], x[i][1], x[i][2], x[i][3]);
+  } else if (k == 0) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      *reinterpret_cast<float4 *>(Linv_out + (Cb + i) * NB + R) = make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4 *>(o + i * NB + 4 * J) = make_float4(x[i][0], x[i][1], x[i][2], x[i][3]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<float4 *>(o + i * NB + 4 * (J + k)) = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 
@@ -390,9 +385,7 @@ __global__ void __launch_bounds__(kFactorThreads) chol_step_kernel(int Dp, int k
   __shared__ __align__(16) TileT sX;
   __shared__ __align__(16) TileT sY;
   __shared__ __align__(16) TileT sL;
-  // threads 0..255 do the tile work; all kFactorThreads factor the next diagonal block
-  const int t = threadIdx.x, ty = (t >> 4) & 15, tx = t & 15;
-  const bool worker = t < 256;
+  const int t = threadIdx.x, ty = t >> 4, tx = t & 15;
   const int lin = blockIdx.x;
   int ii = (int)((sqrtf(8.f * lin + 1.f) - 1.f) * 0.5f);
   while ((ii + 1) * (ii + 2) / 2 <= lin) ++ii;
@@ -403,67 +396,57 @@ __global__ void __launch_bounds__(kFactorThreads) chol_step_kernel(int Dp, int k
   float *tile = M + (long long)i * NB * ld + j * NB;
 
   float aij[4][4];
-  if (worker) {
-    load_tile_t(sX, M + (long long)i * NB * ld + k * NB, ld);
-    if (!diag) load_tile_t(sY, M + (long long)j * NB * ld + k * NB, ld);
-    load_tile_t(sL, Linv + (long long)k * NB * NB, NB);
+  load_tile_t(sX, M + (long long)i * NB * ld + k * NB, ld);
+  if (!diag) load_tile_t(sY, M + (long long)j * NB * ld + k * NB, ld);
+  load_tile_t(sL, Linv + (long long)k * NB * NB, NB);
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const float4 v = *reinterpret_cast<const float4 *>(tile + (long long)(4 * ty + a) * ld + 4 * tx);
-      aij[a][0] = v.x;
-      aij[a][1] = v.y;
-      aij[a][2] = v.z;
-      aij[a][3] = v.w;
-    }
+  for (int a = 0; a < 4; ++a) {
+    const float4 v = *reinterpret_cast<const float4 *>(tile + (long long)(4 * ty + a) * ld + 4 * tx);
+    aij[a][0] = v.x;
+    aij[a][1] = v.y;
+    aij[a][2] = v.z;
+    aij[a][3] = v.w;
   }
   __syncthreads();
 
   // panel tiles: L_ik = A_ik Linv_kk^T, L_jk = A_jk Linv_kk^T
   float p1[4][4], p2[4][4];
-  if (worker) {
-    tile_xyt(sX, sL, p1);
-    if (!diag) tile_xyt(sY, sL, p2);
-  }
+  tile_xyt(sX, sL, p1);
+  if (!diag) tile_xyt(sY, sL, p2);
   __syncthreads();
-  if (worker) {
-    store_acc_t(sX, p1);
-    if (!diag) store_acc_t(sY, p2);
-  }
+  store_acc_t(sX, p1);
+  if (!diag) store_acc_t(sY, p2);
   __syncthreads();
 
-  if (worker) {
-    if (diag) {
-      // upper tile (k, i) = L_ik^T: its row q is column q of L_ik
+  if (diag) {
+    // upper tile (k, i) = L_ik^T: its row q is column q of L_ik
 #pragma unroll
-      for (int pass = 0; pass < 4; ++pass) {
-        const int q = (t >> 4) + 16 * pass, c = t & 15;
-        const float4 v = *reinterpret_cast<const float4 *>(&sX[q][tgrp(c, q)]);
-        *reinterpret_cast<float4 *>(M + (long long)(k * NB + q) * ld + i * NB + 4 * c) = v;
-      }
+    for (int pass = 0; pass < 4; ++pass) {
+      const int q = (t >> 4) + 16 * pass, c = t & 15;
+      const float4 v = *reinterpret_cast<const float4 *>(&sX[q][tgrp(c, q)]);
+      *reinterpret_cast<float4 *>(M + (long long)(k * NB + q) * ld + i * NB + 4 * c) = v;
     }
-    // trailing update A_ij -= L_ik L_jk^T
-    float upd[4][4];
-    tile_xyt(sX, diag ? sX : sY, upd);
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b) aij[a][b] -= upd[a][b];
   }
+  // trailing update A_ij -= L_ik L_jk^T
+  float upd[4][4];
+  tile_xyt(sX, diag ? sX : sY, upd);
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) aij[a][b] -= upd[a][b];
 
   if (i == k + 1) {
     // the next diagonal block: factor and invert it for the next launch
     // (nothing reads the tile itself again, so it is not stored)
     __syncthreads();  // all reads of sX and sY are done
     float *S = &sY[0][0];
-    if (worker) {
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
-        *reinterpret_cast<float4 *>(S + (4 * ty + a) * NB + 4 * tx) =
-            make_float4(aij[a][0], aij[a][1], aij[a][2], aij[a][3]);
-    }
+    for (int a = 0; a < 4; ++a)
+      *reinterpret_cast<float4 *>(S + (4 * ty + a) * NB + 4 * tx) =
+          make_float4(aij[a][0], aij[a][1], aij[a][2], aij[a][3]);
     __syncthreads();
     factor_invert_tile(S, &sX[0][0], Linv + (long long)(k + 1) * NB * NB, (k + 1) * NB, flag, err);
-  } else if (worker) {
+  } else {
 #pragma unroll
     for (int a = 0; a < 4; ++a)
       *reinterpret_cast<float4 *>(tile + (long long)(4 * ty + a) * ld + 4 * tx) =
