@@ -213,7 +213,7 @@ ispa_status ispa_ridge_solve(int D, int Dout, const float *G, const float *C, co
  * Same arguments and results as ispa_ridge_solve, without the workspace.  Its
  * scratch is a static array inside the library sized for the largest problem
  * (2.25 ISPA_RIDGE_NOALLOC_MAX_D^2 + 64 ISPA_RIDGE_NOALLOC_MAX_D +
- * 2 ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_DOUT floats, 17.25 MiB),
+ * 4 ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_DOUT floats, 25.25 MiB),
  * which every GPU that loads the library holds until the process exits; the call
  * itself allocates nothing.  D > ISPA_RIDGE_NOALLOC_MAX_D or Dout >
  * ISPA_RIDGE_NOALLOC_MAX_DOUT returns ISPA_ERR_INVALID_ARG.  The first call on

@@ -5,8 +5,10 @@
 
 namespace ispa {
 
-ispa_status launch_tc_gemm(const CUtensorMap &ta, const CUtensorMap &tb0, const CUtensorMap &tb1,
-                           tcg::Params &P, cudaStream_t s) {
+namespace {
+
+ispa_status launch_kernel(const CUtensorMap &ta, const CUtensorMap &tb0, const CUtensorMap &tb1,
+                          const CUtensorMap &ta_lo, const CUtensorMap &tb_lo, tcg::Params &P, cudaStream_t s) {
   if (P.n_tiles == 0 || P.K == 0) return ISPA_OK;
   static thread_local int configured_device = -1;
   int dev = 0;
@@ -17,9 +19,25 @@ ispa_status launch_tc_gemm(const CUtensorMap &ta, const CUtensorMap &tb0, const 
     if (e != cudaSuccess) return cuda_status(e, "gemm smem attribute");
     configured_device = dev;
   }
-  tcg::gemm_kernel<<<P.n_tiles, tcg::THREADS, tcg::SMEM_BYTES, s>>>(ta, tb0, tb1, P);
+  const int nchunk = P.nchunk > 1 ? P.nchunk : 1;
+  tcg::gemm_kernel<<<P.n_tiles * nchunk, tcg::THREADS, tcg::SMEM_BYTES, s>>>(ta, tb0, tb1, ta_lo, tb_lo, P);
   note_launch();
   return cuda_status(cudaGetLastError(), "tcgen05 gemm launch");
+}
+
+}  // namespace
+
+ispa_status launch_tc_gemm(const CUtensorMap &ta, const CUtensorMap &tb0, const CUtensorMap &tb1,
+                           tcg::Params &P, cudaStream_t s) {
+  P.split3 = 0;
+  return launch_kernel(ta, tb0, tb1, ta, tb0, P, s);
+}
+
+ispa_status launch_tc_gemm_split3(const CUtensorMap &ta, const CUtensorMap &ta_lo, const CUtensorMap &tb,
+                                  const CUtensorMap &tb_lo, tcg::Params &P, cudaStream_t s) {
+  P.split3 = 1;
+  P.n_tiles = P.n_tiles0;  // one sub-problem
+  return launch_kernel(ta, tb, tb, ta_lo, tb_lo, P, s);
 }
 
 // y[M, N] = A[M, K] B[K, N], A and B bf16 row-major (A K-major, B MN-major).

@@ -22,9 +22,22 @@
 // outputs run in one launch: blockIdx.x enumerates the tiles of problem 0,
 // then those of problem 1.  Tiles may be restricted to the upper triangle
 // (used for the symmetric Gram matrix).
+//
+// fp32-accurate products on the tf32 pipe (split3): with x = x_hi + x_lo,
+// x_hi the nearest tf32 and x_lo the remainder, A B is taken as
+// A_hi B_hi + A_hi B_lo + A_lo B_hi, three passes over the K range into one
+// accumulator (the dropped A_lo B_lo is below fp32 rounding).  For these
+// products the K range of a tile may be cut to a triangle of A (lower:
+// k < m0 + BM; upper: k >= m0) and split into chunks of chunk_kt K-tiles, one
+// CTA each (blockIdx.x = tile * nchunk + chunk; an empty chunk exits at once),
+// whose partial products are added to the output with atomics.  The tensor
+// cores accumulate in fp32 with truncation, a bias of about 2^-25 of the sum
+// per MMA step: fine for the solve, not for quantities that are small
+// differences of large sums.
 #pragma once
 
 #include "common.cuh"
+#include "internal.h"
 
 namespace ispa {
 namespace tcg {
@@ -39,8 +52,11 @@ enum Epi : int {
   EPI_STORE_F32 = 0,      // out = acc
   EPI_STORE_TF32_SQ = 1,  // out = tf32_rn(acc); r2 += sum acc^2
   EPI_ACCUM_F32 = 2,      // out += acc
-  EPI_STORE_BF16 = 3      // out = bf16_rn(acc)
+  EPI_STORE_BF16 = 3,     // out = bf16_rn(acc)
+  EPI_ATOMIC_F32 = 4      // out += acc with atomics (split K)
 };
+
+enum Tri : int { TRI_NONE = 0, TRI_A_LOWER = 1, TRI_A_UPPER = 2 };
 
 struct SubProblem {
   int N;          // columns of this problem's output
@@ -60,6 +76,10 @@ struct Params {
   int a_mn, b_mn; // operand majorness (1 = MN-major)
   uint32_t idesc;
   double *r2;     // EPI_STORE_TF32_SQ accumulator
+  int split3;     // 1: three passes (hi hi, hi lo, lo hi) with the lo maps
+  int tri;        // Tri: K range of a tile cut to a triangle of A
+  int nchunk;     // K chunks per tile (0 or 1: none)
+  int chunk_kt;   // K-tiles per chunk
   SubProblem p[2];
   DevErr err;
 };
@@ -95,6 +115,11 @@ __device__ inline void tile_coords(const Params &P, int t, int &prob, int &tm, i
   tn = 0;
 }
 
+__device__ __forceinline__ void red_add_v4(float *p, float4 v) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
+
 template <int EPI>
 __device__ __forceinline__ void epilogue_chunk(const Params &P, const SubProblem &sp, int row, int col0,
                                                const uint32_t (&r)[32], double &sq) {
@@ -119,13 +144,17 @@ __device__ __forceinline__ void epilogue_chunk(const Params &P, const SubProblem
     return;
   }
   float *o = reinterpret_cast<float *>(sp.out) + (long long)row * sp.ldo + col0;
-  const bool full = col0 + 32 <= N && (!sp.upper || col0 >= row);
+  const bool full = col0 + 32 <= N && (!sp.upper || col0 >= row) && (reinterpret_cast<uintptr_t>(o) & 15) == 0;
   if (full) {
     float4 *o4 = reinterpret_cast<float4 *>(o);
 #pragma unroll
     for (int v = 0; v < 8; ++v) {
       float4 x = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]), __uint_as_float(r[4 * v + 2]),
                              __uint_as_float(r[4 * v + 3]));
+      if (EPI == EPI_ATOMIC_F32) {
+        red_add_v4(o + 4 * v, x);
+        continue;
+      }
       if (EPI == EPI_STORE_TF32_SQ) {
         sq += (double)x.x * x.x + (double)x.y * x.y + (double)x.z * x.z + (double)x.w * x.w;
         x = make_float4(to_tf32_rn(x.x), to_tf32_rn(x.y), to_tf32_rn(x.z), to_tf32_rn(x.w));
@@ -145,6 +174,10 @@ __device__ __forceinline__ void epilogue_chunk(const Params &P, const SubProblem
       if (c >= N) break;
       if (sp.upper && c < row) continue;
       float x = __uint_as_float(r[j]);
+      if (EPI == EPI_ATOMIC_F32) {
+        atomicAdd(o + j, x);
+        continue;
+      }
       if (EPI == EPI_STORE_TF32_SQ) {
         sq += (double)x * x;
         x = to_tf32_rn(x);
@@ -156,10 +189,12 @@ __device__ __forceinline__ void epilogue_chunk(const Params &P, const SubProblem
 }
 
 #ifdef ISPA_DEFINE_GEMM_KERNEL
-// tma maps: ta = A operand; tb[prob] = B operand of each sub-problem.
+// tma maps: ta = A operand; tb[prob] = B operand of each sub-problem; with
+// split3, ta_lo and tb_lo hold the remainders of A and of B (problem 0 only).
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb0,
-                const __grid_constant__ CUtensorMap tb1, Params P) {
+                const __grid_constant__ CUtensorMap tb1, const __grid_constant__ CUtensorMap ta_lo,
+                const __grid_constant__ CUtensorMap tb_lo, Params P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = smem;
@@ -172,13 +207,25 @@ __global__ void __launch_bounds__(THREADS, 1)
   volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nchunk = P.nchunk > 1 ? P.nchunk : 1;
   int prob, tm, tn;
-  tile_coords(P, blockIdx.x, prob, tm, tn);
+  tile_coords(P, blockIdx.x / nchunk, prob, tm, tn);
   const SubProblem &sp = P.p[prob];
   const CUtensorMap *tB = prob == 0 ? &tb0 : &tb1;
   const int m0 = tm * BM, n0 = tn * BN;
-  const int k_tiles = (P.K + (P.kind_tf32 ? 31 : 63)) / (P.kind_tf32 ? 32 : 64);
   const int bk = P.kind_tf32 ? 32 : 64;         // K elements per stage
+  // this CTA's K-tiles [kt_begin, kt_end): the tile's range (cut to A's
+  // triangle), then this chunk of it
+  int kt_begin = 0, kt_end = (P.K + bk - 1) / bk;
+  if (P.tri == TRI_A_LOWER) kt_end = min(kt_end, (m0 + BM + bk - 1) / bk);
+  if (P.tri == TRI_A_UPPER) kt_begin = m0 / bk;
+  if (nchunk > 1) {
+    kt_begin += (blockIdx.x % nchunk) * P.chunk_kt;
+    kt_end = min(kt_end, kt_begin + P.chunk_kt);
+  }
+  if (kt_begin >= kt_end) return;  // empty chunk: nothing to add (before any barrier or TMEM)
+  const int k_span = kt_end - kt_begin;
+  const int k_tiles = k_span * (P.split3 ? 3 : 1);  // pipeline iterations
   const int e128 = P.kind_tf32 ? 32 : 64;       // elements per 128-byte row
   const uint32_t kstep_kmajor = 32;             // bytes per MMA K-step inside a K-major row
   const uint32_t kstep_mn = P.kind_tf32 ? 1024 : 2048;  // bytes per MMA K-step in an MN-major tile
@@ -197,6 +244,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&ta);
     tma_prefetch_desc(tB);
+    if (P.split3) {
+      tma_prefetch_desc(&ta_lo);
+      tma_prefetch_desc(&tb_lo);
+    }
   }
   if (warp == 1) tmem_alloc(tmem_slot, BN);
   tc_fence_before();
@@ -213,18 +264,21 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t ph = (kt / STAGES) & 1;
         if (!wait_parity(empty + s, ph ^ 1, P.err, abort, 1)) break;
         mbar_arrive_expect_tx(full + s, TILE_BYTES + TILE_B_BYTES);
-        const int k0 = kt * bk;
+        const int pass = kt / k_span;  // split3: 0 = hi hi, 1 = hi lo, 2 = lo hi
+        const int k0 = (kt_begin + kt - pass * k_span) * bk;
+        const CUtensorMap *mA = pass == 2 ? &ta_lo : &ta;
+        const CUtensorMap *mB = pass == 1 ? &tb_lo : tB;
         uint8_t *a = sA + s * TILE_BYTES;
         uint8_t *b = sB + s * TILE_B_BYTES;
         if (!P.a_mn) {
-          tma_load_2d(a, &ta, full + s, k0, m0);
+          tma_load_2d(a, mA, full + s, k0, m0);
         } else {
-          for (int c = 0; c < BM / e128; ++c) tma_load_2d(a + c * mn_box_bytes, &ta, full + s, m0 + c * e128, k0);
+          for (int c = 0; c < BM / e128; ++c) tma_load_2d(a + c * mn_box_bytes, mA, full + s, m0 + c * e128, k0);
         }
         if (!P.b_mn) {  // 128-row boxes, one after the other
-          for (int c = 0; c < BN / 128; ++c) tma_load_2d(b + c * TILE_BYTES, tB, full + s, k0, n0 + c * 128);
+          for (int c = 0; c < BN / 128; ++c) tma_load_2d(b + c * TILE_BYTES, mB, full + s, k0, n0 + c * 128);
         } else {
-          for (int c = 0; c < BN / e128; ++c) tma_load_2d(b + c * mn_box_bytes, tB, full + s, n0 + c * e128, k0);
+          for (int c = 0; c < BN / e128; ++c) tma_load_2d(b + c * mn_box_bytes, mB, full + s, n0 + c * e128, k0);
         }
         pending |= 1u << s;
         issued_phase = (issued_phase & ~(1u << s)) | (ph << s);
@@ -281,6 +335,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           case EPI_STORE_F32: epilogue_chunk<EPI_STORE_F32>(P, sp, row, n0 + c * 32, r, sq); break;
           case EPI_STORE_TF32_SQ: epilogue_chunk<EPI_STORE_TF32_SQ>(P, sp, row, n0 + c * 32, r, sq); break;
           case EPI_ACCUM_F32: epilogue_chunk<EPI_ACCUM_F32>(P, sp, row, n0 + c * 32, r, sq); break;
+          case EPI_ATOMIC_F32: epilogue_chunk<EPI_ATOMIC_F32>(P, sp, row, n0 + c * 32, r, sq); break;
           default: epilogue_chunk<EPI_STORE_BF16>(P, sp, row, n0 + c * 32, r, sq); break;
         }
       }
@@ -298,4 +353,29 @@ __global__ void __launch_bounds__(THREADS, 1)
 #endif  // ISPA_DEFINE_GEMM_KERNEL
 
 }  // namespace tcg
+
+// fp32 map of a row-major [outer, inner] matrix with leading dimension ld
+// (elements, a multiple of 4).  K-major operands use the 128-byte swizzle;
+// MN-major tf32 operands the 128-byte swizzle with 32-byte atoms.
+inline ispa_status map2d_f32_ld(CUtensorMap *m, const void *base, int inner, int outer, long long ld, int box_inner,
+                                int box_outer, bool mn_major) {
+  const uint64_t dims[2] = {(uint64_t)inner, (uint64_t)outer};
+  const uint64_t strides[1] = {(uint64_t)ld * 4};
+  const uint32_t box[2] = {(uint32_t)box_inner, (uint32_t)box_outer};
+  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box,
+                   mn_major ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+inline ispa_status map2d_f32(CUtensorMap *m, const void *base, int inner, int outer, int box_inner, int box_outer,
+                             bool mn_major) {
+  return map2d_f32_ld(m, base, inner, outer, inner, box_inner, box_outer, mn_major);
+}
+
+// Host launchers (gemm_tc.cu).  launch_tc_gemm: up to two sub-problems, one
+// pass.  launch_tc_gemm_split3: one sub-problem, fp32-accurate three-pass
+// product from the hi and lo maps of A and B.
+ispa_status launch_tc_gemm(const CUtensorMap &ta, const CUtensorMap &tb0, const CUtensorMap &tb1,
+                           tcg::Params &P, cudaStream_t s);
+ispa_status launch_tc_gemm_split3(const CUtensorMap &ta, const CUtensorMap &ta_lo, const CUtensorMap &tb,
+                                  const CUtensorMap &tb_lo, tcg::Params &P, cudaStream_t s);
 }  // namespace ispa

@@ -9,13 +9,24 @@
 //   CTA of tile (k+1, k+1) -- block 0, dispatched first -- goes on to factor
 //   that tile and invert its factor, so the next launch finds Linv_{k+1} ready.
 // One more launch copies L^T from the upper tiles into the lower ones.  Then
-// X = L^-1 by recursive 2 x 2 block inversion (batched GEMMs, one pair per
-// recursion depth), and the solve is two triangular GEMMs,
+// X = L^-1 by recursive 2 x 2 block inversion (batched fp32 GEMMs, one pair
+// per recursion depth), and the solve is two triangular GEMMs,
 //   dW = X^T (X C),
 // fully parallel instead of a chain of block substitutions; the same X serves
 // the optional iterative refinement (residual C - (G + lambda I) dW with fp64
 // accumulation, dW += X^T (X residual)).  epsilon = r2 - 2<dW, C> + <dW, G dW>
 // with fp64 reductions.
+//
+// The two solve products run on the tensor cores' tf32 pipe: every operand x
+// is split into x_hi (the nearest tf32) and x_lo = x - x_hi, and a product is
+// taken as A_hi B_hi + A_hi B_lo + A_lo B_hi in three passes of the tcgen05
+// GEMM into one fp32 accumulator (the dropped A_lo B_lo and the tf32 rounding
+// of the remainders are of order 2^-22 of each term; the accumulator's own
+// truncation adds a bias of about 2^-25 of the sum per MMA step).  Their K
+// ranges are cut to the triangle of X and split into chunks whose partial
+// products are added with atomics.  <dW, G dW> stays on the fp32 CUDA cores:
+// epsilon is a small difference of O(r2) terms and needs round-to-nearest
+// accumulation.
 //
 // Sizes are padded to Dp = 64 * ceil(D / 64) with an identity block, which is
 // decoupled from the problem and keeps every tile whole.
@@ -23,8 +34,10 @@
 #include <utility>
 #include <vector>
 
+#include "gemm_tc.cuh"
 #include "internal.h"
 #include "simt_gemm.cuh"
+#include "simt_gemm_batched.cuh"
 
 namespace ispa {
 
@@ -39,6 +52,8 @@ struct Ws {
   float *T;      // [Dp * Dp / 4] products of the recursive inversion
   float *Y;      // [D, Doutp] L^-1 times the right-hand side
   float *Rres;   // [D, Dout] refinement residual
+  float *Bhi;    // [D, Doutp] tf32 parts (nearest tf32, remainder) of a right-hand operand
+  float *Blo;
   double *acc;   // [0] <dW, C>  [1] <dW, G dW>  [2] trace(G)  [3] lambda_eff
   int *flag;     // non-zero once a pivot failed
 };
@@ -64,6 +79,8 @@ size_t carve_bytes(int D, int Dout, Ws *w, void *base) {
   float *T = reinterpret_cast<float *>(take(Dp * Dp / 4 * sizeof(float)));
   float *Y = reinterpret_cast<float *>(take((size_t)D * padded4(Dout) * sizeof(float)));
   float *R = reinterpret_cast<float *>(take((size_t)D * Dout * sizeof(float)));
+  float *Bhi = reinterpret_cast<float *>(take((size_t)D * padded4(Dout) * sizeof(float)));
+  float *Blo = reinterpret_cast<float *>(take((size_t)D * padded4(Dout) * sizeof(float)));
   char *tail = take(256);
   if (w) {
     w->M = M;
@@ -72,6 +89,8 @@ size_t carve_bytes(int D, int Dout, Ws *w, void *base) {
     w->T = T;
     w->Y = Y;
     w->Rres = R;
+    w->Bhi = Bhi;
+    w->Blo = Blo;
     w->acc = reinterpret_cast<double *>(tail);
     w->flag = reinterpret_cast<int *>(tail + 64);
   }
@@ -487,6 +506,29 @@ struct EpiResidual {
   }
 };
 
+// out[i][j] = G[min(i,j)][max(i,j)]: the full symmetric matrix from its upper triangle.
+// hi = the nearest tf32 of x and lo = x - hi (exact in fp32) for a rows x cols
+// block; src and hi may be the same array (then lds == ldd).
+__global__ void split_tf32_kernel(int rows, int cols, const float *src, long long lds, float *hi, float *lo,
+                                  long long ldd) {
+  const long long n = (long long)rows * cols;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
+    const long long i = e / cols, j = e - i * cols;
+    const float x = src[i * lds + j];
+    const float h = to_tf32_rn(x);
+    hi[i * ldd + j] = h;
+    lo[i * ldd + j] = x - h;
+  }
+}
+
+__global__ void symmetrize_kernel(int D, const float *__restrict__ G, float *out) {
+  const long long n = (long long)D * D;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
+    const int i = (int)(e / D), j = (int)(e - (long long)i * D);
+    out[e] = i <= j ? G[e] : G[(long long)j * D + i];
+  }
+}
+
 // acc[1] += sum dW[m][n] * (G dW)[m][n]
 struct EpiDotG {
   const float *dW;
@@ -500,15 +542,6 @@ struct EpiDotG {
     if ((threadIdx.x & 31) == 0) atomicAdd(acc + 1, s);
   }
 };
-
-// out[i][j] = G[min(i,j)][max(i,j)]: the full symmetric matrix from its upper triangle.
-__global__ void symmetrize_kernel(int D, const float *__restrict__ G, float *out) {
-  const long long n = (long long)D * D;
-  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
-    const int i = (int)(e / D), j = (int)(e - (long long)i * D);
-    out[e] = i <= j ? G[e] : G[(long long)j * D + i];
-  }
-}
 
 __global__ void dot_kernel(long long n, const float *__restrict__ a, const float *__restrict__ b, double *out) {
   double s = 0.0;
@@ -540,7 +573,7 @@ __global__ void x_init_kernel(int Dp, const float *__restrict__ Linv, float *X) 
 // chunks so that every SM gets a few CTAs (balancing the triangular K ranges
 // and giving the small products of the inversion enough parallelism); the
 // outputs must then already hold beta C (zero for beta = 0).
-cudaError_t launch_gemm_batch(const GemmJob *jobs, int n, bool a_trans, bool split_k, cudaStream_t s) {
+cudaError_t launch_gemm_batch(const GemmJob *jobs, int n, bool split_k, cudaStream_t s) {
   for (int b0 = 0; b0 < n; b0 += kMaxGemmJobs) {
     GemmBatch batch{};
     const int cnt = n - b0 < kMaxGemmJobs ? n - b0 : kMaxGemmJobs;
@@ -571,22 +604,14 @@ cudaError_t launch_gemm_batch(const GemmJob *jobs, int n, bool a_trans, bool spl
       int dev = 0;
       cudaGetDevice(&dev);
       if (configured_device != dev) {
-        cudaError_t e = cudaFuncSetAttribute(simt_gemm_pipe_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(simt_gemm_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)kPipeSmemBytes);
-        if (e == cudaSuccess)
-          e = cudaFuncSetAttribute(simt_gemm_pipe_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)kPipeSmemBytes);
         if (e != cudaSuccess) return e;
         configured_device = dev;
       }
-      if (a_trans)
-        simt_gemm_pipe_kernel<true><<<grid, 256, kPipeSmemBytes, s>>>(batch, nsplit, kchunk);
-      else
-        simt_gemm_pipe_kernel<false><<<grid, 256, kPipeSmemBytes, s>>>(batch, nsplit, kchunk);
-    } else if (a_trans) {
-      simt_gemm_batched_kernel<true><<<grid, 256, 0, s>>>(batch, vec, nsplit, kchunk);
+      simt_gemm_pipe_kernel<<<grid, 256, kPipeSmemBytes, s>>>(batch, nsplit, kchunk);
     } else {
-      simt_gemm_batched_kernel<false><<<grid, 256, 0, s>>>(batch, vec, nsplit, kchunk);
+      simt_gemm_batched_kernel<<<grid, 256, 0, s>>>(batch, vec, nsplit, kchunk);
     }
     note_launch();
     cudaError_t e = cudaGetLastError();
@@ -633,27 +658,78 @@ cudaError_t invert_factor(int Dp, const Ws &w, cudaStream_t s) {
     }
     // T starts at zero (split-K accumulates into it); X21 is still zero from x_init
     cudaError_t e = cudaMemsetAsync(w.T, 0, (size_t)t_off * sizeof(float), s);
-    if (e == cudaSuccess) e = launch_gemm_batch(first.data(), (int)first.size(), false, true, s);
-    if (e == cudaSuccess) e = launch_gemm_batch(second.data(), (int)second.size(), false, true, s);
+    if (e == cudaSuccess) e = launch_gemm_batch(first.data(), (int)first.size(), true, s);
+    if (e == cudaSuccess) e = launch_gemm_batch(second.data(), (int)second.size(), true, s);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
 }
 
+cudaError_t split_tf32(int rows, int cols, const float *src, long long lds, float *hi, float *lo, long long ldd,
+                       cudaStream_t s) {
+  split_tf32_kernel<<<sm_count() * 4, 256, 0, s>>>(rows, cols, src, lds, hi, lo, ldd);
+  note_launch();
+  return cudaGetLastError();
+}
+
+// K-tiles (32 elements of K) per CTA of the three-pass products
+constexpr int kTc3ChunkKt = 8;
+
+// out += op(A) B on the tf32 pipe: three passes of the tcgen05 GEMM, K chunks
+// added with atomics (out must hold its start value).  A is given as its tf32
+// parts (a_hi, a_lo), row-major [M, K] with leading dimension lda, or, with
+// a_trans, stored [K, M] (op(A) = A^T); B as (b_hi, b_lo), row-major [K, N],
+// ldb.  tri cuts each tile's K range to the triangle of op(A) that may be
+// non-zero.  Every leading dimension a multiple of 4, every base 16-byte
+// aligned.
+ispa_status tc3_product(int M, int N, int K, const float *a_hi, const float *a_lo, long long lda, bool a_trans,
+                        int tri, const float *b_hi, const float *b_lo, long long ldb, float *out, long long ldo,
+                        const DevErr &err, cudaStream_t s) {
+  if (M <= 0 || N <= 0 || K <= 0) return ISPA_OK;
+  CUtensorMap ta, tal, tb, tbl;
+  ispa_status st;
+  const int a_inner = a_trans ? M : K, a_outer = a_trans ? K : M, a_box_outer = a_trans ? 32 : tcg::BM;
+  if ((st = map2d_f32_ld(&ta, a_hi, a_inner, a_outer, lda, 32, a_box_outer, a_trans)) != ISPA_OK) return st;
+  if ((st = map2d_f32_ld(&tal, a_lo, a_inner, a_outer, lda, 32, a_box_outer, a_trans)) != ISPA_OK) return st;
+  if ((st = map2d_f32_ld(&tb, b_hi, N, K, ldb, 32, 32, true)) != ISPA_OK) return st;
+  if ((st = map2d_f32_ld(&tbl, b_lo, N, K, ldb, 32, 32, true)) != ISPA_OK) return st;
+  tcg::Params P{};
+  P.M = M;
+  P.K = K;
+  P.tiles_m = (M + tcg::BM - 1) / tcg::BM;
+  P.kind_tf32 = 1;
+  P.a_mn = a_trans ? 1 : 0;
+  P.b_mn = 1;
+  P.idesc = make_idesc(tcg::BM, tcg::BN, 2, P.a_mn, 1);
+  P.r2 = nullptr;
+  P.tri = tri;
+  P.chunk_kt = kTc3ChunkKt;
+  P.nchunk = ((K + 31) / 32 + kTc3ChunkKt - 1) / kTc3ChunkKt;
+  P.p[0] = tcg::SubProblem{N, (N + tcg::BN - 1) / tcg::BN, 0, tcg::EPI_ATOMIC_F32, out, ldo};
+  P.p[1] = P.p[0];
+  P.n_tiles0 = P.tiles_m * P.p[0].tiles_n;
+  P.err = err;
+  return launch_tc_gemm_split3(ta, tal, tb, tbl, P, s);
+}
+
 // out = beta out + A^-1 rhs = beta out + X^T (X rhs), rhs and out [D, Dout]
-// (beta 0 or 1).
-cudaError_t apply_inverse(int D, int Dout, const Ws &w, const float *rhs, float *out, float beta, cudaStream_t s) {
+// (leading dimension Dout, beta 0 or 1), with X in tf32 parts (w.X, w.M).
+ispa_status apply_inverse(int D, int Dout, const Ws &w, const float *rhs, float *out, float beta, const DevErr &err,
+                          cudaStream_t s) {
   const int Dp = padded(D), ldy = padded4(Dout);
-  // split-K accumulates into its outputs: Y starts at zero, out at beta out
-  cudaError_t e = cudaMemsetAsync(w.Y, 0, (size_t)D * ldy * sizeof(float), s);
+  // the products add their K chunks with atomics: Y starts at zero, out at beta out
+  cudaError_t e = split_tf32(D, Dout, rhs, Dout, w.Bhi, w.Blo, ldy, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(w.Y, 0, (size_t)D * ldy * sizeof(float), s);
   if (e == cudaSuccess && beta == 0.f) e = cudaMemsetAsync(out, 0, (size_t)D * Dout * sizeof(float), s);
-  if (e != cudaSuccess) return e;
-  const GemmJob y{w.X, rhs, w.Y, Dp, Dout, ldy, D, Dout, D, kTriALower, 1.f, 0.f};
-  e = launch_gemm_batch(&y, 1, false, true, s);
-  if (e != cudaSuccess) return e;
-  // X^T is upper triangular: op(A)[m][k] = X[k][m] = 0 for k < m
-  const GemmJob x{w.X, w.Y, out, Dp, ldy, Dout, D, Dout, D, kTriAUpper, 1.f, beta};
-  return launch_gemm_batch(&x, 1, true, true, s);
+  if (e != cudaSuccess) return cuda_status(e, "ridge solve set-up");
+  // Y = X rhs   (X lower triangular)
+  ispa_status st =
+      tc3_product(D, Dout, D, w.X, w.M, Dp, false, tcg::TRI_A_LOWER, w.Bhi, w.Blo, ldy, w.Y, ldy, err, s);
+  if (st != ISPA_OK) return st;
+  e = split_tf32(D, Dout, w.Y, ldy, w.Y, w.Blo, ldy, s);
+  if (e != cudaSuccess) return cuda_status(e, "ridge solve split");
+  // out += X^T Y   (X^T upper triangular)
+  return tc3_product(D, Dout, D, w.X, w.M, Dp, true, tcg::TRI_A_UPPER, w.Y, w.Blo, ldy, out, Dout, err, s);
 }
 
 }  // namespace
@@ -671,11 +747,11 @@ size_t ridge_workspace_bytes(int D, int Dout) { return carve_bytes(D, Dout, null
 // ---------------------------------------------------------------------------
 // the workspace of the largest size (D a multiple of 64 and Dout of 4, so
 // every part is a multiple of 256 bytes): factor copy, inverse, inversion
-// products, diagonal-block inverses, two D x Dout buffers, accumulators
+// products, diagonal-block inverses, four D x Dout buffers, accumulators
 constexpr size_t kNoAllocScratchBytes =
     (size_t)ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_D * 4 * 2 +
     (size_t)ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_D +
-    (size_t)ISPA_RIDGE_NOALLOC_MAX_D * NB * 4 + (size_t)ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_DOUT * 4 * 2 +
+    (size_t)ISPA_RIDGE_NOALLOC_MAX_D * NB * 4 + (size_t)ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_DOUT * 4 * 4 +
     256;
 static __device__ __align__(256) unsigned char g_ridge_scratch[kNoAllocScratchBytes];
 
@@ -723,18 +799,24 @@ ispa_status launch_ridge(int D, int Dout, const float *G, const float *C, const 
   }
   cudaError_t e = invert_factor(Dp, w, s);
   if (e != cudaSuccess) return cuda_status(e, "ridge inverse");
-  e = apply_inverse(D, Dout, w, C, dW, 0.f, s);
-  if (e != cudaSuccess) return cuda_status(e, "ridge solve");
+  // X in tf32 parts for the solve products: hi in place, lo in M (free after the inversion)
+  e = split_tf32(Dp, Dp, w.X, Dp, w.X, w.M, Dp, s);
+  if (e != cudaSuccess) return cuda_status(e, "ridge inverse split");
+  st = apply_inverse(D, Dout, w, C, dW, 0.f, err, s);
+  if (st != ISPA_OK) return st;
   const long long nDO = (long long)D * Dout;
   for (int r = 0; r < refine_steps; ++r) {
     e = simt_gemm<OP_SYM_UPPER, OP_N, double, 0>(D, Dout, D, Operand{G, nullptr, D}, Operand{dW, nullptr, Dout},
                                                  EpiResidual{w.Rres, C, dW, w.acc, Dout}, s);
     if (e != cudaSuccess) return cuda_status(e, "ridge residual");
-    e = apply_inverse(D, Dout, w, w.Rres, dW, 1.f, s);
-    if (e != cudaSuccess) return cuda_status(e, "ridge refinement solve");
+    st = apply_inverse(D, Dout, w, w.Rres, dW, 1.f, err, s);
+    if (st != ISPA_OK) return st;
   }
   dot_kernel<<<grid, 256, 0, s>>>(nDO, dW, C, w.acc);
   note_launch();
+  // <dW, G dW> on the fp32 CUDA cores: epsilon cancels r2 against 2<dW, C>,
+  // so this term needs round-to-nearest accumulation (the tensor cores' fp32
+  // accumulation truncates, a bias that grows with K)
   if (D % 4 == 0 && Dout % 4 == 0) {
     // the factorisation is no longer needed: expand G to the full symmetric
     // matrix there so that the G dW product reads both operands row-major with

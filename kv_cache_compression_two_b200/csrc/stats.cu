@@ -72,26 +72,12 @@ TF32Ws carve_tf32(void *ws, int T, int D, int Dout) {
   return w;
 }
 
-// fp32 map of a row-major [outer, inner] matrix.  K-major operands use the
-// 128-byte swizzle; MN-major tf32 operands the 128-byte swizzle with 32-byte atoms.
-ispa_status map2d_f32(CUtensorMap *m, const void *base, int inner, int outer, int box_inner, int box_outer,
-                      bool mn_major) {
-  const uint64_t dims[2] = {(uint64_t)inner, (uint64_t)outer};
-  const uint64_t strides[1] = {(uint64_t)inner * 4};
-  const uint32_t box[2] = {(uint32_t)box_inner, (uint32_t)box_outer};
-  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box,
-                   mn_major ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B);
-}
-
 }  // namespace
 
 size_t stats_workspace_bytes(int T, int D, int Dout, ispa_precision prec) {
   if (prec == ISPA_PREC_F32) return a256((size_t)T * Dout * 4);
   return 2 * a256((size_t)T * D * 4) + a256((size_t)D * Dout * 4) + a256((size_t)T * Dout * 4);
 }
-
-ispa_status launch_tc_gemm(const CUtensorMap &ta, const CUtensorMap &tb0, const CUtensorMap &tb1,
-                           tcg::Params &P, cudaStream_t s);
 
 ispa_status launch_stats(int T, int D, int Dout, const float *a_loc, const float *a_full, const float *W,
                          float *G, float *C, double *r2, ispa_precision prec, void *ws, cudaStream_t s) {
