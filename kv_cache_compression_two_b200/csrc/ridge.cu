@@ -30,6 +30,7 @@
 //
 // Sizes are padded to Dp = 64 * ceil(D / 64) with an identity block, which is
 // decoupled from the problem and keeps every tile whole.
+#include <algorithm>
 #include <mutex>
 #include <utility>
 #include <vector>
@@ -521,14 +522,6 @@ __global__ void split_tf32_kernel(int rows, int cols, const float *src, long lon
   }
 }
 
-__global__ void symmetrize_kernel(int D, const float *__restrict__ G, float *out) {
-  const long long n = (long long)D * D;
-  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
-    const int i = (int)(e / D), j = (int)(e - (long long)i * D);
-    out[e] = i <= j ? G[e] : G[(long long)j * D + i];
-  }
-}
-
 // acc[1] += sum dW[m][n] * (G dW)[m][n]
 struct EpiDotG {
   const float *dW;
@@ -542,6 +535,44 @@ struct EpiDotG {
     if ((threadIdx.x & 31) == 0) atomicAdd(acc + 1, s);
   }
 };
+
+// acc[1] += <G, P> over a K slice of P = dW dW^T, from the upper triangles of
+// both (G's upper triangle as given, weight 2 off the diagonal): equal to
+// <dW, G dW> for symmetric G.
+struct EpiSymDot {
+  const float *G;
+  double *acc;
+  int ld;
+  double part;
+  __device__ void begin() { part = 0.0; }
+  __device__ void operator()(int m, int n, float a) {
+    if (m < n)
+      part += 2.0 * (double)G[(long long)m * ld + n] * (double)a;
+    else if (m == n)
+      part += (double)G[(long long)m * ld + m] * (double)a;
+  }
+  __device__ void end() {
+    const double s = warp_sum_d(part);
+    if ((threadIdx.x & 31) == 0) atomicAdd(acc + 1, s);
+  }
+};
+
+// dst [cols, rows] = src [rows, cols]^T through 32 x 32 shared-memory tiles;
+// block (32, 8), grid (ceil(cols / 32), ceil(rows / 32)).
+__global__ void transpose_kernel(int rows, int cols, const float *__restrict__ src, long long lds, float *dst,
+                                 long long ldd) {
+  __shared__ float t[32][33];
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < rows && c < cols) t[i][threadIdx.x] = src[(long long)r * lds + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (r < rows && c < cols) dst[(long long)c * ldd + r] = t[threadIdx.x][i];
+  }
+}
 
 __global__ void dot_kernel(long long n, const float *__restrict__ a, const float *__restrict__ b, double *out) {
   double s = 0.0;
@@ -818,12 +849,14 @@ ispa_status launch_ridge(int D, int Dout, const float *G, const float *C, const 
   // so this term needs round-to-nearest accumulation (the tensor cores' fp32
   // accumulation truncates, a bias that grows with K)
   if (D % 4 == 0 && Dout % 4 == 0) {
-    // the factorisation is no longer needed: expand G to the full symmetric
-    // matrix there so that the G dW product reads both operands row-major with
-    // 16-byte loads
-    symmetrize_kernel<<<grid, 256, 0, s>>>(D, G, w.M);
+    // as <G, dW dW^T>: only the upper-triangle tiles of dW dW^T, G read from
+    // its upper triangle; dW^T goes to the free right-hand-side buffer, and
+    // the K range (Dout) is split so that about two CTAs run per SM
+    transpose_kernel<<<dim3((Dout + 31) / 32, (D + 31) / 32), dim3(32, 8), 0, s>>>(D, Dout, dW, Dout, w.Bhi, D);
     note_launch();
-    e = simt_gemm_nn128(D, Dout, D, w.M, D, dW, Dout, EpiDotG{dW, w.acc, Dout, 0.0}, s);
+    const int tiles = (D + 127) / 128, upper_tiles = tiles * (tiles + 1) / 2;
+    const int nsplit = std::max(1, 2 * sm_count() / upper_tiles);
+    e = simt_gemm_nn128(D, D, Dout, dW, Dout, w.Bhi, D, EpiSymDot{G, w.acc, D, 0.0}, s, nsplit, 1);
   } else {
     e = simt_gemm<OP_SYM_UPPER, OP_N, float, 0>(D, Dout, D, Operand{G, nullptr, D}, Operand{dW, nullptr, Dout},
                                                 EpiDotG{dW, w.acc, Dout, 0.0}, s);

@@ -104,37 +104,43 @@ inline cudaError_t simt_gemm(int M, int N, int K, Operand A, Operand B, Epi epi,
 // 128 x 128 output tile, 256 threads with 8 x 8 accumulators each (two 4 x 4
 // quadrants 64 apart in each dimension, so shared-memory reads are float4 and
 // conflict-free), K staged 8 at a time through double-buffered shared memory
-// with the next stage prefetched into registers.
+// with the next stage prefetched into registers.  Grid z-slice z covers the
+// K range [z kchunk, (z + 1) kchunk) (kchunk a multiple of 8), so the epilogue
+// sees partial sums when gridDim.z > 1; with upper != 0 only tiles that reach
+// the upper triangle (some m <= n) run.
 // ---------------------------------------------------------------------------
 template <class Epi>
 __global__ void __launch_bounds__(256) simt_gemm_nn128_kernel(int M, int N, int K, const float *__restrict__ A,
                                                               long long lda, const float *__restrict__ B,
-                                                              long long ldb, Epi epi) {
+                                                              long long ldb, Epi epi, int kchunk, int upper) {
   __shared__ __align__(16) float As[2][8][128];
   __shared__ __align__(16) float Bs[2][8][128];
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const int m0 = blockIdx.y * 128, n0 = blockIdx.x * 128;
+  if (upper && m0 > n0 + 127) return;
+  const int k_lo = blockIdx.z * kchunk, k_hi = min(K, k_lo + kchunk);
+  if (k_lo >= k_hi) return;
   // A tile 128 x 8: thread loads row (tid >> 1), 4 k values at (tid & 1) * 4
   const int a_row = tid >> 1, a_k = (tid & 1) * 4;
   // B tile 8 x 128: thread loads k row (tid >> 5), 4 columns at (tid & 31) * 4
   const int b_k = tid >> 5, b_col = (tid & 31) * 4;
   auto load_a = [&](int k0, float4 &v) {
     const int gm = m0 + a_row, gk = k0 + a_k;
-    if (gm < M && gk + 3 < K) {
+    if (gm < M && gk + 3 < k_hi) {
       v = *reinterpret_cast<const float4 *>(A + (long long)gm * lda + gk);
     } else {
       float t[4];
-      for (int i = 0; i < 4; ++i) t[i] = (gm < M && gk + i < K) ? A[(long long)gm * lda + gk + i] : 0.f;
+      for (int i = 0; i < 4; ++i) t[i] = (gm < M && gk + i < k_hi) ? A[(long long)gm * lda + gk + i] : 0.f;
       v = make_float4(t[0], t[1], t[2], t[3]);
     }
   };
   auto load_b = [&](int k0, float4 &v) {
     const int gk = k0 + b_k, gn = n0 + b_col;
-    if (gk < K && gn + 3 < N) {
+    if (gk < k_hi && gn + 3 < N) {
       v = *reinterpret_cast<const float4 *>(B + (long long)gk * ldb + gn);
     } else {
       float t[4];
-      for (int i = 0; i < 4; ++i) t[i] = (gk < K && gn + i < N) ? B[(long long)gk * ldb + gn + i] : 0.f;
+      for (int i = 0; i < 4; ++i) t[i] = (gk < k_hi && gn + i < N) ? B[(long long)gk * ldb + gn + i] : 0.f;
       v = make_float4(t[0], t[1], t[2], t[3]);
     }
   };
@@ -144,8 +150,8 @@ __global__ void __launch_bounds__(256) simt_gemm_nn128_kernel(int M, int N, int 
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
   float4 ra, rb;
-  load_a(0, ra);
-  load_b(0, rb);
+  load_a(k_lo, ra);
+  load_b(k_lo, rb);
   int buf = 0;
   As[0][a_k + 0][a_row] = ra.x;
   As[0][a_k + 1][a_row] = ra.y;
@@ -153,8 +159,8 @@ __global__ void __launch_bounds__(256) simt_gemm_nn128_kernel(int M, int N, int 
   As[0][a_k + 3][a_row] = ra.w;
   *reinterpret_cast<float4 *>(&Bs[0][b_k][b_col]) = rb;
   __syncthreads();
-  for (int k0 = 0; k0 < K; k0 += 8) {
-    const bool more = k0 + 8 < K;
+  for (int k0 = k_lo; k0 < k_hi; k0 += 8) {
+    const bool more = k0 + 8 < k_hi;
     if (more) {
       load_a(k0 + 8, ra);
       load_b(k0 + 8, rb);
@@ -196,10 +202,11 @@ __global__ void __launch_bounds__(256) simt_gemm_nn128_kernel(int M, int N, int 
 
 template <class Epi>
 inline cudaError_t simt_gemm_nn128(int M, int N, int K, const float *A, long long lda, const float *B, long long ldb,
-                                   Epi epi, cudaStream_t s) {
-  if (M <= 0 || N <= 0) return cudaSuccess;
-  dim3 grid((N + 127) / 128, (M + 127) / 128);
-  simt_gemm_nn128_kernel<Epi><<<grid, 256, 0, s>>>(M, N, K, A, lda, B, ldb, epi);
+                                   Epi epi, cudaStream_t s, int nsplit = 1, int upper = 0) {
+  if (M <= 0 || N <= 0 || K <= 0) return cudaSuccess;
+  const int kchunk = ((K + nsplit - 1) / nsplit + 7) / 8 * 8;
+  dim3 grid((N + 127) / 128, (M + 127) / 128, (K + kchunk - 1) / kchunk);
+  simt_gemm_nn128_kernel<Epi><<<grid, 256, 0, s>>>(M, N, K, A, lda, B, ldb, epi, kchunk, upper);
   note_launch();
   return cudaGetLastError();
 }
