@@ -120,26 +120,42 @@ __global__ void trace_kernel(int D, const float *__restrict__ G, double *acc) {
   }
 }
 
+// (row block, column block) of tile lin of the lower triangle numbered row by
+// row: (0,0), (1,0), (1,1), (2,0), ...
+__device__ __forceinline__ void lower_tile(int lin, int &I, int &J) {
+  int a = (int)((sqrtf(8.f * lin + 1.f) - 1.f) * 0.5f);
+  while ((a + 1) * (a + 2) / 2 <= lin) ++a;
+  while (a * (a + 1) / 2 > lin) --a;
+  I = a;
+  J = lin - a * (a + 1) / 2;
+}
+
 // M = G + lambda I on the lower tiles (diagonal tiles whole), identity on the
-// padding.
-__global__ void init_kernel(int D, int Dp, const float *__restrict__ G, float lambda, int relative, Ws w) {
+// padding.  One CTA (256 threads) per lower tile: the tile (J, I) of G's upper
+// triangle is read row by row into shared memory and written transposed.
+__global__ void __launch_bounds__(256) init_kernel(int D, int Dp, const float *__restrict__ G, float lambda,
+                                                   int relative, Ws w) {
   const double lam = relative ? (double)lambda * w.acc[2] / D : (double)lambda;
   const float lamf = (float)lam;
-  const long long nDD = (long long)Dp * Dp;
-  const long long stride = (long long)gridDim.x * blockDim.x;
-  const long long t0 = blockIdx.x * (long long)blockDim.x + threadIdx.x;
-  if (t0 == 0) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
     w.acc[0] = 0.0;
     w.acc[1] = 0.0;
     w.acc[3] = (double)lamf;
     *w.flag = 0;
   }
-  for (long long e = t0; e < nDD; e += stride) {
-    const int i = (int)(e / Dp), j = (int)(e - (long long)i * Dp);
-    if (i / NB < j / NB) continue;  // upper tiles are written by the factorisation
-    float x = (i == j) ? 1.f : 0.f;
-    if (i < D && j < D) x = G[(long long)min(i, j) * D + max(i, j)] + (i == j ? lamf : 0.f);
-    w.M[e] = x;
+  __shared__ float t[NB][NB + 1];
+  int I, J;
+  lower_tile(blockIdx.x, I, J);
+  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
+    const int r = e / NB, c = e % NB, gi = J * NB + r, gj = I * NB + c;
+    t[r][c] = (gi < D && gj < D) ? G[(long long)gi * D + gj] : 0.f;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
+    const int r = e / NB, c = e % NB, i = I * NB + r, j = J * NB + c;
+    float x = (I > J || r > c) ? t[c][r] : t[r][c];  // G symmetric from its upper triangle
+    if (i == j) x = i < D ? x + lamf : 1.f;
+    w.M[(long long)i * Dp + j] = x;
   }
 }
 
@@ -508,17 +524,37 @@ struct EpiResidual {
 };
 
 // out[i][j] = G[min(i,j)][max(i,j)]: the full symmetric matrix from its upper triangle.
+__device__ __forceinline__ bool aligned16_dev(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+__device__ __forceinline__ float4 tf32_hi4(float4 x) {
+  return make_float4(to_tf32_rn(x.x), to_tf32_rn(x.y), to_tf32_rn(x.z), to_tf32_rn(x.w));
+}
+
 // hi = the nearest tf32 of x and lo = x - hi (exact in fp32) for a rows x cols
-// block; src and hi may be the same array (then lds == ldd).
-__global__ void split_tf32_kernel(int rows, int cols, const float *src, long long lds, float *hi, float *lo,
-                                  long long ldd) {
-  const long long n = (long long)rows * cols;
-  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
-    const long long i = e / cols, j = e - i * cols;
-    const float x = src[i * lds + j];
-    const float h = to_tf32_rn(x);
-    hi[i * ldd + j] = h;
-    lo[i * ldd + j] = x - h;
+// block; src and hi may be the same array (then lds == ldd).  Blocks stride
+// over rows and threads over the columns of a row, four at a time when every
+// leading dimension is a multiple of 4 and every base 16-byte aligned.
+__global__ void __launch_bounds__(256) split_tf32_kernel(int rows, int cols, const float *src, long long lds,
+                                                         float *hi, float *lo, long long ldd) {
+  const bool vec = ((cols | (int)(lds & 3) | (int)(ldd & 3)) & 3) == 0 && aligned16_dev(src) &&
+                   aligned16_dev(hi) && aligned16_dev(lo);
+  for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+    const float *sr = src + (long long)r * lds;
+    float *hr = hi + (long long)r * ldd, *lr = lo + (long long)r * ldd;
+    if (vec) {
+      for (int c = threadIdx.x; c < cols / 4; c += blockDim.x) {
+        const float4 x = reinterpret_cast<const float4 *>(sr)[c];
+        const float4 h = tf32_hi4(x);
+        reinterpret_cast<float4 *>(hr)[c] = h;
+        reinterpret_cast<float4 *>(lr)[c] = make_float4(x.x - h.x, x.y - h.y, x.z - h.z, x.w - h.w);
+      }
+    } else {
+      for (int c = threadIdx.x; c < cols; c += blockDim.x) {
+        const float x = sr[c], h = to_tf32_rn(x);
+        hr[c] = h;
+        lr[c] = x - h;
+      }
+    }
   }
 }
 
@@ -574,10 +610,24 @@ __global__ void transpose_kernel(int rows, int cols, const float *__restrict__ s
   }
 }
 
-__global__ void dot_kernel(long long n, const float *__restrict__ a, const float *__restrict__ b, double *out) {
+// out += <a, b> over a rows x cols block with leading dimension ld (fp64
+// accumulation); float4 loads when ld is a multiple of 4 and both bases are
+// 16-byte aligned.
+__global__ void __launch_bounds__(256) dot_kernel(int rows, int cols, long long ld, const float *__restrict__ a,
+                                                  const float *__restrict__ b, double *out) {
+  const bool vec = ((cols | (int)(ld & 3)) & 3) == 0 && aligned16_dev(a) && aligned16_dev(b);
   double s = 0.0;
-  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x)
-    s += (double)a[e] * (double)b[e];
+  for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+    const float *ar = a + (long long)r * ld, *br = b + (long long)r * ld;
+    if (vec) {
+      for (int c = threadIdx.x; c < cols / 4; c += blockDim.x) {
+        const float4 x = reinterpret_cast<const float4 *>(ar)[c], y = reinterpret_cast<const float4 *>(br)[c];
+        s += (double)x.x * y.x + (double)x.y * y.y + (double)x.z * y.z + (double)x.w * y.w;
+      }
+    } else {
+      for (int c = threadIdx.x; c < cols; c += blockDim.x) s += (double)ar[c] * (double)br[c];
+    }
+  }
   s = warp_sum_d(s);
   if ((threadIdx.x & 31) == 0) atomicAdd(out, s);
 }
@@ -592,11 +642,15 @@ __global__ void finalize_kernel(long long n, const double *__restrict__ r2, Ws w
 }
 
 // X = 0 with the inverses of L's diagonal blocks on its diagonal tiles.
-__global__ void x_init_kernel(int Dp, const float *__restrict__ Linv, float *X) {
-  const long long n = (long long)Dp * Dp;
-  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
-    const int i = (int)(e / Dp), j = (int)(e - (long long)i * Dp);
-    X[e] = (i / NB == j / NB) ? Linv[(long long)(i / NB) * NB * NB + (i % NB) * NB + j % NB] : 0.f;
+// X = the block diagonal of the diagonal-block inverses, zero elsewhere; one
+// row per block iteration, four columns per thread (Dp is a multiple of 64).
+__global__ void __launch_bounds__(256) x_init_kernel(int Dp, const float *__restrict__ Linv, float *X) {
+  for (int r = blockIdx.x; r < Dp; r += gridDim.x) {
+    const int rb = r / NB;
+    const float4 *lrow = reinterpret_cast<const float4 *>(Linv + (long long)rb * NB * NB + (r % NB) * NB);
+    float4 *xrow = reinterpret_cast<float4 *>(X + (long long)r * Dp);
+    for (int c = threadIdx.x; c < Dp / 4; c += blockDim.x)
+      xrow[c] = (c * 4) / NB == rb ? lrow[c - rb * (NB / 4)] : make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 
@@ -816,7 +870,7 @@ ispa_status launch_ridge(int D, int Dout, const float *G, const float *C, const 
   const int Dp = padded(D), nb = Dp / NB;
   const int grid = sm_count() * 4;
   trace_kernel<<<1, 256, 0, s>>>(D, G, w.acc);
-  init_kernel<<<grid, 256, 0, s>>>(D, Dp, G, lambda, lambda_relative, w);
+  init_kernel<<<nb * (nb + 1) / 2, 256, 0, s>>>(D, Dp, G, lambda, lambda_relative, w);
   chol_first_kernel<<<1, kFactorThreads, 0, s>>>(Dp, w.M, w.Linv, w.flag, err);
   note_launch(3);
   for (int k = 0; k + 1 < nb; ++k) {
@@ -843,7 +897,7 @@ ispa_status launch_ridge(int D, int Dout, const float *G, const float *C, const 
     st = apply_inverse(D, Dout, w, w.Rres, dW, 1.f, err, s);
     if (st != ISPA_OK) return st;
   }
-  dot_kernel<<<grid, 256, 0, s>>>(nDO, dW, C, w.acc);
+  dot_kernel<<<grid, 256, 0, s>>>(D, Dout, Dout, dW, C, w.acc);
   note_launch();
   // <dW, G dW> on the fp32 CUDA cores: epsilon cancels r2 against 2<dW, C>,
   // so this term needs round-to-nearest accumulation (the tensor cores' fp32
