@@ -272,6 +272,39 @@ ispa_status ispa_attn_local_proj(const ispa_attn_desc *desc, const void *q, cons
                                  ispa_dtype y_dtype, void *workspace, size_t workspace_bytes,
                                  ispa_stream_t stream);
 
+/* ------------------------------------------------------------------------- */
+/* KV eviction of post-switch L-layers                                        */
+/* ------------------------------------------------------------------------- */
+/*
+ * After the switch the selected layers drop their historical KV entries and
+ * keep only the local context, sink and current frames [DE-summary 2,
+ * "Speichereffiziente Inferenz"; EN-notes, Key Designs 3 and "A Worked
+ * Example"].  The kept frames are the local group of desc: the union of
+ * [0, sink_frames) and [cur_begin, cur_end), in frame order.
+ *
+ * ispa_kv_evicted_desc: the descriptor of the evicted layout, in which the
+ * kept frames are stored back to back, each renumbered by its rank among the
+ * kept frames: sink_frames' = sink_frames, cur_begin' = min(cur_begin,
+ * sink_frames), cur_end' = cur_begin' + (cur_end - cur_begin), no history,
+ * kv_frames' = the number of kept frames.  The current chunk (the queries)
+ * keeps its length, and the local group of the result holds exactly the keys
+ * and values of the local group of desc, in the same order, so the
+ * post-switch calls (ispa_attn_split, ispa_attn_local_proj) on the evicted
+ * buffers attend to the same entries.  Host only; ISPA_ERR_INVALID_ARG for an
+ * invalid desc.
+ *
+ * ispa_kv_evict_history: copies, for every instance, the kept frames of k and
+ * v (layout of desc: [B, kv_frames * tpf, H, head_dim], in_dtype) into k_out
+ * and v_out (layout of the evicted desc: [B, kv_frames' * tpf, H, head_dim]),
+ * bit for bit.  The caller then releases k and v: per tensor that frees
+ * B * (kv_frames - kv_frames') * tpf * H * head_dim elements.  Outputs must
+ * not overlap inputs; all four pointers 16-byte aligned.  Asynchronous.
+ */
+ispa_status ispa_kv_evicted_desc(const ispa_attn_desc *desc, ispa_attn_desc *evicted);
+
+ispa_status ispa_kv_evict_history(const ispa_attn_desc *desc, const void *k, const void *v,
+                                  void *k_out, void *v_out, ispa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

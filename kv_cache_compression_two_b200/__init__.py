@@ -31,7 +31,7 @@ STATUS_NAMES = {0: "ISPA_OK", 1: "ISPA_ERR_INVALID_ARG", 2: "ISPA_ERR_UNSUPPORTE
 EXPORTED = ("ispa_version", "ispa_last_error", "ispa_launch_count", "ispa_check_device_error", "ispa_attn_split_workspace_bytes", "ispa_attn_split", "ispa_lse_merge",
             "ispa_accum_stats_workspace_bytes", "ispa_accum_stats", "ispa_ridge_workspace_bytes", "ispa_ridge_solve",
             "ispa_select_layers", "ispa_absorb_weight", "ispa_attn_local_proj_workspace_bytes",
-            "ispa_attn_local_proj", "ispa_ridge_solve_noalloc")
+            "ispa_attn_local_proj", "ispa_ridge_solve_noalloc", "ispa_kv_evicted_desc", "ispa_kv_evict_history")
 RIDGE_NOALLOC_MAX_D = RIDGE_NOALLOC_MAX_DOUT = 1024
 
 
@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
         "ispa_absorb_weight": (_ci, [_ci, _ci, _vp, _ci, _vp, _vp, _ci, _vp]),
         "ispa_attn_local_proj_workspace_bytes": (_sz, [ctypes.POINTER(AttnDesc)]),
         "ispa_attn_local_proj": (_ci, [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _ci, _vp, _ci, _vp, _sz, _vp]),
+        "ispa_kv_evicted_desc": (_ci, [ctypes.POINTER(AttnDesc), ctypes.POINTER(AttnDesc)]),
+        "ispa_kv_evict_history": (_ci, [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -226,6 +228,17 @@ def ispa_attn_local_proj(desc: AttnDesc, q, k, v, W_proj, Dout: int, y, y_dtype:
         workspace_bytes = workspace_bytes or workspace.numel() * workspace.element_size()
     _check(lib().ispa_attn_local_proj(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(W_proj), Dout, _ptr(y),
                                       y_dtype, _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def ispa_kv_evicted_desc(desc: AttnDesc) -> AttnDesc:
+    out = AttnDesc()
+    _check(lib().ispa_kv_evicted_desc(ctypes.byref(desc), ctypes.byref(out)))
+    return out
+
+
+def ispa_kv_evict_history(desc: AttnDesc, k, v, k_out, v_out, stream=None) -> None:
+    _check(lib().ispa_kv_evict_history(ctypes.byref(desc), _ptr(k), _ptr(v), _ptr(k_out), _ptr(v_out),
+                                       _stream(stream)))
 
 
 lib()

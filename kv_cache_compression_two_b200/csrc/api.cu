@@ -373,4 +373,49 @@ ispa_status ispa_attn_local_proj(const ispa_attn_desc *desc, const void *q, cons
   return launch_gemm_bf16(d.B * g.Lq, Dout, D, a_loc, W_proj, y, y_dtype, (cudaStream_t)stream);
 }
 
+ispa_status ispa_kv_evicted_desc(const ispa_attn_desc *desc, ispa_attn_desc *evicted) {
+  GroupRanges g;
+  float scale;
+  ispa_status st = attn_ranges(desc, &g, &scale);
+  if (st != ISPA_OK) return st;
+  if (!evicted) return fail(ISPA_ERR_INVALID_ARG, "evicted is NULL");
+  // kept frame f moves to its rank among the kept frames
+  ispa_attn_desc e = *desc;
+  const int S = desc->sink_frames, cb = desc->cur_begin, ce = desc->cur_end;
+  const int rank_cb = cb < S ? cb : S;
+  e.sink_frames = S;
+  e.cur_begin = rank_cb;
+  e.cur_end = rank_cb + (ce - cb);
+  e.hist_begin = e.hist_end = 0;
+  e.kv_frames = ce > S ? rank_cb + (ce - cb) : S;  // |[0, S) u [cb, ce)|
+  *evicted = e;
+  return ISPA_OK;
+}
+
+ispa_status ispa_kv_evict_history(const ispa_attn_desc *desc, const void *k, const void *v, void *k_out, void *v_out,
+                                  ispa_stream_t stream) {
+  GroupRanges g;
+  float scale;
+  ispa_status st = attn_ranges(desc, &g, &scale);
+  if (st != ISPA_OK) return st;
+  if (!ptr_ok(k) || !ptr_ok(v) || !ptr_ok(k_out) || !ptr_ok(v_out))
+    return fail(ISPA_ERR_INVALID_ARG, "k, v, k_out, v_out must be 16-byte aligned device pointers");
+  const long long esize = desc->in_dtype == ISPA_BF16 ? 2 : 4;
+  const long long row_bytes = (long long)desc->H * desc->head_dim * esize;  // a multiple of 64
+  const long long src_rows = g.Lkv;
+  const long long len0 = g.loc_end[0] - g.loc_begin[0];
+  const long long dst_rows = len0 + (g.n_loc > 1 ? g.loc_end[1] - g.loc_begin[1] : 0);
+  const long long in_bytes = desc->B * src_rows * row_bytes, out_bytes = desc->B * dst_rows * row_bytes;
+  auto overlap = [](const void *a, long long na, const void *b, long long nb) {
+    const char *x = (const char *)a, *y = (const char *)b;
+    return x < y + nb && y < x + na;
+  };
+  if (overlap(k_out, out_bytes, k, in_bytes) || overlap(k_out, out_bytes, v, in_bytes) ||
+      overlap(v_out, out_bytes, k, in_bytes) || overlap(v_out, out_bytes, v, in_bytes) ||
+      overlap(k_out, out_bytes, v_out, out_bytes))
+    return fail(ISPA_ERR_INVALID_ARG, "k_out and v_out must not overlap each other or the inputs");
+  return launch_kv_evict(desc->B, src_rows, dst_rows, g.loc_begin[0], len0, g.n_loc > 1 ? g.loc_begin[1] : 0,
+                         row_bytes, k, v, k_out, v_out, (cudaStream_t)stream);
+}
+
 }  // extern "C"

@@ -260,6 +260,31 @@ def kv_retained_fraction(x: float, hist_frac: float) -> float:
 # ---------------------------------------------------------------------------
 # post-switch L-layer  [DE-summary 2, "Speichereffiziente Inferenz"]
 # ---------------------------------------------------------------------------
+def evict_history(shape, kv: np.ndarray) -> np.ndarray:
+    """K or V of an L-layer once its historical entries are evicted: for every
+    instance, the frames of the local group (sink and current, in frame order)
+    back to back.  The selected layers drop K_hist, V_hist and run on the local
+    context alone [DE-summary 2, "Speichereffiziente Inferenz"; EN-notes, Key
+    Designs 3 and "A Worked Example"].  kv [B, kv_frames * tpf, H, d].
+    """
+    return np.ascontiguousarray(np.asarray(kv)[:, _local_rows(shape)])
+
+
+def evicted_shape(shape):
+    """Frame layout of an evicted buffer: every kept frame is renumbered by its
+    rank among the kept frames, so the sink stays [0, sink), the current chunk
+    keeps its length and starts at the number of kept frames before it, and
+    there is no history.  Its local group holds the same keys, in the same
+    order, as the local group of ``shape``, and its queries are the same.
+    """
+    import dataclasses
+    kept = sorted(set(range(shape.sink_frames)) | set(range(shape.cur_begin, shape.cur_end)))
+    rank = {f: i for i, f in enumerate(kept)}
+    cb = rank[shape.cur_begin]
+    return dataclasses.replace(shape, hist_begin=0, hist_end=0, cur_begin=cb,
+                               cur_end=cb + shape.cur_end - shape.cur_begin, kv_frames=len(kept))
+
+
 def local_projection(shape, q, k, v, W: np.ndarray, dW: np.ndarray = None, scale: float = None,
                      rows: Sequence[int] = None) -> np.ndarray:
     """Y = A_loc (W + dW): attention over sink + current only, projected with W_new = W + dW.

@@ -127,3 +127,40 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(ispa, "_lib", None)
     with pytest.raises(ImportError):
         ispa.lib()
+
+
+# ---------------------------------------------------------------- KV eviction (host side)
+@pytest.mark.parametrize("layout", [
+    dict(sink_frames=1, hist_begin=1, hist_end=4, cur_begin=4, cur_end=5, kv_frames=5),   # sink | history | current
+    dict(sink_frames=2, hist_begin=2, hist_end=5, cur_begin=5, cur_end=8, kv_frames=10),  # frames after the chunk
+    dict(sink_frames=0, hist_begin=0, hist_end=3, cur_begin=3, cur_end=5, kv_frames=5),   # no sink
+    dict(sink_frames=3, hist_begin=0, hist_end=0, cur_begin=2, cur_end=4, kv_frames=4),   # current overlaps the sink
+    dict(sink_frames=4, hist_begin=0, hist_end=0, cur_begin=4, cur_end=6, kv_frames=6),   # current right after the sink
+    dict(sink_frames=5, hist_begin=0, hist_end=0, cur_begin=1, cur_end=3, kv_frames=6),   # current inside the sink
+])
+def test_kv_evicted_desc_matches_oracle_layout(layout):
+    import synth_inputs as si
+    from oracle import ispa_oracle as orc
+    d = _desc(**layout)
+    e = ispa.ispa_kv_evicted_desc(d)
+    sh = si.AttnShape(B=d.B, H=d.H, d=d.head_dim, tpf=d.tokens_per_frame, **layout)
+    es = orc.evicted_shape(sh)
+    got = (e.sink_frames, e.hist_begin, e.hist_end, e.cur_begin, e.cur_end, e.kv_frames)
+    assert got == (es.sink_frames, es.hist_begin, es.hist_end, es.cur_begin, es.cur_end, es.kv_frames)
+    assert (e.B, e.H, e.head_dim, e.tokens_per_frame, e.in_dtype) == (d.B, d.H, d.head_dim, d.tokens_per_frame,
+                                                                       d.in_dtype)
+
+
+def test_kv_eviction_validation():
+    L = ispa.lib()
+    bad = _desc(cur_begin=5, cur_end=5)
+    out = ispa.AttnDesc()
+    assert L.ispa_kv_evicted_desc(ctypes.byref(bad), ctypes.byref(out)) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_kv_evicted_desc(ctypes.byref(_desc()), None) == ispa.ISPA_ERR_INVALID_ARG
+    d = _desc()
+    assert L.ispa_kv_evict_history(ctypes.byref(d), FAKE, FAKE, None, FAKE, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_kv_evict_history(ctypes.byref(d), FAKE, FAKE, FAKE + 8, FAKE, None) == ispa.ISPA_ERR_INVALID_ARG
+    # outputs overlapping the inputs are rejected (here k_out == k)
+    assert L.ispa_kv_evict_history(ctypes.byref(d), FAKE, FAKE + (1 << 24), FAKE, FAKE + (1 << 26),
+                                   None) == ispa.ISPA_ERR_INVALID_ARG
+    assert "overlap" in L.ispa_last_error().decode()

@@ -154,3 +154,87 @@ def test_bf16_full_size_1p3b_sampled_rows():
     # unwritten outputs would still hold NaN
     for n in ("loc", "hist", "full"):
         assert not np.isnan(O[n]).any() and not np.isnan(L[n]).any()
+
+
+# ---------------------------------------------------------------- KV eviction of post-switch L-layers
+EVICT_LAYOUTS = [
+    dict(sink_frames=2, hist_begin=2, hist_end=6, cur_begin=6, cur_end=8, kv_frames=9),  # sink | history | current | spare
+    dict(sink_frames=0, hist_begin=0, hist_end=3, cur_begin=3, cur_end=5, kv_frames=5),  # no sink
+    dict(sink_frames=5, hist_begin=0, hist_end=0, cur_begin=1, cur_end=3, kv_frames=6),  # current inside the sink
+]
+
+
+@pytest.mark.parametrize("layout", EVICT_LAYOUTS)
+@pytest.mark.parametrize("in_dt", [ispa.ISPA_BF16, ispa.ISPA_F32])
+def test_kv_evict_history_bit_exact(layout, in_dt):
+    sh = si.AttnShape(B=2, H=3, d=128 if in_dt == ispa.ISPA_BF16 else 64, tpf=37, **layout)
+    data = si.iid_qkv(sh, "bf16" if in_dt == ispa.ISPA_BF16 else "f32", ("gpu", "evict"))
+    tin = torch.bfloat16 if in_dt == ispa.ISPA_BF16 else torch.float32
+    k, v = dev(data["k"], tin), dev(data["v"], tin)
+    desc = ispa.attn_desc(sh, in_dt, ispa.ISPA_F32)
+    ed = ispa.ispa_kv_evicted_desc(desc)
+    es = orc.evicted_shape(sh)
+    assert (ed.kv_frames, ed.sink_frames, ed.cur_begin, ed.cur_end) == (es.kv_frames, es.sink_frames, es.cur_begin,
+                                                                         es.cur_end)
+    shape_out = (sh.B, ed.kv_frames * sh.tpf, sh.H, sh.d)
+    k_out, v_out = nan_like(shape_out, tin), nan_like(shape_out, tin)
+    ispa.ispa_kv_evict_history(desc, k, v, k_out, v_out)
+    torch.cuda.synchronize()
+    for got, name in ((k_out, "k"), (v_out, "v")):
+        ref = orc.evict_history(sh, data[name])
+        assert np.array_equal(host(got), ref.astype(np.float64)), name
+
+
+@pytest.mark.parametrize("layout", EVICT_LAYOUTS[:2])
+def test_attention_after_eviction_matches_oracle(layout):
+    """The post-switch call on the evicted buffers attends to the same local
+    entries: its local output and LSE match the oracle of the original layout."""
+    sh = si.AttnShape(B=2, H=2, d=128, tpf=45, **layout)
+    data = si.iid_qkv(sh, "bf16", ("gpu", "evict-attn"))
+    desc = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_F32)
+    ed = ispa.ispa_kv_evicted_desc(desc)
+    es = orc.evicted_shape(sh)
+    k, v = dev(data["k"], torch.bfloat16), dev(data["v"], torch.bfloat16)
+    shape_out = (sh.B, ed.kv_frames * sh.tpf, sh.H, sh.d)
+    k_ev, v_ev = nan_like(shape_out, torch.bfloat16), nan_like(shape_out, torch.bfloat16)
+    ispa.ispa_kv_evict_history(desc, k, v, k_ev, v_ev)
+    del k, v
+    q = dev(data["q"], torch.bfloat16)
+    o = nan_like((sh.B, sh.Lq, sh.H, sh.d), torch.float32)
+    lse = nan_like((sh.B, sh.Lq, sh.H), torch.float32)
+    ws = torch.empty(max(1, ispa.ispa_attn_split_workspace_bytes(ed)), dtype=torch.uint8, device="cuda")
+    ispa.ispa_attn_split(ed, q, k_ev, v_ev, o, lse, None, None, None, None, workspace=ws)
+    ispa.ispa_check_device_error()
+    torch.cuda.synchronize()
+    ref = orc.split_attention(sh, data["q"], data["k"], data["v"])
+    assert es.Lq == sh.Lq
+    assert max_over_rms(host(o), ref["O_loc"]) <= 1e-2
+    assert_lse(host(lse), ref["L_loc"], 1e-3)
+
+
+def test_kv_eviction_releases_the_history_bytes():
+    """Real eviction: once the caller frees the original K/V, the device
+    allocator holds exactly the kept frames (sizes chosen as multiples of the
+    allocator's 512-byte granule)."""
+    layout = EVICT_LAYOUTS[0]
+    sh = si.AttnShape(B=2, H=4, d=128, tpf=64, **layout)
+    desc = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_BF16)
+    ed = ispa.ispa_kv_evicted_desc(desc)
+    torch.cuda.synchronize()
+    base = torch.cuda.memory_allocated()
+    full = (sh.B, sh.kv_frames * sh.tpf, sh.H, sh.d)
+    k = torch.ones(full, dtype=torch.bfloat16, device="cuda")
+    v = torch.ones(full, dtype=torch.bfloat16, device="cuda")
+    before = torch.cuda.memory_allocated() - base
+    kept = (sh.B, ed.kv_frames * sh.tpf, sh.H, sh.d)
+    k_ev = torch.empty(kept, dtype=torch.bfloat16, device="cuda")
+    v_ev = torch.empty(kept, dtype=torch.bfloat16, device="cuda")
+    ispa.ispa_kv_evict_history(desc, k, v, k_ev, v_ev)
+    torch.cuda.synchronize()
+    del k, v
+    after = torch.cuda.memory_allocated() - base
+    row_bytes = sh.H * sh.d * 2
+    freed_per_tensor = sh.B * (sh.kv_frames - ed.kv_frames) * sh.tpf * row_bytes
+    assert before == 2 * sh.B * sh.kv_frames * sh.tpf * row_bytes
+    assert before - after == 2 * freed_per_tensor
+    assert torch.all(k_ev == 1) and torch.all(v_ev == 1)

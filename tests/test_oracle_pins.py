@@ -375,6 +375,33 @@ def test_local_projection_definition():
     assert np.allclose(Y[0], orc.heads_to_rows(out["O_loc"]) @ (W + dW), atol=1e-13)
 
 
+@pytest.mark.parametrize("layout", [
+    dict(sink_frames=2, hist_begin=2, hist_end=6, cur_begin=6, cur_end=8, kv_frames=9),
+    dict(sink_frames=0, hist_begin=0, hist_end=3, cur_begin=3, cur_end=5, kv_frames=5),
+    dict(sink_frames=3, hist_begin=0, hist_end=0, cur_begin=2, cur_end=4, kv_frames=4),
+    dict(sink_frames=5, hist_begin=0, hist_end=0, cur_begin=1, cur_end=3, kv_frames=6),
+])
+def test_eviction_keeps_exactly_the_local_frames(layout):
+    """Evicting history keeps the sink and current frames, in frame order, and
+    drops everything else [DE-summary 2, "Speichereffiziente Inferenz"]: checked
+    frame by frame, and local attention over the evicted buffer equals local
+    attention over the original (same keys, same order: identical arithmetic)."""
+    sh = si.AttnShape(B=2, H=2, d=8, tpf=3, **layout)
+    d = si.iid_qkv(sh, "f32", ("pin", "evict"))
+    kept_frames = [f for f in range(sh.kv_frames) if f < sh.sink_frames or sh.cur_begin <= f < sh.cur_end]
+    for name in ("k", "v"):
+        ev = orc.evict_history(sh, d[name])
+        brute = np.concatenate([d[name][:, f * sh.tpf:(f + 1) * sh.tpf] for f in kept_frames], axis=1)
+        assert np.array_equal(ev, brute)
+    es = orc.evicted_shape(sh)
+    assert es.kv_frames == len(kept_frames) and es.hist_end == es.hist_begin
+    ek, ev_ = orc.evict_history(sh, d["k"]), orc.evict_history(sh, d["v"])
+    a = orc.split_attention(sh, d["q"], d["k"], d["v"])
+    b = orc.split_attention(es, d["q"], ek, ev_)
+    assert np.array_equal(a["O_loc"], b["O_loc"]) and np.array_equal(a["L_loc"], b["L_loc"])
+    assert np.all(np.isneginf(b["L_hist"]))
+
+
 # ---------------------------------------------------------------------------
 # mutation tests: plausible mistakes planted in copies of oracle functions
 # ---------------------------------------------------------------------------
