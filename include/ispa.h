@@ -305,6 +305,37 @@ ispa_status ispa_kv_evicted_desc(const ispa_attn_desc *desc, ispa_attn_desc *evi
 ispa_status ispa_kv_evict_history(const ispa_attn_desc *desc, const void *k, const void *v,
                                   void *k_out, void *v_out, ispa_stream_t stream);
 
+/*
+ * ispa_kv_restore: the inverse of ispa_kv_evict_history, for a layer that
+ * goes back to full context when warmup is re-entered (recalibration below).
+ * Copies the kept frames from k_ev, v_ev (layout of the evicted desc) to their
+ * places in k_full, v_full (layout of desc, the descriptor the eviction used),
+ * bit for bit; every other row of k_full and v_full is left as it is (the
+ * history that the new warmup fills).  Same pointer rules as
+ * ispa_kv_evict_history.  Asynchronous.
+ */
+ispa_status ispa_kv_restore(const ispa_attn_desc *desc, const void *k_ev, const void *v_ev,
+                            void *k_full, void *v_full, ispa_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* Recalibration                                                              */
+/* ------------------------------------------------------------------------- */
+/*
+ * Warmup can be re-entered after a major scene change, refreshing both the
+ * layer selection and the weight corrections [EN-notes, Key Designs 3].  The
+ * pages give no detector, so the trigger is the caller's.  Recalibration with
+ * this library: for every layer ispa_stats_reset; the L-layers back to full
+ * context (ispa_kv_restore into full-layout buffers, projection with W again);
+ * a new warmup (ispa_attn_split, ispa_accum_stats); at its end the transition
+ * as the first time (ispa_ridge_solve per layer, ispa_select_layers,
+ * ispa_absorb_weight, ispa_kv_evict_history).
+ *
+ * ispa_stats_reset: G [D, D] and C [D, Dout] (fp32) and r2 (one double) back
+ * to zero on stream, so that the next warmup accumulates from nothing.
+ * Asynchronous; ISPA_ERR_INVALID_ARG for D or Dout < 1 or a NULL pointer.
+ */
+ispa_status ispa_stats_reset(int D, int Dout, float *G, float *C, double *r2, ispa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

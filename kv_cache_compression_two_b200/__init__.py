@@ -31,7 +31,8 @@ STATUS_NAMES = {0: "ISPA_OK", 1: "ISPA_ERR_INVALID_ARG", 2: "ISPA_ERR_UNSUPPORTE
 EXPORTED = ("ispa_version", "ispa_last_error", "ispa_launch_count", "ispa_check_device_error", "ispa_attn_split_workspace_bytes", "ispa_attn_split", "ispa_lse_merge",
             "ispa_accum_stats_workspace_bytes", "ispa_accum_stats", "ispa_ridge_workspace_bytes", "ispa_ridge_solve",
             "ispa_select_layers", "ispa_absorb_weight", "ispa_attn_local_proj_workspace_bytes",
-            "ispa_attn_local_proj", "ispa_ridge_solve_noalloc", "ispa_kv_evicted_desc", "ispa_kv_evict_history")
+            "ispa_attn_local_proj", "ispa_ridge_solve_noalloc", "ispa_kv_evicted_desc", "ispa_kv_evict_history",
+            "ispa_kv_restore", "ispa_stats_reset")
 RIDGE_NOALLOC_MAX_D = RIDGE_NOALLOC_MAX_DOUT = 1024
 
 
@@ -87,6 +88,8 @@ def lib() -> ctypes.CDLL:
         "ispa_attn_local_proj": (_ci, [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _ci, _vp, _ci, _vp, _sz, _vp]),
         "ispa_kv_evicted_desc": (_ci, [ctypes.POINTER(AttnDesc), ctypes.POINTER(AttnDesc)]),
         "ispa_kv_evict_history": (_ci, [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp]),
+        "ispa_kv_restore": (_ci, [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp]),
+        "ispa_stats_reset": (_ci, [_ci, _ci, _vp, _vp, _vp, _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -239,6 +242,15 @@ def ispa_kv_evicted_desc(desc: AttnDesc) -> AttnDesc:
 def ispa_kv_evict_history(desc: AttnDesc, k, v, k_out, v_out, stream=None) -> None:
     _check(lib().ispa_kv_evict_history(ctypes.byref(desc), _ptr(k), _ptr(v), _ptr(k_out), _ptr(v_out),
                                        _stream(stream)))
+
+
+def ispa_kv_restore(desc: AttnDesc, k_ev, v_ev, k_full, v_full, stream=None) -> None:
+    _check(lib().ispa_kv_restore(ctypes.byref(desc), _ptr(k_ev), _ptr(v_ev), _ptr(k_full), _ptr(v_full),
+                                 _stream(stream)))
+
+
+def ispa_stats_reset(D: int, Dout: int, G, C, r2, stream=None) -> None:
+    _check(lib().ispa_stats_reset(D, Dout, _ptr(G), _ptr(C), _ptr(r2), _stream(stream)))
 
 
 lib()

@@ -171,6 +171,35 @@ ispa_status attn_ranges(const ispa_attn_desc *d, GroupRanges *g, float *scale) {
 
 bool ptr_ok(const void *p) { return p != nullptr && aligned16(p); }
 
+// Eviction (gather: full layout of desc -> compact layout of the evicted desc)
+// and restore (scatter back).  Validates desc, alignment and overlap.
+ispa_status kv_remap(const ispa_attn_desc *desc, const void *k, const void *v, void *k_out, void *v_out, bool gather,
+                     cudaStream_t s) {
+  GroupRanges g;
+  float scale;
+  ispa_status st = attn_ranges(desc, &g, &scale);
+  if (st != ISPA_OK) return st;
+  if (!ptr_ok(k) || !ptr_ok(v) || !ptr_ok(k_out) || !ptr_ok(v_out))
+    return fail(ISPA_ERR_INVALID_ARG, "the four K/V pointers must be 16-byte aligned device pointers");
+  const long long esize = desc->in_dtype == ISPA_BF16 ? 2 : 4;
+  const long long row_bytes = (long long)desc->H * desc->head_dim * esize;  // a multiple of 64
+  const long long full_rows = g.Lkv;
+  const long long len0 = g.loc_end[0] - g.loc_begin[0];
+  const long long kept_rows = len0 + (g.n_loc > 1 ? g.loc_end[1] - g.loc_begin[1] : 0);
+  const long long full_bytes = desc->B * full_rows * row_bytes, kept_bytes = desc->B * kept_rows * row_bytes;
+  const long long in_bytes = gather ? full_bytes : kept_bytes, out_bytes = gather ? kept_bytes : full_bytes;
+  auto overlap = [](const void *a, long long na, const void *b, long long nb) {
+    const char *x = (const char *)a, *y = (const char *)b;
+    return x < y + nb && y < x + na;
+  };
+  if (overlap(k_out, out_bytes, k, in_bytes) || overlap(k_out, out_bytes, v, in_bytes) ||
+      overlap(v_out, out_bytes, k, in_bytes) || overlap(v_out, out_bytes, v, in_bytes) ||
+      overlap(k_out, out_bytes, v_out, out_bytes))
+    return fail(ISPA_ERR_INVALID_ARG, "the outputs must not overlap each other or the inputs");
+  return launch_kv_remap(desc->B, full_rows, kept_rows, g.loc_begin[0], len0, g.n_loc > 1 ? g.loc_begin[1] : 0,
+                         row_bytes, gather, k, v, k_out, v_out, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -394,28 +423,22 @@ ispa_status ispa_kv_evicted_desc(const ispa_attn_desc *desc, ispa_attn_desc *evi
 
 ispa_status ispa_kv_evict_history(const ispa_attn_desc *desc, const void *k, const void *v, void *k_out, void *v_out,
                                   ispa_stream_t stream) {
-  GroupRanges g;
-  float scale;
-  ispa_status st = attn_ranges(desc, &g, &scale);
-  if (st != ISPA_OK) return st;
-  if (!ptr_ok(k) || !ptr_ok(v) || !ptr_ok(k_out) || !ptr_ok(v_out))
-    return fail(ISPA_ERR_INVALID_ARG, "k, v, k_out, v_out must be 16-byte aligned device pointers");
-  const long long esize = desc->in_dtype == ISPA_BF16 ? 2 : 4;
-  const long long row_bytes = (long long)desc->H * desc->head_dim * esize;  // a multiple of 64
-  const long long src_rows = g.Lkv;
-  const long long len0 = g.loc_end[0] - g.loc_begin[0];
-  const long long dst_rows = len0 + (g.n_loc > 1 ? g.loc_end[1] - g.loc_begin[1] : 0);
-  const long long in_bytes = desc->B * src_rows * row_bytes, out_bytes = desc->B * dst_rows * row_bytes;
-  auto overlap = [](const void *a, long long na, const void *b, long long nb) {
-    const char *x = (const char *)a, *y = (const char *)b;
-    return x < y + nb && y < x + na;
-  };
-  if (overlap(k_out, out_bytes, k, in_bytes) || overlap(k_out, out_bytes, v, in_bytes) ||
-      overlap(v_out, out_bytes, k, in_bytes) || overlap(v_out, out_bytes, v, in_bytes) ||
-      overlap(k_out, out_bytes, v_out, out_bytes))
-    return fail(ISPA_ERR_INVALID_ARG, "k_out and v_out must not overlap each other or the inputs");
-  return launch_kv_evict(desc->B, src_rows, dst_rows, g.loc_begin[0], len0, g.n_loc > 1 ? g.loc_begin[1] : 0,
-                         row_bytes, k, v, k_out, v_out, (cudaStream_t)stream);
+  return kv_remap(desc, k, v, k_out, v_out, true, (cudaStream_t)stream);
+}
+
+ispa_status ispa_kv_restore(const ispa_attn_desc *desc, const void *k_ev, const void *v_ev, void *k_full,
+                            void *v_full, ispa_stream_t stream) {
+  return kv_remap(desc, k_ev, v_ev, k_full, v_full, false, (cudaStream_t)stream);
+}
+
+ispa_status ispa_stats_reset(int D, int Dout, float *G, float *C, double *r2, ispa_stream_t stream) {
+  if (D < 1 || Dout < 1) return fail(ISPA_ERR_INVALID_ARG, "D and Dout must be >= 1");
+  if (!G || !C || !r2) return fail(ISPA_ERR_INVALID_ARG, "G, C and r2 must be device pointers");
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(G, 0, (size_t)D * D * sizeof(float), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(C, 0, (size_t)D * Dout * sizeof(float), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(r2, 0, sizeof(double), s);
+  return cuda_status(e, "statistics reset");
 }
 
 }  // extern "C"

@@ -186,33 +186,41 @@ ispa_status launch_select(int N, const double *eps, int K, unsigned char *is_loc
 }
 
 // ---------------------------------------------------------------------------
-// KV eviction of an L-layer: the kept token rows of every instance, back to
-// back, 16 bytes per thread and iteration.
+// KV eviction of an L-layer and its inverse: the kept token rows of every
+// instance, back to back in the compact layout; 16 bytes per thread and
+// iteration.  Compact row r of an instance is full row b0 + r for r < len0,
+// b1 + r - len0 after.  gather: compact <- full; otherwise full <- compact.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) kv_evict_kernel(int B, long long src_rows, long long dst_rows, long long b0,
-                                                       long long len0, long long b1, int vec_per_row,
+__global__ void __launch_bounds__(256) kv_remap_kernel(int B, long long full_rows, long long kept_rows, long long b0,
+                                                       long long len0, long long b1, int vec_per_row, int gather,
                                                        const uint4 *__restrict__ k, const uint4 *__restrict__ v,
                                                        uint4 *__restrict__ ko, uint4 *__restrict__ vo) {
-  const long long per_inst = dst_rows * vec_per_row;
+  const long long per_inst = kept_rows * vec_per_row;
   const long long n = (long long)B * per_inst;
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
     const long long b = e / per_inst, rem = e - b * per_inst;
     const long long r = rem / vec_per_row, c = rem - r * vec_per_row;
-    const long long sr = r < len0 ? b0 + r : b1 + (r - len0);
-    const long long si = (b * src_rows + sr) * vec_per_row + c;
-    ko[e] = k[si];
-    vo[e] = v[si];
+    const long long fr = r < len0 ? b0 + r : b1 + (r - len0);
+    const long long fi = (b * full_rows + fr) * vec_per_row + c;
+    if (gather) {
+      ko[e] = k[fi];
+      vo[e] = v[fi];
+    } else {
+      ko[fi] = k[e];
+      vo[fi] = v[e];
+    }
   }
 }
 
-ispa_status launch_kv_evict(int B, long long src_rows, long long dst_rows, long long b0, long long len0, long long b1,
-                            long long row_bytes, const void *k, const void *v, void *k_out, void *v_out,
-                            cudaStream_t s) {
-  if (B == 0 || dst_rows == 0) return ISPA_OK;
-  kv_evict_kernel<<<sm_count() * 4, 256, 0, s>>>(B, src_rows, dst_rows, b0, len0, b1, (int)(row_bytes / 16),
-                                                (const uint4 *)k, (const uint4 *)v, (uint4 *)k_out, (uint4 *)v_out);
+ispa_status launch_kv_remap(int B, long long full_rows, long long kept_rows, long long b0, long long len0,
+                            long long b1, long long row_bytes, bool gather, const void *k, const void *v,
+                            void *k_out, void *v_out, cudaStream_t s) {
+  if (B == 0 || kept_rows == 0) return ISPA_OK;
+  kv_remap_kernel<<<sm_count() * 4, 256, 0, s>>>(B, full_rows, kept_rows, b0, len0, b1, (int)(row_bytes / 16),
+                                                gather ? 1 : 0, (const uint4 *)k, (const uint4 *)v, (uint4 *)k_out,
+                                                (uint4 *)v_out);
   note_launch();
-  return cuda_status(cudaGetLastError(), "kv eviction launch");
+  return cuda_status(cudaGetLastError(), "kv remap launch");
 }
 
 }  // namespace ispa

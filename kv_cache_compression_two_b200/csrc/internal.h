@@ -40,12 +40,13 @@ struct GroupRanges {
 // ---- launchers (each returns ISPA_OK or ISPA_ERR_CUDA) ----
 ispa_status launch_lse_merge(int rows, int H, int d, ispa_dtype dt, const void *oa, const float *la,
                              const void *ob, const float *lb, void *oo, float *lo, cudaStream_t s);
-// Copies, per instance, the token rows [b0, b0 + len0) and then
-// [b1, b1 + dst_rows - len0) of k and v (src_rows rows per instance, row_bytes
-// bytes each, a multiple of 16) into k_out, v_out (dst_rows rows per instance).
-ispa_status launch_kv_evict(int B, long long src_rows, long long dst_rows, long long b0, long long len0, long long b1,
-                            long long row_bytes, const void *k, const void *v, void *k_out, void *v_out,
-                            cudaStream_t s);
+// Moves, per instance, the full-layout token rows [b0, b0 + len0) and then
+// [b1, b1 + kept_rows - len0) (full_rows rows per instance, row_bytes bytes
+// each, a multiple of 16) to the compact layout of kept_rows rows (gather), or
+// back from it (scatter; the other full rows are left as they are).
+ispa_status launch_kv_remap(int B, long long full_rows, long long kept_rows, long long b0, long long len0,
+                            long long b1, long long row_bytes, bool gather, const void *k, const void *v,
+                            void *k_out, void *v_out, cudaStream_t s);
 ispa_status launch_select(int N, const double *eps, int K, unsigned char *is_local, int *idx,
                           cudaStream_t s);
 ispa_status launch_absorb_weight(int D, int Dout, const void *W, ispa_dtype wdt, const float *dW,

@@ -270,6 +270,17 @@ def evict_history(shape, kv: np.ndarray) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(kv)[:, _local_rows(shape)])
 
 
+def restore_history(shape, kv_evicted: np.ndarray, kv_full: np.ndarray) -> np.ndarray:
+    """The kept frames of an evicted buffer put back at their places in a
+    full-layout buffer (every other row of ``kv_full`` unchanged), for a layer
+    that returns to full context when warmup is re-entered [EN-notes, Key
+    Designs 3].  kv_evicted [B, kept * tpf, H, d], kv_full [B, kv_frames * tpf, H, d].
+    """
+    out = np.array(kv_full, copy=True)
+    out[:, _local_rows(shape)] = kv_evicted
+    return out
+
+
 def evicted_shape(shape):
     """Frame layout of an evicted buffer: every kept frame is renumbered by its
     rank among the kept frames, so the sink stays [0, sink), the current chunk

@@ -164,3 +164,14 @@ def test_kv_eviction_validation():
     assert L.ispa_kv_evict_history(ctypes.byref(d), FAKE, FAKE + (1 << 24), FAKE, FAKE + (1 << 26),
                                    None) == ispa.ISPA_ERR_INVALID_ARG
     assert "overlap" in L.ispa_last_error().decode()
+
+
+def test_recalibration_validation():
+    L = ispa.lib()
+    assert L.ispa_stats_reset(0, 4, FAKE, FAKE, FAKE, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_stats_reset(4, 4, None, FAKE, FAKE, None) == ispa.ISPA_ERR_INVALID_ARG
+    d = _desc()
+    assert L.ispa_kv_restore(ctypes.byref(d), FAKE, None, FAKE, FAKE, None) == ispa.ISPA_ERR_INVALID_ARG
+    bad = _desc(cur_begin=5, cur_end=5)
+    assert L.ispa_kv_restore(ctypes.byref(bad), FAKE, FAKE, FAKE + (1 << 24), FAKE + (1 << 26),
+                             None) == ispa.ISPA_ERR_INVALID_ARG

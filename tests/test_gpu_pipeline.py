@@ -134,3 +134,114 @@ def test_reduced_model_selection_matches_oracle():
           f"max rel eps dev {max(rel):.3e}")
     assert gap > 2 * max(rel), "selection boundary is a tie within the propagated error"
     assert idx.cpu().numpy().tolist() == ref_idx.tolist()
+
+
+# ---------------------------------------------------------------- recalibration
+def _warm(layers_rows, Ws, G, C, r2, ws):
+    for (chunks_loc, chunks_full), W, g, c, r in zip(layers_rows, Ws, G, C, r2):
+        D, Dout = W.shape
+        for a_loc, a_full in zip(chunks_loc, chunks_full):
+            ispa.ispa_accum_stats(a_loc.shape[0], D, Dout, dev(a_loc), dev(a_full), dev(W), g, c, r,
+                                  ispa.ISPA_PREC_TF32, ws)
+
+
+def _transition(Ws, G, C, r2, K):
+    eps = torch.zeros(len(Ws), dtype=torch.float64, device="cuda")
+    dWs = []
+    for i, W in enumerate(Ws):
+        D, Dout = W.shape
+        dW = torch.empty((D, Dout), device="cuda")
+        rws = torch.empty(ispa.ispa_ridge_workspace_bytes(D, Dout), dtype=torch.uint8, device="cuda")
+        ispa.ispa_ridge_solve(D, Dout, G[i], C[i], r2[i], 1e-3, True, 0, dW, eps[i:i + 1], rws)
+        dWs.append(dW)
+    mask = torch.zeros(len(Ws), dtype=torch.uint8, device="cuda")
+    idx = torch.zeros(K, dtype=torch.int32, device="cuda")
+    ispa.ispa_select_layers(len(Ws), eps, K, mask, idx)
+    ispa.ispa_check_device_error()
+    return [host(d) for d in dWs], host(eps), mask.cpu().numpy(), idx.cpu().numpy()
+
+
+def test_recalibration_equals_a_fresh_warmup():
+    """Re-entering warmup after a scene change [EN-notes, Key Designs 3]: after
+    ispa_stats_reset and a warmup on the new scene only, the statistics, the
+    corrections, the errors and the selection are those of a fresh warmup on
+    the new scene, and they match the oracle on that scene."""
+    N, D, T, K = 4, 256, 384, 2
+    g = np.random.default_rng(21)
+
+    def scene(seed):
+        rows = []
+        r = np.random.default_rng(seed)
+        for layer in range(N):  # a linear part the correction can absorb, and a residual it cannot
+            mix = r.standard_normal((D, D)) * 0.1 / math.sqrt(D)
+            noise = 0.05 * (1 + (layer * 5 + seed) % N)
+            loc = [r.standard_normal((T, D)).astype(np.float32) for _ in range(2)]
+            full = [(a + a @ mix + noise * r.standard_normal((T, D))).astype(np.float32) for a in loc]
+            rows.append((loc, full))
+        return rows
+
+    Ws = [(g.standard_normal((D, D)) / math.sqrt(D)).astype(np.float32) for _ in range(N)]
+    scene1, scene2 = scene(1), scene(2)
+    ws = torch.empty(ispa.ispa_accum_stats_workspace_bytes(T, D, D, ispa.ISPA_PREC_TF32), dtype=torch.uint8,
+                     device="cuda")
+
+    def fresh():
+        return ([torch.zeros((D, D), device="cuda") for _ in range(N)],
+                [torch.zeros((D, D), device="cuda") for _ in range(N)],
+                [torch.zeros(1, dtype=torch.float64, device="cuda") for _ in range(N)])
+
+    G, C, r2 = fresh()
+    _warm(scene1, Ws, G, C, r2, ws)
+    first = _transition(Ws, G, C, r2, K)
+    for i in range(N):  # the trigger: back to warmup
+        ispa.ispa_stats_reset(D, D, G[i], C[i], r2[i])
+    _warm(scene2, Ws, G, C, r2, ws)
+    recal = _transition(Ws, G, C, r2, K)
+
+    G2, C2, r22 = fresh()
+    _warm(scene2, Ws, G2, C2, r22, ws)
+    ref = _transition(Ws, G2, C2, r22, K)
+    torch.cuda.synchronize()
+    for i in range(N):
+        assert torch.equal(torch.triu(G[i]), torch.triu(G2[i])) and torch.equal(C[i], C2[i])
+        assert abs(r2[i].item() - r22[i].item()) <= 1e-12 * r22[i].item()
+        assert rel_fro(recal[0][i], ref[0][i]) <= 1e-5
+    # epsilon: run to run only the summation order of the solve's atomics differs
+    assert np.allclose(recal[1], ref[1], rtol=0, atol=1e-7 * max(r.item() for r in r22))
+    assert np.array_equal(recal[2], ref[2]) and np.array_equal(recal[3], ref[3])
+    assert not np.allclose(first[1], recal[1])  # the scenes differ, so the errors moved ...
+    assert not np.array_equal(first[2], recal[2])  # ... and so does the selection
+
+    # against the oracle on the new scene alone
+    eps_ref = []
+    for i, ((loc, full), W) in enumerate(zip(scene2, Ws)):
+        A_loc = np.concatenate(loc).astype(np.float64)
+        A_full = np.concatenate(full).astype(np.float64)
+        Gr, Cr, r2r = orc.absorption_stats(A_loc, A_full, W.astype(np.float64))
+        lam = float(np.float32(orc.ridge_lambda(Gr, 1e-3, True)))
+        dWr = orc.ridge_solve(Gr, Cr, lam)
+        assert rel_fro(recal[0][i], dWr) <= 1e-2
+        eps_ref.append(orc.eps_from_stats(Gr, Cr, r2r, dWr))
+    mask_ref, idx_ref = orc.select_layers(eps_ref, K)
+    assert np.array_equal(recal[2], mask_ref) and np.array_equal(recal[3], idx_ref)
+
+
+def test_kv_restore_inverts_eviction():
+    sh = si.AttnShape(B=2, H=2, d=128, tpf=40, sink_frames=2, hist_begin=2, hist_end=6, cur_begin=6, cur_end=8,
+                      kv_frames=9)
+    data = si.iid_qkv(sh, "bf16", ("gpu", "restore"))
+    desc = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_BF16)
+    ed = ispa.ispa_kv_evicted_desc(desc)
+    k, v = dev(data["k"], torch.bfloat16), dev(data["v"], torch.bfloat16)
+    kept = (sh.B, ed.kv_frames * sh.tpf, sh.H, sh.d)
+    k_ev, v_ev = torch.empty(kept, dtype=torch.bfloat16, device="cuda"), torch.empty(kept, dtype=torch.bfloat16,
+                                                                                        device="cuda")
+    ispa.ispa_kv_evict_history(desc, k, v, k_ev, v_ev)
+    full = tuple(k.shape)
+    k_back = torch.full(full, 3.0, dtype=torch.bfloat16, device="cuda")
+    v_back = torch.full(full, 3.0, dtype=torch.bfloat16, device="cuda")
+    ispa.ispa_kv_restore(desc, k_ev, v_ev, k_back, v_back)
+    torch.cuda.synchronize()
+    sentinel = np.full(full, 3.0)
+    assert np.array_equal(host(k_back), orc.restore_history(sh, orc.evict_history(sh, data["k"]), sentinel))
+    assert np.array_equal(host(v_back), orc.restore_history(sh, orc.evict_history(sh, data["v"]), sentinel))

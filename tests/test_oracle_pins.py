@@ -402,6 +402,19 @@ def test_eviction_keeps_exactly_the_local_frames(layout):
     assert np.all(np.isneginf(b["L_hist"]))
 
 
+def test_restore_is_the_inverse_of_eviction():
+    sh = si.AttnShape(B=2, H=2, d=8, tpf=3, sink_frames=2, hist_begin=2, hist_end=6, cur_begin=6, cur_end=8,
+                      kv_frames=9)
+    d = si.iid_qkv(sh, "f32", ("pin", "restore"))
+    sentinel = np.full_like(d["k"], 7.0)
+    back = orc.restore_history(sh, orc.evict_history(sh, d["k"]), sentinel)
+    local = np.zeros(sh.kv_frames * sh.tpf, bool)
+    for f in list(range(sh.sink_frames)) + list(range(sh.cur_begin, sh.cur_end)):
+        local[f * sh.tpf:(f + 1) * sh.tpf] = True
+    assert np.array_equal(back[:, local], d["k"][:, local])
+    assert np.all(back[:, ~local] == 7.0)
+
+
 # ---------------------------------------------------------------------------
 # mutation tests: plausible mistakes planted in copies of oracle functions
 # ---------------------------------------------------------------------------
