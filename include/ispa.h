@@ -82,6 +82,19 @@ uint64_t ispa_launch_count(void);
  */
 ispa_status ispa_check_device_error(ispa_stream_t stream, int *detail);
 
+/*
+ * Failure-detection self-test.  Launches one CTA whose thread waits, through
+ * the bounded wait that every kernel of this library uses for its hand-offs,
+ * on a shared-memory mbarrier that nothing ever completes, with the time limit
+ * wait_ns (1 ms to 10 s).  When the limit passes it records ISPA_ERR_TIMEOUT
+ * with the site ISPA_SELFTEST_SITE in the device error word — what a kernel
+ * whose peer role never arrives does — and returns; nothing faults or traps,
+ * so ispa_check_device_error then reports the timeout and the context stays
+ * usable.  Asynchronous; ISPA_ERR_INVALID_ARG for wait_ns out of range.
+ */
+#define ISPA_SELFTEST_SITE 999
+ispa_status ispa_selftest_wait_timeout(long long wait_ns, ispa_stream_t stream);
+
 /* ------------------------------------------------------------------------- */
 /* Two-group attention                                                        */
 /* ------------------------------------------------------------------------- */

@@ -32,7 +32,7 @@ EXPORTED = ("ispa_version", "ispa_last_error", "ispa_launch_count", "ispa_check_
             "ispa_accum_stats_workspace_bytes", "ispa_accum_stats", "ispa_ridge_workspace_bytes", "ispa_ridge_solve",
             "ispa_select_layers", "ispa_absorb_weight", "ispa_attn_local_proj_workspace_bytes",
             "ispa_attn_local_proj", "ispa_ridge_solve_noalloc", "ispa_kv_evicted_desc", "ispa_kv_evict_history",
-            "ispa_kv_restore", "ispa_stats_reset")
+            "ispa_kv_restore", "ispa_stats_reset", "ispa_selftest_wait_timeout")
 RIDGE_NOALLOC_MAX_D = RIDGE_NOALLOC_MAX_DOUT = 1024
 
 
@@ -90,6 +90,7 @@ def lib() -> ctypes.CDLL:
         "ispa_kv_evict_history": (_ci, [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp]),
         "ispa_kv_restore": (_ci, [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp]),
         "ispa_stats_reset": (_ci, [_ci, _ci, _vp, _vp, _vp, _vp]),
+        "ispa_selftest_wait_timeout": (_ci, [ctypes.c_longlong, _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -251,6 +252,13 @@ def ispa_kv_restore(desc: AttnDesc, k_ev, v_ev, k_full, v_full, stream=None) -> 
 
 def ispa_stats_reset(D: int, Dout: int, G, C, r2, stream=None) -> None:
     _check(lib().ispa_stats_reset(D, Dout, _ptr(G), _ptr(C), _ptr(r2), _stream(stream)))
+
+
+ISPA_SELFTEST_SITE = 999
+
+
+def ispa_selftest_wait_timeout(wait_ns: int, stream=None) -> None:
+    _check(lib().ispa_selftest_wait_timeout(int(wait_ns), _stream(stream)))
 
 
 lib()

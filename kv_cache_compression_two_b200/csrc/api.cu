@@ -431,6 +431,16 @@ ispa_status ispa_kv_restore(const ispa_attn_desc *desc, const void *k_ev, const 
   return kv_remap(desc, k_ev, v_ev, k_full, v_full, false, (cudaStream_t)stream);
 }
 
+ispa_status ispa_selftest_wait_timeout(long long wait_ns, ispa_stream_t stream) {
+  if (wait_ns < 1000000LL || wait_ns > 10000000000LL)
+    return fail(ISPA_ERR_INVALID_ARG, "wait_ns must lie in [1 ms, 10 s] (got %lld)", wait_ns);
+  DevErr e;
+  ispa_status st = device_err(&e);
+  if (st != ISPA_OK) return st;
+  e.limit_ns = wait_ns;
+  return launch_selftest_wait(e, (cudaStream_t)stream);
+}
+
 ispa_status ispa_stats_reset(int D, int Dout, float *G, float *C, double *r2, ispa_stream_t stream) {
   if (D < 1 || Dout < 1) return fail(ISPA_ERR_INVALID_ARG, "D and Dout must be >= 1");
   if (!G || !C || !r2) return fail(ISPA_ERR_INVALID_ARG, "G, C and r2 must be device pointers");

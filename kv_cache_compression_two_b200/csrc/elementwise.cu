@@ -223,4 +223,26 @@ ispa_status launch_kv_remap(int B, long long full_rows, long long kept_rows, lon
   return cuda_status(cudaGetLastError(), "kv remap launch");
 }
 
+// ---------------------------------------------------------------------------
+// Failure-detection self-test: the bounded wait of the kernels, on a barrier
+// that no arrival completes, so that it runs out and reports.
+// ---------------------------------------------------------------------------
+__global__ void selftest_wait_kernel(DevErr e) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) wait_parity(&bar, 0, e, &abort_flag, ISPA_SELFTEST_SITE);
+}
+
+ispa_status launch_selftest_wait(const DevErr &e, cudaStream_t s) {
+  selftest_wait_kernel<<<1, 32, 0, s>>>(e);
+  note_launch();
+  return cuda_status(cudaGetLastError(), "self-test launch");
+}
+
 }  // namespace ispa

@@ -47,6 +47,8 @@ ispa_status launch_lse_merge(int rows, int H, int d, ispa_dtype dt, const void *
 ispa_status launch_kv_remap(int B, long long full_rows, long long kept_rows, long long b0, long long len0,
                             long long b1, long long row_bytes, bool gather, const void *k, const void *v,
                             void *k_out, void *v_out, cudaStream_t s);
+// One CTA waiting (bounded by e.limit_ns) on an mbarrier nothing completes.
+ispa_status launch_selftest_wait(const DevErr &e, cudaStream_t s);
 ispa_status launch_select(int N, const double *eps, int K, unsigned char *is_local, int *idx,
                           cudaStream_t s);
 ispa_status launch_absorb_weight(int D, int Dout, const void *W, ispa_dtype wdt, const float *dW,

@@ -175,3 +175,9 @@ def test_recalibration_validation():
     bad = _desc(cur_begin=5, cur_end=5)
     assert L.ispa_kv_restore(ctypes.byref(bad), FAKE, FAKE, FAKE + (1 << 24), FAKE + (1 << 26),
                              None) == ispa.ISPA_ERR_INVALID_ARG
+
+
+def test_selftest_validation():
+    L = ispa.lib()
+    assert L.ispa_selftest_wait_timeout(10, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_selftest_wait_timeout(20_000_000_000, None) == ispa.ISPA_ERR_INVALID_ARG

@@ -255,3 +255,26 @@ def test_attn_local_proj(y_dt):
         assert_bf16_out(got, ref, tol=2e-2)
     else:
         assert max_over_rms(got, ref) <= 2e-2, max_over_rms(got, ref)
+
+
+# ---------------------------------------------------------------- failure detection
+def test_bounded_wait_runs_out_and_the_context_survives():
+    """A wait whose peer never arrives gives up after its limit, reports
+    ISPA_ERR_TIMEOUT with its site, and leaves the context usable (no fault,
+    no trap: the kernel returns)."""
+    import time
+    ispa.ispa_check_device_error()  # starts clean
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    ispa.ispa_selftest_wait_timeout(50_000_000)  # 50 ms
+    with pytest.raises(ispa.IspaError) as err:
+        ispa.ispa_check_device_error()
+    elapsed = time.perf_counter() - t0
+    assert err.value.status == ispa.ISPA_ERR_TIMEOUT
+    assert str(ispa.ISPA_SELFTEST_SITE) in str(err.value)
+    assert elapsed >= 0.045
+    # the error word was cleared by the report, and the device still works
+    G, C, r2 = _spd_problem(64, 64, 192, 3)
+    dW, eps = _run_ridge(G, C, r2, 1e-4, True, 0)
+    assert np.all(np.isfinite(dW)) and math.isfinite(eps)
+    assert ispa.ispa_check_device_error() == 0
