@@ -191,15 +191,20 @@ __device__ __forceinline__ void tile_xyt(const TileT &X, const TileT &Y, float a
   for (int a = 0; a < 4; ++a)
 #pragma unroll
     for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
-#pragma unroll 8
-  for (int q = 0; q < NB; ++q) {
-    const float4 x = *reinterpret_cast<const float4 *>(&X[q][tgrp(ty, q)]);
-    const float4 y = *reinterpret_cast<const float4 *>(&Y[q][tgrp(tx, q)]);
-    const float xa[4] = {x.x, x.y, x.z, x.w}, yb[4] = {y.x, y.y, y.z, y.w};
+  // the swizzled column of a thread is the same for the four rows q0 .. q0 + 3
+#pragma unroll 2
+  for (int q0 = 0; q0 < NB; q0 += 4) {
+    const float *xp = &X[q0][tgrp(ty, q0)], *yp = &Y[q0][tgrp(tx, q0)];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int i = 0; i < 4; ++i) {
+      const float4 x = *reinterpret_cast<const float4 *>(xp + i * NB);
+      const float4 y = *reinterpret_cast<const float4 *>(yp + i * NB);
+      const float xa[4] = {x.x, x.y, x.z, x.w}, yb[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
-      for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(xa[a], yb[b], acc[a][b]);
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(xa[a], yb[b], acc[a][b]);
+    }
   }
 }
 
