@@ -338,3 +338,93 @@ def absorb_layer(chunks: List[Dict[str, np.ndarray]], W: np.ndarray, lam: float,
 def attention_flops(n_query: int, n_key: int, H: int, d: int) -> float:
     """Dot-product FLOPs of one attention call: QK^T and PV, 2 flops per multiply-add."""
     return 4.0 * n_query * n_key * H * d
+
+
+# ---------------------------------------------------------------------------
+# W8A8 post-switch projection  [EN-notes, "Key Findings" (Figure 7);
+# DE-summary §4 "Beschleunigung"]
+# ---------------------------------------------------------------------------
+# The pages report ISPA combined with W8A8 post-training quantisation but do not
+# fix the scheme.  Reading taken: symmetric quantisation with one fp32 scale per
+# activation row and per weight column, s = amax / QMAX, q = Q(x * inv) with
+# inv = QMAX / amax; Q rounds to fp8 e4m3 (to nearest even, saturating at 448)
+# or to int8 (half to even, clamped to +-127).  The scale arithmetic is fp32,
+# the precision that decides the codes on both sides.
+Q8_E4M3, Q8_INT8 = 0, 1
+Q8_MAX = {Q8_E4M3: 448.0, Q8_INT8: 127.0}
+
+
+def e4m3_round(x: np.ndarray) -> np.ndarray:
+    """Nearest fp8 e4m3 value of each x (ties to even mantissa), saturating at +-448.
+
+    The format (OCP 8-bit floating point, E4M3): sign, 4 exponent bits with bias
+    7, 3 mantissa bits; normal values (1 + m/8) 2^(e-7) for e = 1..15 except
+    e = 15, m = 7 (NaN), subnormals m 2^-9; no infinities.  In the binade
+    [2^E, 2^(E+1)) with E >= -6 the spacing is 2^(E-3); below 2^-6 it is 2^-9.
+    """
+    x = np.asarray(x, np.float64)
+    a = np.abs(x)
+    _, ex = np.frexp(a)                      # a = f 2^ex, f in [0.5, 1)
+    E = np.maximum(ex - 1, -6)               # binade exponent, floored at the normal minimum
+    quantum = np.ldexp(1.0, E - 3)
+    q = np.rint(a / quantum) * quantum       # exact: a / quantum is a power-of-two scaling
+    q = np.minimum(q, 448.0)
+    return np.copysign(q, x)
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """Value of each e4m3 byte (NaN for the codes S.1111.111), from the format definition."""
+    c = np.asarray(codes, np.uint8).astype(np.int64)
+    s = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    val = np.where(e == 0, np.ldexp(m.astype(np.float64), -9),
+                   np.ldexp(1.0 + m / 8.0, e - 7))
+    val = np.where((e == 15) & (m == 7), np.nan, val)
+    return s * val
+
+
+def q8_round(t: np.ndarray, fmt: int) -> np.ndarray:
+    """The format's rounding Q of already-scaled values t."""
+    if fmt == Q8_E4M3:
+        return e4m3_round(t)
+    return np.clip(np.rint(np.asarray(t, np.float64)), -127.0, 127.0)
+
+
+def quantize_rows(x: np.ndarray, fmt: int):
+    """Per-row quantisation of x [M, K]: returns (q [M, K] as float64 values, s [M] fp32).
+
+    amax, inv = QMAX / amax and x * inv are fp32 operations (each rounded to
+    nearest); an all-zero row has s = 0, inv = 0, q = 0.
+    """
+    x32 = np.asarray(x, np.float32)
+    qmax = np.float32(Q8_MAX[fmt])
+    amax = np.abs(x32).max(axis=1) if x32.shape[1] else np.zeros(x32.shape[0], np.float32)
+    with np.errstate(divide="ignore"):
+        inv = np.where(amax > 0, qmax / np.where(amax > 0, amax, np.float32(1)), np.float32(0)).astype(np.float32)
+    s = (amax / qmax).astype(np.float32)
+    t = (x32 * inv[:, None]).astype(np.float32)
+    return q8_round(t.astype(np.float64), fmt), s
+
+
+def quantize_cols(W: np.ndarray, fmt: int):
+    """Per-column quantisation of W [K, N]: (q [K, N] values, s [N] fp32)."""
+    q, s = quantize_rows(np.asarray(W, np.float32).T, fmt)
+    return q.T, s
+
+
+def gemm_q8(qa: np.ndarray, sa: np.ndarray, qw: np.ndarray, sw: np.ndarray, fmt: int) -> np.ndarray:
+    """y[m, n] = (sum_k qa[m, k] qw[k, n]) sa[m] sw[n].
+
+    The sum is exact in float64 for both formats (e4m3 products carry at most 8
+    significant bits over a 36-bit range, int8 ones are integers below 2^15).
+    For int8 the kernel's accumulator is that exact integer, and the scaling is
+    taken as the kernel takes it: fp32(acc) * sa, then * sw, each in fp32 with
+    rounding to nearest -- returned as fp32.  For e4m3 the exact value is
+    returned in float64 (the tensor cores add in fp32).
+    """
+    acc = np.asarray(qa, np.float64) @ np.asarray(qw, np.float64)
+    if fmt == Q8_INT8:
+        a32 = acc.astype(np.float32)           # |acc| < 2^31, rounded to nearest fp32
+        return (a32 * np.asarray(sa, np.float32)[:, None]).astype(np.float32) * np.asarray(sw, np.float32)[None, :]
+    return acc * np.asarray(sa, np.float64)[:, None] * np.asarray(sw, np.float64)[None, :]

@@ -251,3 +251,23 @@ def random_groups_shape(g: np.random.Generator, *, max_frames: int = 12, d: Opti
     hb, he = S, S + Hf
     return AttnShape(B=B, H=H, d=d, tpf=tpf, sink_frames=S, hist_begin=hb, hist_end=he,
                      cur_begin=he, cur_end=he + C, kv_frames=he + C)
+
+
+def activation_rows(M: int, K: int, key: Iterable) -> np.ndarray:
+    """Activation-like rows [M, K] in bf16 values for the 8-bit quantisers.
+
+    Row magnitudes log-uniform over 1e-4 .. 1e2 (so some rows reach the e4m3
+    subnormal range after scaling), a few outlier channels at 20x, row 0 all
+    zeros and row 1 a single nonzero entry when M allows.
+    """
+    g = rng(*tuple(key), "act")
+    x = _normal(g, (M, K), 1.0)
+    x *= (10.0 ** g.uniform(-4.0, 2.0, size=(M, 1))).astype(np.float32)
+    if K >= 8:
+        x[:, g.choice(K, size=max(1, K // 128), replace=False)] *= np.float32(20.0)
+    if M >= 1:
+        x[0] = 0.0
+    if M >= 2:
+        x[1] = 0.0
+        x[1, K // 3] = -3.0
+    return round_to_bf16(x)

@@ -463,3 +463,146 @@ def test_mutant_largest_eps_selection_is_caught():
     def largest(eps, K):
         return orc.select_layers(-np.asarray(eps), K)
     assert not check_selection_bruteforce(largest)
+
+
+# ---------------------------------------------------------------------------
+# W8A8: the 8-bit formats and the quantised projection
+# ---------------------------------------------------------------------------
+def e4m3_grid_by_enumeration():
+    """Every positive finite e4m3 value, listed from the format's bit fields with Python floats."""
+    vals = [m * 2.0 ** -9 for m in range(1, 8)]                      # subnormals
+    for e in range(1, 16):
+        for m in range(8):
+            if e == 15 and m == 7:
+                continue                                              # NaN
+            vals.append((1 + m / 8) * 2.0 ** (e - 7))
+    return sorted(vals)
+
+
+def test_e4m3_decode_matches_the_format_definition():
+    grid = e4m3_grid_by_enumeration()
+    assert len(grid) == 126 and grid[-1] == 448.0 and grid[0] == 2.0 ** -9 and grid[7] == 2.0 ** -6
+    v = orc.e4m3_decode(np.arange(256, dtype=np.uint8))
+    assert np.isnan(v[0x7F]) and np.isnan(v[0xFF]) and np.isnan(v).sum() == 2
+    assert v[0x00] == 0.0 and v[0x80] == 0.0 and np.signbit(v[0x80])
+    pos = v[1:0x7F]
+    assert list(pos) == grid                                         # codes 0x01..0x7E in increasing order
+    assert np.array_equal(v[0x81:0xFF], -pos)
+
+
+def test_e4m3_round_is_the_nearest_grid_value_ties_to_even():
+    grid = np.array(e4m3_grid_by_enumeration())
+    assert np.array_equal(orc.e4m3_round(grid), grid)
+    assert np.array_equal(orc.e4m3_round(-grid), -grid)
+    full = np.concatenate([[0.0], grid])
+    codes = np.arange(0, 127)                                        # code of full[i] is i
+    mids = (full[:-1] + full[1:]) / 2
+    got = orc.e4m3_round(mids)
+    even = np.where(codes[:-1] % 2 == 0, full[:-1], full[1:])        # the neighbour with an even code
+    assert np.array_equal(got, even)
+    # off-midpoint values go to the nearer neighbour
+    lo = full[:-1] + (full[1:] - full[:-1]) * 0.49
+    hi = full[:-1] + (full[1:] - full[:-1]) * 0.51
+    assert np.array_equal(orc.e4m3_round(lo), full[:-1]) and np.array_equal(orc.e4m3_round(hi), full[1:])
+    # saturation
+    assert list(orc.e4m3_round(np.array([448.0, 460.0, 464.0, 1e6, -1e30]))) == [448, 448, 448, 448, -448]
+
+
+def test_e4m3_round_agrees_with_torch_float8_in_range():
+    torch = pytest.importorskip("torch")
+    x = np.random.default_rng(11).standard_normal(200000) * np.exp(np.random.default_rng(12).uniform(-12, 6, 200000))
+    x = x[np.abs(x) <= 448]
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(orc.e4m3_round(x), ref)
+
+
+def test_int8_rounding_is_half_to_even_and_clamped():
+    t = np.array([0.5, 1.5, 2.5, -2.5, -0.5, 2.4999, 126.5, 127.49, 128.0, -300.0, 0.0])
+    assert list(orc.q8_round(t, orc.Q8_INT8)) == [0, 2, 2, -2, -0, 2, 126, 127, 127, -127, 0]
+
+
+@pytest.mark.parametrize("fmt", [orc.Q8_E4M3, orc.Q8_INT8])
+def test_quantize_rows_properties(fmt):
+    x = si.activation_rows(37, 96, ("pin", "q8", fmt))
+    q, s = orc.quantize_rows(x, fmt)
+    qmax = orc.Q8_MAX[fmt]
+    amax = np.abs(x).max(axis=1)
+    assert s.dtype == np.float32 and np.array_equal(s, (amax / np.float32(qmax)).astype(np.float32))
+    assert np.all(q[0] == 0) and s[0] == 0                            # zero row
+    nz = amax > 0
+    # the largest entry of each row lands on +-QMAX exactly
+    arg = np.abs(x).argmax(axis=1)
+    assert np.all(np.abs(q[np.arange(len(x)), arg])[nz] == qmax)
+    assert np.all(np.abs(q) <= qmax)
+    # values are on the format's grid
+    if fmt == orc.Q8_INT8:
+        assert np.array_equal(q, np.round(q))
+    else:
+        grid = set(e4m3_grid_by_enumeration()) | {0.0}
+        assert set(np.abs(q).ravel().tolist()) <= grid
+    # dequantisation error: int8 within half a step; e4m3 within half a spacing of the binade
+    t = x.astype(np.float64) * (qmax / np.where(nz, amax, 1.0))[:, None]
+    if fmt == orc.Q8_INT8:
+        assert np.all(np.abs(q - t) <= 0.5 + 1e-5 * qmax)
+    else:
+        bound = np.maximum(np.abs(t) * 2.0 ** -4, 2.0 ** -10) * (1 + 1e-5)
+        assert np.all(np.abs(q - t) <= bound)
+
+
+def brute_gemm_q8(qa, sa, qw, sw):
+    """sum_k qa[m][k] qw[k][n] * sa[m] * sw[n] with exact Python fractions, converted at the end."""
+    from fractions import Fraction
+    M, K = qa.shape
+    N = qw.shape[1]
+    y = np.zeros((M, N))
+    for m in range(M):
+        for n in range(N):
+            acc = sum(Fraction(float(qa[m, k])) * Fraction(float(qw[k, n])) for k in range(K))
+            y[m, n] = float(acc * Fraction(float(sa[m])) * Fraction(float(sw[n])))
+    return y
+
+
+@pytest.mark.parametrize("fmt", [orc.Q8_E4M3, orc.Q8_INT8])
+def test_gemm_q8_against_exact_brute_force(fmt):
+    x = si.activation_rows(5, 48, ("pin", "gemm", fmt))
+    W = si.projection_weight(48, 7, ("pin", "gemm", fmt), "bf16")
+    qa, sa = orc.quantize_rows(x, fmt)
+    qw, sw = orc.quantize_cols(W, fmt)
+    assert qw.shape == (48, 7) and sw.shape == (7,)
+    ref = brute_gemm_q8(qa, sa, qw, sw)
+    got = np.asarray(orc.gemm_q8(qa, sa, qw, sw, fmt), np.float64)
+    if fmt == orc.Q8_INT8:
+        # fp32 epilogue: three roundings to nearest fp32
+        assert np.all(np.abs(got - ref) <= 3 * 2.0 ** -24 * np.abs(ref) + 1e-45)
+    else:
+        assert np.allclose(got, ref, rtol=1e-15, atol=0)
+
+
+@pytest.mark.parametrize("fmt", [orc.Q8_E4M3, orc.Q8_INT8])
+def test_w8a8_projection_is_within_the_quantisation_bound(fmt):
+    """|A W - deq(A) deq(W)| <= sum_k |a||dW| + |da||W| + |da||dW| with the per-element errors."""
+    A = si.activation_rows(40, 256, ("pin", "w8a8", fmt))[2:]
+    W = si.projection_weight(256, 24, ("pin", "w8a8", fmt), "bf16")
+    qa, sa = orc.quantize_rows(A, fmt)
+    qw, sw = orc.quantize_cols(W, fmt)
+    Ad = qa * sa[:, None].astype(np.float64)
+    Wd = qw * sw[None, :].astype(np.float64)
+    dA, dWq = np.abs(A - Ad), np.abs(W - Wd)
+    bound = np.abs(A) @ dWq + dA @ np.abs(W) + dA @ dWq
+    y = np.asarray(orc.gemm_q8(qa, sa, qw, sw, fmt), np.float64)
+    exact = A.astype(np.float64) @ W.astype(np.float64)
+    assert np.all(np.abs(y - exact) <= bound * (1 + 1e-5) + 1e-6 * np.abs(exact))
+    # and the product stays close: a few percent relative error (the 20x outlier
+    # channels of the rows set their scales, which coarsens int8 most)
+    rel = np.linalg.norm(y - exact) / np.linalg.norm(exact)
+    assert rel < 0.06, rel
+
+
+def test_mutant_scale_of_the_wrong_side_is_caught():
+    x = si.activation_rows(5, 48, ("pin", "gemm", 1))
+    W = si.projection_weight(48, 5, ("pin", "gemm", 1), "bf16")
+    qa, sa = orc.quantize_rows(x, orc.Q8_INT8)
+    qw, sw = orc.quantize_cols(W, orc.Q8_INT8)
+    ref = brute_gemm_q8(qa, sa, qw, sw)
+    swapped = np.asarray(orc.gemm_q8(qa, sw, qw, sa, orc.Q8_INT8), np.float64)
+    assert not np.allclose(swapped, ref, rtol=1e-6)
