@@ -428,3 +428,31 @@ def gemm_q8(qa: np.ndarray, sa: np.ndarray, qw: np.ndarray, sw: np.ndarray, fmt:
         a32 = acc.astype(np.float32)           # |acc| < 2^31, rounded to nearest fp32
         return (a32 * np.asarray(sa, np.float32)[:, None]).astype(np.float32) * np.asarray(sw, np.float32)[None, :]
     return acc * np.asarray(sa, np.float64)[:, None] * np.asarray(sw, np.float64)[None, :]
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """Nearest bfloat16 value (8 significand bits, fp32's exponent range), ties to even.
+
+    Written from the format: x is first rounded to fp32, then the low 16 bits of
+    its encoding are rounded away (adding 0x7FFF plus the kept part's lowest bit
+    carries into the kept bits exactly when the dropped part exceeds half, or
+    equals half with an odd kept part).  Inputs must be finite.
+    """
+    b = np.ascontiguousarray(np.asarray(x, np.float32)).view(np.uint32).astype(np.uint64)
+    b = ((b + 0x7FFF + ((b >> 16) & 1)) >> 16) << 16
+    return b.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def local_projection_q8(shape, q, k, v, W_new: np.ndarray, fmt: int, scale: float = None) -> np.ndarray:
+    """The post-switch step with a W8A8 projection: Y [B, n, D_out].
+
+    A_loc from the local-group attention (as in :func:`local_projection`), held
+    in bf16 as the post-switch layer stores it, quantised per row; W_new
+    quantised per column; the 8-bit product scaled back (:func:`gemm_q8`).
+    """
+    B, Lq = q.shape[0], q.shape[1]
+    A = local_projection(shape, q, k, v, np.eye(shape.H * shape.d), None, scale)
+    A = bf16_round(A.reshape(B * Lq, -1))
+    qa, sa = quantize_rows(A, fmt)
+    qw, sw = quantize_cols(W_new, fmt)
+    return np.asarray(gemm_q8(qa, sa, qw, sw, fmt)).reshape(B, Lq, -1)

@@ -606,3 +606,37 @@ def test_mutant_scale_of_the_wrong_side_is_caught():
     ref = brute_gemm_q8(qa, sa, qw, sw)
     swapped = np.asarray(orc.gemm_q8(qa, sw, qw, sa, orc.Q8_INT8), np.float64)
     assert not np.allclose(swapped, ref, rtol=1e-6)
+
+
+def test_bf16_round_agrees_with_torch_bfloat16():
+    torch = pytest.importorskip("torch")
+    g = np.random.default_rng(13)
+    x = (g.standard_normal(100000) * np.exp(g.uniform(-30, 30, 100000))).astype(np.float32)
+    # exact ties: fp32 values whose low 16 bits are 0x8000, with odd and even kept parts
+    ties = ((np.arange(0x3F80, 0x3F80 + 1000, dtype=np.uint32) << 16) | np.uint32(0x8000)).view(np.float32)
+    x = np.concatenate([x, ties, -ties])
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(orc.bf16_round(x), ref)
+    # ties go to the even kept part
+    kept = (ties.view(np.uint32) >> 16)
+    got = orc.bf16_round(ties).astype(np.float32).view(np.uint32) >> 16
+    assert np.all(got % 2 == 0) and np.all((got == kept) | (got == kept + 1))
+
+
+@pytest.mark.parametrize("fmt", [orc.Q8_E4M3, orc.Q8_INT8])
+def test_local_projection_q8_reduces_to_the_unquantised_step(fmt):
+    """The W8A8 step approximates A_loc W_new within the quantisation bound of its own operands."""
+    sh = si.AttnShape(B=1, H=2, d=16, tpf=3, sink_frames=1, hist_begin=1, hist_end=3, cur_begin=3, cur_end=5,
+                      kv_frames=5)
+    data = si.iid_qkv(sh, "f32", ("pin", "lq8"))
+    W = si.projection_weight(sh.D, 8, ("pin", "lq8"))
+    y8 = orc.local_projection_q8(sh, data["q"], data["k"], data["v"], W, fmt)
+    y = orc.local_projection(sh, data["q"], data["k"], data["v"], W)
+    A = orc.bf16_round(orc.local_projection(sh, data["q"], data["k"], data["v"], np.eye(sh.D)).reshape(-1, sh.D))
+    qa, sa = orc.quantize_rows(A, fmt)
+    qw, sw = orc.quantize_cols(W, fmt)
+    A0 = orc.local_projection(sh, data["q"], data["k"], data["v"], np.eye(sh.D)).reshape(-1, sh.D)
+    dA = np.abs(A0 - qa * sa[:, None].astype(np.float64))
+    dW = np.abs(W - qw * sw[None, :].astype(np.float64))
+    bound = np.abs(A0) @ dW + dA @ np.abs(W) + dA @ dW
+    assert np.all(np.abs(y8.reshape(-1, 8) - y.reshape(-1, 8)) <= bound * (1 + 1e-5) + 1e-12)
