@@ -54,6 +54,12 @@ typedef enum {
 
 typedef enum { ISPA_F32 = 0, ISPA_BF16 = 1 } ispa_dtype;
 
+/* 8-bit format of the W8A8 projection (one byte per value). */
+typedef enum {
+  ISPA_Q8_E4M3 = 0, /* fp8 e4m3 (bias 7, max 448), round to nearest even, saturating */
+  ISPA_Q8_INT8 = 1  /* two's-complement int8 in [-127, 127], round half to even        */
+} ispa_q8_format;
+
 /* Arithmetic of the absorption-statistics GEMMs. */
 typedef enum {
   ISPA_PREC_TF32 = 0, /* tcgen05 kind::tf32, operands rounded to nearest tf32, fp32 accumulate */
@@ -107,8 +113,8 @@ ispa_status ispa_selftest_wait_timeout(long long wait_ns, ispa_stream_t stream);
  *                   (a frame in both counts once);
  *   history group = frames [hist_begin, hist_end); it must not intersect the
  *                   local group.  hist_begin == hist_end means no history.
- * "The local group contains the initial sink frame and current frame; the
- * historical group contains the intervening frames" [EN-notes, Key Designs 1].
+ * The local group is the sink frame(s) plus the current frame(s), the history
+ * group the frames between them [EN-notes, Key Designs 1].
  * A post-switch F-layer (full context) is the same call with
  * sink_frames = cur_begin and an empty history.
  */
@@ -348,6 +354,55 @@ ispa_status ispa_kv_restore(const ispa_attn_desc *desc, const void *k_ev, const 
  * Asynchronous; ISPA_ERR_INVALID_ARG for D or Dout < 1 or a NULL pointer.
  */
 ispa_status ispa_stats_reset(int D, int Dout, float *G, float *C, double *r2, ispa_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
+/* W8A8 post-switch projection                                                */
+/* ------------------------------------------------------------------------- */
+/*
+ * ISPA composes with post-training W8A8 quantisation of the projections
+ * [EN-notes, "Key Findings" (Figure 7); DE-summary 4, "Beschleunigung"].  The
+ * pages do not fix the scheme; this library takes the plain symmetric one:
+ * one scale per activation row (token) and per weight column (output
+ * channel), s = amax / QMAX in fp32 (QMAX = 448 for e4m3, 127 for int8), and
+ * the value q = Q(x * inv) with inv = QMAX / amax (fp32, rounded to nearest)
+ * and Q the format's rounding (ispa_q8_format).  An all-zero row or column
+ * gets s = 0 and q = 0.  Inputs must be finite.  The product
+ *   y[m, n] = fp32(sum_k qa[m, k] qw[k, n]) * sa[m] * sw[n]
+ * runs on the 8-bit tensor cores (kind::f8f6f4 for e4m3 with an fp32
+ * accumulator, kind::i8 for int8 with an exact int32 one) and is rounded to
+ * y_dtype at the end.
+ *
+ * ispa_quantize_rows: x [M, K] bf16 row-major -> q [M, K] (bytes), sa [M] fp32.
+ * ispa_quantize_weight: W [K, N] bf16 row-major (the layout of W_new from
+ *   ispa_absorb_weight) -> qT [N, K] (bytes, the transpose, K contiguous) and
+ *   sw [N] fp32.  Once per layer, at the switch.
+ * ispa_gemm_q8: y [M, N] in y_dtype from q, sa, qT, sw of the same format.
+ * Sizes: M, N >= 0 with N % 16 == 0 for the product; K >= 16, K % 16 == 0.
+ * Device pointers, 16-byte aligned, no overlap between inputs and outputs.
+ * Asynchronous on stream; ISPA_ERR_INVALID_ARG for bad sizes, format or pointers.
+ */
+ispa_status ispa_quantize_rows(int M, int K, const void *x, ispa_q8_format fmt, void *q, float *sa,
+                               ispa_stream_t stream);
+ispa_status ispa_quantize_weight(int K, int N, const void *W, ispa_q8_format fmt, void *qT, float *sw,
+                                 ispa_stream_t stream);
+ispa_status ispa_gemm_q8(int M, int N, int K, const void *q, const float *sa, const void *qT,
+                         const float *sw, ispa_q8_format fmt, void *y, ispa_dtype y_dtype,
+                         ispa_stream_t stream);
+
+size_t ispa_attn_local_proj_q8_workspace_bytes(const ispa_attn_desc *desc);
+
+/*
+ * ispa_attn_local_proj_q8: the post-switch layer step of ispa_attn_local_proj
+ * with a W8A8 projection.  The attention runs as there (A_loc in bf16); A_loc
+ * is then quantised per row (ispa_quantize_rows) and multiplied with the
+ * quantised weight (qT, sw from ispa_quantize_weight of W_proj, [D, Dout]).
+ *   Dout % 16 == 0; y [B, Lq, Dout] in y_dtype;
+ *   workspace >= ispa_attn_local_proj_q8_workspace_bytes(desc).
+ */
+ispa_status ispa_attn_local_proj_q8(const ispa_attn_desc *desc, const void *q, const void *k,
+                                    const void *v, const void *qT, const float *sw,
+                                    ispa_q8_format fmt, int Dout, void *y, ispa_dtype y_dtype,
+                                    void *workspace, size_t workspace_bytes, ispa_stream_t stream);
 
 #ifdef __cplusplus
 }

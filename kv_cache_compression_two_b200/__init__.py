@@ -23,6 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libispa.so")
 ISPA_OK, ISPA_ERR_INVALID_ARG, ISPA_ERR_UNSUPPORTED, ISPA_ERR_CUDA, ISPA_ERR_NOT_SPD, ISPA_ERR_TIMEOUT = range(6)
 ISPA_F32, ISPA_BF16 = 0, 1
 ISPA_PREC_TF32, ISPA_PREC_F32 = 0, 1
+ISPA_Q8_E4M3, ISPA_Q8_INT8 = 0, 1
 
 STATUS_NAMES = {0: "ISPA_OK", 1: "ISPA_ERR_INVALID_ARG", 2: "ISPA_ERR_UNSUPPORTED", 3: "ISPA_ERR_CUDA",
                 4: "ISPA_ERR_NOT_SPD", 5: "ISPA_ERR_TIMEOUT"}
@@ -32,7 +33,9 @@ EXPORTED = ("ispa_version", "ispa_last_error", "ispa_launch_count", "ispa_check_
             "ispa_accum_stats_workspace_bytes", "ispa_accum_stats", "ispa_ridge_workspace_bytes", "ispa_ridge_solve",
             "ispa_select_layers", "ispa_absorb_weight", "ispa_attn_local_proj_workspace_bytes",
             "ispa_attn_local_proj", "ispa_ridge_solve_noalloc", "ispa_kv_evicted_desc", "ispa_kv_evict_history",
-            "ispa_kv_restore", "ispa_stats_reset", "ispa_selftest_wait_timeout")
+            "ispa_kv_restore", "ispa_stats_reset", "ispa_selftest_wait_timeout", "ispa_quantize_rows",
+            "ispa_quantize_weight", "ispa_gemm_q8", "ispa_attn_local_proj_q8_workspace_bytes",
+            "ispa_attn_local_proj_q8")
 RIDGE_NOALLOC_MAX_D = RIDGE_NOALLOC_MAX_DOUT = 1024
 
 
@@ -91,6 +94,12 @@ def lib() -> ctypes.CDLL:
         "ispa_kv_restore": (_ci, [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp]),
         "ispa_stats_reset": (_ci, [_ci, _ci, _vp, _vp, _vp, _vp]),
         "ispa_selftest_wait_timeout": (_ci, [ctypes.c_longlong, _vp]),
+        "ispa_quantize_rows": (_ci, [_ci, _ci, _vp, _ci, _vp, _vp, _vp]),
+        "ispa_quantize_weight": (_ci, [_ci, _ci, _vp, _ci, _vp, _vp, _vp]),
+        "ispa_gemm_q8": (_ci, [_ci, _ci, _ci, _vp, _vp, _vp, _vp, _ci, _vp, _ci, _vp]),
+        "ispa_attn_local_proj_q8_workspace_bytes": (_sz, [ctypes.POINTER(AttnDesc)]),
+        "ispa_attn_local_proj_q8": (_ci, [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp, _ci, _ci, _vp, _ci,
+                                          _vp, _sz, _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -232,6 +241,32 @@ def ispa_attn_local_proj(desc: AttnDesc, q, k, v, W_proj, Dout: int, y, y_dtype:
         workspace_bytes = workspace_bytes or workspace.numel() * workspace.element_size()
     _check(lib().ispa_attn_local_proj(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(W_proj), Dout, _ptr(y),
                                       y_dtype, _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def ispa_quantize_rows(M: int, K: int, x, fmt: int, q, sa, stream=None) -> None:
+    _check(lib().ispa_quantize_rows(M, K, _ptr(x), fmt, _ptr(q), _ptr(sa), _stream(stream)))
+
+
+def ispa_quantize_weight(K: int, N: int, W, fmt: int, qT, sw, stream=None) -> None:
+    _check(lib().ispa_quantize_weight(K, N, _ptr(W), fmt, _ptr(qT), _ptr(sw), _stream(stream)))
+
+
+def ispa_gemm_q8(M: int, N: int, K: int, q, sa, qT, sw, fmt: int, y, y_dtype: int, stream=None) -> None:
+    _check(lib().ispa_gemm_q8(M, N, K, _ptr(q), _ptr(sa), _ptr(qT), _ptr(sw), fmt, _ptr(y), y_dtype,
+                              _stream(stream)))
+
+
+def ispa_attn_local_proj_q8_workspace_bytes(desc: AttnDesc) -> int:
+    return int(lib().ispa_attn_local_proj_q8_workspace_bytes(ctypes.byref(desc)))
+
+
+def ispa_attn_local_proj_q8(desc: AttnDesc, q, k, v, qT, sw, fmt: int, Dout: int, y, y_dtype: int, workspace,
+                            workspace_bytes: int = 0, stream=None) -> None:
+    if workspace is not None and not isinstance(workspace, int):
+        workspace_bytes = workspace_bytes or workspace.numel() * workspace.element_size()
+    _check(lib().ispa_attn_local_proj_q8(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(qT), _ptr(sw), fmt,
+                                         Dout, _ptr(y), y_dtype, _ptr(workspace), workspace_bytes,
+                                         _stream(stream)))
 
 
 def ispa_kv_evicted_desc(desc: AttnDesc) -> AttnDesc:

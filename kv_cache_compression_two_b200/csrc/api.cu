@@ -402,6 +402,109 @@ ispa_status ispa_attn_local_proj(const ispa_attn_desc *desc, const void *q, cons
   return launch_gemm_bf16(d.B * g.Lq, Dout, D, a_loc, W_proj, y, y_dtype, (cudaStream_t)stream);
 }
 
+namespace {
+
+bool q8_ok(ispa_q8_format f) { return f == ISPA_Q8_E4M3 || f == ISPA_Q8_INT8; }
+
+bool q8_k_ok(int K) { return K >= 16 && K % 16 == 0; }
+
+// [a, a + na) and [b, b + nb) (bytes) overlap
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+  const char *x = static_cast<const char *>(a), *y = static_cast<const char *>(b);
+  return x < y + nb && y < x + na;
+}
+
+}  // namespace
+
+ispa_status ispa_quantize_rows(int M, int K, const void *x, ispa_q8_format fmt, void *q, float *sa,
+                               ispa_stream_t stream) {
+  if (M < 0 || !q8_k_ok(K)) return fail(ISPA_ERR_INVALID_ARG, "need M >= 0 and K a positive multiple of 16");
+  if (!q8_ok(fmt)) return fail(ISPA_ERR_INVALID_ARG, "bad 8-bit format");
+  if (M == 0) return ISPA_OK;
+  if (!ptr_ok(x) || !ptr_ok(q) || !ptr_ok(sa)) return fail(ISPA_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
+  const size_t xb = (size_t)M * K * 2, qb = (size_t)M * K, sb = (size_t)M * 4;
+  if (overlaps(x, xb, q, qb) || overlaps(x, xb, sa, sb) || overlaps(q, qb, sa, sb))
+    return fail(ISPA_ERR_INVALID_ARG, "x, q and sa must not overlap");
+  return launch_quant_rows(M, K, x, fmt, q, sa, (cudaStream_t)stream);
+}
+
+ispa_status ispa_quantize_weight(int K, int N, const void *W, ispa_q8_format fmt, void *qT, float *sw,
+                                 ispa_stream_t stream) {
+  if (N < 0 || !q8_k_ok(K)) return fail(ISPA_ERR_INVALID_ARG, "need N >= 0 and K a positive multiple of 16");
+  if (!q8_ok(fmt)) return fail(ISPA_ERR_INVALID_ARG, "bad 8-bit format");
+  if (N == 0) return ISPA_OK;
+  if (!ptr_ok(W) || !ptr_ok(qT) || !ptr_ok(sw)) return fail(ISPA_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
+  const size_t wb = (size_t)K * N * 2, qb = (size_t)K * N, sb = (size_t)N * 4;
+  if (overlaps(W, wb, qT, qb) || overlaps(W, wb, sw, sb) || overlaps(qT, qb, sw, sb))
+    return fail(ISPA_ERR_INVALID_ARG, "W, qT and sw must not overlap");
+  return launch_quant_cols(K, N, W, fmt, qT, sw, (cudaStream_t)stream);
+}
+
+ispa_status ispa_gemm_q8(int M, int N, int K, const void *q, const float *sa, const void *qT, const float *sw,
+                         ispa_q8_format fmt, void *y, ispa_dtype y_dtype, ispa_stream_t stream) {
+  if (M < 0 || N < 0 || N % 16 != 0 || !q8_k_ok(K))
+    return fail(ISPA_ERR_INVALID_ARG, "need M >= 0, N a multiple of 16 and K a positive multiple of 16");
+  if (!q8_ok(fmt)) return fail(ISPA_ERR_INVALID_ARG, "bad 8-bit format");
+  if (!dtype_ok(y_dtype)) return fail(ISPA_ERR_INVALID_ARG, "bad y dtype");
+  if (M == 0 || N == 0) return ISPA_OK;
+  if (!ptr_ok(q) || !ptr_ok(sa) || !ptr_ok(qT) || !ptr_ok(sw) || !ptr_ok(y))
+    return fail(ISPA_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
+  const size_t yb = (size_t)M * N * (y_dtype == ISPA_BF16 ? 2 : 4);
+  if (overlaps(y, yb, q, (size_t)M * K) || overlaps(y, yb, sa, (size_t)M * 4) ||
+      overlaps(y, yb, qT, (size_t)N * K) || overlaps(y, yb, sw, (size_t)N * 4))
+    return fail(ISPA_ERR_INVALID_ARG, "y must not overlap the inputs");
+  return launch_gemm_q8(M, N, K, q, sa, qT, sw, fmt, y, y_dtype, (cudaStream_t)stream);
+}
+
+size_t ispa_attn_local_proj_q8_workspace_bytes(const ispa_attn_desc *desc) {
+  const size_t base = (ispa_attn_local_proj_workspace_bytes(desc) + 255) & ~size_t(255);
+  if (base == 0) return 0;
+  const size_t rows = (size_t)desc->B * ((size_t)(desc->cur_end - desc->cur_begin) * desc->tokens_per_frame);
+  const size_t qa = rows * desc->H * desc->head_dim, sa = rows * 4;
+  return base + ((qa + 255) & ~size_t(255)) + ((sa + 255) & ~size_t(255));
+}
+
+ispa_status ispa_attn_local_proj_q8(const ispa_attn_desc *desc, const void *q, const void *k, const void *v,
+                                    const void *qT, const float *sw, ispa_q8_format fmt, int Dout, void *y,
+                                    ispa_dtype y_dtype, void *workspace, size_t workspace_bytes,
+                                    ispa_stream_t stream) {
+  GroupRanges g;
+  float scale;
+  ispa_status st = attn_ranges(desc, &g, &scale);
+  if (st != ISPA_OK) return st;
+  if (desc->in_dtype != ISPA_BF16 || desc->head_dim != 128)
+    return fail(ISPA_ERR_UNSUPPORTED, "post-switch projection is compiled for bf16 inputs with head_dim 128");
+  if (!q8_ok(fmt)) return fail(ISPA_ERR_INVALID_ARG, "bad 8-bit format");
+  if (Dout < 16 || Dout % 16 != 0) return fail(ISPA_ERR_INVALID_ARG, "Dout must be a positive multiple of 16");
+  if (!dtype_ok(y_dtype)) return fail(ISPA_ERR_INVALID_ARG, "bad y dtype");
+  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(qT) || !ptr_ok(sw) || !ptr_ok(y))
+    return fail(ISPA_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
+  const size_t need = ispa_attn_local_proj_q8_workspace_bytes(desc);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return fail(ISPA_ERR_INVALID_ARG, "workspace needs %zu bytes (16-byte aligned)", need);
+  ispa_attn_desc d = *desc;
+  d.hist_begin = d.hist_end = 0;
+  d.out_dtype = ISPA_BF16;
+  g.hist_begin = g.hist_end = 0;
+  const int D = d.H * d.head_dim;
+  const size_t rows = (size_t)d.B * g.Lq;
+  const size_t a_bytes = ((rows * D * 2) + 255) & ~size_t(255);
+  const size_t l_bytes = ((rows * d.H * 4) + 255) & ~size_t(255);
+  const size_t base = (ispa_attn_local_proj_workspace_bytes(desc) + 255) & ~size_t(255);
+  const size_t qa_bytes = (rows * D + 255) & ~size_t(255);
+  char *w = static_cast<char *>(workspace);
+  void *a_loc = w;
+  float *lse = reinterpret_cast<float *>(w + a_bytes);
+  void *attn_ws = w + a_bytes + l_bytes;
+  void *qa = w + base;
+  float *sa = reinterpret_cast<float *>(w + base + qa_bytes);
+  cudaStream_t s = (cudaStream_t)stream;
+  st = launch_attn_tc(d, g, scale, q, k, v, a_loc, lse, nullptr, nullptr, nullptr, nullptr, attn_ws, s);
+  if (st != ISPA_OK) return st;
+  if ((st = launch_quant_rows((int)rows, D, a_loc, fmt, qa, sa, s)) != ISPA_OK) return st;
+  return launch_gemm_q8((int)rows, Dout, D, qa, sa, qT, sw, fmt, y, y_dtype, s);
+}
+
 ispa_status ispa_kv_evicted_desc(const ispa_attn_desc *desc, ispa_attn_desc *evicted) {
   GroupRanges g;
   float scale;

@@ -188,9 +188,23 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 
 // D[tmem] (+)= A[smem] * B[smem]
+// kind: 0 = kind::f16 (fp16 / bf16), 1 = kind::tf32, 2 = kind::f8f6f4 (e4m3 operands),
+// 3 = kind::i8 (int8 operands, exact int32 accumulator).
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate, int kind_tf32) {
-  if (kind_tf32) {
+                                       uint32_t accumulate, int kind) {
+  if (kind == 3) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else if (kind == 2) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else if (kind == 1) {
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
@@ -295,6 +309,12 @@ __host__ __device__ constexpr uint32_t make_idesc(int M, int N, int ab_format, i
          | ((uint32_t)b_mn << 16)                    // B major
          | ((uint32_t)(N >> 3) << 17)                // N
          | ((uint32_t)(M >> 4) << 24);               // M
+}
+
+// Instruction descriptor of kind::i8 with signed 8-bit A and B (format 1) and an
+// int32 accumulator (D format 2), both operands K-major, no saturation.
+__host__ __device__ constexpr uint32_t make_idesc_s8(int M, int N) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 // ---------------------------------------------------------------------------

@@ -53,7 +53,8 @@ enum Epi : int {
   EPI_STORE_TF32_SQ = 1,  // out = tf32_rn(acc); r2 += sum acc^2
   EPI_ACCUM_F32 = 2,      // out += acc
   EPI_STORE_BF16 = 3,     // out = bf16_rn(acc)
-  EPI_ATOMIC_F32 = 4      // out += acc with atomics (split K)
+  EPI_ATOMIC_F32 = 4,     // out += acc with atomics (split K)
+  EPI_SCALED = 5          // out = acc * row_scale[m] * col_scale[n], bf16 or fp32 (out_bf16)
 };
 
 enum Tri : int { TRI_NONE = 0, TRI_A_LOWER = 1, TRI_A_UPPER = 2 };
@@ -73,9 +74,12 @@ struct Params {
   int n_tiles0;   // tiles of problem 0 (upper-triangle filter already applied)
   int n_tiles;    // tiles of both problems (the grid size)
   int kind_tf32;  // 1: kind::tf32 (fp32 operands), 0: kind::f16 with bf16 operands
+  int kind_f8;    // 8-bit K-major operands: 1 = e4m3 (kind::f8f6f4), 2 = int8 (kind::i8, int32 accumulator)
   int a_mn, b_mn; // operand majorness (1 = MN-major)
   uint32_t idesc;
   double *r2;     // EPI_STORE_TF32_SQ accumulator
+  const float *row_scale, *col_scale;  // EPI_SCALED factors
+  int out_bf16;   // EPI_SCALED: bf16 output (else fp32)
   int split3;     // 1: three passes (hi hi, hi lo, lo hi) with the lo maps
   int tri;        // Tri: K range of a tile cut to a triangle of A
   int nchunk;     // K chunks per tile (0 or 1: none)
@@ -125,6 +129,41 @@ __device__ __forceinline__ void epilogue_chunk(const Params &P, const SubProblem
                                                const uint32_t (&r)[32], double &sq) {
   if (row >= P.M) return;
   const int N = sp.N;
+  if (EPI == EPI_SCALED) {
+    const float rs = P.row_scale[row];
+    float x[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float acc = P.kind_f8 == 2 ? __int2float_rn((int)r[j]) : __uint_as_float(r[j]);
+      x[j] = col0 + j < N ? acc * rs * P.col_scale[col0 + j] : 0.f;
+    }
+    if (P.out_bf16) {
+      __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(sp.out) + (long long)row * sp.ldo + col0;
+      if (col0 + 32 <= N && (reinterpret_cast<uintptr_t>(o) & 15) == 0) {
+        uint4 *o4 = reinterpret_cast<uint4 *>(o);
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          o4[v] = make_uint4(pack_bf16x2(x[8 * v], x[8 * v + 1]), pack_bf16x2(x[8 * v + 2], x[8 * v + 3]),
+                             pack_bf16x2(x[8 * v + 4], x[8 * v + 5]), pack_bf16x2(x[8 * v + 6], x[8 * v + 7]));
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (col0 + j < N) o[j] = __float2bfloat16_rn(x[j]);
+      }
+    } else {
+      float *o = reinterpret_cast<float *>(sp.out) + (long long)row * sp.ldo + col0;
+      if (col0 + 32 <= N && (reinterpret_cast<uintptr_t>(o) & 15) == 0) {
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          reinterpret_cast<float4 *>(o)[v] = make_float4(x[4 * v], x[4 * v + 1], x[4 * v + 2], x[4 * v + 3]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (col0 + j < N) o[j] = x[j];
+      }
+    }
+    return;
+  }
   if (EPI == EPI_STORE_BF16) {
     __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(sp.out) + (long long)row * sp.ldo + col0;
     if (col0 + 32 <= N) {
@@ -213,7 +252,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const SubProblem &sp = P.p[prob];
   const CUtensorMap *tB = prob == 0 ? &tb0 : &tb1;
   const int m0 = tm * BM, n0 = tn * BN;
-  const int bk = P.kind_tf32 ? 32 : 64;         // K elements per stage
+  const int bk = P.kind_tf32 ? 32 : (P.kind_f8 ? 128 : 64);  // K elements per stage (128 bytes)
   // this CTA's K-tiles [kt_begin, kt_end): the tile's range (cut to A's
   // triangle), then this chunk of it
   int kt_begin = 0, kt_end = (P.K + bk - 1) / bk;
@@ -226,7 +265,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (kt_begin >= kt_end) return;  // empty chunk: nothing to add (before any barrier or TMEM)
   const int k_span = kt_end - kt_begin;
   const int k_tiles = k_span * (P.split3 ? 3 : 1);  // pipeline iterations
-  const int e128 = P.kind_tf32 ? 32 : 64;       // elements per 128-byte row
+  const int e128 = bk;                          // elements per 128-byte row
   const uint32_t kstep_kmajor = 32;             // bytes per MMA K-step inside a K-major row
   const uint32_t kstep_mn = P.kind_tf32 ? 1024 : 2048;  // bytes per MMA K-step in an MN-major tile
   const uint32_t mn_box_bytes = (uint32_t)bk * 128;     // one 128-byte-wide MN-major box
@@ -311,7 +350,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                                      : smem_desc_sw128(a_base + ks * kstep_kmajor, 16, 1024);
           const uint64_t bd = P.b_mn ? smem_desc(b_base + ks * kstep_mn, mn_box_bytes, mn_sbo, mn_layout)
                                      : smem_desc_sw128(b_base + ks * kstep_kmajor, 16, 1024);
-          mma_ss(tmem, ad, bd, P.idesc, (kt > 0 || ks > 0) ? 1u : 0u, P.kind_tf32);
+          mma_ss(tmem, ad, bd, P.idesc, (kt > 0 || ks > 0) ? 1u : 0u, P.kind_f8 ? P.kind_f8 + 1 : P.kind_tf32);
         }
         mma_commit(empty + s);
       }
@@ -336,6 +375,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           case EPI_STORE_TF32_SQ: epilogue_chunk<EPI_STORE_TF32_SQ>(P, sp, row, n0 + c * 32, r, sq); break;
           case EPI_ACCUM_F32: epilogue_chunk<EPI_ACCUM_F32>(P, sp, row, n0 + c * 32, r, sq); break;
           case EPI_ATOMIC_F32: epilogue_chunk<EPI_ATOMIC_F32>(P, sp, row, n0 + c * 32, r, sq); break;
+          case EPI_SCALED: epilogue_chunk<EPI_SCALED>(P, sp, row, n0 + c * 32, r, sq); break;
           default: epilogue_chunk<EPI_STORE_BF16>(P, sp, row, n0 + c * 32, r, sq); break;
         }
       }

@@ -79,4 +79,10 @@ ispa_status ridge_noalloc_scratch(void **out);
 ispa_status launch_gemm_bf16(int M, int N, int K, const void *A, const void *B, void *Y, ispa_dtype ydt,
                              cudaStream_t s);
 
+// W8A8 projection (quant.cu); fmt is an ispa_q8_format
+ispa_status launch_quant_rows(int M, int K, const void *x, int fmt, void *q, float *scale, cudaStream_t s);
+ispa_status launch_quant_cols(int K, int N, const void *W, int fmt, void *qT, float *scale, cudaStream_t s);
+ispa_status launch_gemm_q8(int M, int N, int K, const void *qa, const float *sa, const void *qT, const float *sw,
+                           int fmt, void *y, ispa_dtype ydt, cudaStream_t s);
+
 }  // namespace ispa

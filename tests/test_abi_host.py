@@ -181,3 +181,40 @@ def test_selftest_validation():
     L = ispa.lib()
     assert L.ispa_selftest_wait_timeout(10, None) == ispa.ISPA_ERR_INVALID_ARG
     assert L.ispa_selftest_wait_timeout(20_000_000_000, None) == ispa.ISPA_ERR_INVALID_ARG
+
+
+def test_w8a8_validation():
+    L = ispa.lib()
+    E8, I8, BAD = ispa.ISPA_Q8_E4M3, ispa.ISPA_Q8_INT8, 7
+    inv = ispa.ISPA_ERR_INVALID_ARG
+    a, b, c = FAKE, FAKE + (1 << 24), FAKE + (1 << 26)
+    # K must be a positive multiple of 16; the format must be known
+    assert L.ispa_quantize_rows(4, 24, a, E8, b, c, None) == inv
+    assert L.ispa_quantize_rows(4, 0, a, E8, b, c, None) == inv
+    assert L.ispa_quantize_rows(4, 32, a, BAD, b, c, None) == inv
+    assert L.ispa_quantize_rows(-1, 32, a, I8, b, c, None) == inv
+    assert L.ispa_quantize_rows(0, 32, None, I8, None, None, None) == ispa.ISPA_OK   # nothing to do
+    assert L.ispa_quantize_rows(4, 32, a + 8, I8, b, c, None) == inv               # unaligned
+    assert L.ispa_quantize_rows(4, 32, a, I8, a + 64, c, None) == inv              # q overlaps x
+    assert L.ispa_quantize_weight(40, 8, a, E8, b, c, None) == inv
+    assert L.ispa_quantize_weight(32, 8, a, E8, b, a + 16, None) == inv           # sw overlaps W
+    assert L.ispa_quantize_weight(32, 8, None, E8, b, c, None) == inv
+    # the product: N a multiple of 16, y apart from the inputs
+    assert L.ispa_gemm_q8(4, 24, 32, a, b, c, c + 4096, E8, c + 8192, ispa.ISPA_BF16, None) == inv
+    assert L.ispa_gemm_q8(4, 32, 40, a, b, c, c + 4096, E8, c + 8192, ispa.ISPA_BF16, None) == inv
+    assert L.ispa_gemm_q8(4, 32, 32, a, b, c, c + 4096, BAD, c + 8192, ispa.ISPA_BF16, None) == inv
+    assert L.ispa_gemm_q8(4, 32, 32, a, b, c, c + 4096, I8, c + 8192, 9, None) == inv
+    assert L.ispa_gemm_q8(4, 32, 32, a, b, c, c + 4096, I8, a, ispa.ISPA_F32, None) == inv
+    assert L.ispa_gemm_q8(0, 32, 32, None, None, None, None, I8, None, ispa.ISPA_F32, None) == ispa.ISPA_OK
+    # the post-switch step: workspace covers the bf16 path plus the 8-bit rows and their scales
+    d = _desc()
+    base = L.ispa_attn_local_proj_workspace_bytes(ctypes.byref(d))
+    need = L.ispa_attn_local_proj_q8_workspace_bytes(ctypes.byref(d))
+    rows = d.B * (d.cur_end - d.cur_begin) * d.tokens_per_frame
+    assert need >= base + rows * d.H * d.head_dim + rows * 4
+    assert L.ispa_attn_local_proj_q8(ctypes.byref(d), a, a, a, b, c, E8, 48, c + 4096, ispa.ISPA_BF16, FAKE,
+                                     need - 1, None) == inv
+    assert L.ispa_attn_local_proj_q8(ctypes.byref(d), a, a, a, b, c, BAD, 48, c + 4096, ispa.ISPA_BF16, FAKE,
+                                     need, None) == inv
+    assert L.ispa_attn_local_proj_q8(ctypes.byref(d), a, a, a, b, c, I8, 40, c + 4096, ispa.ISPA_BF16, FAKE,
+                                     need, None) == inv

@@ -278,3 +278,168 @@ def test_bounded_wait_runs_out_and_the_context_survives():
     dW, eps = _run_ridge(G, C, r2, 1e-4, True, 0)
     assert np.all(np.isfinite(dW)) and math.isfinite(eps)
     assert ispa.ispa_check_device_error() == 0
+
+
+# ---------------------------------------------------------------- W8A8 projection
+Q8_FORMATS = [(ispa.ISPA_Q8_E4M3, orc.Q8_E4M3), (ispa.ISPA_Q8_INT8, orc.Q8_INT8)]
+_E4M3_POS = orc.e4m3_decode(np.arange(0x80, dtype=np.uint8))       # codes 0x00..0x7F, increasing (NaN last)
+
+
+def q8_values(codes: np.ndarray, fmt: int) -> np.ndarray:
+    """Values of the kernels' bytes in the given format."""
+    codes = np.asarray(codes, np.uint8)
+    return orc.e4m3_decode(codes) if fmt == orc.Q8_E4M3 else codes.view(np.int8).astype(np.float64)
+
+
+def q8_codes(vals: np.ndarray, fmt: int) -> np.ndarray:
+    """Bytes of oracle values (values on the format's grid) for the kernels' inputs."""
+    vals = np.asarray(vals, np.float64)
+    if fmt == orc.Q8_INT8:
+        return vals.astype(np.int8).view(np.uint8)
+    a = np.abs(vals)
+    code = np.searchsorted(_E4M3_POS[:0x7F], a).astype(np.uint8)
+    assert np.array_equal(_E4M3_POS[code], a)
+    return np.where(vals < 0, code | 0x80, code).astype(np.uint8)
+
+
+def _gemm_q8_tolerance(qa, sa, qw, sw, fmt):
+    """int8: 0 (the int32 accumulator is exact).  e4m3: the products are exact, their sum is
+    not: one MMA step adds K = 32 of them to the accumulator.  The precision the tensor cores
+    keep inside an 8-bit step is not documented; the bound assumes at least 14 significant
+    bits per step, i.e. an error of at most 2^-13 of sum_k |qa qw| per step, times
+    ceil(K / 32) steps (a wrong tile, operand or scale errs by far more)."""
+    if fmt == orc.Q8_INT8:
+        return 0.0
+    steps = -(-qa.shape[1] // 32)
+    mag = (np.abs(qa) @ np.abs(qw)) * sa[:, None].astype(np.float64) * sw[None, :].astype(np.float64)
+    return steps * 2.0 ** -13 * mag + 1e-38
+
+
+@pytest.mark.parametrize("fmt,ofmt", Q8_FORMATS)
+def test_quantize_rows_bit_exact(fmt, ofmt):
+    M, K = 333, 272
+    x = si.activation_rows(M, K, ("gpu", "q8rows", ofmt))
+    q = torch.full((M, K), 0x55, dtype=torch.uint8, device="cuda")
+    sa = nan_like((M,), torch.float32)
+    ispa.ispa_quantize_rows(M, K, dev(x, torch.bfloat16), fmt, q, sa)
+    torch.cuda.synchronize()
+    ref_q, ref_s = orc.quantize_rows(x, ofmt)
+    assert np.array_equal(host(sa), ref_s)
+    assert np.array_equal(q8_values(host(q), ofmt), ref_q)
+    if ofmt == orc.Q8_E4M3:
+        assert ((ref_q != 0) & (np.abs(ref_q) < 2.0 ** -6)).any()    # the case reaches e4m3 subnormals
+
+
+@pytest.mark.parametrize("fmt,ofmt", Q8_FORMATS)
+def test_quantize_weight_bit_exact(fmt, ofmt):
+    K, N = 272, 208
+    W = si.projection_weight(K, N, ("gpu", "q8w", ofmt), "bf16")
+    W[:, 5] = 0.0
+    W[:, 7] *= 1e-3
+    W = si.round_to_bf16(W)                                          # the values the kernel reads
+    qT = torch.full((N, K), 0x55, dtype=torch.uint8, device="cuda")
+    sw = nan_like((N,), torch.float32)
+    ispa.ispa_quantize_weight(K, N, dev(W, torch.bfloat16), fmt, qT, sw)
+    torch.cuda.synchronize()
+    ref_q, ref_s = orc.quantize_cols(W, ofmt)
+    assert np.array_equal(host(sw), ref_s)
+    assert np.array_equal(q8_values(host(qT), ofmt).T, ref_q)
+
+
+def _gemm_q8_case(M, N, K, ofmt, key):
+    x = si.activation_rows(M, K, ("gpu", "q8g", ofmt) + key)
+    W = si.projection_weight(K, N, ("gpu", "q8g", ofmt) + key, "bf16")
+    qa, sa = orc.quantize_rows(x, ofmt)
+    qw, sw = orc.quantize_cols(W, ofmt)
+    return qa, sa, qw, sw
+
+
+@pytest.mark.parametrize("y_dt", [ispa.ISPA_F32, ispa.ISPA_BF16])
+@pytest.mark.parametrize("fmt,ofmt", Q8_FORMATS)
+def test_gemm_q8_matches_oracle(fmt, ofmt, y_dt):
+    # 3 M tiles (ragged), 3 N tiles (the last 16 wide), 9 K stages (the last 16 deep)
+    M, N, K = 333, 528, 1040
+    qa, sa, qw, sw = _gemm_q8_case(M, N, K, ofmt, ("small",))
+    tdt = torch.bfloat16 if y_dt == ispa.ISPA_BF16 else torch.float32
+    y = nan_like((M, N), tdt)
+    ispa.ispa_gemm_q8(M, N, K, dev(q8_codes(qa, ofmt), torch.uint8), dev(sa),
+                      dev(np.ascontiguousarray(q8_codes(qw, ofmt).T), torch.uint8), dev(sw), fmt, y, y_dt)
+    torch.cuda.synchronize()
+    ref = orc.gemm_q8(qa, sa, qw, sw, ofmt)
+    got = host(y).astype(np.float64)
+    tol = _gemm_q8_tolerance(qa, sa, qw, sw, ofmt)
+    if y_dt == ispa.ISPA_BF16:
+        if ofmt == orc.Q8_INT8:
+            assert np.array_equal(got, orc.bf16_round(ref))
+        else:
+            assert np.all(np.abs(got - ref) <= tol + 2.0 ** -8 * np.abs(ref))
+    elif ofmt == orc.Q8_INT8:
+        assert np.array_equal(got, np.asarray(ref, np.float64))
+    else:
+        assert np.all(np.abs(got - ref) <= tol), np.max(np.abs(got - ref) / (tol + 1e-30))
+        assert rel_fro(got, np.asarray(ref)) <= 1e-3, rel_fro(got, np.asarray(ref))
+    assert np.all(got[0] == 0)                                       # the zero row
+
+
+@pytest.mark.parametrize("fmt,ofmt", Q8_FORMATS)
+def test_gemm_q8_full_size_layer(fmt, ofmt):
+    """The projection of the 1.3B-shaped post-switch layer: 4680 rows (B = 1, 3 frames of 1560
+    tokens), D = Dout = 1536, every output against the oracle."""
+    M, N, K = 4680, 1536, 1536
+    qa, sa, qw, sw = _gemm_q8_case(M, N, K, ofmt, ("full",))
+    y = nan_like((M, N), torch.float32)
+    ispa.ispa_gemm_q8(M, N, K, dev(q8_codes(qa, ofmt), torch.uint8), dev(sa),
+                      dev(np.ascontiguousarray(q8_codes(qw, ofmt).T), torch.uint8), dev(sw), fmt, y, ispa.ISPA_F32)
+    torch.cuda.synchronize()
+    ref = orc.gemm_q8(qa, sa, qw, sw, ofmt)
+    got = host(y).astype(np.float64)
+    if ofmt == orc.Q8_INT8:
+        assert np.array_equal(got, np.asarray(ref, np.float64))
+    else:
+        assert np.all(np.abs(got - ref) <= _gemm_q8_tolerance(qa, sa, qw, sw, ofmt))
+        assert rel_fro(got, np.asarray(ref)) <= 1e-3, rel_fro(got, np.asarray(ref))
+
+
+@pytest.mark.parametrize("fmt,ofmt", Q8_FORMATS)
+def test_attn_local_proj_q8(fmt, ofmt):
+    sh = si.AttnShape(B=2, H=2, d=128, tpf=45, sink_frames=2, hist_begin=2, hist_end=6, cur_begin=6, cur_end=9,
+                      kv_frames=9)
+    data = si.iid_qkv(sh, "bf16", ("gpu", "projq8"))
+    D, Dout = sh.D, 192
+    W = si.projection_weight(D, Dout, ("gpu", "projq8"), "bf16")
+    dW = (0.02 * np.random.default_rng(6).standard_normal((D, Dout))).astype(np.float32)
+    Wn = si.round_to_bf16(W + dW)
+    qT = torch.empty((Dout, D), dtype=torch.uint8, device="cuda")
+    sw = torch.empty((Dout,), dtype=torch.float32, device="cuda")
+    ispa.ispa_quantize_weight(D, Dout, dev(Wn, torch.bfloat16), fmt, qT, sw)
+    desc = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_BF16)
+    ws = torch.empty(ispa.ispa_attn_local_proj_q8_workspace_bytes(desc), dtype=torch.uint8, device="cuda")
+    q, k, v = (dev(data[n], torch.bfloat16) for n in ("q", "k", "v"))
+    y = nan_like((sh.B, sh.Lq, Dout), torch.float32)
+    ispa.ispa_attn_local_proj_q8(desc, q, k, v, qT, sw, fmt, Dout, y, ispa.ISPA_F32, ws)
+    # the same step from its parts: A_loc (bf16) through an identity projection, then the 8-bit product
+    eye = torch.eye(D, dtype=torch.bfloat16, device="cuda")
+    a_loc = torch.empty((sh.B * sh.Lq, D), dtype=torch.bfloat16, device="cuda")
+    ws16 = torch.empty(ispa.ispa_attn_local_proj_workspace_bytes(desc), dtype=torch.uint8, device="cuda")
+    ispa.ispa_attn_local_proj(desc, q, k, v, eye, D, a_loc, ispa.ISPA_BF16, ws16)
+    qa = torch.empty((sh.B * sh.Lq, D), dtype=torch.uint8, device="cuda")
+    sa = torch.empty((sh.B * sh.Lq,), dtype=torch.float32, device="cuda")
+    ispa.ispa_quantize_rows(sh.B * sh.Lq, D, a_loc, fmt, qa, sa)
+    y2 = nan_like((sh.B * sh.Lq, Dout), torch.float32)
+    ispa.ispa_gemm_q8(sh.B * sh.Lq, Dout, D, qa, sa, qT, sw, fmt, y2, ispa.ISPA_F32)
+    torch.cuda.synchronize()
+    got = host(y)
+    assert np.array_equal(got.reshape(-1, Dout), host(y2))
+    # against the oracle's W8A8 step from the same synthetic inputs: the two sides' A_loc differ in
+    # the last bf16 bit of a few entries (fp32/fp16 kernel arithmetic vs fp64), which moves a few
+    # 8-bit codes by one step and, where it changes a row's amax, that row's scale by 2^-8.  One
+    # e4m3 step at a row's largest entry is 2^-4 amax; with amax ~ 4 RMS(a) and a weight ~ 4 RMS(w)
+    # it moves an output by ~2^-4 * 16 / sqrt(D) = 6e-2 of RMS(y) at D = 256, two such steps 0.12.
+    # An int8 step is 1/127 of amax, eight times smaller, but a row whose scale moves re-rounds
+    # every entry: the bound keeps a factor of two over one step at D = 256.
+    ref = orc.local_projection_q8(sh, data["q"], data["k"], data["v"], Wn, ofmt)
+    assert rel_fro(got, ref) <= 1e-2, rel_fro(got, ref)
+    assert max_over_rms(got, ref) <= (0.15 if ofmt == orc.Q8_E4M3 else 6e-2), max_over_rms(got, ref)
+    # and the W8A8 step stays near the bf16 step (quantisation error of a few percent)
+    ref16 = orc.local_projection(sh, data["q"], data["k"], data["v"], Wn)
+    assert rel_fro(got, ref16) <= 6e-2, rel_fro(got, ref16)
