@@ -19,7 +19,10 @@ the evicted L-layer 57 MB); between two uses of one layer's K/V the other
 passes stream 400 MB or more through the 126 MB L2, so no flush is needed.  The step runs on a stream of its own,
 captured once into a CUDA graph and replayed (warm-up and timed steps); the
 solve's component time replays a graph of the solve alone.  The end-to-end
-number calls the public API eagerly, with the host copies in the timed region.  Inputs are seeded synthetic tensors
+number calls the public API eagerly, with the host copies in the timed region.
+Outside the timed steps a component times the L-layer with its projection in
+8 bits (W8A8, e4m3 and int8; ispa_quantize_weight, ispa_attn_local_proj_q8)
+against the bf16 step.  Inputs are seeded synthetic tensors
 shaped like the pages' video generators (the trained models and prompts are
 not available).
 
@@ -119,16 +122,55 @@ def barrier(device):
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock and throttle reasons sampled while the timed region runs.
+
+    NVML (read-only queries, every 2 ms, so that a region of a few tens of ms
+    still gets samples); `nvidia-smi -lms 50` when NVML is not importable.
+    """
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.nvml = None
         self.lines = []
+        self.samples = []  # (sm MHz, max sm MHz, reason bits)
+        self.stop = threading.Event()
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            p = torch.cuda.get_device_properties(self.gpu)
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+
+    def _poll_nvml(self):
+        nv, h = self.nvml
+        mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        while not self.stop.is_set():
+            try:
+                self.samples.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)), mx,
+                                     int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))))
+            except Exception:
+                return
+            time.sleep(0.002)
 
     def __enter__(self):
+        try:
+            self.nvml = self._nvml_handle()
+            self.thread = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "50"], stdout=subprocess.PIPE,
@@ -149,6 +191,13 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def __exit__(self, *exc):
+        if self.nvml:
+            self.stop.set()
+            self.thread.join(timeout=5)
+            try:
+                self.nvml[0].nvmlShutdown()
+            except Exception:
+                pass
         if self.proc:
             self.proc.terminate()
             try:
@@ -158,7 +207,10 @@ class ClockSampler:
 
     def summary(self):
         sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for clk, cmax, bits in self.samples:
+            sm.append(clk)
+            mx.append(cmax)
+            reasons.update(n for n, b in self.REASONS if bits & b)
         for line in self.lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 7:
@@ -168,13 +220,14 @@ class ClockSampler:
                 mx.append(float(parts[1]))
             except ValueError:
                 continue
-            for n, p in zip(names, parts[3:7]):
+            for (n, _), p in zip(self.REASONS, parts[3:7]):
                 if p.lower().startswith("active"):
                     reasons.add(n)
+        src = "nvml" if self.nvml else "nvidia-smi"
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": src}
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": src}
 
 
 # DRAM traffic of the attention kernel (dram__bytes_read.sum + dram__bytes_write.sum
@@ -215,6 +268,70 @@ class Layer:
         data = si.iid_qkv(sh, "bf16", key)
         self.host = {n: torch.from_numpy(data[n]).to(torch.bfloat16).pin_memory() for n in ("q", "k", "v")}
         self.dev = {n: t.to(dev, non_blocking=False) for n, t in self.host.items()}
+
+
+def w8a8_component(ispa, torch, stream, dev, desc_L, LL, W_new, y_bf16, o_loc, T, D, ws_proj):
+    """Times the post-switch L-layer with its projection quantised to 8 bits.
+
+    Per format: the weight quantisation (once per layer at the switch), the
+    whole L-layer step (attention, row quantisation, 8-bit product) and its
+    two quantised parts alone, the product's rate, and the relative Frobenius
+    distance of its output from the bf16 step's.  Events on the launching
+    stream around a graph of repeated launches, mean per launch.
+    """
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(fn, reps=20):
+        # the launches are captured into a graph and replayed, so that the
+        # host's per-call cost (argument marshalling, tensor maps) stays out
+        fn()
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+            for _ in range(reps):
+                fn()
+        torch.cuda.set_stream(stream)
+        g.replay()
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        del g
+        return e0.elapsed_time(e1) / reps
+
+    Bq, Lq = y_bf16.shape[0], y_bf16.shape[1]
+    a16 = o_loc.to(torch.bfloat16).reshape(T, D)      # an A_loc-shaped bf16 operand
+    ws_q8 = torch.empty(ispa.ispa_attn_local_proj_q8_workspace_bytes(desc_L), device=dev, dtype=torch.uint8)
+    qT = torch.empty((D, D), device=dev, dtype=torch.uint8)
+    sw = torch.empty(D, device=dev, dtype=torch.float32)
+    qa = torch.empty((T, D), device=dev, dtype=torch.uint8)
+    sa = torch.empty(T, device=dev, dtype=torch.float32)
+    y8 = torch.empty((Bq, Lq, D), device=dev, dtype=torch.bfloat16)
+    q, k, v = LL.dev["q"], LL.dev["k"], LL.dev["v"]
+
+    def bf16_step():
+        ispa.ispa_attn_local_proj(desc_L, q, k, v, W_new, D, y_bf16, ispa.ISPA_BF16, ws_proj, stream=stream)
+
+    out = {"l_layer_bf16_ms": timed(bf16_step)}
+    out["gemm_bf16_ms"] = timed(lambda: ispa.ispa_gemm_bf16(T, D, D, a16, W_new, y8, ispa.ISPA_BF16, stream=stream))
+    out["gemm_bf16_tflops"] = 2.0 * T * D * D / (out["gemm_bf16_ms"] * 1e-3) / 1e12
+    for name, fmt in (("e4m3", ispa.ISPA_Q8_E4M3), ("int8", ispa.ISPA_Q8_INT8)):
+        r = {"quantize_weight_ms": timed(lambda: ispa.ispa_quantize_weight(D, D, W_new, fmt, qT, sw, stream=stream), 5)}
+
+        def q8_step():
+            ispa.ispa_attn_local_proj_q8(desc_L, q, k, v, qT, sw, fmt, D, y8, ispa.ISPA_BF16, ws_q8, stream=stream)
+
+        r["l_layer_ms"] = timed(q8_step)
+        bf16_step()
+        q8_step()
+        torch.cuda.synchronize(dev)
+        r["rel_diff_vs_bf16"] = float((y8.float() - y_bf16.float()).norm() / y_bf16.float().norm())
+        r["quantize_rows_ms"] = timed(lambda: ispa.ispa_quantize_rows(T, D, a16, fmt, qa, sa, stream=stream))
+        r["gemm_ms"] = timed(lambda: ispa.ispa_gemm_q8(T, D, D, qa, sa, qT, sw, fmt, y8, ispa.ISPA_BF16,
+                                                        stream=stream))
+        r["gemm_tflops"] = 2.0 * T * D * D / (r["gemm_ms"] * 1e-3) / 1e12
+        out[name] = r
+    return out
 
 
 def run_ours(args, world, rank, local):
@@ -359,6 +476,11 @@ def run_ours(args, world, rank, local):
     attn_launch_ms = float(np.mean(comp_attn))
     solve_launch_ms = float(np.mean(comp_solve))
 
+    # ---- the W8A8 post-switch L-layer: the same step with its projection in
+    # 8 bits (e4m3, int8), against the bf16 step; repeated launches, K/V of
+    # the evicted layer L2-resident for both alike
+    w8a8 = w8a8_component(ispa, torch, stream, dev, desc_L, layers[1], W_new, y["L"], o["loc"], T, D, ws_proj)
+
     # ---- end to end through the C ABI with host buffers
     h2d = sum(t.numel() * t.element_size() for Lr in layers for t in Lr.host.values()) + W_host.numel() * 4
     y_host = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in y.items()}
@@ -390,7 +512,7 @@ def run_ours(args, world, rank, local):
     e2e_ms = reduce_over_ranks(e0.elapsed_time(e1) / e2e_steps, "max", dev)
 
     return dict(ms_step=ms_step, work=work, attn_launch_ms=attn_launch_ms, solve_launch_ms=solve_launch_ms,
-                kv_evict=kv_evict,
+                kv_evict=kv_evict, w8a8=w8a8,
                 launches=launches, clocks=clocks.summary(), e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, world=world, rank=rank)
 
 
@@ -484,6 +606,59 @@ def config_block(world):
             "l2": "inputs larger than L2 (per step 457 MB of K/V: warmup and F-layer 200 MB each, evicted L-layer 57 MB)", "parallelism": f"replicas x{world}"}
 
 
+def run_proj_only(args):
+    """The post-switch projection alone at the layer's size (4680 x 1536 x 1536):
+    bf16, e4m3 and int8 products, each a graph of repeated launches, for profiling."""
+    import torch
+
+    import kv_cache_compression_two_b200 as ispa
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    sh = WORKLOAD.shape
+    T, D = sh.B * sh.Lq, sh.D
+    a16 = torch.from_numpy(si.activation_rows(T, D, ("bench", "proj"))).to(dev).to(torch.bfloat16)
+    w16 = torch.from_numpy(si.projection_weight(D, D, ("bench", "proj"), "bf16")).to(dev).to(torch.bfloat16)
+    y = torch.empty((T, D), device=dev, dtype=torch.bfloat16)
+    qa = torch.empty((T, D), device=dev, dtype=torch.uint8)
+    sa = torch.empty(T, device=dev, dtype=torch.float32)
+    qT = torch.empty((D, D), device=dev, dtype=torch.uint8)
+    sw = torch.empty(D, device=dev, dtype=torch.float32)
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(stream)
+    out = {}
+    cases = [("bf16", lambda: ispa.ispa_gemm_bf16(T, D, D, a16, w16, y, ispa.ISPA_BF16, stream=stream))]
+    for name, fmt in (("e4m3", ispa.ISPA_Q8_E4M3), ("int8", ispa.ISPA_Q8_INT8)):
+        cases.append((name, lambda fmt=fmt: (ispa.ispa_quantize_rows(T, D, a16, fmt, qa, sa, stream=stream),
+                                             ispa.ispa_quantize_weight(D, D, w16, fmt, qT, sw, stream=stream),
+                                             ispa.ispa_gemm_q8(T, D, D, qa, sa, qT, sw, fmt, y, ispa.ISPA_BF16,
+                                                               stream=stream))))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for name, fn in cases:
+        if name != "bf16":
+            fn()  # quantise once; the timed graph holds the product only
+            fmt = ispa.ISPA_Q8_E4M3 if name == "e4m3" else ispa.ISPA_Q8_INT8
+            fn = lambda fmt=fmt: ispa.ispa_gemm_q8(T, D, D, qa, sa, qT, sw, fmt, y, ispa.ISPA_BF16, stream=stream)
+        for _ in range(max(1, args.warmup)):
+            fn()
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream, capture_error_mode="thread_local"):
+            for _ in range(args.steps):
+                fn()
+        torch.cuda.set_stream(stream)
+        graph.replay()
+        e0.record(stream)
+        graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / args.steps
+        out[name] = {"ms": ms, "tflops": 2.0 * T * D * D / (ms * 1e-3) / 1e12}
+        del graph
+    ispa.ispa_check_device_error(stream)
+    print(json.dumps({"kernel": "projection", "M": T, "N": D, "K": D, **out}), flush=True)
+    return 0
+
+
 def run_attn_only(args):
     """The warmup split attention (fused merge) alone on the 1.3B-shaped layer, for profiling."""
     import torch
@@ -523,9 +698,12 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-rows", type=int, default=32, help="query rows of the oracle sample (0: skip it)")
-    ap.add_argument("--only", choices=["step", "attn"], default="step",
-                    help="attn: run only the split-attention launches (for profiling); prints their timing")
+    ap.add_argument("--only", choices=["step", "attn", "proj"], default="step",
+                    help="attn: only the split-attention launches; proj: only the post-switch projection "
+                         "(bf16, e4m3, int8 products); both for profiling, printing their timing")
     args = ap.parse_args(argv)
+    if args.only == "proj":
+        return run_proj_only(args)
     if args.only == "attn":
         return run_attn_only(args)
 
@@ -579,7 +757,7 @@ def main(argv=None):
                 "attn_split_tflops": achieved,
                 "query_tok_per_s": world * WORKLOAD.shape.B * WORKLOAD.shape.Lq / (r["attn_launch_ms"] * 1e-3),
                 "attn_split_ms": r["attn_launch_ms"], "solve_ms_per_layer": r["solve_launch_ms"],
-                "step_gflop": work["total"] / 1e9, "kv_eviction": r["kv_evict"]},
+                "step_gflop": work["total"] / 1e9, "kv_eviction": r["kv_evict"], "w8a8_l_layer": r["w8a8"]},
             "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (two-group attention + fused merge)",
                          "achieved": achieved, "peak": peak, "peak_source": peak_src, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": measured_traffic()},

@@ -389,6 +389,15 @@ ispa_status ispa_gemm_q8(int M, int N, int K, const void *q, const float *sa, co
                          const float *sw, ispa_q8_format fmt, void *y, ispa_dtype y_dtype,
                          ispa_stream_t stream);
 
+/*
+ * ispa_gemm_bf16: the bf16 projection of the post-switch layer alone,
+ * y [M, N] = A [M, K] W [K, N] (A, W bf16 row-major; fp32 accumulation on the
+ * tensor cores, rounded to y_dtype at the end) -- the product that W8A8
+ * replaces, with the same size and pointer rules as ispa_gemm_q8.
+ */
+ispa_status ispa_gemm_bf16(int M, int N, int K, const void *A, const void *W, void *y, ispa_dtype y_dtype,
+                           ispa_stream_t stream);
+
 size_t ispa_attn_local_proj_q8_workspace_bytes(const ispa_attn_desc *desc);
 
 /*

@@ -34,7 +34,7 @@ EXPORTED = ("ispa_version", "ispa_last_error", "ispa_launch_count", "ispa_check_
             "ispa_select_layers", "ispa_absorb_weight", "ispa_attn_local_proj_workspace_bytes",
             "ispa_attn_local_proj", "ispa_ridge_solve_noalloc", "ispa_kv_evicted_desc", "ispa_kv_evict_history",
             "ispa_kv_restore", "ispa_stats_reset", "ispa_selftest_wait_timeout", "ispa_quantize_rows",
-            "ispa_quantize_weight", "ispa_gemm_q8", "ispa_attn_local_proj_q8_workspace_bytes",
+            "ispa_quantize_weight", "ispa_gemm_q8", "ispa_gemm_bf16", "ispa_attn_local_proj_q8_workspace_bytes",
             "ispa_attn_local_proj_q8")
 RIDGE_NOALLOC_MAX_D = RIDGE_NOALLOC_MAX_DOUT = 1024
 
@@ -97,6 +97,7 @@ def lib() -> ctypes.CDLL:
         "ispa_quantize_rows": (_ci, [_ci, _ci, _vp, _ci, _vp, _vp, _vp]),
         "ispa_quantize_weight": (_ci, [_ci, _ci, _vp, _ci, _vp, _vp, _vp]),
         "ispa_gemm_q8": (_ci, [_ci, _ci, _ci, _vp, _vp, _vp, _vp, _ci, _vp, _ci, _vp]),
+        "ispa_gemm_bf16": (_ci, [_ci, _ci, _ci, _vp, _vp, _vp, _ci, _vp]),
         "ispa_attn_local_proj_q8_workspace_bytes": (_sz, [ctypes.POINTER(AttnDesc)]),
         "ispa_attn_local_proj_q8": (_ci, [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp, _ci, _ci, _vp, _ci,
                                           _vp, _sz, _vp]),
@@ -254,6 +255,10 @@ def ispa_quantize_weight(K: int, N: int, W, fmt: int, qT, sw, stream=None) -> No
 def ispa_gemm_q8(M: int, N: int, K: int, q, sa, qT, sw, fmt: int, y, y_dtype: int, stream=None) -> None:
     _check(lib().ispa_gemm_q8(M, N, K, _ptr(q), _ptr(sa), _ptr(qT), _ptr(sw), fmt, _ptr(y), y_dtype,
                               _stream(stream)))
+
+
+def ispa_gemm_bf16(M: int, N: int, K: int, A, W, y, y_dtype: int, stream=None) -> None:
+    _check(lib().ispa_gemm_bf16(M, N, K, _ptr(A), _ptr(W), _ptr(y), y_dtype, _stream(stream)))
 
 
 def ispa_attn_local_proj_q8_workspace_bytes(desc: AttnDesc) -> int:

@@ -440,6 +440,19 @@ ispa_status ispa_quantize_weight(int K, int N, const void *W, ispa_q8_format fmt
   return launch_quant_cols(K, N, W, fmt, qT, sw, (cudaStream_t)stream);
 }
 
+ispa_status ispa_gemm_bf16(int M, int N, int K, const void *A, const void *W, void *y, ispa_dtype y_dtype,
+                           ispa_stream_t stream) {
+  if (M < 0 || N < 0 || N % 16 != 0 || K < 16 || K % 16 != 0)
+    return fail(ISPA_ERR_INVALID_ARG, "need M >= 0, N a multiple of 16 and K a positive multiple of 16");
+  if (!dtype_ok(y_dtype)) return fail(ISPA_ERR_INVALID_ARG, "bad y dtype");
+  if (M == 0 || N == 0) return ISPA_OK;
+  if (!ptr_ok(A) || !ptr_ok(W) || !ptr_ok(y)) return fail(ISPA_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
+  const size_t yb = (size_t)M * N * (y_dtype == ISPA_BF16 ? 2 : 4);
+  if (overlaps(y, yb, A, (size_t)M * K * 2) || overlaps(y, yb, W, (size_t)K * N * 2))
+    return fail(ISPA_ERR_INVALID_ARG, "y must not overlap the inputs");
+  return launch_gemm_bf16(M, N, K, A, W, y, y_dtype, (cudaStream_t)stream);
+}
+
 ispa_status ispa_gemm_q8(int M, int N, int K, const void *q, const float *sa, const void *qT, const float *sw,
                          ispa_q8_format fmt, void *y, ispa_dtype y_dtype, ispa_stream_t stream) {
   if (M < 0 || N < 0 || N % 16 != 0 || !q8_k_ok(K))

@@ -381,6 +381,25 @@ def test_gemm_q8_matches_oracle(fmt, ofmt, y_dt):
     assert np.all(got[0] == 0)                                       # the zero row
 
 
+@pytest.mark.parametrize("y_dt", [ispa.ISPA_F32, ispa.ISPA_BF16])
+def test_gemm_bf16_matches_oracle(y_dt):
+    """The bf16 projection alone: exact products of bf16 operands summed in fp32 on the tensor
+    cores (96 MMA steps of K = 16 at K = 1536, each truncating at most 2^-23 of the running sum)."""
+    M, N, K = 333, 528, 1536
+    A = si.activation_rows(M, K, ("gpu", "gbf16"))
+    W = si.projection_weight(K, N, ("gpu", "gbf16"), "bf16")
+    tdt = torch.bfloat16 if y_dt == ispa.ISPA_BF16 else torch.float32
+    y = nan_like((M, N), tdt)
+    ispa.ispa_gemm_bf16(M, N, K, dev(A, torch.bfloat16), dev(W, torch.bfloat16), y, y_dt)
+    torch.cuda.synchronize()
+    ref = A.astype(np.float64) @ W.astype(np.float64)
+    tol = 96 * 2.0 ** -23 * (np.abs(A).astype(np.float64) @ np.abs(W).astype(np.float64))
+    got = host(y)
+    if y_dt == ispa.ISPA_BF16:
+        tol = tol + 2.0 ** -8 * np.abs(ref)
+    assert np.all(np.abs(got - ref) <= tol + 1e-38)
+
+
 @pytest.mark.parametrize("fmt,ofmt", Q8_FORMATS)
 def test_gemm_q8_full_size_layer(fmt, ofmt):
     """The projection of the 1.3B-shaped post-switch layer: 4680 rows (B = 1, 3 frames of 1560
