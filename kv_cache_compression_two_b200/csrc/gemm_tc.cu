@@ -56,7 +56,11 @@ ispa_status launch_gemm_bf16(int M, int N, int K, const void *A, const void *B, 
                         CU_TENSOR_MAP_SWIZZLE_128B)) != ISPA_OK)
       return st;
   }
-  {
+  bool b_blk = false;
+  if ((st = map_mn_blocked(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, N, K, N, 64, tcg::BN / 64,
+                           CU_TENSOR_MAP_SWIZZLE_128B, &b_blk)) != ISPA_OK)
+    return st;
+  if (!b_blk) {
     const uint64_t dims[2] = {(uint64_t)N, (uint64_t)K};
     const uint64_t strides[1] = {(uint64_t)N * 2};
     const uint32_t box[2] = {64, 64};
@@ -74,7 +78,7 @@ ispa_status launch_gemm_bf16(int M, int N, int K, const void *A, const void *B, 
   P.idesc = make_idesc(tcg::BM, tcg::BN, 1, 0, 1);
   P.r2 = nullptr;
   P.p[0] = tcg::SubProblem{N, (N + tcg::BN - 1) / tcg::BN, 0,
-                           ydt == ISPA_BF16 ? tcg::EPI_STORE_BF16 : tcg::EPI_STORE_F32, Y, N};
+                           ydt == ISPA_BF16 ? tcg::EPI_STORE_BF16 : tcg::EPI_STORE_F32, Y, N, b_blk ? 1 : 0};
   P.p[1] = P.p[0];
   P.n_tiles0 = P.tiles_m * P.p[0].tiles_n;
   P.n_tiles = P.n_tiles0;

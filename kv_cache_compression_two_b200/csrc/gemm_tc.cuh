@@ -66,6 +66,7 @@ struct SubProblem {
   int epi;        // Epi
   void *out;      // [M, N] row-major, ld = ldo
   long long ldo;
+  int b_blk;      // 1: B's map delivers a whole stage in one box (see the operand staging note)
 };
 
 struct Params {
@@ -76,6 +77,7 @@ struct Params {
   int kind_tf32;  // 1: kind::tf32 (fp32 operands), 0: kind::f16 with bf16 operands
   int kind_f8;    // 8-bit K-major operands: 1 = e4m3 (kind::f8f6f4), 2 = int8 (kind::i8, int32 accumulator)
   int a_mn, b_mn; // operand majorness (1 = MN-major)
+  int a_blk;      // 1: A's map delivers a whole stage in one box
   uint32_t idesc;
   double *r2;     // EPI_STORE_TF32_SQ accumulator
   const float *row_scale, *col_scale;  // EPI_SCALED factors
@@ -227,6 +229,68 @@ __device__ __forceinline__ void epilogue_chunk(const Params &P, const SubProblem
   }
 }
 
+// Store epilogue through shared memory, for the plain stores (bf16 or fp32)
+// and the scaled 8-bit one, with N % 16 == 0 and 16-byte aligned rows.  Each
+// epilogue warp owns 32 rows of the tile: it moves its accumulator rows out
+// of tensor memory (lane = row), writes them to its own staging area in
+// 16-byte chunks (chunk j of row r at slot j ^ r, so that neither the row-wise
+// writes nor the column-wise reads below collide in a bank), then writes the
+// rows back one at a time with the whole warp: 512 (bf16) or 1024 (fp32)
+// contiguous bytes per row, instead of every store instruction touching 32
+// rows.  The staging areas reuse the operand stages, idle once the
+// accumulator is complete.
+template <bool BF16_OUT, bool SCALED>
+__device__ __forceinline__ void epilogue_staged(const Params &P, const SubProblem &sp, uint32_t tmem_rows, int quarter,
+                                                int lane, int m0, int n0, uint8_t *stage) {
+  constexpr int ELEM = BF16_OUT ? 2 : 4;
+  constexpr int CPR = BN * ELEM / 16;  // 16-byte chunks per row
+  const int N = sp.N;
+  const int row = m0 + quarter * 32 + lane;
+  const float rs = SCALED && row < P.M ? P.row_scale[row] : 1.f;
+  const int n_chunks = min(BN, N - n0 + 31) / 32;
+  uint8_t *my = stage + lane * (CPR * 16);
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(tmem_rows + c * 32, r);
+    tmem_wait_ld();
+    if (c >= n_chunks) continue;
+    float cs = 1.f;
+    if (SCALED) {
+      const int col = n0 + c * 32 + lane;
+      cs = col < N ? P.col_scale[col] : 0.f;
+    }
+    float x[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float acc = SCALED && P.kind_f8 == 2 ? __int2float_rn((int)r[j]) : __uint_as_float(r[j]);
+      x[j] = SCALED ? acc * rs * __shfl_sync(0xffffffffu, cs, j) : acc;
+    }
+    if (BF16_OUT) {
+#pragma unroll
+      for (int v = 0; v < 4; ++v)
+        *reinterpret_cast<uint4 *>(my + (((c * 4 + v) ^ lane) * 16)) =
+            make_uint4(pack_bf16x2(x[8 * v], x[8 * v + 1]), pack_bf16x2(x[8 * v + 2], x[8 * v + 3]),
+                       pack_bf16x2(x[8 * v + 4], x[8 * v + 5]), pack_bf16x2(x[8 * v + 6], x[8 * v + 7]));
+    } else {
+#pragma unroll
+      for (int v = 0; v < 8; ++v)
+        *reinterpret_cast<float4 *>(my + (((c * 8 + v) ^ lane) * 16)) =
+            make_float4(x[4 * v], x[4 * v + 1], x[4 * v + 2], x[4 * v + 3]);
+    }
+  }
+  __syncwarp();
+  for (int rr = 0; rr < 32; ++rr) {
+    const int grow = m0 + quarter * 32 + rr;
+    if (grow >= P.M) break;
+    const uint8_t *src = stage + rr * (CPR * 16);
+    uint8_t *dst = static_cast<uint8_t *>(sp.out) + ((long long)grow * sp.ldo + n0) * ELEM;
+#pragma unroll
+    for (int j = lane; j < CPR; j += 32)
+      if (n0 + j * (16 / ELEM) < N)
+        *reinterpret_cast<uint4 *>(dst + j * 16) = *reinterpret_cast<const uint4 *>(src + ((j ^ rr) * 16));
+  }
+}
+
 #ifdef ISPA_DEFINE_GEMM_KERNEL
 // tma maps: ta = A operand; tb[prob] = B operand of each sub-problem; with
 // split3, ta_lo and tb_lo hold the remainders of A and of B (problem 0 only).
@@ -311,11 +375,19 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint8_t *b = sB + s * TILE_B_BYTES;
         if (!P.a_mn) {
           tma_load_2d(a, mA, full + s, k0, m0);
+        } else if (P.a_blk) {  // 3D map: (element in block, k, block of e128)
+          tma_load_3d(a, mA, full + s, 0, k0, m0 / e128);
         } else {
           for (int c = 0; c < BM / e128; ++c) tma_load_2d(a + c * mn_box_bytes, mA, full + s, m0 + c * e128, k0);
         }
-        if (!P.b_mn) {  // 128-row boxes, one after the other
-          for (int c = 0; c < BN / 128; ++c) tma_load_2d(b + c * TILE_BYTES, mB, full + s, k0, n0 + c * 128);
+        if (!P.b_mn) {
+          if (sp.b_blk) {  // one 256-row box
+            tma_load_2d(b, mB, full + s, k0, n0);
+          } else {         // 128-row boxes, one after the other
+            for (int c = 0; c < BN / 128; ++c) tma_load_2d(b + c * TILE_BYTES, mB, full + s, k0, n0 + c * 128);
+          }
+        } else if (sp.b_blk) {
+          tma_load_3d(b, mB, full + s, 0, k0, n0 / e128);
         } else {
           for (int c = 0; c < BN / e128; ++c) tma_load_2d(b + c * mn_box_bytes, mB, full + s, n0 + c * e128, k0);
         }
@@ -362,7 +434,23 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int quarter = warp & 3;
     const int row = m0 + quarter * 32 + lane;
     double sq = 0.0;
-    if (wait_parity(done, 0, P.err, abort, 3)) {
+    const bool staged = (sp.epi == EPI_STORE_BF16 || sp.epi == EPI_STORE_F32 || sp.epi == EPI_SCALED) &&
+                        sp.N % 16 == 0 && sp.ldo % 16 == 0 && (reinterpret_cast<uintptr_t>(sp.out) & 15) == 0;
+    const uint32_t tmem_rows = tmem + ((uint32_t)(quarter * 32) << 16);
+    uint8_t *stage = smem + quarter * (32 * BN * 4);  // 32 KB per warp inside the operand stages
+    if (staged) {
+      if (wait_parity(done, 0, P.err, abort, 3)) {
+        tc_fence_after();
+        const bool bf16_out = sp.epi == EPI_STORE_BF16 || (sp.epi == EPI_SCALED && P.out_bf16);
+        if (sp.epi == EPI_SCALED) {
+          if (bf16_out) epilogue_staged<true, true>(P, sp, tmem_rows, quarter, lane, m0, n0, stage);
+          else epilogue_staged<false, true>(P, sp, tmem_rows, quarter, lane, m0, n0, stage);
+        } else {
+          if (bf16_out) epilogue_staged<true, false>(P, sp, tmem_rows, quarter, lane, m0, n0, stage);
+          else epilogue_staged<false, false>(P, sp, tmem_rows, quarter, lane, m0, n0, stage);
+        }
+      }
+    } else if (wait_parity(done, 0, P.err, abort, 3)) {
       tc_fence_after();
       const int n_chunks = min(BN, sp.N - n0 + 31) / 32;
       for (int c = 0; c < BN / 32; ++c) {
@@ -404,6 +492,41 @@ inline ispa_status map2d_f32_ld(CUtensorMap *m, const void *base, int inner, int
   const uint32_t box[2] = {(uint32_t)box_inner, (uint32_t)box_outer};
   return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box,
                    mn_major ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Blocked view of an MN-major operand, so that one TMA load fills a whole
+// stage.  The copy engine spends a roughly fixed time per box (a 4 KB box
+// moves at a third of the rate of a 32 KB one), and an MN-major stage of
+// 128-byte-wide column blocks would otherwise take one box per block.  The
+// row-major [outer, inner] matrix (leading dimension ld elements of elem
+// bytes, inner = M or N) is seen as three dimensions: the e128 elements of a
+// 128-byte block, the outer (K) rows, and the blocks, whose stride (128 bytes)
+// is smaller than the row stride; the box {e128, box_k, blocks} lands in
+// shared memory as blocks one after the other, the layout of the per-block
+// boxes.  Only when inner is a whole number of blocks and holds at least one
+// box of them (else *blocked = false and the caller keeps per-block boxes).
+inline ispa_status map_mn_blocked(CUtensorMap *m, CUtensorMapDataType dt, int elem, const void *base, int inner,
+                                  int outer, long long ld, int box_k, int blocks, CUtensorMapSwizzle sw,
+                                  bool *blocked) {
+  const int e128 = 128 / elem;
+  *blocked = inner % e128 == 0 && inner / e128 >= blocks;
+  if (!*blocked) return ISPA_OK;
+  const uint64_t dims[3] = {(uint64_t)e128, (uint64_t)outer, (uint64_t)(inner / e128)};
+  const uint64_t strides[2] = {(uint64_t)ld * elem, 128};
+  const uint32_t box[3] = {(uint32_t)e128, (uint32_t)box_k, (uint32_t)blocks};
+  return make_tmap(m, dt, 3, base, dims, strides, box, sw);
+}
+
+// MN-major fp32 operand map for a tile of `blocks` 32-element blocks: blocked
+// when possible, per-block 2D boxes otherwise.
+inline ispa_status map_f32_mn(CUtensorMap *m, const void *base, int inner, int outer, long long ld, int box_k,
+                              int blocks, int *blk) {
+  bool b = false;
+  ispa_status st = map_mn_blocked(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, inner, outer, ld, box_k, blocks,
+                                  CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B, &b);
+  if (st != ISPA_OK) return st;
+  *blk = b ? 1 : 0;
+  return b ? ISPA_OK : map2d_f32_ld(m, base, inner, outer, ld, 32, box_k, true);
 }
 
 inline ispa_status map2d_f32(CUtensorMap *m, const void *base, int inner, int outer, int box_inner, int box_outer,

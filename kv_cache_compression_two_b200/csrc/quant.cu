@@ -140,17 +140,20 @@ ispa_status launch_gemm_q8(int M, int N, int K, const void *qa, const float *sa,
   DevErr err;
   ispa_status st = device_err(&err);
   if (st != ISPA_OK) return st;
+  // A: 128-row boxes; B: one 256-row box per stage (the copy engine's time is
+  // mostly per box, so a stage in fewer boxes arrives sooner)
   CUtensorMap ta, tb;
   const uint64_t strides[1] = {(uint64_t)K};
-  const uint32_t box[2] = {128, 128};
   {
     const uint64_t dims[2] = {(uint64_t)K, (uint64_t)M};
+    const uint32_t box[2] = {128, (uint32_t)tcg::BM};
     if ((st = make_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, qa, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) !=
         ISPA_OK)
       return st;
   }
   {
     const uint64_t dims[2] = {(uint64_t)K, (uint64_t)N};
+    const uint32_t box[2] = {128, (uint32_t)tcg::BN};
     if ((st = make_tmap(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, qT, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) !=
         ISPA_OK)
       return st;
@@ -167,7 +170,7 @@ ispa_status launch_gemm_q8(int M, int N, int K, const void *qa, const float *sa,
   P.row_scale = sa;
   P.col_scale = sw;
   P.out_bf16 = ydt == ISPA_BF16;
-  P.p[0] = tcg::SubProblem{N, (N + tcg::BN - 1) / tcg::BN, 0, tcg::EPI_SCALED, y, N};
+  P.p[0] = tcg::SubProblem{N, (N + tcg::BN - 1) / tcg::BN, 0, tcg::EPI_SCALED, y, N, 1};
   P.p[1] = P.p[0];
   P.n_tiles0 = P.tiles_m * P.p[0].tiles_n;
   P.n_tiles = P.n_tiles0;

@@ -778,11 +778,16 @@ ispa_status tc3_product(int M, int N, int K, const float *a_hi, const float *a_l
   if (M <= 0 || N <= 0 || K <= 0) return ISPA_OK;
   CUtensorMap ta, tal, tb, tbl;
   ispa_status st;
-  const int a_inner = a_trans ? M : K, a_outer = a_trans ? K : M, a_box_outer = a_trans ? 32 : tcg::BM;
-  if ((st = map2d_f32_ld(&ta, a_hi, a_inner, a_outer, lda, 32, a_box_outer, a_trans)) != ISPA_OK) return st;
-  if ((st = map2d_f32_ld(&tal, a_lo, a_inner, a_outer, lda, 32, a_box_outer, a_trans)) != ISPA_OK) return st;
-  if ((st = map2d_f32_ld(&tb, b_hi, N, K, ldb, 32, 32, true)) != ISPA_OK) return st;
-  if ((st = map2d_f32_ld(&tbl, b_lo, N, K, ldb, 32, 32, true)) != ISPA_OK) return st;
+  int a_blk = 0, b_blk = 0;
+  if (a_trans) {
+    if ((st = map_f32_mn(&ta, a_hi, M, K, lda, 32, tcg::BM / 32, &a_blk)) != ISPA_OK) return st;
+    if ((st = map_f32_mn(&tal, a_lo, M, K, lda, 32, tcg::BM / 32, &a_blk)) != ISPA_OK) return st;
+  } else {
+    if ((st = map2d_f32_ld(&ta, a_hi, K, M, lda, 32, tcg::BM, false)) != ISPA_OK) return st;
+    if ((st = map2d_f32_ld(&tal, a_lo, K, M, lda, 32, tcg::BM, false)) != ISPA_OK) return st;
+  }
+  if ((st = map_f32_mn(&tb, b_hi, N, K, ldb, 32, tcg::BN / 32, &b_blk)) != ISPA_OK) return st;
+  if ((st = map_f32_mn(&tbl, b_lo, N, K, ldb, 32, tcg::BN / 32, &b_blk)) != ISPA_OK) return st;
   tcg::Params P{};
   P.M = M;
   P.K = K;
@@ -790,12 +795,13 @@ ispa_status tc3_product(int M, int N, int K, const float *a_hi, const float *a_l
   P.kind_tf32 = 1;
   P.a_mn = a_trans ? 1 : 0;
   P.b_mn = 1;
+  P.a_blk = a_blk;
   P.idesc = make_idesc(tcg::BM, tcg::BN, 2, P.a_mn, 1);
   P.r2 = nullptr;
   P.tri = tri;
   P.chunk_kt = kTc3ChunkKt;
   P.nchunk = ((K + 31) / 32 + kTc3ChunkKt - 1) / kTc3ChunkKt;
-  P.p[0] = tcg::SubProblem{N, (N + tcg::BN - 1) / tcg::BN, 0, tcg::EPI_ATOMIC_F32, out, ldo};
+  P.p[0] = tcg::SubProblem{N, (N + tcg::BN - 1) / tcg::BN, 0, tcg::EPI_ATOMIC_F32, out, ldo, b_blk};
   P.p[1] = P.p[0];
   P.n_tiles0 = P.tiles_m * P.p[0].tiles_n;
   P.err = err;

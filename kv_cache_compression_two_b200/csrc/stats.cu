@@ -109,8 +109,9 @@ ispa_status launch_stats(int T, int D, int Dout, const float *a_loc, const float
   // launch 1: R = dA W
   {
     CUtensorMap ta, tb;
+    int b_blk = 0;
     if ((st = map2d_f32(&ta, w.dA, D, T, 32, 128, false)) != ISPA_OK) return st;
-    if ((st = map2d_f32(&tb, w.Wr, Dout, D, 32, 32, true)) != ISPA_OK) return st;
+    if ((st = map_f32_mn(&tb, w.Wr, Dout, D, Dout, 32, tcg::BN / 32, &b_blk)) != ISPA_OK) return st;
     tcg::Params P{};
     P.M = T;
     P.K = D;
@@ -120,7 +121,7 @@ ispa_status launch_stats(int T, int D, int Dout, const float *a_loc, const float
     P.b_mn = 1;
     P.idesc = make_idesc(tcg::BM, tcg::BN, 2, 0, 1);
     P.r2 = r2;
-    P.p[0] = tcg::SubProblem{Dout, (Dout + tcg::BN - 1) / tcg::BN, 0, tcg::EPI_STORE_TF32_SQ, w.R, Dout};
+    P.p[0] = tcg::SubProblem{Dout, (Dout + tcg::BN - 1) / tcg::BN, 0, tcg::EPI_STORE_TF32_SQ, w.R, Dout, b_blk};
     P.n_tiles0 = P.tiles_m * P.p[0].tiles_n;
     P.n_tiles = P.n_tiles0;
     P.p[1] = P.p[0];
@@ -129,9 +130,12 @@ ispa_status launch_stats(int T, int D, int Dout, const float *a_loc, const float
   }
   // launch 2: G (upper) += Ar^T Ar, C += Ar^T R
   {
-    CUtensorMap ta, tr;
-    if ((st = map2d_f32(&ta, w.Ar, D, T, 32, 32, true)) != ISPA_OK) return st;
-    if ((st = map2d_f32(&tr, w.R, Dout, T, 32, 32, true)) != ISPA_OK) return st;
+    // Ar is A (128-wide tiles) and the B of G (256-wide tiles): one map each
+    CUtensorMap ta, tg, tr;
+    int a_blk = 0, g_blk = 0, r_blk = 0;
+    if ((st = map_f32_mn(&ta, w.Ar, D, T, D, 32, tcg::BM / 32, &a_blk)) != ISPA_OK) return st;
+    if ((st = map_f32_mn(&tg, w.Ar, D, T, D, 32, tcg::BN / 32, &g_blk)) != ISPA_OK) return st;
+    if ((st = map_f32_mn(&tr, w.R, Dout, T, Dout, 32, tcg::BN / 32, &r_blk)) != ISPA_OK) return st;
     tcg::Params P{};
     P.M = D;
     P.K = T;
@@ -139,14 +143,15 @@ ispa_status launch_stats(int T, int D, int Dout, const float *a_loc, const float
     P.kind_tf32 = 1;
     P.a_mn = 1;
     P.b_mn = 1;
+    P.a_blk = a_blk;
     P.idesc = make_idesc(tcg::BM, tcg::BN, 2, 1, 1);
     P.r2 = nullptr;
-    P.p[0] = tcg::SubProblem{D, (D + tcg::BN - 1) / tcg::BN, 1, tcg::EPI_ACCUM_F32, G, D};
-    P.p[1] = tcg::SubProblem{Dout, (Dout + tcg::BN - 1) / tcg::BN, 0, tcg::EPI_ACCUM_F32, C, Dout};
+    P.p[0] = tcg::SubProblem{D, (D + tcg::BN - 1) / tcg::BN, 1, tcg::EPI_ACCUM_F32, G, D, g_blk};
+    P.p[1] = tcg::SubProblem{Dout, (Dout + tcg::BN - 1) / tcg::BN, 0, tcg::EPI_ACCUM_F32, C, Dout, r_blk};
     P.n_tiles0 = tcg::upper_tile_count(P.tiles_m, P.p[0].tiles_n);
     P.n_tiles = P.n_tiles0 + P.tiles_m * P.p[1].tiles_n;
     P.err = err;
-    if ((st = launch_tc_gemm(ta, ta, tr, P, s)) != ISPA_OK) return st;
+    if ((st = launch_tc_gemm(ta, tg, tr, P, s)) != ISPA_OK) return st;
   }
   return ISPA_OK;
 }
