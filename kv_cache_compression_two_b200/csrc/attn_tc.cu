@@ -328,8 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wait_parity(&empty[st], ph ^ 1, P.err, abort, is_k ? 11 : 12)) break;
         uint8_t *dst = is_k ? sm.k[st] : sm.v[st];
         mbar_arrive_expect_tx(&full[st], kTileBytes);
-        tma_load_3d(dst, map, &full[st], x0, it.t0, b);
-        tma_load_3d(dst + kBoxBytes, map, &full[st], x0 + 64, it.t0, b);
+        tma_load_4d(dst, map, &full[st], 0, it.t0, x0 / 64, b);  // both 64-column halves, one box
         pend |= 1u << st;
         ph_bits = (ph_bits & ~(1u << st)) | (ph << st);
       }
@@ -594,11 +593,17 @@ ispa_status launch_typed(const CUtensorMap &tk, const CUtensorMap &tv, const __n
   return cuda_status(cudaGetLastError(), "tcgen05 attention launch");
 }
 
-ispa_status map3d_16(CUtensorMap *m, const void *base, int D, int rows, int B, CUtensorMapDataType dt) {
-  const uint64_t dims[3] = {(uint64_t)D, (uint64_t)rows, (uint64_t)B};
-  const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)D * 2 * (uint64_t)rows};
-  const uint32_t box[3] = {64, 128, 1};
-  return make_tmap(m, dt, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+// K or V [B, rows, D] (16-bit, D = H * 128) seen as (64 columns of a 128-byte
+// block, row, block of the row, instance): the block stride (128 bytes) is
+// below the row stride, so that one box {64, 128, 2, 1} brings both 64-column
+// halves of a head's 128-row tile, half after half as the swizzled operand
+// layout wants them (half the copy instructions of two 16 KB boxes; the
+// launch time is the same either way, the copies not being the bound here).
+ispa_status map_kv16(CUtensorMap *m, const void *base, int D, int rows, int B, CUtensorMapDataType dt) {
+  const uint64_t dims[4] = {64, (uint64_t)rows, (uint64_t)D / 64, (uint64_t)B};
+  const uint64_t strides[3] = {(uint64_t)D * 2, 128, (uint64_t)D * 2 * (uint64_t)rows};
+  const uint32_t box[4] = {64, 128, 2, 1};
+  return make_tmap(m, dt, 4, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -647,8 +652,8 @@ ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float 
   P.v_unscale = v_unscale;
 
   CUtensorMap tk, tv;
-  if ((st = map3d_16(&tk, k, D, g.Lkv, d.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) != ISPA_OK) return st;
-  if ((st = map3d_16(&tv, v16, D, g.Lkv, d.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16)) != ISPA_OK) return st;
+  if ((st = map_kv16(&tk, k, D, g.Lkv, d.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) != ISPA_OK) return st;
+  if ((st = map_kv16(&tv, v16, D, g.Lkv, d.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16)) != ISPA_OK) return st;
   P.H = d.H;
   P.Lq = g.Lq;
   P.q_tiles = (g.Lq + kTileQ - 1) / kTileQ;
