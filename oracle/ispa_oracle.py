@@ -51,9 +51,9 @@ def attend_group(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> T
     """Softmax attention of queries q [n, d] over one key group k, v [m, d].
 
     Returns the group's normalised output O [n, d] and its log-sum-exp
-    L [n] = log(sum_j exp(scale * q.k_j)).  Each group "returns both its
-    weighted value output and the LSE state associated with softmax
-    normalization" [EN-notes, Key Designs 1].  An empty group returns O = 0 and
+    L [n] = log(sum_j exp(scale * q.k_j)).  Each group yields its normalised
+    value output together with the log-sum-exp of its softmax normaliser
+    [EN-notes, Key Designs 1].  An empty group returns O = 0 and
     L = -inf, so that it carries no attention mass in a merge.
     """
     q = np.asarray(q, np.float64)
@@ -136,8 +136,8 @@ def full_attention(shape, q, k, v, scale: float = None, rows: Sequence[int] = No
                    row_block: int = 512) -> Tuple[np.ndarray, np.ndarray]:
     """Monolithic softmax attention over every KV frame (the F-layer path after the switch).
 
-    F-layers "continue using the full-context path" [EN-notes, Key Designs 3;
-    DE-summary 2, "Speichereffiziente Inferenz"].
+    F-layers keep attending over the full context after the switch [EN-notes,
+    Key Designs 3; DE-summary 2, "Speichereffiziente Inferenz"].
     """
     d = q.shape[-1]
     scale = 1.0 / math.sqrt(d) if not scale else scale
@@ -323,7 +323,7 @@ def absorb_layer(chunks: List[Dict[str, np.ndarray]], W: np.ndarray, lam: float,
 
     ``chunks`` holds the split-attention outputs of every warmup chunk (dicts
     from :func:`split_attention`).  Rows of all chunks are stacked (the
-    statistics are "accumulated during forward passes").  Returns G, C, r2,
+    statistics are summed over the warmup's forward calls).  Returns G, C, r2,
     lambda, dW, eps (direct form) and the stacked rows.
     """
     A_loc = np.concatenate([heads_to_rows(c["O_loc"]) for c in chunks], axis=0)
