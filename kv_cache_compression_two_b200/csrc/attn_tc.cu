@@ -68,10 +68,17 @@ struct AttnParams {
 // fp16 copy of V.  P = exp(S - m) is rounded to 16 bits before the PV product;
 // in fp16 (11 significant bits) that rounding is 8x finer than in bf16, which
 // keeps the output error well inside the parity tolerance.  tcgen05 kind::f16
-// needs both operands in the same type, so V is converted once per call:
-// each head of each instance is scaled by a power of two 2^s so that its
-// largest |v| lies in [2^14, 2^15) (exact in fp16, far from overflow), and the
-// epilogue multiplies O by 2^-s (exact).  Only the rows the tiles read are
+// needs both operands in the same type, so V is converted once per call.  A
+// bf16 value (8 significant bits) is exact in fp16 when its magnitude lies in
+// [2^-17, 65504], and below 2^-14 fp16 keeps an absolute spacing of 2^-24, so
+// a converted entry is off by at most 2^-25.  One pass converts V as it is and
+// records, per head of each instance, the largest |v| and the sum of v^2.  A
+// head whose largest |v| reaches 2^15 (overflow margin), or whose RMS is
+// below 2^-10 (where 2^-25 would no longer be small against the 2^-11
+// relative rounding of its typical entries), is converted again by a second
+// kernel with a power-of-two scale 2^s that puts its largest |v| in
+// [2^14, 2^15), and the epilogue multiplies O by 2^-s (exact); for the other
+// heads that kernel only writes 2^-s = 1.  Only the rows the tiles read are
 // converted: every range rounded up to whole 128-row tiles.
 // ---------------------------------------------------------------------------
 struct VPrep {
@@ -80,11 +87,13 @@ struct VPrep {
   int ext_begin[3], ext_end[3];  // row extents the tiles touch
 };
 
-// Per-(instance, head) max |v|.  Each thread keeps one 16-byte column group c8
-// (8 values of one head) and walks rows; the 16 lanes that cover one head
-// combine by shuffles and one lane per head issues the atomic.
-__global__ void __launch_bounds__(256) v_amax_kernel(VPrep p, const __nv_bfloat16 *__restrict__ v,
-                                                     unsigned int *amax_bits) {
+// Conversion pass.  Each thread keeps one 16-byte column group c8 (8 values
+// of one head) and walks rows, converting them unscaled; the 16 lanes that
+// cover one head combine their largest |v| and sum of squares by shuffles and
+// one lane per head issues the atomics (non-negative floats order like their
+// bit patterns).
+__global__ void __launch_bounds__(256) v_prep_kernel(VPrep p, const __nv_bfloat16 *__restrict__ v, __half *v16,
+                                                     unsigned int *amax_bits, float *sumsq) {
   const int D = p.H * kD;
   const int vec_per_row = D / 8;                       // multiple of 16 (kD / 8 = 16 per head)
   const int b = blockIdx.y;
@@ -93,24 +102,36 @@ __global__ void __launch_bounds__(256) v_amax_kernel(VPrep p, const __nv_bfloat1
   const int tid = blockIdx.x * blockDim.x + threadIdx.x;
   const int c8 = tid % vec_per_row;
   const int r0 = tid / vec_per_row;
-  float m = 0.f;
+  float mx = 0.f, ss = 0.f;
   if (r0 < row_step) {
     for (int e = 0; e < p.n_ext; ++e)
       for (int row = p.ext_begin[e] + r0; row < p.ext_end[e]; row += row_step) {
-        const uint4 in = __ldg(reinterpret_cast<const uint4 *>(v + ((long long)b * p.Lkv + row) * D) + c8);
+        const long long off = ((long long)b * p.Lkv + row) * D + c8 * 8;
+        const uint4 in = __ldg(reinterpret_cast<const uint4 *>(v + off));
         const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+        uint32_t o[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[j]));
-          m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+          mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+          ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+          __half2 hh = __floats2half2_rn(f.x, f.y);
+          o[j] = *reinterpret_cast<uint32_t *>(&hh);
         }
+        *reinterpret_cast<uint4 *>(v16 + off) = make_uint4(o[0], o[1], o[2], o[3]);
       }
   }
   // vec_per_row = 16 H and warps start at multiples of 32, so lanes 16k..16k+15
   // hold the 16 column groups of one head of one row: reduce them by shuffles.
 #pragma unroll
-  for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((threadIdx.x & 15) == 0 && r0 < row_step) atomicMax(amax_bits + b * p.H + (c8 * 8) / kD, __float_as_uint(m));
+  for (int o = 8; o > 0; o >>= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  }
+  if ((threadIdx.x & 15) == 0 && r0 < row_step) {
+    atomicMax(amax_bits + b * p.H + (c8 * 8) / kD, __float_as_uint(mx));
+    atomicAdd(sumsq + b * p.H + (c8 * 8) / kD, ss);
+  }
 }
 
 __device__ __forceinline__ int v_exponent(unsigned int amax_bits) {
@@ -119,23 +140,36 @@ __device__ __forceinline__ int v_exponent(unsigned int amax_bits) {
   return 14 - ilogbf(a);  // a * 2^s in [2^14, 2^15)
 }
 
-__global__ void __launch_bounds__(256) v_to_f16_kernel(VPrep p, const __nv_bfloat16 *__restrict__ v,
-                                                       const unsigned int *__restrict__ amax_bits, __half *v16,
-                                                       float *v_unscale) {
+// The heads the unscaled copy does not serve (see the note above): largest
+// |v| from 2^15 up, or RMS below 2^-10 (sum of squares below count * 2^-20).
+__device__ __forceinline__ bool v_needs_scale(unsigned int amax_bits, float sumsq, float count) {
+  return !(__uint_as_float(amax_bits) < 32768.f) || sumsq < count * 0x1p-20f;
+}
+
+// Second pass: v_unscale for every head, and the scaled copy of the heads
+// v_needs_scale picks (same thread layout as v_prep_kernel).
+__global__ void __launch_bounds__(256) v_fix_kernel(VPrep p, const __nv_bfloat16 *__restrict__ v, __half *v16,
+                                                    const unsigned int *__restrict__ amax_bits,
+                                                    const float *__restrict__ sumsq, float *v_unscale) {
   const int D = p.H * kD;
   const int vec_per_row = D / 8;
-  if (blockIdx.x == 0)
-    for (int i = threadIdx.x; i < p.B * p.H; i += blockDim.x) v_unscale[i] = ldexpf(1.f, -v_exponent(amax_bits[i]));
-  for (int e = 0; e < p.n_ext; ++e) {
-    const long long rows = p.ext_end[e] - p.ext_begin[e];
-    const long long n = (long long)p.B * rows * vec_per_row;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-      const int c8 = (int)(i % vec_per_row);
-      const long long br = i / vec_per_row;
-      const int b = (int)(br / rows);
-      const long long row = p.ext_begin[e] + br % rows;
-      const int h = (c8 * 8) / kD;
-      const float scale = ldexpf(1.f, v_exponent(amax_bits[b * p.H + h]));
+  const int b = blockIdx.y;
+  const int lanes = gridDim.x * blockDim.x;
+  const int row_step = lanes / vec_per_row;
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+  const int c8 = tid % vec_per_row;
+  const int r0 = tid / vec_per_row;
+  if (r0 >= row_step) return;
+  const int hb = b * p.H + (c8 * 8) / kD;
+  float count = 0.f;
+  for (int e = 0; e < p.n_ext; ++e) count += (float)(p.ext_end[e] - p.ext_begin[e]) * kD;
+  const bool fix = v_needs_scale(amax_bits[hb], sumsq[hb], count);
+  const int sexp = fix ? v_exponent(amax_bits[hb]) : 0;
+  if (r0 == 0 && (c8 * 8) % kD == 0) v_unscale[hb] = ldexpf(1.f, -sexp);
+  if (!fix) return;
+  const float scale = ldexpf(1.f, sexp);
+  for (int e = 0; e < p.n_ext; ++e)
+    for (int row = p.ext_begin[e] + r0; row < p.ext_end[e]; row += row_step) {
       const long long off = ((long long)b * p.Lkv + row) * D + c8 * 8;
       const uint4 in = *reinterpret_cast<const uint4 *>(v + off);
       const uint32_t w[4] = {in.x, in.y, in.z, in.w};
@@ -150,7 +184,6 @@ __global__ void __launch_bounds__(256) v_to_f16_kernel(VPrep p, const __nv_bfloa
       }
       *reinterpret_cast<uint4 *>(v16 + off) = make_uint4(o[0], o[1], o[2], o[3]);
     }
-  }
 }
 
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
@@ -611,7 +644,7 @@ size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 }  // namespace
 
 size_t attn_tc_workspace_bytes(int B, int H, int Lkv) {
-  return a256((size_t)B * Lkv * H * kD * 2) + 2 * a256((size_t)B * H * 4);
+  return a256((size_t)B * Lkv * H * kD * 2) + 3 * a256((size_t)B * H * 4);
 }
 
 ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float scale, const void *q,
@@ -626,8 +659,10 @@ ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float 
   // ---- fp16 copy of the V rows the tiles read (workspace)
   char *ws = static_cast<char *>(workspace);
   __half *v16 = reinterpret_cast<__half *>(ws);
+  const size_t head_words = a256((size_t)d.B * d.H * 4);
   unsigned int *amax = reinterpret_cast<unsigned int *>(ws + a256((size_t)d.B * g.Lkv * D * 2));
-  float *v_unscale = reinterpret_cast<float *>(ws + a256((size_t)d.B * g.Lkv * D * 2) + a256((size_t)d.B * d.H * 4));
+  float *sumsq = reinterpret_cast<float *>(reinterpret_cast<char *>(amax) + head_words);
+  float *v_unscale = reinterpret_cast<float *>(reinterpret_cast<char *>(amax) + 2 * head_words);
   VPrep vp{};
   vp.B = d.B;
   vp.H = d.H;
@@ -641,12 +676,14 @@ ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float 
   };
   for (int r = 0; r < g.n_loc; ++r) add_ext(g.loc_begin[r], g.loc_end[r]);
   add_ext(g.hist_begin, g.hist_end);
-  cudaError_t e = cudaMemsetAsync(amax, 0, (size_t)d.B * d.H * 4, s);
+  cudaError_t e = cudaMemsetAsync(amax, 0, 2 * head_words, s);  // amax and sumsq
   if (e != cudaSuccess) return cuda_status(e, "attention workspace clear");
   const int vec_per_row = D / 8;
-  const int amax_blocks = max((vec_per_row + 255) / 256, (sm_count() * 8 + d.B - 1) / d.B);
-  v_amax_kernel<<<dim3(amax_blocks, d.B), 256, 0, s>>>(vp, static_cast<const __nv_bfloat16 *>(v), amax);
-  v_to_f16_kernel<<<sm_count() * 8, 256, 0, s>>>(vp, static_cast<const __nv_bfloat16 *>(v), amax, v16, v_unscale);
+  const int prep_blocks = max((vec_per_row + 255) / 256, (sm_count() * 8 + d.B - 1) / d.B);
+  const int fix_blocks = max((vec_per_row + 255) / 256, 2);
+  const __nv_bfloat16 *vb = static_cast<const __nv_bfloat16 *>(v);
+  v_prep_kernel<<<dim3(prep_blocks, d.B), 256, 0, s>>>(vp, vb, v16, amax, sumsq);
+  v_fix_kernel<<<dim3(fix_blocks, d.B), 256, 0, s>>>(vp, vb, v16, amax, sumsq, v_unscale);
   note_launch(2);
   if ((st = cuda_status(cudaGetLastError(), "V conversion launch")) != ISPA_OK) return st;
   P.v_unscale = v_unscale;

@@ -115,6 +115,36 @@ def test_bf16_optional_outputs():
     assert np.all(np.isnan(O["hist"]))
 
 
+def test_bf16_v_outside_the_fp16_range():
+    """Heads whose V the unscaled fp16 copy does not serve (|v| up to ~2^20; RMS ~2^-20) take
+    the power-of-two-scaled copy; the others, one of them holding a few entries of 2^-19, stay
+    unscaled.  Each (instance, head) is checked against the oracle relative to its own output
+    scale."""
+    sh = si.AttnShape(B=2, H=3, d=128, tpf=40, sink_frames=1, hist_begin=1, hist_end=5, cur_begin=5, cur_end=7,
+                      kv_frames=7)
+    data = si.iid_qkv(sh, "bf16", ("gpu", "vrange"))
+    v = data["v"].copy()
+    v[0, :, 0] *= np.float32(2.0 ** 17)     # largest |v| ~ 5 * 2^17 > 65504
+    v[1, :, 2] *= np.float32(2.0 ** -20)    # nonzero |v| below 2^-17
+    v[1, 5, 1] = np.float32(2.0 ** -19)     # one tiny entry in an otherwise normal head
+    data["v"] = si.round_to_bf16(v)
+    q, k, vv = dev(data["q"], torch.bfloat16), dev(data["k"], torch.bfloat16), dev(data["v"], torch.bfloat16)
+    o = {n: nan_like((sh.B, sh.Lq, sh.H, 128), torch.float32) for n in ("loc", "hist", "full")}
+    l = {n: nan_like((sh.B, sh.Lq, sh.H), torch.float32) for n in ("loc", "hist", "full")}
+    desc = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_F32)
+    ws = torch.empty(ispa.ispa_attn_split_workspace_bytes(desc), dtype=torch.uint8, device="cuda")
+    ispa.ispa_attn_split(desc, q, k, vv, o["loc"], l["loc"], o["hist"], l["hist"], o["full"], l["full"], workspace=ws)
+    torch.cuda.synchronize()
+    ref = orc.split_attention(sh, data["q"], data["k"], data["v"])
+    for n in ("loc", "hist", "full"):
+        got = host(o[n])
+        for b in range(sh.B):
+            for h in range(sh.H):
+                r = ref["O_" + n][b, :, h]
+                rms = np.sqrt(np.mean(r ** 2))
+                assert np.abs(got[b, :, h] - r).max() <= 1e-2 * rms, (n, b, h)
+
+
 def test_bf16_large_scores_and_rescaling():
     """Scores scaled up so the running maximum moves by far more than the rescale threshold."""
     sh = si.AttnShape(B=1, H=1, d=128, tpf=64, sink_frames=1, hist_begin=1, hist_end=6, cur_begin=6, cur_end=8,
