@@ -22,7 +22,9 @@ solve's component time replays a graph of the solve alone.  The end-to-end
 number calls the public API eagerly, with the host copies in the timed region.
 Outside the timed steps a component times the L-layer with its projection in
 8 bits (W8A8, e4m3 and int8; ispa_quantize_weight, ispa_attn_local_proj_q8)
-against the bf16 step.  Inputs are seeded synthetic tensors
+against the bf16 step, and another the fused warmup step (ispa_warmup_fused:
+the attention epilogue writes the statistics' operands) against the two calls
+it replaces.  Inputs are seeded synthetic tensors
 shaped like the pages' video generators (the trained models and prompts are
 not available).
 
@@ -270,6 +272,26 @@ class Layer:
         self.dev = {n: t.to(dev, non_blocking=False) for n, t in self.host.items()}
 
 
+def graph_time(torch, stream, dev, fn, reps):
+    """Mean ms of fn over a CUDA graph of reps calls, replayed between two events
+    on the launching stream (after one eager call and one warm replay)."""
+    fn()
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+        for _ in range(reps):
+            fn()
+    torch.cuda.set_stream(stream)
+    g.replay()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    del g
+    return e0.elapsed_time(e1) / reps
+
+
 def w8a8_component(ispa, torch, stream, dev, desc_L, LL, W_new, y_bf16, o_loc, T, D, ws_proj):
     """Times the post-switch L-layer with its projection quantised to 8 bits.
 
@@ -481,6 +503,25 @@ def run_ours(args, world, rank, local):
     # the evicted layer L2-resident for both alike
     w8a8 = w8a8_component(ispa, torch, stream, dev, desc_L, layers[1], W_new, y["L"], o["loc"], T, D, ws_proj)
 
+    # ---- the fused warmup step (attention writing the statistics' operands)
+    # against the two calls it replaces, on the warmup layer
+    Lw = layers[0]
+
+    def two_calls():
+        ispa.ispa_attn_split(desc_warm, Lw.dev["q"], Lw.dev["k"], Lw.dev["v"], o["loc"], l["loc"], o["hist"],
+                             l["hist"], o["full"], l["full"], workspace=ws_attn, stream=stream)
+        ispa.ispa_accum_stats(T, D, D, o["loc"], o["full"], W32, G, C, r2, ispa.ISPA_PREC_TF32, ws_stats,
+                              stream=stream)
+
+    ws_fused = torch.empty(ispa.ispa_warmup_fused_workspace_bytes(desc_warm, D), device=dev, dtype=torch.uint8)
+
+    def fused():
+        ispa.ispa_warmup_fused(desc_warm, Lw.dev["q"], Lw.dev["k"], Lw.dev["v"], W32, D, o["full"], l["full"], G, C,
+                               r2, ws_fused, stream=stream)
+
+    warm_fused = {"two_calls_ms": graph_time(torch, stream, dev, two_calls, 5),
+                  "fused_ms": graph_time(torch, stream, dev, fused, 5)}
+
     # ---- end to end through the C ABI with host buffers
     h2d = sum(t.numel() * t.element_size() for Lr in layers for t in Lr.host.values()) + W_host.numel() * 4
     y_host = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in y.items()}
@@ -512,7 +553,7 @@ def run_ours(args, world, rank, local):
     e2e_ms = reduce_over_ranks(e0.elapsed_time(e1) / e2e_steps, "max", dev)
 
     return dict(ms_step=ms_step, work=work, attn_launch_ms=attn_launch_ms, solve_launch_ms=solve_launch_ms,
-                kv_evict=kv_evict, w8a8=w8a8,
+                kv_evict=kv_evict, w8a8=w8a8, warm_fused=warm_fused,
                 launches=launches, clocks=clocks.summary(), e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, world=world, rank=rank)
 
 
@@ -757,7 +798,8 @@ def main(argv=None):
                 "attn_split_tflops": achieved,
                 "query_tok_per_s": world * WORKLOAD.shape.B * WORKLOAD.shape.Lq / (r["attn_launch_ms"] * 1e-3),
                 "attn_split_ms": r["attn_launch_ms"], "solve_ms_per_layer": r["solve_launch_ms"],
-                "step_gflop": work["total"] / 1e9, "kv_eviction": r["kv_evict"], "w8a8_l_layer": r["w8a8"]},
+                "step_gflop": work["total"] / 1e9, "kv_eviction": r["kv_evict"], "w8a8_l_layer": r["w8a8"],
+                "warmup_fused": r["warm_fused"]},
             "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (two-group attention + fused merge)",
                          "achieved": achieved, "peak": peak, "peak_source": peak_src, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": measured_traffic()},

@@ -200,6 +200,35 @@ ispa_status ispa_accum_stats(int T, int D, int Dout, const float *a_loc, const f
                              ispa_stream_t stream);
 
 /* ------------------------------------------------------------------------- */
+/* Fused warmup step                                                          */
+/* ------------------------------------------------------------------------- */
+size_t ispa_warmup_fused_workspace_bytes(const ispa_attn_desc *desc, int Dout);
+
+/*
+ * One warmup forward step of a layer in one pass over the attention outputs
+ * [EN-notes, Key Designs 1-2: the two groups' outputs come out of the same
+ * attention pass, and the statistics are gathered during warmup at no extra
+ * attention cost]: the two-group attention with its fused merge writes the
+ * layer's full-context output O_full (fp32) and L_full, and, from the same
+ * epilogue, the operands of the statistics (A_loc and A_full - A_loc rounded to
+ * tf32) straight into the workspace; then G += A_loc^T A_loc (upper triangle),
+ * C += A_loc^T R and r2 += ||R||^2 with R = (A_full - A_loc) W, as
+ * ispa_accum_stats with ISPA_PREC_TF32 computes them from the same values.
+ * The separate per-group outputs O_loc / O_hist and the statistics' rounding
+ * pass over them are not materialised.
+ *   desc      bf16 inputs, head_dim 128 (its out_dtype is ignored: fp32)
+ *   W         [D, Dout] fp32, D = H * 128, Dout % 32 == 0
+ *   o_full    [B, Lq, H, 128] fp32, l_full [B, Lq, H] fp32
+ *   G, C, r2  as for ispa_accum_stats (accumulated into)
+ *   workspace >= ispa_warmup_fused_workspace_bytes(desc, Dout)
+ * Asynchronous; ISPA_ERR_INVALID_ARG / ISPA_ERR_UNSUPPORTED as the calls it
+ * combines.
+ */
+ispa_status ispa_warmup_fused(const ispa_attn_desc *desc, const void *q, const void *k, const void *v,
+                              const float *W, int Dout, float *o_full, float *l_full, float *G, float *C,
+                              double *r2, void *workspace, size_t workspace_bytes, ispa_stream_t stream);
+
+/* ------------------------------------------------------------------------- */
 /* Closed-form absorption                                                     */
 /* ------------------------------------------------------------------------- */
 size_t ispa_ridge_workspace_bytes(int D, int Dout);

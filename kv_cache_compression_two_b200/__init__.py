@@ -35,7 +35,7 @@ EXPORTED = ("ispa_version", "ispa_last_error", "ispa_launch_count", "ispa_check_
             "ispa_attn_local_proj", "ispa_ridge_solve_noalloc", "ispa_kv_evicted_desc", "ispa_kv_evict_history",
             "ispa_kv_restore", "ispa_stats_reset", "ispa_selftest_wait_timeout", "ispa_quantize_rows",
             "ispa_quantize_weight", "ispa_gemm_q8", "ispa_gemm_bf16", "ispa_attn_local_proj_q8_workspace_bytes",
-            "ispa_attn_local_proj_q8")
+            "ispa_attn_local_proj_q8", "ispa_warmup_fused_workspace_bytes", "ispa_warmup_fused")
 RIDGE_NOALLOC_MAX_D = RIDGE_NOALLOC_MAX_DOUT = 1024
 
 
@@ -99,6 +99,9 @@ def lib() -> ctypes.CDLL:
         "ispa_gemm_q8": (_ci, [_ci, _ci, _ci, _vp, _vp, _vp, _vp, _ci, _vp, _ci, _vp]),
         "ispa_gemm_bf16": (_ci, [_ci, _ci, _ci, _vp, _vp, _vp, _ci, _vp]),
         "ispa_attn_local_proj_q8_workspace_bytes": (_sz, [ctypes.POINTER(AttnDesc)]),
+        "ispa_warmup_fused_workspace_bytes": (_sz, [ctypes.POINTER(AttnDesc), _ci]),
+        "ispa_warmup_fused": (_ci, [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _ci, _vp, _vp, _vp, _vp, _vp, _vp,
+                                    _sz, _vp]),
         "ispa_attn_local_proj_q8": (_ci, [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp, _ci, _ci, _vp, _ci,
                                           _vp, _sz, _vp]),
     }
@@ -272,6 +275,19 @@ def ispa_attn_local_proj_q8(desc: AttnDesc, q, k, v, qT, sw, fmt: int, Dout: int
     _check(lib().ispa_attn_local_proj_q8(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(qT), _ptr(sw), fmt,
                                          Dout, _ptr(y), y_dtype, _ptr(workspace), workspace_bytes,
                                          _stream(stream)))
+
+
+def ispa_warmup_fused_workspace_bytes(desc: AttnDesc, Dout: int) -> int:
+    return int(lib().ispa_warmup_fused_workspace_bytes(ctypes.byref(desc), Dout))
+
+
+def ispa_warmup_fused(desc: AttnDesc, q, k, v, W, Dout: int, o_full, l_full, G, C, r2, workspace,
+                      workspace_bytes: int = 0, stream=None) -> None:
+    if workspace is not None and not isinstance(workspace, int):
+        workspace_bytes = workspace_bytes or workspace.numel() * workspace.element_size()
+    _check(lib().ispa_warmup_fused(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(W), Dout, _ptr(o_full),
+                                   _ptr(l_full), _ptr(G), _ptr(C), _ptr(r2), _ptr(workspace), workspace_bytes,
+                                   _stream(stream)))
 
 
 def ispa_kv_evicted_desc(desc: AttnDesc) -> AttnDesc:

@@ -302,6 +302,54 @@ ispa_status ispa_accum_stats(int T, int D, int Dout, const float *a_loc, const f
   return launch_stats(T, D, Dout, a_loc, a_full, W, G, C, r2, prec, workspace, (cudaStream_t)stream);
 }
 
+namespace {
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+}  // namespace
+
+size_t ispa_warmup_fused_workspace_bytes(const ispa_attn_desc *desc, int Dout) {
+  GroupRanges g;
+  float scale;
+  if (!desc || Dout < 1 || attn_ranges(desc, &g, &scale) != ISPA_OK) return 0;
+  const int T = desc->B * g.Lq, D = desc->H * desc->head_dim;
+  return round256(stats_workspace_bytes(T, D, Dout, ISPA_PREC_TF32)) + round256((size_t)T * desc->H * 4) +
+         attn_tc_workspace_bytes(desc->B, desc->H, g.Lkv);
+}
+
+ispa_status ispa_warmup_fused(const ispa_attn_desc *desc, const void *q, const void *k, const void *v,
+                              const float *W, int Dout, float *o_full, float *l_full, float *G, float *C,
+                              double *r2, void *workspace, size_t workspace_bytes, ispa_stream_t stream) {
+  GroupRanges g;
+  float scale;
+  ispa_status st = attn_ranges(desc, &g, &scale);
+  if (st != ISPA_OK) return st;
+  if (desc->in_dtype != ISPA_BF16 || desc->head_dim != 128)
+    return fail(ISPA_ERR_UNSUPPORTED, "the fused warmup is compiled for bf16 inputs with head_dim 128");
+  const int D = desc->H * desc->head_dim;
+  const long long T = (long long)desc->B * g.Lq;
+  if (Dout < 32 || Dout % 32 != 0) return fail(ISPA_ERR_INVALID_ARG, "Dout must be a positive multiple of 32");
+  if (T * D > (1LL << 34) || (long long)D * Dout > (1LL << 31)) return fail(ISPA_ERR_INVALID_ARG, "sizes too large");
+  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(W) || !ptr_ok(o_full) || !ptr_ok(l_full) || !ptr_ok(G) ||
+      !ptr_ok(C) || !r2)
+    return fail(ISPA_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
+  const size_t need = ispa_warmup_fused_workspace_bytes(desc, Dout);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return fail(ISPA_ERR_INVALID_ARG, "workspace needs %zu bytes (16-byte aligned)", need);
+  if (T == 0) return ISPA_OK;
+  ispa_attn_desc d = *desc;
+  d.out_dtype = ISPA_F32;
+  char *w = static_cast<char *>(workspace);
+  const size_t stats_bytes = round256(stats_workspace_bytes((int)T, D, Dout, ISPA_PREC_TF32));
+  float *lse_loc = reinterpret_cast<float *>(w + stats_bytes);
+  void *attn_ws = w + stats_bytes + round256((size_t)T * d.H * 4);
+  float *dA = nullptr, *Ar = nullptr;
+  stats_row_operands(w, (int)T, D, Dout, &dA, &Ar);
+  cudaStream_t s = (cudaStream_t)stream;
+  // O_loc goes to the statistics' Ar buffer (left there rounded to tf32), dA next to it
+  st = launch_attn_tc(d, g, scale, q, k, v, Ar, lse_loc, nullptr, nullptr, o_full, l_full, attn_ws, s, dA);
+  if (st != ISPA_OK) return st;
+  return launch_stats((int)T, D, Dout, nullptr, nullptr, W, G, C, r2, ISPA_PREC_TF32, w, s, true);
+}
+
 size_t ispa_ridge_workspace_bytes(int D, int Dout) {
   if (D < 1 || Dout < 1) return 0;
   return ridge_workspace_bytes(D, Dout);

@@ -61,6 +61,10 @@ struct AttnParams {
   const float *v_unscale;  // [B * H]: 2^-s of the fp16 copy of V (see prepare_v)
   void *o_loc, *o_hist, *o_full;
   float *l_loc, *l_hist, *l_full;
+  // Statistics operands (fp32 outputs only; see launch_attn_tc): when set, the
+  // epilogue writes dA = tf32(O_full - O_loc) here, and leaves tf32(O_loc) in
+  // o_loc, the operands of the absorption statistics.
+  float *stats_dA;
   DevErr err;
 };
 
@@ -576,13 +580,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!row_ok) continue;
         if (dst) store_row32<TO>(dst + c * 32, xo);
         if (write_full) {
+          float y[32];
           if (!is_loc) {
-            float y[32];
             load_row32<TO>(o_loc + c * 32, y);
 #pragma unroll
             for (int t = 0; t < 32; ++t) xo[t] = wa * y[t] + wb * xo[t];
+          } else {
+#pragma unroll
+            for (int t = 0; t < 32; ++t) y[t] = xo[t];  // no history: O_full = O_loc
           }
           store_row32<TO>(o_full + c * 32, xo);
+          if (P.stats_dA) {  // the statistics operands, rounded as the statistics pass rounds them
+            float da[32];
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+              da[t] = to_tf32_rn(xo[t] - y[t]);
+              y[t] = to_tf32_rn(y[t]);
+            }
+            store_row32<float>(P.stats_dA + head_row * kD + c * 32, da);
+            store_row32<TO>(o_loc + c * 32, y);
+          }
         }
       }
       if (write_full && row_ok) P.l_full[head_row] = L_full;
@@ -649,7 +666,7 @@ size_t attn_tc_workspace_bytes(int B, int H, int Lkv) {
 
 ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float scale, const void *q,
                            const void *k, const void *v, void *o_loc, float *l_loc, void *o_hist, float *l_hist,
-                           void *o_full, float *l_full, void *workspace, cudaStream_t s) {
+                           void *o_full, float *l_full, void *workspace, cudaStream_t s, float *stats_dA) {
   if (g.Lq == 0) return ISPA_OK;
   AttnParams P{};
   ispa_status st = device_err(&P.err);
@@ -714,6 +731,7 @@ ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float 
   P.o_loc = o_loc;
   P.o_hist = o_hist;
   P.o_full = o_full;
+  P.stats_dA = (d.out_dtype == ISPA_F32 && o_full) ? stats_dA : nullptr;
   P.l_loc = l_loc;
   P.l_hist = l_hist;
   P.l_full = l_full;

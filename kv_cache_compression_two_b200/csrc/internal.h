@@ -60,12 +60,18 @@ ispa_status launch_attn_simt(const ispa_attn_desc &d, const GroupRanges &g, floa
 size_t attn_tc_workspace_bytes(int B, int H, int Lkv);
 ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float scale, const void *q,
                            const void *k, const void *v, void *o_loc, float *l_loc, void *o_hist,
-                           float *l_hist, void *o_full, float *l_full, void *workspace, cudaStream_t s);
+                           float *l_hist, void *o_full, float *l_full, void *workspace, cudaStream_t s,
+                           float *stats_dA = nullptr);
 
 // stats
 size_t stats_workspace_bytes(int T, int D, int Dout, ispa_precision prec);
+// rows_ready: the tf32 operands dA and Ar of the rows are already in the workspace
+// (written by the attention epilogue); a_loc and a_full are then unused.
 ispa_status launch_stats(int T, int D, int Dout, const float *a_loc, const float *a_full, const float *W,
-                         float *G, float *C, double *r2, ispa_precision prec, void *ws, cudaStream_t s);
+                         float *G, float *C, double *r2, ispa_precision prec, void *ws, cudaStream_t s,
+                         bool rows_ready = false);
+// Where the attention epilogue puts the operands for launch_stats(rows_ready).
+void stats_row_operands(void *ws, int T, int D, int Dout, float **dA, float **Ar);
 
 // ridge
 size_t ridge_workspace_bytes(int D, int Dout);

@@ -79,8 +79,15 @@ size_t stats_workspace_bytes(int T, int D, int Dout, ispa_precision prec) {
   return 2 * a256((size_t)T * D * 4) + a256((size_t)D * Dout * 4) + a256((size_t)T * Dout * 4);
 }
 
+void stats_row_operands(void *ws, int T, int D, int Dout, float **dA, float **Ar) {
+  TF32Ws w = carve_tf32(ws, T, D, Dout);
+  *dA = w.dA;
+  *Ar = w.Ar;
+}
+
 ispa_status launch_stats(int T, int D, int Dout, const float *a_loc, const float *a_full, const float *W,
-                         float *G, float *C, double *r2, ispa_precision prec, void *ws, cudaStream_t s) {
+                         float *G, float *C, double *r2, ispa_precision prec, void *ws, cudaStream_t s,
+                         bool rows_ready) {
   if (T == 0) return ISPA_OK;
   if (prec == ISPA_PREC_F32) {
     float *R = static_cast<float *>(ws);
@@ -99,7 +106,7 @@ ispa_status launch_stats(int T, int D, int Dout, const float *a_loc, const float
   ispa_status st = device_err(&err);
   if (st != ISPA_OK) return st;
   TF32Ws w = carve_tf32(ws, T, D, Dout);
-  const long long n4_rows = (long long)T * D / 4, n4_w = (long long)D * Dout / 4;
+  const long long n4_rows = rows_ready ? 0 : (long long)T * D / 4, n4_w = (long long)D * Dout / 4;
   prep_tf32_kernel<<<sm_count() * 8, 256, 0, s>>>(n4_rows, n4_w, (const float4 *)a_loc, (const float4 *)a_full,
                                                   (const float4 *)W, (float4 *)w.dA, (float4 *)w.Ar, (float4 *)w.Wr);
   note_launch();

@@ -222,3 +222,21 @@ def test_w8a8_validation():
                                      need, None) == inv
     assert L.ispa_attn_local_proj_q8(ctypes.byref(d), a, a, a, b, c, I8, 40, c + 4096, ispa.ISPA_BF16, FAKE,
                                      need, None) == inv
+
+
+def test_warmup_fused_validation():
+    L = ispa.lib()
+    inv = ispa.ISPA_ERR_INVALID_ARG
+    d = _desc()
+    need = L.ispa_warmup_fused_workspace_bytes(ctypes.byref(d), 64)
+    T, D = d.B * (d.cur_end - d.cur_begin) * d.tokens_per_frame, d.H * d.head_dim
+    assert need >= 2 * T * D * 4 + D * 64 * 4 + T * 64 * 4          # dA, Ar, W in tf32, R
+    assert L.ispa_warmup_fused_workspace_bytes(ctypes.byref(d), 0) == 0
+    args = [FAKE] * 3 + [FAKE, 64] + [FAKE] * 5
+    assert L.ispa_warmup_fused(ctypes.byref(d), *args, FAKE, need - 1, None) == inv      # workspace short
+    bad = list(args); bad[4] = 48                                                        # Dout % 32
+    assert L.ispa_warmup_fused(ctypes.byref(d), *bad, FAKE, need, None) == inv
+    bad = list(args); bad[9] = None                                                      # r2
+    assert L.ispa_warmup_fused(ctypes.byref(d), *bad, FAKE, need, None) == inv
+    d32 = _desc(in_dtype=ispa.ISPA_F32)
+    assert L.ispa_warmup_fused(ctypes.byref(d32), *args, FAKE, need, None) == ispa.ISPA_ERR_UNSUPPORTED

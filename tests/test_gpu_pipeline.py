@@ -245,3 +245,62 @@ def test_kv_restore_inverts_eviction():
     sentinel = np.full(full, 3.0)
     assert np.array_equal(host(k_back), orc.restore_history(sh, orc.evict_history(sh, data["k"]), sentinel))
     assert np.array_equal(host(v_back), orc.restore_history(sh, orc.evict_history(sh, data["v"]), sentinel))
+
+
+FUSED_LAYOUTS = [
+    # (sink, hist_begin, hist_end, cur_begin, cur_end, kv_frames, tpf)
+    (2, 2, 6, 6, 9, 9, 45),      # history present, ragged 135-row chunk
+    (3, 3, 3, 3, 5, 5, 64),      # no history (sink adjacent to the chunk)
+    (1, 1, 4, 4, 6, 6, 70),
+]
+
+
+@pytest.mark.parametrize("lay", range(len(FUSED_LAYOUTS)))
+def test_warmup_fused_equals_split_plus_stats(lay):
+    """The fused warmup gives bit for bit the O_full, L_full, G and C of the two-call path
+    (split attention, then the statistics of its outputs) and r2 up to the order of its
+    fp64 atomic additions; and G, C, r2 against the oracle from the synthetic inputs."""
+    S, hb, he, cb, ce, kvf, tpf = FUSED_LAYOUTS[lay]
+    sh = si.AttnShape(B=2, H=2, d=128, tpf=tpf, sink_frames=S, hist_begin=hb, hist_end=he, cur_begin=cb,
+                      cur_end=ce, kv_frames=kvf)
+    data = si.iid_qkv(sh, "bf16", ("gpu", "fused", lay))
+    D, Dout, T = sh.D, 192, sh.B * sh.Lq
+    W = si.projection_weight(D, Dout, ("gpu", "fused", lay))
+    q, k, v = (dev(data[n], torch.bfloat16) for n in ("q", "k", "v"))
+    Wd = dev(W)
+    desc = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_F32)
+    f32 = dict(device="cuda", dtype=torch.float32)
+    # two-call path
+    o = {n: torch.full((sh.B, sh.Lq, sh.H, 128), float("nan"), **f32) for n in ("loc", "hist", "full")}
+    l = {n: torch.full((sh.B, sh.Lq, sh.H), float("nan"), **f32) for n in ("loc", "hist", "full")}
+    ws_a = torch.empty(ispa.ispa_attn_split_workspace_bytes(desc), dtype=torch.uint8, device="cuda")
+    ispa.ispa_attn_split(desc, q, k, v, o["loc"], l["loc"], o["hist"], l["hist"], o["full"], l["full"], workspace=ws_a)
+    G1, C1 = torch.zeros((D, D), **f32), torch.zeros((D, Dout), **f32)
+    r1 = torch.zeros(1, device="cuda", dtype=torch.float64)
+    ws_s = torch.empty(ispa.ispa_accum_stats_workspace_bytes(T, D, Dout, ispa.ISPA_PREC_TF32), dtype=torch.uint8,
+                       device="cuda")
+    ispa.ispa_accum_stats(T, D, Dout, o["loc"], o["full"], Wd, G1, C1, r1, ispa.ISPA_PREC_TF32, ws_s)
+    # fused
+    of = torch.full((sh.B, sh.Lq, sh.H, 128), float("nan"), **f32)
+    lf = torch.full((sh.B, sh.Lq, sh.H), float("nan"), **f32)
+    G2, C2 = torch.zeros((D, D), **f32), torch.zeros((D, Dout), **f32)
+    r2 = torch.zeros(1, device="cuda", dtype=torch.float64)
+    ws_f = torch.empty(ispa.ispa_warmup_fused_workspace_bytes(desc, Dout), dtype=torch.uint8, device="cuda")
+    ispa.ispa_warmup_fused(desc, q, k, v, Wd, Dout, of, lf, G2, C2, r2, ws_f)
+    ispa.ispa_check_device_error()
+    torch.cuda.synchronize()
+    assert torch.equal(of, o["full"]) and torch.equal(lf, l["full"])
+    up = torch.triu(torch.ones((D, D), dtype=torch.bool, device="cuda"))
+    assert torch.equal(G2[up], G1[up]) and torch.equal(C2, C1)
+    assert abs(float(r2) - float(r1)) <= 1e-12 * abs(float(r1))
+    # against the oracle (tf32 operands: the statistics' 1e-3 relative Frobenius bar)
+    ref = orc.split_attention(sh, data["q"], data["k"], data["v"])
+    A_loc, A_full = orc.heads_to_rows(ref["O_loc"]), orc.heads_to_rows(ref["O_full"])
+    Gr, Cr, rr = orc.absorption_stats(A_loc, A_full, W)
+    Gg = np.triu(host(G2))
+    assert rel_fro(Gg + np.triu(Gg, 1).T, Gr) <= 1e-3
+    if rr == 0.0:  # no history: A_full = A_loc, so R, C and r2 vanish exactly
+        assert np.all(host(C2) == 0) and float(r2) == 0.0
+    else:
+        assert rel_fro(host(C2), Cr) <= 1e-3
+        assert abs(float(r2) - rr) <= 1e-3 * rr
