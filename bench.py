@@ -19,7 +19,8 @@ the evicted L-layer 57 MB); between two uses of one layer's K/V the other
 passes stream 400 MB or more through the 126 MB L2, so no flush is needed.  The step runs on a stream of its own,
 captured once into a CUDA graph and replayed (warm-up and timed steps); the
 solve's component time replays a graph of the solve alone.  The end-to-end
-number calls the public API eagerly, with the host copies in the timed region.
+number calls the public API eagerly, with every step's host copies in the timed
+region (the next step's inputs copied on a second stream while a step computes).
 Outside the timed steps a component times the L-layer with its projection in
 8 bits (W8A8, e4m3 and int8; ispa_quantize_weight, ispa_attn_local_proj_q8)
 against the bf16 step, and another the fused warmup step (ispa_warmup_fused:
@@ -370,8 +371,9 @@ def run_ours(args, world, rank, local):
     work = step_work(sh)
 
     layers = [Layer(sh, ("bench", name, rank), dev) for name in ("warm", "local", "full")]
-    W_host = torch.from_numpy(si.projection_weight(D, D, ("bench", "W", rank), "bf16"))
+    W_host = torch.from_numpy(si.projection_weight(D, D, ("bench", "W", rank), "bf16")).pin_memory()
     W32 = W_host.to(dev)
+    wcur = {"W32": W32}  # the buffer set the step reads W from (see the end-to-end pipeline)
     W16 = W_host.to(torch.bfloat16).to(dev)
     f32 = dict(device=dev, dtype=torch.float32)
     o = {n: torch.empty((B, Lq, H, 128), **f32) for n in ("loc", "hist", "full")}
@@ -438,7 +440,7 @@ def run_ours(args, world, rank, local):
                              l["hist"], o["full"], l["full"], workspace=ws_attn, stream=stream)
         if timed_components:
             ev_attn[1].record(stream)
-        ispa.ispa_accum_stats(T, D, D, o["loc"], o["full"], W32, G, C, r2, ispa.ISPA_PREC_TF32, ws_stats,
+        ispa.ispa_accum_stats(T, D, D, o["loc"], o["full"], wcur["W32"], G, C, r2, ispa.ISPA_PREC_TF32, ws_stats,
                               stream=stream)
         solve()
         ispa.ispa_select_layers(N_LAYERS, eps_all, K_sel, is_local, idx, stream=stream)
@@ -529,27 +531,59 @@ def run_ours(args, world, rank, local):
     small_host = torch.empty(N_LAYERS, dtype=torch.float64).pin_memory()
     d2h = sum(t.numel() * t.element_size() for t in y_host.values()) + dW_host.numel() * 4 + N_LAYERS * 8
 
-    def e2e_step():
-        for Lr in layers:
-            for n in ("q", "k", "v"):
-                Lr.dev[n].copy_(Lr.host[n], non_blocking=True)
-        W32.copy_(W_host, non_blocking=True)
-        step(False)
-        for n in ("L", "F"):
-            y_host[n].copy_(y[n], non_blocking=True)
-        dW_host.copy_(dW, non_blocking=True)
-        small_host.copy_(eps_all, non_blocking=True)
+    # Every step copies all of its inputs (Q/K/V of the three layers and W)
+    # from pinned host memory and reads its results back.  The copies of step
+    # i + 1 run on a copy stream into a second set of input buffers while step
+    # i computes on the first (double buffering, ordered by events), so the
+    # step costs max(copy, compute) instead of their sum.
+    sets = [([Lr.dev for Lr in layers], W32),
+            ([{n: torch.empty_like(t) for n, t in Lr.dev.items()} for Lr in layers], torch.empty_like(W32))]
+    copy_stream = torch.cuda.Stream(dev)
+    copied = [torch.cuda.Event(), torch.cuda.Event()]
+    freed = [torch.cuda.Event(), torch.cuda.Event()]
 
-    e2e_steps = max(2, min(args.steps, 5))
-    e2e_step()
+    def issue_copy(i):
+        devs, wd = sets[i % 2]
+        with torch.cuda.stream(copy_stream):
+            if i >= 2:
+                copy_stream.wait_event(freed[i % 2])  # step i - 2 is done with this set
+            for Lr, d in zip(layers, devs):
+                for n in ("q", "k", "v"):
+                    d[n].copy_(Lr.host[n], non_blocking=True)
+            wd.copy_(W_host, non_blocking=True)
+            copied[i % 2].record(copy_stream)
+
+    def e2e_run(n_steps, start_event=None):
+        if start_event is not None:
+            copy_stream.wait_event(start_event)
+        issue_copy(0)
+        for i in range(n_steps):
+            if i + 1 < n_steps:
+                issue_copy(i + 1)
+            stream.wait_event(copied[i % 2])
+            devs, wd = sets[i % 2]
+            for Lr, d in zip(layers, devs):
+                Lr.dev = d
+            wcur["W32"] = wd
+            step(False)
+            for n in ("L", "F"):
+                y_host[n].copy_(y[n], non_blocking=True)
+            dW_host.copy_(dW, non_blocking=True)
+            small_host.copy_(eps_all, non_blocking=True)
+            freed[i % 2].record(stream)
+
+    e2e_steps = max(2, min(args.steps, 6))
+    e2e_run(2)
     torch.cuda.synchronize(dev)
     barrier(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    e2e_run(e2e_steps, e0)
     e1.record(stream)
     torch.cuda.synchronize(dev)
+    for Lr, d in zip(layers, sets[0][0]):
+        Lr.dev = d
+    wcur["W32"] = W32
     e2e_ms = reduce_over_ranks(e0.elapsed_time(e1) / e2e_steps, "max", dev)
 
     return dict(ms_step=ms_step, work=work, attn_launch_ms=attn_launch_ms, solve_launch_ms=solve_launch_ms,
