@@ -229,8 +229,10 @@ __device__ __forceinline__ void epilogue_chunk(const Params &P, const SubProblem
   }
 }
 
-// Store epilogue through shared memory, for the plain stores (bf16 or fp32)
-// and the scaled 8-bit one, with N % 16 == 0 and 16-byte aligned rows.  Each
+// Store epilogue through shared memory, for the plain stores (bf16 or fp32),
+// the scaled 8-bit one, the accumulating one (out += acc, only i <= j for an
+// upper-triangle problem) and the tf32-rounding one with its sum of squares,
+// with N % 16 == 0 and 16-byte aligned rows.  Each
 // epilogue warp owns 32 rows of the tile: it moves its accumulator rows out
 // of tensor memory (lane = row), writes them to its own staging area in
 // 16-byte chunks (chunk j of row r at slot j ^ r, so that neither the row-wise
@@ -239,9 +241,12 @@ __device__ __forceinline__ void epilogue_chunk(const Params &P, const SubProblem
 // contiguous bytes per row, instead of every store instruction touching 32
 // rows.  The staging areas reuse the operand stages, idle once the
 // accumulator is complete.
-template <bool BF16_OUT, bool SCALED>
+enum StageMode { STAGE_STORE = 0, STAGE_SCALED = 1, STAGE_ACCUM = 2, STAGE_TF32_SQ = 3 };
+
+template <bool BF16_OUT, int MODE>
 __device__ __forceinline__ void epilogue_staged(const Params &P, const SubProblem &sp, uint32_t tmem_rows, int quarter,
-                                                int lane, int m0, int n0, uint8_t *stage) {
+                                                int lane, int m0, int n0, uint8_t *stage, double &sq) {
+  constexpr bool SCALED = MODE == STAGE_SCALED;
   constexpr int ELEM = BF16_OUT ? 2 : 4;
   constexpr int CPR = BN * ELEM / 16;  // 16-byte chunks per row
   const int N = sp.N;
@@ -264,6 +269,10 @@ __device__ __forceinline__ void epilogue_staged(const Params &P, const SubProble
     for (int j = 0; j < 32; ++j) {
       const float acc = SCALED && P.kind_f8 == 2 ? __int2float_rn((int)r[j]) : __uint_as_float(r[j]);
       x[j] = SCALED ? acc * rs * __shfl_sync(0xffffffffu, cs, j) : acc;
+      if (MODE == STAGE_TF32_SQ) {
+        if (row < P.M && n0 + c * 32 + j < N) sq += (double)acc * acc;
+        x[j] = to_tf32_rn(acc);
+      }
     }
     if (BF16_OUT) {
 #pragma unroll
@@ -285,9 +294,21 @@ __device__ __forceinline__ void epilogue_staged(const Params &P, const SubProble
     const uint8_t *src = stage + rr * (CPR * 16);
     uint8_t *dst = static_cast<uint8_t *>(sp.out) + ((long long)grow * sp.ldo + n0) * ELEM;
 #pragma unroll
-    for (int j = lane; j < CPR; j += 32)
-      if (n0 + j * (16 / ELEM) < N)
-        *reinterpret_cast<uint4 *>(dst + j * 16) = *reinterpret_cast<const uint4 *>(src + ((j ^ rr) * 16));
+    for (int j = lane; j < CPR; j += 32) {
+      const int col = n0 + j * (16 / ELEM);
+      if (col >= N) continue;
+      uint4 v = *reinterpret_cast<const uint4 *>(src + ((j ^ rr) * 16));
+      if (MODE == STAGE_ACCUM) {  // fp32: old + acc, acc taken as 0 left of the diagonal of an upper problem
+        const float4 old = *reinterpret_cast<const float4 *>(dst + j * 16);
+        const float a[4] = {__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z), __uint_as_float(v.w)};
+        const float o4[4] = {old.x, old.y, old.z, old.w};
+        float s4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s4[e] = (sp.upper && col + e < grow) ? o4[e] : o4[e] + a[e];
+        v = make_uint4(__float_as_uint(s4[0]), __float_as_uint(s4[1]), __float_as_uint(s4[2]), __float_as_uint(s4[3]));
+      }
+      *reinterpret_cast<uint4 *>(dst + j * 16) = v;
+    }
   }
 }
 
@@ -434,7 +455,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int quarter = warp & 3;
     const int row = m0 + quarter * 32 + lane;
     double sq = 0.0;
-    const bool staged = (sp.epi == EPI_STORE_BF16 || sp.epi == EPI_STORE_F32 || sp.epi == EPI_SCALED) &&
+    const bool staged = (sp.epi == EPI_STORE_BF16 || sp.epi == EPI_STORE_F32 || sp.epi == EPI_SCALED ||
+                         sp.epi == EPI_ACCUM_F32 || sp.epi == EPI_STORE_TF32_SQ) &&
                         sp.N % 16 == 0 && sp.ldo % 16 == 0 && (reinterpret_cast<uintptr_t>(sp.out) & 15) == 0;
     const uint32_t tmem_rows = tmem + ((uint32_t)(quarter * 32) << 16);
     uint8_t *stage = smem + quarter * (32 * BN * 4);  // 32 KB per warp inside the operand stages
@@ -443,11 +465,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         const bool bf16_out = sp.epi == EPI_STORE_BF16 || (sp.epi == EPI_SCALED && P.out_bf16);
         if (sp.epi == EPI_SCALED) {
-          if (bf16_out) epilogue_staged<true, true>(P, sp, tmem_rows, quarter, lane, m0, n0, stage);
-          else epilogue_staged<false, true>(P, sp, tmem_rows, quarter, lane, m0, n0, stage);
+          if (bf16_out) epilogue_staged<true, STAGE_SCALED>(P, sp, tmem_rows, quarter, lane, m0, n0, stage, sq);
+          else epilogue_staged<false, STAGE_SCALED>(P, sp, tmem_rows, quarter, lane, m0, n0, stage, sq);
+        } else if (sp.epi == EPI_ACCUM_F32) {
+          epilogue_staged<false, STAGE_ACCUM>(P, sp, tmem_rows, quarter, lane, m0, n0, stage, sq);
+        } else if (sp.epi == EPI_STORE_TF32_SQ) {
+          epilogue_staged<false, STAGE_TF32_SQ>(P, sp, tmem_rows, quarter, lane, m0, n0, stage, sq);
         } else {
-          if (bf16_out) epilogue_staged<true, false>(P, sp, tmem_rows, quarter, lane, m0, n0, stage);
-          else epilogue_staged<false, false>(P, sp, tmem_rows, quarter, lane, m0, n0, stage);
+          if (bf16_out) epilogue_staged<true, STAGE_STORE>(P, sp, tmem_rows, quarter, lane, m0, n0, stage, sq);
+          else epilogue_staged<false, STAGE_STORE>(P, sp, tmem_rows, quarter, lane, m0, n0, stage, sq);
         }
       }
     } else if (wait_parity(done, 0, P.err, abort, 3)) {
