@@ -524,6 +524,25 @@ def run_ours(args, world, rank, local):
     warm_fused = {"two_calls_ms": graph_time(torch, stream, dev, two_calls, 5),
                   "fused_ms": graph_time(torch, stream, dev, fused, 5)}
 
+    # ---- the stand-alone LSE merge (the attention fuses it; this is the
+    # separate call on the same outputs) and the statistics alone
+    merged_o = torch.empty_like(o["full"])
+    merged_l = torch.empty_like(l["full"])
+
+    def merge():
+        ispa.ispa_lse_merge(T, H, 128, ispa.ISPA_F32, o["loc"], l["loc"], o["hist"], l["hist"], merged_o, merged_l,
+                            stream=stream)
+
+    def stats_only():
+        ispa.ispa_accum_stats(T, D, D, o["loc"], o["full"], W32, G, C, r2, ispa.ISPA_PREC_TF32, ws_stats,
+                              stream=stream)
+
+    merge_ms = graph_time(torch, stream, dev, merge, 20)
+    merge_bytes = T * H * (3 * 128 * 4 + 3 * 4)  # two O and L read, one written (fp32)
+    stats_ms = graph_time(torch, stream, dev, stats_only, 5)
+    extra = {"merge_ms": merge_ms, "merge_gb_s": merge_bytes / (merge_ms * 1e-3) / 1e9,
+             "stats_ms": stats_ms, "stats_tflops": work["stats"] / (stats_ms * 1e-3) / 1e12}
+
     # ---- end to end through the C ABI with host buffers
     h2d = sum(t.numel() * t.element_size() for Lr in layers for t in Lr.host.values()) + W_host.numel() * 4
     y_host = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in y.items()}
@@ -587,7 +606,7 @@ def run_ours(args, world, rank, local):
     e2e_ms = reduce_over_ranks(e0.elapsed_time(e1) / e2e_steps, "max", dev)
 
     return dict(ms_step=ms_step, work=work, attn_launch_ms=attn_launch_ms, solve_launch_ms=solve_launch_ms,
-                kv_evict=kv_evict, w8a8=w8a8, warm_fused=warm_fused,
+                kv_evict=kv_evict, w8a8=w8a8, warm_fused=warm_fused, extra=extra,
                 launches=launches, clocks=clocks.summary(), e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, world=world, rank=rank)
 
 
@@ -833,7 +852,7 @@ def main(argv=None):
                 "query_tok_per_s": world * WORKLOAD.shape.B * WORKLOAD.shape.Lq / (r["attn_launch_ms"] * 1e-3),
                 "attn_split_ms": r["attn_launch_ms"], "solve_ms_per_layer": r["solve_launch_ms"],
                 "step_gflop": work["total"] / 1e9, "kv_eviction": r["kv_evict"], "w8a8_l_layer": r["w8a8"],
-                "warmup_fused": r["warm_fused"]},
+                "warmup_fused": r["warm_fused"], **r["extra"]},
             "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (two-group attention + fused merge)",
                          "achieved": achieved, "peak": peak, "peak_source": peak_src, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": measured_traffic()},
