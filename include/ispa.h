@@ -406,7 +406,8 @@ ispa_status ispa_stats_reset(int D, int Dout, float *G, float *C, double *r2, is
  *   ispa_absorb_weight) -> qT [N, K] (bytes, the transpose, K contiguous) and
  *   sw [N] fp32.  Once per layer, at the switch.
  * ispa_gemm_q8: y [M, N] in y_dtype from q, sa, qT, sw of the same format.
- * Sizes: M, N >= 0 with N % 16 == 0 for the product; K >= 16, K % 16 == 0.
+ * Sizes: M, N >= 0 with N % 16 == 0 for the product; K >= 16, K % 16 == 0;
+ * for int8 products K <= 131072 (the exact int32 sum stays below 2^31).
  * Device pointers, 16-byte aligned, no overlap between inputs and outputs.
  * Asynchronous on stream; ISPA_ERR_INVALID_ARG for bad sizes, format or pointers.
  */

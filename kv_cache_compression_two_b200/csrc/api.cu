@@ -456,6 +456,9 @@ bool q8_ok(ispa_q8_format f) { return f == ISPA_Q8_E4M3 || f == ISPA_Q8_INT8; }
 
 bool q8_k_ok(int K) { return K >= 16 && K % 16 == 0; }
 
+// int8 products accumulate exactly in int32: |sum| <= K * 127^2 must stay below 2^31
+constexpr int kQ8Int8MaxK = 131072;
+
 // [a, a + na) and [b, b + nb) (bytes) overlap
 bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
   const char *x = static_cast<const char *>(a), *y = static_cast<const char *>(b);
@@ -506,6 +509,7 @@ ispa_status ispa_gemm_q8(int M, int N, int K, const void *q, const float *sa, co
   if (M < 0 || N < 0 || N % 16 != 0 || !q8_k_ok(K))
     return fail(ISPA_ERR_INVALID_ARG, "need M >= 0, N a multiple of 16 and K a positive multiple of 16");
   if (!q8_ok(fmt)) return fail(ISPA_ERR_INVALID_ARG, "bad 8-bit format");
+  if (fmt == ISPA_Q8_INT8 && K > kQ8Int8MaxK) return fail(ISPA_ERR_INVALID_ARG, "int8 products need K <= 131072");
   if (!dtype_ok(y_dtype)) return fail(ISPA_ERR_INVALID_ARG, "bad y dtype");
   if (M == 0 || N == 0) return ISPA_OK;
   if (!ptr_ok(q) || !ptr_ok(sa) || !ptr_ok(qT) || !ptr_ok(sw) || !ptr_ok(y))
@@ -536,6 +540,8 @@ ispa_status ispa_attn_local_proj_q8(const ispa_attn_desc *desc, const void *q, c
   if (desc->in_dtype != ISPA_BF16 || desc->head_dim != 128)
     return fail(ISPA_ERR_UNSUPPORTED, "post-switch projection is compiled for bf16 inputs with head_dim 128");
   if (!q8_ok(fmt)) return fail(ISPA_ERR_INVALID_ARG, "bad 8-bit format");
+  if (fmt == ISPA_Q8_INT8 && desc->H * desc->head_dim > kQ8Int8MaxK)
+    return fail(ISPA_ERR_INVALID_ARG, "int8 products need D <= 131072");
   if (Dout < 16 || Dout % 16 != 0) return fail(ISPA_ERR_INVALID_ARG, "Dout must be a positive multiple of 16");
   if (!dtype_ok(y_dtype)) return fail(ISPA_ERR_INVALID_ARG, "bad y dtype");
   if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(qT) || !ptr_ok(sw) || !ptr_ok(y))

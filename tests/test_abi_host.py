@@ -206,6 +206,7 @@ def test_w8a8_validation():
     assert L.ispa_gemm_q8(4, 32, 32, a, b, c, c + 4096, I8, c + 8192, 9, None) == inv
     assert L.ispa_gemm_q8(4, 32, 32, a, b, c, c + 4096, I8, a, ispa.ISPA_F32, None) == inv
     assert L.ispa_gemm_q8(0, 32, 32, None, None, None, None, I8, None, ispa.ISPA_F32, None) == ispa.ISPA_OK
+    assert L.ispa_gemm_q8(4, 32, 131088, a, b, c, c + 4096, I8, c + 8192, ispa.ISPA_F32, None) == inv  # int32 range
     assert L.ispa_gemm_bf16(4, 24, 32, a, b, c, ispa.ISPA_BF16, None) == inv
     assert L.ispa_gemm_bf16(4, 32, 24, a, b, c, ispa.ISPA_BF16, None) == inv
     assert L.ispa_gemm_bf16(4, 32, 32, a, b, a + 32, ispa.ISPA_BF16, None) == inv   # y overlaps A
