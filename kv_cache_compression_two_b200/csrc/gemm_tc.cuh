@@ -14,9 +14,15 @@
 //
 // Operand staging.  An A tile is 16 KB and a B tile 32 KB: 128 (A) or 256 (B)
 // rows of M or N by one 128-byte swizzle span of K for K-major operands, or BK
-// rows of K by 128 / 256 M or N elements (several 128-byte boxes) for MN-major
-// operands.  Per stage the MMA warp issues 4 instructions of K = 8 (tf32) or
-// K = 16 (bf16).
+// rows of K by 128 / 256 M or N elements (128-byte column blocks) for MN-major
+// operands.  Per stage the MMA warp issues 4 instructions of K = 8 (tf32),
+// K = 16 (bf16) or K = 32 (e4m3 / int8, K-major only).  The copy engine's time
+// is mostly per box, so a stage arrives in as few boxes as the layout allows:
+// the K-major B tile as one 256-row box, an MN-major operand through a 3D
+// view whose third dimension is its column blocks (map_mn_blocked).
+//
+// Store epilogues go through shared memory (the operand stages are idle once
+// the accumulator is complete) so that each row is written by a whole warp.
 //
 // Up to two sub-problems that share A (same M, K) but have different B and
 // outputs run in one launch: blockIdx.x enumerates the tiles of problem 0,
