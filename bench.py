@@ -853,7 +853,8 @@ def main(argv=None):
                 "attn_split_ms": r["attn_launch_ms"], "solve_ms_per_layer": r["solve_launch_ms"],
                 "step_gflop": work["total"] / 1e9, "kv_eviction": r["kv_evict"], "w8a8_l_layer": r["w8a8"],
                 "warmup_fused": r["warm_fused"], **r["extra"]},
-            "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (two-group attention + fused merge)",
+            "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (two-group attention + fused merge), timed as its "
+                                                   "call: the fp16 V copy (v_prep_kernel, v_fix_kernel) included",
                          "achieved": achieved, "peak": peak, "peak_source": peak_src, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": measured_traffic()},
             "gpu_launches": r["launches"],
