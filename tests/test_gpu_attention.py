@@ -268,3 +268,41 @@ def test_kv_eviction_releases_the_history_bytes():
     assert before == 2 * sh.B * sh.kv_frames * sh.tpf * row_bytes
     assert before - after == 2 * freed_per_tensor
     assert torch.all(k_ev == 1) and torch.all(v_ev == 1)
+
+
+def test_post_switch_full_size_1p3b_sampled_rows():
+    """The post-switch calls as the bench times them, on the 1.3B-shaped layer at full size: the
+    L-layer on its evicted K/V (sink + current, 9360 keys) projected with W + dW, the F-layer over
+    all 32760 keys projected with W; bf16 output, sampled rows against the oracle (the output
+    tolerance of the bf16 projection, 2e-2 of RMS plus the bf16 output rounding)."""
+    import dataclasses
+    sh = si.SHAPE_1P3B
+    D = sh.D
+    data = si.iid_qkv(sh, "bf16", ("gpu", "post1p3b"))
+    W = si.projection_weight(D, D, ("gpu", "post1p3b"), "bf16")
+    dW = (1e-3 * si.rng("gpu", "post1p3b", "dW").standard_normal((D, D))).astype(np.float32)
+    q = dev(data["q"], torch.bfloat16)
+    k_full, v_full = dev(data["k"], torch.bfloat16), dev(data["v"], torch.bfloat16)
+    rows = np.r_[0:2, 1559:1562, 3000, 4600:4680:9, 4679]
+    for layer in ("L", "F"):
+        if layer == "L":
+            desc_full = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_BF16)
+            desc = ispa.ispa_kv_evicted_desc(desc_full)
+            shape_ev = (sh.B, desc.kv_frames * sh.tpf, sh.H, sh.d)
+            k, v = nan_like(shape_ev, torch.bfloat16), nan_like(shape_ev, torch.bfloat16)
+            ispa.ispa_kv_evict_history(desc_full, k_full, v_full, k, v)
+            Wp = si.round_to_bf16(W + dW)   # the absorbed weight as the layer holds it
+            ref_sh = sh                     # local attention of the original layout
+        else:
+            ref_sh = dataclasses.replace(sh, sink_frames=sh.cur_begin, hist_begin=0, hist_end=0)
+            desc = ispa.attn_desc(ref_sh, ispa.ISPA_BF16, ispa.ISPA_BF16)
+            k, v, Wp = k_full, v_full, W
+        ws = torch.empty(ispa.ispa_attn_local_proj_workspace_bytes(desc), dtype=torch.uint8, device="cuda")
+        y = nan_like((sh.B, sh.Lq, D), torch.bfloat16)
+        ispa.ispa_attn_local_proj(desc, q, k, v, dev(Wp, torch.bfloat16), D, y, ispa.ISPA_BF16, ws)
+        ispa.ispa_check_device_error()
+        torch.cuda.synchronize()
+        got = host(y)
+        assert not np.isnan(got).any(), layer
+        ref = orc.local_projection(ref_sh, data["q"], data["k"], data["v"], Wp, None, rows=rows)
+        assert_bf16_out(got[:, rows], ref, tol=2e-2)

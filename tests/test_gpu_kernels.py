@@ -411,6 +411,20 @@ def test_gemm_bf16_matches_oracle(y_dt):
     assert np.all(np.abs(got - ref) <= tol + 1e-38)
 
 
+def test_gemm_bf16_full_size_layer():
+    """The bf16 projection of the 1.3B-shaped post-switch layer, 4680 x 1536 x 1536, every output
+    against the exact product (96 MMA steps of K = 16, each truncating at most 2^-23 of the sum)."""
+    M, N, K = 4680, 1536, 1536
+    A = si.activation_rows(M, K, ("gpu", "gbf16full"))
+    W = si.projection_weight(K, N, ("gpu", "gbf16full"), "bf16")
+    y = nan_like((M, N), torch.float32)
+    ispa.ispa_gemm_bf16(M, N, K, dev(A, torch.bfloat16), dev(W, torch.bfloat16), y, ispa.ISPA_F32)
+    torch.cuda.synchronize()
+    ref = A.astype(np.float64) @ W.astype(np.float64)
+    tol = 96 * 2.0 ** -23 * (np.abs(A).astype(np.float64) @ np.abs(W).astype(np.float64))
+    assert np.all(np.abs(host(y) - ref) <= tol + 1e-38)
+
+
 @pytest.mark.parametrize("fmt,ofmt", Q8_FORMATS)
 def test_gemm_q8_full_size_layer(fmt, ofmt):
     """The projection of the 1.3B-shaped post-switch layer: 4680 rows (B = 1, 3 frames of 1560
