@@ -2,8 +2,8 @@
 
 Argument marshalling only: every step of the path runs in the CUDA kernels of
 ``libispa.so`` (built in-tree by :mod:`kv_cache_compression_two_b200.build`).
-Importing this package fails loudly when the library is missing; there is no
-CPU or PyTorch fallback.
+The first call into the library raises ImportError when it has not been
+built; there is no CPU or PyTorch fallback.
 
 Tensor arguments may be ``torch.Tensor`` objects (their ``data_ptr()`` is
 passed; the binding checks device, dtype and contiguity) or raw integer device
