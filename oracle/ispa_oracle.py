@@ -15,7 +15,9 @@ Autoregressive Video Generation via Instance-Specific Parametric Absorption"):
 * [ZH-notes]   papernotes.org note, the Chinese version of the same sections.
 * [DE-summary] gist.science/de, "Technisches Resümee", section 2 "Methodik",
                 items "Dual-Stream Warmup", "Layer Absorb", "Speichereffiziente
-                Inferenz" and "Dynamische Layerauswahl".
+                Inferenz" and "Dynamische Layerauswahl"; section 4, item
+                "Beschleunigung" (the W8A8 combination, with the English
+                note's "Key Findings").
 
 Readings taken where the pages are silent or garbled (each one is also
 listed in the design notes of the repository):
@@ -29,7 +31,10 @@ listed in the design notes of the repository):
 * W is applied to row vectors, y = a W, W of shape [D_in, D_out];
 * the ridge penalty is squared Frobenius (the DE summary writes ||.||_2^2);
 * epsilon is taken over all warmup rows, without the lambda term;
-* K = floor(x N); ties in epsilon go to the lower layer index.
+* K = floor(x N); ties in epsilon go to the lower layer index;
+* W8A8: symmetric per-row (activation) and per-column (weight) scales
+  s = amax / QMAX in fp32, codes Q(x * QMAX / amax) in fp8 e4m3 (nearest
+  even, saturating) or int8 (half to even, clamped to +-127).
 
 Parity pins for every function live in ``tests/test_oracle_pins.py``.
 """
