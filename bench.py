@@ -780,6 +780,49 @@ def run_proj_only(args):
     return 0
 
 
+def run_parts_only(args):
+    """The LSE merge, the statistics and one ridge solve alone at the 1.3B layer's
+    sizes, each once after a warm call, for profiling (events around each)."""
+    import torch
+
+    import kv_cache_compression_two_b200 as ispa
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    sh = WORKLOAD.shape
+    T, H, D = sh.B * sh.Lq, sh.H, sh.D
+    g = torch.Generator(device="cpu").manual_seed(5)
+    oa, ob = torch.randn((T, H, 128), generator=g).to(dev), torch.randn((T, H, 128), generator=g).to(dev)
+    la, lb = torch.randn((T, H), generator=g).to(dev), torch.randn((T, H), generator=g).to(dev)
+    oo, lo = torch.empty_like(oa), torch.empty_like(la)
+    a_loc = torch.randn((T, D), generator=g).to(dev)
+    a_full = a_loc + 0.1 * torch.randn((T, D), generator=g).to(dev)
+    W = torch.from_numpy(si.projection_weight(D, D, ("bench", "parts"))).to(dev)
+    G, C = torch.zeros((D, D), device=dev), torch.zeros((D, D), device=dev)
+    r2 = torch.zeros(1, device=dev, dtype=torch.float64)
+    ws = torch.empty(ispa.ispa_accum_stats_workspace_bytes(T, D, D), device=dev, dtype=torch.uint8)
+    dW = torch.empty((D, D), device=dev)
+    eps = torch.empty(1, device=dev, dtype=torch.float64)
+    rws = torch.empty(ispa.ispa_ridge_workspace_bytes(D, D), device=dev, dtype=torch.uint8)
+    parts = {
+        "merge": lambda: ispa.ispa_lse_merge(T, H, 128, ispa.ISPA_F32, oa, la, ob, lb, oo, lo),
+        "stats": lambda: ispa.ispa_accum_stats(T, D, D, a_loc, a_full, W, G, C, r2, ispa.ISPA_PREC_TF32, ws),
+        "solve": lambda: ispa.ispa_ridge_solve(D, D, G, C, r2, LAMBDA_REL, True, 0, dW, eps, rws),
+    }
+    out = {}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for name, fn in parts.items():
+        fn()
+        torch.cuda.synchronize()
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        out[name + "_ms"] = e0.elapsed_time(e1)
+    ispa.ispa_check_device_error()
+    print(json.dumps({"kernel": "parts", **out}), flush=True)
+    return 0
+
+
 def run_attn_only(args):
     """The warmup split attention (fused merge) alone on the 1.3B-shaped layer, for profiling."""
     import torch
@@ -819,12 +862,15 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-rows", type=int, default=32, help="query rows of the oracle sample (0: skip it)")
-    ap.add_argument("--only", choices=["step", "attn", "proj"], default="step",
+    ap.add_argument("--only", choices=["step", "attn", "proj", "parts"], default="step",
                     help="attn: only the split-attention launches; proj: only the post-switch projection "
-                         "(bf16, e4m3, int8 products); both for profiling, printing their timing")
+                         "(bf16, e4m3, int8 products); parts: the merge, the statistics and one solve; "
+                         "all for profiling, printing their timing")
     args = ap.parse_args(argv)
     if args.only == "proj":
         return run_proj_only(args)
+    if args.only == "parts":
+        return run_parts_only(args)
     if args.only == "attn":
         return run_attn_only(args)
 
