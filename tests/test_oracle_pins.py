@@ -640,3 +640,79 @@ def test_local_projection_q8_reduces_to_the_unquantised_step(fmt):
     dW = np.abs(W - qw * sw[None, :].astype(np.float64))
     bound = np.abs(A0) @ dW + dA @ np.abs(W) + dA @ dW
     assert np.all(np.abs(y8.reshape(-1, 8) - y.reshape(-1, 8)) <= bound * (1 + 1e-5) + 1e-12)
+
+
+# ---------------------------------------------------------------------------
+# mutation tests of the W8A8 oracle: a planted mistake fails a pin
+# ---------------------------------------------------------------------------
+def check_e4m3_round(fn) -> bool:
+    """The midpoint and saturation pins of test_e4m3_round_is_the_nearest_grid_value_ties_to_even."""
+    grid = np.array(e4m3_grid_by_enumeration())
+    full = np.concatenate([[0.0], grid])
+    mids = (full[:-1] + full[1:]) / 2
+    even = np.where(np.arange(126) % 2 == 0, full[:-1], full[1:])
+    return (np.array_equal(fn(mids), even) and np.array_equal(fn(grid), grid)
+            and fn(np.array([1e6]))[0] == 448.0)
+
+
+def check_quantize_rows(fn, fmt) -> bool:
+    """Per-row scale and the largest entry of each row on +-QMAX."""
+    x = si.activation_rows(37, 96, ("pin", "q8", fmt))
+    q, s = fn(x, fmt)
+    amax = np.abs(x).max(axis=1)
+    nz = amax > 0
+    arg = np.abs(x).argmax(axis=1)
+    return (np.array_equal(s, (amax / np.float32(orc.Q8_MAX[fmt])).astype(np.float32))
+            and bool(np.all(np.abs(q[np.arange(len(x)), arg])[nz] == orc.Q8_MAX[fmt])))
+
+
+def check_gemm_q8(fn) -> bool:
+    x = si.activation_rows(5, 48, ("pin", "gemm", 0))
+    W = si.projection_weight(48, 7, ("pin", "gemm", 0), "bf16")
+    qa, sa = orc.quantize_rows(x, orc.Q8_E4M3)
+    qw, sw = orc.quantize_cols(W, orc.Q8_E4M3)
+    return np.allclose(np.asarray(fn(qa, sa, qw, sw, orc.Q8_E4M3), np.float64), brute_gemm_q8(qa, sa, qw, sw),
+                       rtol=1e-12, atol=0)
+
+
+def test_w8a8_pins_accept_the_oracle():
+    assert check_e4m3_round(orc.e4m3_round)
+    assert check_quantize_rows(orc.quantize_rows, orc.Q8_E4M3) and check_quantize_rows(orc.quantize_rows, orc.Q8_INT8)
+    assert check_gemm_q8(orc.gemm_q8)
+
+
+def test_mutant_e4m3_ties_away_from_zero_is_caught():
+    def ties_away(x):
+        x = np.asarray(x, np.float64)
+        a = np.abs(x)
+        _, ex = np.frexp(a)
+        quantum = np.ldexp(1.0, np.maximum(ex - 1, -6) - 3)
+        q = np.minimum(np.floor(a / quantum + 0.5) * quantum, 448.0)
+        return np.copysign(q, x)
+    assert not check_e4m3_round(ties_away)
+
+
+def test_mutant_e4m3_without_saturation_is_caught():
+    def no_sat(x):
+        x = np.asarray(x, np.float64)
+        a = np.abs(x)
+        _, ex = np.frexp(a)
+        quantum = np.ldexp(1.0, np.maximum(ex - 1, -6) - 3)
+        return np.copysign(np.rint(a / quantum) * quantum, x)
+    assert not check_e4m3_round(no_sat)
+
+
+def test_mutant_per_tensor_scale_is_caught():
+    def per_tensor(x, fmt):
+        x32 = np.asarray(x, np.float32)
+        amax = np.float32(np.abs(x32).max())
+        qmax = np.float32(orc.Q8_MAX[fmt])
+        s = np.full(x32.shape[0], amax / qmax, np.float32)
+        return orc.q8_round((x32 * (qmax / amax)).astype(np.float64), fmt), s
+    assert not check_quantize_rows(per_tensor, orc.Q8_INT8)
+
+
+def test_mutant_gemm_q8_dropped_column_scale_is_caught():
+    def no_sw(qa, sa, qw, sw, fmt):
+        return orc.gemm_q8(qa, sa, qw, np.ones_like(sw), fmt)
+    assert not check_gemm_q8(no_sw)
