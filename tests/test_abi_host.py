@@ -241,3 +241,36 @@ def test_warmup_fused_validation():
     assert L.ispa_warmup_fused(ctypes.byref(d), *bad, FAKE, need, None) == inv
     d32 = _desc(in_dtype=ispa.ISPA_F32)
     assert L.ispa_warmup_fused(ctypes.byref(d32), *args, FAKE, need, None) == ispa.ISPA_ERR_UNSUPPORTED
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/ispa.h compiles as C99 and a C program links against libispa.so and calls it:
+    the boundary needs neither C++ nor torch (no GPU call: version, a rejected argument and the
+    last-error text)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "probe.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "ispa.h"
+int main(void) {
+  const char *v = ispa_version();
+  if (!v || !*v) return 2;
+  ispa_status st = ispa_stats_reset(0, 4, NULL, NULL, NULL, NULL);
+  if (st != ISPA_ERR_INVALID_ARG) return 3;
+  if (strlen(ispa_last_error()) == 0) return 4;
+  printf("%s\n", v);
+  return 0;
+}
+''')
+    lib_dir = os.path.join(ROOT, "kv_cache_compression_two_b200")
+    exe = tmp_path / "probe"
+    subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o",
+                    str(exe), "-L", lib_dir, "-lispa", "-Wl,-rpath," + lib_dir], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, (out.returncode, out.stderr)
+    assert out.stdout.strip() == ispa.lib().ispa_version().decode()
