@@ -716,3 +716,47 @@ def test_mutant_gemm_q8_dropped_column_scale_is_caught():
     def no_sw(qa, sa, qw, sw, fmt):
         return orc.gemm_q8(qa, sa, qw, np.ones_like(sw), fmt)
     assert not check_gemm_q8(no_sw)
+
+
+# ---------------------------------------------------------------------------
+# properties of the 8-bit and bf16 roundings over random inputs (hypothesis)
+# ---------------------------------------------------------------------------
+from hypothesis import given, settings  # noqa: E402
+from hypothesis import strategies as st  # noqa: E402
+
+_finite = st.floats(min_value=-1e4, max_value=1e4, allow_nan=False, allow_infinity=False, width=32)
+
+
+@settings(max_examples=200, deadline=None)
+@given(st.lists(_finite, min_size=2, max_size=64))
+def test_e4m3_round_is_monotone_idempotent_and_odd(xs):
+    x = np.sort(np.asarray(xs, np.float64))
+    q = orc.e4m3_round(x)
+    assert np.all(np.diff(q) >= 0)                      # monotone
+    assert np.array_equal(orc.e4m3_round(q), q)         # idempotent
+    assert np.array_equal(orc.e4m3_round(-x), -q)       # odd
+    assert np.all(np.abs(q) <= 448.0)
+
+
+@settings(max_examples=200, deadline=None)
+@given(st.lists(_finite, min_size=2, max_size=64))
+def test_bf16_round_is_monotone_and_idempotent(xs):
+    x = np.sort(np.asarray(xs, np.float32))
+    q = orc.bf16_round(x)
+    assert np.all(np.diff(q) >= 0)
+    assert np.array_equal(orc.bf16_round(q), q)
+    # half a unit in the last place: 2^-8 relative, or half the subnormal spacing 2^-133
+    assert np.all(np.abs(q - x) <= 2.0 ** -8 * np.abs(x) + 2.0 ** -134)
+
+
+@settings(max_examples=60, deadline=None)
+@given(st.integers(min_value=0, max_value=2 ** 31 - 1), st.integers(min_value=-20, max_value=20),
+       st.sampled_from([orc.Q8_E4M3, orc.Q8_INT8]))
+def test_quantize_rows_commutes_with_power_of_two_scaling(seed, k, fmt):
+    """x -> x 2^k leaves every code unchanged and scales every row's scale by 2^k exactly
+    (amax, QMAX / amax and x * inv all scale exactly while no value leaves fp32's normal range)."""
+    x = si.round_to_bf16(np.random.default_rng(seed).standard_normal((6, 40)).astype(np.float32))
+    q1, s1 = orc.quantize_rows(x, fmt)
+    q2, s2 = orc.quantize_rows((x * np.float32(2.0 ** k)).astype(np.float32), fmt)
+    assert np.array_equal(q1, q2)
+    assert np.array_equal(s2, (s1 * np.float32(2.0 ** k)).astype(np.float32))
