@@ -49,3 +49,19 @@ def test_kv_retained_fraction_of_the_model():
     frac = ((30 - 15) * sh.kv_frames + 15 * kept) / (30 * sh.kv_frames)
     assert kept == 6 and abs(frac - 0.6428571) < 1e-6
     assert abs(orc.kv_retained_fraction(0.5, (sh.kv_frames - kept) / sh.kv_frames) - frac) < 1e-12
+
+
+def test_clock_sampler_summary_maps_reasons():
+    c = bench.ClockSampler(0)
+    # NVML samples: (sm MHz, max MHz, clock-event reason bits); 0x4 = sw power cap, 0x8 = hw slowdown
+    c.samples = [(1965.0, 1965.0, 0), (1900.0, 1965.0, 0x4), (1800.0, 1965.0, 0x4 | 0x8)]
+    s = c.summary()
+    assert s["sm_mhz"] == 1900.0 and s["sm_max_mhz"] == 1965.0 and s["samples"] == 3
+    assert s["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    # nvidia-smi lines (the fallback): fields as queried, "Active" / "Not Active"
+    c2 = bench.ClockSampler(0)
+    c2.lines = ["1965, 1965, 800.0, Not Active, Not Active, Not Active, Active",
+                "1950, 1965, 810.0, Not Active, Active, Not Active, Not Active"]
+    s2 = c2.summary()
+    assert s2["samples"] == 2 and s2["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    assert bench.ClockSampler(0).summary()["sm_mhz"] is None
