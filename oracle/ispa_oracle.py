@@ -240,12 +240,15 @@ def num_selected(x: float, N: int) -> int:
 def select_layers(eps: Sequence[float], K: int):
     """Sort layers by increasing epsilon and take the K lowest as L-layers.
 
-    Ties go to the lower layer index (stable sort).  Returns (is_local uint8 [N],
-    idx int32 [K] ascending by layer index).
+    Ties go to the lower layer index (stable sort).  A NaN epsilon (a layer
+    whose solve failed) orders after every number, NaNs among themselves by
+    layer index.  Returns (is_local uint8 [N], idx int32 [K] ascending by layer
+    index).
     """
     eps = np.asarray(eps, np.float64)
     N = eps.shape[0]
-    order = sorted(range(N), key=lambda i: (eps[i], i))
+    nan = np.isnan(eps)
+    order = sorted(range(N), key=lambda i: (bool(nan[i]), 0.0 if nan[i] else float(eps[i]), i))
     chosen = sorted(order[:K])
     is_local = np.zeros(N, np.uint8)
     is_local[chosen] = 1

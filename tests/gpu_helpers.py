@@ -48,5 +48,6 @@ def assert_bf16_out(got, ref, tol=1e-2):
 def assert_lse(got, ref, tol):
     both_inf = np.isneginf(got) & np.isneginf(ref)
     assert np.array_equal(np.isneginf(got), np.isneginf(ref))
-    d = np.abs(np.where(both_inf, 0.0, got - ref))
+    # mask before subtracting: -inf - (-inf) is NaN
+    d = np.abs(np.where(both_inf, 0.0, got) - np.where(both_inf, 0.0, ref))
     assert float(d.max()) <= tol, float(d.max())

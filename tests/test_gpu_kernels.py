@@ -67,13 +67,22 @@ def test_select_layers_matches_oracle_with_ties():
 
 
 def test_select_layers_nan_sorts_last():
-    eps = np.array([0.5, np.nan, 0.1, np.nan, 0.3])
-    mask = torch.zeros(5, dtype=torch.uint8, device="cuda")
-    idx = torch.zeros(4, dtype=torch.int32, device="cuda")
-    ispa.ispa_select_layers(5, dev(eps, torch.float64), 4, mask, idx)
-    torch.cuda.synchronize()
-    assert mask.cpu().tolist() == [1, 1, 1, 0, 1]
-    assert idx.cpu().tolist() == [0, 1, 2, 4]
+    g = np.random.default_rng(17)
+    cases = [np.array([0.5, np.nan, 0.1, np.nan, 0.3])]
+    for N in (3, 30, 257):
+        e = np.round(g.random(N) * 8) / 8
+        e[g.random(N) < 0.25] = np.nan
+        cases.append(e)
+    for eps in cases:
+        N = eps.shape[0]
+        for K in sorted({0, 1, N // 2, N - 1, N}):
+            mask = torch.full((N,), 7, dtype=torch.uint8, device="cuda")
+            idx = torch.full((max(K, 1),), -1, dtype=torch.int32, device="cuda")
+            ispa.ispa_select_layers(N, dev(eps, torch.float64), K, mask, idx)
+            torch.cuda.synchronize()
+            rm, ri = orc.select_layers(eps, K)
+            assert np.array_equal(mask.cpu().numpy(), rm)
+            assert np.array_equal(idx.cpu().numpy()[:K], ri)
 
 
 # ---------------------------------------------------------------- statistics

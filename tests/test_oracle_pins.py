@@ -324,6 +324,24 @@ def test_selection_bruteforce():
     assert check_selection_bruteforce(orc.select_layers)
 
 
+def test_selection_nan_orders_last():
+    """A NaN epsilon (a failed solve) orders after every number, NaNs by layer index:
+    pinned to NumPy's stable argsort, which sorts NaN to the end in index order."""
+    g = np.random.default_rng(41)
+    for N in (1, 2, 5, 9, 30):
+        for _ in range(20):
+            eps = np.round(g.random(N) * 4) / 4
+            eps[g.random(N) < 0.3] = np.nan
+            order = np.argsort(eps, kind="stable")
+            for K in range(N + 1):
+                mask, idx = orc.select_layers(eps, K)
+                assert idx.tolist() == sorted(order[:K].tolist())
+                assert int(mask.sum()) == K and all(mask[idx] == 1)
+    # a layer with a NaN epsilon is chosen only once every finite one is
+    mask, idx = orc.select_layers([np.nan, 2.0, np.nan, 1.0], 3)
+    assert idx.tolist() == [0, 1, 3]
+
+
 def test_num_selected():
     assert orc.num_selected(0.5, 30) == 15 and orc.num_selected(0.5, 40) == 20
     assert orc.num_selected(0.25, 30) == 7 and orc.num_selected(0.25, 40) == 10
