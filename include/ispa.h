@@ -264,9 +264,13 @@ ispa_status ispa_ridge_solve(int D, int Dout, const float *G, const float *C, co
  * 4 ISPA_RIDGE_NOALLOC_MAX_D * ISPA_RIDGE_NOALLOC_MAX_DOUT floats, 25.25 MiB),
  * which every GPU that loads the library holds until the process exits; the call
  * itself allocates nothing.  D > ISPA_RIDGE_NOALLOC_MAX_D or Dout >
- * ISPA_RIDGE_NOALLOC_MAX_DOUT returns ISPA_ERR_INVALID_ARG.  The first call on
- * a device looks up the array's device address (cudaGetSymbolAddress); make
- * that first call before any stream capture.  All calls share the one array
+ * ISPA_RIDGE_NOALLOC_MAX_DOUT returns ISPA_ERR_INVALID_ARG, as does any size
+ * whose scratch would not fit the array (checked on the host before the
+ * launch).  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it for the CUDA context that was current;
+ * a call from another context (after cudaDeviceReset, for instance) looks it
+ * up again.  Make the first call on a device, and the first after a reset,
+ * before any stream capture.  All calls share the one array
  * and every call rewrites the parts it reads before reading them, so calls
  * that overlap on the GPU (other streams, other host threads) race: serialise
  * them.

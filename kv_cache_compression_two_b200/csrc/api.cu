@@ -45,17 +45,47 @@ int current_device() {
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
   return dev;
 }
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+CtxGetCurrentFn ctx_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+}  // namespace
+
+void *current_context() {
+  CtxGetCurrentFn fn = ctx_fn();
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
+namespace {
+void *g_err_ctx[kMaxDevices] = {};
 }  // namespace
 
 ispa_status device_err(DevErr *out) {
   const int dev = current_device();
   if (dev < 0 || dev >= kMaxDevices) return fail(ISPA_ERR_CUDA, "no current CUDA device");
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_err_addr[dev]) {
+  // looked up again whenever the thread's current context is not the one the
+  // cached address belongs to (a reset device has a new context and module)
+  void *ctx = current_context();
+  if (!g_err_addr[dev] || !ctx || ctx != g_err_ctx[dev]) {
     void *p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_ispa_device_error);
     if (e != cudaSuccess) return cuda_status(e, "cudaGetSymbolAddress(error word)");
     g_err_addr[dev] = static_cast<int *>(p);
+    g_err_ctx[dev] = current_context();
   }
   out->word = g_err_addr[dev];
   out->limit_ns = g_wait_limit_ns;
@@ -384,7 +414,7 @@ ispa_status ispa_ridge_solve_noalloc(int D, int Dout, const float *G, const floa
   if (!ptr_ok(G) || !ptr_ok(C) || !r2 || !ptr_ok(dW) || !eps)
     return fail(ISPA_ERR_INVALID_ARG, "pointers must be non-NULL, matrices 16-byte aligned");
   void *scratch = nullptr;
-  ispa_status st = ridge_noalloc_scratch(&scratch);
+  ispa_status st = ridge_noalloc_scratch(D, Dout, &scratch);
   if (st != ISPA_OK) return st;
   return launch_ridge(D, Dout, G, C, r2, lambda, lambda_relative, refine_steps, dW, eps, scratch,
                       (cudaStream_t)stream);

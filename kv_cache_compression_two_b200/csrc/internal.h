@@ -19,6 +19,9 @@ ispa_status cuda_status(cudaError_t e, const char *what);
 ispa_status device_err(DevErr *out);
 // SM count of the current device.
 int sm_count();
+// The CUDA context current on the calling thread (NULL if none, or if the
+// driver entry point is unavailable); keys the caches of device addresses.
+void *current_context();
 
 // Encodes a tiled TMA descriptor (driver entry point resolved at run time).
 //   dims[0] is the contiguous dimension; strides_bytes has rank-1 entries.
@@ -78,8 +81,9 @@ size_t ridge_workspace_bytes(int D, int Dout);
 ispa_status launch_ridge(int D, int Dout, const float *G, const float *C, const double *r2, float lambda,
                          int lambda_relative, int refine_steps, float *dW, double *eps, void *ws,
                          cudaStream_t s);
-// Device address of the static scratch array of ispa_ridge_solve_noalloc on the current device.
-ispa_status ridge_noalloc_scratch(void **out);
+// Device address of the static scratch array of ispa_ridge_solve_noalloc on the
+// current device, after checking that the workspace of a D x Dout solve fits it.
+ispa_status ridge_noalloc_scratch(int D, int Dout, void **out);
 
 // bf16 projection GEMM y[M, N] = A[M, K] * B[K, N] (A, B bf16 row-major) on tcgen05
 ispa_status launch_gemm_bf16(int M, int N, int K, const void *A, const void *B, void *Y, ispa_dtype ydt,

@@ -851,19 +851,28 @@ constexpr size_t kNoAllocScratchBytes =
     256;
 static __device__ __align__(256) unsigned char g_ridge_scratch[kNoAllocScratchBytes];
 
-ispa_status ridge_noalloc_scratch(void **out) {
+ispa_status ridge_noalloc_scratch(int D, int Dout, void **out) {
+  const size_t need = carve_bytes(D, Dout, nullptr, nullptr);
+  if (need > sizeof(g_ridge_scratch))
+    return fail(ISPA_ERR_INVALID_ARG, "ispa_ridge_solve_noalloc: a %d x %d solve needs %zu bytes of scratch, the "
+                "static array holds %zu", D, Dout, need, sizeof(g_ridge_scratch));
   static std::mutex mu;
   static void *addr[64] = {};
+  static void *ctx_of[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_status(e, "cudaGetDevice");
   if (dev < 0 || dev >= 64) return fail(ISPA_ERR_CUDA, "device index %d out of range", dev);
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  // the address belongs to the context it was looked up in: after a device
+  // reset (a new context, the module loaded again) it is looked up afresh
+  void *ctx = current_context();
+  if (!addr[dev] || !ctx || ctx != ctx_of[dev]) {
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_ridge_scratch);
     if (e != cudaSuccess) return cuda_status(e, "cudaGetSymbolAddress(ridge scratch)");
     addr[dev] = p;
+    ctx_of[dev] = current_context();
   }
   *out = addr[dev];
   static_assert(ISPA_RIDGE_NOALLOC_MAX_D % NB == 0 && ISPA_RIDGE_NOALLOC_MAX_DOUT % 64 == 0,

@@ -65,3 +65,11 @@ def test_clock_sampler_summary_maps_reasons():
     s2 = c2.summary()
     assert s2["samples"] == 2 and s2["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
     assert bench.ClockSampler(0).summary()["sm_mhz"] is None
+
+
+def test_oracle_sample_work_scales_to_the_step():
+    # a sample of all Lq rows is the whole step; the solve is counted once per sample
+    sh = si.SHAPE_1P3B
+    w = bench.step_work(sh)
+    assert abs(bench.sample_work(sh.B * sh.Lq) - w["total"]) <= 1e-9 * w["total"]
+    assert abs(bench.sample_work(0) - w["solve"]) <= 1e-9 * w["solve"]

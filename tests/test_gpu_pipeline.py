@@ -114,12 +114,14 @@ def test_reduced_model_selection_matches_oracle():
             ref_chunks.append(orc.split_attention(sh, data["q"], data["k"], data["v"]))
         G, C, r2, dW, eps = _absorb_gpu(loc_d, full_d, W, ispa.ISPA_PREC_TF32, 1e-4, 0)
         full = orc.absorb_layer(ref_chunks, W, 1e-4, True)
-        dW_err.append(rel_fro(dW, full["dW"]))  # reported: the tf32 statistics' 1e-3 amplified by cond
+        dW_err.append(rel_fro(dW, full["dW"]))
         eps_gpu.append(eps)
         eps_ref.append(full["eps"])
         assert rel_fro(G[np.triu_indices(sh.D)], full["G"][np.triu_indices(sh.D)]) <= 1e-3
         assert rel_fro(C, full["C"]) <= 1e-3
     print(f"end-to-end dW rel errors {np.round(dW_err, 4)}")
+    # the dW bar holds end to end: bf16 attention, tf32 statistics, fp32 solve
+    assert max(dW_err) <= 1e-2, dW_err
     e = torch.tensor(eps_gpu, dtype=torch.float64, device="cuda")
     mask = torch.zeros(N, dtype=torch.uint8, device="cuda")
     idx = torch.zeros(K, dtype=torch.int32, device="cuda")
