@@ -12,7 +12,9 @@
 //   warp 1      TMEM allocator and MMA issuer.  S_j = Q K_j^T (bf16; Q from
 //               tensor memory, K from shared memory) into S buffer j % 2, and
 //               PV_j: O += P_j V_j (fp16 P from tensor memory, fp16 V from shared
-//               memory).  Order: S_0, S_1, then per tile j: PV_j, S_{j+2}.
+//               memory).  Order: S_0, S_1, then per tile j: PV_j, S_{j+2}, issued
+//               back to back once P_j is published (the copies of V_j and
+//               K_{j+2} are waited for before P_j).
 //   warp 3      idle.
 //   warps 4-7   Q into tensor memory once; then per tile the softmax (one row
 //               per thread, TMEM lane = row), the correction of O when the
@@ -229,6 +231,13 @@ struct TileIter {
   }
 };
 
+// max(a, b, c) in one instruction (sm_100); a NaN operand is ignored as by fmaxf.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -423,19 +432,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_s(j);
       }
       for (int j = 0; ok && j < P.n_tiles; ++j) {
-        ok = wait_parity_spin(&sm.p_full[j & 1], (uint32_t)(j >> 1) & 1, P.err, abort, 23);
+        const int jn = j + 2;  // S runs two tiles ahead, into the buffer PV_j reads
+        // The copies of V_j and K_{j+2} are waited for first: they land long
+        // before the softmax of tile j ends, so these waits overlap the MMAs
+        // still queued, and the only wait between P_j and the 16 MMAs of PV_j
+        // and S_{j+2} is P_j itself.  (No cycle: the stages of V_j and K_{j+2}
+        // were released by PV_{j-3} and S_{j-1}, issued earlier.)
+        ok = wait_parity(&sm.v_full[j % kStagesV], (j / kStagesV) & 1, P.err, abort, 25);
+        if (ok && jn < P.n_tiles)
+          ok = wait_parity(&sm.k_full[jn % kStagesK], (jn / kStagesK) & 1, P.err, abort, 26);
+        if (ok) ok = wait_parity_spin(&sm.p_full[j & 1], (uint32_t)(j >> 1) & 1, P.err, abort, 23);
         if (ok && j == P.n_loc_tiles) ok = wait_parity(&sm.o_free, 0, P.err, abort, 24);
-        if (ok) ok = wait_parity(&sm.v_full[j % kStagesV], (j / kStagesV) & 1, P.err, abort, 25);
         if (!ok) break;
         tc_fence_after();
         issue_pv(j);
-        const int jn = j + 2;  // S runs two tiles ahead, into the buffer PV_j has just read
-        if (jn < P.n_tiles) {
-          ok = wait_parity(&sm.k_full[jn % kStagesK], (jn / kStagesK) & 1, P.err, abort, 26);
-          if (!ok) break;
-          tc_fence_after();
-          issue_s(jn);
-        }
+        if (jn < P.n_tiles) issue_s(jn);
       }
       if (!ok) {
         mma_commit(&sm.drain);
@@ -494,13 +505,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 128; ++c)
           if (c >= n_valid) sr[c >> 5][c & 31] = 0xff800000u;
       }
+      // row maximum with three-input max instructions: 64 for 128 values, in
+      // eight independent chains
       float mx[8];
 #pragma unroll
       for (int t = 0; t < 8; ++t) mx[t] = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(sr[c >> 5][c & 31]));
-      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+      for (int c = 0; c < 128; c += 2)
+        mx[(c >> 1) & 7] = fmax3(mx[(c >> 1) & 7], __uint_as_float(sr[c >> 5][c & 31]),
+                                 __uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]));
+      const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
                        P.scale_log2;
       if (grp_first) {
         m_ref = mt;
