@@ -5,6 +5,7 @@ workload (12 heads x 128, 1560 tokens per latent frame, sink 3 frames, history
 15 frames, chunk 3 frames: 4680 queries over 32760 keys, bf16, fp32
 accumulation):
 
+  every layer    ispa_v16_prepare    the chunk's V frames into the layer's prepared fp16 copy
   warmup layer   ispa_attn_split     local + history groups, fused LSE merge (fp32 out)
                  ispa_accum_stats    R = (A_full - A_loc) W, G += A_loc^T A_loc, C += A_loc^T R
   transition     ispa_ridge_solve    dW = (G + lambda I)^-1 C, epsilon   (lambda = 1e-4 tr(G)/D)
@@ -14,13 +15,16 @@ accumulation):
   post-switch    ispa_attn_local_proj  L-layer: sink + current only (evicted layout), projected with W + dW
                  ispa_attn_local_proj  F-layer: every frame, projected with W
 
-Each attention pass reads its own layer's K/V (warmup and F-layer 200 MB each,
-the evicted L-layer 57 MB); between two uses of one layer's K/V the other
-passes stream 400 MB or more through the 126 MB L2, so no flush is needed.  The step runs on a stream of its own,
-captured once into a CUDA graph and replayed (warm-up and timed steps); the
-solve's component time replays a graph of the solve alone.  The end-to-end
-number calls the public API eagerly, with every step's host copies in the timed
-region (the next step's inputs copied on a second stream while a step computes).
+Each attention pass reads its own layer's K and prepared V (warmup and F-layer
+200 MB each, the evicted L-layer 57 MB); between two uses of one layer's K/V
+the other passes stream 400 MB or more through the 126 MB L2, so no flush is
+needed.  The step runs on a stream of its own, captured once into a CUDA graph
+and replayed (warm-up and timed steps); the solve's component time replays a
+graph of the solve alone.  The end-to-end number calls the public API eagerly,
+with every step's host copies in the timed region: each layer's queries and
+the chunk's own K/V frames (the earlier frames are the layers' device-resident
+KV caches) and W, copied on a second stream for the next step while a step
+computes, and the step's outputs read back.
 Outside the timed steps a component times the L-layer with its projection in
 8 bits (W8A8, e4m3 and int8; ispa_quantize_weight, ispa_attn_local_proj_q8)
 against the bf16 step, and another the fused warmup step (ispa_warmup_fused:
@@ -264,13 +268,22 @@ def measured_traffic():
 # our arm
 # ---------------------------------------------------------------------------
 class Layer:
-    """Device buffers of one attention layer of the workload."""
+    """Device buffers of one attention layer of the workload: Q, the KV cache
+    (bf16 K and V) and, once attached to its descriptor, the prepared fp16 V."""
 
     def __init__(self, sh, key, dev):
         import torch
         data = si.iid_qkv(sh, "bf16", key)
         self.host = {n: torch.from_numpy(data[n]).to(torch.bfloat16).pin_memory() for n in ("q", "k", "v")}
         self.dev = {n: t.to(dev, non_blocking=False) for n, t in self.host.items()}
+        self.desc = None
+
+    def attach(self, ispa, desc, dev):
+        """Prepares the fp16 copy of every frame of V once (the cache's first fill)."""
+        import torch
+        self.desc = desc
+        self.dev["v16"] = torch.empty(ispa.ispa_v16_bytes(desc), device=dev, dtype=torch.uint8)
+        ispa.ispa_v16_prepare(desc, self.dev["v"], 0, desc.kv_frames, self.dev["v16"])
 
 
 def graph_time(torch, stream, dev, fn, reps):
@@ -330,7 +343,7 @@ def w8a8_component(ispa, torch, stream, dev, desc_L, LL, W_new, y_bf16, o_loc, T
     qa = torch.empty((T, D), device=dev, dtype=torch.uint8)
     sa = torch.empty(T, device=dev, dtype=torch.float32)
     y8 = torch.empty((Bq, Lq, D), device=dev, dtype=torch.bfloat16)
-    q, k, v = LL.dev["q"], LL.dev["k"], LL.dev["v"]
+    q, k, v = LL.dev["q"], LL.dev["k"], LL.dev["v16"]   # desc_L is the prepared-V descriptor
 
     def bf16_step():
         ispa.ispa_attn_local_proj(desc_L, q, k, v, W_new, D, y_bf16, ispa.ISPA_BF16, ws_proj, stream=stream)
@@ -355,6 +368,365 @@ def w8a8_component(ispa, torch, stream, dev, desc_L, LL, W_new, y_bf16, o_loc, T
         r["gemm_tflops"] = 2.0 * T * D * D / (r["gemm_ms"] * 1e-3) / 1e12
         out[name] = r
     return out
+
+
+# ---------------------------------------------------------------------------
+# the other workloads: the 14B-shaped layer, the 30-layer 1.3B model, the sweep
+# ---------------------------------------------------------------------------
+L2_BYTES = 126 * 2 ** 20
+
+
+def kv_retained(sh, B: int, N: int, x: float):
+    """KV bytes a model of N layers of shape sh keeps per chunk after ISPA-x
+    (K = floor(x N) L-layers keep the sink and current frames, the others every
+    frame; K and the prepared V, 2 bytes per value each), and that as a fraction."""
+    K = int(math.floor(x * N + 1e-9))
+    n_loc = len(sh.local_rows)
+    per_row = sh.D * 2 * 2
+    full = B * N * sh.Lkv * per_row
+    kept = B * ((N - K) * sh.Lkv + K * n_loc) * per_row
+    return {"layers": N, "l_layers": K, "kv_bytes": kept, "kv_bytes_full": full, "fraction": kept / full}
+
+
+def timed_calls(torch, stream, fn, reps: int, warm: int = 1):
+    """Mean ms per call of fn over reps eager calls, events on the launching stream."""
+    for _ in range(warm):
+        fn()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        fn()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def merge_rate(ispa, torch, stream, dev, rows: int, H: int):
+    """The stand-alone fp32 LSE merge of rows x H heads: GB/s over buffer sets
+    rotating through more than 4x the L2."""
+    set_bytes = rows * H * (3 * 128 * 4 + 3 * 4)
+    nsets = max(1, math.ceil(4 * L2_BYTES / set_bytes))
+    sets = [[torch.randn((rows, H, 128), device=dev), torch.zeros((rows, H), device=dev),
+             torch.randn((rows, H, 128), device=dev), torch.zeros((rows, H), device=dev),
+             torch.empty((rows, H, 128), device=dev), torch.empty((rows, H), device=dev)] for _ in range(nsets)]
+    i = [0]
+
+    def merge():
+        oa, la, ob, lb, oo, lo = sets[i[0] % nsets]
+        i[0] += 1
+        ispa.ispa_lse_merge(rows, H, 128, ispa.ISPA_F32, oa, la, ob, lb, oo, lo, stream=stream)
+
+    ms = graph_time(torch, stream, dev, merge, max(12, 2 * nsets))
+    del sets
+    return {"merge_ms": ms, "merge_gb_s": set_bytes / (ms * 1e-3) / 1e9, "merge_bytes": set_bytes}
+
+
+class KVCache:
+    """One layer's K, V and prepared V on the device, sized for the largest
+    frame layout a component uses; smaller layouts view a prefix of it."""
+
+    def __init__(self, ispa, torch, dev, sh_max, gen):
+        self.k = si.device_normal_bf16((sh_max.B, sh_max.Lkv, sh_max.H, sh_max.d), dev, gen)
+        self.v = si.device_normal_bf16((sh_max.B, sh_max.Lkv, sh_max.H, sh_max.d), dev, gen)
+        d = ispa.attn_desc(sh_max, ispa.ISPA_BF16, ispa.ISPA_F32)
+        self.v16 = torch.empty(ispa.ispa_v16_bytes(d), device=dev, dtype=torch.uint8)
+
+
+def attention_point(ispa, torch, stream, dev, sh, cache, reps):
+    """Split attention (fused merge, fp32 out, as in warmup) and the post-switch
+    F-layer (one group over every frame, bf16 out) at frame layout sh on the
+    cache's buffers (prepared V for every frame first, untimed)."""
+    import dataclasses
+    B, Lq, H = sh.B, sh.Lq, sh.H
+    desc = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_F32)
+    ispa.ispa_v16_prepare(desc, cache.v, 0, sh.kv_frames, cache.v16, stream=stream)
+    pd = ispa.prepared(desc)
+    q = si.device_normal_bf16((B, Lq, H, 128), dev, si.torch_generator(dev, "sweep-q", B, H))
+    o = {n: torch.empty((B, Lq, H, 128), device=dev) for n in ("loc", "hist", "full")}
+    l = {n: torch.empty((B, Lq, H), device=dev) for n in ("loc", "hist", "full")}
+    t_split = timed_calls(torch, stream, lambda: ispa.ispa_attn_split(
+        pd, q, cache.k, cache.v16, o["loc"], l["loc"], o["hist"], l["hist"], o["full"], l["full"], stream=stream),
+        reps)
+    shF = dataclasses.replace(sh, sink_frames=sh.cur_begin, hist_begin=0, hist_end=0)
+    pdF = ispa.prepared(ispa.attn_desc(shF, ispa.ISPA_BF16, ispa.ISPA_BF16))
+    ob = torch.empty((B, Lq, H, 128), device=dev, dtype=torch.bfloat16)
+    t_full = timed_calls(torch, stream, lambda: ispa.ispa_attn_split(pdF, q, cache.k, cache.v16, ob, l["loc"],
+                                                                       stream=stream), reps)
+    flops = 4.0 * B * Lq * sh.Lkv * H * 128
+    return {"attn_split_ms": t_split, "attn_split_tflops": flops / (t_split * 1e-3) / 1e12,
+            "query_tok_per_s": B * Lq / (t_split * 1e-3), "f_layer_attn_ms": t_full,
+            "f_layer_attn_tflops": flops / (t_full * 1e-3) / 1e12}
+
+
+def local_attention_ms(ispa, torch, stream, dev, sh, cache, reps):
+    """The post-switch L-layer's attention (sink + current only) at layout sh."""
+    B, Lq, H = sh.B, sh.Lq, sh.H
+    desc = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_BF16)
+    ispa.ispa_v16_prepare(desc, cache.v, 0, sh.kv_frames, cache.v16, stream=stream)
+    pd = ispa.prepared(desc)
+    q = si.device_normal_bf16((B, Lq, H, 128), dev, si.torch_generator(dev, "sweep-ql", B, H))
+    o = torch.empty((B, Lq, H, 128), device=dev, dtype=torch.bfloat16)
+    lse = torch.empty((B, Lq, H), device=dev)
+    return timed_calls(torch, stream, lambda: ispa.ispa_attn_split(pd, q, cache.k, cache.v16, o, lse, stream=stream),
+                       reps)
+
+
+SWEEP_HIST = (3, 9, 15, 30, 60, 90, 117)
+SWEEP_X = (0.0, 0.25, 0.5)
+SWEEP_SHAPES = (("1.3B", 12, 30), ("14B", 40, 40))
+
+
+def sweep_component(ispa, torch, stream, dev, solve_ms: dict, reps: int = 2, emit=None):
+    """History 3 -> 117 frames x ISPA-x in {0, 0.25, 0.5} x batch {1, 2} on both
+    shapes: attention TFLOP/s and query tok/s of the warmup split attention, the
+    F- and L-layer attention, merge GB/s, solve ms/layer, and the KV bytes a
+    model keeps, with the post-switch attention time of a model chunk.  One KV
+    buffer per (shape, batch) sized for 117 history frames is reused."""
+    points = []
+    for name, H, N in SWEEP_SHAPES:
+        for B in (1, 2):
+            sh_max = si.video_shape(H, max(SWEEP_HIST), B=B)
+            cache = KVCache(ispa, torch, dev, sh_max, si.torch_generator(dev, "sweep", name, B))
+            t_loc = local_attention_ms(ispa, torch, stream, dev, si.video_shape(H, min(SWEEP_HIST), B=B), cache, reps)
+            mrate = merge_rate(ispa, torch, stream, dev, B * sh_max.Lq, H)
+            for Hf in SWEEP_HIST:
+                sh = si.video_shape(H, Hf, B=B)
+                pt = {"shape": name, "B": B, "hist_frames": Hf, "Lq": sh.Lq, "Lkv": sh.Lkv, "heads": H,
+                      **attention_point(ispa, torch, stream, dev, sh, cache, reps),
+                      "l_layer_attn_ms": t_loc, "merge_gb_s": mrate["merge_gb_s"],
+                      "solve_ms_per_layer": solve_ms.get(name)}
+                pt["x"] = {}
+                for x in SWEEP_X:
+                    kv = kv_retained(sh, B, N, x)
+                    kv["post_switch_attn_ms_per_chunk"] = ((N - kv["l_layers"]) * pt["f_layer_attn_ms"] +
+                                                           kv["l_layers"] * t_loc)
+                    pt["x"][str(x)] = kv
+                points.append(pt)
+                if emit:
+                    emit(pt)
+            del cache
+            torch.cuda.empty_cache()
+    return points
+
+
+def solve_ms_at(ispa, torch, stream, dev, D: int, T: int, reps: int = 3):
+    """The ridge solve at width D from statistics of T rows (graph-timed)."""
+    g = si.torch_generator(dev, "solve", D)
+    A = torch.randn((T, D), device=dev, generator=g)
+    G = torch.triu(A.T @ A)
+    C = A.T @ torch.randn((T, D), device=dev, generator=g)
+    r2 = torch.ones(1, device=dev, dtype=torch.float64)
+    del A
+    dW = torch.empty((D, D), device=dev)
+    eps = torch.zeros(1, device=dev, dtype=torch.float64)
+    ws = torch.empty(ispa.ispa_ridge_workspace_bytes(D, D), device=dev, dtype=torch.uint8)
+    ms = graph_time(torch, stream, dev, lambda: ispa.ispa_ridge_solve(D, D, G, C, r2, LAMBDA_REL, True, 0, dW, eps, ws,
+                                                                      stream=stream), reps)
+    ispa.ispa_check_device_error(stream)
+    return ms
+
+
+def cfg4_component(ispa, torch, stream, dev):
+    """The 14B-shaped layer (40 x 128, D = 5120, sink 3 + history 60 + chunk 3):
+    split attention, merge, statistics of one chunk (T = 4680) and the 5120^2 solve."""
+    sh = si.SHAPE_14B
+    B, Lq, H, D = sh.B, sh.Lq, sh.H, sh.D
+    T = B * Lq
+    drift = si.drift_layer_kv_device(sh, 0, ("bench", "cfg4"), dev)
+    k = torch.empty((B, sh.Lkv, H, 128), device=dev, dtype=torch.bfloat16)
+    v = torch.empty_like(k)
+    n = sh.cur_begin * sh.tpf
+    k[:, :n], v[:, :n] = drift["k"], drift["v"]
+    del drift
+    g = si.torch_generator(dev, "bench", "cfg4", "chunk")
+    k[:, n:] = si.device_normal_bf16((B, sh.Lkv - n, H, 128), dev, g)
+    v[:, n:] = si.device_normal_bf16((B, sh.Lkv - n, H, 128), dev, g)
+    q = si.device_normal_bf16((B, Lq, H, 128), dev, g)
+    desc = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_F32)
+    v16 = torch.empty(ispa.ispa_v16_bytes(desc), device=dev, dtype=torch.uint8)
+    ispa.ispa_v16_prepare(desc, v, 0, sh.kv_frames, v16, stream=stream)
+    pd = ispa.prepared(desc)
+    o = {nm: torch.empty((B, Lq, H, 128), device=dev) for nm in ("loc", "hist", "full")}
+    l = {nm: torch.empty((B, Lq, H), device=dev) for nm in ("loc", "hist", "full")}
+    t_attn = timed_calls(torch, stream, lambda: ispa.ispa_attn_split(
+        pd, q, k, v16, o["loc"], l["loc"], o["hist"], l["hist"], o["full"], l["full"], stream=stream), 3)
+    t_prep = timed_calls(torch, stream, lambda: ispa.ispa_v16_prepare(desc, v, sh.cur_begin, sh.cur_end, v16,
+                                                                      stream=stream), 5)
+    W = si.device_normal_bf16((D, D), dev, g, 1.0 / math.sqrt(D)).float()
+    G = torch.zeros((D, D), device=dev)
+    C = torch.zeros((D, D), device=dev)
+    r2 = torch.zeros(1, device=dev, dtype=torch.float64)
+    ws = torch.empty(ispa.ispa_accum_stats_workspace_bytes(T, D, D), device=dev, dtype=torch.uint8)
+    a_loc, a_full = o["loc"].reshape(T, D), o["full"].reshape(T, D)
+
+    def stats():
+        ispa.ispa_accum_stats(T, D, D, a_loc, a_full, W, G, C, r2, ispa.ISPA_PREC_TF32, ws, stream=stream)
+
+    t_stats = timed_calls(torch, stream, stats, 3)
+    G.zero_()
+    C.zero_()
+    r2.zero_()
+    stats()
+    dW = torch.empty((D, D), device=dev)
+    eps = torch.zeros(1, device=dev, dtype=torch.float64)
+    del ws, k, v, v16, q
+    torch.cuda.empty_cache()
+    rws = torch.empty(ispa.ispa_ridge_workspace_bytes(D, D), device=dev, dtype=torch.uint8)
+    t_solve = graph_time(torch, stream, dev, lambda: ispa.ispa_ridge_solve(D, D, G, C, r2, LAMBDA_REL, True, 0, dW, eps,
+                                                                           rws, stream=stream), 3)
+    ispa.ispa_check_device_error(stream)
+    w = step_work(sh)
+    mrate = merge_rate(ispa, torch, stream, dev, T, H)
+    out = {"workload": "14B-shaped layer: 40x128 heads (D=5120), 1560 tok/frame, sink 3 + history 60 + chunk 3 "
+                       "(4680 queries x 102960 keys), drift history (device-drawn)",
+           "attn_split_ms": t_attn, "attn_split_tflops": w["attn_split"] / (t_attn * 1e-3) / 1e12,
+           "query_tok_per_s": T / (t_attn * 1e-3), "v16_prepare_chunk_ms": t_prep,
+           "stats_ms": t_stats, "stats_tflops": w["stats"] / (t_stats * 1e-3) / 1e12,
+           "solve_ms_per_layer": t_solve, "solve_gflop": w["solve"] / 1e9, "eps": float(eps.item()),
+           **mrate, "kv_retained_isp_0p5": kv_retained(sh, B, 40, 0.5)}
+    return out
+
+
+def cfg3_component(ispa, torch, stream, dev, n_layers: int = 30, warm_chunks: int = 8, post_chunks: int = 16,
+                   heldout_chunks: int = 2, x: float = 0.5):
+    """The 30-layer 1.3B-shaped warmup and switch on device-drawn drift inputs:
+    per layer 8 warmup chunks (prepared V, split attention, statistics), then a
+    solve; 2 held-out chunks give each layer's held-out epsilon of its dW
+    (ispa_absorb_error); ISPA-0.5 selects 15 L-layers; 16 post-switch chunks run
+    the model (L-layers on evicted K/V projected with W + dW, F-layers over every
+    frame with W), timed per chunk."""
+    import dataclasses
+    sh = si.SHAPE_1P3B
+    B, Lq, H, D = sh.B, sh.Lq, sh.H, sh.D
+    T = B * Lq
+    K_sel = int(math.floor(x * n_layers + 1e-9))
+    desc = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_F32)
+    pd = ispa.prepared(desc)
+    k = torch.empty((B, sh.Lkv, H, 128), device=dev, dtype=torch.bfloat16)
+    v = torch.empty_like(k)
+    v16 = torch.empty(ispa.ispa_v16_bytes(desc), device=dev, dtype=torch.uint8)
+    o = {nm: torch.empty((B, Lq, H, 128), device=dev) for nm in ("loc", "full")}
+    l = {nm: torch.empty((B, Lq, H), device=dev) for nm in ("loc", "full")}
+    ws = torch.empty(ispa.ispa_accum_stats_workspace_bytes(T, D, D), device=dev, dtype=torch.uint8)
+    rws = torch.empty(ispa.ispa_ridge_workspace_bytes(D, D), device=dev, dtype=torch.uint8)
+    ews = torch.empty(ispa.ispa_absorb_error_workspace_bytes(D, D), device=dev, dtype=torch.uint8)
+    G, C = torch.zeros((D, D), device=dev), torch.zeros((D, D), device=dev)
+    Gh, Ch = torch.zeros((D, D), device=dev), torch.zeros((D, D), device=dev)
+    r2, r2h = torch.zeros(1, device=dev, dtype=torch.float64), torch.zeros(1, device=dev, dtype=torch.float64)
+    eps = torch.zeros(n_layers, device=dev, dtype=torch.float64)
+    eps_held = torch.zeros(n_layers, device=dev, dtype=torch.float64)
+    dWs, Ws = [], []
+    n = sh.cur_begin * sh.tpf
+    e0, e1, s0, s1 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
+    warm_ms, solve_ms = 0.0, []
+    for layer in range(n_layers):
+        drift = si.drift_layer_kv_device(sh, layer, ("bench", "cfg3"), dev)
+        k[:, :n], v[:, :n] = drift["k"], drift["v"]
+        del drift
+        W = si.device_normal_bf16((D, D), dev, si.torch_generator(dev, "bench", "cfg3", "W", layer),
+                                  1.0 / math.sqrt(D)).float()
+        for t in (G, C, r2, Gh, Ch, r2h):
+            t.zero_()
+        for c in range(warm_chunks + heldout_chunks):
+            gch = si.torch_generator(dev, "bench", "cfg3", layer, c)
+            k[:, n:] = si.device_normal_bf16((B, Lq, H, 128), dev, gch)
+            v[:, n:] = si.device_normal_bf16((B, Lq, H, 128), dev, gch)
+            q = si.device_normal_bf16((B, Lq, H, 128), dev, gch)
+            heldout = c >= warm_chunks
+            if c == 0:
+                ispa.ispa_v16_prepare(desc, v, 0, sh.kv_frames, v16, stream=stream)
+            if not heldout:
+                e0.record(stream)
+            if c > 0:
+                ispa.ispa_v16_prepare(desc, v, sh.cur_begin, sh.cur_end, v16, stream=stream)
+            ispa.ispa_attn_split(pd, q, k, v16, o["loc"], l["loc"], None, None, o["full"], l["full"], stream=stream)
+            ispa.ispa_accum_stats(T, D, D, o["loc"].reshape(T, D), o["full"].reshape(T, D), W,
+                                  Gh if heldout else G, Ch if heldout else C, r2h if heldout else r2,
+                                  ispa.ISPA_PREC_TF32, ws, stream=stream)
+            if not heldout:
+                e1.record(stream)
+                e1.synchronize()
+                warm_ms += e0.elapsed_time(e1)
+        dW = torch.empty((D, D), device=dev)
+        s0.record(stream)
+        ispa.ispa_ridge_solve(D, D, G, C, r2, LAMBDA_REL, True, 0, dW, eps[layer:layer + 1], rws, stream=stream)
+        s1.record(stream)
+        ispa.ispa_absorb_error(D, D, Gh, Ch, r2h, dW, eps_held[layer:layer + 1], ews, stream=stream)
+        s1.synchronize()
+        solve_ms.append(s0.elapsed_time(s1))
+        dWs.append(dW)
+        Ws.append(W)
+    ispa.ispa_check_device_error(stream)
+    mask = torch.zeros(n_layers, device=dev, dtype=torch.uint8)
+    idx = torch.zeros(max(K_sel, 1), device=dev, dtype=torch.int32)
+    ispa.ispa_select_layers(n_layers, eps, K_sel, mask, idx, stream=stream)
+    torch.cuda.synchronize(dev)
+    chosen = set(idx[:K_sel].cpu().tolist())
+    # post-switch: L-layers on their evicted K/V with W + dW, F-layers on every frame with W
+    # (one buffer of each kind serves every layer of its kind; the weights are each layer's own)
+    descL_full = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_BF16)
+    descL = ispa.ispa_kv_evicted_desc(descL_full)
+    kept = (B, descL.kv_frames * sh.tpf, H, 128)
+    kL, vL = torch.empty(kept, device=dev, dtype=torch.bfloat16), torch.empty(kept, device=dev, dtype=torch.bfloat16)
+    ispa.ispa_kv_evict_history(descL_full, k, v, kL, vL, stream=stream)
+    v16L = torch.empty(ispa.ispa_v16_bytes(descL), device=dev, dtype=torch.uint8)
+    ispa.ispa_v16_prepare(descL, vL, 0, descL.kv_frames, v16L, stream=stream)
+    shF = dataclasses.replace(sh, sink_frames=sh.cur_begin, hist_begin=0, hist_end=0)
+    descF = ispa.attn_desc(shF, ispa.ISPA_BF16, ispa.ISPA_BF16)
+    pL, pF = ispa.prepared(descL), ispa.prepared(descF)
+    w_eff = []
+    for layer in range(n_layers):
+        Wb = Ws[layer].to(torch.bfloat16)
+        if layer in chosen:
+            Wn = torch.empty((D, D), device=dev, dtype=torch.bfloat16)
+            ispa.ispa_absorb_weight(D, D, Wb, ispa.ISPA_BF16, dWs[layer], Wn, ispa.ISPA_BF16, stream=stream)
+            w_eff.append(Wn)
+        else:
+            w_eff.append(Wb)
+    wsp = torch.empty(max(ispa.ispa_attn_local_proj_workspace_bytes(pL), ispa.ispa_attn_local_proj_workspace_bytes(pF),
+                          16), device=dev, dtype=torch.uint8)
+    y = torch.empty((B, Lq, D), device=dev, dtype=torch.bfloat16)
+    qp = si.device_normal_bf16((B, Lq, H, 128), dev, si.torch_generator(dev, "bench", "cfg3", "post"))
+    all_f_ms = []
+    for c in range(4):  # the same model chunk with no layer switched (ISPA-0): every layer an F-layer
+        e0.record(stream)
+        for layer in range(n_layers):
+            ispa.ispa_v16_prepare(descF, v, descF.cur_begin, descF.cur_end, v16, stream=stream)
+            ispa.ispa_attn_local_proj(pF, qp, k, v16, Ws[layer].to(torch.bfloat16), D, y, ispa.ISPA_BF16, wsp,
+                                      stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        if c > 0:
+            all_f_ms.append(e0.elapsed_time(e1))
+    post_ms = []
+    for c in range(post_chunks + 1):
+        e0.record(stream)
+        for layer in range(n_layers):
+            if layer in chosen:
+                ispa.ispa_v16_prepare(descL, vL, descL.cur_begin, descL.cur_end, v16L, stream=stream)
+                ispa.ispa_attn_local_proj(pL, qp, kL, v16L, w_eff[layer], D, y, ispa.ISPA_BF16, wsp, stream=stream)
+            else:
+                ispa.ispa_v16_prepare(descF, v, descF.cur_begin, descF.cur_end, v16, stream=stream)
+                ispa.ispa_attn_local_proj(pF, qp, k, v16, w_eff[layer], D, y, ispa.ISPA_BF16, wsp, stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        if c > 0:  # the first chunk warms up
+            post_ms.append(e0.elapsed_time(e1))
+    ispa.ispa_check_device_error(stream)
+    e_all = eps.cpu().numpy()
+    e_held = eps_held.cpu().numpy()
+    order = np.sort(e_all)
+    return {"workload": "1.3B-shaped model: 30 layers, drift history (device-drawn), 8 warmup chunks per layer, "
+                        "ISPA-0.5, 16 post-switch chunks",
+            "warmup_ms_per_layer_chunk": warm_ms / (n_layers * warm_chunks),
+            "solve_ms_per_layer": float(np.mean(solve_ms)), "solve_ms_per_layer_max": float(np.max(solve_ms)),
+            "eps": e_all.tolist(), "eps_heldout": e_held.tolist(),
+            "selected": sorted(chosen),
+            "eps_gap_at_K": float((order[K_sel] - order[K_sel - 1]) / order[K_sel]) if 0 < K_sel < n_layers else None,
+            "heldout_over_warmup_eps_selected": float(np.mean([e_held[i] / e_all[i] for i in sorted(chosen)])),
+            "post_switch_ms_per_chunk": float(np.mean(post_ms)),
+            "post_switch_ms_per_chunk_no_switch": float(np.mean(all_f_ms)),
+            "kv_retained": kv_retained(sh, B, n_layers, x)}
 
 
 def run_ours(args, world, rank, local):
@@ -390,7 +762,6 @@ def run_ours(args, world, rank, local):
     W_new = torch.empty((D, D), device=dev, dtype=torch.bfloat16)
     y = {n: torch.empty((B, Lq, D), device=dev, dtype=torch.bfloat16) for n in ("L", "F")}
     desc_warm = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_F32)
-    ws_attn = torch.empty(ispa.ispa_attn_split_workspace_bytes(desc_warm), device=dev, dtype=torch.uint8)
     # the switch: the L-layer drops its history (real eviction: the kept frames
     # go to new buffers, the originals are released; bytes from the allocator)
     desc_L_full = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_BF16)
@@ -416,13 +787,21 @@ def run_ours(args, world, rank, local):
         N_LAYERS * sh.kv_frames)
     kept_rows = torch.tensor([f * sh.tpf + t for f in range(sh.kv_frames)
                               if f < sh.sink_frames or sh.cur_begin <= f < sh.cur_end for t in range(sh.tpf)])
-    for n in ("k", "v"):  # the end-to-end path streams the evicted layout from the host
+    for n in ("k", "v"):  # the end-to-end path streams the evicted layout's chunk rows from the host
         LL_.host[n] = LL_.host[n].index_select(1, kept_rows).contiguous().pin_memory()
     import dataclasses
     shF = dataclasses.replace(sh, sink_frames=sh.cur_begin, hist_begin=0, hist_end=0)
     desc_F = ispa.attn_desc(shF, ispa.ISPA_BF16, ispa.ISPA_BF16)
-    ws_proj = torch.empty(max(ispa.ispa_attn_local_proj_workspace_bytes(desc_L),
-                              ispa.ispa_attn_local_proj_workspace_bytes(desc_F)), device=dev, dtype=torch.uint8)
+    # every layer keeps a prepared fp16 copy of its V next to its cache: made
+    # once here for every frame, then each step prepares the chunk's frames only
+    descs = [desc_warm, desc_L, desc_F]
+    pdescs = [ispa.prepared(d_) for d_ in descs]
+    pdesc_warm, pdesc_L, pdesc_F = pdescs
+    for Lr, d_ in zip(layers, descs):
+        Lr.attach(ispa, d_, dev)
+    torch.cuda.synchronize(dev)
+    ws_proj = torch.empty(max(ispa.ispa_attn_local_proj_workspace_bytes(pdesc_L),
+                              ispa.ispa_attn_local_proj_workspace_bytes(pdesc_F), 16), device=dev, dtype=torch.uint8)
     # a stream of its own: the step is captured into a CUDA graph, which the
     # legacy default stream does not allow
     stream = torch.cuda.Stream(dev)
@@ -432,15 +811,20 @@ def run_ours(args, world, rank, local):
     def solve():
         ispa.ispa_ridge_solve(D, D, G, C, r2, LAMBDA_REL, True, 0, dW, eps_all[7:8], ws_ridge, stream=stream)
 
+    def prepare_chunk(Lr):
+        d_ = Lr.desc
+        ispa.ispa_v16_prepare(d_, Lr.dev["v"], d_.cur_begin, d_.cur_end, Lr.dev["v16"], stream=stream)
+
     def step(timed_components: bool):
         Lw, LL, LF = layers
         G.zero_()
         C.zero_()
         r2.zero_()
+        prepare_chunk(Lw)
         if timed_components:
             ev_attn[0].record(stream)
-        ispa.ispa_attn_split(desc_warm, Lw.dev["q"], Lw.dev["k"], Lw.dev["v"], o["loc"], l["loc"], o["hist"],
-                             l["hist"], o["full"], l["full"], workspace=ws_attn, stream=stream)
+        ispa.ispa_attn_split(pdesc_warm, Lw.dev["q"], Lw.dev["k"], Lw.dev["v16"], o["loc"], l["loc"], o["hist"],
+                             l["hist"], o["full"], l["full"], stream=stream)
         if timed_components:
             ev_attn[1].record(stream)
         ispa.ispa_accum_stats(T, D, D, o["loc"], o["full"], wcur["W32"], G, C, r2, ispa.ISPA_PREC_TF32, ws_stats,
@@ -448,9 +832,11 @@ def run_ours(args, world, rank, local):
         solve()
         ispa.ispa_select_layers(N_LAYERS, eps_all, K_sel, is_local, idx, stream=stream)
         ispa.ispa_absorb_weight(D, D, W16, ispa.ISPA_BF16, dW, W_new, ispa.ISPA_BF16, stream=stream)
-        ispa.ispa_attn_local_proj(desc_L, LL.dev["q"], LL.dev["k"], LL.dev["v"], W_new, D, y["L"], ispa.ISPA_BF16,
-                                  ws_proj, stream=stream)
-        ispa.ispa_attn_local_proj(desc_F, LF.dev["q"], LF.dev["k"], LF.dev["v"], W16, D, y["F"], ispa.ISPA_BF16,
+        prepare_chunk(LL)
+        ispa.ispa_attn_local_proj(pdesc_L, LL.dev["q"], LL.dev["k"], LL.dev["v16"], W_new, D, y["L"],
+                                  ispa.ISPA_BF16, ws_proj, stream=stream)
+        prepare_chunk(LF)
+        ispa.ispa_attn_local_proj(pdesc_F, LF.dev["q"], LF.dev["k"], LF.dev["v16"], W16, D, y["F"], ispa.ISPA_BF16,
                                   ws_proj, stream=stream)
 
     # one eager step sets up every kernel's attributes; then the step and the
@@ -506,23 +892,22 @@ def run_ours(args, world, rank, local):
     # ---- the W8A8 post-switch L-layer: the same step with its projection in
     # 8 bits (e4m3, int8), against the bf16 step; repeated launches, K/V of
     # the evicted layer L2-resident for both alike
-    w8a8 = w8a8_component(ispa, torch, stream, dev, desc_L, layers[1], W_new, y["L"], o["loc"], T, D, ws_proj)
+    w8a8 = w8a8_component(ispa, torch, stream, dev, pdesc_L, layers[1], W_new, y["L"], o["loc"], T, D, ws_proj)
 
     # ---- the fused warmup step (attention writing the statistics' operands)
     # against the two calls it replaces, on the warmup layer
     Lw = layers[0]
 
     def two_calls():
-        ispa.ispa_attn_split(desc_warm, Lw.dev["q"], Lw.dev["k"], Lw.dev["v"], o["loc"], l["loc"], o["hist"],
-                             l["hist"], o["full"], l["full"], workspace=ws_attn, stream=stream)
+        ispa.ispa_attn_split(pdesc_warm, Lw.dev["q"], Lw.dev["k"], Lw.dev["v16"], o["loc"], l["loc"], o["hist"],
+                             l["hist"], o["full"], l["full"], stream=stream)
         ispa.ispa_accum_stats(T, D, D, o["loc"], o["full"], W32, G, C, r2, ispa.ISPA_PREC_TF32, ws_stats,
                               stream=stream)
-
-    ws_fused = torch.empty(ispa.ispa_warmup_fused_workspace_bytes(desc_warm, D), device=dev, dtype=torch.uint8)
+    ws_fused = torch.empty(ispa.ispa_warmup_fused_workspace_bytes(pdesc_warm, D), device=dev, dtype=torch.uint8)
 
     def fused():
-        ispa.ispa_warmup_fused(desc_warm, Lw.dev["q"], Lw.dev["k"], Lw.dev["v"], W32, D, o["full"], l["full"], G, C,
-                               r2, ws_fused, stream=stream)
+        ispa.ispa_warmup_fused(pdesc_warm, Lw.dev["q"], Lw.dev["k"], Lw.dev["v16"], W32, D, o["full"], l["full"], G,
+                               C, r2, ws_fused, stream=stream)
 
     warm_fused = {"two_calls_ms": graph_time(torch, stream, dev, two_calls, 5),
                   "fused_ms": graph_time(torch, stream, dev, fused, 5)}
@@ -551,39 +936,50 @@ def run_ours(args, world, rank, local):
     del msets
     merge_bytes = T * H * (3 * 128 * 4 + 3 * 4)  # two O and L read, one written (fp32)
     stats_ms = graph_time(torch, stream, dev, stats_only, 5)
+    prep_ms = graph_time(torch, stream, dev, lambda: prepare_chunk(layers[0]), 10)
     # post-switch attention + projection of an L-layer (evicted, 9360 keys)
     # against an F-layer (all 32760 keys): the analogue of the pages' attention
     # speed-up of the switched layers
     LLr, LFr = layers[1], layers[2]
 
     def l_layer():
-        ispa.ispa_attn_local_proj(desc_L, LLr.dev["q"], LLr.dev["k"], LLr.dev["v"], W_new, D, y["L"], ispa.ISPA_BF16,
-                                  ws_proj, stream=stream)
+        ispa.ispa_attn_local_proj(pdesc_L, LLr.dev["q"], LLr.dev["k"], LLr.dev["v16"], W_new, D, y["L"],
+                                  ispa.ISPA_BF16, ws_proj, stream=stream)
 
     def f_layer():
-        ispa.ispa_attn_local_proj(desc_F, LFr.dev["q"], LFr.dev["k"], LFr.dev["v"], W16, D, y["F"], ispa.ISPA_BF16,
-                                  ws_proj, stream=stream)
+        ispa.ispa_attn_local_proj(pdesc_F, LFr.dev["q"], LFr.dev["k"], LFr.dev["v16"], W16, D, y["F"],
+                                  ispa.ISPA_BF16, ws_proj, stream=stream)
 
     l_ms = graph_time(torch, stream, dev, l_layer, 5)
     f_ms = graph_time(torch, stream, dev, f_layer, 5)
     extra = {"merge_ms": merge_ms, "merge_gb_s": merge_bytes / (merge_ms * 1e-3) / 1e9,
              "stats_ms": stats_ms, "stats_tflops": work["stats"] / (stats_ms * 1e-3) / 1e12,
+             "v16_prepare_chunk_ms": prep_ms,
              "l_layer_ms": l_ms, "f_layer_ms": f_ms, "f_over_l": f_ms / l_ms}
 
     # ---- end to end through the C ABI with host buffers
-    h2d = sum(t.numel() * t.element_size() for Lr in layers for t in Lr.host.values()) + W_host.numel() * 4
+    # Per step the host sends what a generator produces for one chunk: each
+    # layer's queries and the chunk's own K/V frames (the earlier frames are the
+    # layers' device-resident KV caches), and W; the step's outputs come back.
+    chunk_rows = [slice(Lr.desc.cur_begin * sh.tpf, Lr.desc.cur_end * sh.tpf) for Lr in layers]
+    h2d = sum(Lr.host["q"].numel() * 2 + 2 * Lr.host["k"][:, rs].numel() * 2 for Lr, rs in zip(layers, chunk_rows))
+    h2d += W_host.numel() * 4
+    host_chunks = [{"q": Lr.host["q"], "k": Lr.host["k"][:, rs].contiguous().pin_memory(),
+                    "v": Lr.host["v"][:, rs].contiguous().pin_memory()} for Lr, rs in zip(layers, chunk_rows)]
     y_host = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in y.items()}
     dW_host = torch.empty((D, D)).pin_memory()
     small_host = torch.empty(N_LAYERS, dtype=torch.float64).pin_memory()
     d2h = sum(t.numel() * t.element_size() for t in y_host.values()) + dW_host.numel() * 4 + N_LAYERS * 8
 
-    # Every step copies all of its inputs (Q/K/V of the three layers and W)
-    # from pinned host memory and reads its results back.  The copies of step
-    # i + 1 run on a copy stream into a second set of input buffers while step
-    # i computes on the first (double buffering, ordered by events), so the
-    # step costs max(copy, compute) instead of their sum.
-    sets = [([Lr.dev for Lr in layers], W32),
-            ([{n: torch.empty_like(t) for n, t in Lr.dev.items()} for Lr in layers], torch.empty_like(W32))]
+    # Two device sets of every layer's buffers (their cache frames identical):
+    # the copies of step i + 1 run on a copy stream into one set while step i
+    # computes on the other (double buffering, ordered by events), so a step
+    # costs max(copy, compute) instead of their sum.
+    set1 = []
+    for Lr in layers:
+        d1 = {n: t.clone() for n, t in Lr.dev.items()}
+        set1.append(d1)
+    sets = [([Lr.dev for Lr in layers], W32), (set1, torch.empty_like(W32))]
     copy_stream = torch.cuda.Stream(dev)
     copied = [torch.cuda.Event(), torch.cuda.Event()]
     freed = [torch.cuda.Event(), torch.cuda.Event()]
@@ -593,9 +989,10 @@ def run_ours(args, world, rank, local):
         with torch.cuda.stream(copy_stream):
             if i >= 2:
                 copy_stream.wait_event(freed[i % 2])  # step i - 2 is done with this set
-            for Lr, d in zip(layers, devs):
-                for n in ("q", "k", "v"):
-                    d[n].copy_(Lr.host[n], non_blocking=True)
+            for hc, d, rs in zip(host_chunks, devs, chunk_rows):
+                d["q"].copy_(hc["q"], non_blocking=True)
+                d["k"][:, rs].copy_(hc["k"], non_blocking=True)
+                d["v"][:, rs].copy_(hc["v"], non_blocking=True)
             wd.copy_(W_host, non_blocking=True)
             copied[i % 2].record(copy_stream)
 
@@ -631,10 +1028,23 @@ def run_ours(args, world, rank, local):
         Lr.dev = d
     wcur["W32"] = W32
     e2e_ms = reduce_over_ranks(e0.elapsed_time(e1) / e2e_steps, "max", dev)
+    del sets, set1
+
+    # ---- the other workloads (outside the timed steps): the 14B-shaped layer,
+    # the 30-layer 1.3B model through its switch, and the history / ISPA-x /
+    # batch sweep on both shapes
+    workloads = {}
+    if not args.no_workloads:
+        workloads["cfg4_14b_layer"] = cfg4_component(ispa, torch, stream, dev)
+        workloads["cfg3_1p3b_model"] = cfg3_component(ispa, torch, stream, dev)
+        workloads["sweep"] = sweep_component(ispa, torch, stream, dev,
+                                             {"1.3B": solve_launch_ms,
+                                              "14B": workloads["cfg4_14b_layer"]["solve_ms_per_layer"]})
 
     return dict(ms_step=ms_step, work=work, attn_launch_ms=attn_launch_ms, solve_launch_ms=solve_launch_ms,
                 kv_evict=kv_evict, w8a8=w8a8, warm_fused=warm_fused, extra=extra,
-                launches=launches, clocks=clocks.summary(), e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, world=world, rank=rank)
+                launches=launches, clocks=clocks.summary(), e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, world=world, rank=rank,
+                workloads=workloads)
 
 
 # ---------------------------------------------------------------------------
@@ -853,9 +1263,15 @@ def run_attn_only(args):
     o = {n: torch.empty((sh.B, sh.Lq, sh.H, 128), **f32) for n in ("loc", "hist", "full")}
     l = {n: torch.empty((sh.B, sh.Lq, sh.H), **f32) for n in ("loc", "hist", "full")}
     desc = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_F32)
-    ws = torch.empty(ispa.ispa_attn_split_workspace_bytes(desc), device=dev, dtype=torch.uint8)
-    run = lambda: ispa.ispa_attn_split(desc, L.dev["q"], L.dev["k"], L.dev["v"], o["loc"], l["loc"], o["hist"],
-                                       l["hist"], o["full"], l["full"], workspace=ws)
+    if args.plain_v:  # the call converting V itself (no prepared copy)
+        ws = torch.empty(ispa.ispa_attn_split_workspace_bytes(desc), device=dev, dtype=torch.uint8)
+        run = lambda: ispa.ispa_attn_split(desc, L.dev["q"], L.dev["k"], L.dev["v"], o["loc"], l["loc"], o["hist"],
+                                           l["hist"], o["full"], l["full"], workspace=ws)
+    else:
+        L.attach(ispa, desc, dev)
+        pd = ispa.prepared(desc)
+        run = lambda: ispa.ispa_attn_split(pd, L.dev["q"], L.dev["k"], L.dev["v16"], o["loc"], l["loc"], o["hist"],
+                                           l["hist"], o["full"], l["full"])
     for _ in range(args.warmup):
         run()
     torch.cuda.synchronize()
@@ -872,6 +1288,23 @@ def run_attn_only(args):
     return 0
 
 
+def run_sweep_only(args):
+    """The sweep alone, one JSON line per point (history, batch, shape)."""
+    import torch
+
+    import kv_cache_compression_two_b200 as ispa
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(stream)
+    solve = {"1.3B": solve_ms_at(ispa, torch, stream, dev, 1536, 4680),
+             "14B": solve_ms_at(ispa, torch, stream, dev, 5120, 4680)}
+    sweep_component(ispa, torch, stream, dev, solve, reps=max(1, args.steps),
+                    emit=lambda pt: print(json.dumps({"kernel": "sweep", **pt}), flush=True))
+    ispa.ispa_check_device_error(stream)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -879,7 +1312,10 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-rows", type=int, default=32, help="query rows of the oracle sample (0: skip it)")
-    ap.add_argument("--only", choices=["step", "attn", "proj", "parts"], default="step",
+    ap.add_argument("--plain-v", action="store_true", help="--only attn: V converted by every call")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the 14B layer, the 30-layer model and the sweep (components outside the timed steps)")
+    ap.add_argument("--only", choices=["step", "attn", "proj", "parts", "sweep"], default="step",
                     help="attn: only the split-attention launches; proj: only the post-switch projection "
                          "(bf16, e4m3, int8 products); parts: the merge, the statistics and one solve; "
                          "all for profiling, printing their timing")
@@ -890,6 +1326,8 @@ def main(argv=None):
         return run_parts_only(args)
     if args.only == "attn":
         return run_attn_only(args)
+    if args.only == "sweep":
+        return run_sweep_only(args)
 
     if args.impl == "reference":
         world, rank, _ = dist_env()
@@ -941,9 +1379,11 @@ def main(argv=None):
                 "query_tok_per_s": world * WORKLOAD.shape.B * WORKLOAD.shape.Lq / (r["attn_launch_ms"] * 1e-3),
                 "attn_split_ms": r["attn_launch_ms"], "solve_ms_per_layer": r["solve_launch_ms"],
                 "step_gflop": work["total"] / 1e9, "kv_eviction": r["kv_evict"], "w8a8_l_layer": r["w8a8"],
-                "warmup_fused": r["warm_fused"], **r["extra"]},
-            "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (two-group attention + fused merge), timed as its "
-                                                   "call: the fp16 V copy (v_prep_kernel, v_fix_kernel) included",
+                "warmup_fused": r["warm_fused"], **r["extra"], **r["workloads"]},
+            "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (two-group attention + fused merge) on the layer's "
+                                                   "prepared fp16 V: the timed call is the kernel alone (the chunk's "
+                                                   "V frames are prepared by a separate call, components."
+                                                   "v16_prepare_chunk_ms)",
                          "achieved": achieved, "peak": peak, "peak_source": peak_src, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": measured_traffic()},
             "gpu_launches": r["launches"],

@@ -118,6 +118,13 @@ ispa_status ispa_selftest_wait_timeout(long long wait_ns, ispa_stream_t stream);
  * A post-switch F-layer (full context) is the same call with
  * sink_frames = cur_begin and an empty history.
  */
+/* What the v argument of the attention calls points at (ispa_attn_desc.v_layout). */
+typedef enum {
+  ISPA_V_PLAIN = 0,       /* V in in_dtype, [B, kv_frames*tpf, H, d]; a bf16 call
+                             converts the rows it reads into its workspace       */
+  ISPA_V_F16_PREPARED = 1 /* a prepared fp16 copy of a bf16 V (ispa_v16_prepare) */
+} ispa_v_layout;
+
 typedef struct {
   int B;                /* independent instances (batch)                        */
   int H;                /* heads                                                */
@@ -130,6 +137,7 @@ typedef struct {
   ispa_dtype in_dtype;  /* dtype of Q, K, V                                     */
   ispa_dtype out_dtype; /* dtype of the O outputs                               */
   float softmax_scale;  /* <= 0 selects 1/sqrt(head_dim)                        */
+  ispa_v_layout v_layout; /* ISPA_V_PLAIN, or ISPA_V_F16_PREPARED (bf16, d = 128) */
 } ispa_attn_desc;
 
 /*
@@ -150,9 +158,10 @@ typedef struct {
  * head_dim 32/64/128 (fp32 CUDA cores).  Outputs may not alias inputs.
  * Every K/V row that a group's 128-row tiles cover must hold finite values.
  *   workspace  >= ispa_attn_split_workspace_bytes(desc) bytes, 16-byte aligned
- *              (0 for fp32 inputs; for bf16 inputs it holds a power-of-two
- *              scaled fp16 copy of the V rows in use, so that the softmax
- *              weights enter the PV product with 11 significant bits).
+ *              (0 for fp32 inputs and for a prepared V; for bf16 inputs with
+ *              v_layout ISPA_V_PLAIN it holds a power-of-two scaled fp16 copy
+ *              of the V rows in use, so that the softmax weights enter the PV
+ *              product with 11 significant bits).
  */
 size_t ispa_attn_split_workspace_bytes(const ispa_attn_desc *desc);
 
@@ -160,6 +169,44 @@ ispa_status ispa_attn_split(const ispa_attn_desc *desc, const void *q, const voi
                             const void *v, void *o_loc, float *lse_loc, void *o_hist,
                             float *lse_hist, void *o_full, float *lse_full, void *workspace,
                             size_t workspace_bytes, ispa_stream_t stream);
+
+/*
+ * Prepared fp16 V.  The tensor-core attention multiplies the softmax weights P
+ * (fp16, 11 significant bits) with an fp16 copy of V scaled by a power of two
+ * per (instance, head): v16 = v * 2^e, the exact fp16 image of every bf16 value
+ * whose scaled magnitude lies in [2^-14, 65504] (e = 0 unless a head's largest
+ * |v| reaches 2^15 or its RMS falls below 2^-10; then e puts the largest |v| in
+ * [2^14, 2^15)).  A call with v_layout ISPA_V_PLAIN converts the V rows it reads
+ * on every call.  A caller that keeps V across calls -- the KV cache of a
+ * generator, where a chunk writes a few new frames and the earlier ones stay --
+ * keeps the converted copy instead and converts only the frames that change:
+ * the history group's cost is then paid once, when its frames are written,
+ * not on every chunk [EN-notes, Key Designs 1: the split attention should cost
+ * no more than full attention].
+ *
+ * ispa_v16_bytes(desc): bytes of the prepared copy for desc's K/V layout
+ *   (B * kv_frames * tpf * H * 128 fp16 values, then a per-(instance, head)
+ *   state of the scale); 0 for a desc that is invalid or not bf16 with d = 128.
+ * ispa_v16_prepare(desc, v, frame_begin, frame_end, v16, stream): converts the
+ *   frames [frame_begin, frame_end) of every instance of the bf16 v
+ *   ([B, kv_frames * tpf, H, 128]) into v16 (caller-owned, ispa_v16_bytes,
+ *   16-byte aligned, not overlapping v), updating each head's state.  With
+ *   frame_begin == 0 the state starts afresh: the copy then describes frames
+ *   [0, frame_end), and frames past frame_end must be prepared by later calls
+ *   before an attention call reads them.  When the new frames move a head's
+ *   exponent, every row of that head, frames [0, kv_frames), is converted
+ *   again from v, which must then hold all of them.  Asynchronous.
+ * Use: set desc.v_layout = ISPA_V_F16_PREPARED and pass v16 as the v argument
+ *   of ispa_attn_split, ispa_warmup_fused, ispa_attn_local_proj(_q8) (same
+ *   frame layout; every row a group's 128-row tiles cover must have been
+ *   prepared, from finite values).  ispa_kv_evict_history / ispa_kv_restore
+ *   with that desc move a prepared copy and its state (v, v_out of their
+ *   ispa_v16_bytes sizes); after a restore, prepare the history frames again as
+ *   the new warmup writes them.
+ */
+size_t ispa_v16_bytes(const ispa_attn_desc *desc);
+ispa_status ispa_v16_prepare(const ispa_attn_desc *desc, const void *v, int frame_begin, int frame_end, void *v16,
+                             ispa_stream_t stream);
 
 /*
  * LSE-weighted merge of two disjoint groups' results [EN-notes, Key Designs 1]:
@@ -280,6 +327,23 @@ ispa_status ispa_ridge_solve(int D, int Dout, const float *G, const float *C, co
 ispa_status ispa_ridge_solve_noalloc(int D, int Dout, const float *G, const float *C, const double *r2,
                                      float lambda, int lambda_relative, int refine_steps, float *dW,
                                      double *eps, ispa_stream_t stream);
+
+/*
+ * Reconstruction error of a given correction on any statistics [EN-notes, Key
+ * Designs 2 (the error), Key Designs 3 (warmup is re-entered after a scene
+ * change)]: eps = r2 - 2<dW, C> + <dW, G dW> = ||A_loc (W + dW) - A_full W||_F^2
+ * over the rows that G, C, r2 were accumulated from (ispa_accum_stats).  With
+ * the warmup's own statistics and its solve this is the epsilon of
+ * ispa_ridge_solve; with statistics gathered after the switch it is the
+ * held-out error of a layer's absorption, which a caller can watch to decide
+ * when to recalibrate.
+ *   G [D, D] fp32 (upper triangle read), C, dW [D, Dout] fp32, r2 one double:
+ *   inputs; eps one double (device): output.  fp64-accumulated reductions.
+ *   workspace >= ispa_absorb_error_workspace_bytes(D, Dout).  Asynchronous.
+ */
+size_t ispa_absorb_error_workspace_bytes(int D, int Dout);
+ispa_status ispa_absorb_error(int D, int Dout, const float *G, const float *C, const double *r2, const float *dW,
+                              double *eps, void *workspace, size_t workspace_bytes, ispa_stream_t stream);
 
 /*
  * Instance-specific layer selection [EN-notes, Key Designs 3; DE-summary 2,

@@ -24,6 +24,7 @@ ISPA_OK, ISPA_ERR_INVALID_ARG, ISPA_ERR_UNSUPPORTED, ISPA_ERR_CUDA, ISPA_ERR_NOT
 ISPA_F32, ISPA_BF16 = 0, 1
 ISPA_PREC_TF32, ISPA_PREC_F32 = 0, 1
 ISPA_Q8_E4M3, ISPA_Q8_INT8 = 0, 1
+ISPA_V_PLAIN, ISPA_V_F16_PREPARED = 0, 1
 
 STATUS_NAMES = {0: "ISPA_OK", 1: "ISPA_ERR_INVALID_ARG", 2: "ISPA_ERR_UNSUPPORTED", 3: "ISPA_ERR_CUDA",
                 4: "ISPA_ERR_NOT_SPD", 5: "ISPA_ERR_TIMEOUT"}
@@ -35,7 +36,8 @@ EXPORTED = ("ispa_version", "ispa_last_error", "ispa_launch_count", "ispa_check_
             "ispa_attn_local_proj", "ispa_ridge_solve_noalloc", "ispa_kv_evicted_desc", "ispa_kv_evict_history",
             "ispa_kv_restore", "ispa_stats_reset", "ispa_selftest_wait_timeout", "ispa_quantize_rows",
             "ispa_quantize_weight", "ispa_gemm_q8", "ispa_gemm_bf16", "ispa_attn_local_proj_q8_workspace_bytes",
-            "ispa_attn_local_proj_q8", "ispa_warmup_fused_workspace_bytes", "ispa_warmup_fused")
+            "ispa_attn_local_proj_q8", "ispa_warmup_fused_workspace_bytes", "ispa_warmup_fused",
+            "ispa_v16_bytes", "ispa_v16_prepare", "ispa_absorb_error_workspace_bytes", "ispa_absorb_error")
 RIDGE_NOALLOC_MAX_D = RIDGE_NOALLOC_MAX_DOUT = 1024
 
 
@@ -50,13 +52,21 @@ class AttnDesc(ctypes.Structure):
                 ("tokens_per_frame", ctypes.c_int), ("sink_frames", ctypes.c_int), ("hist_begin", ctypes.c_int),
                 ("hist_end", ctypes.c_int), ("cur_begin", ctypes.c_int), ("cur_end", ctypes.c_int),
                 ("kv_frames", ctypes.c_int), ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
-                ("softmax_scale", ctypes.c_float)]
+                ("softmax_scale", ctypes.c_float), ("v_layout", ctypes.c_int)]
 
 
-def attn_desc(shape, in_dtype: int, out_dtype: int, softmax_scale: float = 0.0) -> AttnDesc:
+def attn_desc(shape, in_dtype: int, out_dtype: int, softmax_scale: float = 0.0,
+              v_layout: int = ISPA_V_PLAIN) -> AttnDesc:
     """Builds an AttnDesc from any object with the frame-layout attributes (B, H, d, tpf, ...)."""
     return AttnDesc(shape.B, shape.H, shape.d, shape.tpf, shape.sink_frames, shape.hist_begin, shape.hist_end,
-                    shape.cur_begin, shape.cur_end, shape.kv_frames, in_dtype, out_dtype, softmax_scale)
+                    shape.cur_begin, shape.cur_end, shape.kv_frames, in_dtype, out_dtype, softmax_scale, v_layout)
+
+
+def prepared(desc: AttnDesc) -> AttnDesc:
+    """A copy of desc whose v argument is a prepared fp16 V (ispa_v16_prepare)."""
+    d = AttnDesc.from_buffer_copy(desc)
+    d.v_layout = ISPA_V_F16_PREPARED
+    return d
 
 
 _lib = None
@@ -104,6 +114,10 @@ def lib() -> ctypes.CDLL:
                                     _sz, _vp]),
         "ispa_attn_local_proj_q8": (_ci, [ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp, _ci, _ci, _vp, _ci,
                                           _vp, _sz, _vp]),
+        "ispa_v16_bytes": (_sz, [ctypes.POINTER(AttnDesc)]),
+        "ispa_absorb_error_workspace_bytes": (_sz, [_ci, _ci]),
+        "ispa_absorb_error": (_ci, [_ci, _ci, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+        "ispa_v16_prepare": (_ci, [ctypes.POINTER(AttnDesc), _vp, _ci, _ci, _vp, _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -188,6 +202,15 @@ def ispa_attn_split(desc: AttnDesc, q, k, v, o_loc, lse_loc, o_hist=None, lse_hi
                                  _ptr(lse_full, name="lse_full"), ws, nbytes, _stream(stream)))
 
 
+def ispa_v16_bytes(desc: AttnDesc) -> int:
+    return int(lib().ispa_v16_bytes(ctypes.byref(desc)))
+
+
+def ispa_v16_prepare(desc: AttnDesc, v, frame_begin: int, frame_end: int, v16, stream=None) -> None:
+    _check(lib().ispa_v16_prepare(ctypes.byref(desc), _ptr(v, name="v"), frame_begin, frame_end,
+                                  _ptr(v16, name="v16"), _stream(stream)))
+
+
 def ispa_lse_merge(rows: int, H: int, head_dim: int, o_dtype: int, o_a, lse_a, o_b, lse_b, o_out, lse_out,
                    stream=None) -> None:
     _check(lib().ispa_lse_merge(rows, H, head_dim, o_dtype, _ptr(o_a), _ptr(lse_a), _ptr(o_b), _ptr(lse_b),
@@ -225,6 +248,17 @@ def ispa_ridge_solve_noalloc(D: int, Dout: int, G, C, r2, lam: float, lambda_rel
     (D, Dout <= 1024; the scratch is a static array inside the library, shared by all calls)."""
     _check(lib().ispa_ridge_solve_noalloc(D, Dout, _ptr(G), _ptr(C), _ptr(r2), float(lam), int(bool(lambda_relative)),
                                           int(refine_steps), _ptr(dW), _ptr(eps), _stream(stream)))
+
+
+def ispa_absorb_error_workspace_bytes(D: int, Dout: int) -> int:
+    return int(lib().ispa_absorb_error_workspace_bytes(D, Dout))
+
+
+def ispa_absorb_error(D: int, Dout: int, G, C, r2, dW, eps, workspace, workspace_bytes: int = 0,
+                      stream=None) -> None:
+    ws, nbytes = _ws(workspace, workspace_bytes)
+    _check(lib().ispa_absorb_error(D, Dout, _ptr(G), _ptr(C), _ptr(r2), _ptr(dW), _ptr(eps), ws, nbytes,
+                                   _stream(stream)))
 
 
 def ispa_select_layers(N: int, eps, K: int, is_local, idx, stream=None) -> None:

@@ -154,6 +154,10 @@ ispa_status attn_ranges(const ispa_attn_desc *d, GroupRanges *g, float *scale) {
   if (d->head_dim != 32 && d->head_dim != 64 && d->head_dim != 128)
     return fail(ISPA_ERR_INVALID_ARG, "head_dim must be 32, 64 or 128 (got %d)", d->head_dim);
   if (!dtype_ok(d->in_dtype) || !dtype_ok(d->out_dtype)) return fail(ISPA_ERR_INVALID_ARG, "bad dtype");
+  if (d->v_layout != ISPA_V_PLAIN && d->v_layout != ISPA_V_F16_PREPARED)
+    return fail(ISPA_ERR_INVALID_ARG, "bad v_layout");
+  if (d->v_layout == ISPA_V_F16_PREPARED && (d->in_dtype != ISPA_BF16 || d->head_dim != 128))
+    return fail(ISPA_ERR_INVALID_ARG, "a prepared fp16 V goes with bf16 inputs and head_dim 128");
   const int F = d->kv_frames;
   if (F < 1) return fail(ISPA_ERR_INVALID_ARG, "kv_frames must be >= 1");
   if (d->sink_frames < 0 || d->sink_frames > F) return fail(ISPA_ERR_INVALID_ARG, "sink_frames out of [0, kv_frames]");
@@ -218,16 +222,29 @@ ispa_status kv_remap(const ispa_attn_desc *desc, const void *k, const void *v, v
   const long long kept_rows = len0 + (g.n_loc > 1 ? g.loc_end[1] - g.loc_begin[1] : 0);
   const long long full_bytes = desc->B * full_rows * row_bytes, kept_bytes = desc->B * kept_rows * row_bytes;
   const long long in_bytes = gather ? full_bytes : kept_bytes, out_bytes = gather ? kept_bytes : full_bytes;
+  // a prepared V is longer than K by its per-head state, which moves with it
+  const bool prepared = desc->v_layout == ISPA_V_F16_PREPARED;
+  const long long v_in_bytes =
+      prepared ? (long long)v16_bytes(desc->B, desc->H, (int)(gather ? full_rows : kept_rows)) : in_bytes;
+  const long long v_out_bytes =
+      prepared ? (long long)v16_bytes(desc->B, desc->H, (int)(gather ? kept_rows : full_rows)) : out_bytes;
   auto overlap = [](const void *a, long long na, const void *b, long long nb) {
     const char *x = (const char *)a, *y = (const char *)b;
     return x < y + nb && y < x + na;
   };
-  if (overlap(k_out, out_bytes, k, in_bytes) || overlap(k_out, out_bytes, v, in_bytes) ||
-      overlap(v_out, out_bytes, k, in_bytes) || overlap(v_out, out_bytes, v, in_bytes) ||
-      overlap(k_out, out_bytes, v_out, out_bytes))
+  if (overlap(k_out, out_bytes, k, in_bytes) || overlap(k_out, out_bytes, v, v_in_bytes) ||
+      overlap(v_out, v_out_bytes, k, in_bytes) || overlap(v_out, v_out_bytes, v, v_in_bytes) ||
+      overlap(k_out, out_bytes, v_out, v_out_bytes))
     return fail(ISPA_ERR_INVALID_ARG, "the outputs must not overlap each other or the inputs");
-  return launch_kv_remap(desc->B, full_rows, kept_rows, g.loc_begin[0], len0, g.n_loc > 1 ? g.loc_begin[1] : 0,
-                         row_bytes, gather, k, v, k_out, v_out, s);
+  st = launch_kv_remap(desc->B, full_rows, kept_rows, g.loc_begin[0], len0, g.n_loc > 1 ? g.loc_begin[1] : 0,
+                       row_bytes, gather, k, v, k_out, v_out, s);
+  if (st != ISPA_OK || desc->v_layout != ISPA_V_F16_PREPARED) return st;
+  // a prepared V carries its per-head state (exponent, 2^-e, range statistics) along
+  const int in_rows = (int)(gather ? full_rows : kept_rows), out_rows = (int)(gather ? kept_rows : full_rows);
+  const char *src = static_cast<const char *>(v) + v16_state_offset(desc->B, desc->H, in_rows);
+  char *dst = static_cast<char *>(v_out) + v16_state_offset(desc->B, desc->H, out_rows);
+  return cuda_status(cudaMemcpyAsync(dst, src, v16_state_bytes(desc->B, desc->H), cudaMemcpyDeviceToDevice, s),
+                     "prepared V state copy");
 }
 
 }  // namespace
@@ -265,7 +282,7 @@ size_t ispa_attn_split_workspace_bytes(const ispa_attn_desc *desc) {
   float scale;
   if (attn_ranges(desc, &g, &scale) != ISPA_OK) return 0;
   if (desc->in_dtype != ISPA_BF16) return 0;
-  return attn_tc_workspace_bytes(desc->B, desc->H, g.Lkv);
+  return attn_tc_workspace_bytes(desc->B, desc->H, g.Lkv, desc->v_layout == ISPA_V_F16_PREPARED);
 }
 
 ispa_status ispa_attn_split(const ispa_attn_desc *desc, const void *q, const void *k, const void *v, void *o_loc,
@@ -292,6 +309,34 @@ ispa_status ispa_attn_split(const ispa_attn_desc *desc, const void *q, const voi
   }
   return launch_attn_simt(*desc, g, scale, (const float *)q, (const float *)k, (const float *)v, o_loc, lse_loc, o_hist,
                           lse_hist, o_full, lse_full, (cudaStream_t)stream);
+}
+
+size_t ispa_v16_bytes(const ispa_attn_desc *desc) {
+  GroupRanges g;
+  float scale;
+  if (attn_ranges(desc, &g, &scale) != ISPA_OK) return 0;
+  if (desc->in_dtype != ISPA_BF16 || desc->head_dim != 128) return 0;
+  return v16_bytes(desc->B, desc->H, g.Lkv);
+}
+
+ispa_status ispa_v16_prepare(const ispa_attn_desc *desc, const void *v, int frame_begin, int frame_end, void *v16,
+                             ispa_stream_t stream) {
+  GroupRanges g;
+  float scale;
+  ispa_status st = attn_ranges(desc, &g, &scale);
+  if (st != ISPA_OK) return st;
+  if (desc->in_dtype != ISPA_BF16 || desc->head_dim != 128)
+    return fail(ISPA_ERR_UNSUPPORTED, "a prepared fp16 V is built for bf16 inputs with head_dim 128");
+  if (!(0 <= frame_begin && frame_begin <= frame_end && frame_end <= desc->kv_frames))
+    return fail(ISPA_ERR_INVALID_ARG, "frames [%d, %d) invalid for kv_frames %d", frame_begin, frame_end,
+                desc->kv_frames);
+  if (!ptr_ok(v) || !ptr_ok(v16)) return fail(ISPA_ERR_INVALID_ARG, "v and v16 must be 16-byte aligned device pointers");
+  const long long tpf = desc->tokens_per_frame;
+  const char *a = static_cast<const char *>(v), *b = static_cast<const char *>(v16);
+  const long long vb = (long long)desc->B * g.Lkv * desc->H * 128 * 2, v16b = (long long)v16_bytes(desc->B, desc->H, g.Lkv);
+  if (a < b + v16b && b < a + vb) return fail(ISPA_ERR_INVALID_ARG, "v16 must not overlap v");
+  return launch_v16_prepare(desc->B, desc->H, g.Lkv, (int)(frame_begin * tpf), (int)(frame_end * tpf), v, v16,
+                            (cudaStream_t)stream);
 }
 
 ispa_status ispa_lse_merge(int rows, int H, int head_dim, ispa_dtype o_dtype, const void *o_a, const float *lse_a,
@@ -342,7 +387,7 @@ size_t ispa_warmup_fused_workspace_bytes(const ispa_attn_desc *desc, int Dout) {
   if (!desc || Dout < 1 || attn_ranges(desc, &g, &scale) != ISPA_OK) return 0;
   const int T = desc->B * g.Lq, D = desc->H * desc->head_dim;
   return round256(stats_workspace_bytes(T, D, Dout, ISPA_PREC_TF32)) + round256((size_t)T * desc->H * 4) +
-         attn_tc_workspace_bytes(desc->B, desc->H, g.Lkv);
+         attn_tc_workspace_bytes(desc->B, desc->H, g.Lkv, desc->v_layout == ISPA_V_F16_PREPARED);
 }
 
 ispa_status ispa_warmup_fused(const ispa_attn_desc *desc, const void *q, const void *k, const void *v,
@@ -420,6 +465,22 @@ ispa_status ispa_ridge_solve_noalloc(int D, int Dout, const float *G, const floa
                       (cudaStream_t)stream);
 }
 
+size_t ispa_absorb_error_workspace_bytes(int D, int Dout) {
+  if (D < 1 || Dout < 1) return 0;
+  return absorb_error_workspace_bytes(D, Dout);
+}
+
+ispa_status ispa_absorb_error(int D, int Dout, const float *G, const float *C, const double *r2, const float *dW,
+                              double *eps, void *workspace, size_t workspace_bytes, ispa_stream_t stream) {
+  if (D < 1 || Dout < 1 || (long long)D * Dout > (1LL << 31)) return fail(ISPA_ERR_INVALID_ARG, "bad D, Dout");
+  if (!ptr_ok(G) || !ptr_ok(C) || !r2 || !ptr_ok(dW) || !eps)
+    return fail(ISPA_ERR_INVALID_ARG, "pointers must be non-NULL, matrices 16-byte aligned");
+  const size_t need = absorb_error_workspace_bytes(D, Dout);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return fail(ISPA_ERR_INVALID_ARG, "workspace needs %zu bytes (16-byte aligned)", need);
+  return launch_absorb_error(D, Dout, G, C, r2, dW, eps, workspace, (cudaStream_t)stream);
+}
+
 ispa_status ispa_select_layers(int N, const double *eps, int K, unsigned char *is_local, int *idx,
                                ispa_stream_t stream) {
   if (N < 0 || N > 4096 || K < 0 || K > N) return fail(ISPA_ERR_INVALID_ARG, "need 0 <= K <= N <= 4096");
@@ -445,7 +506,7 @@ size_t ispa_attn_local_proj_workspace_bytes(const ispa_attn_desc *desc) {
   const size_t a = (size_t)desc->B * g.Lq * desc->H * desc->head_dim * 2;
   const size_t l = (size_t)desc->B * g.Lq * desc->H * 4;
   return ((a + 255) & ~size_t(255)) + ((l + 255) & ~size_t(255)) +
-         attn_tc_workspace_bytes(desc->B, desc->H, g.Lkv);
+         attn_tc_workspace_bytes(desc->B, desc->H, g.Lkv, desc->v_layout == ISPA_V_F16_PREPARED);
 }
 
 ispa_status ispa_attn_local_proj(const ispa_attn_desc *desc, const void *q, const void *k, const void *v,

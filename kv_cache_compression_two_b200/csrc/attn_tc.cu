@@ -37,6 +37,8 @@
 //   * At the end of the local group the epilogue reads O after PV of that tile
 //     (o_done) and releases it (o_free) before the first history PV, which
 //     starts O afresh, is issued.
+#include <algorithm>
+
 #include "internal.h"
 
 namespace ispa {
@@ -190,6 +192,130 @@ __global__ void __launch_bounds__(256) v_fix_kernel(VPrep p, const __nv_bfloat16
       }
       *reinterpret_cast<uint4 *>(v16 + off) = make_uint4(o[0], o[1], o[2], o[3]);
     }
+}
+
+// ---------------------------------------------------------------------------
+// Prepared fp16 copy of V (ispa_v16_prepare): the same conversion, kept by the
+// caller across calls so that each call converts only the frames it writes.
+// Per (instance, head) the copy holds v * 2^e with one exponent e; its state
+// records e, 2^-e, the largest |v| and the sum of v^2 over the rows prepared so
+// far (and their count), by which the rule above picks e.  A prepare converts
+// its rows with the current e; when the new rows move a head's e, every row of
+// that head is converted again from v with the new one.
+// ---------------------------------------------------------------------------
+struct V16State {
+  float *unscale;      // 2^-e
+  int *expo;           // e
+  unsigned int *amax;  // largest |v| (bits of a non-negative float)
+  float *sumsq;        // sum of v^2
+  double *count;       // values accumulated
+  int *flag;           // 1: e changed in the last prepare, the head is converted again
+};
+
+__host__ __device__ inline size_t v16_a256(size_t x) { return (x + 255) & ~size_t(255); }
+
+V16State v16_state(void *v16, int B, int H, int Lkv) {
+  char *base = static_cast<char *>(v16) + v16_a256((size_t)B * Lkv * H * kD * 2);
+  const size_t w = v16_a256((size_t)B * H * 4);
+  V16State st;
+  st.unscale = reinterpret_cast<float *>(base);
+  st.expo = reinterpret_cast<int *>(base + w);
+  st.amax = reinterpret_cast<unsigned int *>(base + 2 * w);
+  st.sumsq = reinterpret_cast<float *>(base + 3 * w);
+  st.count = reinterpret_cast<double *>(base + 4 * w);
+  st.flag = reinterpret_cast<int *>(base + 4 * w + v16_a256((size_t)B * H * 8));
+  return st;
+}
+
+// Conversion of the prepared rows (thread layout of v_prep_kernel), scaled by
+// each head's current 2^e; the statistics are taken on the unscaled values.
+__global__ void __launch_bounds__(256) v16_prep_kernel(VPrep p, const __nv_bfloat16 *__restrict__ v, __half *v16,
+                                                       V16State st) {
+  const int D = p.H * kD;
+  const int vec_per_row = D / 8;
+  const int b = blockIdx.y;
+  const int lanes = gridDim.x * blockDim.x;
+  const int row_step = lanes / vec_per_row;
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+  const int c8 = tid % vec_per_row;
+  const int r0 = tid / vec_per_row;
+  const int hb = b * p.H + (c8 * 8) / kD;
+  const float scale = r0 < row_step ? ldexpf(1.f, st.expo[hb]) : 1.f;
+  float mx = 0.f, ss = 0.f;
+  if (r0 < row_step) {
+    for (int e = 0; e < p.n_ext; ++e)
+      for (int row = p.ext_begin[e] + r0; row < p.ext_end[e]; row += row_step) {
+        const long long off = ((long long)b * p.Lkv + row) * D + c8 * 8;
+        const uint4 in = __ldg(reinterpret_cast<const uint4 *>(v + off));
+        const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[j]));
+          mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+          ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+          const float lo = fminf(fmaxf(f.x * scale, -65504.f), 65504.f);
+          const float hi = fminf(fmaxf(f.y * scale, -65504.f), 65504.f);
+          __half2 hh = __floats2half2_rn(lo, hi);
+          o[j] = *reinterpret_cast<uint32_t *>(&hh);
+        }
+        *reinterpret_cast<uint4 *>(v16 + off) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+  }
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  }
+  if ((threadIdx.x & 15) == 0 && r0 < row_step) {
+    atomicMax(st.amax + hb, __float_as_uint(mx));
+    atomicAdd(st.sumsq + hb, ss);
+  }
+}
+
+// One thread per (instance, head): the exponent the rule picks for the rows
+// prepared so far; a change marks the head for conversion again.
+__global__ void __launch_bounds__(256) v16_decide_kernel(int BH, double added, V16State st) {
+  for (int hb = blockIdx.x * blockDim.x + threadIdx.x; hb < BH; hb += gridDim.x * blockDim.x) {
+    const double count = st.count[hb] + added;
+    st.count[hb] = count;
+    const int e = v_needs_scale(st.amax[hb], st.sumsq[hb], (float)count) ? v_exponent(st.amax[hb]) : 0;
+    st.flag[hb] = e != st.expo[hb] ? 1 : 0;
+    st.expo[hb] = e;
+    st.unscale[hb] = ldexpf(1.f, -e);
+  }
+}
+
+// Every row [0, Lkv) of the heads whose exponent changed, converted again.
+__global__ void __launch_bounds__(256) v16_reconvert_kernel(VPrep p, const __nv_bfloat16 *__restrict__ v, __half *v16,
+                                                            V16State st) {
+  const int D = p.H * kD;
+  const int vec_per_row = D / 8;
+  const int b = blockIdx.y;
+  const int lanes = gridDim.x * blockDim.x;
+  const int row_step = lanes / vec_per_row;
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+  const int c8 = tid % vec_per_row;
+  const int r0 = tid / vec_per_row;
+  if (r0 >= row_step) return;
+  const int hb = b * p.H + (c8 * 8) / kD;
+  if (!st.flag[hb]) return;
+  const float scale = ldexpf(1.f, st.expo[hb]);
+  for (int row = r0; row < p.Lkv; row += row_step) {
+    const long long off = ((long long)b * p.Lkv + row) * D + c8 * 8;
+    const uint4 in = *reinterpret_cast<const uint4 *>(v + off);
+    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[j]));
+      const float lo = fminf(fmaxf(f.x * scale, -65504.f), 65504.f);
+      const float hi = fminf(fmaxf(f.y * scale, -65504.f), 65504.f);
+      __half2 hh = __floats2half2_rn(lo, hi);
+      o[j] = *reinterpret_cast<uint32_t *>(&hh);
+    }
+    *reinterpret_cast<uint4 *>(v16 + off) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
 }
 
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
@@ -674,9 +800,55 @@ size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
-size_t attn_tc_workspace_bytes(int B, int H, int Lkv) {
+size_t attn_tc_workspace_bytes(int B, int H, int Lkv, bool v_prepared) {
+  if (v_prepared) return 0;
   return a256((size_t)B * Lkv * H * kD * 2) + 3 * a256((size_t)B * H * 4);
 }
+
+size_t v16_state_offset(int B, int H, int Lkv) { return a256((size_t)B * Lkv * H * kD * 2); }
+
+size_t v16_state_bytes(int B, int H) { return 4 * a256((size_t)B * H * 4) + a256((size_t)B * H * 8) + a256((size_t)B * H * 4); }
+
+size_t v16_bytes(int B, int H, int Lkv) { return v16_state_offset(B, H, Lkv) + v16_state_bytes(B, H); }
+
+ispa_status launch_v16_prepare(int B, int H, int Lkv, int row_begin, int row_end, const void *v, void *v16,
+                               cudaStream_t s) {
+  const int D = H * kD;
+  V16State st = v16_state(v16, B, H, Lkv);
+  cudaError_t e = cudaSuccess;
+  if (row_begin == 0) {  // a prepare from the first frame starts the copy afresh
+    e = cudaMemsetAsync(static_cast<char *>(v16) + v16_state_offset(B, H, Lkv), 0, v16_state_bytes(B, H), s);
+    if (e != cudaSuccess) return cuda_status(e, "prepared V state clear");
+  }
+  VPrep vp{};
+  vp.B = B;
+  vp.H = H;
+  vp.Lkv = Lkv;
+  vp.n_ext = 1;
+  vp.ext_begin[0] = row_begin;
+  vp.ext_end[0] = row_end;
+  const int vec_per_row = D / 8;
+  const __nv_bfloat16 *vb = static_cast<const __nv_bfloat16 *>(v);
+  __half *out = static_cast<__half *>(v16);
+  if (row_end > row_begin) {
+    const int rows = row_end - row_begin;
+    const int want = std::max(1, (int)(((long long)rows * vec_per_row + 255) / 256));
+    const int blocks = std::max((vec_per_row + 255) / 256, std::min(want, (sm_count() * 8 + B - 1) / B));
+    v16_prep_kernel<<<dim3(blocks, B), 256, 0, s>>>(vp, vb, out, st);
+    note_launch();
+  }
+  const int BH = B * H;
+  v16_decide_kernel<<<(BH + 255) / 256, 256, 0, s>>>(BH, (double)(row_end - row_begin) * kD, st);
+  const int fix_blocks = std::max((vec_per_row + 255) / 256, 2);
+  v16_reconvert_kernel<<<dim3(fix_blocks, B), 256, 0, s>>>(vp, vb, out, st);
+  note_launch(2);
+  return cuda_status(cudaGetLastError(), "prepared V launch");
+}
+
+ispa_status launch_prepared(const ispa_attn_desc &d, const GroupRanges &g, float scale, const void *q,
+                            const CUtensorMap &tk, const CUtensorMap &tv, AttnParams &P, void *o_loc, float *l_loc,
+                            void *o_hist, float *l_hist, void *o_full, float *l_full, cudaStream_t s,
+                            float *stats_dA);
 
 ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float scale, const void *q,
                            const void *k, const void *v, void *o_loc, float *l_loc, void *o_hist, float *l_hist,
@@ -687,6 +859,14 @@ ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float 
   if (st != ISPA_OK) return st;
   const int D = d.H * kD;
 
+  CUtensorMap tk, tv;
+  if ((st = map_kv16(&tk, k, D, g.Lkv, d.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) != ISPA_OK) return st;
+  if (d.v_layout == ISPA_V_F16_PREPARED) {
+    // the caller's prepared copy (ispa_v16_prepare) and its per-head 2^-e
+    P.v_unscale = v16_state(const_cast<void *>(v), d.B, d.H, g.Lkv).unscale;
+    if ((st = map_kv16(&tv, v, D, g.Lkv, d.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16)) != ISPA_OK) return st;
+    return launch_prepared(d, g, scale, q, tk, tv, P, o_loc, l_loc, o_hist, l_hist, o_full, l_full, s, stats_dA);
+  }
   // ---- fp16 copy of the V rows the tiles read (workspace)
   char *ws = static_cast<char *>(workspace);
   __half *v16 = reinterpret_cast<__half *>(ws);
@@ -718,10 +898,15 @@ ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float 
   note_launch(2);
   if ((st = cuda_status(cudaGetLastError(), "V conversion launch")) != ISPA_OK) return st;
   P.v_unscale = v_unscale;
-
-  CUtensorMap tk, tv;
-  if ((st = map_kv16(&tk, k, D, g.Lkv, d.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)) != ISPA_OK) return st;
   if ((st = map_kv16(&tv, v16, D, g.Lkv, d.B, CU_TENSOR_MAP_DATA_TYPE_FLOAT16)) != ISPA_OK) return st;
+  return launch_prepared(d, g, scale, q, tk, tv, P, o_loc, l_loc, o_hist, l_hist, o_full, l_full, s, stats_dA);
+}
+
+// The attention launch proper, once V is in fp16 (tv) with its unscale in P.
+ispa_status launch_prepared(const ispa_attn_desc &d, const GroupRanges &g, float scale, const void *q,
+                            const CUtensorMap &tk, const CUtensorMap &tv, AttnParams &P, void *o_loc, float *l_loc,
+                            void *o_hist, float *l_hist, void *o_full, float *l_full, cudaStream_t s,
+                            float *stats_dA) {
   P.H = d.H;
   P.Lq = g.Lq;
   P.q_tiles = (g.Lq + kTileQ - 1) / kTileQ;

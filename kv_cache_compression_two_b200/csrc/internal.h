@@ -59,8 +59,17 @@ ispa_status launch_absorb_weight(int D, int Dout, const void *W, ispa_dtype wdt,
 ispa_status launch_attn_simt(const ispa_attn_desc &d, const GroupRanges &g, float scale, const float *q,
                              const float *k, const float *v, void *o_loc, float *l_loc, void *o_hist,
                              float *l_hist, void *o_full, float *l_full, cudaStream_t s);
-// workspace: an fp16 copy of V (see attn_tc.cu) plus per-head scales
-size_t attn_tc_workspace_bytes(int B, int H, int Lkv);
+// workspace: an fp16 copy of V (see attn_tc.cu) plus per-head scales; none
+// when V comes prepared (ispa_v16_prepare)
+size_t attn_tc_workspace_bytes(int B, int H, int Lkv, bool v_prepared);
+// prepared fp16 V: B * Lkv * H * 128 fp16 values, then the per-head state
+size_t v16_bytes(int B, int H, int Lkv);
+size_t v16_state_offset(int B, int H, int Lkv);
+size_t v16_state_bytes(int B, int H);
+// converts rows [row_begin, row_end) of every instance (a prepare from row 0
+// clears the state first)
+ispa_status launch_v16_prepare(int B, int H, int Lkv, int row_begin, int row_end, const void *v, void *v16,
+                               cudaStream_t s);
 ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float scale, const void *q,
                            const void *k, const void *v, void *o_loc, float *l_loc, void *o_hist,
                            float *l_hist, void *o_full, float *l_full, void *workspace, cudaStream_t s,
@@ -81,6 +90,10 @@ size_t ridge_workspace_bytes(int D, int Dout);
 ispa_status launch_ridge(int D, int Dout, const float *G, const float *C, const double *r2, float lambda,
                          int lambda_relative, int refine_steps, float *dW, double *eps, void *ws,
                          cudaStream_t s);
+// epsilon of a given dW from statistics (ispa_absorb_error)
+size_t absorb_error_workspace_bytes(int D, int Dout);
+ispa_status launch_absorb_error(int D, int Dout, const float *G, const float *C, const double *r2, const float *dW,
+                                double *eps, void *ws, cudaStream_t s);
 // Device address of the static scratch array of ispa_ridge_solve_noalloc on the
 // current device, after checking that the workspace of a D x Dout solve fits it.
 ispa_status ridge_noalloc_scratch(int D, int Dout, void **out);

@@ -833,6 +833,44 @@ ispa_status apply_inverse(int D, int Dout, const Ws &w, const float *rhs, float 
 size_t ridge_workspace_bytes(int D, int Dout) { return carve_bytes(D, Dout, nullptr, nullptr); }
 
 // ---------------------------------------------------------------------------
+// epsilon of a given dW on statistics G, C, r2 (ispa_absorb_error): the same
+// fp64-accumulated reductions as the solve's epsilon.  Workspace: dW^T and
+// two accumulators.
+// ---------------------------------------------------------------------------
+size_t absorb_error_workspace_bytes(int D, int Dout) { return align256((size_t)Dout * D * sizeof(float)) + 256; }
+
+namespace {
+__global__ void eps_finalize_kernel(const double *__restrict__ r2, const double *__restrict__ acc, double *eps) {
+  *eps = *r2 - 2.0 * acc[0] + acc[1];
+}
+}  // namespace
+
+ispa_status launch_absorb_error(int D, int Dout, const float *G, const float *C, const double *r2, const float *dW,
+                                double *eps, void *ws, cudaStream_t s) {
+  float *dWt = static_cast<float *>(ws);
+  double *acc = reinterpret_cast<double *>(static_cast<char *>(ws) + align256((size_t)Dout * D * sizeof(float)));
+  cudaError_t e = cudaMemsetAsync(acc, 0, 2 * sizeof(double), s);
+  if (e != cudaSuccess) return cuda_status(e, "absorb error set-up");
+  const int grid = sm_count() * 4;
+  dot_kernel<<<grid, 256, 0, s>>>(D, Dout, Dout, dW, C, acc);
+  note_launch();
+  if (D % 4 == 0 && Dout % 4 == 0) {
+    transpose_kernel<<<dim3((Dout + 31) / 32, (D + 31) / 32), dim3(32, 8), 0, s>>>(D, Dout, dW, Dout, dWt, D);
+    note_launch();
+    const int tiles = (D + 127) / 128, upper_tiles = tiles * (tiles + 1) / 2;
+    const int nsplit = std::max(1, 2 * sm_count() / upper_tiles);
+    e = simt_gemm_nn128(D, D, Dout, dW, Dout, dWt, D, EpiSymDot{G, acc, D, 0.0}, s, nsplit, 1);
+  } else {
+    e = simt_gemm<OP_SYM_UPPER, OP_N, float, 0>(D, Dout, D, Operand{G, nullptr, D}, Operand{dW, nullptr, Dout},
+                                                EpiDotG{dW, acc, Dout, 0.0}, s);
+  }
+  if (e != cudaSuccess) return cuda_status(e, "absorb error G dW");
+  eps_finalize_kernel<<<1, 1, 0, s>>>(r2, acc, eps);
+  note_launch();
+  return cuda_status(cudaGetLastError(), "absorb error launch");
+}
+
+// ---------------------------------------------------------------------------
 // Allocation-free variant (ispa_ridge_solve_noalloc).  Its scratch -- the
 // working copy of the factorisation, the refinement residual and a few
 // accumulators -- lives in this file-scope device array instead of a

@@ -46,9 +46,15 @@ def rng(*key) -> np.random.Generator:
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round float32 values to bf16 (round to nearest, ties to even); returns uint16 bits."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    bias = ((u >> 16) & 1) + 0x7FFF
-    out = ((u + bias) >> 16).astype(np.uint16)
+    u = x.view(np.uint32)
+    # u + 0x7FFF + (bit 16 of u), in place in one uint32 temporary: only NaN
+    # patterns (overwritten below) can carry out of 32 bits
+    r = u >> 16
+    r &= 1
+    r += 0x7FFF
+    r += u
+    r >>= 16
+    out = r.astype(np.uint16)
     nan = np.isnan(x)
     if nan.any():
         out[nan] = 0x7FC0
@@ -271,3 +277,53 @@ def activation_rows(M: int, K: int, key: Iterable) -> np.ndarray:
         x[1] = 0.0
         x[1, K // 3] = -3.0
     return round_to_bf16(x)
+
+
+# ---------------------------------------------------------------------------
+# device-side draws of the same recipes (timing runs only: the values come
+# from torch's generator, not from the PCG64 streams above, so no oracle
+# comparison uses them)
+# ---------------------------------------------------------------------------
+def torch_generator(device, *key):
+    """A torch generator on `device` seeded from ROOT_SEED and a key tuple."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(np.random.SeedSequence([ROOT_SEED] + [_key_int(k) for k in key]).generate_state(1)[0]))
+    return g
+
+
+def device_normal_bf16(shape, device, gen, std: float = 1.0):
+    """N(0, std^2) draws in fp32 on the device, rounded to bf16."""
+    import torch
+    x = torch.randn(shape, device=device, dtype=torch.float32, generator=gen)
+    if std != 1.0:
+        x.mul_(std)
+    return x.to(torch.bfloat16)
+
+
+def drift_layer_kv_device(shape: AttnShape, layer: int, key: Iterable, device):
+    """The drift history recipe of :func:`drift_layer_kv` drawn on the device:
+    K, V [B, hist_end*tpf, H, d] in bf16 (sink frames, then every history frame
+    as its base sink frame plus alpha (j/Hf) X U Vr^T and N(0, 0.1^2) noise)."""
+    import torch
+    key = tuple(key)
+    S, Hf, tpf, d, H = shape.sink_frames, shape.hist_end - shape.hist_begin, shape.tpf, shape.d, shape.H
+    alpha = float(rng(*key, "alpha", layer).uniform(0.5, 2.0))
+    out = {}
+    for name in ("k", "v"):
+        g = torch_generator(device, *key, "drift", layer, name)
+        sink = torch.randn((shape.B, S * tpf, H, d), device=device, dtype=torch.float32, generator=g)
+        U = torch.randn((H, d, 64), device=device, generator=g) / math.sqrt(d)
+        Vr = torch.randn((H, d, 64), device=device, generator=g) / math.sqrt(d)
+        P = torch.matmul(U, Vr.transpose(1, 2))                      # [H, d, d]
+        buf = torch.empty((shape.B, (S + Hf) * tpf, H, d), device=device, dtype=torch.bfloat16)
+        buf[:, :S * tpf] = sink.to(torch.bfloat16)
+        for j in range(1, Hf + 1):
+            b = (j - 1) % S
+            base = sink[:, b * tpf:(b + 1) * tpf]                     # [B, tpf, H, d]
+            drift = torch.einsum("bthd,hde->bthe", base, P)
+            noise = torch.randn(base.shape, device=device, generator=g) * 0.1
+            buf[:, (S + j - 1) * tpf:(S + j) * tpf] = (base + (alpha * j / Hf) * drift + noise).to(torch.bfloat16)
+        out[name] = buf
+    out["alpha"] = alpha
+    return out

@@ -73,3 +73,21 @@ def test_oracle_sample_work_scales_to_the_step():
     w = bench.step_work(sh)
     assert abs(bench.sample_work(sh.B * sh.Lq) - w["total"]) <= 1e-9 * w["total"]
     assert abs(bench.sample_work(0) - w["solve"]) <= 1e-9 * w["solve"]
+
+
+def test_sweep_kv_retained_matches_the_oracle_accounting():
+    # every sweep point: the bytes the bench reports as kept equal the oracle's
+    # retained fraction 1 - (K/N) h, with K = floor(x N) and h the history share of the keys
+    for name, H, N in bench.SWEEP_SHAPES:
+        for B in (1, 2):
+            for Hf in bench.SWEEP_HIST:
+                sh = si.video_shape(H, Hf, B=B)
+                h_frac = len(sh.hist_rows) / sh.Lkv
+                for x in bench.SWEEP_X:
+                    kv = bench.kv_retained(sh, B, N, x)
+                    K = orc.num_selected(x, N)
+                    assert kv["l_layers"] == K
+                    assert abs(kv["fraction"] - orc.kv_retained_fraction(K / N, h_frac)) < 1e-12
+                    assert kv["kv_bytes_full"] == B * N * sh.Lkv * sh.D * 4
+    # the 30-layer 1.3B model at ISPA-0.5 keeps 64.3 % of its KV
+    assert abs(bench.kv_retained(si.SHAPE_1P3B, 1, 30, 0.5)["fraction"] - 0.6428571428) < 1e-9

@@ -496,3 +496,30 @@ def test_attn_local_proj_q8(fmt, ofmt):
     # and the W8A8 step stays near the bf16 step (quantisation error of a few percent)
     ref16 = orc.local_projection(sh, data["q"], data["k"], data["v"], Wn)
     assert rel_fro(got, ref16) <= 6e-2, rel_fro(got, ref16)
+
+
+# ---------------------------------------------------------------- epsilon of a given correction
+@pytest.mark.parametrize("D,Dout", [(64, 64), (256, 136), (1536, 1536), (333, 77)])
+def test_absorb_error_matches_oracle(D, Dout):
+    """ispa_absorb_error on statistics of other rows than the solve's (the held-out
+    error after the switch): against the oracle's epsilon from the same statistics,
+    and against the direct form on the rows themselves."""
+    g = np.random.default_rng(D * 7 + Dout)
+    T = 2 * D
+    A_loc = g.standard_normal((T, D)).astype(np.float32)
+    A_full = (A_loc + 0.3 * g.standard_normal((T, D))).astype(np.float32)
+    W = (g.standard_normal((D, Dout)) / math.sqrt(D)).astype(np.float32)
+    dW = (0.05 * g.standard_normal((D, Dout))).astype(np.float32)
+    G, C, r2 = orc.absorption_stats(A_loc, A_full, W)
+    G32, C32 = G.astype(np.float32), C.astype(np.float32)
+    eps = torch.zeros(1, dtype=torch.float64, device="cuda")
+    ws = torch.empty(ispa.ispa_absorb_error_workspace_bytes(D, Dout), dtype=torch.uint8, device="cuda")
+    ispa.ispa_absorb_error(D, Dout, dev(np.triu(G32)), dev(C32), dev(np.array([r2]), torch.float64), dev(dW), eps, ws)
+    ispa.ispa_check_device_error()
+    got = float(eps.item())
+    ref = orc.eps_from_stats(G32.astype(np.float64), C32.astype(np.float64), r2, dW.astype(np.float64))
+    t = abs(float(np.sum(dW.astype(np.float64) * C32)))
+    qd = abs(float(np.sum(dW.astype(np.float64) * (G32.astype(np.float64) @ dW))))
+    assert abs(got - ref) <= 1e-5 * (r2 + 2 * t + qd), (got, ref)
+    direct = orc.eps_direct(A_loc, A_full, W, dW)
+    assert abs(got - direct) <= 1e-5 * (r2 + 2 * t + qd) + 1e-6 * direct, (got, direct)
