@@ -88,8 +88,12 @@ def _check_rows(sh, q_np, k_np, v_np, o, l, rows):
 def test_14b_layer_attention_statistics_and_solve():
     """40 heads x 128 (D = 5120), 1560 tokens per frame, sink 3 + history 60 + chunk 3
     (4680 queries over 102 960 keys, 1480 query tiles).  Attention on sampled rows x all
-    heads x all keys; G, C, r2 of the chunk against the fp64 statistics of the GPU's
-    own rows; the full 5120 x 5120 solve (plain and refined) against the oracle's."""
+    heads x all keys; G, C, r2 of the first chunk against the fp64 statistics of the
+    GPU's own rows; after all 8 warmup chunks (T = 37 440 rows) the full 5120 x 5120
+    solve (plain and refined) against the oracle's solve of the GPU's statistics.
+    (One chunk alone has fewer rows than dimensions: its G is singular, and the tf32
+    statistics' rounding, about 1e-3 of G, then outweighs lambda = 1e-4 tr(G) / D on
+    the null space, so G + lambda I is indefinite -- in fp64 as well.)"""
     sh = si.SHAPE_14B
     key = ("gpu", "cfg4")
     prefix = si.drift_layer_kv(sh, "bf16", 0, key)
@@ -116,17 +120,26 @@ def test_14b_layer_attention_statistics_and_solve():
     ws = torch.empty(ispa.ispa_accum_stats_workspace_bytes(T, D, D), dtype=torch.uint8, device="cuda")
     a_loc, a_full = o["loc"].reshape(T, D), o["full"].reshape(T, D)
     ispa.ispa_accum_stats(T, D, D, a_loc, a_full, Wd, G, C, r2, ispa.ISPA_PREC_TF32, ws)
-    del ws
     Gr, Cr, r2r = orc.absorption_stats(host(a_loc), host(a_full), W)
     Gh, Ch = host(G), host(C)
     iu = np.triu_indices(D)
     assert rel_fro(Gh[iu], Gr[iu]) <= 1e-3, rel_fro(Gh[iu], Gr[iu])
     assert rel_fro(Ch, Cr) <= 1e-3, rel_fro(Ch, Cr)
     assert abs(float(r2.item()) - r2r) <= 1e-3 * r2r
-    del o, l, Gr, Cr
+    del o, l, Gr, Cr, Gh, Ch
+    # the other seven warmup chunks of the layer: written into the cache, attended, accumulated
+    for c in range(1, 8):
+        cq = si.chunk_qkv(sh, "bf16", 0, c, key)
+        cache.write_chunk(cq)
+        o, l = cache.attend(dev(cq["q"], torch.bfloat16))
+        ispa.ispa_accum_stats(T, D, D, o["loc"].reshape(T, D), o["full"].reshape(T, D), Wd, G, C, r2,
+                              ispa.ISPA_PREC_TF32, ws)
+        del o, l
+    ispa.ispa_check_device_error()
+    del ws, cache
+    Gh, Ch = host(G), host(C)
 
-    # the 5120 x 5120 solve from the GPU's statistics (fewer rows than dimensions:
-    # G is rank-deficient, lambda = 1e-4 tr(G) / D sets the conditioning)
+    # the 5120 x 5120 solve from the GPU's statistics of the 8 chunks (37 440 rows)
     Gs = _sym(Gh.astype(np.float32).astype(np.float64))
     Cs = Ch.astype(np.float32).astype(np.float64)
     lam32 = float(np.float32(orc.ridge_lambda(Gs, LAMBDA_REL, True)))

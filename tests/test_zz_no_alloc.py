@@ -73,9 +73,13 @@ def test_noalloc_matches_oracle_and_workspace_solve_on_two_calls_in_a_row():
         n2 = float(np.sum(ref * ref))
         bound = 1e-6 * r2 + 2.0 * lam32 * tol * n2 + np.linalg.norm(Gs, 2) * tol ** 2 * n2
         assert abs(eps[1] - ref_eps) <= bound, (eps[1], ref_eps, bound)
-        # and the same arithmetic as the workspace form: the scratch layout is the workspace's
-        assert np.linalg.norm(got - dW_ws) / np.linalg.norm(dW_ws) <= 1e-6
-        assert abs(eps[1] - eps[0]) <= 1e-9 * r2
+        # and the same arithmetic as the workspace form (the scratch layout is the workspace's;
+        # the two differ only by the order of the solve products' atomic additions), epsilon
+        # within the quadratic form's bound for that difference
+        rho = np.linalg.norm(got - dW_ws) / np.linalg.norm(dW_ws)
+        assert rho <= 1e-6, rho
+        n2w = float(np.sum(dW_ws * dW_ws))
+        assert abs(eps[1] - eps[0]) <= 1e-6 * r2 + 2.0 * lam32 * rho * n2w + np.linalg.norm(Gs, 2) * rho ** 2 * n2w
 
 
 def test_noalloc_allocates_no_device_memory():
