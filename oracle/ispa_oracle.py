@@ -464,3 +464,127 @@ def local_projection_q8(shape, q, k, v, W_new: np.ndarray, fmt: int, scale: floa
     qa, sa = quantize_rows(A, fmt)
     qw, sw = quantize_cols(W_new, fmt)
     return np.asarray(gemm_q8(qa, sa, qw, sw, fmt)).reshape(B, Lq, -1)
+
+
+# ---------------------------------------------------------------------------
+# FP8 post-switch attention: the W8A8 combination carried into the attention
+# products (QK^T and PV in fp8 e4m3).  The pages report ISPA combined with
+# post-training 8-bit quantisation [EN-notes, Key Findings (Figure 7);
+# DE-summary 4, "Beschleunigung"] and give no scheme for the attention.
+# Reading taken:
+#  * Q, K, V: one fp32 scale per (instance, head) over that head's rows,
+#    s = amax / 448, codes e4m3(x * (448 / amax)) -- the row quantiser above
+#    applied to the head's values as one row;
+#  * scores in log2 units t = (q8 . k8) s_q s_k scale log2(e);
+#  * each group is taken in blocks of 128 keys in its order (the local group's
+#    sink range, then its current range; the history range), the blocks of a
+#    range starting at the 16-aligned key position at or below its first key; a
+#    running maximum m over the blocks seen so far (the product and the sum are
+#    scaled by 2^(m_old - m_new) when it grows); per block p = 2^(t - m + 8), so
+#    that p <= 256 and the weights of the bulk of the keys lie in e4m3's normal
+#    range; the sum l += p is kept exactly, the product acc += e4m3(p) v8;
+#  * O = acc s_v / l, L = (m - 8 + log2 l) ln 2; the two groups are merged by
+#    their log-sum-exp as in lse_merge.
+# ---------------------------------------------------------------------------
+FP8_BLOCK, FP8_ALIGN, FP8_P_OFFSET = 128, 16, 8.0
+
+
+def quantize_heads(x: np.ndarray):
+    """Per (instance, head) e4m3 quantisation of x [B, n, H, d].
+
+    Returns (codes as float64 values [B, n, H, d], s [B, H] fp32); each head's
+    n x d values are quantised as one row by :func:`quantize_rows`.
+    """
+    B, n, H, d = x.shape
+    q = np.empty(x.shape)
+    s = np.empty((B, H), np.float32)
+    for b in range(B):
+        for h in range(H):
+            qq, ss = quantize_rows(np.asarray(x[b, :, h, :], np.float32).reshape(1, n * d), Q8_E4M3)
+            q[b, :, h, :] = qq.reshape(n, d)
+            s[b, h] = ss[0]
+    return q, s
+
+
+def _runs(rows: np.ndarray):
+    """Contiguous [lo, hi) runs of a sorted index array."""
+    out = []
+    for r in rows:
+        if out and out[-1][1] == r:
+            out[-1][1] = r + 1
+        else:
+            out.append([int(r), int(r) + 1])
+    return [tuple(x) for x in out]
+
+
+def fp8_blocks(ranges) -> List[Tuple[int, int]]:
+    """The blocks of a group: for each key range [lo, hi) in order, windows of
+    FP8_BLOCK keys starting at lo rounded down to FP8_ALIGN; each block is
+    returned as the [first, end) of its keys that belong to the range."""
+    out = []
+    for lo, hi in ranges:
+        w = lo - lo % FP8_ALIGN
+        while w < hi:
+            out.append((max(w, lo), min(w + FP8_BLOCK, hi)))
+            w += FP8_BLOCK
+    return out
+
+
+def attend_group_fp8(t: np.ndarray, v8: np.ndarray, blocks, quantize_p: bool = True):
+    """Blockwise softmax of one group with e4m3 weights (see the reading above).
+
+    t [n, Lkv] scores in log2 units (columns outside the group unused), v8
+    [Lkv, d] dequantisation-free e4m3 codes of V, blocks from :func:`fp8_blocks`.
+    Returns (acc / l [n, d] before the V scale, L in natural log [n]).
+    quantize_p=False keeps the weights exact (the plain online softmax).
+    """
+    n, d = t.shape[0], v8.shape[1]
+    if not blocks:
+        return np.zeros((n, d)), np.full(n, NEG_INF)
+    m = np.full(n, NEG_INF)
+    l = np.zeros(n)
+    acc = np.zeros((n, d))
+    for lo, hi in blocks:
+        tb = t[:, lo:hi]
+        m_new = np.maximum(m, tb.max(axis=1))
+        f = np.where(np.isneginf(m), 0.0, np.exp2(m - m_new))
+        acc *= f[:, None]
+        l *= f
+        m = m_new
+        p = np.exp2(tb - m[:, None] + FP8_P_OFFSET)
+        l += p.sum(axis=1)
+        acc += (e4m3_round(p) if quantize_p else p) @ v8[lo:hi]
+    return acc / l[:, None], (m - FP8_P_OFFSET + np.log2(l)) * math.log(2.0)
+
+
+def split_attention_fp8(shape, q, k, v, scale: float = None, rows: Sequence[int] = None,
+                        quantize_p: bool = True) -> Dict[str, np.ndarray]:
+    """Two-group attention with fp8 e4m3 products (reading above); same outputs
+    as :func:`split_attention`.  q, k, v hold the unquantised (bf16) values; the
+    per-head quantisation is part of the definition."""
+    d = q.shape[-1]
+    scale = 1.0 / math.sqrt(d) if not scale else scale
+    B, Lq, H, _ = q.shape
+    rows = np.arange(Lq) if rows is None else np.asarray(rows)
+    n = len(rows)
+    q8, sq = quantize_heads(q)
+    k8, sk = quantize_heads(k)
+    v8, sv = quantize_heads(v)
+    blk_loc = fp8_blocks(_runs(_local_rows(shape)))
+    blk_hist = fp8_blocks(_runs(_hist_rows(shape)))
+    out = {key: np.zeros((B, n, H, d)) for key in ("O_loc", "O_hist", "O_full")}
+    out.update({key: np.zeros((B, n, H)) for key in ("L_loc", "L_hist", "L_full")})
+    log2e = 1.0 / math.log(2.0)
+    for b in range(B):
+        for h in range(H):
+            c = float(sq[b, h]) * float(sk[b, h]) * scale * log2e
+            t = (q8[b, rows, h, :] @ k8[b, :, h, :].T) * c          # [n, Lkv]
+            res = {}
+            for name, blk in (("loc", blk_loc), ("hist", blk_hist)):
+                o, L = attend_group_fp8(t, v8[b, :, h, :], blk, quantize_p)
+                res[name] = (o * float(sv[b, h]), L)
+            o_f, l_f = lse_merge(res["loc"][0], res["loc"][1], res["hist"][0], res["hist"][1])
+            for name in ("loc", "hist"):
+                out["O_" + name][b, :, h], out["L_" + name][b, :, h] = res[name]
+            out["O_full"][b, :, h], out["L_full"][b, :, h] = o_f, l_f
+    return out

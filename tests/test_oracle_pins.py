@@ -778,3 +778,143 @@ def test_quantize_rows_commutes_with_power_of_two_scaling(seed, k, fmt):
     q2, s2 = orc.quantize_rows((x * np.float32(2.0 ** k)).astype(np.float32), fmt)
     assert np.array_equal(q1, q2)
     assert np.array_equal(s2, (s1 * np.float32(2.0 ** k)).astype(np.float32))
+
+
+# ---------------------------------------------------------------------------
+# FP8 attention (the 8-bit reading of the post-switch attention)
+# ---------------------------------------------------------------------------
+FP8_LAYOUTS = [
+    si.AttnShape(B=1, H=2, d=64, tpf=37, sink_frames=1, hist_begin=1, hist_end=5, cur_begin=5, cur_end=6, kv_frames=6),
+    si.AttnShape(B=2, H=1, d=32, tpf=50, sink_frames=2, hist_begin=2, hist_end=2, cur_begin=2, cur_end=4, kv_frames=4),
+    si.AttnShape(B=1, H=1, d=32, tpf=200, sink_frames=2, hist_begin=2, hist_end=2, cur_begin=0, cur_end=2, kv_frames=2),
+    si.AttnShape(B=1, H=1, d=16, tpf=9, sink_frames=1, hist_begin=1, hist_end=30, cur_begin=30, cur_end=33,
+                 kv_frames=33),
+]
+
+
+def _dequantised(data):
+    out = {}
+    for n in ("q", "k", "v"):
+        c, s = orc.quantize_heads(data[n])
+        out[n] = c * s.astype(np.float64)[:, None, :, None]
+    return out
+
+
+def check_fp8_online_softmax(fn) -> bool:
+    """With the weights kept exact, the blockwise algorithm is softmax attention of
+    the dequantised Q, K, V (online softmax is exact whatever the blocks)."""
+    ok = True
+    for i, sh in enumerate(FP8_LAYOUTS):
+        data = si.iid_qkv(sh, "bf16", ("pin", "fp8", i))
+        got = fn(sh, data["q"], data["k"], data["v"], quantize_p=False)
+        dq = _dequantised(data)
+        ref = orc.split_attention(sh, dq["q"], dq["k"], dq["v"])
+        for n in ("loc", "hist", "full"):
+            ok &= np.allclose(got["O_" + n], ref["O_" + n], rtol=0, atol=1e-12)
+            fin = np.isfinite(ref["L_" + n])
+            ok &= np.array_equal(fin, np.isfinite(got["L_" + n]))
+            ok &= np.allclose(got["L_" + n][fin], ref["L_" + n][fin], rtol=0, atol=1e-12)
+    return bool(ok)
+
+
+def test_fp8_attention_without_weight_rounding_is_softmax_of_the_dequantised_inputs():
+    assert check_fp8_online_softmax(orc.split_attention_fp8)
+
+
+def test_fp8_quantize_heads_is_the_row_quantiser_per_head():
+    x = si.round_to_bf16(si.rng("pin", "qh").standard_normal((2, 33, 3, 16)).astype(np.float32) *
+                         np.array([1.0, 100.0, 1e-3], np.float32)[None, None, :, None])
+    q, s = orc.quantize_heads(x)
+    for b in range(2):
+        for h in range(3):
+            amax = np.float32(np.abs(x[b, :, h]).max())
+            assert s[b, h] == np.float32(amax / np.float32(448.0))
+            assert np.abs(q[b, :, h]).max() == 448.0
+            assert np.array_equal(orc.e4m3_round(q[b, :, h]), q[b, :, h])   # codes on the e4m3 grid
+
+
+def test_fp8_blocks_cover_each_range_in_aligned_128_key_windows():
+    g = np.random.default_rng(5)
+    for _ in range(200):
+        lo = int(g.integers(0, 3000))
+        hi = lo + int(g.integers(1, 1500))
+        lo2 = hi + int(g.integers(0, 300))
+        hi2 = lo2 + int(g.integers(0, 700))
+        ranges = [(lo, hi)] + ([(lo2, hi2)] if hi2 > lo2 else [])
+        blocks = orc.fp8_blocks(ranges)
+        keys = [k for a, b in blocks for k in range(a, b)]
+        assert keys == [k for a, b in ranges for k in range(a, b)]          # every key once, in order
+        for a, b in blocks:
+            w0 = next(r0 - r0 % 16 + 128 * ((a - (r0 - r0 % 16)) // 128) for r0, r1 in ranges if r0 <= a < r1)
+            assert w0 % 16 == 0 and w0 <= a < b <= w0 + 128                # inside one aligned window
+
+
+def test_fp8_weights_on_the_e4m3_grid_pass_exactly():
+    """p = 2^(t - m + 8): weights 2^0 .. 2^-14 relative to the maximum are e4m3 normals
+    after the offset; a weight of 1.125 * 2^-7 (2.25 after it) enters exactly."""
+    v8 = np.array([[1.0, -2.0], [3.0, 0.5]])
+    t = np.array([[0.0, math.log2(1.125 * 2.0 ** -7)]])
+    o, L = orc.attend_group_fp8(t, v8, [(0, 2)])
+    w = np.array([256.0, 2.25])
+    assert np.allclose(o[0], (w @ v8) / w.sum(), rtol=0, atol=1e-15)
+    assert abs(L[0] - math.log(1.0 + 1.125 * 2.0 ** -7)) < 1e-15
+
+
+def test_fp8_weight_rounding_stays_within_its_bound():
+    """With e4m3 weights the output moves by at most 2^-4 of sum_j w_j |v_j| (normal
+    weights) plus 2^-10 per subnormal weight over l >= 2^8; L is unchanged (the
+    normaliser keeps the exact weights); and the rounding is really applied."""
+    for i, sh in enumerate(FP8_LAYOUTS):
+        data = si.iid_qkv(sh, "bf16", ("pin", "fp8b", i))
+        got = orc.split_attention_fp8(sh, data["q"], data["k"], data["v"])
+        exact = orc.split_attention_fp8(sh, data["q"], data["k"], data["v"], quantize_p=False)
+        dq = _dequantised(data)
+        moved = 0.0
+        for name, rows in (("loc", orc._local_rows(sh)), ("hist", orc._hist_rows(sh))):
+            if len(rows) == 0:
+                continue
+            for b in range(sh.B):
+                for h in range(sh.H):
+                    s = (dq["q"][b, :, h] @ dq["k"][b, rows, h].T) / math.sqrt(sh.d)
+                    w = np.exp(s - s.max(axis=1, keepdims=True))
+                    w /= w.sum(axis=1, keepdims=True)
+                    av = np.abs(dq["v"][b, rows, h])
+                    bound = 2.0 ** -4 * (w @ av) + 2.0 ** -18 * av.sum(axis=0)[None, :] + 1e-12
+                    err = np.abs(got["O_" + name][b, :, h] - exact["O_" + name][b, :, h])
+                    assert np.all(err <= bound), (i, name, float((err - bound).max()))
+                    moved = max(moved, float(err.max()))
+            fin = np.isfinite(exact["L_" + name])
+            assert np.allclose(got["L_" + name][fin], exact["L_" + name][fin], rtol=0, atol=1e-12)
+        assert moved > 1e-6
+
+
+def test_mutant_fp8_without_the_weight_offset_is_caught():
+    def no_offset(t, v8, blocks, quantize_p=True):
+        n, d = t.shape[0], v8.shape[1]
+        m, l, acc = np.full(n, -np.inf), np.zeros(n), np.zeros((n, d))
+        for lo, hi in blocks:
+            tb = t[:, lo:hi]
+            m_new = np.maximum(m, tb.max(axis=1))
+            f = np.where(np.isneginf(m), 0.0, np.exp2(m - m_new))
+            acc, l, m = acc * f[:, None], l * f, m_new
+            p = np.exp2(tb - m[:, None])
+            l += p.sum(axis=1)
+            acc += orc.e4m3_round(p) @ v8[lo:hi]
+        return acc / l[:, None], (m + np.log2(l)) * math.log(2.0)
+    v8 = np.array([[1.0, -2.0], [3.0, 0.5]])
+    t = np.array([[0.0, math.log2(1.125 * 2.0 ** -7)]])
+    o, _ = no_offset(t, v8, [(0, 2)])
+    w = np.array([256.0, 2.25])
+    assert not np.allclose(o[0], (w @ v8) / w.sum(), rtol=0, atol=1e-15)
+
+
+def test_mutant_fp8_v_dequantised_with_the_k_scale_is_caught():
+    def wrong_v_scale(shape, q, k, v, scale=None, rows=None, quantize_p=True):
+        out = orc.split_attention_fp8(shape, q, k, v, scale, rows, quantize_p)
+        _, sk = orc.quantize_heads(k)
+        _, sv = orc.quantize_heads(v)
+        f = (sk.astype(np.float64) / sv.astype(np.float64))[:, None, :, None]
+        for n in ("loc", "hist", "full"):
+            out["O_" + n] = out["O_" + n] * f
+        return out
+    assert not check_fp8_online_softmax(wrong_v_scale)
