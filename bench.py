@@ -740,6 +740,56 @@ def cfg3_component(ispa, torch, stream, dev, n_layers: int = 30, warm_chunks: in
             "kv_retained": kv_retained(sh, B, n_layers, x)}
 
 
+def fp8_component(ispa, torch, stream, dev, layers, W_new, W16, D):
+    """The post-switch layers with fp8 e4m3 attention (prepared fp8 K/V) against the
+    bf16 ones on the same buffers: attention + bf16 projection, attention + W8A8
+    projection, the per-chunk prepare, and the output's distance from the bf16 step."""
+    out = {}
+    qT = torch.empty((D, D), device=dev, dtype=torch.uint8)
+    sw = torch.empty(D, device=dev, dtype=torch.float32)
+    for name, Lr, W in (("l_layer", layers[1], W_new), ("f_layer", layers[2], W16)):
+        d_ = Lr.desc
+        p16 = ispa.prepared(d_)
+        p8 = ispa.prepared(d_, ispa.ISPA_KV_E4M3_PREPARED)
+        kv8 = torch.empty(ispa.ispa_kv8_bytes(d_), device=dev, dtype=torch.uint8)
+        ispa.ispa_kv8_prepare(d_, Lr.dev["k"], Lr.dev["v"], 0, d_.kv_frames, kv8, stream=stream)
+        ispa.ispa_quantize_weight(D, D, W, ispa.ISPA_Q8_E4M3, qT, sw, stream=stream)
+        B, Lq = Lr.dev["q"].shape[0], Lr.dev["q"].shape[1]
+        y16 = torch.empty((B, Lq, D), device=dev, dtype=torch.bfloat16)
+        y8 = torch.empty_like(y16)
+        ws = torch.empty(max(ispa.ispa_attn_local_proj_q8_workspace_bytes(p8),
+                             ispa.ispa_attn_local_proj_workspace_bytes(p16), 16), device=dev, dtype=torch.uint8)
+        q = Lr.dev["q"]
+
+        def bf16():
+            ispa.ispa_attn_local_proj(p16, q, Lr.dev["k"], Lr.dev["v16"], W, D, y16, ispa.ISPA_BF16, ws, stream=stream)
+
+        def fp8():
+            ispa.ispa_attn_local_proj(p8, q, kv8, None, W, D, y8, ispa.ISPA_BF16, ws, stream=stream)
+
+        def fp8_w8a8():
+            ispa.ispa_attn_local_proj_q8(p8, q, kv8, None, qT, sw, ispa.ISPA_Q8_E4M3, D, y8, ispa.ISPA_BF16, ws,
+                                         stream=stream)
+
+        r = {"bf16_ms": graph_time(torch, stream, dev, bf16, 5), "fp8_attn_ms": graph_time(torch, stream, dev, fp8, 5),
+             "fp8_attn_w8a8_ms": graph_time(torch, stream, dev, fp8_w8a8, 5),
+             "kv8_prepare_chunk_ms": graph_time(torch, stream, dev, lambda: ispa.ispa_kv8_prepare(
+                 d_, Lr.dev["k"], Lr.dev["v"], d_.cur_begin, d_.cur_end, kv8, stream=stream), 5)}
+        bf16()
+        fp8()
+        torch.cuda.synchronize(dev)
+        r["rel_diff_fp8_attn_vs_bf16"] = float((y8.float() - y16.float()).norm() / y16.float().norm())
+        r["speedup_fp8_attn"] = r["bf16_ms"] / r["fp8_attn_ms"]
+        r["speedup_fp8_attn_w8a8"] = r["bf16_ms"] / r["fp8_attn_w8a8_ms"]
+        n_keys = (len(si.AttnShape(B, d_.H, 128, d_.tokens_per_frame, d_.sink_frames, d_.hist_begin, d_.hist_end,
+                                   d_.cur_begin, d_.cur_end, d_.kv_frames).local_rows))
+        r["attn_tflops_fp8"] = 4.0 * B * Lq * n_keys * d_.H * 128 / (r["fp8_attn_ms"] * 1e-3) / 1e12
+        out[name] = r
+        del kv8
+    ispa.ispa_check_device_error(stream)
+    return out
+
+
 def run_ours(args, world, rank, local):
     import torch
 
@@ -1058,6 +1108,7 @@ def run_ours(args, world, rank, local):
                     pass
                 print(f"component {name} failed: {exc}", file=sys.stderr, flush=True)
 
+        run_component("fp8_post_switch", lambda: fp8_component(ispa, torch, stream, dev, layers, W_new, W16, D))
         run_component("cfg4_14b_layer", lambda: cfg4_component(ispa, torch, stream, dev))
         run_component("cfg3_1p3b_model", lambda: cfg3_component(ispa, torch, stream, dev))
         solve14 = workloads["cfg4_14b_layer"].get("solve_ms_per_layer")

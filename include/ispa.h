@@ -122,7 +122,8 @@ ispa_status ispa_selftest_wait_timeout(long long wait_ns, ispa_stream_t stream);
 typedef enum {
   ISPA_V_PLAIN = 0,       /* V in in_dtype, [B, kv_frames*tpf, H, d]; a bf16 call
                              converts the rows it reads into its workspace       */
-  ISPA_V_F16_PREPARED = 1 /* a prepared fp16 copy of a bf16 V (ispa_v16_prepare) */
+  ISPA_V_F16_PREPARED = 1, /* a prepared fp16 copy of a bf16 V (ispa_v16_prepare) */
+  ISPA_KV_E4M3_PREPARED = 2 /* k: a prepared fp8 K and V (ispa_kv8_prepare); v unused */
 } ispa_v_layout;
 
 typedef struct {
@@ -137,7 +138,7 @@ typedef struct {
   ispa_dtype in_dtype;  /* dtype of Q, K, V                                     */
   ispa_dtype out_dtype; /* dtype of the O outputs                               */
   float softmax_scale;  /* <= 0 selects 1/sqrt(head_dim)                        */
-  ispa_v_layout v_layout; /* ISPA_V_PLAIN, or ISPA_V_F16_PREPARED (bf16, d = 128) */
+  ispa_v_layout v_layout; /* ISPA_V_PLAIN, ISPA_V_F16_PREPARED or ISPA_KV_E4M3_PREPARED (bf16, d = 128) */
 } ispa_attn_desc;
 
 /*
@@ -155,7 +156,8 @@ typedef struct {
  *   o_full     [B, Lq, H, d] out_dtype, lse_full [B, Lq, H] fp32   (both or neither)
  * An empty group yields O = 0 and L = -inf.  Compiled paths: bf16 in with
  * head_dim 128 (tcgen05 tensor cores, fp32 accumulation) and fp32 in with
- * head_dim 32/64/128 (fp32 CUDA cores).  Outputs may not alias inputs.
+ * head_dim 32/64/128 (tcgen05 kind::tf32 in three passes, hi/lo split of every
+ * operand: fp32-accurate).  Outputs may not alias inputs.
  * Every K/V row that a group's 128-row tiles cover must hold finite values.
  *   workspace  >= ispa_attn_split_workspace_bytes(desc) bytes, 16-byte aligned
  *              (0 for fp32 inputs and for a prepared V; for bf16 inputs with
@@ -207,6 +209,42 @@ ispa_status ispa_attn_split(const ispa_attn_desc *desc, const void *q, const voi
 size_t ispa_v16_bytes(const ispa_attn_desc *desc);
 ispa_status ispa_v16_prepare(const ispa_attn_desc *desc, const void *v, int frame_begin, int frame_end, void *v16,
                              ispa_stream_t stream);
+
+/*
+ * Prepared fp8 K and V: attention with 8-bit products for the post-switch
+ * layers.  ISPA combines with post-training 8-bit quantisation [EN-notes, Key
+ * Findings (Figure 7); DE-summary 4, "Beschleunigung"]; the pages give no
+ * scheme for the attention, so this library takes the plain one:
+ *   * Q, K, V in fp8 e4m3 with one fp32 scale per (instance, head) over that
+ *     head's rows, s = amax / 448, codes e4m3(x * (448 / amax)) (as the W8A8
+ *     quantisers; Q is quantised by the attention call itself);
+ *   * S = Q8 K8^T and O = P8 V8 on the 8-bit tensor cores (fp32 accumulation);
+ *   * per group an online softmax over 128-key tiles taken in the group's
+ *     order, each key range's tiles starting at its first key rounded down to
+ *     a multiple of 16: with t = S s_q s_k scale log2(e) and m the running
+ *     maximum over the tiles seen, p = 2^(t - m + 8) <= 256 enters the product
+ *     as e4m3(p) and the normaliser l as it is (fp32); O = acc s_v / l and
+ *     L = (m - 8 + log2 l) ln 2; the groups are merged by their LSE.
+ * ispa_kv8_bytes(desc): bytes of the prepared buffer for desc's K/V layout
+ *   (K8 [B, kv_frames*tpf, H, 128] bytes, V8 transposed [B, H, 128, rows
+ *   rounded up to 16] bytes, then the per-head scales); 0 for an invalid desc
+ *   or one that is not bf16 with d = 128.
+ * ispa_kv8_prepare(desc, k, v, frame_begin, frame_end, kv8, stream): converts
+ *   frames [frame_begin, frame_end) of the bf16 k and v into kv8 (caller-owned,
+ *   16-byte aligned, not overlapping k or v).  frame_begin == 0 starts afresh
+ *   (the scales then cover frames [0, frame_end)); a later prepare whose frames
+ *   raise a head's amax converts every row of that head again from k / v, which
+ *   must then hold all kv_frames frames.  Asynchronous.
+ * Use: set desc.v_layout = ISPA_KV_E4M3_PREPARED and pass kv8 as the k argument
+ *   of ispa_attn_split, ispa_attn_local_proj or ispa_attn_local_proj_q8 (v is
+ *   not read and may be NULL); their workspace then holds Q's per-head amax.
+ *   Not taken by ispa_warmup_fused (the warmup statistics use the bf16
+ *   attention) nor by ispa_kv_evict_history / ispa_kv_restore (evict the bf16
+ *   K/V, then prepare the evicted layout).
+ */
+size_t ispa_kv8_bytes(const ispa_attn_desc *desc);
+ispa_status ispa_kv8_prepare(const ispa_attn_desc *desc, const void *k, const void *v, int frame_begin,
+                             int frame_end, void *kv8, ispa_stream_t stream);
 
 /*
  * LSE-weighted merge of two disjoint groups' results [EN-notes, Key Designs 1]:

@@ -24,7 +24,7 @@ ISPA_OK, ISPA_ERR_INVALID_ARG, ISPA_ERR_UNSUPPORTED, ISPA_ERR_CUDA, ISPA_ERR_NOT
 ISPA_F32, ISPA_BF16 = 0, 1
 ISPA_PREC_TF32, ISPA_PREC_F32 = 0, 1
 ISPA_Q8_E4M3, ISPA_Q8_INT8 = 0, 1
-ISPA_V_PLAIN, ISPA_V_F16_PREPARED = 0, 1
+ISPA_V_PLAIN, ISPA_V_F16_PREPARED, ISPA_KV_E4M3_PREPARED = 0, 1, 2
 
 STATUS_NAMES = {0: "ISPA_OK", 1: "ISPA_ERR_INVALID_ARG", 2: "ISPA_ERR_UNSUPPORTED", 3: "ISPA_ERR_CUDA",
                 4: "ISPA_ERR_NOT_SPD", 5: "ISPA_ERR_TIMEOUT"}
@@ -37,7 +37,8 @@ EXPORTED = ("ispa_version", "ispa_last_error", "ispa_launch_count", "ispa_check_
             "ispa_kv_restore", "ispa_stats_reset", "ispa_selftest_wait_timeout", "ispa_quantize_rows",
             "ispa_quantize_weight", "ispa_gemm_q8", "ispa_gemm_bf16", "ispa_attn_local_proj_q8_workspace_bytes",
             "ispa_attn_local_proj_q8", "ispa_warmup_fused_workspace_bytes", "ispa_warmup_fused",
-            "ispa_v16_bytes", "ispa_v16_prepare", "ispa_absorb_error_workspace_bytes", "ispa_absorb_error")
+            "ispa_v16_bytes", "ispa_v16_prepare", "ispa_absorb_error_workspace_bytes", "ispa_absorb_error",
+            "ispa_kv8_bytes", "ispa_kv8_prepare")
 RIDGE_NOALLOC_MAX_D = RIDGE_NOALLOC_MAX_DOUT = 1024
 
 
@@ -62,10 +63,11 @@ def attn_desc(shape, in_dtype: int, out_dtype: int, softmax_scale: float = 0.0,
                     shape.cur_begin, shape.cur_end, shape.kv_frames, in_dtype, out_dtype, softmax_scale, v_layout)
 
 
-def prepared(desc: AttnDesc) -> AttnDesc:
-    """A copy of desc whose v argument is a prepared fp16 V (ispa_v16_prepare)."""
+def prepared(desc: AttnDesc, layout: int = ISPA_V_F16_PREPARED) -> AttnDesc:
+    """A copy of desc whose V (ISPA_V_F16_PREPARED, ispa_v16_prepare) or K/V
+    (ISPA_KV_E4M3_PREPARED, ispa_kv8_prepare) comes prepared."""
     d = AttnDesc.from_buffer_copy(desc)
-    d.v_layout = ISPA_V_F16_PREPARED
+    d.v_layout = layout
     return d
 
 
@@ -116,6 +118,8 @@ def lib() -> ctypes.CDLL:
                                           _vp, _sz, _vp]),
         "ispa_v16_bytes": (_sz, [ctypes.POINTER(AttnDesc)]),
         "ispa_absorb_error_workspace_bytes": (_sz, [_ci, _ci]),
+        "ispa_kv8_bytes": (_sz, [ctypes.POINTER(AttnDesc)]),
+        "ispa_kv8_prepare": (_ci, [ctypes.POINTER(AttnDesc), _vp, _vp, _ci, _ci, _vp, _vp]),
         "ispa_absorb_error": (_ci, [_ci, _ci, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
         "ispa_v16_prepare": (_ci, [ctypes.POINTER(AttnDesc), _vp, _ci, _ci, _vp, _vp]),
     }
@@ -209,6 +213,15 @@ def ispa_v16_bytes(desc: AttnDesc) -> int:
 def ispa_v16_prepare(desc: AttnDesc, v, frame_begin: int, frame_end: int, v16, stream=None) -> None:
     _check(lib().ispa_v16_prepare(ctypes.byref(desc), _ptr(v, name="v"), frame_begin, frame_end,
                                   _ptr(v16, name="v16"), _stream(stream)))
+
+
+def ispa_kv8_bytes(desc: AttnDesc) -> int:
+    return int(lib().ispa_kv8_bytes(ctypes.byref(desc)))
+
+
+def ispa_kv8_prepare(desc: AttnDesc, k, v, frame_begin: int, frame_end: int, kv8, stream=None) -> None:
+    _check(lib().ispa_kv8_prepare(ctypes.byref(desc), _ptr(k, name="k"), _ptr(v, name="v"), frame_begin, frame_end,
+                                  _ptr(kv8, name="kv8"), _stream(stream)))
 
 
 def ispa_lse_merge(rows: int, H: int, head_dim: int, o_dtype: int, o_a, lse_a, o_b, lse_b, o_out, lse_out,

@@ -154,10 +154,10 @@ ispa_status attn_ranges(const ispa_attn_desc *d, GroupRanges *g, float *scale) {
   if (d->head_dim != 32 && d->head_dim != 64 && d->head_dim != 128)
     return fail(ISPA_ERR_INVALID_ARG, "head_dim must be 32, 64 or 128 (got %d)", d->head_dim);
   if (!dtype_ok(d->in_dtype) || !dtype_ok(d->out_dtype)) return fail(ISPA_ERR_INVALID_ARG, "bad dtype");
-  if (d->v_layout != ISPA_V_PLAIN && d->v_layout != ISPA_V_F16_PREPARED)
+  if (d->v_layout != ISPA_V_PLAIN && d->v_layout != ISPA_V_F16_PREPARED && d->v_layout != ISPA_KV_E4M3_PREPARED)
     return fail(ISPA_ERR_INVALID_ARG, "bad v_layout");
-  if (d->v_layout == ISPA_V_F16_PREPARED && (d->in_dtype != ISPA_BF16 || d->head_dim != 128))
-    return fail(ISPA_ERR_INVALID_ARG, "a prepared fp16 V goes with bf16 inputs and head_dim 128");
+  if (d->v_layout != ISPA_V_PLAIN && (d->in_dtype != ISPA_BF16 || d->head_dim != 128))
+    return fail(ISPA_ERR_INVALID_ARG, "a prepared V (fp16) or K/V (fp8) goes with bf16 inputs and head_dim 128");
   const int F = d->kv_frames;
   if (F < 1) return fail(ISPA_ERR_INVALID_ARG, "kv_frames must be >= 1");
   if (d->sink_frames < 0 || d->sink_frames > F) return fail(ISPA_ERR_INVALID_ARG, "sink_frames out of [0, kv_frames]");
@@ -213,6 +213,9 @@ ispa_status kv_remap(const ispa_attn_desc *desc, const void *k, const void *v, v
   float scale;
   ispa_status st = attn_ranges(desc, &g, &scale);
   if (st != ISPA_OK) return st;
+  if (desc->v_layout == ISPA_KV_E4M3_PREPARED)
+    return fail(ISPA_ERR_INVALID_ARG, "a prepared fp8 K/V is not evicted or restored: move the bf16 K/V and "
+                "prepare the result (ispa_kv8_prepare)");
   if (!ptr_ok(k) || !ptr_ok(v) || !ptr_ok(k_out) || !ptr_ok(v_out))
     return fail(ISPA_ERR_INVALID_ARG, "the four K/V pointers must be 16-byte aligned device pointers");
   const long long esize = desc->in_dtype == ISPA_BF16 ? 2 : 4;
@@ -282,7 +285,7 @@ size_t ispa_attn_split_workspace_bytes(const ispa_attn_desc *desc) {
   float scale;
   if (attn_ranges(desc, &g, &scale) != ISPA_OK) return 0;
   if (desc->in_dtype != ISPA_BF16) return 0;
-  return attn_tc_workspace_bytes(desc->B, desc->H, g.Lkv, desc->v_layout == ISPA_V_F16_PREPARED);
+  return attn_tc_workspace_bytes(desc->B, desc->H, g.Lkv, desc->v_layout);
 }
 
 ispa_status ispa_attn_split(const ispa_attn_desc *desc, const void *q, const void *k, const void *v, void *o_loc,
@@ -295,7 +298,8 @@ ispa_status ispa_attn_split(const ispa_attn_desc *desc, const void *q, const voi
   const size_t need = ispa_attn_split_workspace_bytes(desc);
   if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
     return fail(ISPA_ERR_INVALID_ARG, "workspace needs %zu bytes (16-byte aligned)", need);
-  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v)) return fail(ISPA_ERR_INVALID_ARG, "q, k, v must be 16-byte aligned device pointers");
+  if (!ptr_ok(q) || !ptr_ok(k) || (!ptr_ok(v) && desc->v_layout != ISPA_KV_E4M3_PREPARED))
+    return fail(ISPA_ERR_INVALID_ARG, "q, k, v must be 16-byte aligned device pointers");
   if (!ptr_ok(o_loc) || !ptr_ok(lse_loc)) return fail(ISPA_ERR_INVALID_ARG, "o_loc and lse_loc are required (16-byte aligned)");
   if ((o_hist == nullptr) != (lse_hist == nullptr)) return fail(ISPA_ERR_INVALID_ARG, "o_hist and lse_hist: both or neither");
   if ((o_full == nullptr) != (lse_full == nullptr)) return fail(ISPA_ERR_INVALID_ARG, "o_full and lse_full: both or neither");
@@ -307,7 +311,7 @@ ispa_status ispa_attn_split(const ispa_attn_desc *desc, const void *q, const voi
     return launch_attn_tc(*desc, g, scale, q, k, v, o_loc, lse_loc, o_hist, lse_hist, o_full, lse_full, workspace,
                           (cudaStream_t)stream);
   }
-  return launch_attn_simt(*desc, g, scale, (const float *)q, (const float *)k, (const float *)v, o_loc, lse_loc, o_hist,
+  return launch_attn_tf32(*desc, g, scale, (const float *)q, (const float *)k, (const float *)v, o_loc, lse_loc, o_hist,
                           lse_hist, o_full, lse_full, (cudaStream_t)stream);
 }
 
@@ -336,6 +340,38 @@ ispa_status ispa_v16_prepare(const ispa_attn_desc *desc, const void *v, int fram
   const long long vb = (long long)desc->B * g.Lkv * desc->H * 128 * 2, v16b = (long long)v16_bytes(desc->B, desc->H, g.Lkv);
   if (a < b + v16b && b < a + vb) return fail(ISPA_ERR_INVALID_ARG, "v16 must not overlap v");
   return launch_v16_prepare(desc->B, desc->H, g.Lkv, (int)(frame_begin * tpf), (int)(frame_end * tpf), v, v16,
+                            (cudaStream_t)stream);
+}
+
+size_t ispa_kv8_bytes(const ispa_attn_desc *desc) {
+  GroupRanges g;
+  float scale;
+  if (attn_ranges(desc, &g, &scale) != ISPA_OK) return 0;
+  if (desc->in_dtype != ISPA_BF16 || desc->head_dim != 128) return 0;
+  return kv8_bytes(desc->B, desc->H, g.Lkv);
+}
+
+ispa_status ispa_kv8_prepare(const ispa_attn_desc *desc, const void *k, const void *v, int frame_begin,
+                             int frame_end, void *kv8, ispa_stream_t stream) {
+  GroupRanges g;
+  float scale;
+  ispa_status st = attn_ranges(desc, &g, &scale);
+  if (st != ISPA_OK) return st;
+  if (desc->in_dtype != ISPA_BF16 || desc->head_dim != 128)
+    return fail(ISPA_ERR_UNSUPPORTED, "a prepared fp8 K/V is built for bf16 inputs with head_dim 128");
+  if (!(0 <= frame_begin && frame_begin <= frame_end && frame_end <= desc->kv_frames))
+    return fail(ISPA_ERR_INVALID_ARG, "frames [%d, %d) invalid for kv_frames %d", frame_begin, frame_end,
+                desc->kv_frames);
+  if (!ptr_ok(k) || !ptr_ok(v) || !ptr_ok(kv8))
+    return fail(ISPA_ERR_INVALID_ARG, "k, v and kv8 must be 16-byte aligned device pointers");
+  const long long nb = (long long)desc->B * g.Lkv * desc->H * 128 * 2, n8 = (long long)kv8_bytes(desc->B, desc->H, g.Lkv);
+  auto overlap = [](const void *a, long long na, const void *b, long long nbb) {
+    const char *x = (const char *)a, *y = (const char *)b;
+    return x < y + nbb && y < x + na;
+  };
+  if (overlap(kv8, n8, k, nb) || overlap(kv8, n8, v, nb)) return fail(ISPA_ERR_INVALID_ARG, "kv8 must not overlap k or v");
+  const long long tpf = desc->tokens_per_frame;
+  return launch_kv8_prepare(desc->B, desc->H, g.Lkv, (int)(frame_begin * tpf), (int)(frame_end * tpf), k, v, kv8,
                             (cudaStream_t)stream);
 }
 
@@ -387,7 +423,7 @@ size_t ispa_warmup_fused_workspace_bytes(const ispa_attn_desc *desc, int Dout) {
   if (!desc || Dout < 1 || attn_ranges(desc, &g, &scale) != ISPA_OK) return 0;
   const int T = desc->B * g.Lq, D = desc->H * desc->head_dim;
   return round256(stats_workspace_bytes(T, D, Dout, ISPA_PREC_TF32)) + round256((size_t)T * desc->H * 4) +
-         attn_tc_workspace_bytes(desc->B, desc->H, g.Lkv, desc->v_layout == ISPA_V_F16_PREPARED);
+         attn_tc_workspace_bytes(desc->B, desc->H, g.Lkv, desc->v_layout);
 }
 
 ispa_status ispa_warmup_fused(const ispa_attn_desc *desc, const void *q, const void *k, const void *v,
@@ -399,6 +435,8 @@ ispa_status ispa_warmup_fused(const ispa_attn_desc *desc, const void *q, const v
   if (st != ISPA_OK) return st;
   if (desc->in_dtype != ISPA_BF16 || desc->head_dim != 128)
     return fail(ISPA_ERR_UNSUPPORTED, "the fused warmup is compiled for bf16 inputs with head_dim 128");
+  if (desc->v_layout == ISPA_KV_E4M3_PREPARED)
+    return fail(ISPA_ERR_UNSUPPORTED, "the fused warmup runs the bf16 attention (fp8 K/V is a post-switch layout)");
   const int D = desc->H * desc->head_dim;
   const long long T = (long long)desc->B * g.Lq;
   if (Dout < 32 || Dout % 32 != 0) return fail(ISPA_ERR_INVALID_ARG, "Dout must be a positive multiple of 32");
@@ -506,7 +544,7 @@ size_t ispa_attn_local_proj_workspace_bytes(const ispa_attn_desc *desc) {
   const size_t a = (size_t)desc->B * g.Lq * desc->H * desc->head_dim * 2;
   const size_t l = (size_t)desc->B * g.Lq * desc->H * 4;
   return ((a + 255) & ~size_t(255)) + ((l + 255) & ~size_t(255)) +
-         attn_tc_workspace_bytes(desc->B, desc->H, g.Lkv, desc->v_layout == ISPA_V_F16_PREPARED);
+         attn_tc_workspace_bytes(desc->B, desc->H, g.Lkv, desc->v_layout);
 }
 
 ispa_status ispa_attn_local_proj(const ispa_attn_desc *desc, const void *q, const void *k, const void *v,
@@ -520,7 +558,8 @@ ispa_status ispa_attn_local_proj(const ispa_attn_desc *desc, const void *q, cons
     return fail(ISPA_ERR_UNSUPPORTED, "post-switch projection is compiled for bf16 inputs with head_dim 128");
   if (Dout < 16 || Dout % 16 != 0) return fail(ISPA_ERR_INVALID_ARG, "Dout must be a positive multiple of 16");
   if (!dtype_ok(y_dtype)) return fail(ISPA_ERR_INVALID_ARG, "bad y dtype");
-  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(W_proj) || !ptr_ok(y))
+  if (!ptr_ok(q) || !ptr_ok(k) || (!ptr_ok(v) && desc->v_layout != ISPA_KV_E4M3_PREPARED) || !ptr_ok(W_proj) ||
+      !ptr_ok(y))
     return fail(ISPA_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
   const size_t need = ispa_attn_local_proj_workspace_bytes(desc);
   if (!workspace || workspace_bytes < need || !aligned16(workspace))
@@ -635,7 +674,8 @@ ispa_status ispa_attn_local_proj_q8(const ispa_attn_desc *desc, const void *q, c
     return fail(ISPA_ERR_INVALID_ARG, "int8 products need D <= 131072");
   if (Dout < 16 || Dout % 16 != 0) return fail(ISPA_ERR_INVALID_ARG, "Dout must be a positive multiple of 16");
   if (!dtype_ok(y_dtype)) return fail(ISPA_ERR_INVALID_ARG, "bad y dtype");
-  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(qT) || !ptr_ok(sw) || !ptr_ok(y))
+  if (!ptr_ok(q) || !ptr_ok(k) || (!ptr_ok(v) && desc->v_layout != ISPA_KV_E4M3_PREPARED) || !ptr_ok(qT) ||
+      !ptr_ok(sw) || !ptr_ok(y))
     return fail(ISPA_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
   const size_t need = ispa_attn_local_proj_q8_workspace_bytes(desc);
   if (!workspace || workspace_bytes < need || !aligned16(workspace))

@@ -800,8 +800,9 @@ size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
-size_t attn_tc_workspace_bytes(int B, int H, int Lkv, bool v_prepared) {
-  if (v_prepared) return 0;
+size_t attn_tc_workspace_bytes(int B, int H, int Lkv, int v_layout) {
+  if (v_layout == ISPA_V_F16_PREPARED) return 0;
+  if (v_layout == ISPA_KV_E4M3_PREPARED) return attn_f8_workspace_bytes(B, H);
   return a256((size_t)B * Lkv * H * kD * 2) + 3 * a256((size_t)B * H * 4);
 }
 
@@ -854,6 +855,8 @@ ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float 
                            const void *k, const void *v, void *o_loc, float *l_loc, void *o_hist, float *l_hist,
                            void *o_full, float *l_full, void *workspace, cudaStream_t s, float *stats_dA) {
   if (g.Lq == 0) return ISPA_OK;
+  if (d.v_layout == ISPA_KV_E4M3_PREPARED)  // k is the prepared fp8 K/V, v is not used
+    return launch_attn_f8(d, g, scale, q, k, o_loc, l_loc, o_hist, l_hist, o_full, l_full, workspace, s);
   AttnParams P{};
   ispa_status st = device_err(&P.err);
   if (st != ISPA_OK) return st;

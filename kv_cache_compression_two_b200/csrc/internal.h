@@ -59,9 +59,13 @@ ispa_status launch_absorb_weight(int D, int Dout, const void *W, ispa_dtype wdt,
 ispa_status launch_attn_simt(const ispa_attn_desc &d, const GroupRanges &g, float scale, const float *q,
                              const float *k, const float *v, void *o_loc, float *l_loc, void *o_hist,
                              float *l_hist, void *o_full, float *l_full, cudaStream_t s);
+// fp32 inputs on the tf32 tensor cores in three passes (attn_tf32.cu)
+ispa_status launch_attn_tf32(const ispa_attn_desc &d, const GroupRanges &g, float scale, const float *q,
+                             const float *k, const float *v, void *o_loc, float *l_loc, void *o_hist, float *l_hist,
+                             void *o_full, float *l_full, cudaStream_t s);
 // workspace: an fp16 copy of V (see attn_tc.cu) plus per-head scales; none
 // when V comes prepared (ispa_v16_prepare)
-size_t attn_tc_workspace_bytes(int B, int H, int Lkv, bool v_prepared);
+size_t attn_tc_workspace_bytes(int B, int H, int Lkv, int v_layout);
 // prepared fp16 V: B * Lkv * H * 128 fp16 values, then the per-head state
 size_t v16_bytes(int B, int H, int Lkv);
 size_t v16_state_offset(int B, int H, int Lkv);
@@ -70,6 +74,16 @@ size_t v16_state_bytes(int B, int H);
 // clears the state first)
 ispa_status launch_v16_prepare(int B, int H, int Lkv, int row_begin, int row_end, const void *v, void *v16,
                                cudaStream_t s);
+// fp8 e4m3 attention (attn_f8.cu): the prepared K/V buffer (K8, V8 transposed,
+// per-head scales), its prepare, the call's workspace (Q's per-head amax) and
+// the launch (kv8 in place of K and V)
+size_t kv8_bytes(int B, int H, int Lkv);
+size_t attn_f8_workspace_bytes(int B, int H);
+ispa_status launch_kv8_prepare(int B, int H, int Lkv, int row_begin, int row_end, const void *k, const void *v,
+                               void *kv8, cudaStream_t s);
+ispa_status launch_attn_f8(const ispa_attn_desc &d, const GroupRanges &g, float scale, const void *q,
+                           const void *kv8, void *o_loc, float *l_loc, void *o_hist, float *l_hist, void *o_full,
+                           float *l_full, void *workspace, cudaStream_t s);
 ispa_status launch_attn_tc(const ispa_attn_desc &d, const GroupRanges &g, float scale, const void *q,
                            const void *k, const void *v, void *o_loc, float *l_loc, void *o_hist,
                            float *l_hist, void *o_full, float *l_full, void *workspace, cudaStream_t s,
