@@ -1337,7 +1337,14 @@ def run_attn_only(args):
     o = {n: torch.empty((sh.B, sh.Lq, sh.H, 128), **f32) for n in ("loc", "hist", "full")}
     l = {n: torch.empty((sh.B, sh.Lq, sh.H), **f32) for n in ("loc", "hist", "full")}
     desc = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_F32)
-    if args.plain_v:  # the call converting V itself (no prepared copy)
+    if args.kv8:  # the fp8 e4m3 attention on a prepared fp8 K/V
+        kv8 = torch.empty(ispa.ispa_kv8_bytes(desc), device=dev, dtype=torch.uint8)
+        ispa.ispa_kv8_prepare(desc, L.dev["k"], L.dev["v"], 0, sh.kv_frames, kv8)
+        pd8 = ispa.prepared(desc, ispa.ISPA_KV_E4M3_PREPARED)
+        ws8 = torch.empty(ispa.ispa_attn_split_workspace_bytes(pd8), device=dev, dtype=torch.uint8)
+        run = lambda: ispa.ispa_attn_split(pd8, L.dev["q"], kv8, None, o["loc"], l["loc"], o["hist"], l["hist"],
+                                           o["full"], l["full"], workspace=ws8)
+    elif args.plain_v:  # the call converting V itself (no prepared copy)
         ws = torch.empty(ispa.ispa_attn_split_workspace_bytes(desc), device=dev, dtype=torch.uint8)
         run = lambda: ispa.ispa_attn_split(desc, L.dev["q"], L.dev["k"], L.dev["v"], o["loc"], l["loc"], o["hist"],
                                            l["hist"], o["full"], l["full"], workspace=ws)
@@ -1387,6 +1394,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-rows", type=int, default=32, help="query rows of the oracle sample (0: skip it)")
     ap.add_argument("--plain-v", action="store_true", help="--only attn: V converted by every call")
+    ap.add_argument("--kv8", action="store_true", help="--only attn: the fp8 attention on a prepared fp8 K/V")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the 14B layer, the 30-layer model and the sweep (components outside the timed steps)")
     ap.add_argument("--only", choices=["step", "attn", "proj", "parts", "sweep"], default="step",

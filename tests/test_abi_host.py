@@ -274,3 +274,53 @@ int main(void) {
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0, (out.returncode, out.stderr)
     assert out.stdout.strip() == ispa.lib().ispa_version().decode()
+
+
+def test_descriptor_layout_matches_the_binding(tmp_path):
+    """sizeof(ispa_attn_desc) and the offset of every field agree between the C header and the
+    ctypes structure the binding passes."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    fields = [f for f, _ in ispa.AttnDesc._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "ispa.h"\nint main(void) {\n'
+                   '  printf("%zu\\n", sizeof(ispa_attn_desc));\n' +
+                   "".join(f'  printf("%zu\\n", offsetof(ispa_attn_desc, {f}));\n' for f in fields) +
+                   "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    vals = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    assert vals[0] == ctypes.sizeof(ispa.AttnDesc)
+    assert vals[1:] == [getattr(ispa.AttnDesc, f).offset for f in fields]
+
+
+def test_prepare_and_error_entry_points_validate_on_the_host():
+    L = ispa.lib()
+    d = _desc()
+    # prepared fp16 V / fp8 K/V: frame ranges and dtypes are checked before any launch
+    assert L.ispa_v16_prepare(ctypes.byref(d), FAKE, 3, 2, FAKE, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_v16_prepare(ctypes.byref(d), FAKE, 0, 6, FAKE, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_kv8_prepare(ctypes.byref(d), FAKE, FAKE, 0, 9, FAKE, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_kv8_prepare(ctypes.byref(d), FAKE, FAKE, 0, 1, FAKE, None) == ispa.ISPA_ERR_INVALID_ARG  # overlap
+    f32 = _desc(in_dtype=ispa.ISPA_F32, head_dim=64)
+    assert L.ispa_v16_bytes(ctypes.byref(f32)) == 0 and L.ispa_kv8_bytes(ctypes.byref(f32)) == 0
+    assert L.ispa_v16_prepare(ctypes.byref(f32), FAKE, 0, 1, FAKE * 2, None) == ispa.ISPA_ERR_UNSUPPORTED
+    assert L.ispa_v16_bytes(ctypes.byref(d)) > 5 * 16 * 2 * 128 * 2
+    # a prepared layout needs bf16 inputs with head_dim 128; an unknown layout is rejected
+    bad = _desc(in_dtype=ispa.ISPA_F32, head_dim=64, v_layout=ispa.ISPA_V_F16_PREPARED)
+    assert _split(bad) == ispa.ISPA_ERR_INVALID_ARG
+    assert _split(_desc(v_layout=7)) == ispa.ISPA_ERR_INVALID_ARG
+    # the fp8 layout is not evicted (the bf16 K/V is), nor run by the fused warmup
+    d8 = _desc(v_layout=ispa.ISPA_KV_E4M3_PREPARED)
+    assert L.ispa_kv_evict_history(ctypes.byref(d8), FAKE, FAKE, FAKE * 2, FAKE * 3, None) == \
+        ispa.ISPA_ERR_INVALID_ARG
+    assert "evict" in L.ispa_last_error().decode()
+    assert L.ispa_warmup_fused(ctypes.byref(d8), FAKE, FAKE, FAKE, FAKE, 256, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                               1 << 40, None) == ispa.ISPA_ERR_UNSUPPORTED
+    # the epsilon entry point
+    assert L.ispa_absorb_error(0, 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_absorb_error(64, 64, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, None) == ispa.ISPA_ERR_INVALID_ARG
+    assert L.ispa_absorb_error_workspace_bytes(64, 64) >= 64 * 64 * 4
