@@ -306,3 +306,26 @@ def test_post_switch_full_size_1p3b_sampled_rows():
         assert not np.isnan(got).any(), layer
         ref = orc.local_projection(ref_sh, data["q"], data["k"], data["v"], Wp, None, rows=rows)
         assert_bf16_out(got[:, rows], ref, tol=2e-2)
+
+
+@pytest.mark.parametrize("B,hist", [(2, 15), (1, 117)])
+def test_bf16_sweep_extremes_sampled_rows(B, hist):
+    """Points of the history / batch sweep at full size: the 1.3B layout with two
+    instances, and with the longest history (117 frames, 191 880 keys), on the
+    prepared V as the bench runs them; sampled rows of every instance against the
+    oracle."""
+    sh = si.video_shape(12, hist, B=B)
+    data = si.iid_qkv(sh, "bf16", ("gpu", "sweep", B, hist))
+    q, k, v = dev(data["q"], torch.bfloat16), dev(data["k"], torch.bfloat16), dev(data["v"], torch.bfloat16)
+    desc = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_F32)
+    v16 = torch.empty(ispa.ispa_v16_bytes(desc), dtype=torch.uint8, device="cuda")
+    ispa.ispa_v16_prepare(desc, v, 0, sh.kv_frames, v16)
+    o = {n: nan_like((B, sh.Lq, sh.H, 128), torch.float32) for n in ("loc", "hist", "full")}
+    l = {n: nan_like((B, sh.Lq, sh.H), torch.float32) for n in ("loc", "hist", "full")}
+    ispa.ispa_attn_split(ispa.prepared(desc), q, k, v16, o["loc"], l["loc"], o["hist"], l["hist"], o["full"],
+                         l["full"])
+    ispa.ispa_check_device_error()
+    torch.cuda.synchronize()
+    rows = np.r_[0, 127, 1560, 3119, 4600:4680:16, 4679]
+    check(sh, data, {n: host(t) for n, t in o.items()}, {n: host(t) for n, t in l.items()}, ispa.ISPA_BF16,
+          ispa.ISPA_F32, rows=rows)
