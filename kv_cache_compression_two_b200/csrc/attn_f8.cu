@@ -38,9 +38,14 @@
 // commit fires when all earlier ones have completed):
 //   * S_{j+2} overwrites S buffer j % 2 after s_free(j): the softmax of tile j
 //     has finished its tcgen05.ld of S_j.
-//   * P_j goes to P buffer j % 2 after p_free(j - 2): PV_{j-2} has read P_{j-2}.
-//   * The correction of O in the softmax of tile j waits o_done for PV_{j-1};
-//     PV_j cannot have run (it waits for P_j), so the phase cannot alias.
+//   * P_j goes to P buffer j % 2 once PV_{j-2} (pv_done) has read P_{j-2}.
+//   * PV_j commits to pv_done[j % 2], so each barrier advances once per two
+//     PVs and a wait names its PV by index: the correction of O in the softmax
+//     of tile j waits for PV_{j-1} (PVs complete in order, so PV_{j-2} too) --
+//     with S issued ahead of PV, PV_{j-2} may still be running when S_j has
+//     landed, and one barrier over every PV would then be two phases behind;
+//     the next phase of pv_done[(j-1) % 2] is PV_{j+1}, which waits for
+//     P_{j+1}, so the wait cannot alias.  The same barriers free P buffers.
 //   * At the end of the local group the epilogue reads O after PV of that tile
 //     and releases it (o_free) before the first history PV starts O afresh.
 #include <algorithm>
@@ -257,8 +262,8 @@ struct SmemLayout8 {
   uint64_t v_full[kStagesV], v_empty[kStagesV];
   uint64_t q_ready;
   uint64_t s_full[2], s_free[2];
-  uint64_t p_full[2], p_free[2];
-  uint64_t o_done, o_free, drain;
+  uint64_t p_full[2], pv_done[2];  // pv_done[b]: PV_j done for j % 2 == b (P buffer b free again)
+  uint64_t o_free, drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -288,6 +293,27 @@ __device__ __forceinline__ float ex2f(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Packed fp32 pair arithmetic (sm_100): one instruction for two lanes of work.
+__device__ __forceinline__ float2 ffma2f(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 fadd2f(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
 }
 
 __device__ __forceinline__ float fmax3f(float a, float b, float c) {
@@ -381,9 +407,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.s_free[s], 128);
       mbar_init(&sm.p_full[s], 128);
-      mbar_init(&sm.p_free[s], 1);
+      mbar_init(&sm.pv_done[s], 1);
     }
-    mbar_init(&sm.o_done, 1);
     mbar_init(&sm.o_free, 128);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
@@ -459,8 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kTileK / 32; ++kk)
           mma_ts_f8(tmem + kColO, a_p + kk * 8, vd + (uint64_t)((kk * 32) >> 4), idesc, (first && kk == 0) ? 0u : 1u);
-        mma_commit(&sm.o_done);
-        mma_commit(&sm.p_free[j & 1]);
+        mma_commit(&sm.pv_done[j & 1]);
         mma_commit(&sm.v_empty[j % kStagesV]);
       };
       bool ok = wait_parity(&sm.q_ready, 0, P.err, abort, 50);
@@ -566,7 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         l = 0.f;
       } else if (__any_sync(0xffffffffu, mt > m_ref)) {
         // the running maximum grows: O (after PV_{j-1}) and l scale by 2^(m_ref - m_new)
-        ok = wait_parity(&sm.o_done, (uint32_t)(j - 1) & 1, P.err, abort, 62);
+        ok = wait_parity(&sm.pv_done[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1, P.err, abort, 62);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
         const float m_new = fmaxf(m_ref, mt);
@@ -585,22 +609,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // p = 2^(t - m_ref + 8) in (0, 256]; l in fp32; P8 = e4m3(p), four per column
-      const float nm = kPOffset - m_ref;
+      // (pairs on the packed fp32 pipe: one FFMA2 and one FADD2 per two weights)
+      const float2 c2 = make_float2(c_log2, c_log2), nm2 = make_float2(kPOffset - m_ref, kPOffset - m_ref);
       uint32_t pk[32];
-      float ls0 = 0.f, ls1 = 0.f;
+      float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        const float p0 = ex2f(fmaf(__uint_as_float(sr[c >> 3][(4 * c) & 31]), c_log2, nm));
-        const float p1 = ex2f(fmaf(__uint_as_float(sr[c >> 3][(4 * c + 1) & 31]), c_log2, nm));
-        const float p2 = ex2f(fmaf(__uint_as_float(sr[c >> 3][(4 * c + 2) & 31]), c_log2, nm));
-        const float p3 = ex2f(fmaf(__uint_as_float(sr[c >> 3][(4 * c + 3) & 31]), c_log2, nm));
-        ls0 += p0 + p1;
-        ls1 += p2 + p3;
-        pk[c] = e4m3x4(p0, p1, p2, p3);
+        const uint32_t *row = &sr[c >> 3][(4 * c) & 31];
+        const float2 x01 = ffma2f(make_float2(__uint_as_float(row[0]), __uint_as_float(row[1])), c2, nm2);
+        const float2 x23 = ffma2f(make_float2(__uint_as_float(row[2]), __uint_as_float(row[3])), c2, nm2);
+        const float2 p01 = make_float2(ex2f(x01.x), ex2f(x01.y));
+        const float2 p23 = make_float2(ex2f(x23.x), ex2f(x23.y));
+        ls[0] = fadd2f(ls[0], p01);
+        ls[1] = fadd2f(ls[1], p23);
+        pk[c] = e4m3x4(p01.x, p01.y, p23.x, p23.y);
       }
-      l += ls0 + ls1;
+      l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
       if (j >= 2) {  // PV_{j-2} has read this P buffer
-        ok = wait_parity(&sm.p_free[j & 1], (uint32_t)((j - 2) >> 1) & 1, P.err, abort, 63);
+        ok = wait_parity(&sm.pv_done[j & 1], (uint32_t)((j - 2) >> 1) & 1, P.err, abort, 63);
         if (!__all_sync(0xffffffffu, ok)) break;
       }
       tmem_st16(lane_base + kColP + (uint32_t)(j & 1) * 32, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
@@ -610,7 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&sm.p_full[j & 1]);
 
       if (!grp_last) continue;
-      ok = wait_parity(&sm.o_done, (uint32_t)j & 1, P.err, abort, 64);
+      ok = wait_parity(&sm.pv_done[j & 1], (uint32_t)(j >> 1) & 1, P.err, abort, 64);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const bool is_loc = j < P.n_loc_tiles;

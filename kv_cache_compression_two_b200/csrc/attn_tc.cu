@@ -33,7 +33,10 @@
 //     reading S_j.
 //   * When the softmax of tile j starts (S_j complete), PV_{j-2} has completed
 //     (S_j was issued after it); PV_{j-1} may still run, so a correction of O
-//     first waits for PV_{j-1} (o_done); PV_j itself waits for P_j.
+//     first waits for PV_{j-1}; PV_j itself waits for P_j.  PV_j commits to
+//     o_done[j % 2], so a wait names its PV by index and the barrier it waits
+//     on cannot be a phase ahead (its next PV, PV_{j+2}, needs P_{j+2}) nor
+//     behind in a way the parity would hide.
 //   * At the end of the local group the epilogue reads O after PV of that tile
 //     (o_done) and releases it (o_free) before the first history PV, which
 //     starts O afresh, is issued.
@@ -331,7 +334,7 @@ struct SmemLayout {
   uint64_t q_ready;   // Q is in tensor memory (128 arrivals)
   uint64_t s_full[2]; // S_j complete in buffer j % 2
   uint64_t p_full[2]; // P_j written into buffer j % 2 (128 arrivals)
-  uint64_t o_done;    // one phase per PV_j
+  uint64_t o_done[2]; // PV_j complete, on o_done[j % 2]
   uint64_t o_free;    // the local-group epilogue has read O (128 arrivals)
   uint64_t drain;
   uint32_t tmem_base;
@@ -466,7 +469,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.p_full[s], 128);
     }
-    mbar_init(&sm.o_done, 1);
+    mbar_init(&sm.o_done[0], 1);
+    mbar_init(&sm.o_done[1], 1);
     mbar_init(&sm.o_free, 128);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
@@ -547,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < kTileK / 16; ++kk)
           mma_ts(tmem + kColO, a_p + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
                  (first && kk == 0) ? 0u : 1u);
-        mma_commit(&sm.o_done);
+        mma_commit(&sm.o_done[j & 1]);
         mma_commit(&sm.v_empty[j % kStagesV]);
       };
       bool ok = wait_parity(&sm.q_ready, 0, P.err, abort, 20);
@@ -648,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (__any_sync(0xffffffffu, mt > m_ref + kRescaleThreshold)) {
         // O may still be accumulating PV_{j-1}; it is final once that PV lands (PV_j
         // waits for P_j, which this warpgroup has not published yet).
-        ok = wait_parity(&sm.o_done, (uint32_t)(j - 1) & 1, P.err, abort, 32);
+        ok = wait_parity(&sm.o_done[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1, P.err, abort, 32);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
         const float m_new = fmaxf(m_ref, mt);
@@ -689,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!grp_last) continue;
       // ---- end of a group: O is final once PV_j has landed (PV_{j+1} needs P_{j+1},
       // which this warpgroup has not produced, so the wait cannot alias).
-      ok = wait_parity(&sm.o_done, (uint32_t)j & 1, P.err, abort, 33);
+      ok = wait_parity(&sm.o_done[j & 1], (uint32_t)(j >> 1) & 1, P.err, abort, 33);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const bool is_loc = j < P.n_loc_tiles;

@@ -28,10 +28,14 @@ def _eps_bound(Gs, Cs, r2, dW_ref, lam, rel_dw, stats_rel=0.0):
     r2 - 2<dW, C> + <dW, G dW> and (G + lam I) dW* = C), plus 1e-6 r2 for the
     kernel's rounding and stats_rel of each term for statistics that carry an error."""
     n2 = float(np.sum(dW_ref * dW_ref))
-    t = abs(float(np.sum(dW_ref * Cs)))
-    qd = abs(float(np.sum(dW_ref * (Gs @ dW_ref))))
-    return (1e-6 * r2 + 2.0 * lam * rel_dw * n2 + np.linalg.norm(Gs, 2) * rel_dw ** 2 * n2 +
-            stats_rel * (r2 + 2 * t + qd))
+    # |G|_2 <= the largest absolute row sum (G symmetric): an O(D^2) bound in place of an SVD
+    g2 = float(np.abs(Gs).sum(axis=1).max())
+    extra = 0.0
+    if stats_rel > 0:
+        t = abs(float(np.sum(dW_ref * Cs)))
+        qd = abs(float(np.sum(dW_ref * (Gs @ dW_ref))))
+        extra = stats_rel * (r2 + 2 * t + qd)
+    return 1e-6 * r2 + 2.0 * lam * rel_dw * n2 + g2 * rel_dw ** 2 * n2 + extra
 
 
 def _sym(G_upper):

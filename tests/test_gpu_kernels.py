@@ -162,7 +162,8 @@ def eps_bound(Gs, Cs, r2, dW_ref, lam, rel_dw):
     2 lam rel_dw |dW*|^2 + |G|_2 rel_dw^2 |dW*|^2; plus 1e-6 r2 for the kernel's own rounding
     (the terms that cancel are of size r2).  Every quantity here is the oracle's."""
     n2 = float(np.sum(dW_ref * dW_ref))
-    return 1e-6 * r2 + 2.0 * lam * rel_dw * n2 + np.linalg.norm(Gs, 2) * rel_dw ** 2 * n2
+    g2 = float(np.abs(Gs).sum(axis=1).max())   # >= |G|_2 for symmetric G (no SVD)
+    return 1e-6 * r2 + 2.0 * lam * rel_dw * n2 + g2 * rel_dw ** 2 * n2
 
 
 def _run_ridge(G, C, r2, lam, rel, refine):
