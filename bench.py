@@ -822,6 +822,8 @@ def run_ours(args, world, rank, local):
     idx = torch.zeros(K_sel, device=dev, dtype=torch.int32)
     W_new = torch.empty((D, D), device=dev, dtype=torch.bfloat16)
     y = {n: torch.empty((B, Lq, D), device=dev, dtype=torch.bfloat16) for n in ("L", "F")}
+    # the step's outputs (the end-to-end run swaps in a second set while the first is read back)
+    ocur = {"y": y, "dW": dW, "eps": eps_all}
     desc_warm = ispa.attn_desc(sh, ispa.ISPA_BF16, ispa.ISPA_F32)
     # the switch: the L-layer drops its history (real eviction: the kept frames
     # go to new buffers, the originals are released; bytes from the allocator)
@@ -870,7 +872,8 @@ def run_ours(args, world, rank, local):
     ev_attn = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
 
     def solve():
-        ispa.ispa_ridge_solve(D, D, G, C, r2, LAMBDA_REL, True, 0, dW, eps_all[7:8], ws_ridge, stream=stream)
+        ispa.ispa_ridge_solve(D, D, G, C, r2, LAMBDA_REL, True, 0, ocur["dW"], ocur["eps"][7:8], ws_ridge,
+                              stream=stream)
 
     def prepare_chunk(Lr):
         d_ = Lr.desc
@@ -891,14 +894,14 @@ def run_ours(args, world, rank, local):
         ispa.ispa_accum_stats(T, D, D, o["loc"], o["full"], wcur["W32"], G, C, r2, ispa.ISPA_PREC_TF32, ws_stats,
                               stream=stream)
         solve()
-        ispa.ispa_select_layers(N_LAYERS, eps_all, K_sel, is_local, idx, stream=stream)
-        ispa.ispa_absorb_weight(D, D, W16, ispa.ISPA_BF16, dW, W_new, ispa.ISPA_BF16, stream=stream)
+        ispa.ispa_select_layers(N_LAYERS, ocur["eps"], K_sel, is_local, idx, stream=stream)
+        ispa.ispa_absorb_weight(D, D, W16, ispa.ISPA_BF16, ocur["dW"], W_new, ispa.ISPA_BF16, stream=stream)
         prepare_chunk(LL)
-        ispa.ispa_attn_local_proj(pdesc_L, LL.dev["q"], LL.dev["k"], LL.dev["v16"], W_new, D, y["L"],
+        ispa.ispa_attn_local_proj(pdesc_L, LL.dev["q"], LL.dev["k"], LL.dev["v16"], W_new, D, ocur["y"]["L"],
                                   ispa.ISPA_BF16, ws_proj, stream=stream)
         prepare_chunk(LF)
-        ispa.ispa_attn_local_proj(pdesc_F, LF.dev["q"], LF.dev["k"], LF.dev["v16"], W16, D, y["F"], ispa.ISPA_BF16,
-                                  ws_proj, stream=stream)
+        ispa.ispa_attn_local_proj(pdesc_F, LF.dev["q"], LF.dev["k"], LF.dev["v16"], W16, D, ocur["y"]["F"],
+                                  ispa.ISPA_BF16, ws_proj, stream=stream)
 
     # one eager step sets up every kernel's attributes; then the step and the
     # solve alone are captured into CUDA graphs (the chain of dependent
@@ -1032,49 +1035,70 @@ def run_ours(args, world, rank, local):
     small_host = torch.empty(N_LAYERS, dtype=torch.float64).pin_memory()
     d2h = sum(t.numel() * t.element_size() for t in y_host.values()) + dW_host.numel() * 4 + N_LAYERS * 8
 
-    # Two device sets of every layer's buffers (their cache frames identical):
-    # the copies of step i + 1 run on a copy stream into one set while step i
-    # computes on the other (double buffering, ordered by events), so a step
-    # costs max(copy, compute) instead of their sum.
+    # Two device sets of every layer's buffers (their cache frames identical)
+    # and of the step's outputs.  The host->device copies of step i + 1 run on
+    # two copy streams into one set while step i computes on the other, and the
+    # device->host copies of step i on a third stream while step i + 1 computes
+    # (double buffering, ordered by events), so a step costs max(copies,
+    # compute) instead of their sum; every copy of every timed step is inside
+    # the timed region.
     set1 = []
     for Lr in layers:
         d1 = {n: t.clone() for n, t in Lr.dev.items()}
         set1.append(d1)
     sets = [([Lr.dev for Lr in layers], W32), (set1, torch.empty_like(W32))]
-    copy_stream = torch.cuda.Stream(dev)
-    copied = [torch.cuda.Event(), torch.cuda.Event()]
+    outs = [dict(ocur), {"y": {n: torch.empty_like(t) for n, t in y.items()}, "dW": torch.empty_like(dW),
+                         "eps": eps_all.clone()}]
+    h2d_streams = [torch.cuda.Stream(dev), torch.cuda.Stream(dev)]
+    d2h_stream = torch.cuda.Stream(dev)
+    copied = [[torch.cuda.Event(), torch.cuda.Event()] for _ in range(2)]
     freed = [torch.cuda.Event(), torch.cuda.Event()]
+    computed = [torch.cuda.Event(), torch.cuda.Event()]
+    read_back = [torch.cuda.Event(), torch.cuda.Event()]
 
     def issue_copy(i):
         devs, wd = sets[i % 2]
-        with torch.cuda.stream(copy_stream):
-            if i >= 2:
-                copy_stream.wait_event(freed[i % 2])  # step i - 2 is done with this set
-            for hc, d, rs in zip(host_chunks, devs, chunk_rows):
-                d["q"].copy_(hc["q"], non_blocking=True)
-                d["k"][:, rs].copy_(hc["k"], non_blocking=True)
-                d["v"][:, rs].copy_(hc["v"], non_blocking=True)
-            wd.copy_(W_host, non_blocking=True)
-            copied[i % 2].record(copy_stream)
+        jobs = []
+        for hc, d, rs in zip(host_chunks, devs, chunk_rows):
+            jobs += [(d["q"], hc["q"]), (d["k"][:, rs], hc["k"]), (d["v"][:, rs], hc["v"])]
+        jobs.append((wd, W_host))
+        for si_, cs in enumerate(h2d_streams):
+            with torch.cuda.stream(cs):
+                if i >= 2:
+                    cs.wait_event(freed[i % 2])  # step i - 2 is done with this set
+                for dst, src in jobs[si_::2]:
+                    dst.copy_(src, non_blocking=True)
+                copied[i % 2][si_].record(cs)
 
     def e2e_run(n_steps, start_event=None):
         if start_event is not None:
-            copy_stream.wait_event(start_event)
+            for cs in h2d_streams:
+                cs.wait_event(start_event)
         issue_copy(0)
         for i in range(n_steps):
             if i + 1 < n_steps:
                 issue_copy(i + 1)
-            stream.wait_event(copied[i % 2])
+            for ev in copied[i % 2]:
+                stream.wait_event(ev)
+            if i >= 2:
+                stream.wait_event(read_back[i % 2])  # step i - 2's outputs are on the host
             devs, wd = sets[i % 2]
             for Lr, d in zip(layers, devs):
                 Lr.dev = d
             wcur["W32"] = wd
+            ocur.update(outs[i % 2])
             step(False)
-            for n in ("L", "F"):
-                y_host[n].copy_(y[n], non_blocking=True)
-            dW_host.copy_(dW, non_blocking=True)
-            small_host.copy_(eps_all, non_blocking=True)
             freed[i % 2].record(stream)
+            computed[i % 2].record(stream)
+            with torch.cuda.stream(d2h_stream):
+                d2h_stream.wait_event(computed[i % 2])
+                o_ = outs[i % 2]
+                for n in ("L", "F"):
+                    y_host[n].copy_(o_["y"][n], non_blocking=True)
+                dW_host.copy_(o_["dW"], non_blocking=True)
+                small_host.copy_(o_["eps"], non_blocking=True)
+                read_back[i % 2].record(d2h_stream)
+        stream.wait_event(read_back[(n_steps - 1) % 2])  # the last step's outputs are read back
 
     e2e_steps = max(2, min(args.steps, 6))
     e2e_run(2)
@@ -1088,6 +1112,7 @@ def run_ours(args, world, rank, local):
     for Lr, d in zip(layers, sets[0][0]):
         Lr.dev = d
     wcur["W32"] = W32
+    ocur.update(outs[0])
     e2e_ms = reduce_over_ranks(e0.elapsed_time(e1) / e2e_steps, "max", dev)
     del sets, set1
 
