@@ -156,8 +156,7 @@ typedef struct {
  *   o_full     [B, Lq, H, d] out_dtype, lse_full [B, Lq, H] fp32   (both or neither)
  * An empty group yields O = 0 and L = -inf.  Compiled paths: bf16 in with
  * head_dim 128 (tcgen05 tensor cores, fp32 accumulation) and fp32 in with
- * head_dim 32/64/128 (tcgen05 kind::tf32 in three passes, hi/lo split of every
- * operand: fp32-accurate).  Outputs may not alias inputs.
+ * head_dim 32/64/128 (fp32 CUDA cores).  Outputs may not alias inputs.
  * Every K/V row that a group's 128-row tiles cover must hold finite values.
  *   workspace  >= ispa_attn_split_workspace_bytes(desc) bytes, 16-byte aligned
  *              (0 for fp32 inputs and for a prepared V; for bf16 inputs with

@@ -311,7 +311,7 @@ ispa_status ispa_attn_split(const ispa_attn_desc *desc, const void *q, const voi
     return launch_attn_tc(*desc, g, scale, q, k, v, o_loc, lse_loc, o_hist, lse_hist, o_full, lse_full, workspace,
                           (cudaStream_t)stream);
   }
-  return launch_attn_tf32(*desc, g, scale, (const float *)q, (const float *)k, (const float *)v, o_loc, lse_loc, o_hist,
+  return launch_attn_simt(*desc, g, scale, (const float *)q, (const float *)k, (const float *)v, o_loc, lse_loc, o_hist,
                           lse_hist, o_full, lse_full, (cudaStream_t)stream);
 }
 

@@ -59,10 +59,6 @@ ispa_status launch_absorb_weight(int D, int Dout, const void *W, ispa_dtype wdt,
 ispa_status launch_attn_simt(const ispa_attn_desc &d, const GroupRanges &g, float scale, const float *q,
                              const float *k, const float *v, void *o_loc, float *l_loc, void *o_hist,
                              float *l_hist, void *o_full, float *l_full, cudaStream_t s);
-// fp32 inputs on the tf32 tensor cores in three passes (attn_tf32.cu)
-ispa_status launch_attn_tf32(const ispa_attn_desc &d, const GroupRanges &g, float scale, const float *q,
-                             const float *k, const float *v, void *o_loc, float *l_loc, void *o_hist, float *l_hist,
-                             void *o_full, float *l_full, cudaStream_t s);
 // workspace: an fp16 copy of V (see attn_tc.cu) plus per-head scales; none
 // when V comes prepared (ispa_v16_prepare)
 size_t attn_tc_workspace_bytes(int B, int H, int Lkv, int v_layout);
