@@ -220,10 +220,12 @@ ispa_status ispa_v16_prepare(const ispa_attn_desc *desc, const void *v, int fram
  *   * S = Q8 K8^T and O = P8 V8 on the 8-bit tensor cores (fp32 accumulation);
  *   * per group an online softmax over 128-key tiles taken in the group's
  *     order, each key range's tiles starting at its first key rounded down to
- *     a multiple of 16: with t = S s_q s_k scale log2(e) and m the running
- *     maximum over the tiles seen, p = 2^(t - m + 8) <= 256 enters the product
- *     as e4m3(p) and the normaliser l as it is (fp32); O = acc s_v / l and
- *     L = (m - 8 + log2 l) ln 2; the groups are merged by their LSE.
+ *     a multiple of 16: with t = S s_q s_k scale log2(e) and a reference m
+ *     per query row -- the group's first tile maximum, moved to a later tile's
+ *     maximum only when that exceeds m by more than 2.75 (O and l rescaled
+ *     then) -- p = 2^(t - m + 6) <= 2^8.75 (below e4m3's 448) enters the
+ *     product as e4m3(p) and the normaliser l as it is (fp32); O = acc s_v / l
+ *     and L = (m - 6 + log2 l) ln 2; the groups are merged by their LSE.
  * ispa_kv8_bytes(desc): bytes of the prepared buffer for desc's K/V layout
  *   (K8 [B, kv_frames*tpf, H, 128] bytes, V8 transposed [B, H, 128, rows
  *   rounded up to 16] bytes, then the per-head scales); 0 for an invalid desc

@@ -5,11 +5,17 @@
 // one fp32 scale per (instance, head), S = Q K^T and O = P V on the 8-bit
 // tensor cores with fp32 accumulation, P in e4m3.  The scheme:
 //   * s_X = amax_X / 448 over the head's rows, codes e4m3(x * (448 / amax_X));
-//   * t = S s_q s_k scale log2(e); per group a running maximum m over the
-//     128-key tiles seen (O and the sum scaled by 2^(m_old - m_new) whenever it
-//     grows), p = 2^(t - m + 8) <= 256 (the weights of the bulk of the keys in
-//     e4m3's normal range), l += p in fp32, O += e4m3(p) V8;
-//   * O = O s_v / l, L = (m - 8 + log2 l) ln 2, the groups merged by their LSE.
+//   * t = S s_q s_k scale log2(e); per group and query row a reference m: the
+//     first 128-key tile's maximum, moved to a later tile's maximum only when
+//     that exceeds m by more than 2.75 (O and the sum then scaled by
+//     2^(m_old - m_new)); p = 2^(t - m + 6) <= 2^8.75 < 448 (finite in e4m3,
+//     the weights of the bulk of the keys in its normal range), l += p in
+//     fp32, O += e4m3(p) V8;
+//   * O = O s_v / l, L = (m - 6 + log2 l) ln 2, the groups merged by their LSE.
+// The softmax forms a tile's weights against the current reference and finds
+// the tile's maximum in the same pass; only when the maximum passes the
+// threshold (after the first tiles of a group, rarely) does it wait for the
+// previous PV, rescale O and form the weights again.
 // The tiles of a key range start at its first key rounded down to a multiple
 // of 16 (the 16-byte rule of the transposed V copy's TMA coordinate); keys of
 // a tile outside the range are masked.
@@ -64,7 +70,8 @@ constexpr int kTileBytes = 128 * 128;  // 128 rows x 128 bytes
 constexpr int kStagesK = 4, kStagesV = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS = 128, kColQ = 384, kColP = 416;
-constexpr float kPOffset = 8.0f;  // p = 2^(t - m + 8) <= 256
+constexpr float kPOffset = 6.0f;  // p = 2^(t - m + 6)
+constexpr float kTau = 2.75f;     // m moves when a tile's maximum exceeds it by more: p <= 2^8.75 < 448
 constexpr int kAlign = 16;        // tiles of a range start at a multiple of 16 keys
 
 size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -405,8 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.q_ready, 128);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.s_free[s], 128);
-      mbar_init(&sm.p_full[s], 128);
+      mbar_init(&sm.s_free[s], 4);  // one arrival per softmax warp
+      mbar_init(&sm.p_full[s], 4);
       mbar_init(&sm.pv_done[s], 1);
     }
     mbar_init(&sm.o_free, 128);
@@ -498,13 +505,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int jn = j + 2;
         if (jn < P.n_tiles) {  // S two tiles ahead, as soon as the softmax has read S_j
           ok = wait_parity(&sm.k_full[jn % kStagesK], (jn / kStagesK) & 1, P.err, abort, 52);
-          if (ok) ok = wait_parity_spin(&sm.s_free[j & 1], (uint32_t)(j >> 1) & 1, P.err, abort, 53);
+          if (ok) ok = wait_parity(&sm.s_free[j & 1], (uint32_t)(j >> 1) & 1, P.err, abort, 53);
           if (!ok) break;
           tc_fence_after();
           issue_s(jn);
         }
         ok = wait_parity(&sm.v_full[j % kStagesV], (j / kStagesV) & 1, P.err, abort, 54);
-        if (ok) ok = wait_parity_spin(&sm.p_full[j & 1], (uint32_t)(j >> 1) & 1, P.err, abort, 55);
+        if (ok) ok = wait_parity(&sm.p_full[j & 1], (uint32_t)(j >> 1) & 1, P.err, abort, 55);
         if (ok && j == P.n_loc_tiles) ok = wait_parity(&sm.o_free, 0, P.err, abort, 56);
         if (!ok) break;
         tc_fence_after();
@@ -570,61 +577,84 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + col_s + c * 32, sr[c]);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(&sm.s_free[j & 1]);  // S_{j+2} may overwrite the buffer now
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.s_free[j & 1]);  // S_{j+2} may overwrite the buffer now
       if (lo > 0 || hi < kTileK) {     // keys of the tile outside the range
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c < lo || c >= hi) sr[c >> 5][c & 31] = 0xff800000u;
       }
-      float mx[8];
+      // p = 2^(t - m_ref + 6); l in fp32; P8 = e4m3(p), four per column (pairs on
+      // the packed fp32 pipe: one FFMA2 and one FADD2 per two weights).  With
+      // track_max the tile's maximum score is taken in the same pass.
+      const float2 c2 = make_float2(c_log2, c_log2);
+      uint32_t pk[32];
+      auto weights = [&](float mref, bool track_max, float &mt) -> float {
+        const float2 nm2 = make_float2(kPOffset - mref, kPOffset - mref);
+        float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int t = 0; t < 8; ++t) mx[t] = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 128; c += 2)
-        mx[(c >> 1) & 7] = fmax3f(mx[(c >> 1) & 7], __uint_as_float(sr[c >> 5][c & 31]),
-                                  __uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]));
-      const float mt =
-          fmax3f(fmax3f(mx[0], mx[1], mx[2]), fmax3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * c_log2;
+        for (int c = 0; c < 32; ++c) {
+          const uint32_t *row = &sr[c >> 3][(4 * c) & 31];
+          const float s0 = __uint_as_float(row[0]), s1 = __uint_as_float(row[1]);
+          const float s2 = __uint_as_float(row[2]), s3 = __uint_as_float(row[3]);
+          if (track_max) {
+            mx[c & 3] = fmax3f(mx[c & 3], s0, s1);
+            mx[c & 3] = fmax3f(mx[c & 3], s2, s3);
+          }
+          const float2 x01 = ffma2f(make_float2(s0, s1), c2, nm2);
+          const float2 x23 = ffma2f(make_float2(s2, s3), c2, nm2);
+          const float2 p01 = make_float2(ex2f(x01.x), ex2f(x01.y));
+          const float2 p23 = make_float2(ex2f(x23.x), ex2f(x23.y));
+          ls[0] = fadd2f(ls[0], p01);
+          ls[1] = fadd2f(ls[1], p23);
+          pk[c] = e4m3x4(p01.x, p01.y, p23.x, p23.y);
+        }
+        if (track_max) mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c_log2;
+        return (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
+      };
+      float l_tile, mt = 0.f;
       if (grp_first) {
-        m_ref = mt;
-        l = 0.f;
-      } else if (__any_sync(0xffffffffu, mt > m_ref)) {
-        // the running maximum grows: O (after PV_{j-1}) and l scale by 2^(m_ref - m_new)
-        ok = wait_parity(&sm.pv_done[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1, P.err, abort, 62);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        tc_fence_after();
-        const float m_new = fmaxf(m_ref, mt);
-        const float f = ex2f(m_ref - m_new);
-        m_ref = m_new;
-        l *= f;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tmem_ld32(lane_base + kColO + c * 32, o);
-          tmem_wait_ld();
+        float mxs[8];
 #pragma unroll
-          for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * f);
-          tmem_st16(lane_base + kColO + c * 32, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
-          tmem_st16(lane_base + kColO + c * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
+        for (int t = 0; t < 8; ++t) mxs[t] = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; c += 2)
+          mxs[(c >> 1) & 7] = fmax3f(mxs[(c >> 1) & 7], __uint_as_float(sr[c >> 5][c & 31]),
+                                     __uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]));
+        m_ref = fmax3f(fmax3f(mxs[0], mxs[1], mxs[2]), fmax3f(mxs[3], mxs[4], mxs[5]), fmaxf(mxs[6], mxs[7])) *
+                c_log2;
+        l = 0.f;
+        l_tile = weights(m_ref, false, mt);
+      } else {
+        // weights against the current reference, the tile maximum alongside; the
+        // reference moves (and the pass is redone) only when the maximum exceeds
+        // it by more than kTau
+        l_tile = weights(m_ref, true, mt);
+        const bool moves = mt > m_ref + kTau;
+        if (__any_sync(0xffffffffu, moves)) {
+          // O (after PV_{j-1}) and l scale by 2^(m_ref - m_new)
+          ok = wait_parity(&sm.pv_done[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1, P.err, abort, 62);
+          if (!__all_sync(0xffffffffu, ok)) break;
+          tc_fence_after();
+          const float m_new = moves ? mt : m_ref;
+          const float f = ex2f(m_ref - m_new);
+          m_ref = m_new;
+          l *= f;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(lane_base + kColO + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int t = 0; t < 32; ++t) o[t] = __float_as_uint(__uint_as_float(o[t]) * f);
+            tmem_st16(lane_base + kColO + c * 32, *reinterpret_cast<uint32_t(*)[16]>(&o[0]));
+            tmem_st16(lane_base + kColO + c * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&o[16]));
+          }
+          l_tile = weights(m_ref, false, mt);
         }
       }
-      // p = 2^(t - m_ref + 8) in (0, 256]; l in fp32; P8 = e4m3(p), four per column
-      // (pairs on the packed fp32 pipe: one FFMA2 and one FADD2 per two weights)
-      const float2 c2 = make_float2(c_log2, c_log2), nm2 = make_float2(kPOffset - m_ref, kPOffset - m_ref);
-      uint32_t pk[32];
-      float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const uint32_t *row = &sr[c >> 3][(4 * c) & 31];
-        const float2 x01 = ffma2f(make_float2(__uint_as_float(row[0]), __uint_as_float(row[1])), c2, nm2);
-        const float2 x23 = ffma2f(make_float2(__uint_as_float(row[2]), __uint_as_float(row[3])), c2, nm2);
-        const float2 p01 = make_float2(ex2f(x01.x), ex2f(x01.y));
-        const float2 p23 = make_float2(ex2f(x23.x), ex2f(x23.y));
-        ls[0] = fadd2f(ls[0], p01);
-        ls[1] = fadd2f(ls[1], p23);
-        pk[c] = e4m3x4(p01.x, p01.y, p23.x, p23.y);
-      }
-      l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
+      l += l_tile;
       if (j >= 2) {  // PV_{j-2} has read this P buffer
         ok = wait_parity(&sm.pv_done[j & 1], (uint32_t)((j - 2) >> 1) & 1, P.err, abort, 63);
         if (!__all_sync(0xffffffffu, ok)) break;
@@ -633,7 +663,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_st16(lane_base + kColP + (uint32_t)(j & 1) * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sm.p_full[j & 1]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.p_full[j & 1]);
 
       if (!grp_last) continue;
       ok = wait_parity(&sm.pv_done[j & 1], (uint32_t)(j >> 1) & 1, P.err, abort, 64);

@@ -478,15 +478,24 @@ def local_projection_q8(shape, q, k, v, W_new: np.ndarray, fmt: int, scale: floa
 #  * scores in log2 units t = (q8 . k8) s_q s_k scale log2(e);
 #  * each group is taken in blocks of 128 keys in its order (the local group's
 #    sink range, then its current range; the history range), the blocks of a
-#    range starting at the 16-aligned key position at or below its first key; a
-#    running maximum m over the blocks seen so far (the product and the sum are
-#    scaled by 2^(m_old - m_new) when it grows); per block p = 2^(t - m + 8), so
-#    that p <= 256 and the weights of the bulk of the keys lie in e4m3's normal
-#    range; the sum l += p is kept exactly, the product acc += e4m3(p) v8;
-#  * O = acc s_v / l, L = (m - 8 + log2 l) ln 2; the two groups are merged by
+#    range starting at the 16-aligned key position at or below its first key;
+#  * a reference m per query row: the first block's maximum, then moved to a
+#    block's maximum only when that maximum exceeds m by more than TAU = 2.75
+#    (log2 units; the product and the sum are scaled by 2^(m_old - m_new) when
+#    it moves); per block p = 2^(t - m + 6), so that p <= 2^8.75 < 448 (e4m3's
+#    largest finite value) and the weights of the bulk of the keys lie in
+#    e4m3's normal range; the sum l += p is kept exactly, the product
+#    acc += e4m3(p) v8;
+#  * O = acc s_v / l, L = (m - 6 + log2 l) ln 2; the two groups are merged by
 #    their log-sum-exp as in lse_merge.
+# With the weights kept exact the result is softmax attention whatever m is;
+# the reference only decides where each weight falls on the e4m3 grid.  A
+# reference that follows the running maximum at every block (TAU = 0) needs an
+# offset of at most log2(448) and rescales O whenever any row's maximum grows,
+# which on long histories is most blocks; with TAU the reference settles after
+# the first blocks.
 # ---------------------------------------------------------------------------
-FP8_BLOCK, FP8_ALIGN, FP8_P_OFFSET = 128, 16, 8.0
+FP8_BLOCK, FP8_ALIGN, FP8_P_OFFSET, FP8_TAU = 128, 16, 6.0, 2.75
 
 
 def quantize_heads(x: np.ndarray):
@@ -530,38 +539,66 @@ def fp8_blocks(ranges) -> List[Tuple[int, int]]:
     return out
 
 
-def attend_group_fp8(t: np.ndarray, v8: np.ndarray, blocks, quantize_p: bool = True):
+def attend_group_fp8(t: np.ndarray, v8: np.ndarray, blocks, quantize_p: bool = True, tie_rel: float = 0.0):
     """Blockwise softmax of one group with e4m3 weights (see the reading above).
 
     t [n, Lkv] scores in log2 units (columns outside the group unused), v8
     [Lkv, d] dequantisation-free e4m3 codes of V, blocks from :func:`fp8_blocks`.
     Returns (acc / l [n, d] before the V scale, L in natural log [n]).
     quantize_p=False keeps the weights exact (the plain online softmax).
+
+    With tie_rel > 0 a third array [n, d] is returned: for the weights that lie
+    within a relative tie_rel of a rounding boundary of the e4m3 grid -- where a
+    weight computed in another precision may round to the neighbouring code --
+    the sum of (code step) |v8| / l, the most the output can move by those
+    roundings; +inf for a row where a block maximum lies within tie_rel of the
+    threshold that moves the reference (there the reference itself is a tie).
     """
     n, d = t.shape[0], v8.shape[1]
     if not blocks:
-        return np.zeros((n, d)), np.full(n, NEG_INF)
-    m = np.full(n, NEG_INF)
+        empty = (np.zeros((n, d)), np.full(n, NEG_INF))
+        return empty + (np.zeros((n, d)),) if tie_rel > 0 else empty
+    m = None
     l = np.zeros(n)
     acc = np.zeros((n, d))
+    amb = np.zeros((n, d))
+    undecided = np.zeros(n, bool)
     for lo, hi in blocks:
         tb = t[:, lo:hi]
-        m_new = np.maximum(m, tb.max(axis=1))
-        f = np.where(np.isneginf(m), 0.0, np.exp2(m - m_new))
-        acc *= f[:, None]
-        l *= f
-        m = m_new
+        bm = tb.max(axis=1)
+        if m is None:
+            m = bm
+        else:
+            if tie_rel > 0:  # the decision itself is a tie: any output of the row is admissible
+                undecided |= np.abs(bm - (m + FP8_TAU)) <= tie_rel * np.maximum(1.0, np.abs(bm))
+            m_new = np.where(bm > m + FP8_TAU, bm, m)
+            f = np.exp2(m - m_new)
+            acc *= f[:, None]
+            amb *= f[:, None]
+            l *= f
+            m = m_new
         p = np.exp2(tb - m[:, None] + FP8_P_OFFSET)
         l += p.sum(axis=1)
         acc += (e4m3_round(p) if quantize_p else p) @ v8[lo:hi]
-    return acc / l[:, None], (m - FP8_P_OFFSET + np.log2(l)) * math.log(2.0)
+        if tie_rel > 0:
+            step = np.abs(e4m3_round(p * (1.0 + tie_rel)) - e4m3_round(p * (1.0 - tie_rel)))
+            amb += step @ np.abs(v8[lo:hi])
+    out = (acc / l[:, None], (m - FP8_P_OFFSET + np.log2(l)) * math.log(2.0))
+    if tie_rel <= 0:
+        return out
+    amb = amb / l[:, None]
+    amb[undecided] = np.inf
+    return out + (amb,)
 
 
 def split_attention_fp8(shape, q, k, v, scale: float = None, rows: Sequence[int] = None,
-                        quantize_p: bool = True) -> Dict[str, np.ndarray]:
+                        quantize_p: bool = True, tie_rel: float = 0.0) -> Dict[str, np.ndarray]:
     """Two-group attention with fp8 e4m3 products (reading above); same outputs
     as :func:`split_attention`.  q, k, v hold the unquantised (bf16) values; the
-    per-head quantisation is part of the definition."""
+    per-head quantisation is part of the definition.  With tie_rel > 0 the
+    outputs also hold A_loc, A_hist, A_full [B, n, H, d]: how far each output may
+    move by weights that sit within tie_rel of an e4m3 rounding boundary (see
+    attend_group_fp8), after the V scale (A_full by the merge weights)."""
     d = q.shape[-1]
     scale = 1.0 / math.sqrt(d) if not scale else scale
     B, Lq, H, _ = q.shape
@@ -574,6 +611,8 @@ def split_attention_fp8(shape, q, k, v, scale: float = None, rows: Sequence[int]
     blk_hist = fp8_blocks(_runs(_hist_rows(shape)))
     out = {key: np.zeros((B, n, H, d)) for key in ("O_loc", "O_hist", "O_full")}
     out.update({key: np.zeros((B, n, H)) for key in ("L_loc", "L_hist", "L_full")})
+    if tie_rel > 0:
+        out.update({key: np.zeros((B, n, H, d)) for key in ("A_loc", "A_hist", "A_full")})
     log2e = 1.0 / math.log(2.0)
     for b in range(B):
         for h in range(H):
@@ -581,10 +620,15 @@ def split_attention_fp8(shape, q, k, v, scale: float = None, rows: Sequence[int]
             t = (q8[b, rows, h, :] @ k8[b, :, h, :].T) * c          # [n, Lkv]
             res = {}
             for name, blk in (("loc", blk_loc), ("hist", blk_hist)):
-                o, L = attend_group_fp8(t, v8[b, :, h, :], blk, quantize_p)
-                res[name] = (o * float(sv[b, h]), L)
+                r = attend_group_fp8(t, v8[b, :, h, :], blk, quantize_p, tie_rel)
+                res[name] = (r[0] * float(sv[b, h]), r[1])
+                if tie_rel > 0:
+                    out["A_" + name][b, :, h] = r[2] * float(sv[b, h])
             o_f, l_f = lse_merge(res["loc"][0], res["loc"][1], res["hist"][0], res["hist"][1])
             for name in ("loc", "hist"):
                 out["O_" + name][b, :, h], out["L_" + name][b, :, h] = res[name]
             out["O_full"][b, :, h], out["L_full"][b, :, h] = o_f, l_f
+            if tie_rel > 0:  # the merge weighs the allowances like the outputs
+                out["A_full"][b, :, h] = lse_merge(out["A_loc"][b, :, h], res["loc"][1],
+                                                   out["A_hist"][b, :, h], res["hist"][1])[0]
     return out

@@ -3,10 +3,15 @@ oracle's fp8 attention (per-head e4m3 scales, blockwise online softmax with
 e4m3 weights), and its distance from the exact attention of the bf16 inputs.
 
 Tolerance: the oracle follows the same definition in fp64, so the kernel
-differs from it only by fp32 arithmetic (scores, exponentials, sums) and the
-rare weight whose e4m3 rounding that moves across a rounding boundary (one
-code step, 2^-3 of that weight); max |dO| <= 1e-2 of each head's output RMS,
-as for the bf16 path, and LSE within 1e-3."""
+differs from it by fp32 arithmetic (scores, exponentials, sums) -- max |dO| <=
+1e-2 of each head's output RMS, as for the bf16 path, and LSE within 1e-3 --
+and by the weights that sit so close to a rounding boundary of the e4m3 grid
+that fp32 may round them to the neighbouring code.  The oracle reports how far
+those can move each output (split_attention_fp8's A_* at TIE_REL) and the bound
+adds it.  TIE_REL: the kernel forms p = 2^x with x = t - m + 6 in fp32 from
+scores accumulated in fp32 over 128 products; for |t| up to ~32 (log2 units)
+their error stays below 2^-19 |t|, so p is within a relative 2^-14 of the
+exact weight."""
 import dataclasses
 
 import numpy as np
@@ -60,8 +65,11 @@ def run_fp8(sh, data, out_dt=ispa.ISPA_F32, prepare=None):
     return {n: host(t) for n, t in o.items()}, {n: host(t) for n, t in l.items()}
 
 
+TIE_REL = 2.0 ** -14
+
+
 def check_against_oracle(sh, data, O, L, rows=None, tol=1e-2, bf16_out=False):
-    ref = orc.split_attention_fp8(sh, data["q"], data["k"], data["v"], rows=rows)
+    ref = orc.split_attention_fp8(sh, data["q"], data["k"], data["v"], rows=rows, tie_rel=TIE_REL)
     sel = slice(None) if rows is None else np.asarray(rows)
     for n in ("loc", "hist", "full"):
         got, r = O[n][:, sel], ref["O_" + n]
@@ -72,7 +80,7 @@ def check_against_oracle(sh, data, O, L, rows=None, tol=1e-2, bf16_out=False):
                     assert np.all(got[b, :, h] == 0), (n, b, h)
                     continue
                 rms = np.sqrt(np.mean(rr ** 2))
-                bound = tol * rms + (2.0 ** -8 * np.abs(rr) if bf16_out else 0.0)
+                bound = tol * rms + ref["A_" + n][b, :, h] + (2.0 ** -8 * np.abs(rr) if bf16_out else 0.0)
                 err = np.abs(got[b, :, h] - rr)
                 assert np.all(err <= bound), (n, b, h, float((err / rms).max()))
         assert_lse(L[n][:, sel], ref["L_" + n], 1e-3)
@@ -140,22 +148,22 @@ def test_fp8_post_switch_full_size_1p3b_sampled_rows():
     ev = {"q": data["q"], "k": orc.evict_history(sh, data["k"]).astype(np.float32),
           "v": orc.evict_history(sh, data["v"]).astype(np.float32)}
     O, L = run_fp8(es, ev, ispa.ISPA_BF16)
-    ref = orc.split_attention_fp8(es, ev["q"], ev["k"], ev["v"], rows=rows)
+    ref = orc.split_attention_fp8(es, ev["q"], ev["k"], ev["v"], rows=rows, tie_rel=TIE_REL)
     for b in range(sh.B):
         for h in range(sh.H):
             r = ref["O_loc"][b, :, h]
             err = np.abs(O["loc"][b, rows, h] - r)
-            assert np.all(err <= 1e-2 * np.sqrt(np.mean(r ** 2)) + 2.0 ** -8 * np.abs(r)), (b, h)
+            assert np.all(err <= 1e-2 * np.sqrt(np.mean(r ** 2)) + ref["A_loc"][b, :, h] + 2.0 ** -8 * np.abs(r)), (b, h)
     assert_lse(L["loc"][:, rows], ref["L_loc"], 1e-3)
     # F-layer: one group over every frame
     shF = dataclasses.replace(sh, sink_frames=sh.cur_begin, hist_begin=0, hist_end=0)
     O, L = run_fp8(shF, data, ispa.ISPA_BF16)
-    ref = orc.split_attention_fp8(shF, data["q"], data["k"], data["v"], rows=rows)
+    ref = orc.split_attention_fp8(shF, data["q"], data["k"], data["v"], rows=rows, tie_rel=TIE_REL)
     for b in range(sh.B):
         for h in range(sh.H):
             r = ref["O_loc"][b, :, h]
             err = np.abs(O["loc"][b, rows, h] - r)
-            assert np.all(err <= 1e-2 * np.sqrt(np.mean(r ** 2)) + 2.0 ** -8 * np.abs(r)), (b, h)
+            assert np.all(err <= 1e-2 * np.sqrt(np.mean(r ** 2)) + ref["A_loc"][b, :, h] + 2.0 ** -8 * np.abs(r)), (b, h)
     assert_lse(L["loc"][:, rows], ref["L_loc"], 1e-3)
 
 

@@ -850,19 +850,105 @@ def test_fp8_blocks_cover_each_range_in_aligned_128_key_windows():
 
 
 def test_fp8_weights_on_the_e4m3_grid_pass_exactly():
-    """p = 2^(t - m + 8): weights 2^0 .. 2^-14 relative to the maximum are e4m3 normals
-    after the offset; a weight of 1.125 * 2^-7 (2.25 after it) enters exactly."""
+    """p = 2^(t - m + 6): the block's maximum enters as 64, and a weight of
+    1.125 * 2^-7 relative to it (0.5625 after the offset) is an e4m3 normal and
+    enters exactly."""
     v8 = np.array([[1.0, -2.0], [3.0, 0.5]])
     t = np.array([[0.0, math.log2(1.125 * 2.0 ** -7)]])
     o, L = orc.attend_group_fp8(t, v8, [(0, 2)])
-    w = np.array([256.0, 2.25])
+    w = np.array([64.0, 0.5625])
     assert np.allclose(o[0], (w @ v8) / w.sum(), rtol=0, atol=1e-15)
     assert abs(L[0] - math.log(1.0 + 1.125 * 2.0 ** -7)) < 1e-15
 
 
+# Three blocks of one row: the second block's maximum is 2.5 above the first's
+# (within TAU = 2.75: the reference stays at 0), the third's is 3.0 above it (the
+# reference moves to 3 and the earlier sums scale by 2^-3).  Weights by hand:
+# block 1: 2^6 = 64; block 2: 2^8.5 = 362.04 -> e4m3 352 (grid step 32 in
+# [256, 512)), 2^5 = 32; block 3: 2^6 = 64.
+LAZY_T = np.array([[0.0, 2.5, -1.0, 3.0]])
+LAZY_V = np.array([[1.0, 0.0], [0.0, 1.0], [2.0, -1.0], [-1.0, 3.0]])
+LAZY_BLOCKS = [(0, 1), (1, 3), (3, 4)]
+
+
+def _lazy_expected():
+    acc = (64.0 * LAZY_V[0] + 352.0 * LAZY_V[1] + 32.0 * LAZY_V[2]) / 8.0 + 64.0 * LAZY_V[3]
+    l = (64.0 + 2.0 ** 8.5 + 32.0) / 8.0 + 64.0
+    return acc / l
+
+
+def test_fp8_reference_moves_only_past_the_threshold():
+    o, L = orc.attend_group_fp8(LAZY_T, LAZY_V, LAZY_BLOCKS)
+    assert np.allclose(o[0], _lazy_expected(), rtol=0, atol=1e-14)
+    # L keeps the exact weights: the log-sum-exp of the scores (log2 units)
+    assert abs(L[0] - math.log(float(np.sum(np.exp2(LAZY_T[0]))))) < 1e-14
+    # the largest weight the threshold admits stays below e4m3's 448
+    assert 2.0 ** (orc.FP8_P_OFFSET + orc.FP8_TAU) < 448.0
+
+
+def test_fp8_tie_allowance_covers_weights_on_a_rounding_boundary():
+    """Weights 64 and 42 (42 = halfway between the e4m3 codes 40 and 44, so the tie
+    rounds to even: 40): the allowance is the code step 4 times |v| over l = 106;
+    weights away from every boundary (the three-block example) have none."""
+    v8 = np.array([[1.0, -2.0], [3.0, 0.5]])
+    t = np.array([[0.0, math.log2(42.0 / 64.0)]])
+    o, _, amb = orc.attend_group_fp8(t, v8, [(0, 2)], tie_rel=2.0 ** -14)
+    assert np.allclose(o[0], (64.0 * v8[0] + 40.0 * v8[1]) / 106.0, rtol=0, atol=1e-14)
+    assert np.allclose(amb[0], 4.0 * np.abs(v8[1]) / 106.0, rtol=0, atol=1e-14)
+    # the other rounding of the tie lies at the edge of the allowance
+    assert np.allclose(np.abs((64.0 * v8[0] + 44.0 * v8[1]) / 106.0 - o[0]), amb[0], rtol=0, atol=1e-14)
+    _, _, amb = orc.attend_group_fp8(LAZY_T, LAZY_V, LAZY_BLOCKS, tie_rel=2.0 ** -14)
+    assert np.all(amb == 0)
+    # a block maximum within tie_rel of the threshold leaves the reference undecided
+    t = np.array([[0.0, 2.75], [0.0, 2.0]])
+    _, _, amb = orc.attend_group_fp8(t, v8, [(0, 1), (1, 2)], tie_rel=2.0 ** -14)
+    assert np.all(np.isinf(amb[0])) and np.all(np.isfinite(amb[1]))
+
+
+def test_fp8_tie_allowance_bounds_every_rounding_of_perturbed_weights():
+    """Scores moved by a relative 2^-16 give, through the oracle itself, outputs
+    that stay within the allowance computed at tie_rel = 2^-14 (brute force over
+    seeded perturbations of a small layout)."""
+    sh = FP8_LAYOUTS[0]
+    data = si.iid_qkv(sh, "bf16", ("pin", "fp8tie"))
+    q8, sq = orc.quantize_heads(data["q"])
+    k8, sk = orc.quantize_heads(data["k"])
+    v8, _ = orc.quantize_heads(data["v"])
+    blk = orc.fp8_blocks(orc._runs(orc._hist_rows(sh)))
+    g = np.random.default_rng(11)
+    for h in range(sh.H):
+        c = float(sq[0, h]) * float(sk[0, h]) / math.sqrt(sh.d) / math.log(2.0)
+        t = (q8[0, :, h, :] @ k8[0, :, h, :].T) * c
+        o, _, amb = orc.attend_group_fp8(t, v8[0, :, h, :], blk, tie_rel=2.0 ** -14)
+        for _ in range(5):
+            tp = t + np.log2(1.0 + g.uniform(-2.0 ** -16, 2.0 ** -16, t.shape))
+            op, _ = orc.attend_group_fp8(tp, v8[0, :, h, :], blk)
+            # the exact weights move by 2^-16 too: their own share of the difference
+            assert np.all(np.abs(op - o) <= amb + 2.0 ** -15 * np.abs(o) + 1e-12)
+
+
+def test_mutant_fp8_reference_following_every_maximum_is_caught():
+    """A reference that follows the running maximum at every block rounds the
+    second block's weights at another place of the grid (64 and 2^2.5 -> 5.5)."""
+    def every_block(t, v8, blocks):
+        n, d = t.shape[0], v8.shape[1]
+        m, l, acc = np.full(n, -np.inf), np.zeros(n), np.zeros((n, d))
+        for lo, hi in blocks:
+            tb = t[:, lo:hi]
+            m_new = np.maximum(m, tb.max(axis=1))
+            f = np.where(np.isneginf(m), 0.0, np.exp2(m - m_new))
+            acc, l, m = acc * f[:, None], l * f, m_new
+            p = np.exp2(tb - m[:, None] + orc.FP8_P_OFFSET)
+            l += p.sum(axis=1)
+            acc += orc.e4m3_round(p) @ v8[lo:hi]
+        return acc / l[:, None]
+    assert not np.allclose(every_block(LAZY_T, LAZY_V, LAZY_BLOCKS)[0], _lazy_expected(), rtol=0, atol=1e-6)
+
+
 def test_fp8_weight_rounding_stays_within_its_bound():
     """With e4m3 weights the output moves by at most 2^-4 of sum_j w_j |v_j| (normal
-    weights) plus 2^-10 per subnormal weight over l >= 2^8; L is unchanged (the
+    weights) plus 2^-10 per subnormal weight over l >= 2^6 (the key that set the
+    reference weighs 2^6); L is unchanged (the
     normaliser keeps the exact weights); and the rounding is really applied."""
     for i, sh in enumerate(FP8_LAYOUTS):
         data = si.iid_qkv(sh, "bf16", ("pin", "fp8b", i))
@@ -879,7 +965,7 @@ def test_fp8_weight_rounding_stays_within_its_bound():
                     w = np.exp(s - s.max(axis=1, keepdims=True))
                     w /= w.sum(axis=1, keepdims=True)
                     av = np.abs(dq["v"][b, rows, h])
-                    bound = 2.0 ** -4 * (w @ av) + 2.0 ** -18 * av.sum(axis=0)[None, :] + 1e-12
+                    bound = 2.0 ** -4 * (w @ av) + 2.0 ** -16 * av.sum(axis=0)[None, :] + 1e-12
                     err = np.abs(got["O_" + name][b, :, h] - exact["O_" + name][b, :, h])
                     assert np.all(err <= bound), (i, name, float((err - bound).max()))
                     moved = max(moved, float(err.max()))
@@ -904,7 +990,7 @@ def test_mutant_fp8_without_the_weight_offset_is_caught():
     v8 = np.array([[1.0, -2.0], [3.0, 0.5]])
     t = np.array([[0.0, math.log2(1.125 * 2.0 ** -7)]])
     o, _ = no_offset(t, v8, [(0, 2)])
-    w = np.array([256.0, 2.25])
+    w = np.array([64.0, 0.5625])
     assert not np.allclose(o[0], (w @ v8) / w.sum(), rtol=0, atol=1e-15)
 
 
