@@ -273,25 +273,26 @@ struct SmemLayout8 {
   uint64_t o_free, drain;
   uint32_t tmem_base;
   int abort;
+  int rng[8];  // range begins [0,3), ends [3,6), count [6]: read by the tile walks
 };
 
 constexpr int kSmemBytes8 = sizeof(SmemLayout8) + 1024;
 
 // Tile walk over the ranges: each range's tiles start at its first key rounded
 // down to a multiple of 16; lo / hi are the tile's valid columns.
-struct TileIter8 {
+struct TileIter8 {  // the ranges come from shared memory (copied from the parameters at the start)
   int range, t0;
-  __device__ void start(const AttnParams8 &P) {
+  __device__ void start(const int *rng) {
     range = 0;
-    t0 = P.n_ranges > 0 ? P.r_begin[0] - P.r_begin[0] % kAlign : 0;
+    t0 = rng[6] > 0 ? rng[0] - rng[0] % kAlign : 0;
   }
-  __device__ int lo(const AttnParams8 &P) const { return max(0, P.r_begin[range] - t0); }
-  __device__ int hi(const AttnParams8 &P) const { return min(kTileK, P.r_end[range] - t0); }
-  __device__ void next(const AttnParams8 &P) {
+  __device__ int lo(const int *rng) const { return max(0, rng[range] - t0); }
+  __device__ int hi(const int *rng) const { return min(kTileK, rng[3 + range] - t0); }
+  __device__ void next(const int *rng) {
     t0 += kTileK;
-    if (t0 >= P.r_end[range]) {
+    if (t0 >= rng[3 + range]) {
       ++range;
-      if (range < P.n_ranges) t0 = P.r_begin[range] - P.r_begin[range] % kAlign;
+      if (range < rng[6]) t0 = rng[range] - rng[range] % kAlign;
     }
   }
 };
@@ -419,6 +420,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.o_free, 128);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
+    for (int r = 0; r < 3; ++r) {
+      sm.rng[r] = P.r_begin[r];
+      sm.rng[3 + r] = P.r_end[r];
+    }
+    sm.rng[6] = P.n_ranges;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -441,8 +447,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint64_t *empty = is_k ? sm.k_empty : sm.v_empty;
       uint32_t pend = 0, ph_bits = 0;
       TileIter8 it;
-      it.start(P);
-      for (int j = 0; j < P.n_tiles; ++j, it.next(P)) {
+      it.start(sm.rng);
+      for (int j = 0; j < P.n_tiles; ++j, it.next(sm.rng)) {
         const int st = j % n_stages;
         const uint32_t ph = (j / n_stages) & 1;
         if (!wait_parity(&empty[st], ph ^ 1, P.err, abort, is_k ? 41 : 42)) break;
@@ -563,11 +569,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     float m_ref = 0.f, l = 0.f, L_loc = -INFINITY;
     TileIter8 it;
-    it.start(P);
-    for (int j = 0; j < P.n_tiles; ++j, it.next(P)) {
+    it.start(sm.rng);
+    for (int j = 0; j < P.n_tiles; ++j, it.next(sm.rng)) {
       const bool grp_first = (j == 0) || (j == P.n_loc_tiles);
       const bool grp_last = (j == P.n_loc_tiles - 1) || (j == P.n_tiles - 1);
-      const int lo = it.lo(P), hi = it.hi(P);
+      const int lo = it.lo(sm.rng), hi = it.hi(sm.rng);
       const uint32_t col_s = kColS + (uint32_t)(j & 1) * 128;
       bool ok = wait_parity_spin(&sm.s_full[j & 1], (uint32_t)(j >> 1) & 1, P.err, abort, 61);
       if (!__all_sync(0xffffffffu, ok)) break;

@@ -339,23 +339,26 @@ struct SmemLayout {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  int rng[8];  // range begins [0,3), ends [3,6), count [6]: read by the tile walks
 };
 
 constexpr int kSmemBytes = sizeof(SmemLayout) + 1024;
 
 // Walks the tile sequence: local ranges first, then history.
+// The ranges come from shared memory (copied from the parameters at the start):
+// an indexed load of a kernel parameter sat on the softmax's per-tile path.
 struct TileIter {
   int range, t0;
-  __device__ void start(const AttnParams &P) {
+  __device__ void start(const int *rng) {
     range = 0;
-    t0 = P.n_ranges > 0 ? P.r_begin[0] : 0;
+    t0 = rng[6] > 0 ? rng[0] : 0;
   }
-  __device__ int valid(const AttnParams &P) const { return min(kTileK, P.r_end[range] - t0); }
-  __device__ void next(const AttnParams &P) {
+  __device__ int valid(const int *rng) const { return min(kTileK, rng[3 + range] - t0); }
+  __device__ void next(const int *rng) {
     t0 += kTileK;
-    if (t0 >= P.r_end[range]) {
+    if (t0 >= rng[3 + range]) {
       ++range;
-      if (range < P.n_ranges) t0 = P.r_begin[range];
+      if (range < rng[6]) t0 = rng[range];
     }
   }
 };
@@ -474,6 +477,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.o_free, 128);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
+    for (int r = 0; r < 3; ++r) {
+      sm.rng[r] = P.r_begin[r];
+      sm.rng[3 + r] = P.r_end[r];
+    }
+    sm.rng[6] = P.n_ranges;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -497,8 +505,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int x0 = h * kD;
       uint32_t pend = 0, ph_bits = 0;
       TileIter it;
-      it.start(P);
-      for (int j = 0; j < P.n_tiles; ++j, it.next(P)) {
+      it.start(sm.rng);
+      for (int j = 0; j < P.n_tiles; ++j, it.next(sm.rng)) {
         const int st = j % n_stages;
         const uint32_t ph = (j / n_stages) & 1;
         if (!wait_parity(&empty[st], ph ^ 1, P.err, abort, is_k ? 11 : 12)) break;
@@ -617,11 +625,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     float m_ref = 0.f, l = 0.f, L_loc = -INFINITY;
     TileIter it;
-    it.start(P);
-    for (int j = 0; j < P.n_tiles; ++j, it.next(P)) {
+    it.start(sm.rng);
+    for (int j = 0; j < P.n_tiles; ++j, it.next(sm.rng)) {
       const bool grp_first = (j == 0) || (j == P.n_loc_tiles);
       const bool grp_last = (j == P.n_loc_tiles - 1) || (j == P.n_tiles - 1);
-      const int n_valid = it.valid(P);
+      const int n_valid = it.valid(sm.rng);
       const uint32_t col_s = kColS + (uint32_t)(j & 1) * 128;
       bool ok = wait_parity_spin(&sm.s_full[j & 1], (uint32_t)(j >> 1) & 1, P.err, abort, 31);
       if (!__all_sync(0xffffffffu, ok)) break;
