@@ -191,3 +191,31 @@ def test_fp8_local_projection_equals_attention_then_product():
     ispa.ispa_gemm_bf16(sh.B * sh.Lq, D, D, o.reshape(sh.B * sh.Lq, D), W, y2, ispa.ISPA_F32)
     ispa.ispa_check_device_error()
     assert torch.equal(y.reshape(-1, D), y2)
+
+
+def test_fp8_post_switch_full_size_14b_sampled_rows():
+    """The F-layer in fp8 at the 14B size: 40 heads, all 102 960 keys of a drift
+    history as one group, 1480 query tiles; sampled rows of two heads (the first
+    and the last: the per-head scales make heads independent) against the fp8
+    oracle of those heads."""
+    sh = si.SHAPE_14B
+    key = ("gpu", "fp8-14b")
+    prefix = si.drift_layer_kv(sh, "bf16", 0, key)
+    cq = si.chunk_qkv(sh, "bf16", 0, 0, key)
+    data = {"q": cq["q"], "k": si.assemble_kv(prefix["k"], cq["k"], sh),
+            "v": si.assemble_kv(prefix["v"], cq["v"], sh)}
+    del prefix
+    shF = dataclasses.replace(sh, sink_frames=sh.cur_begin, hist_begin=0, hist_end=0)
+    O, L = run_fp8(shF, data, ispa.ISPA_BF16)
+    heads = [0, sh.H - 1]
+    sub = {n: np.ascontiguousarray(data[n][:, :, heads]) for n in ("q", "k", "v")}
+    del data
+    rows = np.r_[0, 1, 127, 128, 2339, 4608:4680:24, 4679]
+    ref = orc.split_attention_fp8(dataclasses.replace(shF, H=len(heads)), sub["q"], sub["k"], sub["v"], rows=rows,
+                                  tie_rel=TIE_REL)
+    for b in range(sh.B):
+        for x, h in enumerate(heads):
+            r = ref["O_loc"][b, :, x]
+            err = np.abs(O["loc"][b, rows, h] - r)
+            assert np.all(err <= 1e-2 * np.sqrt(np.mean(r ** 2)) + ref["A_loc"][b, :, x] + 2.0 ** -8 * np.abs(r)), (b, h)
+    assert_lse(L["loc"][:, rows][:, :, heads], ref["L_loc"], 1e-3)
