@@ -219,6 +219,9 @@ __device__ __forceinline__ void store_acc_t(TileT &T, const float acc[4][4]) {
 }
 
 constexpr int kFactorThreads = 256;
+// Steps with at least this many trailing block rows run as two launches (panel,
+// update); below it the fused step, whose single launch is shorter on the chain.
+constexpr int kTwoLaunchRows = 32;
 constexpr int kFactorBcast = 2 * 8 * NB;  // floats of the factor routine's broadcast buffers (two generations)
 
 // Inverse m (lower triangular) of the Cholesky factor of the symmetric 4 x 4
@@ -479,6 +482,96 @@ __global__ void __launch_bounds__(kFactorThreads) chol_step_kernel(int Dp, int k
   if (i == k + 1) {
     // the next diagonal block: factor and invert it for the next launch
     // (nothing reads the tile itself again, so it is not stored)
+    __syncthreads();  // all reads of sX and sY are done
+    float *S = &sY[0][0];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+      *reinterpret_cast<float4 *>(S + (4 * ty + a) * NB + 4 * tx) =
+          make_float4(aij[a][0], aij[a][1], aij[a][2], aij[a][3]);
+    __syncthreads();
+    factor_invert_tile(S, &sX[0][0], Linv + (long long)(k + 1) * NB * NB, (k + 1) * NB, flag, err);
+  } else {
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+      *reinterpret_cast<float4 *>(tile + (long long)(4 * ty + a) * ld + 4 * tx) =
+          make_float4(aij[a][0], aij[a][1], aij[a][2], aij[a][3]);
+  }
+}
+
+// Loads the row-major 64 x 64 tile at src into T layout transposed: element
+// (row, col) of src becomes element (col, row) of the tile.
+__device__ __forceinline__ void load_tile_tt(TileT &T, const float *__restrict__ src, long long ld) {
+  const int t = threadIdx.x, c = t & 15;
+#pragma unroll
+  for (int pass = 0; pass < 4; ++pass) {
+    const int q = (t >> 4) + 16 * pass;
+    *reinterpret_cast<float4 *>(&T[q][tgrp(c, q)]) = *reinterpret_cast<const float4 *>(src + (long long)q * ld + 4 * c);
+  }
+}
+
+// Block step k in two launches, for steps with many trailing block rows: the
+// fused step above forms each panel tile once per trailing tile that needs it
+// (three 64^3 products per CTA, two of them repeated across a block row); here
+// chol_panel_kernel forms each L_ik once, and chol_update_kernel applies
+// A_ij -= L_ik L_jk^T with one product per CTA.
+// Panel: one CTA per block row i > k; writes upper tile (k, i) = L_ik^T.
+__global__ void __launch_bounds__(kFactorThreads) chol_panel_kernel(int Dp, int k, float *M, const float *Linv) {
+  __shared__ __align__(16) TileT sX;
+  __shared__ __align__(16) TileT sL;
+  const int i = k + 1 + blockIdx.x;
+  const long long ld = Dp;
+  load_tile_t(sX, M + (long long)i * NB * ld + k * NB, ld);
+  load_tile_t(sL, Linv + (long long)k * NB * NB, NB);
+  __syncthreads();
+  float p[4][4];
+  tile_xyt(sX, sL, p);
+  __syncthreads();
+  store_acc_t(sX, p);
+  __syncthreads();
+  const int t = threadIdx.x;
+#pragma unroll
+  for (int pass = 0; pass < 4; ++pass) {  // row q of the upper tile is column q of L_ik
+    const int q = (t >> 4) + 16 * pass, c = t & 15;
+    const float4 v = *reinterpret_cast<const float4 *>(&sX[q][tgrp(c, q)]);
+    *reinterpret_cast<float4 *>(M + (long long)(k * NB + q) * ld + i * NB + 4 * c) = v;
+  }
+}
+
+// Update: one CTA per trailing tile (i, j), j <= i, numbered as in
+// chol_step_kernel (block 0 is the next diagonal tile, which it then factors and
+// inverts for the next step).  Reads upper tiles (k, i), (k, j) and tile (i, j).
+__global__ void __launch_bounds__(kFactorThreads) chol_update_kernel(int Dp, int k, float *M, float *Linv, int *flag,
+                                                                      DevErr err) {
+  __shared__ __align__(16) TileT sX;
+  __shared__ __align__(16) TileT sY;
+  const int t = threadIdx.x, ty = t >> 4, tx = t & 15;
+  const int lin = blockIdx.x;
+  int ii = (int)((sqrtf(8.f * lin + 1.f) - 1.f) * 0.5f);
+  while ((ii + 1) * (ii + 2) / 2 <= lin) ++ii;
+  while (ii * (ii + 1) / 2 > lin) --ii;
+  const int i = k + 1 + ii, j = k + 1 + (lin - ii * (ii + 1) / 2);
+  const bool diag = i == j;
+  const long long ld = Dp;
+  float *tile = M + (long long)i * NB * ld + j * NB;
+  load_tile_tt(sX, M + (long long)k * NB * ld + i * NB, ld);  // L_ik
+  if (!diag) load_tile_tt(sY, M + (long long)k * NB * ld + j * NB, ld);  // L_jk
+  float aij[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const float4 v = *reinterpret_cast<const float4 *>(tile + (long long)(4 * ty + a) * ld + 4 * tx);
+    aij[a][0] = v.x;
+    aij[a][1] = v.y;
+    aij[a][2] = v.z;
+    aij[a][3] = v.w;
+  }
+  __syncthreads();
+  float upd[4][4];
+  tile_xyt(sX, diag ? sX : sY, upd);
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) aij[a][b] -= upd[a][b];
+  if (i == k + 1) {
     __syncthreads();  // all reads of sX and sY are done
     float *S = &sY[0][0];
 #pragma unroll
@@ -933,8 +1026,14 @@ ispa_status launch_ridge(int D, int Dout, const float *G, const float *C, const 
   note_launch(3);
   for (int k = 0; k + 1 < nb; ++k) {
     const int m = nb - k - 1;
-    chol_step_kernel<<<m * (m + 1) / 2, kFactorThreads, 0, s>>>(Dp, k, w.M, w.Linv, w.flag, err);
-    note_launch();
+    if (m >= kTwoLaunchRows) {  // many trailing tiles: panel once, then one product per tile
+      chol_panel_kernel<<<m, kFactorThreads, 0, s>>>(Dp, k, w.M, w.Linv);
+      chol_update_kernel<<<m * (m + 1) / 2, kFactorThreads, 0, s>>>(Dp, k, w.M, w.Linv, w.flag, err);
+      note_launch(2);
+    } else {
+      chol_step_kernel<<<m * (m + 1) / 2, kFactorThreads, 0, s>>>(Dp, k, w.M, w.Linv, w.flag, err);
+      note_launch();
+    }
   }
   if (nb > 1) {
     upper_to_lower_kernel<<<nb * (nb - 1) / 2, 256, 0, s>>>(Dp, w.M);
