@@ -1100,7 +1100,10 @@ def run_ours(args, world, rank, local):
                 read_back[i % 2].record(d2h_stream)
         stream.wait_event(read_back[(n_steps - 1) % 2])  # the last step's outputs are read back
 
-    e2e_steps = max(2, min(args.steps, 6))
+    # as many steps as the device-timed run: the first step's copy in and the last
+    # step's read-back are not overlapped with any compute, so few steps would
+    # time the pipeline's fill and drain rather than its rate
+    e2e_steps = max(2, args.steps)
     e2e_run(2)
     torch.cuda.synchronize(dev)
     barrier(dev)
@@ -1411,6 +1414,21 @@ def run_sweep_only(args):
     return 0
 
 
+def run_solve_only(args):
+    """The ridge solve alone at width --solve-d from statistics of 2 D rows (graph-timed)."""
+    import torch
+
+    import kv_cache_compression_two_b200 as ispa
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(stream)
+    D = args.solve_d
+    ms = solve_ms_at(ispa, torch, stream, dev, D, 2 * D, reps=max(1, args.steps))
+    print(json.dumps({"kernel": "ridge_solve", "D": D, "Dout": D, "ms": ms}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1422,10 +1440,11 @@ def main(argv=None):
     ap.add_argument("--kv8", action="store_true", help="--only attn: the fp8 attention on a prepared fp8 K/V")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the 14B layer, the 30-layer model and the sweep (components outside the timed steps)")
-    ap.add_argument("--only", choices=["step", "attn", "proj", "parts", "sweep"], default="step",
+    ap.add_argument("--only", choices=["step", "attn", "proj", "parts", "sweep", "solve"], default="step",
                     help="attn: only the split-attention launches; proj: only the post-switch projection "
                          "(bf16, e4m3, int8 products); parts: the merge, the statistics and one solve; "
-                         "all for profiling, printing their timing")
+                         "solve: the ridge solve at --solve-d; all for profiling, printing their timing")
+    ap.add_argument("--solve-d", type=int, default=5120, help="--only solve: the width D = Dout")
     args = ap.parse_args(argv)
     if args.only == "proj":
         return run_proj_only(args)
@@ -1435,6 +1454,8 @@ def main(argv=None):
         return run_attn_only(args)
     if args.only == "sweep":
         return run_sweep_only(args)
+    if args.only == "solve":
+        return run_solve_only(args)
 
     if args.impl == "reference":
         world, rank, _ = dist_env()
