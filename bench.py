@@ -1070,6 +1070,25 @@ def run_ours(args, world, rank, local):
                     dst.copy_(src, non_blocking=True)
                 copied[i % 2][si_].record(cs)
 
+    # The step's calls are captured once per buffer set into a CUDA graph, as a
+    # serving loop would do: replaying it costs no per-call host work, which
+    # issued eagerly from Python (about 70 library calls a step) would otherwise
+    # pace the device.
+    graphs_e2e = []
+    for i in range(2):
+        devs, wd = sets[i]
+        for Lr, d in zip(layers, devs):
+            Lr.dev = d
+        wcur["W32"] = wd
+        ocur.update(outs[i])
+        step(False)
+        torch.cuda.synchronize(dev)
+        g_ = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_, stream=stream, capture_error_mode="thread_local"):
+            step(False)
+        graphs_e2e.append(g_)
+    torch.cuda.set_stream(stream)
+
     def e2e_run(n_steps, start_event=None):
         if start_event is not None:
             for cs in h2d_streams:
@@ -1082,12 +1101,7 @@ def run_ours(args, world, rank, local):
                 stream.wait_event(ev)
             if i >= 2:
                 stream.wait_event(read_back[i % 2])  # step i - 2's outputs are on the host
-            devs, wd = sets[i % 2]
-            for Lr, d in zip(layers, devs):
-                Lr.dev = d
-            wcur["W32"] = wd
-            ocur.update(outs[i % 2])
-            step(False)
+            graphs_e2e[i % 2].replay()
             freed[i % 2].record(stream)
             computed[i % 2].record(stream)
             with torch.cuda.stream(d2h_stream):
@@ -1117,7 +1131,34 @@ def run_ours(args, world, rank, local):
     wcur["W32"] = W32
     ocur.update(outs[0])
     e2e_ms = reduce_over_ranks(e0.elapsed_time(e1) / e2e_steps, "max", dev)
-    del sets, set1
+    # the transfers alone, without the compute: the floor the end-to-end step
+    # can reach (host->device on the two copy streams, device->host on its own)
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    for cs in h2d_streams:
+        cs.wait_event(c0)
+    for i in range(e2e_steps):
+        issue_copy(i)
+    for ev in copied[(e2e_steps - 1) % 2] + copied[e2e_steps % 2]:
+        stream.wait_event(ev)
+    c1.record(stream)
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(d2h_stream):
+        d2h_stream.wait_event(c1)
+        d0.record(d2h_stream)
+        for i in range(e2e_steps):
+            o_ = outs[i % 2]
+            for n in ("L", "F"):
+                y_host[n].copy_(o_["y"][n], non_blocking=True)
+            dW_host.copy_(o_["dW"], non_blocking=True)
+            small_host.copy_(o_["eps"], non_blocking=True)
+        d1.record(d2h_stream)
+    torch.cuda.synchronize(dev)
+    extra["e2e_transfers"] = {"h2d_ms_per_step": c0.elapsed_time(c1) / e2e_steps,
+                              "d2h_ms_per_step": d0.elapsed_time(d1) / e2e_steps,
+                              "h2d_gb_s": h2d * e2e_steps / (c0.elapsed_time(c1) * 1e-3) / 1e9,
+                              "d2h_gb_s": d2h * e2e_steps / (d0.elapsed_time(d1) * 1e-3) / 1e9}
+    del sets, set1, graphs_e2e
 
     # ---- the other workloads (outside the timed steps): the 14B-shaped layer,
     # the 30-layer 1.3B model through its switch, and the history / ISPA-x /

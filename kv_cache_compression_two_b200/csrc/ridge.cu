@@ -426,6 +426,7 @@ __global__ void __launch_bounds__(kFactorThreads) chol_first_kernel(int Dp, cons
 // tiles (k, i) and Linv_{k+1}, so no CTA reads what another CTA writes.
 __global__ void __launch_bounds__(kFactorThreads) chol_step_kernel(int Dp, int k, float *M, float *Linv, int *flag,
                                                                     DevErr err) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ __align__(16) TileT sX;
   __shared__ __align__(16) TileT sY;
   __shared__ __align__(16) TileT sL;
@@ -516,6 +517,7 @@ __device__ __forceinline__ void load_tile_tt(TileT &T, const float *__restrict__
 // A_ij -= L_ik L_jk^T with one product per CTA.
 // Panel: one CTA per block row i > k; writes upper tile (k, i) = L_ik^T.
 __global__ void __launch_bounds__(kFactorThreads) chol_panel_kernel(int Dp, int k, float *M, const float *Linv) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ __align__(16) TileT sX;
   __shared__ __align__(16) TileT sL;
   const int i = k + 1 + blockIdx.x;
@@ -542,6 +544,7 @@ __global__ void __launch_bounds__(kFactorThreads) chol_panel_kernel(int Dp, int 
 // inverts for the next step).  Reads upper tiles (k, i), (k, j) and tile (i, j).
 __global__ void __launch_bounds__(kFactorThreads) chol_update_kernel(int Dp, int k, float *M, float *Linv, int *flag,
                                                                       DevErr err) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ __align__(16) TileT sX;
   __shared__ __align__(16) TileT sY;
   const int t = threadIdx.x, ty = t >> 4, tx = t & 15;
@@ -1026,12 +1029,29 @@ ispa_status launch_ridge(int D, int Dout, const float *G, const float *C, const 
   note_launch(3);
   for (int k = 0; k + 1 < nb; ++k) {
     const int m = nb - k - 1;
+    // Programmatic dependent launch: a step's grid is set up while the previous
+    // step drains (its last CTA is the diagonal factor); each step kernel waits
+    // (griddepcontrol.wait) for the previous grid before reading anything.
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kFactorThreads);
+    cfg.stream = s;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
     if (m >= kTwoLaunchRows) {  // many trailing tiles: panel once, then one product per tile
-      chol_panel_kernel<<<m, kFactorThreads, 0, s>>>(Dp, k, w.M, w.Linv);
-      chol_update_kernel<<<m * (m + 1) / 2, kFactorThreads, 0, s>>>(Dp, k, w.M, w.Linv, w.flag, err);
+      cfg.gridDim = dim3(m);
+      cudaError_t le = cudaLaunchKernelEx(&cfg, chol_panel_kernel, Dp, k, w.M, (const float *)w.Linv);
+      if (le != cudaSuccess) return cuda_status(le, "ridge factor panel launch");
+      cfg.gridDim = dim3(m * (m + 1) / 2);
+      le = cudaLaunchKernelEx(&cfg, chol_update_kernel, Dp, k, w.M, w.Linv, w.flag, err);
+      if (le != cudaSuccess) return cuda_status(le, "ridge factor update launch");
       note_launch(2);
     } else {
-      chol_step_kernel<<<m * (m + 1) / 2, kFactorThreads, 0, s>>>(Dp, k, w.M, w.Linv, w.flag, err);
+      cfg.gridDim = dim3(m * (m + 1) / 2);
+      const cudaError_t le = cudaLaunchKernelEx(&cfg, chol_step_kernel, Dp, k, w.M, w.Linv, w.flag, err);
+      if (le != cudaSuccess) return cuda_status(le, "ridge factor step launch");
       note_launch();
     }
   }
