@@ -54,6 +54,9 @@
 //     P_{j+1}, so the wait cannot alias.  The same barriers free P buffers.
 //   * At the end of the local group the epilogue reads O after PV of that tile
 //     and releases it (o_free) before the first history PV starts O afresh.
+//   * s_free and p_full count one arrival per softmax warp: lane 0 arrives
+//     after the warp's tcgen05.wait (the load, or the store, of all 32 lanes
+//     has completed), a tcgen05 fence and a __syncwarp.
 #include <algorithm>
 
 #include <cuda_fp8.h>
