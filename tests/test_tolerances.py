@@ -68,3 +68,21 @@ def test_fp8_kernel_weights_stay_within_the_tie_tolerance_of_the_oracle():
                 rel = np.abs(np.exp2(x32[keep] - x64[keep]) - 1.0)
                 worst = max(worst, float(rel.max()))
     assert worst < TIE_REL / 4, worst
+
+
+def test_bf16_projection_error_model_sits_well_inside_its_bound():
+    """The post-switch projection y = A_loc (W + dW) runs in bf16 (both operands
+    rounded to bf16, fp32 accumulation); its parity bound is 2e-2 of the output's
+    RMS.  Modelled on the CPU at the tests' shapes -- A_loc unit-scale like an
+    attention output, W a projection weight -- the largest deviation from the
+    fp64 product stays under half the bound."""
+    g = si.rng("tol", "proj")
+    for T, D, Dout in ((405, 256, 192), (780, 1536, 1536)):
+        A = g.standard_normal((T, D)) * 0.5
+        W = si.projection_weight(D, Dout, ("tol", "proj", D), "bf16").astype(np.float64)
+        dW = 0.02 * g.standard_normal((D, Dout))
+        Wn = si.round_to_bf16((W + dW).astype(np.float32)).astype(np.float64)
+        exact = A @ Wn
+        model = (si.round_to_bf16(A.astype(np.float32)).astype(np.float32) @ Wn.astype(np.float32)).astype(np.float64)
+        rel = np.abs(model - exact).max() / np.sqrt(np.mean(exact ** 2))
+        assert rel < 1e-2, (T, D, rel)
