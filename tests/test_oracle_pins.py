@@ -223,6 +223,46 @@ def test_exact_absorption_closed_form():
     assert check_exact_absorption(orc.absorption_stats, orc.ridge_solve, orc.eps_direct)
 
 
+def test_absorb_layer_stacks_every_chunk_and_absorbs_exactly():
+    """Three warmup chunks of a layer (two instances, two heads of d = 4) whose full
+    output is an exact linear map of the local one, A_full = A_loc M: with lambda -> 0
+    the layer's absorption is dW = (M - I) W and eps = 0; its statistics are the sums
+    of the chunks' own (explicit loops over every row of every chunk); the relative
+    lambda takes the trace of the summed G; and the history output plays no part."""
+    g = np.random.default_rng(21)
+    B, n, H, d = 2, 7, 2, 4
+    D = H * d
+    M = np.eye(D) + 0.3 * g.standard_normal((D, D))
+    W = g.standard_normal((D, 5))
+    chunks = []
+    for _ in range(3):
+        o_loc = g.standard_normal((B, n, H, d))
+        o_full = (o_loc.reshape(B * n, D) @ M).reshape(B, n, H, d)
+        chunks.append({"O_loc": o_loc, "O_full": o_full, "O_hist": np.full((B, n, H, d), np.nan)})
+    out = orc.absorb_layer(chunks, W, 1e-14, False)
+    assert np.allclose(out["dW"], (M - np.eye(D)) @ W, atol=1e-8)
+    assert out["eps"] <= 1e-12 * out["r2"]
+    G = np.zeros((D, D))
+    C = np.zeros((D, 5))
+    r2 = 0.0
+    for c in chunks:
+        for b in range(B):
+            for i in range(n):
+                a = [c["O_loc"][b, i, h, e] for h in range(H) for e in range(d)]
+                f = [c["O_full"][b, i, h, e] for h in range(H) for e in range(d)]
+                r = [sum((f[k] - a[k]) * W[k, j] for k in range(D)) for j in range(5)]
+                for x in range(D):
+                    for y in range(D):
+                        G[x, y] += a[x] * a[y]
+                    for j in range(5):
+                        C[x, j] += a[x] * r[j]
+                r2 += sum(v * v for v in r)
+    assert np.allclose(out["G"], G, rtol=1e-12, atol=1e-12) and np.allclose(out["C"], C, rtol=1e-12, atol=1e-12)
+    assert abs(out["r2"] - r2) <= 1e-12 * r2
+    rel = orc.absorb_layer(chunks, W, 1e-3, True)
+    assert abs(rel["lam"] - 1e-3 * np.trace(G) / D) <= 1e-12 * rel["lam"]
+
+
 def check_normal_equations(stats, solve, lam=0.7, seed=7):
     A_loc, A_full, W = _absorb_problem(seed)
     G, C, r2 = stats(A_loc, A_full, W)
